@@ -1,0 +1,204 @@
+"""NumPy front end of the C oracle (``msda_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY: the test suite, the smoke check and the benchmark's
+CPU-baseline leg may import this package; the library itself never does.
+
+Every function takes NumPy arrays (any float dtype is widened exactly to
+float64), returns float64 results and follows the layouts documented in
+``msda_oracle.h``.  ``coord_f32=True`` takes the corner decision in binary32,
+as the CUDA kernels do; ``False`` takes it in double (finite differences).
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+_D = ctypes.POINTER(ctypes.c_double)
+_I64 = ctypes.POINTER(ctypes.c_int64)
+_I32 = ctypes.POINTER(ctypes.c_int32)
+_U8 = ctypes.POINTER(ctypes.c_uint8)
+_i = ctypes.c_int
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        L.oracle_softmax.argtypes = [_D, ctypes.c_int64, _i, _D]
+        L.oracle_msda_forward.argtypes = [_D, _i, _i, _i, _i, _i, _I64, _I64, _i, _i, _D, _D, _i, _D]
+        L.oracle_msda_forward_fused.argtypes = [_D, _i, _i, _i, _i, _i, _I64, _I64, _i, _i, _i,
+                                                _D, _D, _D, _i, _D]
+        L.oracle_fused_locations.argtypes = [_i, _i, _i, _I64, _i, _i, _i, _D, _D, _D, _i, _D, _D]
+        L.oracle_msda_backward.argtypes = [_D, _i, _i, _i, _i, _i, _I64, _I64, _i, _i, _D, _D, _D,
+                                           _i, _D, _D, _D]
+        L.oracle_sca_compact.argtypes = [_U8, _i, _i, _i, _i, _I32, _I32, _I32, _I32]
+        L.oracle_sca_forward.argtypes = [_D, _i, _i, _i, _i, _i, _i, _I64, _I64, _i, _i, _i, _D,
+                                         _U8, _D, _D, _i, _D, _D]
+        L.oracle_sca_backward.argtypes = [_D, _i, _i, _i, _i, _i, _i, _I64, _I64, _i, _i, _i, _D,
+                                          _U8, _D, _D, _D, _i, _D, _D, _D]
+        for f in ("oracle_softmax", "oracle_msda_forward", "oracle_msda_forward_fused",
+                  "oracle_fused_locations", "oracle_msda_backward", "oracle_sca_compact",
+                  "oracle_sca_forward", "oracle_sca_backward"):
+            getattr(L, f).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _d(a):
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _p(a, t):
+    return a.ctypes.data_as(t)
+
+
+def _levels(spatial_shapes, level_start_index):
+    shapes = np.ascontiguousarray(spatial_shapes, dtype=np.int64).reshape(-1, 2)
+    if level_start_index is None:
+        sizes = shapes[:, 0] * shapes[:, 1]
+        level_start_index = np.concatenate([[0], np.cumsum(sizes)[:-1]])
+    starts = np.ascontiguousarray(level_start_index, dtype=np.int64).reshape(-1)
+    return shapes, starts
+
+
+def _check(rc, name):
+    if rc != 0:
+        raise ValueError(f"{name}: invalid arguments")
+
+
+def softmax(logits, axis_len):
+    a = _d(logits)
+    out = np.empty_like(a)
+    _check(lib().oracle_softmax(_p(a, _D), a.size // axis_len, axis_len, _p(out, _D)), "softmax")
+    return out
+
+
+def msda_forward(value, spatial_shapes, level_start_index, sampling_locations,
+                 attention_weights, coord_f32=True):
+    """value [B, Nv, H, Dh]; locations [B, Nq, H, L, P, 2]; weights [B, Nq, H, L, P]
+    -> out [B, Nq, H*Dh]."""
+    v, loc, w = _d(value), _d(sampling_locations), _d(attention_weights)
+    shapes, starts = _levels(spatial_shapes, level_start_index)
+    B, Nv, H, Dh = v.shape
+    _, Nq, _, L, P, _ = loc.shape
+    out = np.empty((B, Nq, H * Dh))
+    rc = lib().oracle_msda_forward(_p(v, _D), B, Nv, H, Dh, L, _p(shapes, _I64), _p(starts, _I64),
+                                   Nq, P, _p(loc, _D), _p(w, _D), int(coord_f32), _p(out, _D))
+    _check(rc, "msda_forward")
+    return out
+
+
+def fused_locations(spatial_shapes, reference_points, sampling_offsets, attention_logits,
+                    coord_f32=True):
+    """-> (sampling_locations [B, Nq, H, L, P, 2], attention_weights [B, Nq, H, L, P])."""
+    shapes, _ = _levels(spatial_shapes, None)
+    ref, off, lg = _d(reference_points), _d(sampling_offsets), _d(attention_logits)
+    B, Nq, H, L, P, _ = off.shape
+    R = ref.shape[2]
+    loc = np.empty(off.shape)
+    w = np.empty(lg.shape)
+    rc = lib().oracle_fused_locations(B, H, L, _p(shapes, _I64), Nq, P, R, _p(ref, _D),
+                                      _p(off, _D), _p(lg, _D), int(coord_f32), _p(loc, _D),
+                                      _p(w, _D))
+    _check(rc, "fused_locations")
+    return loc, w
+
+
+def msda_forward_fused(value, spatial_shapes, level_start_index, reference_points,
+                       sampling_offsets, attention_logits, coord_f32=True):
+    """ref [B, Nq, R, 2]; offsets [B, Nq, H, L, P, 2] (level pixels);
+    logits [B, Nq, H, L, P] -> out [B, Nq, H*Dh]."""
+    v = _d(value)
+    shapes, starts = _levels(spatial_shapes, level_start_index)
+    ref, off, lg = _d(reference_points), _d(sampling_offsets), _d(attention_logits)
+    B, Nv, H, Dh = v.shape
+    _, Nq, _, L, P, _ = off.shape
+    R = ref.shape[2]
+    out = np.empty((B, Nq, H * Dh))
+    rc = lib().oracle_msda_forward_fused(_p(v, _D), B, Nv, H, Dh, L, _p(shapes, _I64),
+                                         _p(starts, _I64), Nq, P, R, _p(ref, _D), _p(off, _D),
+                                         _p(lg, _D), int(coord_f32), _p(out, _D))
+    _check(rc, "msda_forward_fused")
+    return out
+
+
+def msda_backward(value, spatial_shapes, level_start_index, sampling_locations,
+                  attention_weights, grad_out, coord_f32=True):
+    """-> (grad_value [B, Nv, H, Dh], grad_locations, grad_weights)."""
+    v, loc, w, go = _d(value), _d(sampling_locations), _d(attention_weights), _d(grad_out)
+    shapes, starts = _levels(spatial_shapes, level_start_index)
+    B, Nv, H, Dh = v.shape
+    _, Nq, _, L, P, _ = loc.shape
+    gv = np.empty(v.shape)
+    gl = np.empty(loc.shape)
+    gw = np.empty(w.shape)
+    rc = lib().oracle_msda_backward(_p(v, _D), B, Nv, H, Dh, L, _p(shapes, _I64), _p(starts, _I64),
+                                    Nq, P, _p(loc, _D), _p(w, _D), _p(go, _D), int(coord_f32),
+                                    _p(gv, _D), _p(gl, _D), _p(gw, _D))
+    _check(rc, "msda_backward")
+    return gv, gl, gw
+
+
+def sca_compact(bev_mask):
+    """bev_mask [Ncam, B, Nq, R] -> (idx [B, Ncam, Nq], count [B, Ncam],
+    pos [B, Ncam, Nq], hits [B, Nq]), all int32."""
+    m = np.ascontiguousarray(bev_mask).astype(np.uint8)
+    Ncam, B, Nq, R = m.shape
+    idx = np.empty((B, Ncam, Nq), np.int32)
+    cnt = np.empty((B, Ncam), np.int32)
+    pos = np.empty((B, Ncam, Nq), np.int32)
+    hits = np.empty((B, Nq), np.int32)
+    rc = lib().oracle_sca_compact(_p(m, _U8), Ncam, B, Nq, R, _p(idx, _I32), _p(cnt, _I32),
+                                  _p(pos, _I32), _p(hits, _I32))
+    _check(rc, "sca_compact")
+    return idx, cnt, pos, hits
+
+
+def sca_forward(value, spatial_shapes, level_start_index, reference_points_cam, bev_mask,
+                sampling_offsets, attention_logits, coord_f32=True, return_rebatched=False):
+    """value [B, Ncam, Nv, H, Dh]; ref [Ncam, B, Nq, R, 2]; mask [Ncam, B, Nq, R];
+    offsets [B, Nq, H, L, P, 2]; logits [B, Nq, H, L, P] -> out [B, Nq, H*Dh]
+    (and the rebatched rows [B, Ncam, Nq, H*Dh] when asked)."""
+    v = _d(value)
+    shapes, starts = _levels(spatial_shapes, level_start_index)
+    ref, off, lg = _d(reference_points_cam), _d(sampling_offsets), _d(attention_logits)
+    m = np.ascontiguousarray(bev_mask).astype(np.uint8)
+    B, Ncam, Nv, H, Dh = v.shape
+    _, Nq, _, L, P, _ = off.shape
+    R = ref.shape[3]
+    out = np.empty((B, Nq, H * Dh))
+    rb = np.empty((B, Ncam, Nq, H * Dh)) if return_rebatched else None
+    rc = lib().oracle_sca_forward(_p(v, _D), B, Ncam, Nv, H, Dh, L, _p(shapes, _I64),
+                                  _p(starts, _I64), Nq, P, R, _p(ref, _D), _p(m, _U8), _p(off, _D),
+                                  _p(lg, _D), int(coord_f32), _p(out, _D),
+                                  _p(rb, _D) if rb is not None else None)
+    _check(rc, "sca_forward")
+    return (out, rb) if return_rebatched else out
+
+
+def sca_backward(value, spatial_shapes, level_start_index, reference_points_cam, bev_mask,
+                 sampling_offsets, attention_logits, grad_out, coord_f32=True):
+    """-> (grad_value [B, Ncam, Nv, H, Dh], grad_loc_rb [B, Ncam, Nq, H, L, P, 2],
+    grad_attn_rb [B, Ncam, Nq, H, L, P])."""
+    v = _d(value)
+    shapes, starts = _levels(spatial_shapes, level_start_index)
+    ref, off, lg = _d(reference_points_cam), _d(sampling_offsets), _d(attention_logits)
+    go = _d(grad_out)
+    m = np.ascontiguousarray(bev_mask).astype(np.uint8)
+    B, Ncam, Nv, H, Dh = v.shape
+    _, Nq, _, L, P, _ = off.shape
+    R = ref.shape[3]
+    gv = np.empty(v.shape)
+    gl = np.empty((B, Ncam, Nq, H, L, P, 2))
+    gw = np.empty((B, Ncam, Nq, H, L, P))
+    rc = lib().oracle_sca_backward(_p(v, _D), B, Ncam, Nv, H, Dh, L, _p(shapes, _I64),
+                                   _p(starts, _I64), Nq, P, R, _p(ref, _D), _p(m, _U8),
+                                   _p(off, _D), _p(lg, _D), _p(go, _D), int(coord_f32),
+                                   _p(gv, _D), _p(gl, _D), _p(gw, _D))
+    _check(rc, "sca_backward")
+    return gv, gl, gw

@@ -1,0 +1,575 @@
+"""Pins of the oracle against facts fixed by the pages and by mathematics.
+
+Every test here runs on the CPU.  None of them re-types the oracle's formula:
+each checks it against a worked example from the pages, a closed form, an
+invariant, a library routine the special case reduces to (torch's
+grid_sample), a brute-force loop with a different structure, or central
+finite differences.
+
+Sources: "BEV(三) BEVFormer: how the Query interacts with the 8 Heads of the
+Feature" (sections 4.2, 5, 6, 7, 10, 15) and the Tencent Cloud "Spatial
+Cross-Attention" walkthrough (rebatch and average listings).
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from scale_deformable_attention_03_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rng(seed):
+    return np.random.Generator(np.random.PCG64(seed))
+
+
+def _levels(shapes):
+    s, starts, nv = inputs.level_table(shapes)
+    return s, starts, nv
+
+
+def _value_rows(value_b, starts, shapes, l, h):
+    """[Dh, H_l, W_l] view of head h of level l of one batch item's value."""
+    Hl, Wl = shapes[l]
+    rows = value_b[starts[l]:starts[l] + Hl * Wl, h, :]
+    return rows.reshape(Hl, Wl, -1).transpose(2, 0, 1)
+
+
+def _grid_sample_msda(value, shapes, starts, loc, attn):
+    """Brute force with torch's grid_sample (bilinear, zero padding,
+    align_corners=False) for every (b, q, h, l, k), summed with the weights."""
+    B, Nv, H, Dh = value.shape
+    _, Nq, _, L, P, _ = loc.shape
+    out = np.zeros((B, Nq, H, Dh))
+    for b in range(B):
+        for h in range(H):
+            for l in range(L):
+                img = torch.from_numpy(np.ascontiguousarray(
+                    _value_rows(value[b], starts, shapes, l, h)))[None]
+                grid = torch.from_numpy(2.0 * loc[b, :, h, l, :, :] - 1.0)[None]  # [1, Nq, P, 2]
+                f = torch.nn.functional.grid_sample(img, grid, mode="bilinear",
+                                                    padding_mode="zeros", align_corners=False)
+                f = f[0].numpy().transpose(1, 2, 0)  # [Nq, P, Dh]
+                out[b, :, h, :] += np.einsum("qp,qpd->qd", attn[b, :, h, l, :], f)
+    return out.reshape(B, Nq, H * Dh)
+
+
+# --------------------------------------------------------------------------
+# softmax (section 4.2)
+# --------------------------------------------------------------------------
+
+def test_softmax_sums_to_one_per_head():
+    a = _rng(1).standard_normal((7, 3, 32)) * 4
+    w = oracle.softmax(a, 32)
+    assert np.all(w > 0)
+    np.testing.assert_allclose(w.sum(-1), 1.0, rtol=0, atol=1e-12)
+    # ordering is preserved and a shift of all logits changes nothing
+    np.testing.assert_array_equal(np.argsort(w, -1), np.argsort(a, -1))
+    np.testing.assert_allclose(oracle.softmax(a + 123.0, 32), w, rtol=1e-12, atol=0)
+
+
+def test_softmax_zero_logits_uniform():
+    # zero-initialised weight head: every one of the L*P = 32 weights is 1/32
+    w = oracle.softmax(np.zeros((5, 8, 32)), 32)
+    assert np.all(w == 1.0 / 32.0)
+    w = oracle.softmax(np.zeros((2, 12)), 12)
+    np.testing.assert_allclose(w, 1.0 / 12.0, rtol=1e-15)
+
+
+def test_softmax_large_logits_stable():
+    w = oracle.softmax(np.array([[1000.0, 1000.0, -1000.0, 999.0]]), 4)
+    e = np.exp([0.0, 0.0, -2000.0, -1.0])
+    np.testing.assert_allclose(w[0], e / e.sum(), rtol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# bilinear read (section 6)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("coord_f32", [True, False])
+def test_pixel_centres_reproduce_pixels(coord_f32):
+    shapes, starts, Nv = _levels([(5, 7), (3, 4), (2, 9)])
+    H, Dh = 3, 5
+    rng = _rng(2)
+    value = rng.standard_normal((1, Nv, H, Dh))
+    L, P = len(shapes), 1
+    targets = [(l, y, x) for l in range(L) for y in range(shapes[l][0]) for x in range(shapes[l][1])]
+    Nq = len(targets)
+    loc = rng.uniform(0.2, 0.8, (1, Nq, H, L, P, 2)).astype(np.float32)
+    attn = np.zeros((1, Nq, H, L, P))
+    expect = np.zeros((1, Nq, H, Dh))
+    for q, (l, y, x) in enumerate(targets):
+        Hl, Wl = shapes[l]
+        loc[0, q, :, l, 0, 0] = np.float32((x + 0.5) / Wl)
+        loc[0, q, :, l, 0, 1] = np.float32((y + 0.5) / Hl)
+        attn[0, q, :, l, 0] = 1.0
+        expect[0, q] = value[0, starts[l] + y * Wl + x]
+    out = oracle.msda_forward(value, shapes, starts, loc, attn, coord_f32=coord_f32)
+    np.testing.assert_allclose(out, expect.reshape(1, Nq, H * Dh), rtol=1e-6, atol=1e-6)
+
+
+def test_constant_map_gives_constant():
+    shapes, starts, Nv = _levels([(6, 9), (3, 5)])
+    H, Dh, L, P, Nq = 2, 4, 2, 3, 40
+    rng = _rng(3)
+    value = np.full((1, Nv, H, Dh), 2.5)
+    loc = np.empty((1, Nq, H, L, P, 2), np.float32)
+    for l, (Hl, Wl) in enumerate(shapes):
+        # x = W s - 1/2 in [0, W-1]: all four neighbours inside the map
+        loc[..., l, :, 0] = rng.uniform(0.5 / Wl, 1 - 0.5 / Wl, (1, Nq, H, P))
+        loc[..., l, :, 1] = rng.uniform(0.5 / Hl, 1 - 0.5 / Hl, (1, Nq, H, P))
+    attn = rng.uniform(0, 1, (1, Nq, H, L, P))
+    out = oracle.msda_forward(value, shapes, starts, loc, attn).reshape(1, Nq, H, Dh)
+    expect = 2.5 * attn.sum(axis=(3, 4))[..., None]
+    np.testing.assert_allclose(out, np.broadcast_to(expect, out.shape), rtol=1e-12)
+
+
+def test_fully_out_of_bounds_is_zero():
+    shapes, starts, Nv = _levels([(4, 6)])
+    H, Dh, L, P, Nq = 2, 3, 1, 4, 64
+    rng = _rng(4)
+    value = rng.standard_normal((1, Nv, H, Dh)) + 10.0
+    Hl, Wl = shapes[0]
+    loc = rng.uniform(0.0, 1.0, (1, Nq, H, L, P, 2))
+    side = rng.integers(0, 4, (1, Nq, H, L, P))
+    # x <= -1 (s_x <= -0.5/W), x >= W (s_x >= 1 + 0.5/W), same for y
+    loc[..., 0] = np.where(side == 0, rng.uniform(-2.0, -0.5 / Wl, side.shape), loc[..., 0])
+    loc[..., 0] = np.where(side == 1, rng.uniform(1 + 0.5 / Wl, 3.0, side.shape), loc[..., 0])
+    loc[..., 1] = np.where(side == 2, rng.uniform(-2.0, -0.5 / Hl, side.shape), loc[..., 1])
+    loc[..., 1] = np.where(side == 3, rng.uniform(1 + 0.5 / Hl, 3.0, side.shape), loc[..., 1])
+    loc = loc.astype(np.float32)
+    attn = rng.uniform(0.1, 1, (1, Nq, H, L, P))
+    out = oracle.msda_forward(value, shapes, starts, loc, attn)
+    assert np.all(out == 0.0)
+
+
+def test_non_finite_location_reads_nothing():
+    shapes, starts, Nv = _levels([(4, 6)])
+    value = _rng(5).standard_normal((1, Nv, 1, 2))
+    loc = np.full((1, 3, 1, 1, 1, 2), 0.5, np.float32)
+    loc[0, 0, 0, 0, 0, 0] = np.nan
+    loc[0, 1, 0, 0, 0, 1] = np.inf
+    attn = np.ones((1, 3, 1, 1, 1))
+    out = oracle.msda_forward(value, shapes, starts, loc, attn)
+    assert np.all(out[0, :2] == 0.0) and np.any(out[0, 2] != 0.0)
+    go = np.ones_like(out)
+    gv, gl, gw = oracle.msda_backward(value, shapes, starts, loc, attn, go)
+    assert np.all(gl[0, :2] == 0.0) and np.all(gw[0, :2] == 0.0)
+
+
+@pytest.mark.parametrize("coord_f32,tol", [(False, 1e-12), (True, 2e-5)])
+def test_matches_torch_grid_sample(coord_f32, tol):
+    """The bilinear read with zero padding and align_corners=False is exactly
+    torch.nn.functional.grid_sample (bilinear, zeros) at grid = 2 s - 1."""
+    shapes, starts, Nv = _levels([(7, 11), (4, 5), (3, 2), (1, 1)])
+    B, H, Dh, L, P, Nq = 2, 3, 6, 4, 5, 23
+    rng = _rng(6)
+    value = rng.standard_normal((B, Nv, H, Dh))
+    loc = rng.uniform(-0.25, 1.25, (B, Nq, H, L, P, 2)).astype(np.float32).astype(np.float64)
+    attn = rng.standard_normal((B, Nq, H, L, P))
+    out = oracle.msda_forward(value, shapes, starts, loc, attn, coord_f32=coord_f32)
+    ref = _grid_sample_msda(value, shapes, starts, loc, attn)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=tol)
+
+
+def test_one_hot_weight_returns_the_sample():
+    shapes, starts, Nv = _levels([(5, 8), (3, 3)])
+    B, H, Dh, L, P, Nq = 1, 2, 4, 2, 3, 12
+    rng = _rng(7)
+    value = rng.standard_normal((B, Nv, H, Dh))
+    loc = rng.uniform(-0.1, 1.1, (B, Nq, H, L, P, 2))
+    pick = rng.integers(0, L * P, (B, Nq, H))
+    attn = np.zeros((B, Nq, H, L * P))
+    np.put_along_axis(attn, pick[..., None], 1.0, axis=-1)
+    attn = attn.reshape(B, Nq, H, L, P)
+    out = oracle.msda_forward(value, shapes, starts, loc, attn, coord_f32=False)
+    ref = _grid_sample_msda(value, shapes, starts, loc, attn)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# weighted sum and head concat (sections 7-9, 15)
+# --------------------------------------------------------------------------
+
+def _pixel_centre(x, y, W, H):
+    return np.float32((x + 0.5) / W), np.float32((y + 0.5) / H)
+
+
+def test_section7_alpha_times_f():
+    g = json.load(open(os.path.join(GOLDEN, "bq_s7_alpha_times_f.json")))
+    f = np.asarray(g["f"])
+    shapes, starts, Nv = _levels([(1, 1)])
+    value = f.reshape(1, 1, 1, 3)
+    loc = np.full((1, 1, 1, 1, 1, 2), 0.5, np.float32)
+    attn = np.full((1, 1, 1, 1, 1), g["alpha"])
+    out = oracle.msda_forward(value, shapes, starts, loc, attn)
+    np.testing.assert_allclose(out.reshape(-1), g["expected"], rtol=1e-15)
+
+
+def _section15_problem(g):
+    """A 1x2 value map whose pixel centres hold the example's sampled vectors:
+    pixel 0 holds f_1 and pixel 1 holds f_2 of each head."""
+    f = np.asarray(g["f"])                  # [head, sample, channel]
+    H, S, Dh = f.shape
+    shapes, starts, Nv = _levels([(1, S)])
+    value = f.transpose(1, 0, 2)[None]      # [1, Nv = S, H, Dh]
+    loc = np.zeros((1, 1, H, 1, S, 2), np.float32)
+    for k in range(S):
+        loc[0, 0, :, 0, k, :] = _pixel_centre(k, 0, S, 1)
+    return value, shapes, starts, loc
+
+
+def test_section15_two_head_example():
+    g = json.load(open(os.path.join(GOLDEN, "bq_s15_two_head_example.json")))
+    value, shapes, starts, loc = _section15_problem(g)
+    attn = np.asarray(g["alpha"])[None, None, :, None, :]
+    out = oracle.msda_forward(value, shapes, starts, loc, attn)
+    np.testing.assert_allclose(out.reshape(-1), g["g"], rtol=1e-14)
+    # identity output projection, dropout off: q_hat = q + g
+    np.testing.assert_allclose(np.asarray(g["q"]) + out.reshape(-1), g["q_hat"], rtol=1e-14)
+
+
+def test_section15_through_the_fused_path():
+    """Logits log(alpha) softmax back to alpha; zero offsets from the pixel
+    centres (one reference point per sample, R = 2) read the same vectors."""
+    g = json.load(open(os.path.join(GOLDEN, "bq_s15_two_head_example.json")))
+    value, shapes, starts, loc = _section15_problem(g)
+    H, S = np.asarray(g["alpha"]).shape
+    ref = loc[:, :, 0, 0, :, :].copy()            # [1, 1, R = S, 2]
+    off = np.zeros((1, 1, H, 1, S, 2))
+    logits = np.log(np.asarray(g["alpha"]))[None, None, :, None, :]
+    out = oracle.msda_forward_fused(value, shapes, starts, ref, off, logits)
+    np.testing.assert_allclose(out.reshape(-1), g["g"], rtol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# location (section 5)
+# --------------------------------------------------------------------------
+
+def test_anchor_of_point_k_is_k_mod_R():
+    """Section 5: with 4 anchors, point k = 4 j + m starts from anchor m.
+    Each anchor sits on a pixel centre holding a distinct value; a one-hot
+    weight on point k must read the pixel of anchor k mod 4."""
+    shapes, starts, Nv = _levels([(3, 10)])
+    R, P, H, Dh = 4, 8, 1, 1
+    value = np.arange(Nv, dtype=np.float64).reshape(1, Nv, 1, 1) + 100
+    anchors = [(1, 0), (4, 1), (7, 2), (9, 1)]   # (x, y) per anchor
+    ref = np.array([[_pixel_centre(x, y, 10, 3) for (x, y) in anchors]], np.float32)[None]
+    off = np.zeros((1, P, H, 1, P, 2))
+    logits = np.full((1, P, H, 1, P), -1e30)
+    for q in range(P):
+        logits[0, q, 0, 0, q] = 0.0
+    ref = np.repeat(ref, P, axis=1)
+    out = oracle.msda_forward_fused(value, shapes, starts, ref, off, logits).reshape(-1)
+    expect = [100 + anchors[k % 4][1] * 10 + anchors[k % 4][0] for k in range(P)]
+    np.testing.assert_array_equal(out, expect)
+
+
+def test_offsets_are_in_level_pixels():
+    """Section 5: the offset is divided by the level's width (x) and height
+    (y), so an offset of (+1, 0) / (0, +1) moves the read by exactly one pixel
+    on every level, whatever its size."""
+    shapes, starts, Nv = _levels([(6, 10), (3, 5), (2, 7)])
+    L, P, R, H, Dh = 3, 3, 1, 1, 1
+    value = np.arange(Nv, dtype=np.float64).reshape(1, Nv, 1, 1)
+    # anchor on the centre of pixel (2, 1) of a 10x6 grid: normalised, it is a
+    # different pixel on each level; read one level at a time
+    for l, (Hl, Wl) in enumerate(shapes):
+        x, y = 1, 0
+        ref = np.array(_pixel_centre(x, y, Wl, Hl), np.float32).reshape(1, 1, 1, 2)
+        ref = np.repeat(ref, P, axis=1)
+        off = np.zeros((1, P, H, L, P, 2))
+        off[0, 1, 0, :, 1, 0] = 1.0       # query 1: point 1 one pixel right
+        off[0, 2, 0, :, 2, 1] = 1.0       # query 2: point 2 one pixel down
+        logits = np.full((1, P, H, L, P), -1e30)
+        for q in range(P):
+            logits[0, q, 0, l, q] = 0.0
+        out = oracle.msda_forward_fused(value, shapes, starts, ref, off, logits).reshape(-1)
+        base = starts[l] + y * Wl + x
+        np.testing.assert_allclose(out, [base, base + 1, base + Wl], rtol=0, atol=1e-4)
+
+
+# --------------------------------------------------------------------------
+# compaction (rebatch listing) and camera average (section 10, average listing)
+# --------------------------------------------------------------------------
+
+def _random_mask(rng, Ncam, B, Nq, R, p=0.3):
+    return (rng.random((Ncam, B, Nq, R)) < p).astype(np.uint8)
+
+
+def test_compaction_brute_force():
+    rng = _rng(8)
+    Ncam, B, Nq, R = 5, 3, 97, 3
+    mask = _random_mask(rng, Ncam, B, Nq, R, 0.2)
+    idx, cnt, pos, hits = oracle.sca_compact(mask)
+    for b in range(B):
+        for c in range(Ncam):
+            seen = [q for q in range(Nq) if any(mask[c, b, q, r] for r in range(R))]
+            n = len(seen)
+            assert cnt[b, c] == n
+            assert list(idx[b, c, :n]) == seen
+            assert np.all(idx[b, c, n:] == -1)
+            # numpy's nonzero of the summed mask, as the rebatch listing does
+            np.testing.assert_array_equal(idx[b, c, :n], np.nonzero(mask[c, b].sum(-1))[0])
+            for q in range(Nq):
+                assert pos[b, c, q] == (seen.index(q) if q in seen else -1)
+    np.testing.assert_array_equal(hits, (mask.sum(-1) > 0).transpose(1, 2, 0).sum(-1))
+    assert cnt.sum() == hits.sum()
+
+
+def test_compaction_edge_cases():
+    for (Ncam, B, Nq, R) in [(1, 1, 1, 1), (3, 2, 0, 2), (2, 1, 33, 4)]:
+        for fill in (0, 1):
+            mask = np.full((Ncam, B, Nq, R), fill, np.uint8)
+            idx, cnt, pos, hits = oracle.sca_compact(mask)
+            assert np.all(cnt == (Nq if fill else 0))
+            if Nq:
+                assert np.all(hits == (Ncam if fill else 0))
+                if fill:
+                    assert np.all(idx == np.arange(Nq)) and np.all(pos == np.arange(Nq))
+                else:
+                    assert np.all(idx == -1) and np.all(pos == -1)
+
+
+def _tiny_sca(seed, B=2, Ncam=3, bev=(2, 4), shapes=((3, 5), (2, 2)), H=2, Dh=3, P=4, R=2,
+              p_mask=0.35):
+    rng = _rng(seed)
+    shapes, starts, Nv = _levels(list(shapes))
+    L = len(shapes)
+    Nq = bev[0] * bev[1]
+    value = rng.standard_normal((B, Ncam, Nv, H, Dh))
+    ref = rng.uniform(0.05, 0.95, (Ncam, B, Nq, R, 2))
+    mask = _random_mask(rng, Ncam, B, Nq, R, p_mask)
+    mask[:, 0, 0, :] = 0          # a query no camera sees
+    mask[:, 0, 1, 0] = 1          # a query every camera sees
+    off = rng.standard_normal((B, Nq, H, L, P, 2)) * 0.7
+    logits = rng.standard_normal((B, Nq, H, L, P))
+    return dict(value=value, shapes=shapes, starts=starts, ref=ref, mask=mask, off=off,
+                logits=logits, B=B, Ncam=Ncam, Nq=Nq, H=H, Dh=Dh, L=L, P=P, R=R)
+
+
+@pytest.mark.parametrize("coord_f32", [True, False])
+def test_sca_equals_per_query_camera_mean(coord_f32):
+    """The rebatch / scatter-add / clamp(count, 1) pipeline equals a direct
+    per-query mean over the cameras that see the query, with no rebatching."""
+    t = _tiny_sca(9)
+    ref32 = t["ref"].astype(np.float32) if coord_f32 else t["ref"]
+    off32 = t["off"].astype(np.float32) if coord_f32 else t["off"]
+    out = oracle.sca_forward(t["value"], t["shapes"], t["starts"], ref32, t["mask"], off32,
+                             t["logits"], coord_f32=coord_f32)
+    expect = np.zeros_like(out)
+    for b in range(t["B"]):
+        for q in range(t["Nq"]):
+            cams = [c for c in range(t["Ncam"]) if t["mask"][c, b, q].any()]
+            for c in cams:
+                one = oracle.msda_forward_fused(
+                    t["value"][b:b + 1, c], t["shapes"], t["starts"],
+                    ref32[c, b:b + 1, q:q + 1], off32[b:b + 1, q:q + 1],
+                    t["logits"][b:b + 1, q:q + 1], coord_f32=coord_f32)
+                expect[b, q] += one[0, 0] / len(cams)
+    np.testing.assert_allclose(out, expect, rtol=1e-12, atol=1e-14)
+    assert np.all(out[0, 0] == 0.0)  # seen by no camera: zero
+
+
+def test_sca_single_camera_is_plain_msda():
+    t = _tiny_sca(10)
+    mask = np.zeros_like(t["mask"])
+    mask[1, :, :, 0] = 1          # only camera 1 sees every query
+    out = oracle.sca_forward(t["value"], t["shapes"], t["starts"], t["ref"], mask, t["off"],
+                             t["logits"], coord_f32=False)
+    plain = oracle.msda_forward_fused(t["value"][:, 1], t["shapes"], t["starts"], t["ref"][1],
+                                      t["off"], t["logits"], coord_f32=False)
+    np.testing.assert_allclose(out, plain, rtol=1e-14, atol=0)
+
+
+def test_sca_rebatched_rows_follow_compaction():
+    t = _tiny_sca(11)
+    out, rb = oracle.sca_forward(t["value"], t["shapes"], t["starts"], t["ref"], t["mask"],
+                                 t["off"], t["logits"], coord_f32=False, return_rebatched=True)
+    idx, cnt, pos, hits = oracle.sca_compact(t["mask"])
+    for b in range(t["B"]):
+        acc = np.zeros_like(out[b])
+        for c in range(t["Ncam"]):
+            n = cnt[b, c]
+            assert np.all(rb[b, c, n:] == 0.0)
+            acc[idx[b, c, :n]] += rb[b, c, :n]
+        np.testing.assert_allclose(out[b], acc / np.maximum(hits[b], 1)[:, None], rtol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# backward: central finite differences and linearity
+# --------------------------------------------------------------------------
+
+def _fd_locations(rng, shape, shapes, margin=1e-3):
+    """Locations whose pixel coordinates stay >= margin away from integers,
+    so that +-h never crosses a cell boundary."""
+    loc = rng.uniform(-0.15, 1.15, shape)
+    L = shape[3]
+    for l in range(L):
+        Hl, Wl = shapes[l]
+        for ax, n in ((0, Wl), (1, Hl)):
+            x = loc[..., l, :, ax] * n - 0.5
+            fr = x - np.floor(x)
+            x = np.floor(x) + np.clip(fr, margin, 1 - margin)
+            loc[..., l, :, ax] = (x + 0.5) / n
+    return loc
+
+
+def _tiny_msda(seed):
+    rng = _rng(seed)
+    shapes, starts, Nv = _levels([(3, 5), (2, 2)])
+    B, H, Dh, L, P, Nq = 1, 2, 3, 2, 2, 3
+    value = rng.standard_normal((B, Nv, H, Dh))
+    loc = _fd_locations(rng, (B, Nq, H, L, P, 2), shapes)
+    attn = rng.uniform(0.1, 1.0, (B, Nq, H, L, P))
+    go = rng.standard_normal((B, Nq, H * Dh))
+    return value, shapes, starts, loc, attn, go
+
+
+def _central_fd(f, x, h):
+    g = np.zeros_like(x)
+    flat = x.reshape(-1)
+    gf = g.reshape(-1)
+    for i in range(flat.size):
+        keep = flat[i]
+        flat[i] = keep + h
+        up = f()
+        flat[i] = keep - h
+        dn = f()
+        flat[i] = keep
+        gf[i] = (up - dn) / (2 * h)
+    return g
+
+
+def test_msda_backward_matches_finite_differences():
+    value, shapes, starts, loc, attn, go = _tiny_msda(12)
+
+    def loss():
+        return float(np.sum(go * oracle.msda_forward(value, shapes, starts, loc, attn,
+                                                     coord_f32=False)))
+
+    gv, gl, gw = oracle.msda_backward(value, shapes, starts, loc, attn, go, coord_f32=False)
+    h = 1e-6
+    np.testing.assert_allclose(gv, _central_fd(loss, value, h), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(gw, _central_fd(loss, attn, h), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(gl, _central_fd(loss, loc, h), rtol=1e-6, atol=1e-7)
+    assert np.abs(gl).max() > 0.1  # the check is not vacuous
+
+
+def test_msda_backward_with_partly_outside_samples():
+    """Samples whose neighbourhood straddles the border (zero padding)."""
+    rng = _rng(13)
+    shapes, starts, Nv = _levels([(3, 4)])
+    B, H, Dh, L, P, Nq = 1, 1, 2, 1, 6, 4
+    value = rng.standard_normal((B, Nv, H, Dh))
+    # pixel coordinates in (-1, 0) or (W-1, W): one neighbour column outside
+    loc = _fd_locations(rng, (B, Nq, H, L, P, 2), shapes)
+    loc[..., 0, 0::2, 0] = (rng.uniform(-0.9, -0.1, (B, Nq, H, 3)) + 0.5) / 4
+    loc[..., 0, 1::2, 1] = (rng.uniform(2.1, 2.9, (B, Nq, H, 3)) + 0.5) / 3
+    attn = rng.uniform(0.1, 1.0, (B, Nq, H, L, P))
+    go = rng.standard_normal((B, Nq, H * Dh))
+
+    def loss():
+        return float(np.sum(go * oracle.msda_forward(value, shapes, starts, loc, attn,
+                                                     coord_f32=False)))
+
+    gv, gl, gw = oracle.msda_backward(value, shapes, starts, loc, attn, go, coord_f32=False)
+    h = 1e-6
+    np.testing.assert_allclose(gv, _central_fd(loss, value, h), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(gl, _central_fd(loss, loc, h), rtol=1e-6, atol=1e-7)
+    np.testing.assert_allclose(gw, _central_fd(loss, attn, h), rtol=1e-6, atol=1e-8)
+
+
+def test_msda_backward_linearity():
+    """out is linear in the weights and in the value: <gO, out> equals
+    sum(gW * alpha) and sum(gV * V)."""
+    rng = _rng(14)
+    shapes, starts, Nv = _levels([(9, 13), (4, 7), (2, 3)])
+    B, H, Dh, L, P, Nq = 2, 3, 8, 3, 4, 31
+    value = rng.standard_normal((B, Nv, H, Dh))
+    loc = rng.uniform(-0.1, 1.1, (B, Nq, H, L, P, 2)).astype(np.float32)
+    attn = rng.uniform(0, 1, (B, Nq, H, L, P))
+    go = rng.standard_normal((B, Nq, H * Dh))
+    out = oracle.msda_forward(value, shapes, starts, loc, attn)
+    gv, gl, gw = oracle.msda_backward(value, shapes, starts, loc, attn, go)
+    lhs = np.sum(go * out)
+    np.testing.assert_allclose(np.sum(gw * attn), lhs, rtol=1e-12)
+    np.testing.assert_allclose(np.sum(gv * value), lhs, rtol=1e-12)
+
+
+def test_sca_backward_matches_finite_differences():
+    """FD through the whole SCA forward.  grad_value directly; the rebatched
+    location and weight gradients through the chain rule of the fused inputs:
+    d/d offset = sum over seeing cameras of grad_loc / (W_l, H_l),
+    d/d reference point of camera c = sum over points of that anchor,
+    d/d logits = softmax Jacobian of the camera-summed grad_attn."""
+    t = _tiny_sca(15)
+    rng = _rng(16)
+    B, Ncam, Nq, H, Dh, L, P, R = (t[k] for k in ("B", "Ncam", "Nq", "H", "Dh", "L", "P", "R"))
+    go = rng.standard_normal((B, Nq, H * Dh))
+    shapes, starts = t["shapes"], t["starts"]
+    # keep pixel coordinates away from cell boundaries
+    for _ in range(50):
+        loc, _w = oracle.fused_locations(shapes, t["ref"][0], t["off"], t["logits"], coord_f32=False)
+        ok = True
+        for c in range(Ncam):
+            loc_c, _ = oracle.fused_locations(shapes, t["ref"][c], t["off"], t["logits"],
+                                              coord_f32=False)
+            for l, (Hl, Wl) in enumerate(shapes):
+                for ax, n in ((0, Wl), (1, Hl)):
+                    x = loc_c[..., l, :, ax] * n - 0.5
+                    fr = x - np.floor(x)
+                    ok &= bool(np.all((fr > 1e-3) & (fr < 1 - 1e-3)))
+        if ok:
+            break
+        t["off"] += rng.uniform(-0.05, 0.05, t["off"].shape)
+    assert ok
+
+    def loss():
+        return float(np.sum(go * oracle.sca_forward(t["value"], shapes, starts, t["ref"],
+                                                     t["mask"], t["off"], t["logits"],
+                                                     coord_f32=False)))
+
+    gv, gl_rb, gw_rb = oracle.sca_backward(t["value"], shapes, starts, t["ref"], t["mask"],
+                                           t["off"], t["logits"], go, coord_f32=False)
+    h = 1e-6
+    np.testing.assert_allclose(gv, _central_fd(loss, t["value"], h), rtol=1e-6, atol=1e-8)
+
+    idx, cnt, pos, hits = oracle.sca_compact(t["mask"])
+    g_off = np.zeros_like(t["off"])
+    g_ref = np.zeros_like(t["ref"])
+    g_alpha = np.zeros_like(t["logits"])
+    norm = np.array([[Wl, Hl] for (Hl, Wl) in shapes], dtype=np.float64)  # [L, 2]
+    for b in range(B):
+        for c in range(Ncam):
+            for i in range(cnt[b, c]):
+                q = idx[b, c, i]
+                g_off[b, q] += gl_rb[b, c, i] / norm[None, :, None, :]
+                g_alpha[b, q] += gw_rb[b, c, i]
+                for k in range(P):
+                    g_ref[c, b, q, k % R] += gl_rb[b, c, i, :, :, k, :].sum(axis=(0, 1))
+            assert np.all(gl_rb[b, c, cnt[b, c]:] == 0) and np.all(gw_rb[b, c, cnt[b, c]:] == 0)
+    alpha = oracle.softmax(t["logits"], L * P).reshape(g_alpha.shape)
+    ga = g_alpha.reshape(B, Nq, H, L * P)
+    al = alpha.reshape(B, Nq, H, L * P)
+    g_logits = (al * (ga - np.sum(al * ga, -1, keepdims=True))).reshape(g_alpha.shape)
+
+    np.testing.assert_allclose(g_off, _central_fd(loss, t["off"], h), rtol=1e-6, atol=1e-7)
+    np.testing.assert_allclose(g_ref, _central_fd(loss, t["ref"], h), rtol=1e-6, atol=1e-7)
+    np.testing.assert_allclose(g_logits, _central_fd(loss, t["logits"], h), rtol=1e-6, atol=1e-8)
+    assert np.abs(g_off).max() > 0.05
+
+
+def test_empty_problems():
+    shapes, starts, Nv = _levels([(2, 3)])
+    value = np.zeros((1, Nv, 1, 2))
+    out = oracle.msda_forward(value, shapes, starts, np.zeros((1, 0, 1, 1, 1, 2)),
+                              np.zeros((1, 0, 1, 1, 1)))
+    assert out.shape == (1, 0, 2)
+    with pytest.raises(ValueError):
+        oracle.msda_forward(value, [(3, 3)], [0], np.zeros((1, 1, 1, 1, 1, 2)),
+                            np.zeros((1, 1, 1, 1, 1)))  # level larger than the value map
