@@ -1,0 +1,472 @@
+"""Benchmark: BEVFormer-base Spatial Cross-Attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+                    [--value-dtype f32|bf16] [--rho coherent|uniform]
+
+One step = one pass of the whole SCA forward over one synthetic batch: mask
+compaction, the fused rebatched MSDA of all six cameras, the camera average
+(sca_compact + sca_rebatched_forward + sca_camera_average, the same kernels
+sca_forward launches).  Inputs are resident in HBM before timing; the L2 is
+flushed (a 256 MiB write) before every step, outside the timed events.  Each
+step is timed with CUDA events on the launching stream, per stage, and the
+job time is the maximum over ranks of the summed step times.
+
+N > 1 (torchrun, one process per GPU): every rank runs an independent replica
+on its own seeded batch (weak scaling; the path has no exchange step).
+
+Printed (rank 0): one JSON line with the metric, the roofline of the dominant
+kernel (the rebatched gather) against the measured HBM copy bandwidth, the
+oracle timed on the host as the CPU baseline, an end-to-end figure through
+the one-call C ABI with host buffers, and the SM clocks seen during timing.
+
+--impl reference times the oracle (plain C, one host core) on the same
+workload and metric, and prints the same kind of line with "impl":
+"reference".
+"""
+import argparse
+import hashlib
+import json
+import os
+import re
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MSDA sampled points/sec (G/s) + HBM GB/s fraction, BEVFormer-base SCA"
+UNIT = "Gsamples/s"
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "sca_gather_bevformer_base.md")
+KERNEL_SOURCES = ("scale_deformable_attention_03_b200/csrc/msda_device.cuh",
+                  "scale_deformable_attention_03_b200/csrc/sca.cu")
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=("native", "reference"), default="native")
+    p.add_argument("--value-dtype", choices=("f32", "bf16"), default="f32")
+    p.add_argument("--rho", choices=("coherent", "uniform"), default="coherent")
+    p.add_argument("--e2e-steps", type=int, default=5)
+    p.add_argument("--cpu-seconds", type=float, default=10.0,
+                   help="minimum host time of the oracle CPU baseline")
+    return p.parse_args(argv)
+
+
+# --------------------------------------------------------------------------
+# helpers shared with the tests (no GPU needed)
+# --------------------------------------------------------------------------
+
+def rank_seed(rank):
+    """Seed of a replica's synthetic batch: the workload's seed for rank 0,
+    distinct seeds for the other ranks."""
+    return 1003 + 1000 * rank
+
+
+def workload_config(args):
+    from scale_deformable_attention_03_b200 import inputs
+    return {
+        "workload": "bevformer-base-sca-forward",
+        "B": 1, "Ncam": 6, "bev": "200x200", "Nq": 40000,
+        "levels": [list(s) for s in inputs.SHAPES_BEVFORMER], "Nv_per_camera": 30825,
+        "H": 8, "head_dim": 32, "P": 8, "R": 4,
+        "value_dtype": args.value_dtype, "rho": args.rho,
+        "mask": "1 + Bernoulli(0.5) cameras per query, non-zero anchor pattern",
+        "l2": "flushed before every step (256 MiB write, outside the timed events)",
+        "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU",
+    }
+
+
+def algorithmic_bytes(w, rows, hit_queries, value_elem):
+    """Bytes each kernel / the whole step must move at least once.
+    rows: rebatched rows (sum of count); hit_queries: queries seen by at
+    least one camera."""
+    S = w.H * w.L * w.P
+    value = w.value.size * value_elem
+    offsets_logits_per_query = S * 3 * 4
+    ref_per_row = w.R * 2 * 4
+    out_row = w.H * 32 * 4
+    gather = (value + hit_queries * offsets_logits_per_query + rows * ref_per_row + rows * 4
+              + rows * out_row)
+    step = (value + w.B * w.Nq * offsets_logits_per_query + w.reference_points.nbytes
+            + w.bev_mask.nbytes + w.B * w.Nq * out_row)
+    return {"gather": int(gather), "step": int(step)}
+
+
+def aggregate(local_ms_total, local_samples, world):
+    """Job time = max over ranks of the summed device time; work = sum."""
+    if world == 1:
+        return local_ms_total, local_samples
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([local_ms_total], dtype=torch.float64, device=dev)
+    n = torch.tensor([float(local_samples)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(n, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(n.item())
+
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured (MEASURED_PEAKS.json hbm_gbs, copy burst)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s pool measurement)"
+
+
+def kernel_source_digest():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(value_dtype):
+    """DRAM bytes per gather launch from the committed ncu summary, when it
+    was taken on the current kernel sources; None otherwise."""
+    try:
+        text = open(PROFILE_TRAFFIC).read()
+    except OSError:
+        return None
+    m = re.search(r"kernel_sources_sha256_16:\s*([0-9a-f]+)", text)
+    t = re.search(rf"traffic_bytes_per_launch_{value_dtype}:\s*([0-9]+)", text)
+    if not m or not t or m.group(1) != kernel_source_digest():
+        return None
+    return int(t.group(1))
+
+
+class ClockSampler:
+    """SM clock and clock-event reasons sampled through NVML every few
+    milliseconds while the timed region runs (a background thread)."""
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, torch_device):
+        import threading
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.stop_flag = threading.Event()
+        self.thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = self._handle(torch_device)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.handle,
+                                                                  pynvml.NVML_CLOCK_SM))
+        except Exception:
+            self.nvml = None
+
+    def _handle(self, dev):
+        import torch
+        pynvml = self.nvml
+        p = torch.cuda.get_device_properties(dev)
+        try:
+            bus = "%08x:%02x:%02x.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+            return pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(dev)
+
+    def _run(self):
+        pynvml = self.nvml
+        get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.stop_flag.is_set():
+            try:
+                self.samples.append(float(pynvml.nvmlDeviceGetClockInfo(self.handle,
+                                                                        pynvml.NVML_CLOCK_SM)))
+                bits = get_reasons(self.handle)
+                for b, name in self.REASONS.items():
+                    if bits & b:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            self.stop_flag.wait(0.005)
+
+    def start(self):
+        if self.nvml is None:
+            return
+        import threading
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+
+    def stop(self):
+        if self.thread is None:
+            return None
+        self.stop_flag.set()
+        self.thread.join()
+        if not self.samples:
+            return None
+        return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples),
+                "source": "NVML, every 5 ms during the timed steps"}
+
+
+# --------------------------------------------------------------------------
+# CPU baseline: the oracle as it stands, one host core
+# --------------------------------------------------------------------------
+
+def oracle_step(w, n_queries):
+    """One oracle SCA forward over the first n_queries BEV queries of the
+    workload (all cameras, full value maps). Returns sampled points."""
+    import oracle
+    q = slice(0, n_queries)
+    out = oracle.sca_forward(w.value, w.spatial_shapes, w.level_start_index,
+                             np.ascontiguousarray(w.reference_points[:, :, q]),
+                             np.ascontiguousarray(w.bev_mask[:, :, q]),
+                             np.ascontiguousarray(w.sampling_offsets[:, q]),
+                             np.ascontiguousarray(w.attention_logits[:, q]))
+    assert out.shape[1] == n_queries
+    rows = int(np.count_nonzero(w.bev_mask[:, :, q].any(-1)))
+    return rows * w.H * w.L * w.P
+
+
+def cpu_baseline(w, min_seconds):
+    done, samples, t0 = 0, 0, time.perf_counter()
+    while True:
+        samples += oracle_step(w, w.Nq)
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds:
+            break
+    return {"value": samples / el / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{done} full workload pass(es) of the C oracle (double), "
+                      f"{el:.1f} s on one host core"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from scale_deformable_attention_03_b200 import inputs
+    from oracle import build as oracle_build
+    oracle_build.build()
+    w = inputs.workload3(seed=rank_seed(0), value_dtype=args.value_dtype, rho=args.rho)
+    t0 = time.perf_counter()
+    oracle_step(w, w.Nq)
+    t_full = time.perf_counter() - t0
+    budget = 150.0  # seconds for warm-up + timed steps
+    frac = min(1.0, budget / max(1e-9, (args.steps + args.warmup) * t_full))
+    nq = max(200, int(w.Nq * frac) // 200 * 200)  # whole BEV rows of 200 cells
+    for _ in range(args.warmup):
+        oracle_step(w, nq)
+    samples, t0 = 0, time.perf_counter()
+    for _ in range(args.steps):
+        samples += oracle_step(w, nq)
+    el = time.perf_counter() - t0
+    value = samples / el / 1e9
+    sample = (f"first {nq} of {w.Nq} BEV queries per step (all 6 cameras, full value maps), "
+              f"C oracle in double on one host core")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(args),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------
+# native arm
+# --------------------------------------------------------------------------
+
+def run_native(args):
+    import torch
+    import torch.distributed as dist
+
+    import scale_deformable_attention_03_b200 as msda
+    from scale_deformable_attention_03_b200 import inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    msda.lib()  # fail loudly before any work when the library is missing
+    stream = torch.cuda.current_stream()
+
+    w = inputs.workload3(seed=rank_seed(rank), value_dtype=args.value_dtype, rho=args.rho)
+    bf16 = args.value_dtype == "bf16"
+
+    def d(a):
+        return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+    value = d(w.value_bf16.view(np.int16)).view(torch.bfloat16) if bf16 else d(w.value)
+    ref, mask = d(w.reference_points), d(w.bev_mask)
+    off, logits = d(w.sampling_offsets), d(w.attention_logits)
+    shapes, starts = w.spatial_shapes, w.level_start_index
+    dims = msda.Dims(w.B, w.Ncam, w.Nq, w.Nv, w.H, w.L, w.P, w.R)
+    cws = torch.empty(max(16, msda.sca_compact_workspace_size(dims)), dtype=torch.uint8,
+                      device="cuda")
+    idx = torch.empty((w.B, w.Ncam, w.Nq), dtype=torch.int32, device="cuda")
+    count = torch.empty((w.B, w.Ncam), dtype=torch.int32, device="cuda")
+    pos = torch.empty_like(idx)
+    hits = torch.empty((w.B, w.Nq), dtype=torch.int32, device="cuda")
+    out_rb = torch.empty((w.B, w.Ncam, w.Nq, w.H * 32), dtype=torch.float32, device="cuda")
+    out = torch.empty((w.B, w.Nq, w.H * 32), dtype=torch.float32, device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    L = msda.lib()
+    i64 = msda._i64p
+    vdt = msda.MSDA_BF16 if bf16 else msda.MSDA_F32
+    sp, st = shapes.ctypes.data_as(i64), starts.ctypes.data_as(i64)
+    P = msda._ptr
+    sptr = msda._stream(stream)
+
+    def compact():
+        msda._check(L.sca_compact(P(mask), dims, P(cws), cws.numel(), P(idx), P(count), P(pos),
+                                  P(hits), sptr), "sca_compact")
+
+    def gather():
+        msda._check(L.sca_rebatched_forward(P(value), vdt, sp, st, P(ref), P(off), P(logits),
+                                            P(idx), P(count), dims, P(out_rb), sptr),
+                    "sca_rebatched_forward")
+
+    def average():
+        msda._check(L.sca_camera_average(P(out_rb), P(pos), P(hits), dims, P(out), sptr),
+                    "sca_camera_average")
+
+    launches_per_step = 4  # two compaction kernels, the gather, the average
+    compact()
+    torch.cuda.synchronize()
+    rows = int(count.sum().item())
+    hit_queries = int((hits > 0).sum().item())
+    samples_per_step = rows * w.H * w.L * w.P
+    nbytes = algorithmic_bytes(w, rows, hit_queries, 2 if bf16 else 4)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        compact()
+        gather()
+        average()
+    torch.cuda.synchronize()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+    for e in evs:
+        flush.zero_()
+        e[0].record(stream)
+        compact()
+        e[1].record(stream)
+        gather()
+        e[2].record(stream)
+        average()
+        e[3].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    gather_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    compact_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    avg_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    total_ms, total_samples = aggregate(sum(step_ms), samples_per_step * args.steps, world)
+    value_gs = total_samples / (total_ms * 1e-3) / 1e9
+
+    # ---- end to end through the one-call C ABI, host buffers ----
+    host = {k: torch.from_numpy(np.ascontiguousarray(a)).pin_memory() for k, a in (
+        ("value", w.value_bf16.view(np.int16) if bf16 else w.value),
+        ("ref", w.reference_points), ("mask", w.bev_mask), ("off", w.sampling_offsets),
+        ("logits", w.attention_logits))}
+    host_out = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+    ws = torch.empty(msda.msda_workspace_size(dims), dtype=torch.uint8, device="cuda")
+    dev_in = {k: torch.empty(v.shape, dtype=v.dtype, device="cuda") for k, v in host.items()}
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = host_out.numel() * 4
+
+    def e2e_step():
+        for k in host:
+            dev_in[k].copy_(host[k], non_blocking=True)
+        v = dev_in["value"].view(torch.bfloat16) if bf16 else dev_in["value"]
+        msda._check(L.sca_forward(P(v), vdt, sp, st, P(dev_in["ref"]), P(dev_in["mask"]),
+                                  P(dev_in["off"]), P(dev_in["logits"]), dims, P(ws), ws.numel(),
+                                  P(out), sptr), "sca_forward")
+        host_out.copy_(out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms, e2e_samples = aggregate(e0.elapsed_time(e1), samples_per_step * args.e2e_steps, world)
+    e2e_gs = e2e_samples / (e2e_ms * 1e-3) / 1e9
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peak, peak_src = measured_hbm_peak()
+    g_ms = float(np.mean(gather_ms))
+    achieved = nbytes["gather"] / (g_ms * 1e-3) / 1e9
+    traffic = recorded_traffic(args.value_dtype)
+    step_mean = float(np.mean(step_ms))
+    line = {
+        "metric": METRIC, "value": value_gs, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "config": workload_config(args),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "kernel": "sca_gather_kernel", "peak_source": peak_src,
+                     "algorithmic_bytes_per_launch": nbytes["gather"],
+                     "launch_ms": g_ms},
+        "step": {"algorithmic_bytes": nbytes["step"],
+                 "hbm_gbs": nbytes["step"] / (step_mean * 1e-3) / 1e9,
+                 "hbm_frac": nbytes["step"] / (step_mean * 1e-3) / 1e9 / peak,
+                 "ms": {"compact": float(np.mean(compact_ms)), "gather": g_ms,
+                        "average": float(np.mean(avg_ms)), "step": step_mean},
+                 "samples": samples_per_step, "rebatched_rows": rows},
+        "e2e": {"value": e2e_gs, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h), "api": "sca_forward (one call)",
+                "steps": args.e2e_steps},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if world == 1:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.steps < 1 or args.warmup < 3:
+        raise SystemExit("need --steps >= 1 and --warmup >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_native(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,244 @@
+/*
+ * msda.h - C ABI of libmsda.so: multi-scale deformable attention (MSDA) and
+ * BEVFormer Spatial Cross-Attention (SCA) on NVIDIA B200 (sm_100a).
+ *
+ * Sources of the operations (pages this library was written from):
+ *   [BQ]  "BEV(三) BEVFormer: how the Query interacts with the 8 Heads of the
+ *         Feature" (leheavengame.com repost of a CSDN article).
+ *   [SCA] "Spatial Cross-Attention" walkthrough, Tencent Cloud developer
+ *         article 2321140 (rebatch listing, scatter-add / average listing).
+ *
+ * What one MSDA output row computes ([BQ] sections 4.2, 5, 6, 8, 9):
+ *   alpha_{h,l,k} = softmax over the L*P logits of head h        (4.2)
+ *   s_{h,l,k}     = rho_{m(k)} + (dx / W_l, dy / H_l), m(k) = k mod R (5)
+ *   x = W_l s_x - 1/2, y = H_l s_y - 1/2; bilinear read of the 32-channel
+ *   head-h slice at (x, y), four neighbours, zero outside the map  (6)
+ *   g^(h) = sum_{l,k} alpha_{h,l,k} * read_{h,l,k};  out = concat_h g^(h) (8, 9)
+ * The corner decision (x, then floor) is made in IEEE binary32 with
+ * round-to-nearest and no fused multiply-add; a location with x <= -1,
+ * x >= W_l (same for y) or a non-finite coordinate reads nothing.
+ *
+ * Conventions of every call:
+ *   - Tensor pointers are caller-owned DEVICE memory, contiguous, row-major
+ *     in the shapes given.  spatial_shapes and level_start_index are HOST
+ *     arrays (read during the call, not kept).
+ *   - The library allocates no memory and keeps no pointer after returning.
+ *     The only state it holds is a per-thread error message and a per-device
+ *     cache of the SM count.
+ *   - Calls are asynchronous on `stream` (NULL = the legacy default stream).
+ *     The status covers argument checks and kernel launch errors; errors that
+ *     happen while the kernels run surface at the caller's next
+ *     synchronisation.  Nothing is launched when the arguments are rejected.
+ *   - Outputs are fully overwritten (including gradients and padded rows).
+ *   - Value rows: pixel (y, x) of level l is row level_start_index[l] +
+ *     y * W_l + x; a row holds H heads of MSDA_HEAD_DIM channels.
+ *     spatial_shapes[2*l] = H_l (rows), spatial_shapes[2*l+1] = W_l.
+ *   - Locations are (x, y), normalised to [0, 1] over the level's width and
+ *     height; offsets are (dx, dy) in pixels of the level they are read on.
+ *   - Alignment: value, out, grad_value and the workspace 16 bytes;
+ *     location, offset and reference-point arrays 8 bytes.
+ */
+#ifndef MSDA_H
+#define MSDA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MSDA_HEAD_DIM 32    /* channels per head */
+#define MSDA_MAX_LEVELS 8   /* L */
+#define MSDA_MAX_POINTS 16  /* P */
+#define MSDA_MAX_CAMERAS 32 /* Ncam */
+#define MSDA_MAX_BATCH_CAMERAS 1024 /* B * Ncam for the sca_* calls */
+
+struct CUstream_st;
+typedef struct CUstream_st* msda_stream_t; /* the same type as cudaStream_t */
+
+/* Problem sizes.  head_dim is fixed at MSDA_HEAD_DIM. */
+typedef struct {
+    int32_t B;    /* batch items (BEVFormer TSA: the two queues prev_bev, bev) */
+    int32_t Ncam; /* cameras (sca_* calls; ignored by msda_* calls) */
+    int32_t Nq;   /* queries per batch item (SCA: BEV queries) */
+    int32_t Nv;   /* value rows per batch item (and camera), >= every
+                     level_start_index[l] + H_l * W_l */
+    int32_t H;    /* heads; a value or output row has H * MSDA_HEAD_DIM channels */
+    int32_t L;    /* levels, 1 .. MSDA_MAX_LEVELS */
+    int32_t P;    /* points per (head, level), 1 .. MSDA_MAX_POINTS */
+    int32_t R;    /* reference anchors per query, divides P (m(k) = k mod R) */
+} msda_dims_t;
+
+typedef enum {
+    MSDA_F32 = 0, /* value stored as fp32 */
+    MSDA_BF16 = 1 /* value stored as bf16; arithmetic and outputs stay fp32 */
+} msda_dtype_t;
+
+typedef enum {
+    MSDA_OK = 0,
+    MSDA_ERR_INVALID_ARG = 1, /* null pointer, bad size, bad alignment, inconsistent levels */
+    MSDA_ERR_UNSUPPORTED = 2, /* outside the compiled limits (L, P, Ncam, index range) */
+    MSDA_ERR_WORKSPACE = 3,   /* workspace missing or smaller than msda_workspace_size() */
+    MSDA_ERR_CUDA = 4         /* a CUDA runtime call or kernel launch failed */
+} msda_status_t;
+
+/* MSDA forward from given sampling locations and attention weights
+ * ([BQ] 6, 8, 9 and the operator inputs of 18.5).
+ *   value              [B, Nv, H, 32]       fp32 or bf16 (vdt)
+ *   sampling_locations [B, Nq, H, L, P, 2]  fp32, (x, y) normalised
+ *   attention_weights  [B, Nq, H, L, P]     fp32, used as given (normally
+ *                                           already softmax-normalised)
+ *   out                [B, Nq, H * 32]      fp32, written */
+msda_status_t msda_forward(const void* value, msda_dtype_t vdt,
+                           const int64_t* spatial_shapes, const int64_t* level_start_index,
+                           const float* sampling_locations, const float* attention_weights,
+                           msda_dims_t d, float* out, msda_stream_t stream);
+
+/* MSDA forward fused with its producers: softmax of the logits ([BQ] 4.2),
+ * location from reference points and pixel offsets ([BQ] 5, 18.4), then the
+ * read and weighted sum of msda_forward.  One kernel.
+ *   reference_points  [B, Nq, R, 2]        fp32, (x, y) normalised
+ *   sampling_offsets  [B, Nq, H, L, P, 2]  fp32, level pixels
+ *   attention_logits  [B, Nq, H, L, P]     fp32
+ *   out               [B, Nq, H * 32]      fp32, written */
+msda_status_t msda_forward_fused(const void* value, msda_dtype_t vdt,
+                                 const int64_t* spatial_shapes, const int64_t* level_start_index,
+                                 const float* reference_points, const float* sampling_offsets,
+                                 const float* attention_logits, msda_dims_t d, float* out,
+                                 msda_stream_t stream);
+
+/* MSDA backward: the derivative of msda_forward (the pages give no backward;
+ * this is the analytic derivative of [BQ] 6 and 8).
+ *   grad_out                [B, Nq, H * 32]      fp32
+ *   grad_value              [B, Nv, H, 32]       fp32, written (zeroed, then
+ *                                                accumulated with atomics:
+ *                                                the summation order varies)
+ *   grad_sampling_locations [B, Nq, H, L, P, 2]  fp32, written
+ *   grad_attention_weights  [B, Nq, H, L, P]     fp32, written
+ * At an integer pixel coordinate the derivative is that of the cell floor()
+ * selects; a location that reads nothing has zero gradients. */
+msda_status_t msda_backward(const void* value, msda_dtype_t vdt,
+                            const int64_t* spatial_shapes, const int64_t* level_start_index,
+                            const float* sampling_locations, const float* attention_weights,
+                            const float* grad_out, msda_dims_t d, float* grad_value,
+                            float* grad_sampling_locations, float* grad_attention_weights,
+                            msda_stream_t stream);
+
+/* Bytes of device workspace sca_forward / sca_backward need for these
+ * sizes: the compaction lists and, for the forward, the rebatched rows
+ * (B * Ncam * Nq * H * 32 floats, of which only the seeing rows are used). */
+size_t msda_workspace_size(msda_dims_t d);
+
+/* Bytes of device workspace sca_compact needs (per-chunk counts and the
+ * per-(batch, camera) row offsets, a few KB). */
+size_t sca_compact_workspace_size(msda_dims_t d);
+
+/* SCA mask compaction ([SCA] rebatch listing; counts of the average listing).
+ * A camera c sees query q of batch item b when any of its R anchors is set.
+ *   bev_mask  [Ncam, B, Nq, R] uint8 (0 = not visible)
+ *   workspace >= sca_compact_workspace_size(d) bytes of device memory,
+ *             caller-owned, contents ignored and overwritten
+ *   idx       [B, Ncam, Nq] int32: the seeing queries in ascending order, then -1
+ *   count     [B, Ncam]     int32: number of seeing queries
+ *   pos       [B, Ncam, Nq] int32: rank of q in idx, -1 when not seen
+ *   hits      [B, Nq]       int32: number of cameras seeing q
+ * Bit-exact and deterministic; no host synchronisation. */
+msda_status_t sca_compact(const uint8_t* bev_mask, msda_dims_t d, void* workspace,
+                          size_t workspace_bytes, int32_t* idx, int32_t* count, int32_t* pos,
+                          int32_t* hits, msda_stream_t stream);
+
+/* SCA, stage 2 ([SCA] rebatch listing and MSDA call; [BQ] 10): the fused
+ * MSDA of every camera's seeing queries, on the compaction of sca_compact.
+ * Row i of camera c of batch item b reads BEV query q = idx[b, c, i]: its
+ * offsets and logits (shared by every camera, [BQ] 10) and camera c's
+ * reference points of q.  All rows of the batch and all cameras run in one
+ * persistent kernel; the row counts are read on the device.
+ *   value                [B, Ncam, Nv, H, 32]   fp32 or bf16
+ *   reference_points_cam [Ncam, B, Nq, R, 2]    fp32
+ *   sampling_offsets     [B, Nq, H, L, P, 2]    fp32, level pixels
+ *   attention_logits     [B, Nq, H, L, P]       fp32
+ *   idx, count           from sca_compact
+ *   out_rb               [B, Ncam, Nq, H * 32]  fp32; rows < count[b, c]
+ *                        written, the others left untouched */
+msda_status_t sca_rebatched_forward(const void* value, msda_dtype_t vdt,
+                                    const int64_t* spatial_shapes,
+                                    const int64_t* level_start_index,
+                                    const float* reference_points_cam,
+                                    const float* sampling_offsets, const float* attention_logits,
+                                    const int32_t* idx, const int32_t* count, msda_dims_t d,
+                                    float* out_rb, msda_stream_t stream);
+
+/* SCA, stage 3 ([SCA] scatter-add and clamp(count, 1) listing; [BQ] 10):
+ *   out[b, q] = (sum over c with pos[b, c, q] >= 0, ascending c, of
+ *                out_rb[b, c, pos[b, c, q]]) / max(1, hits[b, q]).
+ * A gather (one thread per 16 bytes of output), no atomics: deterministic.
+ *   out_rb [B, Ncam, Nq, H * 32]; pos, hits from sca_compact;
+ *   out    [B, Nq, H * 32] fp32, written */
+msda_status_t sca_camera_average(const float* out_rb, const int32_t* pos, const int32_t* hits,
+                                 msda_dims_t d, float* out, msda_stream_t stream);
+
+/* SCA forward ([BQ] 10; [SCA] listings): sca_compact, sca_rebatched_forward
+ * and sca_camera_average in one call, with the lists and the rebatched rows
+ * in the caller's workspace.  A query no camera sees gets 0.
+ *   value                [B, Ncam, Nv, H, 32]   fp32 or bf16
+ *   reference_points_cam [Ncam, B, Nq, R, 2]    fp32
+ *   bev_mask             [Ncam, B, Nq, R]       uint8
+ *   sampling_offsets     [B, Nq, H, L, P, 2]    fp32, level pixels
+ *   attention_logits     [B, Nq, H, L, P]       fp32
+ *   workspace            >= msda_workspace_size(d) bytes of device memory,
+ *                        caller-owned, contents ignored and overwritten
+ *   out                  [B, Nq, H * 32]        fp32, written */
+msda_status_t sca_forward(const void* value, msda_dtype_t vdt,
+                          const int64_t* spatial_shapes, const int64_t* level_start_index,
+                          const float* reference_points_cam, const uint8_t* bev_mask,
+                          const float* sampling_offsets, const float* attention_logits,
+                          msda_dims_t d, void* workspace, size_t workspace_bytes, float* out,
+                          msda_stream_t stream);
+
+/* SCA backward on a given compaction: derivative of sca_forward with respect
+ * to the value and to the per-camera (rebatched) sampling locations and
+ * attention weights.  The upstream gradient of row i of camera c is
+ * grad_out[b, idx[b, c, i]] / max(1, hits[b, idx[b, c, i]]).
+ *   grad_out                   [B, Nq, H * 32]              fp32
+ *   idx, count, hits           from sca_compact
+ *   grad_value                 [B, Ncam, Nv, H, 32]         fp32, written
+ *                                                           (atomics)
+ *   grad_sampling_locations_rb [B, Ncam, Nq, H, L, P, 2]    fp32, written;
+ *   grad_attention_weights_rb  [B, Ncam, Nq, H, L, P]       fp32, written;
+ *                              rows >= count[b, c] are zero */
+msda_status_t sca_rebatched_backward(const void* value, msda_dtype_t vdt,
+                                     const int64_t* spatial_shapes,
+                                     const int64_t* level_start_index,
+                                     const float* reference_points_cam,
+                                     const float* sampling_offsets,
+                                     const float* attention_logits, const float* grad_out,
+                                     const int32_t* idx, const int32_t* count,
+                                     const int32_t* hits, msda_dims_t d, float* grad_value,
+                                     float* grad_sampling_locations_rb,
+                                     float* grad_attention_weights_rb, msda_stream_t stream);
+
+/* SCA backward: sca_compact then sca_rebatched_backward, the lists in the
+ * caller's workspace (>= msda_workspace_size(d) bytes).  Outputs as above. */
+msda_status_t sca_backward(const void* value, msda_dtype_t vdt,
+                           const int64_t* spatial_shapes, const int64_t* level_start_index,
+                           const float* reference_points_cam, const uint8_t* bev_mask,
+                           const float* sampling_offsets, const float* attention_logits,
+                           const float* grad_out, msda_dims_t d, void* workspace,
+                           size_t workspace_bytes, float* grad_value,
+                           float* grad_sampling_locations_rb, float* grad_attention_weights_rb,
+                           msda_stream_t stream);
+
+/* Fixed text for a status code. */
+const char* msda_status_string(msda_status_t status);
+
+/* Detail of the last failure on the calling thread ("" after a success). */
+const char* msda_last_error(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int32_t msda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MSDA_H */

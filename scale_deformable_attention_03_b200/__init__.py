@@ -1,1 +1,359 @@
-"""B200-native multi-scale deformable attention (placeholder; binding below)."""
+"""B200-native multi-scale deformable attention (MSDA) and BEVFormer Spatial
+Cross-Attention (SCA).
+
+The compute lives in ``libmsda.so`` (hand-written sm_100a CUDA kernels behind
+the C ABI of ``include/msda.h``).  This module only marshals arguments: it
+reads shapes and device pointers from torch tensors, allocates outputs with
+torch, passes the current CUDA stream and raises ``MsdaError`` on a non-zero
+status.  There is no fallback: without the built library every call raises.
+
+Functions (same names as the C ABI): ``msda_forward``, ``msda_forward_fused``,
+``msda_backward``, ``sca_compact``, ``sca_rebatched_forward``,
+``sca_camera_average``, ``sca_forward``, ``sca_rebatched_backward``,
+``sca_backward``, ``msda_workspace_size``, ``sca_compact_workspace_size``.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+HEAD_DIM = 32
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmsda.so")
+
+MSDA_F32, MSDA_BF16 = 0, 1
+
+
+class MsdaError(RuntimeError):
+    pass
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("B", "Ncam", "Nq", "Nv", "H", "L", "P", "R")]
+
+
+_lib = None
+_vp = ctypes.c_void_p
+_i64p = ctypes.POINTER(ctypes.c_int64)
+
+
+def lib():
+    """The loaded libmsda.so (raises MsdaError when it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise MsdaError(f"{LIB_PATH} is missing: build it with "
+                            "`python -m scale_deformable_attention_03_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        st = ctypes.c_int
+        L.msda_forward.argtypes = [_vp, st, _i64p, _i64p, _vp, _vp, Dims, _vp, _vp]
+        L.msda_forward_fused.argtypes = [_vp, st, _i64p, _i64p, _vp, _vp, _vp, Dims, _vp, _vp]
+        L.msda_backward.argtypes = [_vp, st, _i64p, _i64p, _vp, _vp, _vp, Dims, _vp, _vp, _vp, _vp]
+        L.msda_workspace_size.argtypes = [Dims]
+        L.msda_workspace_size.restype = ctypes.c_size_t
+        L.sca_compact_workspace_size.argtypes = [Dims]
+        L.sca_compact_workspace_size.restype = ctypes.c_size_t
+        L.sca_compact.argtypes = [_vp, Dims, _vp, ctypes.c_size_t, _vp, _vp, _vp, _vp, _vp]
+        L.sca_forward.argtypes = [_vp, st, _i64p, _i64p, _vp, _vp, _vp, _vp, Dims, _vp,
+                                  ctypes.c_size_t, _vp, _vp]
+        L.sca_backward.argtypes = [_vp, st, _i64p, _i64p, _vp, _vp, _vp, _vp, _vp, Dims, _vp,
+                                   ctypes.c_size_t, _vp, _vp, _vp, _vp]
+        L.sca_rebatched_forward.argtypes = [_vp, st, _i64p, _i64p, _vp, _vp, _vp, _vp, _vp, Dims,
+                                            _vp, _vp]
+        L.sca_camera_average.argtypes = [_vp, _vp, _vp, Dims, _vp, _vp]
+        L.sca_rebatched_backward.argtypes = [_vp, st, _i64p, _i64p, _vp, _vp, _vp, _vp, _vp, _vp,
+                                             _vp, Dims, _vp, _vp, _vp, _vp]
+        for f in ("msda_forward", "msda_forward_fused", "msda_backward", "sca_compact",
+                  "sca_forward", "sca_backward", "sca_rebatched_forward", "sca_camera_average",
+                  "sca_rebatched_backward"):
+            getattr(L, f).restype = ctypes.c_int
+        L.msda_status_string.argtypes = [ctypes.c_int]
+        L.msda_status_string.restype = ctypes.c_char_p
+        L.msda_last_error.restype = ctypes.c_char_p
+        L.msda_version.restype = ctypes.c_int32
+        _lib = L
+    return _lib
+
+
+def _check(status, name):
+    if status != 0:
+        L = lib()
+        raise MsdaError(f"{name}: {L.msda_status_string(status).decode()}: "
+                        f"{L.msda_last_error().decode()}")
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    torch = _torch()
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _levels(spatial_shapes, level_start_index):
+    """Host int64 copies of the level tables (kept alive by the caller)."""
+    torch = _torch()
+
+    def host(a):
+        if isinstance(a, torch.Tensor):
+            a = a.detach().cpu().numpy()
+        return np.ascontiguousarray(np.asarray(a, dtype=np.int64))
+    shapes = host(spatial_shapes).reshape(-1, 2)
+    if level_start_index is None:
+        sizes = shapes[:, 0] * shapes[:, 1]
+        level_start_index = np.concatenate([[0], np.cumsum(sizes)[:-1]])
+    starts = host(level_start_index).reshape(-1)
+    return shapes, starts
+
+
+def _vdt(value):
+    torch = _torch()
+    if value.dtype == torch.float32:
+        return MSDA_F32
+    if value.dtype == torch.bfloat16:
+        return MSDA_BF16
+    raise MsdaError(f"value dtype {value.dtype} is not float32 or bfloat16")
+
+
+def _contig(*ts):
+    for t in ts:
+        if t is not None and not t.is_contiguous():
+            raise MsdaError("tensors must be contiguous")
+
+
+def msda_forward(value, spatial_shapes, level_start_index, sampling_locations,
+                 attention_weights, out=None, stream=None):
+    """value [B, Nv, H, 32] (f32/bf16); locations [B, Nq, H, L, P, 2];
+    weights [B, Nq, H, L, P] -> out [B, Nq, H*32] fp32."""
+    torch = _torch()
+    _contig(value, sampling_locations, attention_weights, out)
+    B, Nv, H, _ = value.shape
+    _, Nq, _, L, P, _ = sampling_locations.shape
+    shapes, starts = _levels(spatial_shapes, level_start_index)
+    if out is None:
+        out = torch.empty((B, Nq, H * HEAD_DIM), device=value.device, dtype=torch.float32)
+    d = Dims(B, 1, Nq, Nv, H, L, P, 1)
+    _check(lib().msda_forward(_ptr(value), _vdt(value), shapes.ctypes.data_as(_i64p),
+                              starts.ctypes.data_as(_i64p), _ptr(sampling_locations),
+                              _ptr(attention_weights), d, _ptr(out), _stream(stream)),
+           "msda_forward")
+    return out
+
+
+def msda_forward_fused(value, spatial_shapes, level_start_index, reference_points,
+                       sampling_offsets, attention_logits, out=None, stream=None):
+    """reference_points [B, Nq, R, 2]; offsets [B, Nq, H, L, P, 2] (level
+    pixels); logits [B, Nq, H, L, P] -> out [B, Nq, H*32] fp32."""
+    torch = _torch()
+    _contig(value, reference_points, sampling_offsets, attention_logits, out)
+    B, Nv, H, _ = value.shape
+    _, Nq, _, L, P, _ = sampling_offsets.shape
+    R = reference_points.shape[2]
+    shapes, starts = _levels(spatial_shapes, level_start_index)
+    if out is None:
+        out = torch.empty((B, Nq, H * HEAD_DIM), device=value.device, dtype=torch.float32)
+    d = Dims(B, 1, Nq, Nv, H, L, P, R)
+    _check(lib().msda_forward_fused(_ptr(value), _vdt(value), shapes.ctypes.data_as(_i64p),
+                                    starts.ctypes.data_as(_i64p), _ptr(reference_points),
+                                    _ptr(sampling_offsets), _ptr(attention_logits), d, _ptr(out),
+                                    _stream(stream)),
+           "msda_forward_fused")
+    return out
+
+
+def msda_backward(value, spatial_shapes, level_start_index, sampling_locations,
+                  attention_weights, grad_out, grad_value=None, grad_sampling_locations=None,
+                  grad_attention_weights=None, stream=None):
+    """-> (grad_value [B, Nv, H, 32] fp32, grad_sampling_locations,
+    grad_attention_weights)."""
+    torch = _torch()
+    _contig(value, sampling_locations, attention_weights, grad_out)
+    B, Nv, H, _ = value.shape
+    _, Nq, _, L, P, _ = sampling_locations.shape
+    shapes, starts = _levels(spatial_shapes, level_start_index)
+    dev = value.device
+    if grad_value is None:
+        grad_value = torch.empty(value.shape, device=dev, dtype=torch.float32)
+    if grad_sampling_locations is None:
+        grad_sampling_locations = torch.empty(sampling_locations.shape, device=dev,
+                                              dtype=torch.float32)
+    if grad_attention_weights is None:
+        grad_attention_weights = torch.empty(attention_weights.shape, device=dev,
+                                             dtype=torch.float32)
+    d = Dims(B, 1, Nq, Nv, H, L, P, 1)
+    _check(lib().msda_backward(_ptr(value), _vdt(value), shapes.ctypes.data_as(_i64p),
+                               starts.ctypes.data_as(_i64p), _ptr(sampling_locations),
+                               _ptr(attention_weights), _ptr(grad_out), d, _ptr(grad_value),
+                               _ptr(grad_sampling_locations), _ptr(grad_attention_weights),
+                               _stream(stream)),
+           "msda_backward")
+    return grad_value, grad_sampling_locations, grad_attention_weights
+
+
+def _sca_dims(value, sampling_offsets, reference_points_cam):
+    B, Ncam, Nv, H, _ = value.shape
+    _, Nq, _, L, P, _ = sampling_offsets.shape
+    R = reference_points_cam.shape[3]
+    return Dims(B, Ncam, Nq, Nv, H, L, P, R)
+
+
+def msda_workspace_size(dims):
+    return int(lib().msda_workspace_size(dims))
+
+
+def sca_compact_workspace_size(dims):
+    return int(lib().sca_compact_workspace_size(dims))
+
+
+def _workspace(nbytes, device, workspace):
+    torch = _torch()
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+    return workspace
+
+
+def sca_compact(bev_mask, workspace=None, stream=None):
+    """bev_mask [Ncam, B, Nq, R] (uint8 / bool) -> (idx [B, Ncam, Nq],
+    count [B, Ncam], pos [B, Ncam, Nq], hits [B, Nq]), int32."""
+    torch = _torch()
+    _contig(bev_mask)
+    if bev_mask.dtype == torch.bool:
+        bev_mask = bev_mask.view(torch.uint8)
+    Ncam, B, Nq, R = bev_mask.shape
+    dev = bev_mask.device
+    idx = torch.empty((B, Ncam, Nq), dtype=torch.int32, device=dev)
+    count = torch.empty((B, Ncam), dtype=torch.int32, device=dev)
+    pos = torch.empty((B, Ncam, Nq), dtype=torch.int32, device=dev)
+    hits = torch.empty((B, Nq), dtype=torch.int32, device=dev)
+    d = Dims(B, Ncam, Nq, 1, 1, 1, 1, R)
+    nbytes = sca_compact_workspace_size(d)
+    workspace = _workspace(nbytes, dev, workspace)
+    _check(lib().sca_compact(_ptr(bev_mask), d, _ptr(workspace), workspace.numel(), _ptr(idx),
+                             _ptr(count), _ptr(pos), _ptr(hits), _stream(stream)),
+           "sca_compact")
+    return idx, count, pos, hits
+
+
+def sca_forward(value, spatial_shapes, level_start_index, reference_points_cam, bev_mask,
+                sampling_offsets, attention_logits, out=None, workspace=None, stream=None):
+    """value [B, Ncam, Nv, H, 32]; reference_points_cam [Ncam, B, Nq, R, 2];
+    bev_mask [Ncam, B, Nq, R]; offsets [B, Nq, H, L, P, 2]; logits
+    [B, Nq, H, L, P] -> out [B, Nq, H*32] fp32."""
+    torch = _torch()
+    _contig(value, reference_points_cam, bev_mask, sampling_offsets, attention_logits, out)
+    if bev_mask.dtype == torch.bool:
+        bev_mask = bev_mask.view(torch.uint8)
+    d = _sca_dims(value, sampling_offsets, reference_points_cam)
+    shapes, starts = _levels(spatial_shapes, level_start_index)
+    if out is None:
+        out = torch.empty((d.B, d.Nq, d.H * HEAD_DIM), device=value.device, dtype=torch.float32)
+    workspace = _workspace(msda_workspace_size(d), value.device, workspace)
+    _check(lib().sca_forward(_ptr(value), _vdt(value), shapes.ctypes.data_as(_i64p),
+                             starts.ctypes.data_as(_i64p), _ptr(reference_points_cam),
+                             _ptr(bev_mask), _ptr(sampling_offsets), _ptr(attention_logits), d,
+                             _ptr(workspace), workspace.numel(), _ptr(out), _stream(stream)),
+           "sca_forward")
+    return out
+
+
+def sca_backward(value, spatial_shapes, level_start_index, reference_points_cam, bev_mask,
+                 sampling_offsets, attention_logits, grad_out, grad_value=None,
+                 grad_sampling_locations_rb=None, grad_attention_weights_rb=None,
+                 workspace=None, stream=None):
+    """-> (grad_value [B, Ncam, Nv, H, 32], grad_sampling_locations_rb
+    [B, Ncam, Nq, H, L, P, 2], grad_attention_weights_rb [B, Ncam, Nq, H, L, P])."""
+    torch = _torch()
+    _contig(value, reference_points_cam, bev_mask, sampling_offsets, attention_logits, grad_out)
+    if bev_mask.dtype == torch.bool:
+        bev_mask = bev_mask.view(torch.uint8)
+    d = _sca_dims(value, sampling_offsets, reference_points_cam)
+    shapes, starts = _levels(spatial_shapes, level_start_index)
+    dev = value.device
+    if grad_value is None:
+        grad_value = torch.empty(value.shape, device=dev, dtype=torch.float32)
+    if grad_sampling_locations_rb is None:
+        grad_sampling_locations_rb = torch.empty((d.B, d.Ncam, d.Nq, d.H, d.L, d.P, 2),
+                                                 device=dev, dtype=torch.float32)
+    if grad_attention_weights_rb is None:
+        grad_attention_weights_rb = torch.empty((d.B, d.Ncam, d.Nq, d.H, d.L, d.P), device=dev,
+                                                dtype=torch.float32)
+    workspace = _workspace(msda_workspace_size(d), dev, workspace)
+    _check(lib().sca_backward(_ptr(value), _vdt(value), shapes.ctypes.data_as(_i64p),
+                              starts.ctypes.data_as(_i64p), _ptr(reference_points_cam),
+                              _ptr(bev_mask), _ptr(sampling_offsets), _ptr(attention_logits),
+                              _ptr(grad_out), d, _ptr(workspace), workspace.numel(),
+                              _ptr(grad_value), _ptr(grad_sampling_locations_rb),
+                              _ptr(grad_attention_weights_rb), _stream(stream)),
+           "sca_backward")
+    return grad_value, grad_sampling_locations_rb, grad_attention_weights_rb
+
+
+def sca_rebatched_forward(value, spatial_shapes, level_start_index, reference_points_cam,
+                          sampling_offsets, attention_logits, idx, count, out_rb=None,
+                          stream=None):
+    """Fused MSDA of every camera's seeing queries (idx, count from
+    sca_compact) -> out_rb [B, Ncam, Nq, H*32]; rows >= count untouched."""
+    torch = _torch()
+    _contig(value, reference_points_cam, sampling_offsets, attention_logits, idx, count, out_rb)
+    d = _sca_dims(value, sampling_offsets, reference_points_cam)
+    shapes, starts = _levels(spatial_shapes, level_start_index)
+    if out_rb is None:
+        out_rb = torch.empty((d.B, d.Ncam, d.Nq, d.H * HEAD_DIM), device=value.device,
+                             dtype=torch.float32)
+    _check(lib().sca_rebatched_forward(_ptr(value), _vdt(value), shapes.ctypes.data_as(_i64p),
+                                       starts.ctypes.data_as(_i64p), _ptr(reference_points_cam),
+                                       _ptr(sampling_offsets), _ptr(attention_logits), _ptr(idx),
+                                       _ptr(count), d, _ptr(out_rb), _stream(stream)),
+           "sca_rebatched_forward")
+    return out_rb
+
+
+def sca_camera_average(out_rb, pos, hits, out=None, stream=None):
+    """out[b, q] = sum over seeing cameras of out_rb rows / max(1, hits)."""
+    torch = _torch()
+    _contig(out_rb, pos, hits, out)
+    B, Ncam, Nq, C = out_rb.shape
+    if out is None:
+        out = torch.empty((B, Nq, C), device=out_rb.device, dtype=torch.float32)
+    d = Dims(B, Ncam, Nq, 1, C // HEAD_DIM, 1, 1, 1)
+    _check(lib().sca_camera_average(_ptr(out_rb), _ptr(pos), _ptr(hits), d, _ptr(out),
+                                    _stream(stream)),
+           "sca_camera_average")
+    return out
+
+
+def sca_rebatched_backward(value, spatial_shapes, level_start_index, reference_points_cam,
+                           sampling_offsets, attention_logits, grad_out, idx, count, hits,
+                           grad_value=None, grad_sampling_locations_rb=None,
+                           grad_attention_weights_rb=None, stream=None):
+    """Backward of sca_rebatched_forward + sca_camera_average on a given
+    compaction -> (grad_value, grad_sampling_locations_rb, grad_attention_weights_rb)."""
+    torch = _torch()
+    _contig(value, reference_points_cam, sampling_offsets, attention_logits, grad_out, idx, count,
+            hits)
+    d = _sca_dims(value, sampling_offsets, reference_points_cam)
+    shapes, starts = _levels(spatial_shapes, level_start_index)
+    dev = value.device
+    if grad_value is None:
+        grad_value = torch.empty(value.shape, device=dev, dtype=torch.float32)
+    if grad_sampling_locations_rb is None:
+        grad_sampling_locations_rb = torch.empty((d.B, d.Ncam, d.Nq, d.H, d.L, d.P, 2),
+                                                 device=dev, dtype=torch.float32)
+    if grad_attention_weights_rb is None:
+        grad_attention_weights_rb = torch.empty((d.B, d.Ncam, d.Nq, d.H, d.L, d.P), device=dev,
+                                                dtype=torch.float32)
+    _check(lib().sca_rebatched_backward(_ptr(value), _vdt(value), shapes.ctypes.data_as(_i64p),
+                                        starts.ctypes.data_as(_i64p), _ptr(reference_points_cam),
+                                        _ptr(sampling_offsets), _ptr(attention_logits),
+                                        _ptr(grad_out), _ptr(idx), _ptr(count), _ptr(hits), d,
+                                        _ptr(grad_value), _ptr(grad_sampling_locations_rb),
+                                        _ptr(grad_attention_weights_rb), _stream(stream)),
+           "sca_rebatched_backward")
+    return grad_value, grad_sampling_locations_rb, grad_attention_weights_rb

@@ -1,0 +1,489 @@
+// The C ABI of libmsda.so (declared in include/msda.h): argument validation,
+// workspace carving and kernel dispatch.  Host code only; no allocation.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "msda.h"
+#include "msda_launch.h"
+
+namespace {
+
+thread_local char g_error[512] = "";
+
+msda_status_t fail(msda_status_t code, const char* fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_error, sizeof(g_error), fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+msda_status_t ok()
+{
+    g_error[0] = '\0';
+    return MSDA_OK;
+}
+
+msda_status_t cuda_status(cudaError_t e, const char* where)
+{
+    if (e == cudaSuccess) return ok();
+    return fail(MSDA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+#define MSDA_CHECK(cond, code, ...)                                                              \
+    do {                                                                                         \
+        if (!(cond)) return fail(code, __VA_ARGS__);                                             \
+    } while (0)
+
+// Sizes common to every call; `sca` adds the camera checks.
+msda_status_t check_dims(const msda_dims_t& d, bool sca)
+{
+    MSDA_CHECK(d.B >= 0 && d.Nq >= 0, MSDA_ERR_INVALID_ARG, "B (%d) and Nq (%d) must be >= 0",
+               d.B, d.Nq);
+    MSDA_CHECK(d.Nv >= 1 && d.H >= 1, MSDA_ERR_INVALID_ARG, "Nv (%d) and H (%d) must be >= 1",
+               d.Nv, d.H);
+    MSDA_CHECK(d.L >= 1 && d.L <= MSDA_MAX_LEVELS, MSDA_ERR_UNSUPPORTED, "L = %d outside 1..%d",
+               d.L, MSDA_MAX_LEVELS);
+    MSDA_CHECK(d.P >= 1 && d.P <= MSDA_MAX_POINTS, MSDA_ERR_UNSUPPORTED, "P = %d outside 1..%d",
+               d.P, MSDA_MAX_POINTS);
+    MSDA_CHECK(d.R >= 1 && d.P % d.R == 0, MSDA_ERR_INVALID_ARG,
+               "R = %d must be >= 1 and divide P = %d", d.R, d.P);
+    // per-(batch, camera) value element offsets are 32-bit inside the kernels
+    MSDA_CHECK((int64_t)d.Nv * d.H * MSDA_HEAD_DIM <= INT32_MAX, MSDA_ERR_UNSUPPORTED,
+               "Nv * H * 32 = %lld exceeds the 32-bit index range",
+               (long long)d.Nv * d.H * MSDA_HEAD_DIM);
+    if (sca) {
+        MSDA_CHECK(d.Ncam >= 1 && d.Ncam <= MSDA_MAX_CAMERAS, MSDA_ERR_UNSUPPORTED,
+                   "Ncam = %d outside 1..%d", d.Ncam, MSDA_MAX_CAMERAS);
+        MSDA_CHECK((int64_t)d.B * d.Ncam * d.Nq <= INT32_MAX, MSDA_ERR_UNSUPPORTED,
+                   "B * Ncam * Nq exceeds the 32-bit row range");
+    }
+    return MSDA_OK;
+}
+
+msda_status_t check_levels(const msda_dims_t& d, const int64_t* shapes, const int64_t* starts,
+                           msda::Levels& lv)
+{
+    MSDA_CHECK(shapes != nullptr && starts != nullptr, MSDA_ERR_INVALID_ARG,
+               "spatial_shapes and level_start_index must be host arrays");
+    std::memset(&lv, 0, sizeof(lv));
+    for (int l = 0; l < d.L; ++l) {
+        const int64_t Hl = shapes[2 * l], Wl = shapes[2 * l + 1], st = starts[l];
+        MSDA_CHECK(Hl >= 1 && Wl >= 1 && Hl <= (1 << 24) && Wl <= (1 << 24), MSDA_ERR_INVALID_ARG,
+                   "level %d has shape %lld x %lld", l, (long long)Hl, (long long)Wl);
+        MSDA_CHECK(st >= 0 && st + Hl * Wl <= d.Nv, MSDA_ERR_INVALID_ARG,
+                   "level %d (start %lld, %lld x %lld) does not fit in Nv = %d", l, (long long)st,
+                   (long long)Hl, (long long)Wl, d.Nv);
+        lv.h[l] = (int)Hl;
+        lv.w[l] = (int)Wl;
+        lv.start[l] = (int)st;
+    }
+    return MSDA_OK;
+}
+
+msda_status_t check_value(const void* value, msda_dtype_t vdt)
+{
+    MSDA_CHECK(vdt == MSDA_F32 || vdt == MSDA_BF16, MSDA_ERR_INVALID_ARG, "unknown value dtype %d",
+               (int)vdt);
+    MSDA_CHECK(value != nullptr, MSDA_ERR_INVALID_ARG, "value is null");
+    MSDA_CHECK(aligned(value, 16), MSDA_ERR_INVALID_ARG, "value must be 16-byte aligned");
+    return MSDA_OK;
+}
+
+#define MSDA_TRY(expr)                                                                           \
+    do {                                                                                         \
+        msda_status_t st_ = (expr);                                                              \
+        if (st_ != MSDA_OK) return st_;                                                          \
+    } while (0)
+
+#define MSDA_PTR(p, align)                                                                       \
+    do {                                                                                         \
+        MSDA_CHECK((p) != nullptr, MSDA_ERR_INVALID_ARG, #p " is null");                         \
+        MSDA_CHECK(aligned((p), (align)), MSDA_ERR_INVALID_ARG,                                  \
+                   #p " must be " #align "-byte aligned");                                       \
+    } while (0)
+
+msda::Problem make_problem(const void* value, msda_dtype_t vdt, const msda_dims_t& d,
+                           const msda::Levels& lv)
+{
+    msda::Problem p;
+    p.value = value;
+    p.bf16 = vdt == MSDA_BF16;
+    p.B = d.B;
+    p.Ncam = d.Ncam;
+    p.Nq = d.Nq;
+    p.Nv = d.Nv;
+    p.H = d.H;
+    p.L = d.L;
+    p.P = d.P;
+    p.R = d.R;
+    p.lv = lv;
+    return p;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+}  // namespace
+
+namespace msda {
+
+int device_sm_count()
+{
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+            n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+size_t compact_scratch_bytes(int B, int Ncam, int Nq)
+{
+    const size_t nbc = (size_t)B * Ncam;
+    const size_t nchunks = Nq > 0 ? ((size_t)Nq + kCompactChunk - 1) / kCompactChunk : 1;
+    return align256(sizeof(int32_t) * nbc * nchunks);
+}
+
+CompactScratch compact_scratch_carve(void* base, int, int, int)
+{
+    CompactScratch c;
+    c.chunk_counts = static_cast<int32_t*>(base);
+    return c;
+}
+
+size_t sca_workspace_bytes(int B, int Ncam, int Nq, int H, bool with_rows)
+{
+    const size_t nbc = (size_t)B * Ncam;
+    size_t n = compact_scratch_bytes(B, Ncam, Nq);
+    n += align256(sizeof(int32_t) * nbc * Nq);        // idx
+    n += align256(sizeof(int32_t) * nbc * Nq);        // pos
+    n += align256(sizeof(int32_t) * nbc);             // count
+    n += align256(sizeof(int32_t) * (size_t)B * Nq);  // hits
+    if (with_rows) n += align256(sizeof(float) * nbc * Nq * (size_t)H * kHeadDim);
+    return n;
+}
+
+ScaWorkspace sca_workspace_carve(void* base, int B, int Ncam, int Nq, int H, bool with_rows)
+{
+    const size_t nbc = (size_t)B * Ncam;
+    const CompactScratch cs = compact_scratch_carve(base, B, Ncam, Nq);
+    char* p = static_cast<char*>(base) + compact_scratch_bytes(B, Ncam, Nq);
+    ScaWorkspace w;
+    w.chunk_counts = cs.chunk_counts;
+    w.idx = reinterpret_cast<int32_t*>(p);
+    p += align256(sizeof(int32_t) * nbc * Nq);
+    w.pos = reinterpret_cast<int32_t*>(p);
+    p += align256(sizeof(int32_t) * nbc * Nq);
+    w.count = reinterpret_cast<int32_t*>(p);
+    p += align256(sizeof(int32_t) * nbc);
+    w.hits = reinterpret_cast<int32_t*>(p);
+    p += align256(sizeof(int32_t) * (size_t)B * Nq);
+    w.out_rb = with_rows ? reinterpret_cast<float*>(p) : nullptr;
+    return w;
+}
+
+}  // namespace msda
+
+extern "C" {
+
+int32_t msda_version(void) { return 10000; }  // 1.0.0
+
+const char* msda_status_string(msda_status_t status)
+{
+    switch (status) {
+        case MSDA_OK: return "success";
+        case MSDA_ERR_INVALID_ARG: return "invalid argument";
+        case MSDA_ERR_UNSUPPORTED: return "unsupported size";
+        case MSDA_ERR_WORKSPACE: return "workspace missing or too small";
+        case MSDA_ERR_CUDA: return "CUDA error";
+    }
+    return "unknown status";
+}
+
+const char* msda_last_error(void) { return g_error; }
+
+msda_status_t msda_forward(const void* value, msda_dtype_t vdt, const int64_t* spatial_shapes,
+                           const int64_t* level_start_index, const float* sampling_locations,
+                           const float* attention_weights, msda_dims_t d, float* out,
+                           msda_stream_t stream)
+{
+    MSDA_TRY(check_dims(d, false));
+    msda::Levels lv;
+    MSDA_TRY(check_levels(d, spatial_shapes, level_start_index, lv));
+    MSDA_TRY(check_value(value, vdt));
+    if ((int64_t)d.B * d.Nq == 0) return ok();
+    MSDA_PTR(sampling_locations, 8);
+    MSDA_PTR(attention_weights, 4);
+    MSDA_PTR(out, 16);
+    const msda::Problem p = make_problem(value, vdt, d, lv);
+    return cuda_status(msda::launch_msda_forward(p, sampling_locations, attention_weights, out,
+                                                 (cudaStream_t)stream),
+                       "msda_forward");
+}
+
+msda_status_t msda_forward_fused(const void* value, msda_dtype_t vdt,
+                                 const int64_t* spatial_shapes, const int64_t* level_start_index,
+                                 const float* reference_points, const float* sampling_offsets,
+                                 const float* attention_logits, msda_dims_t d, float* out,
+                                 msda_stream_t stream)
+{
+    MSDA_TRY(check_dims(d, false));
+    msda::Levels lv;
+    MSDA_TRY(check_levels(d, spatial_shapes, level_start_index, lv));
+    MSDA_TRY(check_value(value, vdt));
+    if ((int64_t)d.B * d.Nq == 0) return ok();
+    MSDA_PTR(reference_points, 8);
+    MSDA_PTR(sampling_offsets, 8);
+    MSDA_PTR(attention_logits, 4);
+    MSDA_PTR(out, 16);
+    const msda::Problem p = make_problem(value, vdt, d, lv);
+    return cuda_status(msda::launch_msda_forward_fused(p, reference_points, sampling_offsets,
+                                                       attention_logits, out,
+                                                       (cudaStream_t)stream),
+                       "msda_forward_fused");
+}
+
+msda_status_t msda_backward(const void* value, msda_dtype_t vdt, const int64_t* spatial_shapes,
+                            const int64_t* level_start_index, const float* sampling_locations,
+                            const float* attention_weights, const float* grad_out, msda_dims_t d,
+                            float* grad_value, float* grad_sampling_locations,
+                            float* grad_attention_weights, msda_stream_t stream)
+{
+    MSDA_TRY(check_dims(d, false));
+    msda::Levels lv;
+    MSDA_TRY(check_levels(d, spatial_shapes, level_start_index, lv));
+    MSDA_TRY(check_value(value, vdt));
+    MSDA_PTR(grad_value, 16);
+    if ((int64_t)d.B * d.Nq > 0) {
+        MSDA_PTR(sampling_locations, 8);
+        MSDA_PTR(attention_weights, 4);
+        MSDA_PTR(grad_out, 16);
+        MSDA_PTR(grad_sampling_locations, 8);
+        MSDA_PTR(grad_attention_weights, 4);
+    }
+    const cudaStream_t s = (cudaStream_t)stream;
+    const msda::Problem p = make_problem(value, vdt, d, lv);
+    cudaError_t e = msda::launch_zero(grad_value, (int64_t)d.B * d.Nv * d.H * MSDA_HEAD_DIM, s);
+    if (e == cudaSuccess)
+        e = msda::launch_msda_backward(p, sampling_locations, attention_weights, grad_out,
+                                       grad_value, grad_sampling_locations,
+                                       grad_attention_weights, s);
+    return cuda_status(e, "msda_backward");
+}
+
+size_t msda_workspace_size(msda_dims_t d)
+{
+    if (d.B < 0 || d.Ncam < 1 || d.Nq < 0 || d.H < 1) return 0;
+    return msda::sca_workspace_bytes(d.B, d.Ncam, d.Nq, d.H, true);
+}
+
+size_t sca_compact_workspace_size(msda_dims_t d)
+{
+    if (d.B < 0 || d.Ncam < 1 || d.Nq < 0) return 0;
+    return msda::compact_scratch_bytes(d.B, d.Ncam, d.Nq);
+}
+
+static msda_status_t check_compact(const msda_dims_t& d)
+{
+    MSDA_CHECK(d.B >= 0 && d.Nq >= 0, MSDA_ERR_INVALID_ARG, "B (%d) and Nq (%d) must be >= 0",
+               d.B, d.Nq);
+    MSDA_CHECK(d.Ncam >= 1 && d.Ncam <= MSDA_MAX_CAMERAS, MSDA_ERR_UNSUPPORTED,
+               "Ncam = %d outside 1..%d", d.Ncam, MSDA_MAX_CAMERAS);
+    MSDA_CHECK(d.R >= 1, MSDA_ERR_INVALID_ARG, "R = %d must be >= 1", d.R);
+    MSDA_CHECK((int64_t)d.B * d.Ncam <= MSDA_MAX_BATCH_CAMERAS, MSDA_ERR_UNSUPPORTED,
+               "B * Ncam = %lld exceeds %d", (long long)d.B * d.Ncam, MSDA_MAX_BATCH_CAMERAS);
+    MSDA_CHECK((int64_t)d.B * d.Ncam * d.Nq <= INT32_MAX, MSDA_ERR_UNSUPPORTED,
+               "B * Ncam * Nq exceeds the 32-bit row range");
+    return MSDA_OK;
+}
+
+static msda_status_t check_workspace(const void* ws, size_t have, size_t need)
+{
+    MSDA_CHECK(ws != nullptr && have >= need, MSDA_ERR_WORKSPACE,
+               "workspace %p of %zu bytes, %zu needed", ws, have, need);
+    MSDA_CHECK(aligned(ws, 16), MSDA_ERR_WORKSPACE, "workspace must be 16-byte aligned");
+    return MSDA_OK;
+}
+
+msda_status_t sca_compact(const uint8_t* bev_mask, msda_dims_t d, void* workspace,
+                          size_t workspace_bytes, int32_t* idx, int32_t* count, int32_t* pos,
+                          int32_t* hits, msda_stream_t stream)
+{
+    MSDA_TRY(check_compact(d));
+    if (d.B == 0) return ok();
+    MSDA_TRY(check_workspace(workspace, workspace_bytes,
+                             msda::compact_scratch_bytes(d.B, d.Ncam, d.Nq)));
+    MSDA_PTR(count, 4);
+    if (d.Nq > 0) {
+        MSDA_PTR(bev_mask, 1);
+        MSDA_PTR(idx, 4);
+        MSDA_PTR(pos, 4);
+        MSDA_PTR(hits, 4);
+    }
+    const msda::CompactScratch cs = msda::compact_scratch_carve(workspace, d.B, d.Ncam, d.Nq);
+    return cuda_status(msda::launch_sca_compact(bev_mask, d.B, d.Ncam, d.Nq, d.R, idx, count, pos,
+                                                hits, cs.chunk_counts, (cudaStream_t)stream),
+                       "sca_compact");
+}
+
+static msda_status_t check_sca_inputs(const void* value, msda_dtype_t vdt, const msda_dims_t& d,
+                                      const int64_t* spatial_shapes,
+                                      const int64_t* level_start_index,
+                                      const float* reference_points_cam,
+                                      const float* sampling_offsets,
+                                      const float* attention_logits, msda::Levels& lv)
+{
+    MSDA_TRY(check_dims(d, true));
+    MSDA_TRY(check_compact(d));
+    MSDA_TRY(check_levels(d, spatial_shapes, level_start_index, lv));
+    MSDA_TRY(check_value(value, vdt));
+    if ((int64_t)d.B * d.Nq > 0) {
+        MSDA_PTR(reference_points_cam, 8);
+        MSDA_PTR(sampling_offsets, 8);
+        MSDA_PTR(attention_logits, 4);
+    }
+    return MSDA_OK;
+}
+
+msda_status_t sca_rebatched_forward(const void* value, msda_dtype_t vdt,
+                                    const int64_t* spatial_shapes,
+                                    const int64_t* level_start_index,
+                                    const float* reference_points_cam,
+                                    const float* sampling_offsets, const float* attention_logits,
+                                    const int32_t* idx, const int32_t* count, msda_dims_t d,
+                                    float* out_rb, msda_stream_t stream)
+{
+    msda::Levels lv;
+    MSDA_TRY(check_sca_inputs(value, vdt, d, spatial_shapes, level_start_index,
+                              reference_points_cam, sampling_offsets, attention_logits, lv));
+    if ((int64_t)d.B * d.Nq == 0) return ok();
+    MSDA_PTR(idx, 4);
+    MSDA_PTR(count, 4);
+    MSDA_PTR(out_rb, 16);
+    const msda::Problem p = make_problem(value, vdt, d, lv);
+    return cuda_status(msda::launch_sca_gather(p, reference_points_cam, sampling_offsets,
+                                               attention_logits, idx, count, out_rb,
+                                               (cudaStream_t)stream),
+                       "sca_rebatched_forward");
+}
+
+msda_status_t sca_camera_average(const float* out_rb, const int32_t* pos, const int32_t* hits,
+                                 msda_dims_t d, float* out, msda_stream_t stream)
+{
+    MSDA_TRY(check_compact(d));
+    MSDA_CHECK(d.H >= 1, MSDA_ERR_INVALID_ARG, "H (%d) must be >= 1", d.H);
+    if ((int64_t)d.B * d.Nq == 0) return ok();
+    MSDA_PTR(out_rb, 16);
+    MSDA_PTR(pos, 4);
+    MSDA_PTR(hits, 4);
+    MSDA_PTR(out, 16);
+    return cuda_status(msda::launch_sca_average(out_rb, pos, hits, d.B, d.Ncam, d.Nq, d.H, out,
+                                                (cudaStream_t)stream),
+                       "sca_camera_average");
+}
+
+msda_status_t sca_forward(const void* value, msda_dtype_t vdt, const int64_t* spatial_shapes,
+                          const int64_t* level_start_index, const float* reference_points_cam,
+                          const uint8_t* bev_mask, const float* sampling_offsets,
+                          const float* attention_logits, msda_dims_t d, void* workspace,
+                          size_t workspace_bytes, float* out, msda_stream_t stream)
+{
+    msda::Levels lv;
+    MSDA_TRY(check_sca_inputs(value, vdt, d, spatial_shapes, level_start_index,
+                              reference_points_cam, sampling_offsets, attention_logits, lv));
+    if ((int64_t)d.B * d.Nq == 0) return ok();
+    MSDA_PTR(bev_mask, 1);
+    MSDA_PTR(out, 16);
+    MSDA_TRY(check_workspace(workspace, workspace_bytes,
+                             msda::sca_workspace_bytes(d.B, d.Ncam, d.Nq, d.H, true)));
+    const cudaStream_t s = (cudaStream_t)stream;
+    const msda::ScaWorkspace w = msda::sca_workspace_carve(workspace, d.B, d.Ncam, d.Nq, d.H, true);
+    const msda::Problem p = make_problem(value, vdt, d, lv);
+    cudaError_t e = msda::launch_sca_compact(bev_mask, d.B, d.Ncam, d.Nq, d.R, w.idx, w.count,
+                                             w.pos, w.hits, w.chunk_counts, s);
+    if (e == cudaSuccess)
+        e = msda::launch_sca_gather(p, reference_points_cam, sampling_offsets, attention_logits,
+                                    w.idx, w.count, w.out_rb, s);
+    if (e == cudaSuccess)
+        e = msda::launch_sca_average(w.out_rb, w.pos, w.hits, d.B, d.Ncam, d.Nq, d.H, out, s);
+    return cuda_status(e, "sca_forward");
+}
+
+msda_status_t sca_rebatched_backward(const void* value, msda_dtype_t vdt,
+                                     const int64_t* spatial_shapes,
+                                     const int64_t* level_start_index,
+                                     const float* reference_points_cam,
+                                     const float* sampling_offsets,
+                                     const float* attention_logits, const float* grad_out,
+                                     const int32_t* idx, const int32_t* count,
+                                     const int32_t* hits, msda_dims_t d, float* grad_value,
+                                     float* grad_sampling_locations_rb,
+                                     float* grad_attention_weights_rb, msda_stream_t stream)
+{
+    msda::Levels lv;
+    MSDA_TRY(check_sca_inputs(value, vdt, d, spatial_shapes, level_start_index,
+                              reference_points_cam, sampling_offsets, attention_logits, lv));
+    if (d.B == 0) return ok();
+    MSDA_PTR(grad_value, 16);
+    if (d.Nq > 0) {
+        MSDA_PTR(grad_out, 16);
+        MSDA_PTR(idx, 4);
+        MSDA_PTR(count, 4);
+        MSDA_PTR(hits, 4);
+        MSDA_PTR(grad_sampling_locations_rb, 8);
+        MSDA_PTR(grad_attention_weights_rb, 4);
+    }
+    const cudaStream_t s = (cudaStream_t)stream;
+    const msda::Problem p = make_problem(value, vdt, d, lv);
+    cudaError_t e = msda::launch_zero(grad_value,
+                                      (int64_t)d.B * d.Ncam * d.Nv * d.H * MSDA_HEAD_DIM, s);
+    if (e == cudaSuccess && d.Nq > 0)
+        e = msda::launch_sca_backward_rows(p, reference_points_cam, sampling_offsets,
+                                           attention_logits, grad_out, idx, hits, count,
+                                           grad_value, grad_sampling_locations_rb,
+                                           grad_attention_weights_rb, s);
+    if (e == cudaSuccess && d.Nq > 0)
+        e = msda::launch_sca_zero_tail(count, d.B, d.Ncam, d.Nq, d.H * d.L * d.P,
+                                       grad_sampling_locations_rb, grad_attention_weights_rb, s);
+    return cuda_status(e, "sca_rebatched_backward");
+}
+
+msda_status_t sca_backward(const void* value, msda_dtype_t vdt, const int64_t* spatial_shapes,
+                           const int64_t* level_start_index, const float* reference_points_cam,
+                           const uint8_t* bev_mask, const float* sampling_offsets,
+                           const float* attention_logits, const float* grad_out, msda_dims_t d,
+                           void* workspace, size_t workspace_bytes, float* grad_value,
+                           float* grad_sampling_locations_rb, float* grad_attention_weights_rb,
+                           msda_stream_t stream)
+{
+    msda::Levels lv;
+    MSDA_TRY(check_sca_inputs(value, vdt, d, spatial_shapes, level_start_index,
+                              reference_points_cam, sampling_offsets, attention_logits, lv));
+    if (d.B == 0) return ok();
+    if (d.Nq > 0) MSDA_PTR(bev_mask, 1);
+    MSDA_TRY(check_workspace(workspace, workspace_bytes,
+                             msda::sca_workspace_bytes(d.B, d.Ncam, d.Nq, d.H, false)));
+    const msda::ScaWorkspace w = msda::sca_workspace_carve(workspace, d.B, d.Ncam, d.Nq, d.H, false);
+    if (d.Nq > 0) {
+        const cudaError_t e = msda::launch_sca_compact(bev_mask, d.B, d.Ncam, d.Nq, d.R, w.idx,
+                                                       w.count, w.pos, w.hits, w.chunk_counts,
+                                                       (cudaStream_t)stream);
+        if (e != cudaSuccess) return cuda_status(e, "sca_backward");
+    }
+    return sca_rebatched_backward(value, vdt, spatial_shapes, level_start_index,
+                                  reference_points_cam, sampling_offsets, attention_logits,
+                                  grad_out, w.idx, w.count, w.hits, d, grad_value,
+                                  grad_sampling_locations_rb, grad_attention_weights_rb, stream);
+}
+
+}  // extern "C"

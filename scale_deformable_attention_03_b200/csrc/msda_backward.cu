@@ -1,0 +1,446 @@
+// MSDA / SCA backward: the analytic derivative of the forward read and sum
+// (the pages give no backward; it follows from "BEV(三) BEVFormer: how the
+// Query interacts with the 8 Heads of the Feature", sections 6 and 8).
+//   f = sum_g w_g V_g,  d out / d alpha = f,
+//   d f / d x = (1-ly)(V_10 - V_00) + ly (V_11 - V_01),
+//   d f / d y = (1-lx)(V_01 - V_00) + lx (V_11 - V_10),
+//   x = W s_x - 1/2  =>  d / d s_x = W * d / d x   (same for y with H),
+//   d out / d V_g = alpha w_g   (neighbours inside the map only).
+// One warp per (row, head) with the forward's lane layout.  For every sample
+// each lane forms dot_g = <grad_out, V_g> over its channels and adds
+// alpha w_g grad_out to grad_value with one 16-byte vector reduction
+// (red.global.add.v4.f32); the per-sample scalars are reduced with shuffles
+// and land on the lane that owns the sample, which writes them coalesced.
+#include <algorithm>
+
+#include "msda_launch.h"
+
+namespace msda {
+
+constexpr int kBwdRowsPerWarp = 1;
+
+struct BwdTable {
+    int off[4][kMetaStride];
+    float wb[4][kMetaStride];  // bilinear weight without alpha
+    float lx[kMetaStride];
+    float ly[kMetaStride];
+};
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d)
+{
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
+                 "f"(c), "f"(d)
+                 : "memory");
+}
+
+// d w_g / d lx and d w_g / d ly for neighbour g.
+__device__ __forceinline__ float dw_dlx(int g, float ly)
+{
+    const float a = (g >> 1) ? ly : 1.f - ly;
+    return (g & 1) ? a : -a;
+}
+__device__ __forceinline__ float dw_dly(int g, float lx)
+{
+    const float a = (g & 1) ? lx : 1.f - lx;
+    return (g >> 1) ? a : -a;
+}
+
+template <typename VT>
+struct BwdLanes;
+
+// fp32 value: lanes 8g..8g+7 hold corner g, channels 4t..4t+3.
+template <>
+struct BwdLanes<float> {
+    static constexpr int kSamplesPerStep = 1;
+    float4 go;
+    __device__ __forceinline__ void load_grad(const float* __restrict__ grow, float scale,
+                                              int lane)
+    {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(grow) + (lane & 7));
+        go = make_float4(v.x / scale, v.y / scale, v.z / scale, v.w / scale);
+    }
+    // partial dot for corner g of sample jj, plus the grad_value reduction
+    __device__ __forceinline__ float step(const float* __restrict__ vb, float* __restrict__ gvb,
+                                          const BwdTable& tab, int jj, bool valid, float alpha,
+                                          int lane)
+    {
+        const int g = lane >> 3, t = lane & 7;
+        const int o = valid ? tab.off[g][jj] : -1;
+        float d = 0.f;
+        if (o >= 0) {
+            const float4 v = __ldg(reinterpret_cast<const float4*>(vb + o + 4 * t));
+            d = go.x * v.x + go.y * v.y + go.z * v.z + go.w * v.w;
+            const float w = alpha * tab.wb[g][jj];
+            if (w != 0.f) red_add_v4(gvb + o + 4 * t, w * go.x, w * go.y, w * go.z, w * go.w);
+        }
+        d += __shfl_xor_sync(0xffffffffu, d, 1);
+        d += __shfl_xor_sync(0xffffffffu, d, 2);
+        d += __shfl_xor_sync(0xffffffffu, d, 4);
+        return d;  // <grad_out, V_g> in every lane of group g
+    }
+    __device__ __forceinline__ static int group(int lane) { return lane >> 3; }
+    __device__ __forceinline__ static float reduce_groups(float v)
+    {
+        v += __shfl_xor_sync(0xffffffffu, v, 8);
+        v += __shfl_xor_sync(0xffffffffu, v, 16);
+        return v;
+    }
+};
+
+// bf16 value: lanes 16s + 4g + t hold corner g of sample 2p + s, channels
+// 8t..8t+7.
+template <>
+struct BwdLanes<__nv_bfloat16> {
+    static constexpr int kSamplesPerStep = 2;
+    float go[8];
+    __device__ __forceinline__ void load_grad(const float* __restrict__ grow, float scale,
+                                              int lane)
+    {
+        const float4* g4 = reinterpret_cast<const float4*>(grow) + 2 * (lane & 3);
+        const float4 a = __ldg(g4), b = __ldg(g4 + 1);
+        go[0] = a.x / scale; go[1] = a.y / scale; go[2] = a.z / scale; go[3] = a.w / scale;
+        go[4] = b.x / scale; go[5] = b.y / scale; go[6] = b.z / scale; go[7] = b.w / scale;
+    }
+    __device__ __forceinline__ float step(const __nv_bfloat16* __restrict__ vb,
+                                          float* __restrict__ gvb, const BwdTable& tab, int jj,
+                                          bool valid, float alpha, int lane)
+    {
+        const int g = (lane >> 2) & 3, t = lane & 3;
+        const int o = valid ? tab.off[g][jj] : -1;
+        float d = 0.f;
+        if (o >= 0) {
+            const uint4 r = __ldg(reinterpret_cast<const uint4*>(vb + o + 8 * t));
+            float v[8];
+            bf16x2_to_f32(r.x, v[0], v[1]);
+            bf16x2_to_f32(r.y, v[2], v[3]);
+            bf16x2_to_f32(r.z, v[4], v[5]);
+            bf16x2_to_f32(r.w, v[6], v[7]);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) d += go[i] * v[i];
+            const float w = alpha * tab.wb[g][jj];
+            if (w != 0.f) {
+                float* dst = gvb + o + 8 * t;
+                red_add_v4(dst, w * go[0], w * go[1], w * go[2], w * go[3]);
+                red_add_v4(dst + 4, w * go[4], w * go[5], w * go[6], w * go[7]);
+            }
+        }
+        d += __shfl_xor_sync(0xffffffffu, d, 1);
+        d += __shfl_xor_sync(0xffffffffu, d, 2);
+        return d;
+    }
+    __device__ __forceinline__ static int group(int lane) { return (lane >> 2) & 3; }
+    __device__ __forceinline__ static float reduce_groups(float v)
+    {
+        v += __shfl_xor_sync(0xffffffffu, v, 4);
+        v += __shfl_xor_sync(0xffffffffu, v, 8);
+        return v;
+    }
+};
+
+// Backward of one (row, head).  grow: grad_out of the row's head (32 floats),
+// divided by `scale` (1 for MSDA, max(1, hits) for SCA).  gvb: grad_value of
+// the batch item (and camera).  gloc_row [L, P, 2], gattn_row [L, P].
+template <typename VT, bool FUSED, int NC>
+__device__ __forceinline__ void row_backward(const VT* __restrict__ vb, int H, int h,
+                                             const float* __restrict__ lo,
+                                             const float* __restrict__ wl,
+                                             const float* __restrict__ ref, int L, int P, int R,
+                                             const SmemLevels& lv, BwdTable& tab,
+                                             const float* __restrict__ grow, float scale,
+                                             float* __restrict__ gvb, float* __restrict__ gloc_row,
+                                             float* __restrict__ gattn_row, int lane)
+{
+    const int n = L * P;
+    float a[NC];
+    row_weights<FUSED, NC>(wl, n, lane, a);
+    BwdLanes<VT> lanes;
+    lanes.load_grad(grow, scale, lane);
+    const int g = BwdLanes<VT>::group(lane);
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+        const int j = c * 32 + lane;
+        Corners cr;
+        float Wl = 0.f, Hl = 0.f;
+        if (j < n) {
+            const int l = j / P, k = j - l * P;
+            const int hl = lv.h[l], wlv = lv.w[l];
+            float sx, sy;
+            sample_location<FUSED>(lo, ref, j, k, R, hl, wlv, sx, sy);
+            locate(sx, sy, hl, wlv, lv.start[l], H, h, cr);
+            Wl = (float)wlv;
+            Hl = (float)hl;
+        } else {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                cr.off[q] = -1;
+                cr.w[q] = 0.f;
+            }
+            cr.lx = cr.ly = 0.f;
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            tab.off[q][lane] = cr.off[q];
+            tab.wb[q][lane] = cr.w[q];
+        }
+        tab.lx[lane] = cr.lx;
+        tab.ly[lane] = cr.ly;
+        __syncwarp();
+        float res_w = 0.f, res_x = 0.f, res_y = 0.f;
+        const int cnt = min(32, n - c * 32);
+        for (int p = 0; p < cnt; p += BwdLanes<VT>::kSamplesPerStep) {
+            const int jraw = (BwdLanes<VT>::kSamplesPerStep == 2) ? p + (lane >> 4) : p;
+            const bool valid = jraw < cnt;
+            const int jj = valid ? jraw : 0;
+            // alpha of sample jj lives in lane jj
+            const float alpha = __shfl_sync(0xffffffffu, a[c], jj);
+            const float d = lanes.step(vb, gvb, tab, jj, valid, alpha, lane);
+            float cw = valid ? tab.wb[g][jj] * d : 0.f;
+            float cx = valid ? dw_dlx(g, tab.ly[jj]) * d : 0.f;
+            float cy = valid ? dw_dly(g, tab.lx[jj]) * d : 0.f;
+            cw = BwdLanes<VT>::reduce_groups(cw);
+            cx = BwdLanes<VT>::reduce_groups(cx);
+            cy = BwdLanes<VT>::reduce_groups(cy);
+            if (BwdLanes<VT>::kSamplesPerStep == 1) {
+                if (lane == p) {
+                    res_w = cw;
+                    res_x = cx;
+                    res_y = cy;
+                }
+            } else {
+                // sample p sits in half 0 (lane 0), sample p + 1 in half 1 (lane 16)
+                const int src = (lane & 1) << 4;
+                const float tw = __shfl_sync(0xffffffffu, cw, src);
+                const float tx = __shfl_sync(0xffffffffu, cx, src);
+                const float ty = __shfl_sync(0xffffffffu, cy, src);
+                if ((lane & ~1) == p) {
+                    res_w = tw;
+                    res_x = tx;
+                    res_y = ty;
+                }
+            }
+        }
+        if (j < n) {
+            gattn_row[j] = res_w;
+            const float al = a[c];
+            *reinterpret_cast<float2*>(gloc_row + 2 * j) =
+                make_float2(cr.valid ? al * Wl * res_x : 0.f, cr.valid ? al * Hl * res_y : 0.f);
+        }
+        __syncwarp();
+    }
+}
+
+template <typename VT, int NC>
+__global__ void __launch_bounds__(kThreads)
+msda_backward_kernel(const VT* __restrict__ value, const float* __restrict__ loc,
+                     const float* __restrict__ attn, const float* __restrict__ grad_out,
+                     float* __restrict__ grad_value, float* __restrict__ grad_loc,
+                     float* __restrict__ grad_attn, int B, int Nq, int Nv, int H, int L, int P,
+                     Levels levels)
+{
+    __shared__ SmemLevels s_lv;
+    __shared__ __align__(16) BwdTable s_tab[kWarps];
+    stage_levels(s_lv, levels);
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t items = (int64_t)B * Nq * H;
+    const int S = L * P;
+    const int64_t tile0 = (int64_t)blockIdx.x * kWarps * kBwdRowsPerWarp;
+    for (int t = 0; t < kBwdRowsPerWarp; ++t) {
+        const int64_t item = tile0 + (int64_t)t * kWarps + warp;
+        if (item >= items) break;
+        const int h = (int)(item % H);
+        const int b = (int)(item / H / Nq);
+        const int64_t vofs = (int64_t)b * Nv * H * kHeadDim;
+        row_backward<VT, false, NC>(value + vofs, H, h, loc + item * S * 2, attn + item * S,
+                                    nullptr, L, P, 1, s_lv, s_tab[warp],
+                                    grad_out + item * kHeadDim, 1.f, grad_value + vofs,
+                                    grad_loc + item * S * 2, grad_attn + item * S, lane);
+    }
+}
+
+template <typename VT, int NC>
+__global__ void __launch_bounds__(kThreads)
+sca_backward_kernel(const VT* __restrict__ value, const float* __restrict__ off,
+                    const float* __restrict__ logits, const float* __restrict__ ref_cam,
+                    const float* __restrict__ grad_out, const int32_t* __restrict__ idx,
+                    const int32_t* __restrict__ hits, const int32_t* __restrict__ count,
+                    float* __restrict__ grad_value, float* __restrict__ grad_loc_rb,
+                    float* __restrict__ grad_attn_rb, int B, int Ncam, int Nq, int Nv, int H,
+                    int L, int P, int R, Levels levels)
+{
+    __shared__ SmemLevels s_lv;
+    __shared__ __align__(16) BwdTable s_tab[kWarps];
+    __shared__ int s_prefix[kMaxBatchCameras + 1];
+    const int nbc = B * Ncam;
+    stage_levels(s_lv, levels);
+    stage_row_prefix(count, nbc, s_prefix);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t items = (int64_t)s_prefix[nbc] * H;
+    const int S = L * P;
+    for (int64_t item = (int64_t)blockIdx.x * kWarps + warp; item < items;
+         item += (int64_t)gridDim.x * kWarps) {
+        const int r = (int)(item / H), h = (int)(item % H);
+        const int bc = find_segment(s_prefix, nbc, r);
+        const int i = r - s_prefix[bc];
+        const int b = bc / Ncam, c = bc - b * Ncam;
+        const int q = __ldg(idx + (int64_t)bc * Nq + i);
+        if ((unsigned)q >= (unsigned)Nq) continue;  // inconsistent lists: read nothing
+        const int64_t bq = (int64_t)b * Nq + q;
+        const int64_t bqh = bq * H + h;
+        const int64_t vofs = (int64_t)bc * Nv * H * kHeadDim;
+        const int64_t rowh = ((int64_t)bc * Nq + i) * H + h;
+        const float scale = (float)max(1, __ldg(hits + bq));
+        row_backward<VT, true, NC>(value + vofs, H, h, off + bqh * S * 2, logits + bqh * S,
+                                   ref_cam + (((int64_t)c * B + b) * Nq + q) * R * 2, L, P, R,
+                                   s_lv, s_tab[warp], grad_out + bqh * kHeadDim, scale,
+                                   grad_value + vofs, grad_loc_rb + rowh * S * 2,
+                                   grad_attn_rb + rowh * S, lane);
+    }
+}
+
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void zero_range(float* __restrict__ p, int64_t n, int64_t tid,
+                                           int64_t nthreads)
+{
+    // scalar head up to 16-byte alignment, float4 body, scalar tail
+    const int64_t head = std::min<int64_t>(n, (int64_t)((16 - ((uintptr_t)p & 15)) & 15) / 4);
+    for (int64_t i = tid; i < head; i += nthreads) p[i] = 0.f;
+    float4* body = reinterpret_cast<float4*>(p + head);
+    const int64_t n4 = (n - head) / 4;
+    for (int64_t i = tid; i < n4; i += nthreads) body[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int64_t i = head + n4 * 4 + tid; i < n; i += nthreads) p[i] = 0.f;
+}
+
+__global__ void zero_kernel(float* __restrict__ p, int64_t n)
+{
+    zero_range(p, n, (int64_t)blockIdx.x * blockDim.x + threadIdx.x,
+               (int64_t)gridDim.x * blockDim.x);
+}
+
+// Rebatched rows count[bc] .. Nq-1 of every (batch, camera) are contiguous in
+// both gradient arrays; zero them.
+__global__ void sca_zero_tail_kernel(const int32_t* __restrict__ count, int Nq, int S,
+                                     float* __restrict__ grad_loc_rb,
+                                     float* __restrict__ grad_attn_rb)
+{
+    const int bc = blockIdx.y;
+    const int64_t first = (int64_t)bc * Nq + __ldg(count + bc), last = (int64_t)bc * Nq + Nq;
+    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t nthreads = (int64_t)gridDim.x * blockDim.x;
+    zero_range(grad_loc_rb + first * S * 2, (last - first) * S * 2, tid, nthreads);
+    zero_range(grad_attn_rb + first * S, (last - first) * S, tid, nthreads);
+}
+
+cudaError_t launch_zero(float* p, int64_t n, cudaStream_t s)
+{
+    if (n <= 0) return cudaSuccess;
+    const int64_t blocks = std::min<int64_t>((n / 4 + 255) / 256 + 1, (int64_t)device_sm_count() * 16);
+    zero_kernel<<<(unsigned)blocks, 256, 0, s>>>(p, n);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_sca_zero_tail(const int32_t* count, int B, int Ncam, int Nq, int S,
+                                 float* grad_loc_rb, float* grad_attn_rb, cudaStream_t s)
+{
+    if (B == 0 || Nq == 0) return cudaSuccess;
+    const int64_t per_bc = (int64_t)Nq * S * 3;
+    const int bx = (int)std::min<int64_t>((per_bc / 4 + 255) / 256 + 1, 64);
+    sca_zero_tail_kernel<<<dim3(bx, B * Ncam), 256, 0, s>>>(count, Nq, S, grad_loc_rb,
+                                                            grad_attn_rb);
+    return cudaGetLastError();
+}
+
+template <typename VT>
+static cudaError_t launch_msda_backward_t(const Problem& p, const float* loc, const float* attn,
+                                          const float* grad_out, float* grad_value,
+                                          float* grad_loc, float* grad_attn, cudaStream_t s)
+{
+    const int64_t items = (int64_t)p.B * p.Nq * p.H;
+    if (items == 0) return cudaSuccess;
+    const int64_t per_cta = (int64_t)kWarps * kBwdRowsPerWarp;
+    const unsigned grid = (unsigned)((items + per_cta - 1) / per_cta);
+    const VT* v = static_cast<const VT*>(p.value);
+    const int nc = (p.L * p.P + 31) / 32;
+#define MSDA_BWD_CASE(NCV)                                                                       \
+    case NCV:                                                                                    \
+        msda_backward_kernel<VT, NCV><<<grid, kThreads, 0, s>>>(                                 \
+            v, loc, attn, grad_out, grad_value, grad_loc, grad_attn, p.B, p.Nq, p.Nv, p.H, p.L,  \
+            p.P, p.lv);                                                                          \
+        break;
+    switch (nc) {
+        MSDA_BWD_CASE(1)
+        MSDA_BWD_CASE(2)
+        MSDA_BWD_CASE(3)
+        MSDA_BWD_CASE(4)
+        default: return cudaErrorInvalidValue;
+    }
+#undef MSDA_BWD_CASE
+    return cudaGetLastError();
+}
+
+cudaError_t launch_msda_backward(const Problem& p, const float* loc, const float* attn,
+                                 const float* grad_out, float* grad_value, float* grad_loc,
+                                 float* grad_attn, cudaStream_t s)
+{
+    return p.bf16 ? launch_msda_backward_t<__nv_bfloat16>(p, loc, attn, grad_out, grad_value,
+                                                          grad_loc, grad_attn, s)
+                  : launch_msda_backward_t<float>(p, loc, attn, grad_out, grad_value, grad_loc,
+                                                  grad_attn, s);
+}
+
+template <typename K>
+static int bwd_resident_ctas(K kernel)
+{
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kThreads, 0) != cudaSuccess || n < 1)
+        n = 1;
+    return n;
+}
+
+template <typename VT>
+static cudaError_t launch_sca_backward_t(const Problem& p, const float* ref_cam, const float* off,
+                                         const float* logits, const float* grad_out,
+                                         const int32_t* idx, const int32_t* hits,
+                                         const int32_t* count, float* grad_value,
+                                         float* grad_loc_rb, float* grad_attn_rb, cudaStream_t s)
+{
+    const int64_t max_items = (int64_t)p.B * p.Ncam * p.Nq * p.H;
+    if (max_items == 0) return cudaSuccess;
+    const int64_t max_ctas = (max_items + kWarps - 1) / kWarps;
+    const VT* v = static_cast<const VT*>(p.value);
+    const int nc = (p.L * p.P + 31) / 32;
+#define SCA_BWD_CASE(NCV)                                                                        \
+    case NCV: {                                                                                  \
+        static int occ = bwd_resident_ctas(sca_backward_kernel<VT, NCV>);                        \
+        const int64_t grid = std::min<int64_t>(max_ctas, (int64_t)occ * device_sm_count());      \
+        sca_backward_kernel<VT, NCV><<<(unsigned)grid, kThreads, 0, s>>>(                        \
+            v, off, logits, ref_cam, grad_out, idx, hits, count, grad_value, grad_loc_rb,        \
+            grad_attn_rb, p.B, p.Ncam, p.Nq, p.Nv, p.H, p.L, p.P, p.R, p.lv);                    \
+        break;                                                                                   \
+    }
+    switch (nc) {
+        SCA_BWD_CASE(1)
+        SCA_BWD_CASE(2)
+        SCA_BWD_CASE(3)
+        SCA_BWD_CASE(4)
+        default: return cudaErrorInvalidValue;
+    }
+#undef SCA_BWD_CASE
+    return cudaGetLastError();
+}
+
+cudaError_t launch_sca_backward_rows(const Problem& p, const float* ref_cam, const float* off,
+                                     const float* logits, const float* grad_out,
+                                     const int32_t* idx, const int32_t* hits,
+                                     const int32_t* count, float* grad_value,
+                                     float* grad_loc_rb, float* grad_attn_rb, cudaStream_t s)
+{
+    return p.bf16 ? launch_sca_backward_t<__nv_bfloat16>(p, ref_cam, off, logits, grad_out, idx,
+                                                         hits, count, grad_value,
+                                                         grad_loc_rb, grad_attn_rb, s)
+                  : launch_sca_backward_t<float>(p, ref_cam, off, logits, grad_out, idx, hits,
+                                                 count, grad_value, grad_loc_rb, grad_attn_rb, s);
+}
+
+}  // namespace msda

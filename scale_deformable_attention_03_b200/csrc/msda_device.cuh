@@ -1,0 +1,367 @@
+// Device building blocks of the MSDA / SCA kernels (sm_100a).
+//
+// One warp computes one output row of one head: the 32 channels of
+//   g^(h) = sum_{l,k} alpha_{h,l,k} * bilinear(V_l^(h), s_{h,l,k})
+// ("BEV(三) BEVFormer: how the Query interacts with the 8 Heads of the
+// Feature", sections 6 and 8).  The warp works in chunks of 32 samples:
+//   1. lane j owns sample j of the chunk: it forms the location, the corner
+//      decision and the four corner offsets and weights (alpha folded in) and
+//      writes them to a per-warp table in shared memory (structure of arrays,
+//      rows padded to 36 words so that the quad reads below are free of bank
+//      conflicts);
+//   2. the warp walks the table four samples at a time.  fp32 value: lanes
+//      8g..8g+7 read corner g of one sample, 16 bytes each, so one warp load
+//      fetches the four 128-byte corner slices of a sample.  bf16 value: lanes
+//      16s + 4g + t read corner g of sample 2p + s (16 bytes = 8 channels), so
+//      one warp load fetches two samples.  Each lane accumulates its own
+//      corner and channels; the corners (and sample halves) are summed with
+//      shuffles once per row, not once per sample.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace msda {
+
+constexpr int kHeadDim = 32;
+constexpr int kMaxLevels = 8;
+constexpr int kWarps = 8;               // warps per CTA
+constexpr int kThreads = kWarps * 32;
+constexpr int kMetaStride = 36;         // words per corner row of the sample table
+constexpr int kMaxBatchCameras = 1024;  // B * Ncam limit of the SCA kernels
+
+// Level geometry, passed by value to every kernel.
+struct Levels {
+    int h[kMaxLevels];      // rows H_l
+    int w[kMaxLevels];      // columns W_l
+    int start[kMaxLevels];  // first value row of the level
+};
+
+struct SmemLevels {
+    int h[kMaxLevels], w[kMaxLevels], start[kMaxLevels];
+};
+
+// Per-warp sample table: corner g of sample j is (off[g][j], w[g][j]).
+struct WarpTable {
+    int off[4][kMetaStride];
+    float w[4][kMetaStride];
+};
+
+__device__ __forceinline__ void stage_levels(SmemLevels& s, const Levels& lv)
+{
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int i = 0; i < kMaxLevels; ++i) {
+            s.h[i] = lv.h[i];
+            s.w[i] = lv.w[i];
+            s.start[i] = lv.start[i];
+        }
+    }
+}
+
+__device__ __forceinline__ float warp_max(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Streaming loads for data read once per row (evict-first).
+__device__ __forceinline__ float ld_stream(const float* p) { return __ldcs(p); }
+__device__ __forceinline__ float2 ld_stream2(const float* p)
+{
+    return __ldcs(reinterpret_cast<const float2*>(p));
+}
+
+// Attention weights of one (row, head): lane holds samples lane + 32c.
+// FUSED: softmax over the L*P logits, max-subtracted (section 4.2).
+template <bool FUSED, int NC>
+__device__ __forceinline__ void row_weights(const float* __restrict__ src, int n, int lane,
+                                            float (&a)[NC])
+{
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+        const int j = c * 32 + lane;
+        a[c] = (j < n) ? ld_stream(src + j) : (FUSED ? -INFINITY : 0.f);
+    }
+    if (FUSED) {
+        float m = a[0];
+#pragma unroll
+        for (int c = 1; c < NC; ++c) m = fmaxf(m, a[c]);
+        m = warp_max(m);
+        float z = 0.f;
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+            const int j = c * 32 + lane;
+            a[c] = (j < n) ? expf(a[c] - m) : 0.f;
+            z += a[c];
+        }
+        z = warp_sum(z);
+#pragma unroll
+        for (int c = 0; c < NC; ++c) a[c] = a[c] / z;
+    }
+}
+
+// Corner decision of one sample (section 6): x = W s_x - 1/2, y = H s_y - 1/2
+// in binary32, round-to-nearest, never contracted; four neighbours with
+// bilinear weights; a neighbour outside the map gets offset -1.  A location
+// with x <= -1 or x >= W (same for y), or a NaN, reads nothing.
+struct Corners {
+    int off[4];    // element offset of the head slice, -1 when outside
+    float w[4];    // bilinear weight (without alpha)
+    float lx, ly;  // fractional parts
+    bool valid;
+};
+
+__device__ __forceinline__ void locate(float sx, float sy, int Hl, int Wl, int start, int H,
+                                       int h, Corners& c)
+{
+    const float fW = (float)Wl, fH = (float)Hl;
+    const float x = __fsub_rn(__fmul_rn(fW, sx), 0.5f);
+    const float y = __fsub_rn(__fmul_rn(fH, sy), 0.5f);
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+        c.off[g] = -1;
+        c.w[g] = 0.f;
+    }
+    c.lx = c.ly = 0.f;
+    c.valid = (x > -1.f) && (x < fW) && (y > -1.f) && (y < fH);
+    if (c.valid) {
+        const float x0f = floorf(x), y0f = floorf(y);
+        const float lx = __fsub_rn(x, x0f), ly = __fsub_rn(y, y0f);
+        const int x0 = (int)x0f, y0 = (int)y0f;  // x0 in [-1, W-1], y0 in [-1, H-1]
+        const float hx = __fsub_rn(1.f, lx), hy = __fsub_rn(1.f, ly);
+        c.lx = lx;
+        c.ly = ly;
+        c.w[0] = __fmul_rn(hx, hy);
+        c.w[1] = __fmul_rn(lx, hy);
+        c.w[2] = __fmul_rn(hx, ly);
+        c.w[3] = __fmul_rn(lx, ly);
+        const bool x0in = x0 >= 0, x1in = x0 + 1 < Wl, y0in = y0 >= 0, y1in = y0 + 1 < Hl;
+        const int p = start + y0 * Wl + x0;  // pixel of neighbour 0 (used only when inside)
+        if (x0in && y0in) c.off[0] = (p * H + h) * kHeadDim;
+        if (x1in && y0in) c.off[1] = ((p + 1) * H + h) * kHeadDim;
+        if (x0in && y1in) c.off[2] = ((p + Wl) * H + h) * kHeadDim;
+        if (x1in && y1in) c.off[3] = ((p + Wl + 1) * H + h) * kHeadDim;
+    }
+}
+
+// Sampling location of sample j = (l, k) of one (row, head).
+// FUSED: rho_{k mod R} + (dx / W_l, dy / H_l), each step one rounded binary32
+// operation (section 5); otherwise the given location.
+template <bool FUSED>
+__device__ __forceinline__ void sample_location(const float* __restrict__ lo,
+                                                const float* __restrict__ ref, int j, int k,
+                                                int R, int Hl, int Wl, float& sx, float& sy)
+{
+    const float2 v = ld_stream2(lo + 2 * j);
+    if (FUSED) {
+        const float2 r = __ldg(reinterpret_cast<const float2*>(ref) + (k % R));
+        sx = __fadd_rn(r.x, __fdiv_rn(v.x, (float)Wl));
+        sy = __fadd_rn(r.y, __fdiv_rn(v.y, (float)Hl));
+    } else {
+        sx = v.x;
+        sy = v.y;
+    }
+}
+
+// bf16 pair (packed in 32 bits) -> two floats, exact.
+__device__ __forceinline__ void bf16x2_to_f32(uint32_t u, float& lo, float& hi)
+{
+    lo = __uint_as_float(u << 16);
+    hi = __uint_as_float(u & 0xffff0000u);
+}
+
+// Gather over the first `cnt` samples of the table; see the file comment for
+// the lane layout.  acc: fp32 value -> 4 channels (4t..4t+3) of corner g;
+// bf16 value -> 8 channels (8t..8t+7) of corner g for the lane's half.
+template <typename VT>
+struct Gather;
+
+template <>
+struct Gather<float> {
+    static constexpr int kAcc = 4;
+    __device__ __forceinline__ static void run(const float* __restrict__ vb,
+                                               const WarpTable& tab, int cnt, int lane,
+                                               float (&acc)[4])
+    {
+        const int g = lane >> 3, t = lane & 7;
+        const float* v = vb + 4 * t;
+        const int quads = (cnt + 3) >> 2;
+#pragma unroll 2
+        for (int p = 0; p < quads; ++p) {
+            const int4 o = *reinterpret_cast<const int4*>(&tab.off[g][4 * p]);
+            const float4 w = *reinterpret_cast<const float4*>(&tab.w[g][4 * p]);
+            float4 x0 = make_float4(0.f, 0.f, 0.f, 0.f), x1 = x0, x2 = x0, x3 = x0;
+            if (o.x >= 0) x0 = __ldg(reinterpret_cast<const float4*>(v + o.x));
+            if (o.y >= 0) x1 = __ldg(reinterpret_cast<const float4*>(v + o.y));
+            if (o.z >= 0) x2 = __ldg(reinterpret_cast<const float4*>(v + o.z));
+            if (o.w >= 0) x3 = __ldg(reinterpret_cast<const float4*>(v + o.w));
+            acc[0] += w.x * x0.x + w.y * x1.x + w.z * x2.x + w.w * x3.x;
+            acc[1] += w.x * x0.y + w.y * x1.y + w.z * x2.y + w.w * x3.y;
+            acc[2] += w.x * x0.z + w.y * x1.z + w.z * x2.z + w.w * x3.z;
+            acc[3] += w.x * x0.w + w.y * x1.w + w.z * x2.w + w.w * x3.w;
+        }
+    }
+    // Sum the four corners; lanes 0..7 store channels 4t..4t+3.
+    __device__ __forceinline__ static void store(float (&acc)[4], int lane, float* __restrict__ out)
+    {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 8);
+            acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 16);
+        }
+        if (lane < 8)
+            *reinterpret_cast<float4*>(out + 4 * lane) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    }
+};
+
+template <>
+struct Gather<__nv_bfloat16> {
+    static constexpr int kAcc = 8;
+    __device__ __forceinline__ static void fma8(float (&acc)[8], float w, uint4 r)
+    {
+        float a, b;
+        bf16x2_to_f32(r.x, a, b);
+        acc[0] += w * a;
+        acc[1] += w * b;
+        bf16x2_to_f32(r.y, a, b);
+        acc[2] += w * a;
+        acc[3] += w * b;
+        bf16x2_to_f32(r.z, a, b);
+        acc[4] += w * a;
+        acc[5] += w * b;
+        bf16x2_to_f32(r.w, a, b);
+        acc[6] += w * a;
+        acc[7] += w * b;
+    }
+    __device__ __forceinline__ static void run(const __nv_bfloat16* __restrict__ vb,
+                                               const WarpTable& tab, int cnt, int lane,
+                                               float (&acc)[8])
+    {
+        const int half = lane >> 4, g = (lane >> 2) & 3, t = lane & 3;
+        const __nv_bfloat16* v = vb + 8 * t;
+        const int quads = (cnt + 3) >> 2;
+#pragma unroll 2
+        for (int p = 0; p < quads; ++p) {
+            const int4 o = *reinterpret_cast<const int4*>(&tab.off[g][4 * p]);
+            const float4 w = *reinterpret_cast<const float4*>(&tab.w[g][4 * p]);
+            const int oa = half ? o.y : o.x, ob = half ? o.w : o.z;
+            const float wa = half ? w.y : w.x, wb = half ? w.w : w.z;
+            uint4 ra = make_uint4(0u, 0u, 0u, 0u), rb = ra;
+            if (oa >= 0) ra = __ldg(reinterpret_cast<const uint4*>(v + oa));
+            if (ob >= 0) rb = __ldg(reinterpret_cast<const uint4*>(v + ob));
+            fma8(acc, wa, ra);
+            fma8(acc, wb, rb);
+        }
+    }
+    // Sum corners and halves; lanes 0..3 store channels 8t..8t+7.
+    __device__ __forceinline__ static void store(float (&acc)[8], int lane, float* __restrict__ out)
+    {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 4);
+            acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 8);
+            acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 16);
+        }
+        if (lane < 4) {
+            float4* o = reinterpret_cast<float4*>(out + 8 * lane);
+            o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        }
+    }
+};
+
+// One output row of one head (all L*P samples), written to out_row[0..32).
+//   vb      value of this batch item (and camera): [Nv, H, 32]
+//   lo      FUSED: pixel offsets, else locations, of this (row, head): [L, P, 2]
+//   wl      FUSED: logits, else weights, of this (row, head): [L, P]
+//   ref     FUSED only: reference points of this row: [R, 2]
+template <typename VT, bool FUSED, int NC>
+__device__ __forceinline__ void row_forward(const VT* __restrict__ vb, int H, int h,
+                                            const float* __restrict__ lo,
+                                            const float* __restrict__ wl,
+                                            const float* __restrict__ ref, int L, int P, int R,
+                                            const SmemLevels& lv, WarpTable& tab,
+                                            float* __restrict__ out_row, int lane)
+{
+    const int n = L * P;
+    float a[NC];
+    row_weights<FUSED, NC>(wl, n, lane, a);
+    float acc[Gather<VT>::kAcc];
+#pragma unroll
+    for (int i = 0; i < Gather<VT>::kAcc; ++i) acc[i] = 0.f;
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+        const int j = c * 32 + lane;
+        Corners cr;
+        if (j < n) {
+            const int l = j / P, k = j - l * P;
+            const int Hl = lv.h[l], Wl = lv.w[l];
+            float sx, sy;
+            sample_location<FUSED>(lo, ref, j, k, R, Hl, Wl, sx, sy);
+            locate(sx, sy, Hl, Wl, lv.start[l], H, h, cr);
+        } else {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                cr.off[g] = -1;
+                cr.w[g] = 0.f;
+            }
+        }
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            tab.off[g][lane] = cr.off[g];
+            tab.w[g][lane] = cr.w[g] * a[c];
+        }
+        __syncwarp();
+        Gather<VT>::run(vb, tab, min(32, n - c * 32), lane, acc);
+        __syncwarp();
+    }
+    Gather<VT>::store(acc, lane, out_row);
+}
+
+// Row offsets of the rebatched layout: s_prefix[bc] = sum of count[0..bc),
+// s_prefix[n] = total rows.  Warp 0 scans; the whole block must call this.
+__device__ __forceinline__ void stage_row_prefix(const int32_t* __restrict__ count, int n,
+                                                 int* s_prefix)
+{
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        int run = 0;
+        for (int base = 0; base < n; base += 32) {
+            const int v = (base + lane < n) ? __ldg(count + base + lane) : 0;
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += u;
+            }
+            if (base + lane < n) s_prefix[base + lane] = run + incl - v;
+            run += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) s_prefix[n] = run;
+    }
+    __syncthreads();
+}
+
+// Largest bc in [0, n) with prefix[bc] <= r, given prefix[n] > r.
+__device__ __forceinline__ int find_segment(const int* prefix, int n, int r)
+{
+    int lo = 0, hi = n;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (prefix[mid] <= r) lo = mid;
+        else hi = mid;
+    }
+    return lo;
+}
+
+}  // namespace msda

@@ -1,0 +1,76 @@
+// Internal launcher interface between the C ABI (msda_api.cu) and the kernel
+// translation units.  Arguments are already validated when these are called.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "msda_device.cuh"
+
+namespace msda {
+
+struct Problem {
+    const void* value;   // [B, (Ncam,) Nv, H, 32]
+    bool bf16;
+    int B, Ncam, Nq, Nv, H, L, P, R;
+    Levels lv;
+};
+
+// Workspace layout of sca_forward / sca_backward: compaction scratch, the
+// compaction lists, then (forward only) the rebatched rows.
+struct ScaWorkspace {
+    int32_t* idx;           // [B, Ncam, Nq]
+    int32_t* pos;           // [B, Ncam, Nq]
+    int32_t* count;         // [B, Ncam]
+    int32_t* hits;          // [B, Nq]
+    int32_t* chunk_counts;  // [B, Ncam, nchunks]
+    float* out_rb;          // [B, Ncam, Nq, H * 32] (forward only)
+};
+
+constexpr int kCompactChunk = 1024;  // queries per compaction CTA
+
+struct CompactScratch {
+    int32_t* chunk_counts;  // [B, Ncam, nchunks]
+};
+
+size_t compact_scratch_bytes(int B, int Ncam, int Nq);
+CompactScratch compact_scratch_carve(void* base, int B, int Ncam, int Nq);
+size_t sca_workspace_bytes(int B, int Ncam, int Nq, int H, bool with_rows);
+ScaWorkspace sca_workspace_carve(void* base, int B, int Ncam, int Nq, int H, bool with_rows);
+
+int device_sm_count();
+
+// K1 / K1f: msda_forward (given locations, weights) and msda_forward_fused.
+cudaError_t launch_msda_forward(const Problem& p, const float* loc, const float* attn,
+                                float* out, cudaStream_t s);
+cudaError_t launch_msda_forward_fused(const Problem& p, const float* ref, const float* off,
+                                      const float* logits, float* out, cudaStream_t s);
+
+// K2: compaction (two launches).
+cudaError_t launch_sca_compact(const uint8_t* mask, int B, int Ncam, int Nq, int R,
+                               int32_t* idx, int32_t* count, int32_t* pos, int32_t* hits,
+                               int32_t* chunk_counts, cudaStream_t s);
+
+// K3: fused MSDA over the rebatched rows of every (batch, camera).
+cudaError_t launch_sca_gather(const Problem& p, const float* ref_cam, const float* off,
+                              const float* logits, const int32_t* idx, const int32_t* count,
+                              float* out_rb, cudaStream_t s);
+
+// K4: deterministic camera average.
+cudaError_t launch_sca_average(const float* out_rb, const int32_t* pos, const int32_t* hits,
+                               int B, int Ncam, int Nq, int H, float* out, cudaStream_t s);
+
+// Backward.
+cudaError_t launch_zero(float* p, int64_t n, cudaStream_t s);
+cudaError_t launch_msda_backward(const Problem& p, const float* loc, const float* attn,
+                                 const float* grad_out, float* grad_value, float* grad_loc,
+                                 float* grad_attn, cudaStream_t s);
+cudaError_t launch_sca_backward_rows(const Problem& p, const float* ref_cam, const float* off,
+                                     const float* logits, const float* grad_out,
+                                     const int32_t* idx, const int32_t* hits,
+                                     const int32_t* count, float* grad_value,
+                                     float* grad_loc_rb, float* grad_attn_rb, cudaStream_t s);
+cudaError_t launch_sca_zero_tail(const int32_t* count, int B, int Ncam, int Nq, int S,
+                                 float* grad_loc_rb, float* grad_attn_rb, cudaStream_t s);
+
+}  // namespace msda

@@ -1,0 +1,113 @@
+"""MSDA and SCA backward on the GPU against the oracle's analytic derivative
+(itself pinned to central finite differences), through the C ABI.
+
+grad_value is accumulated with fp32 atomics, so its summation order differs
+from the oracle's; the fp32 tolerance still applies at these sizes.
+Workload 5 (the BEVFormer-base SCA training step, bf16 value) runs at full
+size against the 2e-2 bf16 bound.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import scale_deformable_attention_03_b200 as msda
+from scale_deformable_attention_03_b200 import inputs
+
+from .gpu_util import assert_close, dev, softmax_weights, value_tensor
+
+pytestmark = pytest.mark.gpu
+
+
+def _problem(seed, B, Nq, H, shapes, P, lo=-0.2, hi=1.2):
+    rng = np.random.Generator(np.random.PCG64(seed))
+    s, starts, Nv = inputs.level_table(shapes)
+    L = len(shapes)
+    value = rng.standard_normal((B, Nv, H, 32)).astype(np.float32)
+    loc = rng.uniform(lo, hi, (B, Nq, H, L, P, 2)).astype(np.float32)
+    weights = softmax_weights(rng.standard_normal((B, Nq, H, L, P)), L * P)
+    gout = rng.standard_normal((B, Nq, H * 32)).astype(np.float32)
+    return s, starts, value, loc, weights, gout
+
+
+CASES = [
+    (1, 1, 29, 1, [(5, 7)], 2),
+    (2, 2, 300, 8, [(20, 30), (10, 15), (5, 8), (3, 4)], 4),
+    (3, 1, 77, 2, [(6, 5), (3, 3), (1, 9)], 12),     # two chunks
+    (4, 1, 40, 3, [(7, 9)] * 8, 16),                 # four chunks
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[f"case{c[0]}" for c in CASES])
+@pytest.mark.parametrize("bf16", [False, True])
+def test_msda_backward_random(case, bf16):
+    seed, B, Nq, H, shapes, P = case
+    s, starts, value, loc, weights, gout = _problem(seed, B, Nq, H, shapes, P)
+    if bf16:
+        bits = inputs.to_bf16_bits(value)
+        value = inputs.bf16_bits_to_f32(bits)
+        vt = dev(bits.view(np.int16)).view(torch.bfloat16)
+    else:
+        vt = dev(value)
+    gv, gl, gw = msda.msda_backward(vt, s, starts, dev(loc), dev(weights), dev(gout))
+    torch.cuda.synchronize()
+    rv, rl, rw = oracle.msda_backward(value, s, starts, loc, weights, gout)
+    assert_close(gw, rw, False, "grad_attention_weights")
+    assert_close(gl, rl, False, "grad_sampling_locations")
+    assert_close(gv, rv, False, "grad_value")
+
+
+def test_msda_backward_workload2():
+    w = inputs.workload2(max_queries=6000)
+    loc, weights = oracle.fused_locations(w.spatial_shapes, w.reference_points,
+                                          w.sampling_offsets, w.attention_logits)
+    loc, weights = loc.astype(np.float32), weights.astype(np.float32)
+    gout = np.random.Generator(np.random.PCG64(5)).standard_normal(
+        (1, w.Nq, w.H * 32)).astype(np.float32)
+    gv, gl, gw = msda.msda_backward(dev(w.value), w.spatial_shapes, w.level_start_index,
+                                    dev(loc), dev(weights), dev(gout))
+    torch.cuda.synchronize()
+    rv, rl, rw = oracle.msda_backward(w.value, w.spatial_shapes, w.level_start_index, loc,
+                                      weights, gout)
+    assert_close(gw, rw, False, "grad_attention_weights")
+    assert_close(gl, rl, False, "grad_sampling_locations")
+    assert_close(gv, rv, False, "grad_value")
+
+
+def _sca_bwd(w, bf16):
+    grads = msda.sca_backward(value_tensor(w, bf16), w.spatial_shapes, w.level_start_index,
+                              dev(w.reference_points), dev(w.bev_mask), dev(w.sampling_offsets),
+                              dev(w.attention_logits), dev(w.grad_out))
+    torch.cuda.synchronize()
+    ref = oracle.sca_backward(w.value, w.spatial_shapes, w.level_start_index, w.reference_points,
+                              w.bev_mask, w.sampling_offsets, w.attention_logits, w.grad_out)
+    return grads, ref
+
+
+@pytest.mark.parametrize("seed,B,Ncam,bev,shapes,H,P,R", [
+    (31, 2, 3, (7, 9), [(9, 13), (4, 7)], 2, 4, 2),
+    (32, 1, 6, (30, 40), [(16, 20), (8, 10), (4, 5), (2, 3)], 8, 8, 4),
+    (33, 2, 2, (5, 13), [(6, 7)] * 3, 1, 12, 3),
+])
+def test_sca_backward_random(seed, B, Ncam, bev, shapes, H, P, R):
+    w = inputs.workload3(seed=seed, B=B, Ncam=Ncam, bev_h=bev[0], bev_w=bev[1], shapes=shapes,
+                         H=H, P=P, R=R, rho="uniform", same_mask=False, with_grad=True)
+    (gv, gl, gw), (rv, rl, rw) = _sca_bwd(w, False)
+    assert_close(gw, rw, False, "grad_attention_weights_rb")
+    assert_close(gl, rl, False, "grad_sampling_locations_rb")
+    assert_close(gv, rv, False, "grad_value")
+
+
+def test_workload5_training_step_full_size():
+    w = inputs.workload5()
+    out = msda.sca_forward(value_tensor(w, True), w.spatial_shapes, w.level_start_index,
+                           dev(w.reference_points), dev(w.bev_mask), dev(w.sampling_offsets),
+                           dev(w.attention_logits))
+    (gv, gl, gw), (rv, rl, rw) = _sca_bwd(w, True)
+    ref_out = oracle.sca_forward(w.value, w.spatial_shapes, w.level_start_index,
+                                 w.reference_points, w.bev_mask, w.sampling_offsets,
+                                 w.attention_logits)
+    assert_close(out, ref_out, True, "workload 5 forward")
+    assert_close(gw, rw, True, "workload 5 grad_attention_weights_rb")
+    assert_close(gl, rl, True, "workload 5 grad_sampling_locations_rb")
+    assert_close(gv, rv, True, "workload 5 grad_value")

@@ -1,0 +1,133 @@
+"""SCA on the GPU against the oracle, through the C ABI: the compaction
+bit-exact, the forward element by element at the full BEVFormer-base size
+(fp32 and bf16 value, coherent and uniform reference points) and on small
+randomised problems with several batch items and cameras."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import scale_deformable_attention_03_b200 as msda
+from scale_deformable_attention_03_b200 import inputs
+
+from .gpu_util import assert_close, dev, value_tensor
+
+pytestmark = pytest.mark.gpu
+
+
+def _compact_gpu(mask):
+    idx, cnt, pos, hits = msda.sca_compact(dev(mask))
+    torch.cuda.synchronize()
+    return [t.cpu().numpy() for t in (idx, cnt, pos, hits)]
+
+
+def _assert_compaction_equal(mask):
+    got = _compact_gpu(mask)
+    want = oracle.sca_compact(mask)
+    for name, g, w in zip(("idx", "count", "pos", "hits"), got, want):
+        assert g.dtype == np.int32 and g.shape == w.shape, name
+        assert np.array_equal(g, w), f"{name} differs at {np.argwhere(g != w)[:5]}"
+
+
+def test_compaction_workload3_bit_exact():
+    w = inputs.workload3()
+    _assert_compaction_equal(w.bev_mask)
+
+
+@pytest.mark.parametrize("shape,p", [
+    ((6, 1, 40000, 4), 0.1),
+    ((6, 2, 1025, 4), 0.3),     # two chunks, ragged tail of one query
+    ((3, 3, 1023, 1), 0.5),
+    ((1, 1, 31, 2), 0.5),       # less than a warp
+    ((32, 1, 2048, 3), 0.05),   # the camera limit
+    ((5, 2, 4097, 8), 0.02),
+])
+def test_compaction_random_bit_exact(shape, p):
+    rng = np.random.Generator(np.random.PCG64(sum(shape)))
+    _assert_compaction_equal((rng.random(shape) < p).astype(np.uint8))
+
+
+@pytest.mark.parametrize("fill", [0, 1])
+def test_compaction_all_or_nothing(fill):
+    _assert_compaction_equal(np.full((6, 2, 3000, 4), fill, np.uint8))
+
+
+def test_compaction_non_binary_mask_bytes():
+    rng = np.random.Generator(np.random.PCG64(3))
+    mask = rng.integers(0, 256, (4, 1, 999, 4)).astype(np.uint8) * (rng.random((4, 1, 999, 4)) < 0.2)
+    _assert_compaction_equal(mask.astype(np.uint8))
+
+
+def _sca(w, bf16):
+    out = msda.sca_forward(value_tensor(w, bf16), w.spatial_shapes, w.level_start_index,
+                           dev(w.reference_points), dev(w.bev_mask), dev(w.sampling_offsets),
+                           dev(w.attention_logits))
+    torch.cuda.synchronize()
+    ref = oracle.sca_forward(w.value, w.spatial_shapes, w.level_start_index, w.reference_points,
+                             w.bev_mask, w.sampling_offsets, w.attention_logits)
+    return out, ref
+
+
+@pytest.mark.parametrize("bf16", [False, True])
+def test_workload3_bevformer_base(bf16):
+    w = inputs.workload3(value_dtype="bf16" if bf16 else "f32")
+    out, ref = _sca(w, bf16)
+    assert_close(out, ref, bf16, "workload 3 SCA")
+
+
+def test_workload3_uniform_reference_points():
+    w = inputs.workload3(rho="uniform", bev_h=100, bev_w=200)
+    out, ref = _sca(w, False)
+    assert_close(out, ref, False, "workload 3 SCA, uniform rho")
+
+
+@pytest.mark.parametrize("seed,B,Ncam,bev,shapes,H,P,R", [
+    (11, 2, 3, (7, 9), [(9, 13), (4, 7)], 2, 4, 2),
+    (12, 3, 6, (33, 35), [(16, 20), (8, 10), (4, 5), (2, 3)], 8, 8, 4),
+    (13, 1, 1, (1, 3), [(5, 5)], 1, 2, 1),
+    (14, 2, 5, (20, 52), [(6, 7)] * 3, 4, 12, 3),   # L*P = 36: two chunks
+])
+def test_random_sca(seed, B, Ncam, bev, shapes, H, P, R):
+    w = inputs.workload3(seed=seed, B=B, Ncam=Ncam, bev_h=bev[0], bev_w=bev[1], shapes=shapes,
+                         H=H, P=P, R=R, rho="uniform", same_mask=False)
+    # widen the offsets so that many reads leave the maps
+    w.sampling_offsets *= 3
+    out, ref = _sca(w, False)
+    assert_close(out, ref, False, f"random SCA {seed}")
+
+
+def test_queries_seen_by_no_camera_are_zero():
+    w = inputs.workload3(seed=21, bev_h=16, bev_w=16)
+    w.bev_mask[:, :, :50, :] = 0
+    out, ref = _sca(w, False)
+    assert torch.all(out[:, :50] == 0)
+    assert_close(out, ref, False, "unseen queries")
+
+
+def test_empty_mask():
+    w = inputs.workload3(seed=22, bev_h=8, bev_w=8)
+    w.bev_mask[:] = 0
+    out, _ = _sca(w, False)
+    assert torch.all(out == 0)
+
+
+def test_staged_calls_equal_sca_forward():
+    """sca_compact + sca_rebatched_forward + sca_camera_average is sca_forward,
+    bit for bit, and the rebatched rows match the oracle's."""
+    w = inputs.workload3(seed=23, bev_h=50, bev_w=60)
+    args = (dev(w.value), w.spatial_shapes, w.level_start_index, dev(w.reference_points))
+    idx, count, pos, hits = msda.sca_compact(dev(w.bev_mask))
+    rows = msda.sca_rebatched_forward(*args, dev(w.sampling_offsets), dev(w.attention_logits),
+                                      idx, count)
+    staged = msda.sca_camera_average(rows, pos, hits)
+    whole = msda.sca_forward(*args, dev(w.bev_mask), dev(w.sampling_offsets),
+                             dev(w.attention_logits))
+    torch.cuda.synchronize()
+    assert torch.equal(staged, whole)
+    ref, ref_rb = oracle.sca_forward(w.value, w.spatial_shapes, w.level_start_index,
+                                     w.reference_points, w.bev_mask, w.sampling_offsets,
+                                     w.attention_logits, return_rebatched=True)
+    cnt = count.cpu().numpy()
+    for c in range(w.Ncam):
+        n = cnt[0, c]
+        assert_close(rows[0, c, :n], ref_rb[0, c, :n], False, f"rebatched rows, camera {c}")
