@@ -87,10 +87,15 @@ msda_status_t check_levels(const msda_dims_t& d, const int64_t* shapes, const in
     return MSDA_OK;
 }
 
-msda_status_t check_value(const void* value, msda_dtype_t vdt)
+msda_status_t check_dtype(msda_dtype_t vdt)
 {
     MSDA_CHECK(vdt == MSDA_F32 || vdt == MSDA_BF16, MSDA_ERR_INVALID_ARG, "unknown value dtype %d",
                (int)vdt);
+    return MSDA_OK;
+}
+
+msda_status_t check_value(const void* value)
+{
     MSDA_CHECK(value != nullptr, MSDA_ERR_INVALID_ARG, "value is null");
     MSDA_CHECK(aligned(value, 16), MSDA_ERR_INVALID_ARG, "value must be 16-byte aligned");
     return MSDA_OK;
@@ -220,8 +225,9 @@ msda_status_t msda_forward(const void* value, msda_dtype_t vdt, const int64_t* s
     MSDA_TRY(check_dims(d, false));
     msda::Levels lv;
     MSDA_TRY(check_levels(d, spatial_shapes, level_start_index, lv));
-    MSDA_TRY(check_value(value, vdt));
+    MSDA_TRY(check_dtype(vdt));
     if ((int64_t)d.B * d.Nq == 0) return ok();
+    MSDA_TRY(check_value(value));
     MSDA_PTR(sampling_locations, 8);
     MSDA_PTR(attention_weights, 4);
     MSDA_PTR(out, 16);
@@ -240,8 +246,9 @@ msda_status_t msda_forward_fused(const void* value, msda_dtype_t vdt,
     MSDA_TRY(check_dims(d, false));
     msda::Levels lv;
     MSDA_TRY(check_levels(d, spatial_shapes, level_start_index, lv));
-    MSDA_TRY(check_value(value, vdt));
+    MSDA_TRY(check_dtype(vdt));
     if ((int64_t)d.B * d.Nq == 0) return ok();
+    MSDA_TRY(check_value(value));
     MSDA_PTR(reference_points, 8);
     MSDA_PTR(sampling_offsets, 8);
     MSDA_PTR(attention_logits, 4);
@@ -262,9 +269,11 @@ msda_status_t msda_backward(const void* value, msda_dtype_t vdt, const int64_t* 
     MSDA_TRY(check_dims(d, false));
     msda::Levels lv;
     MSDA_TRY(check_levels(d, spatial_shapes, level_start_index, lv));
-    MSDA_TRY(check_value(value, vdt));
+    MSDA_TRY(check_dtype(vdt));
+    if (d.B == 0) return ok();
     MSDA_PTR(grad_value, 16);
-    if ((int64_t)d.B * d.Nq > 0) {
+    if (d.Nq > 0) {
+        MSDA_TRY(check_value(value));
         MSDA_PTR(sampling_locations, 8);
         MSDA_PTR(attention_weights, 4);
         MSDA_PTR(grad_out, 16);
@@ -274,7 +283,7 @@ msda_status_t msda_backward(const void* value, msda_dtype_t vdt, const int64_t* 
     const cudaStream_t s = (cudaStream_t)stream;
     const msda::Problem p = make_problem(value, vdt, d, lv);
     cudaError_t e = msda::launch_zero(grad_value, (int64_t)d.B * d.Nv * d.H * MSDA_HEAD_DIM, s);
-    if (e == cudaSuccess)
+    if (e == cudaSuccess && d.Nq > 0)
         e = msda::launch_msda_backward(p, sampling_locations, attention_weights, grad_out,
                                        grad_value, grad_sampling_locations,
                                        grad_attention_weights, s);
@@ -346,8 +355,9 @@ static msda_status_t check_sca_inputs(const void* value, msda_dtype_t vdt, const
     MSDA_TRY(check_dims(d, true));
     MSDA_TRY(check_compact(d));
     MSDA_TRY(check_levels(d, spatial_shapes, level_start_index, lv));
-    MSDA_TRY(check_value(value, vdt));
+    MSDA_TRY(check_dtype(vdt));
     if ((int64_t)d.B * d.Nq > 0) {
+        MSDA_TRY(check_value(value));
         MSDA_PTR(reference_points_cam, 8);
         MSDA_PTR(sampling_offsets, 8);
         MSDA_PTR(attention_logits, 4);

@@ -11,6 +11,10 @@
 // alpha w_g grad_out to grad_value with one 16-byte vector reduction
 // (red.global.add.v4.f32); the per-sample scalars are reduced with shuffles
 // and land on the lane that owns the sample, which writes them coalesced.
+// The dot products and everything derived from them are formed in double
+// (a product of two fp32 numbers is exact in double): the location gradient
+// multiplies a difference of dot products by alpha * W_l (up to ~40 at
+// W_l = 200), and fp32 sums of the 32 products leave errors near 1e-4 there.
 #include <algorithm>
 
 #include "msda_launch.h"
@@ -34,14 +38,14 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
 }
 
 // d w_g / d lx and d w_g / d ly for neighbour g.
-__device__ __forceinline__ float dw_dlx(int g, float ly)
+__device__ __forceinline__ double dw_dlx(int g, float ly)
 {
-    const float a = (g >> 1) ? ly : 1.f - ly;
+    const double a = (g >> 1) ? (double)ly : 1.0 - (double)ly;
     return (g & 1) ? a : -a;
 }
-__device__ __forceinline__ float dw_dly(int g, float lx)
+__device__ __forceinline__ double dw_dly(int g, float lx)
 {
-    const float a = (g & 1) ? lx : 1.f - lx;
+    const double a = (g & 1) ? (double)lx : 1.0 - (double)lx;
     return (g >> 1) ? a : -a;
 }
 
@@ -60,16 +64,16 @@ struct BwdLanes<float> {
         go = make_float4(v.x / scale, v.y / scale, v.z / scale, v.w / scale);
     }
     // partial dot for corner g of sample jj, plus the grad_value reduction
-    __device__ __forceinline__ float step(const float* __restrict__ vb, float* __restrict__ gvb,
-                                          const BwdTable& tab, int jj, bool valid, float alpha,
-                                          int lane)
+    __device__ __forceinline__ double step(const float* __restrict__ vb, float* __restrict__ gvb,
+                                           const BwdTable& tab, int jj, bool valid, float alpha,
+                                           int lane)
     {
         const int g = lane >> 3, t = lane & 7;
         const int o = valid ? tab.off[g][jj] : -1;
-        float d = 0.f;
+        double d = 0.0;
         if (o >= 0) {
             const float4 v = __ldg(reinterpret_cast<const float4*>(vb + o + 4 * t));
-            d = go.x * v.x + go.y * v.y + go.z * v.z + go.w * v.w;
+            d = (double)go.x * v.x + (double)go.y * v.y + (double)go.z * v.z + (double)go.w * v.w;
             const float w = alpha * tab.wb[g][jj];
             if (w != 0.f) red_add_v4(gvb + o + 4 * t, w * go.x, w * go.y, w * go.z, w * go.w);
         }
@@ -79,7 +83,7 @@ struct BwdLanes<float> {
         return d;  // <grad_out, V_g> in every lane of group g
     }
     __device__ __forceinline__ static int group(int lane) { return lane >> 3; }
-    __device__ __forceinline__ static float reduce_groups(float v)
+    __device__ __forceinline__ static double reduce_groups(double v)
     {
         v += __shfl_xor_sync(0xffffffffu, v, 8);
         v += __shfl_xor_sync(0xffffffffu, v, 16);
@@ -101,13 +105,13 @@ struct BwdLanes<__nv_bfloat16> {
         go[0] = a.x / scale; go[1] = a.y / scale; go[2] = a.z / scale; go[3] = a.w / scale;
         go[4] = b.x / scale; go[5] = b.y / scale; go[6] = b.z / scale; go[7] = b.w / scale;
     }
-    __device__ __forceinline__ float step(const __nv_bfloat16* __restrict__ vb,
-                                          float* __restrict__ gvb, const BwdTable& tab, int jj,
-                                          bool valid, float alpha, int lane)
+    __device__ __forceinline__ double step(const __nv_bfloat16* __restrict__ vb,
+                                           float* __restrict__ gvb, const BwdTable& tab, int jj,
+                                           bool valid, float alpha, int lane)
     {
         const int g = (lane >> 2) & 3, t = lane & 3;
         const int o = valid ? tab.off[g][jj] : -1;
-        float d = 0.f;
+        double d = 0.0;
         if (o >= 0) {
             const uint4 r = __ldg(reinterpret_cast<const uint4*>(vb + o + 8 * t));
             float v[8];
@@ -116,7 +120,7 @@ struct BwdLanes<__nv_bfloat16> {
             bf16x2_to_f32(r.z, v[4], v[5]);
             bf16x2_to_f32(r.w, v[6], v[7]);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) d += go[i] * v[i];
+            for (int i = 0; i < 8; ++i) d += (double)go[i] * v[i];
             const float w = alpha * tab.wb[g][jj];
             if (w != 0.f) {
                 float* dst = gvb + o + 8 * t;
@@ -129,7 +133,7 @@ struct BwdLanes<__nv_bfloat16> {
         return d;
     }
     __device__ __forceinline__ static int group(int lane) { return (lane >> 2) & 3; }
-    __device__ __forceinline__ static float reduce_groups(float v)
+    __device__ __forceinline__ static double reduce_groups(double v)
     {
         v += __shfl_xor_sync(0xffffffffu, v, 4);
         v += __shfl_xor_sync(0xffffffffu, v, 8);
@@ -185,7 +189,7 @@ __device__ __forceinline__ void row_backward(const VT* __restrict__ vb, int H, i
         tab.lx[lane] = cr.lx;
         tab.ly[lane] = cr.ly;
         __syncwarp();
-        float res_w = 0.f, res_x = 0.f, res_y = 0.f;
+        double res_w = 0.0, res_x = 0.0, res_y = 0.0;
         const int cnt = min(32, n - c * 32);
         for (int p = 0; p < cnt; p += BwdLanes<VT>::kSamplesPerStep) {
             const int jraw = (BwdLanes<VT>::kSamplesPerStep == 2) ? p + (lane >> 4) : p;
@@ -193,10 +197,10 @@ __device__ __forceinline__ void row_backward(const VT* __restrict__ vb, int H, i
             const int jj = valid ? jraw : 0;
             // alpha of sample jj lives in lane jj
             const float alpha = __shfl_sync(0xffffffffu, a[c], jj);
-            const float d = lanes.step(vb, gvb, tab, jj, valid, alpha, lane);
-            float cw = valid ? tab.wb[g][jj] * d : 0.f;
-            float cx = valid ? dw_dlx(g, tab.ly[jj]) * d : 0.f;
-            float cy = valid ? dw_dly(g, tab.lx[jj]) * d : 0.f;
+            const double d = lanes.step(vb, gvb, tab, jj, valid, alpha, lane);
+            double cw = valid ? (double)tab.wb[g][jj] * d : 0.0;
+            double cx = valid ? dw_dlx(g, tab.ly[jj]) * d : 0.0;
+            double cy = valid ? dw_dly(g, tab.lx[jj]) * d : 0.0;
             cw = BwdLanes<VT>::reduce_groups(cw);
             cx = BwdLanes<VT>::reduce_groups(cx);
             cy = BwdLanes<VT>::reduce_groups(cy);
@@ -209,9 +213,9 @@ __device__ __forceinline__ void row_backward(const VT* __restrict__ vb, int H, i
             } else {
                 // sample p sits in half 0 (lane 0), sample p + 1 in half 1 (lane 16)
                 const int src = (lane & 1) << 4;
-                const float tw = __shfl_sync(0xffffffffu, cw, src);
-                const float tx = __shfl_sync(0xffffffffu, cx, src);
-                const float ty = __shfl_sync(0xffffffffu, cy, src);
+                const double tw = __shfl_sync(0xffffffffu, cw, src);
+                const double tx = __shfl_sync(0xffffffffu, cx, src);
+                const double ty = __shfl_sync(0xffffffffu, cy, src);
                 if ((lane & ~1) == p) {
                     res_w = tw;
                     res_x = tx;
@@ -220,10 +224,11 @@ __device__ __forceinline__ void row_backward(const VT* __restrict__ vb, int H, i
             }
         }
         if (j < n) {
-            gattn_row[j] = res_w;
-            const float al = a[c];
+            gattn_row[j] = (float)res_w;
+            const double al = a[c];
             *reinterpret_cast<float2*>(gloc_row + 2 * j) =
-                make_float2(cr.valid ? al * Wl * res_x : 0.f, cr.valid ? al * Hl * res_y : 0.f);
+                make_float2(cr.valid ? (float)(al * Wl * res_x) : 0.f,
+                            cr.valid ? (float)(al * Hl * res_y) : 0.f);
         }
         __syncwarp();
     }
