@@ -21,7 +21,7 @@
 
 namespace msda {
 
-constexpr int kBwdRowsPerWarp = 1;
+constexpr int kBwdRowsPerTile = 2;
 
 struct BwdTable {
     int off[4][kMetaStride];
@@ -148,13 +148,12 @@ template <typename VT, bool FUSED, int NC>
 __device__ __forceinline__ void row_backward(const VT* __restrict__ vb, int H, int h,
                                              const float* __restrict__ lo,
                                              const float* __restrict__ wl,
-                                             const float* __restrict__ ref, int L, int P, int R,
-                                             const SmemLevels& lv, BwdTable& tab,
+                                             const float* __restrict__ ref, int n,
+                                             const LaneSamples<NC>& ls, BwdTable& tab,
                                              const float* __restrict__ grow, float scale,
                                              float* __restrict__ gvb, float* __restrict__ gloc_row,
                                              float* __restrict__ gattn_row, int lane)
 {
-    const int n = L * P;
     float a[NC];
     row_weights<FUSED, NC>(wl, n, lane, a);
     BwdLanes<VT> lanes;
@@ -165,14 +164,12 @@ __device__ __forceinline__ void row_backward(const VT* __restrict__ vb, int H, i
         const int j = c * 32 + lane;
         Corners cr;
         float Wl = 0.f, Hl = 0.f;
-        if (j < n) {
-            const int l = j / P, k = j - l * P;
-            const int hl = lv.h[l], wlv = lv.w[l];
+        if (ls.in[c]) {
             float sx, sy;
-            sample_location<FUSED>(lo, ref, j, k, R, hl, wlv, sx, sy);
-            locate(sx, sy, hl, wlv, lv.start[l], H, h, cr);
-            Wl = (float)wlv;
-            Hl = (float)hl;
+            sample_location<FUSED>(lo, ref, j, ls.m[c], ls.h[c], ls.w[c], sx, sy);
+            locate(sx, sy, ls.h[c], ls.w[c], ls.start[c], H, h, cr);
+            Wl = (float)ls.w[c];
+            Hl = (float)ls.h[c];
         } else {
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -247,19 +244,28 @@ msda_backward_kernel(const VT* __restrict__ value, const float* __restrict__ loc
     stage_levels(s_lv, levels);
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t items = (int64_t)B * Nq * H;
+    LaneSamples<NC> ls;
+    lane_samples<NC>(s_lv, L, P, 1, lane, ls);
     const int S = L * P;
-    const int64_t tile0 = (int64_t)blockIdx.x * kWarps * kBwdRowsPerWarp;
-    for (int t = 0; t < kBwdRowsPerWarp; ++t) {
-        const int64_t item = tile0 + (int64_t)t * kWarps + warp;
-        if (item >= items) break;
-        const int h = (int)(item % H);
-        const int b = (int)(item / H / Nq);
+    const int64_t rows = (int64_t)B * Nq;
+    const int64_t row0 = (int64_t)blockIdx.x * kBwdRowsPerTile;
+    const int b0 = (int)(row0 / Nq);
+    const int q0 = (int)(row0 - (int64_t)b0 * Nq);
+    ItemCursor cur(warp, H);
+    for (int it = warp; it < kBwdRowsPerTile * H; it += kWarps, cur.next()) {
+        const int64_t bq = row0 + cur.rr;
+        if (bq >= rows) break;
+        int q = q0 + cur.rr, b = b0;
+        while (q >= Nq) {
+            q -= Nq;
+            ++b;
+        }
+        const int64_t item = bq * H + cur.h;
         const int64_t vofs = (int64_t)b * Nv * H * kHeadDim;
-        row_backward<VT, false, NC>(value + vofs, H, h, loc + item * S * 2, attn + item * S,
-                                    nullptr, L, P, 1, s_lv, s_tab[warp],
-                                    grad_out + item * kHeadDim, 1.f, grad_value + vofs,
-                                    grad_loc + item * S * 2, grad_attn + item * S, lane);
+        row_backward<VT, false, NC>(value + vofs, H, cur.h, loc + item * S * 2, attn + item * S,
+                                    nullptr, S, ls, s_tab[warp], grad_out + item * kHeadDim, 1.f,
+                                    grad_value + vofs, grad_loc + item * S * 2,
+                                    grad_attn + item * S, lane);
     }
 }
 
@@ -280,26 +286,38 @@ sca_backward_kernel(const VT* __restrict__ value, const float* __restrict__ off,
     stage_levels(s_lv, levels);
     stage_row_prefix(count, nbc, s_prefix);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t items = (int64_t)s_prefix[nbc] * H;
+    LaneSamples<NC> ls;
+    lane_samples<NC>(s_lv, L, P, R, lane, ls);
     const int S = L * P;
-    for (int64_t item = (int64_t)blockIdx.x * kWarps + warp; item < items;
-         item += (int64_t)gridDim.x * kWarps) {
-        const int r = (int)(item / H), h = (int)(item % H);
-        const int bc = find_segment(s_prefix, nbc, r);
-        const int i = r - s_prefix[bc];
-        const int b = bc / Ncam, c = bc - b * Ncam;
-        const int q = __ldg(idx + (int64_t)bc * Nq + i);
-        if ((unsigned)q >= (unsigned)Nq) continue;  // inconsistent lists: read nothing
-        const int64_t bq = (int64_t)b * Nq + q;
-        const int64_t bqh = bq * H + h;
-        const int64_t vofs = (int64_t)bc * Nv * H * kHeadDim;
-        const int64_t rowh = ((int64_t)bc * Nq + i) * H + h;
-        const float scale = (float)max(1, __ldg(hits + bq));
-        row_backward<VT, true, NC>(value + vofs, H, h, off + bqh * S * 2, logits + bqh * S,
-                                   ref_cam + (((int64_t)c * B + b) * Nq + q) * R * 2, L, P, R,
-                                   s_lv, s_tab[warp], grad_out + bqh * kHeadDim, scale,
-                                   grad_value + vofs, grad_loc_rb + rowh * S * 2,
-                                   grad_attn_rb + rowh * S, lane);
+    const int total = s_prefix[nbc];
+    int bc = 0, b = 0, c = 0, bc_cached = -1;
+    for (int64_t tile = blockIdx.x; tile * kBwdRowsPerTile < total; tile += gridDim.x) {
+        const int r0 = (int)(tile * kBwdRowsPerTile);
+        ItemCursor cur(warp, H);
+        for (int it = warp; it < kBwdRowsPerTile * H; it += kWarps, cur.next()) {
+            const int r = r0 + cur.rr;
+            if (r >= total) break;
+            while (r >= s_prefix[bc + 1]) ++bc;  // rows only grow: bc is monotone
+            if (bc != bc_cached) {
+                b = bc / Ncam;
+                c = bc - b * Ncam;
+                bc_cached = bc;
+            }
+            const int i = r - s_prefix[bc];
+            const int q = __ldg(idx + (int64_t)bc * Nq + i);
+            if ((unsigned)q >= (unsigned)Nq) continue;  // inconsistent lists: read nothing
+            const int h = cur.h;
+            const int64_t bq = (int64_t)b * Nq + q;
+            const int64_t bqh = bq * H + h;
+            const int64_t vofs = (int64_t)bc * Nv * H * kHeadDim;
+            const int64_t rowh = ((int64_t)bc * Nq + i) * H + h;
+            const float scale = (float)max(1, __ldg(hits + bq));
+            row_backward<VT, true, NC>(value + vofs, H, h, off + bqh * S * 2, logits + bqh * S,
+                                       ref_cam + (((int64_t)c * B + b) * Nq + q) * R * 2, S, ls,
+                                       s_tab[warp], grad_out + bqh * kHeadDim, scale,
+                                       grad_value + vofs, grad_loc_rb + rowh * S * 2,
+                                       grad_attn_rb + rowh * S, lane);
+        }
     }
 }
 
@@ -361,10 +379,9 @@ static cudaError_t launch_msda_backward_t(const Problem& p, const float* loc, co
                                           const float* grad_out, float* grad_value,
                                           float* grad_loc, float* grad_attn, cudaStream_t s)
 {
-    const int64_t items = (int64_t)p.B * p.Nq * p.H;
-    if (items == 0) return cudaSuccess;
-    const int64_t per_cta = (int64_t)kWarps * kBwdRowsPerWarp;
-    const unsigned grid = (unsigned)((items + per_cta - 1) / per_cta);
+    const int64_t rows = (int64_t)p.B * p.Nq;
+    if (rows == 0) return cudaSuccess;
+    const unsigned grid = (unsigned)((rows + kBwdRowsPerTile - 1) / kBwdRowsPerTile);
     const VT* v = static_cast<const VT*>(p.value);
     const int nc = (p.L * p.P + 31) / 32;
 #define MSDA_BWD_CASE(NCV)                                                                       \
@@ -410,9 +427,9 @@ static cudaError_t launch_sca_backward_t(const Problem& p, const float* ref_cam,
                                          const int32_t* count, float* grad_value,
                                          float* grad_loc_rb, float* grad_attn_rb, cudaStream_t s)
 {
-    const int64_t max_items = (int64_t)p.B * p.Ncam * p.Nq * p.H;
-    if (max_items == 0) return cudaSuccess;
-    const int64_t max_ctas = (max_items + kWarps - 1) / kWarps;
+    const int64_t max_rows = (int64_t)p.B * p.Ncam * p.Nq;
+    if (max_rows == 0) return cudaSuccess;
+    const int64_t max_ctas = (max_rows + kBwdRowsPerTile - 1) / kBwdRowsPerTile;
     const VT* v = static_cast<const VT*>(p.value);
     const int nc = (p.L * p.P + 31) / 32;
 #define SCA_BWD_CASE(NCV)                                                                        \

@@ -31,6 +31,18 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kMetaStride = 36;         // words per corner row of the sample table
 constexpr int kMaxBatchCameras = 1024;  // B * Ncam limit of the SCA kernels
 
+// Build-time tuning of the gather kernels (defaults are the tuned values).
+#ifndef MSDA_GATHER_UNROLL
+#define MSDA_GATHER_UNROLL 4   // table quads unrolled in the gather loop
+#endif
+#ifndef MSDA_ROWS_PER_TILE
+#define MSDA_ROWS_PER_TILE 8   // consecutive rows per CTA tile (<= 32)
+#endif
+#ifndef MSDA_MIN_CTAS
+#define MSDA_MIN_CTAS 1        // __launch_bounds__ minimum resident CTAs per SM
+#endif
+constexpr int kGatherUnroll = MSDA_GATHER_UNROLL;
+
 // Level geometry, passed by value to every kernel.
 struct Levels {
     int h[kMaxLevels];      // rows H_l
@@ -60,11 +72,13 @@ __device__ __forceinline__ void stage_levels(SmemLevels& s, const Levels& lv)
     }
 }
 
+// Maximum over the warp in one instruction (sm_100a redux.sync on f32; a NaN
+// lane is ignored like fmaxf ignores it).
 __device__ __forceinline__ float warp_max(float v)
 {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    return v;
+    float r;
+    asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+    return r;
 }
 
 __device__ __forceinline__ float warp_sum(float v)
@@ -154,17 +168,44 @@ __device__ __forceinline__ void locate(float sx, float sy, int Hl, int Wl, int s
     }
 }
 
-// Sampling location of sample j = (l, k) of one (row, head).
-// FUSED: rho_{k mod R} + (dx / W_l, dy / H_l), each step one rounded binary32
+// What lane `lane` needs to know about its samples j = c * 32 + lane of every
+// row: the sample's level geometry and its anchor m(k) = k mod R.  The same for
+// every row and head, so a warp computes it once, before its row loop.
+template <int NC>
+struct LaneSamples {
+    int w[NC], h[NC], start[NC];  // level of sample j (W_l, H_l, first row)
+    int m[NC];                    // anchor of point k: k mod R
+    bool in[NC];                  // j < L * P
+};
+
+template <int NC>
+__device__ __forceinline__ void lane_samples(const SmemLevels& lv, int L, int P, int R, int lane,
+                                             LaneSamples<NC>& ls)
+{
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+        const int j = c * 32 + lane;
+        ls.in[c] = j < L * P;
+        const int l = ls.in[c] ? j / P : 0;
+        const int k = j - l * P;
+        ls.w[c] = lv.w[l];
+        ls.h[c] = lv.h[l];
+        ls.start[c] = lv.start[l];
+        ls.m[c] = ls.in[c] ? k % R : 0;
+    }
+}
+
+// Sampling location of sample j of one (row, head).
+// FUSED: rho_{m} + (dx / W_l, dy / H_l), each step one rounded binary32
 // operation (section 5); otherwise the given location.
 template <bool FUSED>
 __device__ __forceinline__ void sample_location(const float* __restrict__ lo,
-                                                const float* __restrict__ ref, int j, int k,
-                                                int R, int Hl, int Wl, float& sx, float& sy)
+                                                const float* __restrict__ ref, int j, int m,
+                                                int Hl, int Wl, float& sx, float& sy)
 {
     const float2 v = ld_stream2(lo + 2 * j);
     if (FUSED) {
-        const float2 r = __ldg(reinterpret_cast<const float2*>(ref) + (k % R));
+        const float2 r = __ldg(reinterpret_cast<const float2*>(ref) + m);
         sx = __fadd_rn(r.x, __fdiv_rn(v.x, (float)Wl));
         sy = __fadd_rn(r.y, __fdiv_rn(v.y, (float)Hl));
     } else {
@@ -196,7 +237,7 @@ struct Gather<float> {
         const int g = lane >> 3, t = lane & 7;
         const float* v = vb + 4 * t;
         const int quads = (cnt + 3) >> 2;
-#pragma unroll 2
+#pragma unroll kGatherUnroll
         for (int p = 0; p < quads; ++p) {
             const int4 o = *reinterpret_cast<const int4*>(&tab.off[g][4 * p]);
             const float4 w = *reinterpret_cast<const float4*>(&tab.w[g][4 * p]);
@@ -250,7 +291,7 @@ struct Gather<__nv_bfloat16> {
         const int half = lane >> 4, g = (lane >> 2) & 3, t = lane & 3;
         const __nv_bfloat16* v = vb + 8 * t;
         const int quads = (cnt + 3) >> 2;
-#pragma unroll 2
+#pragma unroll kGatherUnroll
         for (int p = 0; p < quads; ++p) {
             const int4 o = *reinterpret_cast<const int4*>(&tab.off[g][4 * p]);
             const float4 w = *reinterpret_cast<const float4*>(&tab.w[g][4 * p]);
@@ -280,46 +321,101 @@ struct Gather<__nv_bfloat16> {
     }
 };
 
-// One output row of one head (all L*P samples), written to out_row[0..32).
-//   vb      value of this batch item (and camera): [Nv, H, 32]
-//   lo      FUSED: pixel offsets, else locations, of this (row, head): [L, P, 2]
-//   wl      FUSED: logits, else weights, of this (row, head): [L, P]
-//   ref     FUSED only: reference points of this row: [R, 2]
+// Inputs of one row for HP heads, per lane (samples j = c * 32 + lane): the
+// logits (or weights), the pixel offsets (or locations) and, fused, the
+// reference point of the sample's anchor.  Loaded one row ahead of their use
+// so that their memory latency overlaps the previous row's gather.
+template <bool FUSED, int NC, int HP>
+struct RowIn {
+    float a[HP][NC];
+    float2 lo[HP][NC];
+    float2 rf[NC];
+};
+
+// lo, wl: the row's first head; head s follows at +2 s n (lo) and +s n (wl).
+template <bool FUSED, int NC, int HP>
+__device__ __forceinline__ void load_row(const float* __restrict__ lo,
+                                         const float* __restrict__ wl,
+                                         const float* __restrict__ ref, int n,
+                                         const LaneSamples<NC>& ls, int lane,
+                                         RowIn<FUSED, NC, HP>& in)
+{
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+        const int j = c * 32 + lane;
+#pragma unroll
+        for (int s = 0; s < HP; ++s) {
+            in.a[s][c] = ls.in[c] ? ld_stream(wl + s * n + j) : (FUSED ? -INFINITY : 0.f);
+            in.lo[s][c] = ls.in[c] ? ld_stream2(lo + s * 2 * n + 2 * j) : make_float2(0.f, 0.f);
+        }
+        in.rf[c] = (FUSED && ls.in[c]) ? __ldg(reinterpret_cast<const float2*>(ref) + ls.m[c])
+                                       : make_float2(0.f, 0.f);
+    }
+}
+
+// Softmax over the L*P logits of one head, in place (section 4.2).
+template <bool FUSED, int NC>
+__device__ __forceinline__ void normalise(float (&a)[NC], const LaneSamples<NC>& ls)
+{
+    if (!FUSED) return;
+    float m = a[0];
+#pragma unroll
+    for (int c = 1; c < NC; ++c) m = fmaxf(m, a[c]);
+    m = warp_max(m);
+    float z = 0.f;
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+        a[c] = ls.in[c] ? expf(a[c] - m) : 0.f;
+        z += a[c];
+    }
+    z = warp_sum(z);
+#pragma unroll
+    for (int c = 0; c < NC; ++c) a[c] = a[c] / z;
+}
+
+// Corners of the lane's sample of chunk c, head h (section 5 location, section
+// 6 corner decision).
+template <bool FUSED, int NC>
+__device__ __forceinline__ void lane_corners(float2 v, float2 r, const LaneSamples<NC>& ls, int c,
+                                             int H, int h, Corners& cr)
+{
+    if (ls.in[c]) {
+        float sx = v.x, sy = v.y;
+        if (FUSED) {
+            sx = __fadd_rn(r.x, __fdiv_rn(v.x, (float)ls.w[c]));
+            sy = __fadd_rn(r.y, __fdiv_rn(v.y, (float)ls.h[c]));
+        }
+        locate(sx, sy, ls.h[c], ls.w[c], ls.start[c], H, h, cr);
+    } else {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            cr.off[g] = -1;
+            cr.w[g] = 0.f;
+        }
+    }
+}
+
+// One output row of one head (all n = L*P samples) from its loaded inputs,
+// written to out_row[0..32).  vb: value of this batch item (and camera),
+// [Nv, H, 32].
 template <typename VT, bool FUSED, int NC>
-__device__ __forceinline__ void row_forward(const VT* __restrict__ vb, int H, int h,
-                                            const float* __restrict__ lo,
-                                            const float* __restrict__ wl,
-                                            const float* __restrict__ ref, int L, int P, int R,
-                                            const SmemLevels& lv, WarpTable& tab,
+__device__ __forceinline__ void row_compute(const VT* __restrict__ vb, int H, int h,
+                                            RowIn<FUSED, NC, 1>& in, int n,
+                                            const LaneSamples<NC>& ls, WarpTable& tab,
                                             float* __restrict__ out_row, int lane)
 {
-    const int n = L * P;
-    float a[NC];
-    row_weights<FUSED, NC>(wl, n, lane, a);
+    normalise<FUSED, NC>(in.a[0], ls);
     float acc[Gather<VT>::kAcc];
 #pragma unroll
     for (int i = 0; i < Gather<VT>::kAcc; ++i) acc[i] = 0.f;
 #pragma unroll
     for (int c = 0; c < NC; ++c) {
-        const int j = c * 32 + lane;
         Corners cr;
-        if (j < n) {
-            const int l = j / P, k = j - l * P;
-            const int Hl = lv.h[l], Wl = lv.w[l];
-            float sx, sy;
-            sample_location<FUSED>(lo, ref, j, k, R, Hl, Wl, sx, sy);
-            locate(sx, sy, Hl, Wl, lv.start[l], H, h, cr);
-        } else {
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                cr.off[g] = -1;
-                cr.w[g] = 0.f;
-            }
-        }
+        lane_corners<FUSED, NC>(in.lo[0][c], in.rf[c], ls, c, H, h, cr);
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
             tab.off[g][lane] = cr.off[g];
-            tab.w[g][lane] = cr.w[g] * a[c];
+            tab.w[g][lane] = cr.w[g] * in.a[0][c];
         }
         __syncwarp();
         Gather<VT>::run(vb, tab, min(32, n - c * 32), lane, acc);
@@ -327,6 +423,100 @@ __device__ __forceinline__ void row_forward(const VT* __restrict__ vb, int H, in
     }
     Gather<VT>::store(acc, lane, out_row);
 }
+
+// bf16 value, two heads per warp.  A bf16 head slice is 64 bytes, and every
+// slice of head h sits in the same half of its 128-byte line ((h * 64) mod
+// 128), so four corners of one head always collide on the same L1 banks.
+// Pairing heads 2m and 2m+1 in one warp puts the two halves of every warp load
+// on opposite bank halves: lanes 16s + 4g + t read corner g of a sample of
+// head 2m + s, channels 8t..8t+7.
+struct PairTable {
+    int off[2][4][kMetaStride];
+    float w[2][4][kMetaStride];
+};
+
+// Heads h0 and h0 + 1 of one row; out_row0 is head h0's output, head h0 + 1
+// follows at +32.
+template <bool FUSED, int NC>
+__device__ __forceinline__ void row_compute_pair(const __nv_bfloat16* __restrict__ vb, int H,
+                                                 int h0, RowIn<FUSED, NC, 2>& in, int n,
+                                                 const LaneSamples<NC>& ls, PairTable& tab,
+                                                 float* __restrict__ out_row0, int lane)
+{
+    normalise<FUSED, NC>(in.a[0], ls);
+    normalise<FUSED, NC>(in.a[1], ls);
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    const int half = lane >> 4, g = (lane >> 2) & 3, t = lane & 3;
+    const __nv_bfloat16* v = vb + 8 * t;
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+#pragma unroll
+        for (int sh = 0; sh < 2; ++sh) {
+            Corners cr;
+            lane_corners<FUSED, NC>(in.lo[sh][c], in.rf[c], ls, c, H, h0 + sh, cr);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                tab.off[sh][q][lane] = cr.off[q];
+                tab.w[sh][q][lane] = cr.w[q] * in.a[sh][c];
+            }
+        }
+        __syncwarp();
+        const int quads = (min(32, n - c * 32) + 3) >> 2;
+#pragma unroll kGatherUnroll
+        for (int p = 0; p < quads; ++p) {
+            const int4 o = *reinterpret_cast<const int4*>(&tab.off[half][g][4 * p]);
+            const float4 w = *reinterpret_cast<const float4*>(&tab.w[half][g][4 * p]);
+            uint4 r0 = make_uint4(0u, 0u, 0u, 0u), r1 = r0, r2 = r0, r3 = r0;
+            if (o.x >= 0) r0 = __ldg(reinterpret_cast<const uint4*>(v + o.x));
+            if (o.y >= 0) r1 = __ldg(reinterpret_cast<const uint4*>(v + o.y));
+            if (o.z >= 0) r2 = __ldg(reinterpret_cast<const uint4*>(v + o.z));
+            if (o.w >= 0) r3 = __ldg(reinterpret_cast<const uint4*>(v + o.w));
+            Gather<__nv_bfloat16>::fma8(acc, w.x, r0);
+            Gather<__nv_bfloat16>::fma8(acc, w.y, r1);
+            Gather<__nv_bfloat16>::fma8(acc, w.z, r2);
+            Gather<__nv_bfloat16>::fma8(acc, w.w, r3);
+        }
+        __syncwarp();
+    }
+    // sum the four corners; lanes 16s + t (g = 0) store head h0 + s, channels 8t..8t+7
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 4);
+        acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 8);
+    }
+    if (g == 0) {
+        float4* o = reinterpret_cast<float4*>(out_row0 + half * kHeadDim + 8 * t);
+        o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    }
+}
+
+// Walks the (row, head) items of one warp without divisions: items are
+// row * H + h, a warp takes every kWarps-th item of its CTA's tile of
+// `rows` consecutive rows, so each step adds kWarps / H rows and
+// kWarps % H heads (with a carry).
+struct ItemCursor {
+    int rr, h;        // row within the tile, head
+    int drr, dh, H;
+    __device__ __forceinline__ ItemCursor(int warp, int H_) : H(H_)
+    {
+        rr = warp / H;
+        h = warp - rr * H;
+        drr = kWarps / H;
+        dh = kWarps - drr * H;
+    }
+    __device__ __forceinline__ void next()
+    {
+        rr += drr;
+        h += dh;
+        if (h >= H) {
+            h -= H;
+            ++rr;
+        }
+    }
+};
 
 // Row offsets of the rebatched layout: s_prefix[bc] = sum of count[0..bc),
 // s_prefix[n] = total rows.  Warp 0 scans; the whole block must call this.

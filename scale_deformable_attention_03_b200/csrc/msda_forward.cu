@@ -1,57 +1,103 @@
 // K1 / K1f: MSDA forward, one warp per (batch, query, head).
 //
-// Item order is (b, q, h) with h fastest, so the eight warps of a CTA take
-// the eight heads of one query; a CTA then walks kRowsPerWarp consecutive
-// queries, which keeps neighbouring queries' reads of the same head slices in
-// the SM's L1.
+// Item order is (b, q, h) with h fastest.  A CTA owns a tile of
+// kRowsPerTile consecutive queries; with H = 8 each of its eight warps keeps
+// one head and walks the tile's queries, so neighbouring queries' reads of the
+// same head slices meet in the SM's L1.  No integer division in the loop; each
+// warp loads the next query's inputs before gathering the current one.
+#include <type_traits>
+
 #include "msda_launch.h"
 
 namespace msda {
 
-constexpr int kRowsPerWarp = 2;
+constexpr int kRowsPerTile = MSDA_ROWS_PER_TILE;
 
-template <typename VT, bool FUSED, int NC>
-__global__ void __launch_bounds__(kThreads)
+template <typename VT, bool FUSED, int NC, int HP>
+__global__ void __launch_bounds__(kThreads, MSDA_MIN_CTAS)
 msda_forward_kernel(const VT* __restrict__ value, const float* __restrict__ lo,
                     const float* __restrict__ wl, const float* __restrict__ ref,
                     float* __restrict__ out, int B, int Nq, int Nv, int H, int L, int P, int R,
                     Levels levels)
 {
+    using Table = typename std::conditional<HP == 2, PairTable, WarpTable>::type;
     __shared__ SmemLevels s_lv;
-    __shared__ __align__(16) WarpTable s_tab[kWarps];
+    __shared__ __align__(16) Table s_tab[kWarps];
     stage_levels(s_lv, levels);
     __syncthreads();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t items = (int64_t)B * Nq * H;
-    const int64_t tile0 = (int64_t)blockIdx.x * kWarps * kRowsPerWarp;
+    LaneSamples<NC> ls;
+    lane_samples<NC>(s_lv, L, P, R, lane, ls);
     const int S = L * P;
-    for (int t = 0; t < kRowsPerWarp; ++t) {
-        const int64_t item = tile0 + (int64_t)t * kWarps + warp;  // (b * Nq + q) * H + h
-        if (item >= items) break;
-        const int h = (int)(item % H);
-        const int64_t bq = item / H;
-        const int b = (int)(bq / Nq);
-        const VT* vb = value + (int64_t)b * Nv * H * kHeadDim;
-        row_forward<VT, FUSED, NC>(vb, H, h, lo + item * S * 2, wl + item * S,
-                                   FUSED ? ref + bq * R * 2 : nullptr, L, P, R, s_lv, s_tab[warp],
-                                   out + item * kHeadDim, lane);
+    const int64_t rows = (int64_t)B * Nq;
+    const int64_t row0 = (int64_t)blockIdx.x * kRowsPerTile;
+    const int b0 = (int)(row0 / Nq);
+    const int q0 = (int)(row0 - (int64_t)b0 * Nq);
+    const int HG = H / HP;  // head groups: one per warp item
+    const int n_items = kRowsPerTile * HG;
+
+    struct Item {
+        bool ok;
+        int b, h;
+        int64_t bq;
+    };
+    auto resolve = [&](int it, const ItemCursor& cur) {
+        Item x;
+        x.bq = row0 + cur.rr;
+        x.ok = it < n_items && x.bq < rows;
+        x.h = cur.h * HP;
+        int q = q0 + cur.rr;
+        x.b = b0;
+        while (q >= Nq) {
+            q -= Nq;
+            ++x.b;
+        }
+        return x;
+    };
+    auto fetch = [&](const Item& x, RowIn<FUSED, NC, HP>& in) {
+        const int64_t item = x.bq * H + x.h;
+        load_row<FUSED, NC, HP>(lo + item * S * 2, wl + item * S, FUSED ? ref + x.bq * R * 2 : nullptr,
+                                S, ls, lane, in);
+    };
+
+    ItemCursor cur(warp, HG);
+    int it = warp;
+    Item x0 = resolve(it, cur);
+    RowIn<FUSED, NC, HP> in0, in1;
+    if (x0.ok) fetch(x0, in0);
+    while (x0.ok) {
+        ItemCursor nx = cur;
+        nx.next();
+        const Item x1 = resolve(it + kWarps, nx);
+        if (x1.ok) fetch(x1, in1);  // next row's inputs in flight during this gather
+        const int64_t item = x0.bq * H + x0.h;
+        const VT* vb = value + (int64_t)x0.b * Nv * H * kHeadDim;
+        if constexpr (HP == 2)
+            row_compute_pair<FUSED, NC>(vb, H, x0.h, in0, S, ls, s_tab[warp],
+                                        out + item * kHeadDim, lane);
+        else
+            row_compute<VT, FUSED, NC>(vb, H, x0.h, in0, S, ls, s_tab[warp],
+                                       out + item * kHeadDim, lane);
+        x0 = x1;
+        in0 = in1;
+        cur = nx;
+        it += kWarps;
     }
 }
 
-template <typename VT, bool FUSED>
+template <typename VT, bool FUSED, int HP>
 static cudaError_t launch_fwd(const Problem& p, const float* lo, const float* wl,
                               const float* ref, float* out, cudaStream_t s)
 {
-    const int64_t items = (int64_t)p.B * p.Nq * p.H;
-    if (items == 0) return cudaSuccess;
-    const int64_t per_cta = (int64_t)kWarps * kRowsPerWarp;
-    const unsigned grid = (unsigned)((items + per_cta - 1) / per_cta);
+    const int64_t rows = (int64_t)p.B * p.Nq;
+    if (rows == 0) return cudaSuccess;
+    const unsigned grid = (unsigned)((rows + kRowsPerTile - 1) / kRowsPerTile);
     const VT* v = static_cast<const VT*>(p.value);
     const int nc = (p.L * p.P + 31) / 32;
 #define MSDA_FWD_CASE(NCV)                                                                       \
     case NCV:                                                                                    \
-        msda_forward_kernel<VT, FUSED, NCV><<<grid, kThreads, 0, s>>>(                           \
+        msda_forward_kernel<VT, FUSED, NCV, HP><<<grid, kThreads, 0, s>>>(                       \
             v, lo, wl, ref, out, p.B, p.Nq, p.Nv, p.H, p.L, p.P, p.R, p.lv);                     \
         break;
     switch (nc) {
@@ -68,15 +114,17 @@ static cudaError_t launch_fwd(const Problem& p, const float* lo, const float* wl
 cudaError_t launch_msda_forward(const Problem& p, const float* loc, const float* attn,
                                 float* out, cudaStream_t s)
 {
-    return p.bf16 ? launch_fwd<__nv_bfloat16, false>(p, loc, attn, nullptr, out, s)
-                  : launch_fwd<float, false>(p, loc, attn, nullptr, out, s);
+    if (!p.bf16) return launch_fwd<float, false, 1>(p, loc, attn, nullptr, out, s);
+    if (p.H % 2 == 0) return launch_fwd<__nv_bfloat16, false, 2>(p, loc, attn, nullptr, out, s);
+    return launch_fwd<__nv_bfloat16, false, 1>(p, loc, attn, nullptr, out, s);
 }
 
 cudaError_t launch_msda_forward_fused(const Problem& p, const float* ref, const float* off,
                                       const float* logits, float* out, cudaStream_t s)
 {
-    return p.bf16 ? launch_fwd<__nv_bfloat16, true>(p, off, logits, ref, out, s)
-                  : launch_fwd<float, true>(p, off, logits, ref, out, s);
+    if (!p.bf16) return launch_fwd<float, true, 1>(p, off, logits, ref, out, s);
+    if (p.H % 2 == 0) return launch_fwd<__nv_bfloat16, true, 2>(p, off, logits, ref, out, s);
+    return launch_fwd<__nv_bfloat16, true, 1>(p, off, logits, ref, out, s);
 }
 
 }  // namespace msda

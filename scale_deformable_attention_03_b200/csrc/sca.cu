@@ -7,13 +7,14 @@
 // Nothing here synchronises with the host: the rebatched row counts live in
 // device memory and K3 is a persistent kernel that reads them.
 #include <algorithm>
+#include <type_traits>
 
 #include "msda_launch.h"
 
 namespace msda {
 
 constexpr int kMaxCameras = 32;
-constexpr int kScaRowsPerWarp = 2;
+constexpr int kScaRowsPerTile = MSDA_ROWS_PER_TILE;  // <= 32: a lane resolves each row
 
 __device__ __forceinline__ int warp_sum_int(int v)
 {
@@ -139,45 +140,98 @@ cudaError_t launch_sca_compact(const uint8_t* mask, int B, int Ncam, int Nq, int
 }
 
 // Rows are ordered (b, c, i): at any time the whole GPU works on a narrow
-// window of rows of one camera, so that camera's value stays in L2.  Offsets
-// and logits come from the BEV query and are shared by its cameras; the
-// reference points are the camera's own.
-template <typename VT, int NC>
-__global__ void __launch_bounds__(kThreads)
+// window of rows of one camera, so that camera's value stays in L2.  A CTA
+// takes tiles of kScaRowsPerTile consecutive rows (with H = 8, one head per
+// warp), so neighbouring queries' reads of the same head slices meet in L1.
+// Offsets and logits come from the BEV query and are shared by its cameras;
+// the reference points are the camera's own.
+template <typename VT, int NC, int HP>
+__global__ void __launch_bounds__(kThreads, MSDA_MIN_CTAS)
 sca_gather_kernel(const VT* __restrict__ value, const float* __restrict__ off,
                   const float* __restrict__ logits, const float* __restrict__ ref_cam,
                   const int32_t* __restrict__ idx, const int32_t* __restrict__ count,
                   float* __restrict__ out_rb, int B, int Ncam, int Nq, int Nv, int H, int L,
                   int P, int R, Levels levels)
 {
+    using Table = typename std::conditional<HP == 2, PairTable, WarpTable>::type;
     __shared__ SmemLevels s_lv;
-    __shared__ __align__(16) WarpTable s_tab[kWarps];
+    __shared__ __align__(16) Table s_tab[kWarps];
     __shared__ int s_prefix[kMaxBatchCameras + 1];
     const int nbc = B * Ncam;
     stage_levels(s_lv, levels);
     stage_row_prefix(count, nbc, s_prefix);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t items = (int64_t)s_prefix[nbc] * H;
-    const int64_t per_tile = (int64_t)kWarps * kScaRowsPerWarp;
+    LaneSamples<NC> ls;
+    lane_samples<NC>(s_lv, L, P, R, lane, ls);
     const int S = L * P;
-    for (int64_t tile0 = (int64_t)blockIdx.x * per_tile; tile0 < items;
-         tile0 += (int64_t)gridDim.x * per_tile) {
-        for (int t = 0; t < kScaRowsPerWarp; ++t) {
-            const int64_t item = tile0 + (int64_t)t * kWarps + warp;  // row * H + h
-            if (item >= items) break;
-            const int r = (int)(item / H), h = (int)(item % H);
-            const int bc = find_segment(s_prefix, nbc, r);
-            const int i = r - s_prefix[bc];
-            const int b = bc / Ncam, c = bc - b * Ncam;
-            const int q = __ldg(idx + (int64_t)bc * Nq + i);
-            if ((unsigned)q >= (unsigned)Nq) continue;  // inconsistent lists: read nothing
-            const int64_t bqh = ((int64_t)b * Nq + q) * H + h;
-            const VT* vb = value + (int64_t)bc * Nv * H * kHeadDim;
-            const float* rf = ref_cam + (((int64_t)c * B + b) * Nq + q) * R * 2;
-            float* orow = out_rb + (((int64_t)bc * Nq + i) * H + h) * kHeadDim;
-            row_forward<VT, true, NC>(vb, H, h, off + bqh * S * 2, logits + bqh * S, rf, L, P, R,
-                                      s_lv, s_tab[warp], orow, lane);
+    const int total = s_prefix[nbc];
+    const int HG = H / HP;  // head groups: one per warp item
+    const int n_items = kScaRowsPerTile * HG;
+    int bc_lane = 0;  // lane's (batch, camera) search start: its rows only grow
+
+    struct Item {
+        bool ok, skip;
+        int h, bc, in_row, ref_row, out_row;
+    };
+    for (int64_t tile = blockIdx.x; tile * kScaRowsPerTile < total; tile += gridDim.x) {
+        const int r0 = (int)(tile * kScaRowsPerTile);
+        // lane i < kScaRowsPerTile resolves row r0 + i of the tile: one coalesced index load
+        int my_bc = 0, my_in = -1, my_ref = 0, my_out = 0;
+        {
+            const int r = r0 + lane;
+            if (lane < kScaRowsPerTile && r < total) {
+                while (r >= s_prefix[bc_lane + 1]) ++bc_lane;
+                const int i = r - s_prefix[bc_lane];
+                const int b = bc_lane / Ncam, c = bc_lane - b * Ncam;
+                const int q = __ldg(idx + (int64_t)bc_lane * Nq + i);
+                if ((unsigned)q < (unsigned)Nq) {  // inconsistent lists: read nothing
+                    my_bc = bc_lane;
+                    my_in = b * Nq + q;
+                    my_ref = (c * B + b) * Nq + q;
+                    my_out = bc_lane * Nq + i;
+                }
+            }
+        }
+        auto resolve = [&](int it, const ItemCursor& cur) {
+            Item x;
+            const int rr = cur.rr;
+            x.ok = it < n_items && r0 + rr < total;  // warp-uniform
+            x.h = cur.h * HP;
+            x.bc = __shfl_sync(0xffffffffu, my_bc, rr & 31);
+            x.in_row = __shfl_sync(0xffffffffu, my_in, rr & 31);
+            x.ref_row = __shfl_sync(0xffffffffu, my_ref, rr & 31);
+            x.out_row = __shfl_sync(0xffffffffu, my_out, rr & 31);
+            x.skip = x.in_row < 0;
+            return x;
+        };
+        auto fetch = [&](const Item& x, RowIn<true, NC, HP>& in) {
+            const int64_t bqh = (int64_t)x.in_row * H + x.h;
+            load_row<true, NC, HP>(off + bqh * S * 2, logits + bqh * S,
+                                   ref_cam + (int64_t)x.ref_row * R * 2, S, ls, lane, in);
+        };
+        ItemCursor cur(warp, HG);
+        int it = warp;
+        Item x0 = resolve(it, cur);
+        RowIn<true, NC, HP> in0, in1;
+        if (x0.ok && !x0.skip) fetch(x0, in0);
+        while (x0.ok) {
+            ItemCursor nx = cur;
+            nx.next();
+            const Item x1 = resolve(it + kWarps, nx);
+            if (x1.ok && !x1.skip) fetch(x1, in1);  // next row's inputs in flight during this gather
+            if (!x0.skip) {
+                const VT* vb = value + (int64_t)x0.bc * Nv * H * kHeadDim;
+                float* orow = out_rb + ((int64_t)x0.out_row * H + x0.h) * kHeadDim;
+                if constexpr (HP == 2)
+                    row_compute_pair<true, NC>(vb, H, x0.h, in0, S, ls, s_tab[warp], orow, lane);
+                else
+                    row_compute<VT, true, NC>(vb, H, x0.h, in0, S, ls, s_tab[warp], orow, lane);
+            }
+            x0 = x1;
+            in0 = in1;
+            cur = nx;
+            it += kWarps;
         }
     }
 }
@@ -191,22 +245,22 @@ static int resident_ctas(K kernel, int threads)
     return n;
 }
 
-template <typename VT>
+template <typename VT, int HP>
 static cudaError_t launch_gather_t(const Problem& p, const float* ref_cam, const float* off,
                                    const float* logits, const int32_t* idx,
                                    const int32_t* count, float* out_rb, cudaStream_t s)
 {
     const int64_t max_items = (int64_t)p.B * p.Ncam * p.Nq * p.H;
     if (max_items == 0) return cudaSuccess;
-    const int64_t per_tile = (int64_t)kWarps * kScaRowsPerWarp;
-    const int64_t max_tiles = (max_items + per_tile - 1) / per_tile;
+    const int64_t max_rows = (int64_t)p.B * p.Ncam * p.Nq;
+    const int64_t max_tiles = (max_rows + kScaRowsPerTile - 1) / kScaRowsPerTile;
     const VT* v = static_cast<const VT*>(p.value);
     const int nc = (p.L * p.P + 31) / 32;
 #define SCA_GATHER_CASE(NCV)                                                                     \
     case NCV: {                                                                                  \
-        static int occ = resident_ctas(sca_gather_kernel<VT, NCV>, kThreads);                    \
+        static int occ = resident_ctas(sca_gather_kernel<VT, NCV, HP>, kThreads);                \
         const int64_t grid = std::min<int64_t>(max_tiles, (int64_t)occ * device_sm_count());     \
-        sca_gather_kernel<VT, NCV><<<(unsigned)grid, kThreads, 0, s>>>(                          \
+        sca_gather_kernel<VT, NCV, HP><<<(unsigned)grid, kThreads, 0, s>>>(                      \
             v, off, logits, ref_cam, idx, count, out_rb, p.B, p.Ncam, p.Nq, p.Nv, p.H, p.L,      \
             p.P, p.R, p.lv);                                                                     \
         break;                                                                                   \
@@ -226,12 +280,19 @@ cudaError_t launch_sca_gather(const Problem& p, const float* ref_cam, const floa
                               const float* logits, const int32_t* idx, const int32_t* count,
                               float* out_rb, cudaStream_t s)
 {
-    return p.bf16 ? launch_gather_t<__nv_bfloat16>(p, ref_cam, off, logits, idx, count, out_rb, s)
-                  : launch_gather_t<float>(p, ref_cam, off, logits, idx, count, out_rb, s);
+    if (!p.bf16) return launch_gather_t<float, 1>(p, ref_cam, off, logits, idx, count, out_rb, s);
+    if (p.H % 2 == 0)
+        return launch_gather_t<__nv_bfloat16, 2>(p, ref_cam, off, logits, idx, count, out_rb, s);
+    return launch_gather_t<__nv_bfloat16, 1>(p, ref_cam, off, logits, idx, count, out_rb, s);
 }
 
 // One thread per 16-byte piece of an output row; cameras summed in ascending
 // order, then divided by max(1, hits) (the clamp of the average listing).
+// Cameras are taken eight at a time: all eight positions are loaded, then all
+// eight rows, then summed, so a thread waits for two memory latencies per
+// eight cameras instead of two per camera.
+constexpr int kAvgCams = 8;
+
 __global__ void __launch_bounds__(256)
 sca_average_kernel(const float4* __restrict__ out_rb, const int32_t* __restrict__ pos,
                    const int32_t* __restrict__ hits, int B, int Ncam, int Nq, int row4,
@@ -244,19 +305,31 @@ sca_average_kernel(const float4* __restrict__ out_rb, const int32_t* __restrict_
     const int64_t bq = t / row4;
     const int b = (int)(bq / Nq), q = (int)(bq - (int64_t)b * Nq);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int c = 0; c < Ncam; ++c) {
-        const int64_t bc = (int64_t)b * Ncam + c;
-        const int p = __ldg(pos + bc * Nq + q);
-        if (p >= 0) {
-            const float4 x = out_rb[(bc * Nq + p) * row4 + v4];
-            acc.x += x.x;
-            acc.y += x.y;
-            acc.z += x.z;
-            acc.w += x.w;
+    for (int c0 = 0; c0 < Ncam; c0 += kAvgCams) {
+        int p[kAvgCams];
+#pragma unroll
+        for (int k = 0; k < kAvgCams; ++k) {
+            const int c = c0 + k;
+            p[k] = c < Ncam ? __ldg(pos + ((int64_t)b * Ncam + c) * Nq + q) : -1;
+        }
+        float4 x[kAvgCams];
+#pragma unroll
+        for (int k = 0; k < kAvgCams; ++k) {
+            x[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (p[k] >= 0) x[k] = __ldcs(out_rb + (((int64_t)b * Ncam + c0 + k) * Nq + p[k]) * row4 + v4);
+        }
+#pragma unroll
+        for (int k = 0; k < kAvgCams; ++k) {
+            if (p[k] >= 0) {
+                acc.x += x[k].x;
+                acc.y += x[k].y;
+                acc.z += x[k].z;
+                acc.w += x[k].w;
+            }
         }
     }
     const float n = (float)max(1, __ldg(hits + bq));
-    out[bq * row4 + v4] = make_float4(acc.x / n, acc.y / n, acc.z / n, acc.w / n);
+    __stcs(out + bq * row4 + v4, make_float4(acc.x / n, acc.y / n, acc.z / n, acc.w / n));
 }
 
 cudaError_t launch_sca_average(const float* out_rb, const int32_t* pos, const int32_t* hits,
