@@ -16,6 +16,7 @@
 // multiplies a difference of dot products by alpha * W_l (up to ~40 at
 // W_l = 200), and fp32 sums of the 32 products leave errors near 1e-4 there.
 #include <algorithm>
+#include <type_traits>
 
 #include "msda_launch.h"
 
@@ -28,6 +29,7 @@ struct BwdTable {
     float wb[4][kMetaStride];  // bilinear weight without alpha
     float lx[kMetaStride];
     float ly[kMetaStride];
+    float alpha[kMetaStride];
 };
 
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d)
@@ -49,13 +51,18 @@ __device__ __forceinline__ double dw_dly(int g, float lx)
     return (g >> 1) ? a : -a;
 }
 
+// Samples are processed eight at a time.  Each lane forms its partial dot
+// products <grad_out, V_g> for the eight samples (over its own channels), and
+// a butterfly reduce-scatter over the lanes that share a corner leaves every
+// lane with the full dot product of one sample: 7 (fp32) or 3 (bf16) double
+// shuffles per eight samples instead of 3 (or 2) per sample.
 template <typename VT>
 struct BwdLanes;
 
-// fp32 value: lanes 8g..8g+7 hold corner g, channels 4t..4t+3.
+// fp32 value: lanes 8g + t hold corner g, channels 4t..4t+3.  After batch(),
+// lane (g, t) holds D_g of sample j0 + t.
 template <>
 struct BwdLanes<float> {
-    static constexpr int kSamplesPerStep = 1;
     float4 go;
     __device__ __forceinline__ void load_grad(const float* __restrict__ grow, float scale,
                                               int lane)
@@ -63,26 +70,43 @@ struct BwdLanes<float> {
         const float4 v = __ldg(reinterpret_cast<const float4*>(grow) + (lane & 7));
         go = make_float4(v.x / scale, v.y / scale, v.z / scale, v.w / scale);
     }
-    // partial dot for corner g of sample jj, plus the grad_value reduction
-    __device__ __forceinline__ double step(const float* __restrict__ vb, float* __restrict__ gvb,
-                                           const BwdTable& tab, int jj, bool valid, float alpha,
-                                           int lane)
+    __device__ __forceinline__ static int group(int lane) { return lane >> 3; }
+    // sample (within the batch) whose dot product the lane holds after batch()
+    __device__ __forceinline__ static int held(int lane) { return lane & 7; }
+    __device__ __forceinline__ double batch(const float* __restrict__ vb,
+                                            float* __restrict__ gvb, const BwdTable& tab,
+                                            int j0, int cnt, int lane) const
     {
         const int g = lane >> 3, t = lane & 7;
-        const int o = valid ? tab.off[g][jj] : -1;
-        double d = 0.0;
-        if (o >= 0) {
-            const float4 v = __ldg(reinterpret_cast<const float4*>(vb + o + 4 * t));
-            d = (double)go.x * v.x + (double)go.y * v.y + (double)go.z * v.z + (double)go.w * v.w;
-            const float w = alpha * tab.wb[g][jj];
-            if (w != 0.f) red_add_v4(gvb + o + 4 * t, w * go.x, w * go.y, w * go.z, w * go.w);
+        double part[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int j = j0 + k;
+            const int o = j < cnt ? tab.off[g][j] : -1;
+            part[k] = 0.0;
+            if (o >= 0) {
+                const float4 v = __ldg(reinterpret_cast<const float4*>(vb + o + 4 * t));
+                part[k] = (double)go.x * v.x + (double)go.y * v.y + (double)go.z * v.z +
+                          (double)go.w * v.w;
+                const float w = tab.alpha[j] * tab.wb[g][j];
+                if (w != 0.f) red_add_v4(gvb + o + 4 * t, w * go.x, w * go.y, w * go.z, w * go.w);
+            }
         }
-        d += __shfl_xor_sync(0xffffffffu, d, 1);
-        d += __shfl_xor_sync(0xffffffffu, d, 2);
-        d += __shfl_xor_sync(0xffffffffu, d, 4);
-        return d;  // <grad_out, V_g> in every lane of group g
+        double q[4], r[2];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const bool hi = t & 4;
+            q[i] = (hi ? part[i + 4] : part[i]) +
+                   __shfl_xor_sync(0xffffffffu, hi ? part[i] : part[i + 4], 4);
+        }
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const bool hi = t & 2;
+            r[i] = (hi ? q[i + 2] : q[i]) + __shfl_xor_sync(0xffffffffu, hi ? q[i] : q[i + 2], 2);
+        }
+        const bool hi = t & 1;
+        return (hi ? r[1] : r[0]) + __shfl_xor_sync(0xffffffffu, hi ? r[0] : r[1], 1);
     }
-    __device__ __forceinline__ static int group(int lane) { return lane >> 3; }
     __device__ __forceinline__ static double reduce_groups(double v)
     {
         v += __shfl_xor_sync(0xffffffffu, v, 8);
@@ -91,11 +115,11 @@ struct BwdLanes<float> {
     }
 };
 
-// bf16 value: lanes 16s + 4g + t hold corner g of sample 2p + s, channels
-// 8t..8t+7.
+// bf16 value: lanes 16s + 4g + t hold corner g, channels 8t..8t+7, of the
+// samples j0 + 2k + s.  After batch(), lane (s, g, t) holds D_g of sample
+// j0 + 2t + s.
 template <>
 struct BwdLanes<__nv_bfloat16> {
-    static constexpr int kSamplesPerStep = 2;
     float go[8];
     __device__ __forceinline__ void load_grad(const float* __restrict__ grow, float scale,
                                               int lane)
@@ -105,34 +129,48 @@ struct BwdLanes<__nv_bfloat16> {
         go[0] = a.x / scale; go[1] = a.y / scale; go[2] = a.z / scale; go[3] = a.w / scale;
         go[4] = b.x / scale; go[5] = b.y / scale; go[6] = b.z / scale; go[7] = b.w / scale;
     }
-    __device__ __forceinline__ double step(const __nv_bfloat16* __restrict__ vb,
-                                           float* __restrict__ gvb, const BwdTable& tab, int jj,
-                                           bool valid, float alpha, int lane)
+    __device__ __forceinline__ static int group(int lane) { return (lane >> 2) & 3; }
+    __device__ __forceinline__ static int held(int lane) { return 2 * (lane & 3) + (lane >> 4); }
+    __device__ __forceinline__ double batch(const __nv_bfloat16* __restrict__ vb,
+                                            float* __restrict__ gvb, const BwdTable& tab,
+                                            int j0, int cnt, int lane) const
     {
-        const int g = (lane >> 2) & 3, t = lane & 3;
-        const int o = valid ? tab.off[g][jj] : -1;
-        double d = 0.0;
-        if (o >= 0) {
-            const uint4 r = __ldg(reinterpret_cast<const uint4*>(vb + o + 8 * t));
-            float v[8];
-            bf16x2_to_f32(r.x, v[0], v[1]);
-            bf16x2_to_f32(r.y, v[2], v[3]);
-            bf16x2_to_f32(r.z, v[4], v[5]);
-            bf16x2_to_f32(r.w, v[6], v[7]);
+        const int s = lane >> 4, g = (lane >> 2) & 3, t = lane & 3;
+        double part[4];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) d += (double)go[i] * v[i];
-            const float w = alpha * tab.wb[g][jj];
-            if (w != 0.f) {
-                float* dst = gvb + o + 8 * t;
-                red_add_v4(dst, w * go[0], w * go[1], w * go[2], w * go[3]);
-                red_add_v4(dst + 4, w * go[4], w * go[5], w * go[6], w * go[7]);
+        for (int k = 0; k < 4; ++k) {
+            const int j = j0 + 2 * k + s;
+            const int o = j < cnt ? tab.off[g][j] : -1;
+            part[k] = 0.0;
+            if (o >= 0) {
+                const uint4 raw = __ldg(reinterpret_cast<const uint4*>(vb + o + 8 * t));
+                float v[8];
+                bf16x2_to_f32(raw.x, v[0], v[1]);
+                bf16x2_to_f32(raw.y, v[2], v[3]);
+                bf16x2_to_f32(raw.z, v[4], v[5]);
+                bf16x2_to_f32(raw.w, v[6], v[7]);
+                double d = 0.0;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) d += (double)go[i] * v[i];
+                part[k] = d;
+                const float w = tab.alpha[j] * tab.wb[g][j];
+                if (w != 0.f) {
+                    float* dst = gvb + o + 8 * t;
+                    red_add_v4(dst, w * go[0], w * go[1], w * go[2], w * go[3]);
+                    red_add_v4(dst + 4, w * go[4], w * go[5], w * go[6], w * go[7]);
+                }
             }
         }
-        d += __shfl_xor_sync(0xffffffffu, d, 1);
-        d += __shfl_xor_sync(0xffffffffu, d, 2);
-        return d;
+        double q[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const bool hi = t & 2;
+            q[i] = (hi ? part[i + 2] : part[i]) +
+                   __shfl_xor_sync(0xffffffffu, hi ? part[i] : part[i + 2], 2);
+        }
+        const bool hi = t & 1;
+        return (hi ? q[1] : q[0]) + __shfl_xor_sync(0xffffffffu, hi ? q[0] : q[1], 1);
     }
-    __device__ __forceinline__ static int group(int lane) { return (lane >> 2) & 3; }
     __device__ __forceinline__ static double reduce_groups(double v)
     {
         v += __shfl_xor_sync(0xffffffffu, v, 4);
@@ -159,6 +197,7 @@ __device__ __forceinline__ void row_backward(const VT* __restrict__ vb, int H, i
     BwdLanes<VT> lanes;
     lanes.load_grad(grow, scale, lane);
     const int g = BwdLanes<VT>::group(lane);
+    const int held = BwdLanes<VT>::held(lane);
 #pragma unroll
     for (int c = 0; c < NC; ++c) {
         const int j = c * 32 + lane;
@@ -185,47 +224,37 @@ __device__ __forceinline__ void row_backward(const VT* __restrict__ vb, int H, i
         }
         tab.lx[lane] = cr.lx;
         tab.ly[lane] = cr.ly;
+        tab.alpha[lane] = a[c];
         __syncwarp();
-        double res_w = 0.0, res_x = 0.0, res_y = 0.0;
+        float res_w = 0.f, res_x = 0.f, res_y = 0.f;
         const int cnt = min(32, n - c * 32);
-        for (int p = 0; p < cnt; p += BwdLanes<VT>::kSamplesPerStep) {
-            const int jraw = (BwdLanes<VT>::kSamplesPerStep == 2) ? p + (lane >> 4) : p;
-            const bool valid = jraw < cnt;
-            const int jj = valid ? jraw : 0;
-            // alpha of sample jj lives in lane jj
-            const float alpha = __shfl_sync(0xffffffffu, a[c], jj);
-            const double d = lanes.step(vb, gvb, tab, jj, valid, alpha, lane);
-            double cw = valid ? (double)tab.wb[g][jj] * d : 0.0;
-            double cx = valid ? dw_dlx(g, tab.ly[jj]) * d : 0.0;
-            double cy = valid ? dw_dly(g, tab.lx[jj]) * d : 0.0;
+        for (int j0 = 0; j0 < cnt; j0 += 8) {
+            const double d = lanes.batch(vb, gvb, tab, j0, cnt, lane);
+            const int js = j0 + held;  // the sample whose D_g this lane holds
+            const bool valid = js < cnt;
+            double cw = valid ? (double)tab.wb[g][js] * d : 0.0;
+            double cx = valid ? dw_dlx(g, tab.ly[js]) * d : 0.0;
+            double cy = valid ? dw_dly(g, tab.lx[js]) * d : 0.0;
             cw = BwdLanes<VT>::reduce_groups(cw);
             cx = BwdLanes<VT>::reduce_groups(cx);
             cy = BwdLanes<VT>::reduce_groups(cy);
-            if (BwdLanes<VT>::kSamplesPerStep == 1) {
-                if (lane == p) {
-                    res_w = cw;
-                    res_x = cx;
-                    res_y = cy;
-                }
-            } else {
-                // sample p sits in half 0 (lane 0), sample p + 1 in half 1 (lane 16)
-                const int src = (lane & 1) << 4;
-                const double tw = __shfl_sync(0xffffffffu, cw, src);
-                const double tx = __shfl_sync(0xffffffffu, cx, src);
-                const double ty = __shfl_sync(0xffffffffu, cy, src);
-                if ((lane & ~1) == p) {
-                    res_w = tw;
-                    res_x = tx;
-                    res_y = ty;
-                }
+            // the owner of sample j0 + u is lane j0 + u; fetch from a lane holding it
+            const int u = lane & 7;
+            const int src = std::is_same<VT, float>::value ? u : 16 * (u & 1) + (u >> 1);
+            const float tw = __shfl_sync(0xffffffffu, (float)cw, src);
+            const float tx = __shfl_sync(0xffffffffu, (float)cx, src);
+            const float ty = __shfl_sync(0xffffffffu, (float)cy, src);
+            if ((lane & ~7) == j0) {
+                res_w = tw;
+                res_x = tx;
+                res_y = ty;
             }
         }
         if (j < n) {
-            gattn_row[j] = (float)res_w;
-            const double al = a[c];
+            gattn_row[j] = res_w;
+            const float al = a[c];
             *reinterpret_cast<float2*>(gloc_row + 2 * j) =
-                make_float2(cr.valid ? (float)(al * Wl * res_x) : 0.f,
-                            cr.valid ? (float)(al * Hl * res_y) : 0.f);
+                make_float2(cr.valid ? al * Wl * res_x : 0.f, cr.valid ? al * Hl * res_y : 0.f);
         }
         __syncwarp();
     }

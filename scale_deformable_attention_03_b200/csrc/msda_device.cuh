@@ -38,10 +38,17 @@ constexpr int kMaxBatchCameras = 1024;  // B * Ncam limit of the SCA kernels
 #ifndef MSDA_ROWS_PER_TILE
 #define MSDA_ROWS_PER_TILE 8   // consecutive rows per CTA tile (<= 32)
 #endif
-#ifndef MSDA_MIN_CTAS
-#define MSDA_MIN_CTAS 1        // __launch_bounds__ minimum resident CTAs per SM
+// Optional minimum resident CTAs per SM for the forward gathers (register cap).
+#ifdef MSDA_MIN_CTAS
+#define MSDA_GATHER_BOUNDS __launch_bounds__(kThreads, MSDA_MIN_CTAS)
+#else
+#define MSDA_GATHER_BOUNDS __launch_bounds__(kThreads)
+#endif
+#ifndef MSDA_PAIR_UNROLL
+#define MSDA_PAIR_UNROLL 2     // the same for the bf16 head-pair gather
 #endif
 constexpr int kGatherUnroll = MSDA_GATHER_UNROLL;
+constexpr int kPairUnroll = MSDA_PAIR_UNROLL;
 
 // Level geometry, passed by value to every kernel.
 struct Levels {
@@ -464,7 +471,7 @@ __device__ __forceinline__ void row_compute_pair(const __nv_bfloat16* __restrict
         }
         __syncwarp();
         const int quads = (min(32, n - c * 32) + 3) >> 2;
-#pragma unroll kGatherUnroll
+#pragma unroll kPairUnroll
         for (int p = 0; p < quads; ++p) {
             const int4 o = *reinterpret_cast<const int4*>(&tab.off[half][g][4 * p]);
             const float4 w = *reinterpret_cast<const float4*>(&tab.w[half][g][4 * p]);

@@ -14,7 +14,7 @@ namespace msda {
 constexpr int kRowsPerTile = MSDA_ROWS_PER_TILE;
 
 template <typename VT, bool FUSED, int NC, int HP>
-__global__ void __launch_bounds__(kThreads, MSDA_MIN_CTAS)
+__global__ void MSDA_GATHER_BOUNDS
 msda_forward_kernel(const VT* __restrict__ value, const float* __restrict__ lo,
                     const float* __restrict__ wl, const float* __restrict__ ref,
                     float* __restrict__ out, int B, int Nq, int Nv, int H, int L, int P, int R,

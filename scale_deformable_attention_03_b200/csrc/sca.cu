@@ -146,7 +146,7 @@ cudaError_t launch_sca_compact(const uint8_t* mask, int B, int Ncam, int Nq, int
 // Offsets and logits come from the BEV query and are shared by its cameras;
 // the reference points are the camera's own.
 template <typename VT, int NC, int HP>
-__global__ void __launch_bounds__(kThreads, MSDA_MIN_CTAS)
+__global__ void MSDA_GATHER_BOUNDS
 sca_gather_kernel(const VT* __restrict__ value, const float* __restrict__ off,
                   const float* __restrict__ logits, const float* __restrict__ ref_cam,
                   const int32_t* __restrict__ idx, const int32_t* __restrict__ count,
@@ -286,62 +286,93 @@ cudaError_t launch_sca_gather(const Problem& p, const float* ref_cam, const floa
     return launch_gather_t<__nv_bfloat16, 1>(p, ref_cam, off, logits, idx, count, out_rb, s);
 }
 
-// One thread per 16-byte piece of an output row; cameras summed in ascending
-// order, then divided by max(1, hits) (the clamp of the average listing).
-// Cameras are taken eight at a time: all eight positions are loaded, then all
-// eight rows, then summed, so a thread waits for two memory latencies per
-// eight cameras instead of two per camera.
-constexpr int kAvgCams = 8;
+// One warp per (batch, query): lane c loads the query's position in camera c,
+// a ballot gives the seeing cameras, and the warp reads their rows (fully
+// coalesced, four cameras' loads in flight at a time), sums them in ascending
+// camera order and divides by max(1, hits) (the clamp of the average listing).
+constexpr int kAvgWarps = 8;
 
-__global__ void __launch_bounds__(256)
+// PL: float4 per lane (a power of two >= row4 / 32); rows of up to 16 heads.
+// kAvgBatch cameras' rows are loaded together (8 float4 per lane in flight).
+template <int PL>
+__global__ void __launch_bounds__(kAvgWarps * 32)
 sca_average_kernel(const float4* __restrict__ out_rb, const int32_t* __restrict__ pos,
                    const int32_t* __restrict__ hits, int B, int Ncam, int Nq, int row4,
                    float4* __restrict__ out)
 {
-    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t total = (int64_t)B * Nq * row4;
-    if (t >= total) return;
-    const int v4 = (int)(t % row4);
-    const int64_t bq = t / row4;
+    constexpr int kAvgBatch = PL >= 8 ? 1 : 8 / PL;
+    const int lane = threadIdx.x & 31;
+    const int64_t bq = (int64_t)blockIdx.x * kAvgWarps + (threadIdx.x >> 5);
+    if (bq >= (int64_t)B * Nq) return;  // warp-uniform
     const int b = (int)(bq / Nq), q = (int)(bq - (int64_t)b * Nq);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int c0 = 0; c0 < Ncam; c0 += kAvgCams) {
-        int p[kAvgCams];
+    const int p = lane < Ncam ? __ldg(pos + ((int64_t)b * Ncam + lane) * Nq + q) : -1;
+    unsigned seen = __ballot_sync(0xffffffffu, p >= 0);
+    float4 acc[PL];
 #pragma unroll
-        for (int k = 0; k < kAvgCams; ++k) {
-            const int c = c0 + k;
-            p[k] = c < Ncam ? __ldg(pos + ((int64_t)b * Ncam + c) * Nq + q) : -1;
+    for (int k = 0; k < PL; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    while (seen) {
+        int cams[kAvgBatch], rows[kAvgBatch];
+#pragma unroll
+        for (int k = 0; k < kAvgBatch; ++k) {
+            cams[k] = seen ? __ffs(seen) - 1 : -1;  // ascending camera order
+            seen &= seen - 1;
+            rows[k] = __shfl_sync(0xffffffffu, p, cams[k] < 0 ? 0 : cams[k]);
         }
-        float4 x[kAvgCams];
+        float4 x[kAvgBatch][PL];
 #pragma unroll
-        for (int k = 0; k < kAvgCams; ++k) {
-            x[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (p[k] >= 0) x[k] = __ldcs(out_rb + (((int64_t)b * Ncam + c0 + k) * Nq + p[k]) * row4 + v4);
-        }
+        for (int k = 0; k < kAvgBatch; ++k)
 #pragma unroll
-        for (int k = 0; k < kAvgCams; ++k) {
-            if (p[k] >= 0) {
-                acc.x += x[k].x;
-                acc.y += x[k].y;
-                acc.z += x[k].z;
-                acc.w += x[k].w;
+            for (int e = 0; e < PL; ++e) {
+                const int v4 = lane + 32 * e;
+                x[k][e] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (cams[k] >= 0 && v4 < row4)
+                    x[k][e] =
+                        __ldcs(out_rb + (((int64_t)b * Ncam + cams[k]) * Nq + rows[k]) * row4 + v4);
             }
-        }
+#pragma unroll
+        for (int k = 0; k < kAvgBatch; ++k)
+            if (cams[k] >= 0)
+#pragma unroll
+                for (int e = 0; e < PL; ++e) {
+                    acc[e].x += x[k][e].x;
+                    acc[e].y += x[k][e].y;
+                    acc[e].z += x[k][e].z;
+                    acc[e].w += x[k][e].w;
+                }
     }
     const float n = (float)max(1, __ldg(hits + bq));
-    __stcs(out + bq * row4 + v4, make_float4(acc.x / n, acc.y / n, acc.z / n, acc.w / n));
+#pragma unroll
+    for (int e = 0; e < PL; ++e) {
+        const int v4 = lane + 32 * e;
+        if (v4 < row4)
+            __stcs(out + bq * row4 + v4,
+                   make_float4(acc[e].x / n, acc[e].y / n, acc[e].z / n, acc[e].w / n));
+    }
 }
 
 cudaError_t launch_sca_average(const float* out_rb, const int32_t* pos, const int32_t* hits,
                                int B, int Ncam, int Nq, int H, float* out, cudaStream_t s)
 {
     const int row4 = H * kHeadDim / 4;
-    const int64_t total = (int64_t)B * Nq * row4;
-    if (total == 0) return cudaSuccess;
-    const unsigned grid = (unsigned)((total + 255) / 256);
-    sca_average_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const float4*>(out_rb), pos, hits,
-                                            B, Ncam, Nq, row4, reinterpret_cast<float4*>(out));
-    return cudaGetLastError();
+    const int64_t rows = (int64_t)B * Nq;
+    if (rows == 0) return cudaSuccess;
+    const unsigned grid = (unsigned)((rows + kAvgWarps - 1) / kAvgWarps);
+    const float4* in = reinterpret_cast<const float4*>(out_rb);
+    float4* o = reinterpret_cast<float4*>(out);
+    const int pl = (row4 + 31) / 32;
+#define SCA_AVG_CASE(PLV)                                                                        \
+    if (pl <= PLV) {                                                                             \
+        sca_average_kernel<PLV><<<grid, kAvgWarps * 32, 0, s>>>(in, pos, hits, B, Ncam, Nq,      \
+                                                                row4, o);                        \
+        return cudaGetLastError();                                                               \
+    }
+    SCA_AVG_CASE(1)
+    SCA_AVG_CASE(2)
+    SCA_AVG_CASE(4)
+    SCA_AVG_CASE(8)
+    SCA_AVG_CASE(16)
+#undef SCA_AVG_CASE
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace msda
