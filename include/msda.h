@@ -148,6 +148,31 @@ msda_status_t sca_compact(const uint8_t* bev_mask, msda_dims_t d, void* workspac
                           size_t workspace_bytes, int32_t* idx, int32_t* count, int32_t* pos,
                           int32_t* hits, msda_stream_t stream);
 
+/* sca_compact for callers that cannot allocate device memory.  (The pages
+ * have no counterpart: this is a library convenience.)
+ * Some callers cannot call cudaMalloc: the framework around them owns all
+ * device memory and hands out no scratch for this step, or the pipeline
+ * forbids allocation once it runs, because cudaMalloc can block and cudaFree
+ * synchronises the device.  This call takes no workspace: the per-chunk
+ * counts of the two compaction passes live in a fixed array inside the
+ * library, MSDA_NO_ALLOC_COUNT_SLOTS ints (256 KiB), which every GPU that
+ * loads the library holds until the process exits.  It allocates nothing.
+ * Arguments and outputs are those of sca_compact (without the workspace).
+ *   - Limit: B * Ncam * ceil(Nq / 1024) <= MSDA_NO_ALLOC_COUNT_SLOTS, else
+ *     MSDA_ERR_UNSUPPORTED with a message (e.g. B = 1, Ncam = 6 allows
+ *     Nq up to about 11 million).
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and remembers it; make
+ *     that first call before any stream capture.
+ *   - Every call shares the one array per device and leaves its counts
+ *     there; calls whose work overlaps on the GPU (different streams, or
+ *     different host threads, without ordering) race on it.  Calls on one
+ *     stream are safe.  Nothing in it needs to start at zero. */
+#define MSDA_NO_ALLOC_COUNT_SLOTS 65536
+msda_status_t sca_compact_no_alloc(const uint8_t* bev_mask, msda_dims_t d, int32_t* idx,
+                                   int32_t* count, int32_t* pos, int32_t* hits,
+                                   msda_stream_t stream);
+
 /* SCA, stage 2 ([SCA] rebatch listing and MSDA call; [BQ] 10): the fused
  * MSDA of every camera's seeing queries, on the compaction of sca_compact.
  * Row i of camera c of batch item b reads BEV query q = idx[b, c, i]: its

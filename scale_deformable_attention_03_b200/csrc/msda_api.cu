@@ -497,3 +497,11 @@ msda_status_t sca_backward(const void* value, msda_dtype_t vdt, const int64_t* s
 }
 
 }  // extern "C"
+
+// Status helpers for entry points defined in other translation units (they
+// share this file's per-thread error message).
+namespace msda {
+msda_status_t api_fail(msda_status_t code, const char* message) { return fail(code, "%s", message); }
+msda_status_t api_ok() { return ok(); }
+msda_status_t api_cuda(cudaError_t e, const char* where) { return cuda_status(e, where); }
+}  // namespace msda

@@ -74,3 +74,12 @@ cudaError_t launch_sca_zero_tail(const int32_t* count, int B, int Ncam, int Nq, 
                                  float* grad_loc_rb, float* grad_attn_rb, cudaStream_t s);
 
 }  // namespace msda
+
+#include "msda.h"
+
+namespace msda {
+// Set the per-thread error message of msda_last_error() and return the code.
+msda_status_t api_fail(msda_status_t code, const char* message);
+msda_status_t api_ok();
+msda_status_t api_cuda(cudaError_t e, const char* where);
+}  // namespace msda
