@@ -237,17 +237,18 @@ struct Gather;
 template <>
 struct Gather<float> {
     static constexpr int kAcc = 4;
+    // samples base .. base + cnt - 1 of the table (base a multiple of 4)
     __device__ __forceinline__ static void run(const float* __restrict__ vb,
                                                const WarpTable& tab, int cnt, int lane,
-                                               float (&acc)[4])
+                                               float (&acc)[4], int base = 0)
     {
         const int g = lane >> 3, t = lane & 7;
         const float* v = vb + 4 * t;
         const int quads = (cnt + 3) >> 2;
 #pragma unroll kGatherUnroll
         for (int p = 0; p < quads; ++p) {
-            const int4 o = *reinterpret_cast<const int4*>(&tab.off[g][4 * p]);
-            const float4 w = *reinterpret_cast<const float4*>(&tab.w[g][4 * p]);
+            const int4 o = *reinterpret_cast<const int4*>(&tab.off[g][base + 4 * p]);
+            const float4 w = *reinterpret_cast<const float4*>(&tab.w[g][base + 4 * p]);
             float4 x0 = make_float4(0.f, 0.f, 0.f, 0.f), x1 = x0, x2 = x0, x3 = x0;
             if (o.x >= 0) x0 = __ldg(reinterpret_cast<const float4*>(v + o.x));
             if (o.y >= 0) x1 = __ldg(reinterpret_cast<const float4*>(v + o.y));
@@ -291,17 +292,18 @@ struct Gather<__nv_bfloat16> {
         acc[6] += w * a;
         acc[7] += w * b;
     }
+    // samples base .. base + cnt - 1 of the table (base a multiple of 4)
     __device__ __forceinline__ static void run(const __nv_bfloat16* __restrict__ vb,
                                                const WarpTable& tab, int cnt, int lane,
-                                               float (&acc)[8])
+                                               float (&acc)[8], int base = 0)
     {
         const int half = lane >> 4, g = (lane >> 2) & 3, t = lane & 3;
         const __nv_bfloat16* v = vb + 8 * t;
         const int quads = (cnt + 3) >> 2;
 #pragma unroll kGatherUnroll
         for (int p = 0; p < quads; ++p) {
-            const int4 o = *reinterpret_cast<const int4*>(&tab.off[g][4 * p]);
-            const float4 w = *reinterpret_cast<const float4*>(&tab.w[g][4 * p]);
+            const int4 o = *reinterpret_cast<const int4*>(&tab.off[g][base + 4 * p]);
+            const float4 w = *reinterpret_cast<const float4*>(&tab.w[g][base + 4 * p]);
             const int oa = half ? o.y : o.x, ob = half ? o.w : o.z;
             const float wa = half ? w.y : w.x, wb = half ? w.w : w.z;
             uint4 ra = make_uint4(0u, 0u, 0u, 0u), rb = ra;
@@ -498,6 +500,97 @@ __device__ __forceinline__ void row_compute_pair(const __nv_bfloat16* __restrict
         o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
         o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
     }
+}
+
+// Rows with few samples (L*P <= 16): one warp serves G heads of a row at
+// once.  Lane j handles sample k = j mod npad of head h0 + j / npad, where
+// npad is L*P rounded up to a power of two (at least 4, so that every head's
+// samples start on a quad of the table) and G = 32 / npad.  The softmax is a
+// segmented reduction over each head's npad lanes; the gather then walks the
+// heads' table segments one after the other.
+struct GroupLane {
+    int npad_log2;  // log2(npad)
+    int s, k;       // head within the group, sample within the head
+    bool in;        // k < L * P
+    int w, h, start, m;
+};
+
+__device__ __forceinline__ void group_lane(const SmemLevels& lv, int L, int P, int R, int npad_log2,
+                                           int lane, GroupLane& gl)
+{
+    gl.npad_log2 = npad_log2;
+    gl.s = lane >> npad_log2;
+    gl.k = lane & ((1 << npad_log2) - 1);
+    gl.in = gl.k < L * P;
+    const int l = gl.in ? gl.k / P : 0;
+    const int kk = gl.k - l * P;
+    gl.w = lv.w[l];
+    gl.h = lv.h[l];
+    gl.start = lv.start[l];
+    gl.m = gl.in ? kk % R : 0;
+}
+
+__device__ __forceinline__ float segment_max(float v, int npad)
+{
+    for (int o = npad >> 1; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ float segment_sum(float v, int npad)
+{
+    for (int o = npad >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// One row, heads h0 .. h0 + G - 1 (those < H).  lo, wl: head h0 of the row
+// (the other heads follow at +2n, +n per head); ref: the row's reference
+// points; out_row0: head h0's output (+32 per head).  The lane's inputs come
+// preloaded in (a, v, r); `valid` = the lane's sample exists.
+template <typename VT, bool FUSED>
+__device__ __forceinline__ void group_compute(const VT* __restrict__ vb, int H, int h0, float a,
+                                              float2 v, float2 r, bool valid, int n,
+                                              const GroupLane& gl, WarpTable& tab,
+                                              float* __restrict__ out_row0, int lane)
+{
+    const int npad = 1 << gl.npad_log2;
+    if (FUSED) {
+        const float m = segment_max(a, npad);
+        const float e = valid ? expf(a - m) : 0.f;
+        const float z = segment_sum(e, npad);
+        a = valid ? e / z : 0.f;
+    } else if (!valid) {
+        a = 0.f;
+    }
+    Corners cr;
+    if (valid) {
+        float sx = v.x, sy = v.y;
+        if (FUSED) {
+            sx = __fadd_rn(r.x, __fdiv_rn(v.x, (float)gl.w));
+            sy = __fadd_rn(r.y, __fdiv_rn(v.y, (float)gl.h));
+        }
+        locate(sx, sy, gl.h, gl.w, gl.start, H, h0 + gl.s, cr);
+    } else {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            cr.off[g] = -1;
+            cr.w[g] = 0.f;
+        }
+    }
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+        tab.off[g][lane] = cr.off[g];
+        tab.w[g][lane] = cr.w[g] * a;
+    }
+    __syncwarp();
+    const int G = 32 >> gl.npad_log2;
+    for (int s = 0; s < G && h0 + s < H; ++s) {
+        float acc[Gather<VT>::kAcc];
+#pragma unroll
+        for (int i = 0; i < Gather<VT>::kAcc; ++i) acc[i] = 0.f;
+        Gather<VT>::run(vb, tab, n, lane, acc, s << gl.npad_log2);
+        Gather<VT>::store(acc, lane, out_row0 + s * kHeadDim);
+    }
+    __syncwarp();
 }
 
 // Walks the (row, head) items of one warp without divisions: items are

@@ -86,6 +86,103 @@ msda_forward_kernel(const VT* __restrict__ value, const float* __restrict__ lo,
     }
 }
 
+// K1g: rows with L*P <= 16, G = 32 / npad heads per warp item (see
+// group_compute).  Items are (row, head group), head groups fastest.
+template <typename VT, bool FUSED>
+__global__ void MSDA_GATHER_BOUNDS
+msda_forward_group_kernel(const VT* __restrict__ value, const float* __restrict__ lo,
+                          const float* __restrict__ wl, const float* __restrict__ ref,
+                          float* __restrict__ out, int B, int Nq, int Nv, int H, int L, int P,
+                          int R, int npad_log2, Levels levels)
+{
+    __shared__ SmemLevels s_lv;
+    __shared__ __align__(16) WarpTable s_tab[kWarps];
+    stage_levels(s_lv, levels);
+    __syncthreads();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    GroupLane gl;
+    group_lane(s_lv, L, P, R, npad_log2, lane, gl);
+    const int S = L * P;
+    const int G = 32 >> npad_log2;
+    const int HG = (H + G - 1) / G;  // head groups per row
+    const int64_t rows = (int64_t)B * Nq;
+    const int64_t row0 = (int64_t)blockIdx.x * kRowsPerTile;
+    const int b0 = (int)(row0 / Nq);
+    const int q0 = (int)(row0 - (int64_t)b0 * Nq);
+    const int n_items = kRowsPerTile * HG;
+
+    struct Item {
+        bool ok, valid;
+        int b, h0;
+        int64_t bq;
+    };
+    auto resolve = [&](int it, const ItemCursor& cur) {
+        Item x;
+        x.bq = row0 + cur.rr;
+        x.ok = it < n_items && x.bq < rows;
+        x.h0 = cur.h * G;
+        x.valid = gl.in && x.h0 + gl.s < H;
+        int q = q0 + cur.rr;
+        x.b = b0;
+        while (q >= Nq) {
+            q -= Nq;
+            ++x.b;
+        }
+        return x;
+    };
+    struct In {
+        float a;
+        float2 v, r;
+    };
+    auto fetch = [&](const Item& x, In& in) {
+        const int64_t row_h = (x.bq * H + x.h0 + gl.s) * S + gl.k;  // this lane's sample
+        in.a = x.valid ? ld_stream(wl + row_h) : (FUSED ? -INFINITY : 0.f);
+        in.v = x.valid ? ld_stream2(lo + 2 * row_h) : make_float2(0.f, 0.f);
+        in.r = (FUSED && x.valid) ? __ldg(reinterpret_cast<const float2*>(ref + x.bq * R * 2) + gl.m)
+                                  : make_float2(0.f, 0.f);
+    };
+
+    ItemCursor cur(warp, HG);
+    int it = warp;
+    Item x0 = resolve(it, cur);
+    In in0, in1;
+    if (x0.ok) fetch(x0, in0);
+    while (x0.ok) {
+        ItemCursor nx = cur;
+        nx.next();
+        const Item x1 = resolve(it + kWarps, nx);
+        if (x1.ok) fetch(x1, in1);
+        const VT* vb = value + (int64_t)x0.b * Nv * H * kHeadDim;
+        group_compute<VT, FUSED>(vb, H, x0.h0, in0.a, in0.v, in0.r, x0.valid, S, gl, s_tab[warp],
+                                 out + (x0.bq * H + x0.h0) * kHeadDim, lane);
+        x0 = x1;
+        in0 = in1;
+        cur = nx;
+        it += kWarps;
+    }
+}
+
+template <typename VT, bool FUSED>
+static cudaError_t launch_group(const Problem& p, const float* lo, const float* wl,
+                                const float* ref, float* out, cudaStream_t s)
+{
+    const int64_t rows = (int64_t)p.B * p.Nq;
+    if (rows == 0) return cudaSuccess;
+    const int S = p.L * p.P;
+    int npad_log2 = 2;
+    while ((1 << npad_log2) < S) ++npad_log2;
+    const unsigned grid = (unsigned)((rows + kRowsPerTile - 1) / kRowsPerTile);
+    msda_forward_group_kernel<VT, FUSED><<<grid, kThreads, 0, s>>>(
+        static_cast<const VT*>(p.value), lo, wl, ref, out, p.B, p.Nq, p.Nv, p.H, p.L, p.P, p.R,
+        npad_log2, p.lv);
+    return cudaGetLastError();
+}
+
+// Warp layout choice: several heads per warp when a row has at most 16
+// samples per head and there is more than one head.
+static bool use_group(const Problem& p) { return p.L * p.P <= 16 && p.H > 1; }
+
 template <typename VT, bool FUSED, int HP>
 static cudaError_t launch_fwd(const Problem& p, const float* lo, const float* wl,
                               const float* ref, float* out, cudaStream_t s)
@@ -114,6 +211,9 @@ static cudaError_t launch_fwd(const Problem& p, const float* lo, const float* wl
 cudaError_t launch_msda_forward(const Problem& p, const float* loc, const float* attn,
                                 float* out, cudaStream_t s)
 {
+    if (use_group(p))
+        return p.bf16 ? launch_group<__nv_bfloat16, false>(p, loc, attn, nullptr, out, s)
+                      : launch_group<float, false>(p, loc, attn, nullptr, out, s);
     if (!p.bf16) return launch_fwd<float, false, 1>(p, loc, attn, nullptr, out, s);
     if (p.H % 2 == 0) return launch_fwd<__nv_bfloat16, false, 2>(p, loc, attn, nullptr, out, s);
     return launch_fwd<__nv_bfloat16, false, 1>(p, loc, attn, nullptr, out, s);
@@ -122,6 +222,9 @@ cudaError_t launch_msda_forward(const Problem& p, const float* loc, const float*
 cudaError_t launch_msda_forward_fused(const Problem& p, const float* ref, const float* off,
                                       const float* logits, float* out, cudaStream_t s)
 {
+    if (use_group(p))
+        return p.bf16 ? launch_group<__nv_bfloat16, true>(p, off, logits, ref, out, s)
+                      : launch_group<float, true>(p, off, logits, ref, out, s);
     if (!p.bf16) return launch_fwd<float, true, 1>(p, off, logits, ref, out, s);
     if (p.H % 2 == 0) return launch_fwd<__nv_bfloat16, true, 2>(p, off, logits, ref, out, s);
     return launch_fwd<__nv_bfloat16, true, 1>(p, off, logits, ref, out, s);
