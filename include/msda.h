@@ -125,6 +125,27 @@ msda_status_t msda_backward(const void* value, msda_dtype_t vdt,
                             float* grad_sampling_locations, float* grad_attention_weights,
                             msda_stream_t stream);
 
+/* Dense projection on the tensor cores ([BQ] 3 value projection W_v, 4.1
+ * offset head W_Delta, 4.2 weight head W_alpha, 11 output projection W_o, 13
+ * residual):  y = x w^T (+ bias) (+ residual).
+ *   x        [M, K] bf16, row-major
+ *   w        [N, K] bf16 (the nn.Linear weight layout, out x in)
+ *   bias     [N] fp32 or NULL
+ *   residual [M, N] fp32 or NULL, added after the bias (the SCA module's
+ *            q_hat = q + output_proj(g) with dropout off, [BQ] 13)
+ *   y        [M, N] fp32 (y_dtype MSDA_F32) or bf16 (MSDA_BF16), written
+ * Products are exact and accumulate in fp32 (tensor memory).  Limits: N a
+ * positive multiple of 256, K one of 64, 128, 192, 256, M >= 0; every pointer
+ * 16-byte aligned. */
+msda_status_t msda_linear(const void* x, const void* w, const float* bias,
+                          const float* residual, int32_t M, int32_t N, int32_t K,
+                          msda_dtype_t y_dtype, void* y, msda_stream_t stream);
+
+/* Number of msda_linear tiles that gave up waiting on their load or MMA
+ * pipeline (each wait is bounded, about a second); 0 in normal operation.
+ * Reads a device word, so it synchronises with the device. */
+uint32_t msda_linear_timeouts(void);
+
 /* Bytes of device workspace sca_forward / sca_backward need for these
  * sizes: the compaction lists and, for the forward, the rebatched rows
  * (B * Ncam * Nq * H * 32 floats, of which only the seeing rows are used). */

@@ -41,9 +41,10 @@ def lib():
                                          _U8, _D, _D, _i, _D, _D]
         L.oracle_sca_backward.argtypes = [_D, _i, _i, _i, _i, _i, _i, _I64, _I64, _i, _i, _i, _D,
                                           _U8, _D, _D, _D, _i, _D, _D, _D]
+        L.oracle_linear.argtypes = [_D, _D, _D, _D, _i, _i, _i, _D]
         for f in ("oracle_softmax", "oracle_msda_forward", "oracle_msda_forward_fused",
                   "oracle_fused_locations", "oracle_msda_backward", "oracle_sca_compact",
-                  "oracle_sca_forward", "oracle_sca_backward"):
+                  "oracle_sca_forward", "oracle_sca_backward", "oracle_linear"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -202,3 +203,17 @@ def sca_backward(value, spatial_shapes, level_start_index, reference_points_cam,
                                    _p(gv, _D), _p(gl, _D), _p(gw, _D))
     _check(rc, "sca_backward")
     return gv, gl, gw
+
+
+def linear(x, w, bias=None, residual=None):
+    """y = x w^T (+ bias) (+ residual); x [M, K], w [N, K] -> y [M, N]."""
+    xd, wd = _d(x), _d(w)
+    M, K = xd.shape
+    N = wd.shape[0]
+    b = _d(bias) if bias is not None else None
+    r = _d(residual) if residual is not None else None
+    y = np.empty((M, N))
+    rc = lib().oracle_linear(_p(xd, _D), _p(wd, _D), _p(b, _D) if b is not None else None,
+                             _p(r, _D) if r is not None else None, M, N, K, _p(y, _D))
+    _check(rc, "linear")
+    return y

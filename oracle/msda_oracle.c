@@ -484,3 +484,22 @@ int oracle_sca_backward(const double* value, int B, int Ncam, int Nv, int H, int
     scratch_free(&sc);
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Dense projection ([BQ] 3, 4.1, 4.2, 11, 13)                              */
+/* ------------------------------------------------------------------------ */
+
+int oracle_linear(const double* x, const double* w, const double* bias, const double* residual,
+                  int M, int N, int K, double* y)
+{
+    if (!x || !w || !y || M < 0 || N < 1 || K < 1) return -1;
+    for (int m = 0; m < M; ++m)
+        for (int n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int k = 0; k < K; ++k) acc += x[(int64_t)m * K + k] * w[(int64_t)n * K + k];
+            if (bias) acc += bias[n];
+            if (residual) acc += residual[(int64_t)m * N + n];
+            y[(int64_t)m * N + n] = acc;
+        }
+    return 0;
+}

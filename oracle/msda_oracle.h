@@ -110,6 +110,14 @@ int oracle_sca_backward(const double* value, int B, int Ncam, int Nv, int H, int
                         const double* logits, const double* grad_out, int coord_f32,
                         double* grad_value, double* grad_loc_rb, double* grad_attn_rb);
 
+/* Dense projection ([BQ] 3 value projection, 4.1 offset head, 4.2 weight
+ * head, 11 output projection, 13 residual):
+ *   y[m, n] = sum_k x[m, k] w[n, k] + bias[n] + residual[m, n]
+ * x [M, K]; w [N, K] (nn.Linear layout); bias [N] or NULL; residual [M, N]
+ * or NULL; y [M, N]. */
+int oracle_linear(const double* x, const double* w, const double* bias, const double* residual,
+                  int M, int N, int K, double* y);
+
 #ifdef __cplusplus
 }
 #endif

@@ -10,7 +10,8 @@ status.  There is no fallback: without the built library every call raises.
 Functions (same names as the C ABI): ``msda_forward``, ``msda_forward_fused``,
 ``msda_backward``, ``sca_compact``, ``sca_rebatched_forward``,
 ``sca_camera_average``, ``sca_forward``, ``sca_rebatched_backward``,
-``sca_backward``, ``msda_workspace_size``, ``sca_compact_workspace_size``.
+``sca_backward``, ``msda_linear``, ``msda_workspace_size``,
+``sca_compact_workspace_size``.
 """
 import ctypes
 import os
@@ -67,6 +68,10 @@ def lib():
                   "sca_forward", "sca_backward", "sca_rebatched_forward", "sca_camera_average",
                   "sca_rebatched_backward"):
             getattr(L, f).restype = ctypes.c_int
+        L.msda_linear.argtypes = [_vp, _vp, _vp, _vp, ctypes.c_int32, ctypes.c_int32,
+                                  ctypes.c_int32, st, _vp, _vp]
+        L.msda_linear.restype = ctypes.c_int
+        L.msda_linear_timeouts.restype = ctypes.c_uint32
         L.msda_status_string.argtypes = [ctypes.c_int]
         L.msda_status_string.restype = ctypes.c_char_p
         L.msda_last_error.restype = ctypes.c_char_p
@@ -357,3 +362,22 @@ def sca_rebatched_backward(value, spatial_shapes, level_start_index, reference_p
                                         _ptr(grad_attention_weights_rb), _stream(stream)),
            "sca_rebatched_backward")
     return grad_value, grad_sampling_locations_rb, grad_attention_weights_rb
+
+
+def msda_linear(x, w, bias=None, residual=None, out=None, out_dtype=None, stream=None):
+    """y = x w^T (+ bias) (+ residual) on the tensor cores.  x [M, K] bf16,
+    w [N, K] bf16, bias [N] fp32, residual [M, N] fp32 -> y [M, N] (fp32, or
+    bf16 when out_dtype / out is bfloat16)."""
+    torch = _torch()
+    _contig(x, w, bias, residual, out)
+    if x.dtype != torch.bfloat16 or w.dtype != torch.bfloat16:
+        raise MsdaError("msda_linear takes bfloat16 x and w")
+    M, K = x.shape
+    N = w.shape[0]
+    if out is None:
+        out = torch.empty((M, N), device=x.device, dtype=out_dtype or torch.float32)
+    ydt = MSDA_BF16 if out.dtype == torch.bfloat16 else MSDA_F32
+    _check(lib().msda_linear(_ptr(x), _ptr(w), _ptr(bias), _ptr(residual), M, N, K, ydt,
+                             _ptr(out), _stream(stream)),
+           "msda_linear")
+    return out

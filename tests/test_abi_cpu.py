@@ -35,6 +35,7 @@ def test_header_declares_the_boundary():
     for n in ("msda_forward", "msda_forward_fused", "msda_backward", "msda_workspace_size",
               "sca_compact_workspace_size", "sca_compact", "sca_forward", "sca_backward",
               "sca_rebatched_forward", "sca_camera_average", "sca_rebatched_backward",
+              "sca_compact_no_alloc", "msda_linear", "msda_linear_timeouts",
               "msda_status_string", "msda_last_error", "msda_version"):
         assert n in names
 
@@ -167,3 +168,14 @@ def test_binding_raises_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(msda, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(msda.MsdaError):
         msda.lib()
+
+
+def test_linear_rejects_unsupported_shapes(L):
+    f = L.msda_linear
+    assert f(FAKE, FAKE, None, None, 128, 100, 256, 0, FAKE, None) == UNSUPPORTED   # N
+    assert f(FAKE, FAKE, None, None, 128, 256, 320, 0, FAKE, None) == UNSUPPORTED   # K
+    assert f(FAKE, FAKE, None, None, 128, 256, 96, 0, FAKE, None) == UNSUPPORTED    # K
+    assert f(FAKE + 8, FAKE, None, None, 128, 256, 256, 0, FAKE, None) == INVALID   # alignment
+    assert f(FAKE, FAKE, FAKE + 4, None, 128, 256, 256, 0, FAKE, None) == INVALID   # bias
+    assert f(FAKE, FAKE, None, None, 128, 256, 256, 9, FAKE, None) == INVALID       # dtype
+    assert f(0, 0, None, None, 0, 256, 256, 0, 0, None) == OK                        # empty

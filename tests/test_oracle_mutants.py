@@ -60,6 +60,9 @@ MUTANTS = [
     ("grad_value missing the weight", "double w = alpha * corner_weight(&c, q);",
      "double w = corner_weight(&c, q);", 0),
     ("grad_attn missing the bilinear weight", "gw += corner_weight(&c, q) * dot[q];", "gw += dot[q];", 0),
+    ("projection weight transposed", "acc += x[(int64_t)m * K + k] * w[(int64_t)n * K + k];",
+     "acc += x[(int64_t)m * K + k] * w[(int64_t)k * N + n];", 0),
+    ("projection bias dropped", "if (bias) acc += bias[n];", "", 0),
     ("SCA backward not divided by the count",
      "sc.row[d] = grad_out[bq * HD + d] / (double)n;", "sc.row[d] = grad_out[bq * HD + d];", 0),
 ]
@@ -85,6 +88,8 @@ PIN_CALLS = [
     ("msda_fd_border", lambda: pins.test_msda_backward_with_partly_outside_samples()),
     ("linearity", lambda: pins.test_msda_backward_linearity()),
     ("sca_fd", lambda: pins.test_sca_backward_matches_finite_differences()),
+    ("linear_numpy", lambda: pins.test_linear_matches_numpy_matmul()),
+    ("linear_s15", lambda: pins.test_section15_output_projection_and_residual()),
 ]
 
 
@@ -110,7 +115,7 @@ def test_pins_catch_planted_mistake(tmp_path, monkeypatch, name, old, new, occ):
     mutant = ctypes.CDLL(str(so))
     for fname in ("oracle_softmax", "oracle_msda_forward", "oracle_msda_forward_fused",
                   "oracle_fused_locations", "oracle_msda_backward", "oracle_sca_compact",
-                  "oracle_sca_forward", "oracle_sca_backward"):
+                  "oracle_sca_forward", "oracle_sca_backward", "oracle_linear"):
         fn = getattr(mutant, fname)
         fn.argtypes = getattr(good, fname).argtypes
         fn.restype = ctypes.c_int

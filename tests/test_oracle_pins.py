@@ -573,3 +573,29 @@ def test_empty_problems():
     with pytest.raises(ValueError):
         oracle.msda_forward(value, [(3, 3)], [0], np.zeros((1, 1, 1, 1, 1, 2)),
                             np.zeros((1, 1, 1, 1, 1)))  # level larger than the value map
+
+
+# --------------------------------------------------------------------------
+# dense projections (sections 3, 4.1, 4.2, 11, 13)
+# --------------------------------------------------------------------------
+
+def test_linear_matches_numpy_matmul():
+    rng = _rng(40)
+    x = rng.standard_normal((37, 24))
+    w = rng.standard_normal((11, 24))
+    b = rng.standard_normal(11)
+    r = rng.standard_normal((37, 11))
+    np.testing.assert_allclose(oracle.linear(x, w, b, r), x @ w.T + b + r, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(oracle.linear(x, w), x @ w.T, rtol=1e-12, atol=1e-12)
+
+
+def test_linear_identity_weight():
+    x = _rng(41).standard_normal((5, 8))
+    np.testing.assert_array_equal(oracle.linear(x, np.eye(8)), x)
+
+
+def test_section15_output_projection_and_residual():
+    """Identity W_o, dropout off: q_hat = q + W_o g = [9, 3.6, 9, 3]."""
+    g = json.load(open(os.path.join(GOLDEN, "bq_s15_two_head_example.json")))
+    q_hat = oracle.linear(np.asarray(g["g"])[None], np.eye(4), None, np.asarray(g["q"])[None])
+    np.testing.assert_allclose(q_hat[0], g["q_hat"], rtol=1e-15)
