@@ -42,9 +42,17 @@ def lib():
         L.oracle_sca_backward.argtypes = [_D, _i, _i, _i, _i, _i, _i, _I64, _I64, _i, _i, _i, _D,
                                           _U8, _D, _D, _D, _i, _D, _D, _D]
         L.oracle_linear.argtypes = [_D, _D, _D, _D, _i, _i, _i, _D]
+        L.oracle_sca_backward_inputs.argtypes = [_i, _i, _i, _i, _i, _I64, _i, _i, _U8, _D, _D,
+                                                 _D, _D, _D, _D]
+        L.oracle_tsa_reference_points.argtypes = [_i, _i, _i, _i, ctypes.c_double,
+                                                  ctypes.c_double, _D, _D]
+        L.oracle_tsa_forward.argtypes = [_D, _i, _i, _i, _i, _i, _i, _I64, _I64, _i, _i, _i, _D,
+                                         _D, _D, _i, _D]
         for f in ("oracle_softmax", "oracle_msda_forward", "oracle_msda_forward_fused",
                   "oracle_fused_locations", "oracle_msda_backward", "oracle_sca_compact",
-                  "oracle_sca_forward", "oracle_sca_backward", "oracle_linear"):
+                  "oracle_sca_forward", "oracle_sca_backward", "oracle_linear",
+                  "oracle_sca_backward_inputs", "oracle_tsa_reference_points",
+                  "oracle_tsa_forward"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -217,3 +225,88 @@ def linear(x, w, bias=None, residual=None):
                              _p(r, _D) if r is not None else None, M, N, K, _p(y, _D))
     _check(rc, "linear")
     return y
+
+
+def round_bf16(a):
+    """Round to the nearest bfloat16 (ties to even), returned as float64: the
+    storage step of the module's bf16 operands."""
+    f = np.ascontiguousarray(a, dtype=np.float32)
+    u = f.view(np.uint32)
+    u = ((u + ((u >> 16) & 1) + np.uint32(0x7FFF)) >> 16) << 16
+    return u.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def sca_module_forward(query, query_pos, features, w_value, b_value, w_offsets, b_offsets,
+                       w_weights, b_weights, w_output, b_output, reference_points_cam, bev_mask,
+                       spatial_shapes, level_start_index, num_levels, num_points,
+                       value_bf16=False):
+    """The SCA module forward ([BQ] 3, 4, 10-13), composed of the oracle's
+    projection and SCA: q~ = bf16(q + pos); V = F~ W_v^T + b_v; Delta, a from
+    q~; g = SCA; q_hat = q + bf16(g) W_o^T + b_o.  features [B, Ncam, Nv, C]."""
+    q = _d(query)
+    B, Nq, C = q.shape
+    _, Ncam, Nv, _ = features.shape
+    H, L, P = C // 32, num_levels, num_points
+    qt = round_bf16(q + (0.0 if query_pos is None else _d(query_pos))).reshape(B * Nq, C)
+    V = linear(_d(features).reshape(-1, C), w_value, b_value)
+    if value_bf16:
+        V = round_bf16(V)
+    off = linear(qt, w_offsets, b_offsets).reshape(B, Nq, H, L, P, 2)
+    lg = linear(qt, w_weights, b_weights).reshape(B, Nq, H, L, P)
+    g = sca_forward(V.reshape(B, Ncam, Nv, H, 32), spatial_shapes, level_start_index,
+                    reference_points_cam, bev_mask, off, lg)
+    y = linear(round_bf16(g).reshape(B * Nq, C), w_output, b_output, q.reshape(B * Nq, C))
+    return y.reshape(B, Nq, C)
+
+
+def sca_backward_inputs(spatial_shapes, bev_mask, attention_logits, grad_loc_rb, grad_attn_rb):
+    """-> (grad_sampling_offsets [B, Nq, H, L, P, 2], grad_attention_logits
+    [B, Nq, H, L, P], grad_reference_points_cam [Ncam, B, Nq, R, 2])."""
+    shapes, _ = _levels(spatial_shapes, None)
+    m = np.ascontiguousarray(bev_mask).astype(np.uint8)
+    Ncam, B, Nq, R = m.shape
+    lg, gl, gw = _d(attention_logits), _d(grad_loc_rb), _d(grad_attn_rb)
+    _, _, H, L, P = lg.shape
+    g_off = np.empty((B, Nq, H, L, P, 2))
+    g_lg = np.empty((B, Nq, H, L, P))
+    g_ref = np.empty((Ncam, B, Nq, R, 2))
+    rc = lib().oracle_sca_backward_inputs(B, Ncam, Nq, H, L, _p(shapes, _I64), P, R, _p(m, _U8),
+                                          _p(lg, _D), _p(gl, _D), _p(gw, _D), _p(g_off, _D),
+                                          _p(g_lg, _D), _p(g_ref, _D))
+    _check(rc, "sca_backward_inputs")
+    return g_off, g_lg, g_ref
+
+
+def tsa_reference_points(bev_h, bev_w, ego_motion, grid_length=(0.512, 0.512)):
+    """ego_motion [B, T, 3] = (dx m, dy m, angle degrees) of each queue;
+    grid_length = (gy, gx) metres per cell -> ref [B, T, bev_h * bev_w, 2]."""
+    e = _d(ego_motion)
+    B, T, _ = e.shape
+    gy, gx = grid_length
+    ref = np.empty((B, T, bev_h * bev_w, 2))
+    rc = lib().oracle_tsa_reference_points(B, T, bev_h, bev_w, float(gx), float(gy), _p(e, _D),
+                                           _p(ref, _D))
+    _check(rc, "tsa_reference_points")
+    return ref
+
+
+def tsa_forward(value, spatial_shapes, level_start_index, reference_points, sampling_offsets,
+                attention_logits, num_queues, coord_f32=True):
+    """value [B*T, Nv, H, Dh] (row b*T + t); ref [B*T, Nq, R, 2];
+    offsets [B*T, Nq, H, L, P, 2]; logits [B*T, Nq, H, L, P] -> out [B, Nq, H*Dh],
+    the mean over the T queues."""
+    v = _d(value)
+    shapes, starts = _levels(spatial_shapes, level_start_index)
+    ref, off, lg = _d(reference_points), _d(sampling_offsets), _d(attention_logits)
+    BT, Nv, H, Dh = v.shape
+    T = int(num_queues)
+    if T < 1 or BT % T:
+        raise ValueError("tsa_forward: batch is not a multiple of num_queues")
+    _, Nq, _, L, P, _ = off.shape
+    R = ref.shape[2]
+    out = np.empty((BT // T, Nq, H * Dh))
+    rc = lib().oracle_tsa_forward(_p(v, _D), BT // T, T, Nv, H, Dh, L, _p(shapes, _I64),
+                                  _p(starts, _I64), Nq, P, R, _p(ref, _D), _p(off, _D),
+                                  _p(lg, _D), int(coord_f32), _p(out, _D))
+    _check(rc, "tsa_forward")
+    return out

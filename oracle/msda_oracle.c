@@ -503,3 +503,124 @@ int oracle_linear(const double* x, const double* w, const double* bias, const do
         }
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Gradients of the SCA inputs ([BQ] 4.2, 5, 10)                            */
+/* ------------------------------------------------------------------------ */
+
+int oracle_sca_backward_inputs(int B, int Ncam, int Nq, int H, int L, const int64_t* shapes,
+                               int P, int R, const uint8_t* bev_mask, const double* logits,
+                               const double* grad_loc_rb, const double* grad_attn_rb,
+                               double* grad_off, double* grad_logits, double* grad_ref_cam)
+{
+    if (B < 0 || Ncam < 1 || Nq < 0 || H < 1 || L < 1 || P < 1 || R < 1 || P % R || !shapes ||
+        !bev_mask || !logits || !grad_loc_rb || !grad_attn_rb || !grad_off || !grad_logits ||
+        !grad_ref_cam)
+        return -1;
+    const int64_t S = (int64_t)H * L * P;
+    int32_t* idx = (int32_t*)malloc(sizeof(int32_t) * (size_t)((int64_t)B * Ncam * Nq + 1));
+    int32_t* count = (int32_t*)malloc(sizeof(int32_t) * (size_t)((int64_t)B * Ncam + 1));
+    int32_t* pos = (int32_t*)malloc(sizeof(int32_t) * (size_t)((int64_t)B * Ncam * Nq + 1));
+    int32_t* hits = (int32_t*)malloc(sizeof(int32_t) * (size_t)((int64_t)B * Nq + 1));
+    double* G = (double*)malloc(sizeof(double) * (size_t)((int64_t)B * Nq * S + 1));
+    double* alpha = (double*)malloc(sizeof(double) * (size_t)(S + 1));
+    if (!idx || !count || !pos || !hits || !G || !alpha) {
+        free(idx); free(count); free(pos); free(hits); free(G); free(alpha);
+        return -1;
+    }
+    oracle_sca_compact(bev_mask, Ncam, B, Nq, R, idx, count, pos, hits);
+    memset(grad_off, 0, sizeof(double) * (size_t)((int64_t)B * Nq * S * 2));
+    memset(grad_ref_cam, 0, sizeof(double) * (size_t)((int64_t)Ncam * B * Nq * R * 2));
+    memset(G, 0, sizeof(double) * (size_t)((int64_t)B * Nq * S));
+    for (int b = 0; b < B; ++b)
+        for (int c = 0; c < Ncam; ++c) {
+            const int64_t bc = (int64_t)b * Ncam + c;
+            for (int i = 0; i < count[bc]; ++i) {
+                const int q = idx[bc * Nq + i];
+                const int64_t bq = (int64_t)b * Nq + q;
+                const double* gl = grad_loc_rb + (bc * Nq + i) * S * 2;
+                const double* ga = grad_attn_rb + (bc * Nq + i) * S;
+                double* gr = grad_ref_cam + (((int64_t)c * B + b) * Nq + q) * R * 2;
+                for (int h = 0; h < H; ++h)
+                    for (int l = 0; l < L; ++l) {
+                        const double Hl = (double)shapes[2 * l], Wl = (double)shapes[2 * l + 1];
+                        for (int k = 0; k < P; ++k) {
+                            const int64_t s = ((int64_t)h * L + l) * P + k;
+                            grad_off[(bq * S + s) * 2 + 0] += gl[2 * s + 0] / Wl;
+                            grad_off[(bq * S + s) * 2 + 1] += gl[2 * s + 1] / Hl;
+                            G[bq * S + s] += ga[s];
+                            gr[2 * (k % R) + 0] += gl[2 * s + 0];
+                            gr[2 * (k % R) + 1] += gl[2 * s + 1];
+                        }
+                    }
+            }
+        }
+    const int n = L * P;
+    for (int64_t bq = 0; bq < (int64_t)B * Nq; ++bq)
+        for (int h = 0; h < H; ++h) {
+            const int64_t base = bq * S + (int64_t)h * n;
+            oracle_softmax(logits + base, 1, n, alpha);
+            double dot = 0.0;
+            for (int j = 0; j < n; ++j) dot += alpha[j] * G[base + j];
+            for (int j = 0; j < n; ++j) grad_logits[base + j] = alpha[j] * (G[base + j] - dot);
+        }
+    free(idx); free(count); free(pos); free(hits); free(G); free(alpha);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Temporal Self-Attention ([TS] section 二.2 and the BEV encoder listing)  */
+/* ------------------------------------------------------------------------ */
+
+int oracle_tsa_reference_points(int B, int T, int bev_h, int bev_w, double gx, double gy,
+                                const double* ego, double* ref)
+{
+    if (B < 0 || T < 1 || bev_h < 1 || bev_w < 1 || !(gx > 0.0) || !(gy > 0.0) || !ego || !ref)
+        return -1;
+    const double pi = 3.14159265358979323846;
+    const int64_t Nq = (int64_t)bev_h * bev_w;
+    for (int b = 0; b < B; ++b)
+        for (int t = 0; t < T; ++t) {
+            const double* e = ego + ((int64_t)b * T + t) * 3;
+            const double dx = e[0], dy = e[1], theta = e[2] * pi / 180.0;
+            const double cs = cos(theta), sn = sin(theta);
+            for (int i = 0; i < bev_h; ++i)
+                for (int j = 0; j < bev_w; ++j) {
+                    /* cell centre in metres about the BEV centre (x along the width) */
+                    const double px = ((double)j + 0.5 - 0.5 * bev_w) * gx;
+                    const double py = ((double)i + 0.5 - 0.5 * bev_h) * gy;
+                    /* the same point in queue t's frame: rotation, then translation */
+                    const double qx = cs * px - sn * py + dx;
+                    const double qy = sn * px + cs * py + dy;
+                    double* r = ref + (((int64_t)b * T + t) * Nq + (int64_t)i * bev_w + j) * 2;
+                    r[0] = qx / (bev_w * gx) + 0.5;
+                    r[1] = qy / (bev_h * gy) + 0.5;
+                }
+        }
+    return 0;
+}
+
+int oracle_tsa_forward(const double* value, int B, int T, int Nv, int H, int Dh,
+                       int L, const int64_t* shapes, const int64_t* starts,
+                       int Nq, int P, int R, const double* ref,
+                       const double* off, const double* logits,
+                       int coord_f32, double* out)
+{
+    if (T < 1 || B < 0 || out == NULL) return -1;
+    const int64_t HD = (int64_t)H * Dh;
+    double* per_queue = (double*)malloc(sizeof(double) * (size_t)((int64_t)B * T * Nq * HD + 1));
+    if (!per_queue) return -1;
+    int rc = oracle_msda_forward_fused(value, B * T, Nv, H, Dh, L, shapes, starts, Nq, P, R, ref,
+                                       off, logits, coord_f32, per_queue);
+    if (rc == 0)
+        for (int b = 0; b < B; ++b)
+            for (int q = 0; q < Nq; ++q)
+                for (int64_t d = 0; d < HD; ++d) {
+                    double sum = 0.0;
+                    for (int t = 0; t < T; ++t)
+                        sum += per_queue[(((int64_t)b * T + t) * Nq + q) * HD + d];
+                    out[((int64_t)b * Nq + q) * HD + d] = sum / T;
+                }
+    free(per_queue);
+    return rc;
+}

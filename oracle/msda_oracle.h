@@ -15,6 +15,14 @@
  *   [SCA] "Spatial Cross-Attention" walkthrough, Tencent Cloud developer
  *         article 2321140: the bev_mask query rebatch listing and the
  *         scatter-add / clamp(count, 1) average listing.
+ *   [TS]  "【论文阅读】BEVFormer论文解析及Temporal Self-Attention、Spatial
+ *         Cross-Attention注意力机制详解及代码示例" (wsisp.com): section 二.2
+ *         (TSA between the previous and the current BEV) and the BEV encoder
+ *         listing (ego motion delta_x, delta_y, ego_angle in degrees from the
+ *         CAN bus; grid_length 0.512 m per BEV cell).  The listing stops
+ *         before it applies the motion and the section gives TSA only as
+ *         generic attention; the two TSA entry points below state the
+ *         reading they take.
  *
  * Conventions shared by every entry point below:
  *   - every array is host memory, contiguous, row-major in the shape given;
@@ -110,6 +118,20 @@ int oracle_sca_backward(const double* value, int B, int Ncam, int Nv, int H, int
                         const double* logits, const double* grad_out, int coord_f32,
                         double* grad_value, double* grad_loc_rb, double* grad_attn_rb);
 
+/* Gradients of the SCA inputs from the rebatched gradients of
+ * oracle_sca_backward.  Offsets and logits belong to the BEV query and are
+ * shared by every camera ([BQ] 10), so their gradients sum over the cameras
+ * that see the query; s = rho_{k mod R} + (dx / W_l, dy / H_l) ([BQ] 5) gives
+ * d/d dx = d/d s_x / W_l and d/d rho_m = sum over the points k with
+ * k mod R = m; alpha = softmax(a) ([BQ] 4.2) gives
+ * d/d a_j = alpha_j (G_j - sum_i alpha_i G_i).
+ *   grad_off [B, Nq, H, L, P, 2], grad_logits [B, Nq, H, L, P],
+ *   grad_ref_cam [Ncam, B, Nq, R, 2] (zero for cameras that do not see q). */
+int oracle_sca_backward_inputs(int B, int Ncam, int Nq, int H, int L, const int64_t* shapes,
+                               int P, int R, const uint8_t* bev_mask, const double* logits,
+                               const double* grad_loc_rb, const double* grad_attn_rb,
+                               double* grad_off, double* grad_logits, double* grad_ref_cam);
+
 /* Dense projection ([BQ] 3 value projection, 4.1 offset head, 4.2 weight
  * head, 11 output projection, 13 residual):
  *   y[m, n] = sum_k x[m, k] w[n, k] + bias[n] + residual[m, n]
@@ -117,6 +139,30 @@ int oracle_sca_backward(const double* value, int B, int Ncam, int Nv, int H, int
  * or NULL; y [M, N]. */
 int oracle_linear(const double* x, const double* w, const double* bias, const double* residual,
                   int M, int N, int K, double* y);
+
+/* TSA reference points ([TS] BEV encoder listing; the transform is this
+ * oracle's reading of "align the previous BEV with the ego motion"):
+ * BEV query q = i * bev_w + j has the cell centre ((j + 1/2) / bev_w,
+ * (i + 1/2) / bev_h), in metres about the BEV centre
+ * p = ((j + 1/2 - bev_w / 2) gx, (i + 1/2 - bev_h / 2) gy).  Queue t sees
+ * that point at p' = Rot(theta) p + (dx, dy), returned normalised:
+ * (p'_x / (bev_w gx) + 1/2, p'_y / (bev_h gy) + 1/2).
+ * ego [B, T, 3] = (dx metres, dy metres, theta degrees, counter-clockwise
+ * from +x towards +y); a queue with (0, 0, 0) gets the cell centres.
+ * ref [B, T, bev_h * bev_w, 2]. */
+int oracle_tsa_reference_points(int B, int T, int bev_h, int bev_w, double gx, double gy,
+                                const double* ego, double* ref);
+
+/* TSA forward ([TS] 二.2 read as: every BEV query samples each of the T
+ * queues with its own offsets and logits, by the fused MSDA above, and its
+ * output is the mean over the queues, summed in ascending t):
+ * value [B*T, Nv, H, Dh] (row b*T + t); ref [B*T, Nq, R, 2];
+ * off [B*T, Nq, H, L, P, 2]; logits [B*T, Nq, H, L, P]; out [B, Nq, H*Dh]. */
+int oracle_tsa_forward(const double* value, int B, int T, int Nv, int H, int Dh,
+                       int L, const int64_t* shapes, const int64_t* starts,
+                       int Nq, int P, int R, const double* ref,
+                       const double* off, const double* logits,
+                       int coord_f32, double* out);
 
 #ifdef __cplusplus
 }

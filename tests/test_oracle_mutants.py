@@ -63,8 +63,26 @@ MUTANTS = [
     ("projection weight transposed", "acc += x[(int64_t)m * K + k] * w[(int64_t)n * K + k];",
      "acc += x[(int64_t)m * K + k] * w[(int64_t)k * N + n];", 0),
     ("projection bias dropped", "if (bias) acc += bias[n];", "", 0),
+    ("offset gradient not divided by the width",
+     "grad_off[(bq * S + s) * 2 + 0] += gl[2 * s + 0] / Wl;", "grad_off[(bq * S + s) * 2 + 0] += gl[2 * s + 0];", 0),
+    ("softmax backward without the centring",
+     "grad_logits[base + j] = alpha[j] * (G[base + j] - dot);", "grad_logits[base + j] = alpha[j] * G[base + j];", 0),
+    ("reference gradient on anchor k / (P/R)", "gr[2 * (k % R) + 0] += gl[2 * s + 0];",
+     "gr[2 * (k / (P / R)) + 0] += gl[2 * s + 0];", 0),
     ("SCA backward not divided by the count",
      "sc.row[d] = grad_out[bq * HD + d] / (double)n;", "sc.row[d] = grad_out[bq * HD + d];", 0),
+    ("ego rotation sign flipped", "const double qx = cs * px - sn * py + dx;",
+     "const double qx = cs * px + sn * py + dx;", 0),
+    ("ego rotation about the corner", "const double px = ((double)j + 0.5 - 0.5 * bev_w) * gx;",
+     "const double px = ((double)j + 0.5) * gx;", 0),
+    ("ego translation in cells", "const double qy = sn * px + cs * py + dy;",
+     "const double qy = sn * px + cs * py + dy * gy;", 0),
+    ("BEV x normalised by the height grid", "r[0] = qx / (bev_w * gx) + 0.5;",
+     "r[0] = qx / (bev_w * gy) + 0.5;", 0),
+    ("queue mean not divided", "out[((int64_t)b * Nq + q) * HD + d] = sum / T;",
+     "out[((int64_t)b * Nq + q) * HD + d] = sum;", 0),
+    ("every queue reads queue 0", "sum += per_queue[(((int64_t)b * T + t) * Nq + q) * HD + d];",
+     "sum += per_queue[(((int64_t)b * T + 0) * Nq + q) * HD + d];", 0),
 ]
 
 PIN_CALLS = [
@@ -90,6 +108,11 @@ PIN_CALLS = [
     ("sca_fd", lambda: pins.test_sca_backward_matches_finite_differences()),
     ("linear_numpy", lambda: pins.test_linear_matches_numpy_matmul()),
     ("linear_s15", lambda: pins.test_section15_output_projection_and_residual()),
+    ("tsa_centres", lambda: pins.test_tsa_reference_points_without_motion_are_cell_centres()),
+    ("tsa_translation", lambda: pins.test_tsa_reference_points_whole_cell_translation()),
+    ("tsa_rigid", lambda: pins.test_tsa_reference_points_are_a_rigid_motion()),
+    ("tsa_rot90", lambda: pins.test_tsa_quarter_turns_rotate_the_previous_map(90.0, 1)),
+    ("tsa_shift", lambda: pins.test_tsa_whole_cell_shift_moves_the_previous_map()),
 ]
 
 
@@ -115,7 +138,9 @@ def test_pins_catch_planted_mistake(tmp_path, monkeypatch, name, old, new, occ):
     mutant = ctypes.CDLL(str(so))
     for fname in ("oracle_softmax", "oracle_msda_forward", "oracle_msda_forward_fused",
                   "oracle_fused_locations", "oracle_msda_backward", "oracle_sca_compact",
-                  "oracle_sca_forward", "oracle_sca_backward", "oracle_linear"):
+                  "oracle_sca_forward", "oracle_sca_backward", "oracle_linear",
+                  "oracle_sca_backward_inputs", "oracle_tsa_reference_points",
+                  "oracle_tsa_forward"):
         fn = getattr(mutant, fname)
         fn.argtypes = getattr(good, fname).argtypes
         fn.restype = ctypes.c_int

@@ -502,11 +502,10 @@ def test_msda_backward_linearity():
 
 
 def test_sca_backward_matches_finite_differences():
-    """FD through the whole SCA forward.  grad_value directly; the rebatched
-    location and weight gradients through the chain rule of the fused inputs:
-    d/d offset = sum over seeing cameras of grad_loc / (W_l, H_l),
-    d/d reference point of camera c = sum over points of that anchor,
-    d/d logits = softmax Jacobian of the camera-summed grad_attn."""
+    """FD through the whole SCA forward: grad_value directly, and the
+    gradients of the offsets, reference points and logits that
+    oracle.sca_backward_inputs forms from the rebatched location and weight
+    gradients."""
     t = _tiny_sca(15)
     rng = _rng(16)
     B, Ncam, Nq, H, Dh, L, P, R = (t[k] for k in ("B", "Ncam", "Nq", "H", "Dh", "L", "P", "R"))
@@ -540,24 +539,11 @@ def test_sca_backward_matches_finite_differences():
     np.testing.assert_allclose(gv, _central_fd(loss, t["value"], h), rtol=1e-6, atol=1e-8)
 
     idx, cnt, pos, hits = oracle.sca_compact(t["mask"])
-    g_off = np.zeros_like(t["off"])
-    g_ref = np.zeros_like(t["ref"])
-    g_alpha = np.zeros_like(t["logits"])
-    norm = np.array([[Wl, Hl] for (Hl, Wl) in shapes], dtype=np.float64)  # [L, 2]
     for b in range(B):
         for c in range(Ncam):
-            for i in range(cnt[b, c]):
-                q = idx[b, c, i]
-                g_off[b, q] += gl_rb[b, c, i] / norm[None, :, None, :]
-                g_alpha[b, q] += gw_rb[b, c, i]
-                for k in range(P):
-                    g_ref[c, b, q, k % R] += gl_rb[b, c, i, :, :, k, :].sum(axis=(0, 1))
             assert np.all(gl_rb[b, c, cnt[b, c]:] == 0) and np.all(gw_rb[b, c, cnt[b, c]:] == 0)
-    alpha = oracle.softmax(t["logits"], L * P).reshape(g_alpha.shape)
-    ga = g_alpha.reshape(B, Nq, H, L * P)
-    al = alpha.reshape(B, Nq, H, L * P)
-    g_logits = (al * (ga - np.sum(al * ga, -1, keepdims=True))).reshape(g_alpha.shape)
-
+    g_off, g_logits, g_ref = oracle.sca_backward_inputs(shapes, t["mask"], t["logits"], gl_rb,
+                                                        gw_rb)
     np.testing.assert_allclose(g_off, _central_fd(loss, t["off"], h), rtol=1e-6, atol=1e-7)
     np.testing.assert_allclose(g_ref, _central_fd(loss, t["ref"], h), rtol=1e-6, atol=1e-7)
     np.testing.assert_allclose(g_logits, _central_fd(loss, t["logits"], h), rtol=1e-6, atol=1e-8)
@@ -599,3 +585,141 @@ def test_section15_output_projection_and_residual():
     g = json.load(open(os.path.join(GOLDEN, "bq_s15_two_head_example.json")))
     q_hat = oracle.linear(np.asarray(g["g"])[None], np.eye(4), None, np.asarray(g["q"])[None])
     np.testing.assert_allclose(q_hat[0], g["q_hat"], rtol=1e-15)
+
+
+def test_round_bf16_ties_to_even():
+    # 1 + 2^-8 is halfway between the bf16 neighbours 1 and 1 + 2^-7: to even (1)
+    x = np.array([1.0, 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -2.5, 3.0e-3])
+    r = oracle.round_bf16(x)
+    assert r[0] == 1.0 and r[1] == 1.0 and r[2] == 1.0 + 2.0 ** -6 and r[3] == -2.5
+    assert abs(r[4] - 3.0e-3) <= 2.0 ** -8 * 3.0e-3  # half an ulp of an 8-bit significand
+
+
+def test_module_with_identity_projections_is_residual_plus_sca():
+    """W_v = I, zero offset/weight heads except their biases, W_o = I: the
+    module returns q + bf16(SCA(V = F~)) (sections 13 and 10)."""
+    rng = _rng(42)
+    B, Ncam, Nq, C, L, P, R = 1, 2, 6, 32, 2, 2, 2
+    shapes, starts, Nv = _levels([(3, 4), (2, 2)])
+    q = rng.standard_normal((B, Nq, C))
+    feats = oracle.round_bf16(rng.standard_normal((B, Ncam, Nv, C)))
+    ref = rng.uniform(0.1, 0.9, (Ncam, B, Nq, R, 2))
+    mask = (rng.random((Ncam, B, Nq, R)) < 0.6).astype(np.uint8)
+    S = 1 * L * P
+    b_off = rng.standard_normal(S * 2) * 0.5
+    b_w = rng.standard_normal(S)
+    y = oracle.sca_module_forward(q, None, feats, np.eye(C), None, np.zeros((2 * S, C)), b_off,
+                                  np.zeros((S, C)), b_w, np.eye(C), None, ref, mask, shapes,
+                                  starts, L, P)
+    off = np.broadcast_to(b_off.reshape(1, 1, 1, L, P, 2), (B, Nq, 1, L, P, 2))
+    lg = np.broadcast_to(b_w.reshape(1, 1, 1, L, P), (B, Nq, 1, L, P))
+    g = oracle.sca_forward(feats.reshape(B, Ncam, Nv, 1, C), shapes, starts, ref, mask, off, lg)
+    np.testing.assert_allclose(y, q + oracle.round_bf16(g), rtol=1e-12, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# TSA: ego-motion reference points and the queue mean ("【论文阅读】BEVFormer
+# 论文解析及Temporal Self-Attention、Spatial Cross-Attention注意力机制详解及
+# 代码示例", section 二.2 and the BEV encoder listing)
+# --------------------------------------------------------------------------
+
+def _cell_centres(bev_h, bev_w):
+    i, j = np.meshgrid(np.arange(bev_h), np.arange(bev_w), indexing="ij")
+    return np.stack([(j + 0.5) / bev_w, (i + 0.5) / bev_h], -1).reshape(-1, 2)
+
+
+def test_tsa_reference_points_without_motion_are_cell_centres():
+    ref = oracle.tsa_reference_points(5, 7, np.zeros((2, 2, 3)))
+    for b in range(2):
+        for t in range(2):
+            np.testing.assert_allclose(ref[b, t], _cell_centres(5, 7), rtol=0, atol=1e-15)
+
+
+def test_tsa_reference_points_whole_cell_translation():
+    """No rotation, a motion of (3 cells, -2 cells): the point seen is the
+    centre of cell (i - 2, j + 3).  Unequal grid lengths pin x to the width."""
+    gy, gx = 0.3, 0.512
+    ego = np.array([[[3 * gx, -2 * gy, 0.0]]])
+    ref = oracle.tsa_reference_points(6, 9, ego, grid_length=(gy, gx))[0, 0]
+    want = _cell_centres(6, 9) + np.array([3 / 9, -2 / 6])
+    np.testing.assert_allclose(ref, want, rtol=0, atol=1e-14)
+
+
+def test_tsa_reference_points_are_a_rigid_motion():
+    """Distances in metres are kept, and the centroid of the cell centres
+    (the BEV centre) lands on the translation."""
+    gy, gx = 0.4, 0.512
+    H, W = 7, 10
+    ego = np.array([[[1.3, -0.7, 33.0]]])
+    ref = oracle.tsa_reference_points(H, W, ego, grid_length=(gy, gx))[0, 0]
+    metres = (ref - 0.5) * np.array([W * gx, H * gy])
+    base = (_cell_centres(H, W) - 0.5) * np.array([W * gx, H * gy])
+    d_new = np.linalg.norm(metres[:, None] - metres[None], axis=-1)
+    d_old = np.linalg.norm(base[:, None] - base[None], axis=-1)
+    np.testing.assert_allclose(d_new, d_old, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(metres.mean(0), [1.3, -0.7], rtol=0, atol=1e-12)
+
+
+def _tsa_point_sampler(prev, cur, ego_prev):
+    """Both queues sampled with one point, zero offsets: the output is the
+    mean of the two maps read at each queue's reference point."""
+    N, _, D = prev.shape
+    shapes, starts, Nv = _levels([(N, N)])
+    value = np.stack([prev.reshape(Nv, 1, D), cur.reshape(Nv, 1, D)])
+    ego = np.array([[ego_prev, [0.0, 0.0, 0.0]]])
+    ref = oracle.tsa_reference_points(N, N, ego).reshape(2, N * N, 1, 2)
+    off = np.zeros((2, N * N, 1, 1, 1, 2))
+    lg = np.zeros((2, N * N, 1, 1, 1))
+    return oracle.tsa_forward(value, shapes, starts, ref, off, lg, 2)[0].reshape(N, N, D)
+
+
+@pytest.mark.parametrize("angle,turns", [(90.0, 1), (180.0, 2), (-90.0, 3)])
+def test_tsa_quarter_turns_rotate_the_previous_map(angle, turns):
+    """A yaw of k * 90 degrees about the BEV centre moves cell centres onto
+    cell centres: the previous queue then returns its map turned like
+    numpy's rot90 (x along the columns, counter-clockwise from +x to +y), and
+    the output is the mean with the current map."""
+    rng = _rng(60)
+    N, D = 6, 3
+    prev, cur = rng.standard_normal((N, N, D)), rng.standard_normal((N, N, D))
+    out = _tsa_point_sampler(prev, cur, [0.0, 0.0, angle])
+    want = 0.5 * (np.rot90(prev, turns, axes=(0, 1)) + cur)
+    np.testing.assert_allclose(out, want, rtol=0, atol=1e-6)
+
+
+def test_tsa_whole_cell_shift_moves_the_previous_map():
+    """A motion of one cell along +x and two along -y reads cell (i - 2, j + 1)
+    of the previous map; cells whose source leaves the map read zero."""
+    rng = _rng(61)
+    N, D = 7, 2
+    prev, cur = rng.standard_normal((N, N, D)), rng.standard_normal((N, N, D))
+    out = _tsa_point_sampler(prev, cur, [0.512, -2 * 0.512, 0.0])
+    shifted = np.zeros_like(prev)
+    shifted[2:, :N - 1] = prev[:N - 2, 1:]
+    np.testing.assert_allclose(out, 0.5 * (shifted + cur), rtol=0, atol=1e-6)
+
+
+def test_tsa_single_queue_is_the_fused_msda():
+    w = inputs.workload4(bev_h=9, bev_w=11)
+    out = oracle.tsa_forward(w.value[:1], w.spatial_shapes, w.level_start_index,
+                             w.reference_points[:1], w.sampling_offsets[:1],
+                             w.attention_logits[:1], 1)
+    ref = oracle.msda_forward_fused(w.value[:1], w.spatial_shapes, w.level_start_index,
+                                    w.reference_points[:1], w.sampling_offsets[:1],
+                                    w.attention_logits[:1])
+    np.testing.assert_array_equal(out, ref)
+
+
+def test_tsa_mean_is_symmetric_in_the_queues():
+    w = inputs.workload4(bev_h=9, bev_w=11)
+    args = (w.value, w.reference_points, w.sampling_offsets, w.attention_logits)
+    a = oracle.tsa_forward(args[0], w.spatial_shapes, w.level_start_index, *args[1:], 2)
+    b = oracle.tsa_forward(*(x[::-1] for x in args[:1]), w.spatial_shapes, w.level_start_index,
+                           *(x[::-1] for x in args[1:]), 2)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-14)
+    same = oracle.tsa_forward(np.concatenate([args[0][:1]] * 2), w.spatial_shapes,
+                              w.level_start_index,
+                              *(np.concatenate([x[:1]] * 2) for x in args[1:]), 2)
+    one = oracle.msda_forward_fused(args[0][:1], w.spatial_shapes, w.level_start_index,
+                                    *(x[:1] for x in args[1:]))
+    np.testing.assert_allclose(same, one, rtol=0, atol=1e-14)
