@@ -39,6 +39,7 @@ sys.path.insert(0, ROOT)
 METRIC = "MSDA sampled points/sec (G/s) + HBM GB/s fraction, BEVFormer-base SCA"
 UNIT = "Gsamples/s"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 L2_FLUSH_BYTES = 256 << 20
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "sca_gather_bevformer_base.md")
 KERNEL_SOURCES = ("scale_deformable_attention_03_b200/csrc/msda_device.cuh",
@@ -54,6 +55,8 @@ def parse_args(argv=None):
     p.add_argument("--value-dtype", choices=("f32", "bf16"), default="f32")
     p.add_argument("--rho", choices=("coherent", "uniform"), default="coherent")
     p.add_argument("--e2e-steps", type=int, default=5)
+    p.add_argument("--rows-iters", type=int, default=20,
+                   help="timed calls per entry point in the next_rows section (0 = skip)")
     p.add_argument("--cpu-seconds", type=float, default=10.0,
                    help="minimum host time of the oracle CPU baseline")
     return p.parse_args(argv)
@@ -121,6 +124,37 @@ def measured_hbm_peak():
         return v, "measured (MEASURED_PEAKS.json hbm_gbs, copy burst)"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback (6.65 TB/s pool measurement)"
+
+
+def measured_bf16_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops)"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback (1.59 PFLOP/s pool measurement)"
+
+
+def tsa_algorithmic_bytes(w, T, value_elem):
+    """tsa_forward: every queue's value, offsets, logits and reference points
+    once, the averaged output once."""
+    S = w.H * w.L * w.P
+    return int(w.value.size * value_elem + w.B * w.Nq * S * 3 * 4
+               + w.B * w.Nq * w.R * 2 * 4 + (w.B // T) * w.Nq * w.H * 32 * 4)
+
+
+def linear_algorithmic_bytes(M, N, K, y_elem, bias=True, residual=False):
+    """msda_linear: x, w (and bias, residual) read once, y written once."""
+    return int(M * K * 2 + N * K * 2 + (N * 4 if bias else 0) + (M * N * 4 if residual else 0)
+               + M * N * y_elem)
+
+
+def input_grads_algorithmic_bytes(w, rows):
+    """sca_backward_inputs: logits, positions, the rebatched gradients of the
+    seen rows once; the three gradients written once."""
+    S = w.H * w.L * w.P
+    return int(w.B * w.Nq * S * 4 + w.B * w.Ncam * w.Nq * 4 + rows * S * 3 * 4
+               + w.B * w.Nq * S * 3 * 4 + w.Ncam * w.B * w.Nq * w.R * 2 * 4)
 
 
 def kernel_source_digest():
@@ -453,10 +487,142 @@ def run_native(args):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
+    if world == 1 and args.rows_iters > 0:
+        tensors = {"value": value, "ref": ref, "mask": mask, "off": off, "logits": logits,
+                   "step_bytes": nbytes["step"], "samples": samples_per_step}
+        line["next_rows"] = measure_next_rows(args, w, tensors, flush, stream, peak)
     if world == 1:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     print(json.dumps(line), flush=True)
     return 0
+
+
+# --------------------------------------------------------------------------
+# the other entry points of the path, each on its full workload
+# --------------------------------------------------------------------------
+
+def measure_next_rows(args, w, tensors, flush, stream, hbm_peak):
+    """Mean CUDA-event time of each further entry point (after three warm-up
+    calls, the L2 flushed before every call, outside the events), with its
+    algorithmic bytes against the measured HBM copy bandwidth."""
+    import torch
+
+    import scale_deformable_attention_03_b200 as msda
+    from scale_deformable_attention_03_b200 import inputs
+
+    iters = args.rows_iters
+
+    def timed(fn, n=iters):
+        for _ in range(3):
+            flush.zero_()
+            fn()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n)]
+        for a, b in evs:
+            flush.zero_()
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        return float(np.mean([a.elapsed_time(b) for a, b in evs]))
+
+    def hbm(nbytes, ms):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        return {"ms": ms, "algorithmic_bytes": int(nbytes), "achieved_gbs": gbs,
+                "hbm_frac": gbs / hbm_peak}
+
+    rows = {}
+    bf16 = args.value_dtype == "bf16"
+    value, ref, mask, off, logits = (tensors[k] for k in ("value", "ref", "mask", "off",
+                                                          "logits"))
+    shapes, starts = w.spatial_shapes, w.level_start_index
+
+    # f2: query-major SCA forward (one kernel, the whole step's algorithmic bytes)
+    out = torch.empty((w.B, w.Nq, w.H * 32), dtype=torch.float32, device="cuda")
+    ms = timed(lambda: msda.sca_forward_query_major(value, shapes, starts, ref, mask, off,
+                                                    logits, out=out))
+    r = hbm(tensors["step_bytes"], ms)
+    r.update(kernel="sca_query_major_kernel", workload="bevformer-base-sca-forward",
+             gsamples_per_s=tensors["samples"] / (ms * 1e-3) / 1e9)
+    rows["sca_forward_query_major"] = r
+
+    # f4: TSA, two queues of the 200x200 BEV, ego motion (1.7 m, -0.9 m, 4 deg)
+    w4 = inputs.workload4()
+    ego = torch.tensor([[[1.7, -0.9, 4.0], [0.0, 0.0, 0.0]]], dtype=torch.float32,
+                       device="cuda")
+    ref4 = msda.tsa_reference_points(ego, 200, 200)
+    v4 = torch.from_numpy(w4.value).cuda()
+    off4 = torch.from_numpy(w4.sampling_offsets).cuda()
+    lg4 = torch.from_numpy(w4.attention_logits).cuda()
+    out4 = torch.empty((1, w4.Nq, w4.H * 32), dtype=torch.float32, device="cuda")
+    ref4v = ref4.view(2, w4.Nq, 1, 2)
+    ms = timed(lambda: msda.tsa_forward(v4, w4.spatial_shapes, w4.level_start_index, ref4v,
+                                        off4, lg4, 2, out=out4))
+    r = hbm(tsa_algorithmic_bytes(w4, 2, 4), ms)
+    r.update(kernel="tsa_forward_group_kernel<float, 2, 2>",
+             workload="bevformer-tsa 2 queues x 200x200, H=8, P=4, fp32",
+             gsamples_per_s=2 * w4.Nq * w4.H * w4.L * w4.P / (ms * 1e-3) / 1e9)
+    rows["tsa_forward"] = r
+    ms = timed(lambda: msda.tsa_reference_points(ego, 200, 200, out=ref4))
+    rows["tsa_reference_points"] = hbm(2 * w4.Nq * 8 + 24, ms)
+    del v4, off4, lg4, out4, ref4
+
+    # A12: the value projection of all six cameras' features, M = 6 * 30825
+    g = torch.Generator(device="cuda").manual_seed(7)
+    M, N, K = w.Ncam * w.Nv, 256, 256
+    x = torch.randn((M, K), device="cuda", generator=g).to(torch.bfloat16)
+    wt = (torch.randn((N, K), device="cuda", generator=g) / 16).to(torch.bfloat16)
+    bias = torch.randn(N, device="cuda", generator=g)
+    peak_tf, peak_tf_src = measured_bf16_peak()
+    for y_dtype, y_elem in (("f32", 4), ("bf16", 2)):
+        y = torch.empty((M, N), device="cuda",
+                        dtype=torch.float32 if y_dtype == "f32" else torch.bfloat16)
+        ms = timed(lambda: msda.msda_linear(x, wt, bias, out=y))
+        r = hbm(linear_algorithmic_bytes(M, N, K, y_elem), ms)
+        tflops = 2.0 * M * N * K / (ms * 1e-3) / 1e12
+        r.update(kernel="proj_gemm_kernel (tcgen05)", shape=[M, N, K], y_dtype=y_dtype,
+                 tflops=tflops, tensor_frac=tflops / peak_tf, tensor_peak_source=peak_tf_src)
+        rows[f"msda_linear_value_proj_{y_dtype}"] = r
+    del x, y
+
+    # f1: the whole SCA module forward (projections + SCA + output projection)
+    C = w.H * 32
+    S = w.H * w.L * w.P
+    q = torch.randn((w.B, w.Nq, C), device="cuda", generator=g)
+    feats = torch.randn((w.B, w.Ncam, w.Nv, C), device="cuda", generator=g).to(torch.bfloat16)
+
+    def lin(n_out):
+        return ((torch.randn((n_out, C), device="cuda", generator=g) / 16).to(torch.bfloat16),
+                torch.randn(n_out, device="cuda", generator=g) * 0.1)
+
+    (wv, bv), (wo_, bo_), (wa, ba), (wout, bout) = lin(C), lin(2 * S), lin(S), lin(C)
+    mod_out = torch.empty_like(q)
+    vdt = torch.bfloat16 if bf16 else None
+    mod_dims = msda.Dims(w.B, w.Ncam, w.Nq, w.Nv, w.H, w.L, w.P, w.R)
+    mod_ws = torch.empty(int(msda.lib().sca_module_workspace_size(
+        mod_dims, msda.MSDA_BF16 if bf16 else msda.MSDA_F32)), dtype=torch.uint8, device="cuda")
+    ms = timed(lambda: msda.sca_module_forward(q, None, feats, wv, bv, wo_, bo_, wa, ba, wout,
+                                               bout, ref, mask, shapes, starts, w.L, w.P,
+                                               value_dtype=vdt, out=mod_out,
+                                               workspace=mod_ws))
+    rows["sca_module_forward"] = {"ms": ms, "workload": "bevformer-base SCA module, C=256",
+                                  "gsamples_per_s": tensors["samples"] / (ms * 1e-3) / 1e9}
+    del feats, q, mod_out, mod_ws
+
+    # f3: gradients of offsets, logits and reference points from the rebatched ones
+    idx, cnt, pos, hits = msda.sca_compact(mask)
+    gout = torch.randn((w.B, w.Nq, C), device="cuda", generator=g)
+    _, gl, gw = msda.sca_rebatched_backward(value, shapes, starts, ref, off, logits, gout, idx,
+                                            cnt, hits)
+    n_rows = int(cnt.sum().item())
+    bufs = msda.sca_backward_inputs(shapes, starts, logits, pos, gl, gw, w.Ncam, w.R)
+    ms = timed(lambda: msda.sca_backward_inputs(shapes, starts, logits, pos, gl, gw, w.Ncam,
+                                                w.R, out=bufs))
+    r = hbm(input_grads_algorithmic_bytes(w, n_rows), ms)
+    r.update(kernel="sca_offset_logit_grads_kernel + sca_reference_grads_kernel")
+    rows["sca_backward_inputs"] = r
+    return rows
 
 
 def main(argv=None):

@@ -7,6 +7,10 @@
  *         Feature" (leheavengame.com repost of a CSDN article).
  *   [SCA] "Spatial Cross-Attention" walkthrough, Tencent Cloud developer
  *         article 2321140 (rebatch listing, scatter-add / average listing).
+ *   [TS]  "【论文阅读】BEVFormer论文解析及Temporal Self-Attention、Spatial
+ *         Cross-Attention注意力机制详解及代码示例" (wsisp.com): section 二.2
+ *         (TSA) and the BEV encoder listing (ego motion from the CAN bus,
+ *         0.512 m BEV cells).
  *
  * What one MSDA output row computes ([BQ] sections 4.2, 5, 6, 8, 9):
  *   alpha_{h,l,k} = softmax over the L*P logits of head h        (4.2)
@@ -53,6 +57,7 @@ extern "C" {
 #define MSDA_MAX_POINTS 16  /* P */
 #define MSDA_MAX_CAMERAS 32 /* Ncam */
 #define MSDA_MAX_BATCH_CAMERAS 1024 /* B * Ncam for the sca_* calls */
+#define MSDA_MAX_QUEUES 4   /* T, BEV queues of tsa_forward */
 
 struct CUstream_st;
 typedef struct CUstream_st* msda_stream_t; /* the same type as cudaStream_t */
@@ -107,6 +112,48 @@ msda_status_t msda_forward_fused(const void* value, msda_dtype_t vdt,
                                  const float* reference_points, const float* sampling_offsets,
                                  const float* attention_logits, msda_dims_t d, float* out,
                                  msda_stream_t stream);
+
+/* TSA reference points ([TS] BEV encoder listing).  The listing takes the
+ * ego motion (delta_x, delta_y in metres, the yaw in degrees) from the CAN
+ * bus and 0.512 m BEV cells, and stops before it applies them; this call
+ * reads "align the BEV of queue t with the current frame" as a rigid motion
+ * of the cell centres:
+ *   query q = i * bev_w + j has the centre p = ((j + 1/2 - bev_w/2) gx,
+ *   (i + 1/2 - bev_h/2) gy) metres about the BEV centre; queue t sees it at
+ *   p' = Rot(theta) p + (dx, dy), returned normalised as
+ *   (p'_x / (bev_w gx) + 1/2, p'_y / (bev_h gy) + 1/2).
+ * A queue with zero motion gets the cell centres ((j + 1/2) / bev_w,
+ * (i + 1/2) / bev_h).  Computed in double, rounded once to fp32.
+ *   ego_motion        [B, T, 3]             fp32 (dx m, dy m, theta degrees,
+ *                                           counter-clockwise from +x to +y)
+ *   reference_points  [B, T, bev_h*bev_w, 2] fp32, written; as [B*T, Nq, 1, 2]
+ *                                           it is tsa_forward's input (R = 1)
+ * grid_length_y, grid_length_x: metres per BEV cell along the height and the
+ * width (BEVFormer: 0.512, 0.512), finite and > 0. */
+msda_status_t tsa_reference_points(const float* ego_motion, int32_t B, int32_t num_queues,
+                                   int32_t bev_h, int32_t bev_w, double grid_length_y,
+                                   double grid_length_x, float* reference_points,
+                                   msda_stream_t stream);
+
+/* TSA forward ([TS] 二.2): every BEV query attends to T = num_queues BEV
+ * queues (BEVFormer: the ego-aligned previous BEV, then the current one),
+ * each with its own offsets and logits, through the fused MSDA of
+ * msda_forward_fused; the output is the mean over the queues (the pages give
+ * TSA only as generic attention: the mean is this library's reading).  One
+ * kernel: the per-queue rows stay in registers.
+ *   d.B                 BEV samples; the value holds d.B * T batch items,
+ *                       item b * T + t being queue t of sample b
+ *   value               [B*T, Nv, H, 32]        fp32 or bf16 (vdt)
+ *   reference_points    [B*T, Nq, R, 2]         fp32, (x, y) normalised
+ *   sampling_offsets    [B*T, Nq, H, L, P, 2]   fp32, level pixels
+ *   attention_logits    [B*T, Nq, H, L, P]      fp32
+ *   out                 [B, Nq, H * 32]         fp32, written:
+ *                       (1/T) sum_t msda_forward_fused(item b*T + t)
+ * num_queues: 1 .. MSDA_MAX_QUEUES, else MSDA_ERR_UNSUPPORTED. */
+msda_status_t tsa_forward(const void* value, msda_dtype_t vdt, const int64_t* spatial_shapes,
+                          const int64_t* level_start_index, const float* reference_points,
+                          const float* sampling_offsets, const float* attention_logits,
+                          int32_t num_queues, msda_dims_t d, float* out, msda_stream_t stream);
 
 /* MSDA backward: the derivative of msda_forward (the pages give no backward;
  * this is the analytic derivative of [BQ] 6 and 8).
@@ -242,6 +289,24 @@ msda_status_t sca_forward(const void* value, msda_dtype_t vdt,
                           msda_dims_t d, void* workspace, size_t workspace_bytes, float* out,
                           msda_stream_t stream);
 
+/* SCA forward, query-major ([BQ] 10: each BEV query samples the cameras that
+ * see it and averages them; [SCA] average listing: the count is clamped at
+ * one).  The same result as sca_forward, from one kernel and without
+ * workspace: one warp per (query, head) takes the softmax once, walks the
+ * seeing cameras in ascending order into the same partial sums and writes
+ * the mean once.  Arguments and layouts as sca_forward's; B * Ncam is not
+ * limited to MSDA_MAX_BATCH_CAMERAS here.  The camera sum is formed before
+ * the four-corner reduction, so results differ from sca_forward's in
+ * rounding only. */
+msda_status_t sca_forward_query_major(const void* value, msda_dtype_t vdt,
+                                      const int64_t* spatial_shapes,
+                                      const int64_t* level_start_index,
+                                      const float* reference_points_cam, const uint8_t* bev_mask,
+                                      const float* sampling_offsets,
+                                      const float* attention_logits, msda_dims_t d, float* out,
+                                      msda_stream_t stream);
+
+
 /* SCA backward on a given compaction: derivative of sca_forward with respect
  * to the value and to the per-camera (rebatched) sampling locations and
  * attention weights.  The upstream gradient of row i of camera c is
@@ -274,6 +339,65 @@ msda_status_t sca_backward(const void* value, msda_dtype_t vdt,
                            size_t workspace_bytes, float* grad_value,
                            float* grad_sampling_locations_rb, float* grad_attention_weights_rb,
                            msda_stream_t stream);
+
+/* The BEVFormer SCA module forward, end to end on the GPU ([BQ] 3, 4, 10-14;
+ * [SCA] listings):
+ *   q~ = bf16(q + pos);  V = F~ W_v^T + b_v;  Delta = q~ W_Delta^T + b_Delta;
+ *   a = q~ W_alpha^T + b_alpha;  g = sca_forward(V, Delta, a, rho, mask);
+ *   q_hat = q + bf16(g) W_o^T + b_o   (dropout is the identity, [BQ] 12;
+ *   the LayerNorm after it belongs to the outer layer, [BQ] 13).
+ * C = H * 32.  The projections run on msda_linear, so C and H*L*P must be
+ * multiples of 256 and C one of 64..256 (BEVFormer-base: C = 256, H = 8,
+ * L = 4, P = 8).  Weights use the nn.Linear layout (out x in), bf16; biases
+ * fp32 (may be NULL). */
+typedef struct {
+    const float* query;                /* [B, Nq, C] fp32: q, also the residual */
+    const float* query_pos;            /* [B, Nq, C] fp32 or NULL: pos */
+    const void* features;              /* [B, Ncam, Nv, C] bf16: F~ = FPN + camera + level
+                                          embeddings, level rows as level_start_index */
+    const void* w_value;               /* [C, C] bf16 */
+    const float* b_value;              /* [C] */
+    const void* w_offsets;             /* [H*L*P*2, C] bf16 (rows h, l, k, xy) */
+    const float* b_offsets;            /* [H*L*P*2] */
+    const void* w_weights;             /* [H*L*P, C] bf16 */
+    const float* b_weights;            /* [H*L*P] */
+    const void* w_output;              /* [C, C] bf16 */
+    const float* b_output;             /* [C] */
+    const float* reference_points_cam; /* [Ncam, B, Nq, R, 2] */
+    const uint8_t* bev_mask;           /* [Ncam, B, Nq, R] */
+    msda_dtype_t value_dtype;          /* storage of V for the sampling: fp32 or bf16 */
+} sca_module_params_t;
+
+/* Bytes of device workspace sca_module_forward needs (q~, V, Delta, a, g and
+ * the sca_forward workspace), 256-byte alignment included. */
+size_t sca_module_workspace_size(msda_dims_t d, msda_dtype_t value_dtype);
+
+/*   q_hat [B, Nq, C] fp32, written.  workspace 256-byte aligned. */
+msda_status_t sca_module_forward(const sca_module_params_t* params,
+                                 const int64_t* spatial_shapes,
+                                 const int64_t* level_start_index, msda_dims_t d,
+                                 void* workspace, size_t workspace_bytes, float* q_hat,
+                                 msda_stream_t stream);
+
+/* Gradients of the SCA inputs from sca_rebatched_backward's rebatched
+ * gradients ([BQ] 4.2 softmax, 5 location, 10: offsets and logits are the
+ * BEV query's and every camera shares them, so their gradients sum over the
+ * cameras that see the query, in ascending camera order, without atomics):
+ *   grad_sampling_offsets     [B, Nq, H, L, P, 2] = sum_c grad_loc / (W_l, H_l)
+ *   grad_attention_logits     [B, Nq, H, L, P]    = alpha (G - <alpha, G>),
+ *                                                   G = sum_c grad_attn
+ *   grad_reference_points_cam [Ncam, B, Nq, R, 2] = sum over the points k with
+ *                                 k mod R = m of the camera's grad_loc (zero
+ *                                 where the camera does not see the query)
+ *   attention_logits          [B, Nq, H, L, P] (alpha is recomputed)
+ *   pos                       from sca_compact
+ *   grad_*_rb                 from sca_rebatched_backward */
+msda_status_t sca_backward_inputs(const int64_t* spatial_shapes, const int64_t* level_start_index,
+                                  const float* attention_logits, const int32_t* pos,
+                                  const float* grad_sampling_locations_rb,
+                                  const float* grad_attention_weights_rb, msda_dims_t d,
+                                  float* grad_sampling_offsets, float* grad_attention_logits,
+                                  float* grad_reference_points_cam, msda_stream_t stream);
 
 /* Fixed text for a status code. */
 const char* msda_status_string(msda_status_t status);

@@ -10,8 +10,8 @@ status.  There is no fallback: without the built library every call raises.
 Functions (same names as the C ABI): ``msda_forward``, ``msda_forward_fused``,
 ``msda_backward``, ``sca_compact``, ``sca_rebatched_forward``,
 ``sca_camera_average``, ``sca_forward``, ``sca_rebatched_backward``,
-``sca_backward``, ``msda_linear``, ``msda_workspace_size``,
-``sca_compact_workspace_size``.
+``sca_backward``, ``msda_linear``, ``sca_module_forward``,
+``msda_workspace_size``, ``sca_compact_workspace_size``.
 """
 import ctypes
 import os
@@ -33,8 +33,17 @@ class Dims(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("B", "Ncam", "Nq", "Nv", "H", "L", "P", "R")]
 
 
-_lib = None
 _vp = ctypes.c_void_p
+
+
+class ScaModuleParams(ctypes.Structure):
+    _fields_ = [("query", _vp), ("query_pos", _vp), ("features", _vp), ("w_value", _vp),
+                ("b_value", _vp), ("w_offsets", _vp), ("b_offsets", _vp), ("w_weights", _vp),
+                ("b_weights", _vp), ("w_output", _vp), ("b_output", _vp),
+                ("reference_points_cam", _vp), ("bev_mask", _vp), ("value_dtype", ctypes.c_int)]
+
+
+_lib = None
 _i64p = ctypes.POINTER(ctypes.c_int64)
 
 
@@ -72,6 +81,22 @@ def lib():
                                   ctypes.c_int32, st, _vp, _vp]
         L.msda_linear.restype = ctypes.c_int
         L.msda_linear_timeouts.restype = ctypes.c_uint32
+        L.sca_module_workspace_size.argtypes = [Dims, ctypes.c_int]
+        L.sca_module_workspace_size.restype = ctypes.c_size_t
+        L.sca_module_forward.argtypes = [ctypes.POINTER(ScaModuleParams), _i64p, _i64p, Dims, _vp,
+                                         ctypes.c_size_t, _vp, _vp]
+        L.sca_module_forward.restype = ctypes.c_int
+        L.sca_backward_inputs.argtypes = [_i64p, _i64p, _vp, _vp, _vp, _vp, Dims, _vp, _vp, _vp,
+                                          _vp]
+        L.sca_backward_inputs.restype = ctypes.c_int
+        i32, f64 = ctypes.c_int32, ctypes.c_double
+        L.tsa_reference_points.argtypes = [_vp, i32, i32, i32, i32, f64, f64, _vp, _vp]
+        L.tsa_reference_points.restype = ctypes.c_int
+        L.tsa_forward.argtypes = [_vp, st, _i64p, _i64p, _vp, _vp, _vp, i32, Dims, _vp, _vp]
+        L.tsa_forward.restype = ctypes.c_int
+        L.sca_forward_query_major.argtypes = [_vp, st, _i64p, _i64p, _vp, _vp, _vp, _vp, Dims,
+                                              _vp, _vp]
+        L.sca_forward_query_major.restype = ctypes.c_int
         L.msda_status_string.argtypes = [ctypes.c_int]
         L.msda_status_string.restype = ctypes.c_char_p
         L.msda_last_error.restype = ctypes.c_char_p
@@ -173,6 +198,49 @@ def msda_forward_fused(value, spatial_shapes, level_start_index, reference_point
     return out
 
 
+def tsa_reference_points(ego_motion, bev_h, bev_w, grid_length=(0.512, 0.512), out=None,
+                         stream=None):
+    """ego_motion [B, T, 3] fp32 (dx m, dy m, yaw degrees) on the device ->
+    reference points [B, T, bev_h * bev_w, 2] fp32; grid_length = (gy, gx)."""
+    torch = _torch()
+    _contig(ego_motion, out)
+    B, T, _ = ego_motion.shape
+    if out is None:
+        out = torch.empty((B, T, bev_h * bev_w, 2), device=ego_motion.device,
+                          dtype=torch.float32)
+    gy, gx = grid_length
+    _check(lib().tsa_reference_points(_ptr(ego_motion), B, T, bev_h, bev_w, float(gy), float(gx),
+                                      _ptr(out), _stream(stream)),
+           "tsa_reference_points")
+    return out
+
+
+def tsa_forward(value, spatial_shapes, level_start_index, reference_points, sampling_offsets,
+                attention_logits, num_queues, out=None, stream=None):
+    """value [B*T, Nv, H, 32] (item b*T + t = queue t of sample b);
+    reference_points [B*T, Nq, R, 2]; offsets [B*T, Nq, H, L, P, 2];
+    logits [B*T, Nq, H, L, P] -> out [B, Nq, H*32] fp32, the mean over the
+    T = num_queues queues of the fused MSDA."""
+    torch = _torch()
+    _contig(value, reference_points, sampling_offsets, attention_logits, out)
+    BT, Nv, H, _ = value.shape
+    T = int(num_queues)
+    if T < 1 or BT % T:
+        raise MsdaError("tsa_forward: the value batch is not a multiple of num_queues")
+    _, Nq, _, L, P, _ = sampling_offsets.shape
+    R = reference_points.shape[2]
+    shapes, starts = _levels(spatial_shapes, level_start_index)
+    if out is None:
+        out = torch.empty((BT // T, Nq, H * HEAD_DIM), device=value.device, dtype=torch.float32)
+    d = Dims(BT // T, 1, Nq, Nv, H, L, P, R)
+    _check(lib().tsa_forward(_ptr(value), _vdt(value), shapes.ctypes.data_as(_i64p),
+                             starts.ctypes.data_as(_i64p), _ptr(reference_points),
+                             _ptr(sampling_offsets), _ptr(attention_logits), T, d, _ptr(out),
+                             _stream(stream)),
+           "tsa_forward")
+    return out
+
+
 def msda_backward(value, spatial_shapes, level_start_index, sampling_locations,
                   attention_weights, grad_out, grad_value=None, grad_sampling_locations=None,
                   grad_attention_weights=None, stream=None):
@@ -265,6 +333,25 @@ def sca_forward(value, spatial_shapes, level_start_index, reference_points_cam, 
                              _ptr(bev_mask), _ptr(sampling_offsets), _ptr(attention_logits), d,
                              _ptr(workspace), workspace.numel(), _ptr(out), _stream(stream)),
            "sca_forward")
+    return out
+
+
+def sca_forward_query_major(value, spatial_shapes, level_start_index, reference_points_cam,
+                            bev_mask, sampling_offsets, attention_logits, out=None, stream=None):
+    """sca_forward's result from one query-major kernel, without workspace."""
+    torch = _torch()
+    _contig(value, reference_points_cam, bev_mask, sampling_offsets, attention_logits, out)
+    if bev_mask.dtype == torch.bool:
+        bev_mask = bev_mask.view(torch.uint8)
+    d = _sca_dims(value, sampling_offsets, reference_points_cam)
+    shapes, starts = _levels(spatial_shapes, level_start_index)
+    if out is None:
+        out = torch.empty((d.B, d.Nq, d.H * HEAD_DIM), device=value.device, dtype=torch.float32)
+    _check(lib().sca_forward_query_major(_ptr(value), _vdt(value), shapes.ctypes.data_as(_i64p),
+                                         starts.ctypes.data_as(_i64p), _ptr(reference_points_cam),
+                                         _ptr(bev_mask), _ptr(sampling_offsets),
+                                         _ptr(attention_logits), d, _ptr(out), _stream(stream)),
+           "sca_forward_query_major")
     return out
 
 
@@ -381,3 +468,70 @@ def msda_linear(x, w, bias=None, residual=None, out=None, out_dtype=None, stream
                              _ptr(out), _stream(stream)),
            "msda_linear")
     return out
+
+
+def sca_module_forward(query, query_pos, features, w_value, b_value, w_offsets, b_offsets,
+                       w_weights, b_weights, w_output, b_output, reference_points_cam, bev_mask,
+                       spatial_shapes, level_start_index, num_levels, num_points,
+                       value_dtype=None, out=None, workspace=None, stream=None):
+    """The SCA module forward: q_hat = q + output_proj(SCA(value_proj(F~),
+    offsets(q + pos), weights(q + pos))).  query, query_pos [B, Nq, C] fp32;
+    features [B, Ncam, Nv, C] bf16; weights bf16 [out, in]; biases fp32;
+    reference_points_cam [Ncam, B, Nq, R, 2]; bev_mask [Ncam, B, Nq, R]
+    -> q_hat [B, Nq, C] fp32."""
+    torch = _torch()
+    _contig(query, query_pos, features, w_value, w_offsets, w_weights, w_output,
+            reference_points_cam, bev_mask)
+    if bev_mask.dtype == torch.bool:
+        bev_mask = bev_mask.view(torch.uint8)
+    B, Nq, C = query.shape
+    _, Ncam, Nv, _ = features.shape
+    H = C // HEAD_DIM
+    R = reference_points_cam.shape[3]
+    vdt = MSDA_BF16 if value_dtype == torch.bfloat16 else MSDA_F32
+    d = Dims(B, Ncam, Nq, Nv, H, num_levels, num_points, R)
+    shapes, starts = _levels(spatial_shapes, level_start_index)
+    if out is None:
+        out = torch.empty((B, Nq, C), device=query.device, dtype=torch.float32)
+    nbytes = int(lib().sca_module_workspace_size(d, vdt))
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=query.device)
+    prm = ScaModuleParams(*[_ptr(t) for t in (query, query_pos, features, w_value, b_value,
+                                              w_offsets, b_offsets, w_weights, b_weights,
+                                              w_output, b_output, reference_points_cam,
+                                              bev_mask)], vdt)
+    _check(lib().sca_module_forward(ctypes.byref(prm), shapes.ctypes.data_as(_i64p),
+                                    starts.ctypes.data_as(_i64p), d, _ptr(workspace),
+                                    workspace.numel(), _ptr(out), _stream(stream)),
+           "sca_module_forward")
+    return out
+
+
+def sca_backward_inputs(spatial_shapes, level_start_index, attention_logits, pos,
+                        grad_sampling_locations_rb, grad_attention_weights_rb, num_cameras,
+                        num_anchors, out=None, stream=None):
+    """-> (grad_sampling_offsets [B, Nq, H, L, P, 2], grad_attention_logits
+    [B, Nq, H, L, P], grad_reference_points_cam [Ncam, B, Nq, R, 2]); `out`
+    may supply the three tensors."""
+    torch = _torch()
+    _contig(attention_logits, pos, grad_sampling_locations_rb, grad_attention_weights_rb)
+    B, Nq, H, L, P = attention_logits.shape
+    Ncam, R = num_cameras, num_anchors
+    shapes, starts = _levels(spatial_shapes, level_start_index)
+    nv = int(np.max(starts + shapes[:, 0] * shapes[:, 1]))  # value rows the levels span
+    d = Dims(B, Ncam, Nq, nv, H, L, P, R)
+    dev = attention_logits.device
+    if out is not None:
+        g_off, g_lg, g_ref = out
+        _contig(g_off, g_lg, g_ref)
+    else:
+        g_off = torch.empty((B, Nq, H, L, P, 2), device=dev, dtype=torch.float32)
+        g_lg = torch.empty((B, Nq, H, L, P), device=dev, dtype=torch.float32)
+        g_ref = torch.empty((Ncam, B, Nq, R, 2), device=dev, dtype=torch.float32)
+    _check(lib().sca_backward_inputs(shapes.ctypes.data_as(_i64p), starts.ctypes.data_as(_i64p),
+                                     _ptr(attention_logits), _ptr(pos),
+                                     _ptr(grad_sampling_locations_rb),
+                                     _ptr(grad_attention_weights_rb), d, _ptr(g_off), _ptr(g_lg),
+                                     _ptr(g_ref), _stream(stream)),
+           "sca_backward_inputs")
+    return g_off, g_lg, g_ref

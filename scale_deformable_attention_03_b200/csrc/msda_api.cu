@@ -260,6 +260,53 @@ msda_status_t msda_forward_fused(const void* value, msda_dtype_t vdt,
                        "msda_forward_fused");
 }
 
+msda_status_t tsa_reference_points(const float* ego_motion, int32_t B, int32_t num_queues,
+                                   int32_t bev_h, int32_t bev_w, double grid_length_y,
+                                   double grid_length_x, float* reference_points,
+                                   msda_stream_t stream)
+{
+    MSDA_CHECK(B >= 0 && num_queues >= 1, MSDA_ERR_INVALID_ARG,
+               "B (%d) must be >= 0 and num_queues (%d) >= 1", B, num_queues);
+    MSDA_CHECK(bev_h >= 1 && bev_w >= 1 && (int64_t)bev_h * bev_w <= INT32_MAX,
+               MSDA_ERR_INVALID_ARG, "BEV grid %d x %d is empty or too large", bev_h, bev_w);
+    MSDA_CHECK(grid_length_y > 0.0 && grid_length_x > 0.0 && grid_length_y < 1e30 &&
+                   grid_length_x < 1e30,
+               MSDA_ERR_INVALID_ARG, "grid lengths (%g, %g) must be finite and > 0",
+               grid_length_y, grid_length_x);
+    if (B == 0) return ok();
+    MSDA_PTR(ego_motion, 4);
+    MSDA_PTR(reference_points, 8);
+    return cuda_status(msda::launch_tsa_reference(ego_motion, B, num_queues, bev_h, bev_w,
+                                                  grid_length_x, grid_length_y, reference_points,
+                                                  (cudaStream_t)stream),
+                       "tsa_reference_points");
+}
+
+msda_status_t tsa_forward(const void* value, msda_dtype_t vdt, const int64_t* spatial_shapes,
+                          const int64_t* level_start_index, const float* reference_points,
+                          const float* sampling_offsets, const float* attention_logits,
+                          int32_t num_queues, msda_dims_t d, float* out, msda_stream_t stream)
+{
+    MSDA_TRY(check_dims(d, false));
+    MSDA_CHECK(num_queues >= 1 && num_queues <= MSDA_MAX_QUEUES, MSDA_ERR_UNSUPPORTED,
+               "num_queues = %d outside 1..%d", num_queues, MSDA_MAX_QUEUES);
+    MSDA_CHECK((int64_t)d.B * num_queues <= INT32_MAX, MSDA_ERR_UNSUPPORTED,
+               "B * num_queues exceeds the 32-bit range");
+    msda::Levels lv;
+    MSDA_TRY(check_levels(d, spatial_shapes, level_start_index, lv));
+    MSDA_TRY(check_dtype(vdt));
+    if ((int64_t)d.B * d.Nq == 0) return ok();
+    MSDA_TRY(check_value(value));
+    MSDA_PTR(reference_points, 8);
+    MSDA_PTR(sampling_offsets, 8);
+    MSDA_PTR(attention_logits, 4);
+    MSDA_PTR(out, 16);
+    const msda::Problem p = make_problem(value, vdt, d, lv);
+    return cuda_status(msda::launch_tsa_forward(p, num_queues, reference_points, sampling_offsets,
+                                                attention_logits, out, (cudaStream_t)stream),
+                       "tsa_forward");
+}
+
 msda_status_t msda_backward(const void* value, msda_dtype_t vdt, const int64_t* spatial_shapes,
                             const int64_t* level_start_index, const float* sampling_locations,
                             const float* attention_weights, const float* grad_out, msda_dims_t d,
@@ -429,6 +476,32 @@ msda_status_t sca_forward(const void* value, msda_dtype_t vdt, const int64_t* sp
     return cuda_status(e, "sca_forward");
 }
 
+msda_status_t sca_forward_query_major(const void* value, msda_dtype_t vdt,
+                                      const int64_t* spatial_shapes,
+                                      const int64_t* level_start_index,
+                                      const float* reference_points_cam, const uint8_t* bev_mask,
+                                      const float* sampling_offsets,
+                                      const float* attention_logits, msda_dims_t d, float* out,
+                                      msda_stream_t stream)
+{
+    MSDA_TRY(check_dims(d, true));
+    msda::Levels lv;
+    MSDA_TRY(check_levels(d, spatial_shapes, level_start_index, lv));
+    MSDA_TRY(check_dtype(vdt));
+    if ((int64_t)d.B * d.Nq == 0) return ok();
+    MSDA_TRY(check_value(value));
+    MSDA_PTR(reference_points_cam, 8);
+    MSDA_PTR(bev_mask, 1);
+    MSDA_PTR(sampling_offsets, 8);
+    MSDA_PTR(attention_logits, 4);
+    MSDA_PTR(out, 16);
+    const msda::Problem p = make_problem(value, vdt, d, lv);
+    return cuda_status(msda::launch_sca_query_major(p, reference_points_cam, bev_mask,
+                                                    sampling_offsets, attention_logits, out,
+                                                    (cudaStream_t)stream),
+                       "sca_forward_query_major");
+}
+
 msda_status_t sca_rebatched_backward(const void* value, msda_dtype_t vdt,
                                      const int64_t* spatial_shapes,
                                      const int64_t* level_start_index,
@@ -497,6 +570,36 @@ msda_status_t sca_backward(const void* value, msda_dtype_t vdt, const int64_t* s
 }
 
 }  // extern "C"
+
+extern "C" msda_status_t sca_backward_inputs(const int64_t* spatial_shapes,
+                                             const int64_t* level_start_index,
+                                             const float* attention_logits, const int32_t* pos,
+                                             const float* grad_sampling_locations_rb,
+                                             const float* grad_attention_weights_rb,
+                                             msda_dims_t d, float* grad_sampling_offsets,
+                                             float* grad_attention_logits,
+                                             float* grad_reference_points_cam,
+                                             msda_stream_t stream)
+{
+    MSDA_TRY(check_dims(d, true));
+    MSDA_TRY(check_compact(d));
+    msda::Levels lv;
+    MSDA_TRY(check_levels(d, spatial_shapes, level_start_index, lv));
+    if ((int64_t)d.B * d.Nq == 0) return ok();
+    MSDA_PTR(attention_logits, 4);
+    MSDA_PTR(pos, 4);
+    MSDA_PTR(grad_sampling_locations_rb, 8);
+    MSDA_PTR(grad_attention_weights_rb, 4);
+    MSDA_PTR(grad_sampling_offsets, 8);
+    MSDA_PTR(grad_attention_logits, 4);
+    MSDA_PTR(grad_reference_points_cam, 4);
+    return cuda_status(msda::launch_sca_input_grads(
+                           attention_logits, pos, grad_sampling_locations_rb,
+                           grad_attention_weights_rb, d.B, d.Ncam, d.Nq, d.H, d.L, d.P, d.R, lv,
+                           grad_sampling_offsets, grad_attention_logits,
+                           grad_reference_points_cam, (cudaStream_t)stream),
+                       "sca_backward_inputs");
+}
 
 // Status helpers for entry points defined in other translation units (they
 // share this file's per-thread error message).

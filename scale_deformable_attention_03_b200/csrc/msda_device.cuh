@@ -260,6 +260,34 @@ struct Gather<float> {
             acc[3] += w.x * x0.w + w.y * x1.w + w.z * x2.w + w.w * x3.w;
         }
     }
+    // Q quads of the table from `base`, straight-line (entries past the
+    // row's samples hold offset -1 and read nothing).
+    template <int Q>
+    __device__ __forceinline__ static void run_quads(const float* __restrict__ vb,
+                                                     const WarpTable& tab, int lane,
+                                                     float (&acc)[4], int base)
+    {
+        const int g = lane >> 3, t = lane & 7;
+        const float* v = vb + 4 * t;
+#pragma unroll
+        for (int p = 0; p < Q; ++p) {
+            const int4 o = *reinterpret_cast<const int4*>(&tab.off[g][base + 4 * p]);
+            const float4 w = *reinterpret_cast<const float4*>(&tab.w[g][base + 4 * p]);
+            float4 x0 = make_float4(0.f, 0.f, 0.f, 0.f), x1 = x0, x2 = x0, x3 = x0;
+            if (o.x >= 0) x0 = __ldg(reinterpret_cast<const float4*>(v + o.x));
+            if (o.y >= 0) x1 = __ldg(reinterpret_cast<const float4*>(v + o.y));
+            if (o.z >= 0) x2 = __ldg(reinterpret_cast<const float4*>(v + o.z));
+            if (o.w >= 0) x3 = __ldg(reinterpret_cast<const float4*>(v + o.w));
+            acc[0] += w.x * x0.x + w.y * x1.x + w.z * x2.x + w.w * x3.x;
+            acc[1] += w.x * x0.y + w.y * x1.y + w.z * x2.y + w.w * x3.y;
+            acc[2] += w.x * x0.z + w.y * x1.z + w.z * x2.z + w.w * x3.z;
+            acc[3] += w.x * x0.w + w.y * x1.w + w.z * x2.w + w.w * x3.w;
+        }
+    }
+    // Lane bits over which the partial sums of one output are spread: the
+    // corner g (bits 4 and 3).  Channel quad t = lane & 7.
+    static constexpr int kSumMasks[2] = {16, 8};
+    __device__ __forceinline__ static int channel0(int lane) { return 4 * (lane & 7); }
     // Sum the four corners; lanes 0..7 store channels 4t..4t+3.
     __device__ __forceinline__ static void store(float (&acc)[4], int lane, float* __restrict__ out)
     {
@@ -313,6 +341,30 @@ struct Gather<__nv_bfloat16> {
             fma8(acc, wb, rb);
         }
     }
+    template <int Q>
+    __device__ __forceinline__ static void run_quads(const __nv_bfloat16* __restrict__ vb,
+                                                     const WarpTable& tab, int lane,
+                                                     float (&acc)[8], int base)
+    {
+        const int half = lane >> 4, g = (lane >> 2) & 3, t = lane & 3;
+        const __nv_bfloat16* v = vb + 8 * t;
+#pragma unroll
+        for (int p = 0; p < Q; ++p) {
+            const int4 o = *reinterpret_cast<const int4*>(&tab.off[g][base + 4 * p]);
+            const float4 w = *reinterpret_cast<const float4*>(&tab.w[g][base + 4 * p]);
+            const int oa = half ? o.y : o.x, ob = half ? o.w : o.z;
+            const float wa = half ? w.y : w.x, wb = half ? w.w : w.z;
+            uint4 ra = make_uint4(0u, 0u, 0u, 0u), rb = ra;
+            if (oa >= 0) ra = __ldg(reinterpret_cast<const uint4*>(v + oa));
+            if (ob >= 0) rb = __ldg(reinterpret_cast<const uint4*>(v + ob));
+            fma8(acc, wa, ra);
+            fma8(acc, wb, rb);
+        }
+    }
+    // Partial sums spread over the sample half (bit 4) and the corner (bits 3,
+    // 2); channel group t = lane & 3.
+    static constexpr int kSumMasks[3] = {16, 8, 4};
+    __device__ __forceinline__ static int channel0(int lane) { return 8 * (lane & 3); }
     // Sum corners and halves; lanes 0..3 store channels 8t..8t+7.
     __device__ __forceinline__ static void store(float (&acc)[8], int lane, float* __restrict__ out)
     {
@@ -329,6 +381,71 @@ struct Gather<__nv_bfloat16> {
         }
     }
 };
+
+// Several heads' partial sums at once (acc[s] = head s, partial over the
+// lanes named by Gather<VT>::kSumMasks).  A butterfly reduce-scatter: at each
+// lane bit, the lane keeps half of the heads it holds (the lower half if the
+// bit is clear) and adds its partner's copy of that half, so G heads cost
+// (G/2 + G/4 + ...) shuffles per element instead of G per bit.  Once a lane
+// holds one head, the remaining bits are plain butterfly sums.
+template <int HELD, int G, int NA>
+__device__ __forceinline__ void reduce_level(float (&acc)[G][NA], int mask, int lane,
+                                             int& head0, bool& writer)
+{
+    if constexpr (HELD > 1) {
+        const bool upper = (lane & mask) != 0;
+#pragma unroll
+        for (int i = 0; i < HELD / 2; ++i)
+#pragma unroll
+            for (int e = 0; e < NA; ++e) {
+                const float keep = upper ? acc[i + HELD / 2][e] : acc[i][e];
+                const float send = upper ? acc[i][e] : acc[i + HELD / 2][e];
+                acc[i][e] = keep + __shfl_xor_sync(0xffffffffu, send, mask);
+            }
+        if (upper) head0 += HELD / 2;
+    } else {
+#pragma unroll
+        for (int e = 0; e < NA; ++e) acc[0][e] += __shfl_xor_sync(0xffffffffu, acc[0][e], mask);
+        writer = writer && (lane & mask) == 0;
+    }
+}
+
+template <int G>
+__host__ __device__ constexpr int held_after(int levels)
+{
+    return (G >> levels) > 0 ? (G >> levels) : 1;
+}
+
+// Reduce G heads' partial sums and store heads 0 .. nheads - 1 of them, each
+// scaled by `scale`, to out_row0 + 32 s.
+template <typename VT, int G>
+__device__ __forceinline__ void store_heads(float (&acc)[G][Gather<VT>::kAcc], int lane,
+                                            float* __restrict__ out_row0, int nheads,
+                                            float scale = 1.f)
+{
+    constexpr int NA = Gather<VT>::kAcc;
+    constexpr int NM = sizeof(Gather<VT>::kSumMasks) / sizeof(int);
+    int head0 = 0;
+    bool writer = true;
+    reduce_level<held_after<G>(0), G, NA>(acc, Gather<VT>::kSumMasks[0], lane, head0, writer);
+    reduce_level<held_after<G>(1), G, NA>(acc, Gather<VT>::kSumMasks[1], lane, head0, writer);
+    if constexpr (NM > 2)
+        reduce_level<held_after<G>(2), G, NA>(acc, Gather<VT>::kSumMasks[2], lane, head0, writer);
+    constexpr int kHeld = held_after<G>(NM);
+    if (!writer) return;
+    const int c0 = Gather<VT>::channel0(lane);
+#pragma unroll
+    for (int i = 0; i < kHeld; ++i) {
+        const int s = head0 + i;
+        if (s < nheads) {
+            float4* o = reinterpret_cast<float4*>(out_row0 + s * kHeadDim + c0);
+#pragma unroll
+            for (int j = 0; j < NA / 4; ++j)
+                o[j] = make_float4(acc[i][4 * j] * scale, acc[i][4 * j + 1] * scale,
+                                   acc[i][4 * j + 2] * scale, acc[i][4 * j + 3] * scale);
+        }
+    }
+}
 
 // Inputs of one row for HP heads, per lane (samples j = c * 32 + lane): the
 // logits (or weights), the pixel offsets (or locations) and, fused, the
@@ -404,32 +521,54 @@ __device__ __forceinline__ void lane_corners(float2 v, float2 r, const LaneSampl
     }
 }
 
-// One output row of one head (all n = L*P samples) from its loaded inputs,
-// written to out_row[0..32).  vb: value of this batch item (and camera),
-// [Nv, H, 32].
+// One head of one row (all n = L*P samples) from its normalised weights a,
+// offsets (or locations) lo and reference points rf, added to the lane's
+// partial sums acc (corners not yet reduced: Gather::store does that).
+// vb: value of this batch item (and camera), [Nv, H, 32].
+template <typename VT, bool FUSED, int NC>
+__device__ __forceinline__ void head_gather(const VT* __restrict__ vb, int H, int h,
+                                            const float (&a)[NC], const float2 (&lo)[NC],
+                                            const float2 (&rf)[NC], int n,
+                                            const LaneSamples<NC>& ls, WarpTable& tab,
+                                            float (&acc)[Gather<VT>::kAcc], int lane)
+{
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+        Corners cr;
+        lane_corners<FUSED, NC>(lo[c], rf[c], ls, c, H, h, cr);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            tab.off[g][lane] = cr.off[g];
+            tab.w[g][lane] = cr.w[g] * a[c];
+        }
+        __syncwarp();
+        Gather<VT>::run(vb, tab, min(32, n - c * 32), lane, acc);
+        __syncwarp();
+    }
+}
+
+// head_gather after the softmax of the row's logits (in place).
+template <typename VT, bool FUSED, int NC>
+__device__ __forceinline__ void row_accumulate(const VT* __restrict__ vb, int H, int h,
+                                               RowIn<FUSED, NC, 1>& in, int n,
+                                               const LaneSamples<NC>& ls, WarpTable& tab,
+                                               float (&acc)[Gather<VT>::kAcc], int lane)
+{
+    normalise<FUSED, NC>(in.a[0], ls);
+    head_gather<VT, FUSED, NC>(vb, H, h, in.a[0], in.lo[0], in.rf, n, ls, tab, acc, lane);
+}
+
+// One output row of one head, written to out_row[0..32).
 template <typename VT, bool FUSED, int NC>
 __device__ __forceinline__ void row_compute(const VT* __restrict__ vb, int H, int h,
                                             RowIn<FUSED, NC, 1>& in, int n,
                                             const LaneSamples<NC>& ls, WarpTable& tab,
                                             float* __restrict__ out_row, int lane)
 {
-    normalise<FUSED, NC>(in.a[0], ls);
     float acc[Gather<VT>::kAcc];
 #pragma unroll
     for (int i = 0; i < Gather<VT>::kAcc; ++i) acc[i] = 0.f;
-#pragma unroll
-    for (int c = 0; c < NC; ++c) {
-        Corners cr;
-        lane_corners<FUSED, NC>(in.lo[0][c], in.rf[c], ls, c, H, h, cr);
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-            tab.off[g][lane] = cr.off[g];
-            tab.w[g][lane] = cr.w[g] * in.a[0][c];
-        }
-        __syncwarp();
-        Gather<VT>::run(vb, tab, min(32, n - c * 32), lane, acc);
-        __syncwarp();
-    }
+    row_accumulate<VT, FUSED, NC>(vb, H, h, in, n, ls, tab, acc, lane);
     Gather<VT>::store(acc, lane, out_row);
 }
 
@@ -444,19 +583,15 @@ struct PairTable {
     float w[2][4][kMetaStride];
 };
 
-// Heads h0 and h0 + 1 of one row; out_row0 is head h0's output, head h0 + 1
-// follows at +32.
+// Heads h0 and h0 + 1 of one row from normalised weights, added to the
+// lane's partial sums (see pair_store for the lane layout).
 template <bool FUSED, int NC>
-__device__ __forceinline__ void row_compute_pair(const __nv_bfloat16* __restrict__ vb, int H,
-                                                 int h0, RowIn<FUSED, NC, 2>& in, int n,
-                                                 const LaneSamples<NC>& ls, PairTable& tab,
-                                                 float* __restrict__ out_row0, int lane)
+__device__ __forceinline__ void pair_gather(const __nv_bfloat16* __restrict__ vb, int H, int h0,
+                                            const RowIn<FUSED, NC, 2>& in,
+                                            const float2 (&rf)[NC], int n,
+                                            const LaneSamples<NC>& ls, PairTable& tab,
+                                            float (&acc)[8], int lane)
 {
-    normalise<FUSED, NC>(in.a[0], ls);
-    normalise<FUSED, NC>(in.a[1], ls);
-    float acc[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
     const int half = lane >> 4, g = (lane >> 2) & 3, t = lane & 3;
     const __nv_bfloat16* v = vb + 8 * t;
 #pragma unroll
@@ -464,7 +599,7 @@ __device__ __forceinline__ void row_compute_pair(const __nv_bfloat16* __restrict
 #pragma unroll
         for (int sh = 0; sh < 2; ++sh) {
             Corners cr;
-            lane_corners<FUSED, NC>(in.lo[sh][c], in.rf[c], ls, c, H, h0 + sh, cr);
+            lane_corners<FUSED, NC>(in.lo[sh][c], rf[c], ls, c, H, h0 + sh, cr);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 tab.off[sh][q][lane] = cr.off[q];
@@ -489,7 +624,13 @@ __device__ __forceinline__ void row_compute_pair(const __nv_bfloat16* __restrict
         }
         __syncwarp();
     }
-    // sum the four corners; lanes 16s + t (g = 0) store head h0 + s, channels 8t..8t+7
+}
+
+// Sum the four corners; lanes 16s + t (g = 0) store head h0 + s, channels
+// 8t..8t+7; out_row0 is head h0's output, head h0 + 1 follows at +32.
+__device__ __forceinline__ void pair_store(float (&acc)[8], int lane, float* __restrict__ out_row0)
+{
+    const int half = lane >> 4, g = (lane >> 2) & 3, t = lane & 3;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 4);
@@ -500,6 +641,23 @@ __device__ __forceinline__ void row_compute_pair(const __nv_bfloat16* __restrict
         o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
         o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
     }
+}
+
+// Heads h0 and h0 + 1 of one row; out_row0 is head h0's output, head h0 + 1
+// follows at +32.
+template <bool FUSED, int NC>
+__device__ __forceinline__ void row_compute_pair(const __nv_bfloat16* __restrict__ vb, int H,
+                                                 int h0, RowIn<FUSED, NC, 2>& in, int n,
+                                                 const LaneSamples<NC>& ls, PairTable& tab,
+                                                 float* __restrict__ out_row0, int lane)
+{
+    normalise<FUSED, NC>(in.a[0], ls);
+    normalise<FUSED, NC>(in.a[1], ls);
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    pair_gather<FUSED, NC>(vb, H, h0, in, in.rf, n, ls, tab, acc, lane);
+    pair_store(acc, lane, out_row0);
 }
 
 // Rows with few samples (L*P <= 16): one warp serves G heads of a row at
@@ -542,15 +700,13 @@ __device__ __forceinline__ float segment_sum(float v, int npad)
     return v;
 }
 
-// One row, heads h0 .. h0 + G - 1 (those < H).  lo, wl: head h0 of the row
-// (the other heads follow at +2n, +n per head); ref: the row's reference
-// points; out_row0: head h0's output (+32 per head).  The lane's inputs come
-// preloaded in (a, v, r); `valid` = the lane's sample exists.
-template <typename VT, bool FUSED>
-__device__ __forceinline__ void group_compute(const VT* __restrict__ vb, int H, int h0, float a,
-                                              float2 v, float2 r, bool valid, int n,
-                                              const GroupLane& gl, WarpTable& tab,
-                                              float* __restrict__ out_row0, int lane)
+// The table of one row for heads h0 .. h0 + G - 1: softmax of each head's
+// segment, locations and corners.  The lane's inputs come preloaded in
+// (a, v, r); `valid` = the lane's sample exists.  The caller syncs the warp
+// before reading the table.
+template <bool FUSED>
+__device__ __forceinline__ void group_table(int H, int h0, float a, float2 v, float2 r, bool valid,
+                                            const GroupLane& gl, WarpTable& tab, int lane)
 {
     const int npad = 1 << gl.npad_log2;
     if (FUSED) {
@@ -581,16 +737,42 @@ __device__ __forceinline__ void group_compute(const VT* __restrict__ vb, int H, 
         tab.off[g][lane] = cr.off[g];
         tab.w[g][lane] = cr.w[g] * a;
     }
-    __syncwarp();
-    const int G = 32 >> gl.npad_log2;
-    for (int s = 0; s < G && h0 + s < H; ++s) {
-        float acc[Gather<VT>::kAcc];
+}
+
+// The gathers of heads h0 .. h0 + G - 1 (the first nheads of them) from a
+// filled group table, added to acc[s]; NPL = log2(npad), G = 32 >> NPL.  All
+// heads' loads are straight-line code, so they are in flight together.
+template <typename VT, int NPL>
+__device__ __forceinline__ void group_gather(const VT* __restrict__ vb, const WarpTable& tab,
+                                             int nheads, int lane,
+                                             float (&acc)[32 >> NPL][Gather<VT>::kAcc])
+{
+    constexpr int G = 32 >> NPL, Q = (1 << NPL) / 4;
 #pragma unroll
-        for (int i = 0; i < Gather<VT>::kAcc; ++i) acc[i] = 0.f;
-        Gather<VT>::run(vb, tab, n, lane, acc, s << gl.npad_log2);
-        Gather<VT>::store(acc, lane, out_row0 + s * kHeadDim);
-    }
+    for (int s = 0; s < G; ++s)
+        if (s < nheads) Gather<VT>::template run_quads<Q>(vb, tab, lane, acc[s], s << NPL);
+}
+
+// One row, heads h0 .. h0 + G - 1 (those < H), from the lane's preloaded
+// inputs (see group_table); out_row0: head h0's output (+32 per head).
+template <typename VT, bool FUSED, int NPL>
+__device__ __forceinline__ void group_compute(const VT* __restrict__ vb, int H, int h0, float a,
+                                              float2 v, float2 r, bool valid,
+                                              const GroupLane& gl, WarpTable& tab,
+                                              float* __restrict__ out_row0, int lane)
+{
+    constexpr int G = 32 >> NPL;
+    group_table<FUSED>(H, h0, a, v, r, valid, gl, tab, lane);
     __syncwarp();
+    float acc[G][Gather<VT>::kAcc];
+#pragma unroll
+    for (int s = 0; s < G; ++s)
+#pragma unroll
+        for (int i = 0; i < Gather<VT>::kAcc; ++i) acc[s][i] = 0.f;
+    const int nheads = min(G, H - h0);
+    group_gather<VT, NPL>(vb, tab, nheads, lane, acc);
+    __syncwarp();
+    store_heads<VT, G>(acc, lane, out_row0, nheads);
 }
 
 // Walks the (row, head) items of one warp without divisions: items are

@@ -88,13 +88,14 @@ msda_forward_kernel(const VT* __restrict__ value, const float* __restrict__ lo,
 
 // K1g: rows with L*P <= 16, G = 32 / npad heads per warp item (see
 // group_compute).  Items are (row, head group), head groups fastest.
-template <typename VT, bool FUSED>
+template <typename VT, bool FUSED, int NPL>
 __global__ void MSDA_GATHER_BOUNDS
 msda_forward_group_kernel(const VT* __restrict__ value, const float* __restrict__ lo,
                           const float* __restrict__ wl, const float* __restrict__ ref,
                           float* __restrict__ out, int B, int Nq, int Nv, int H, int L, int P,
-                          int R, int npad_log2, Levels levels)
+                          int R, Levels levels)
 {
+    constexpr int npad_log2 = NPL;
     __shared__ SmemLevels s_lv;
     __shared__ __align__(16) WarpTable s_tab[kWarps];
     stage_levels(s_lv, levels);
@@ -154,8 +155,8 @@ msda_forward_group_kernel(const VT* __restrict__ value, const float* __restrict_
         const Item x1 = resolve(it + kWarps, nx);
         if (x1.ok) fetch(x1, in1);
         const VT* vb = value + (int64_t)x0.b * Nv * H * kHeadDim;
-        group_compute<VT, FUSED>(vb, H, x0.h0, in0.a, in0.v, in0.r, x0.valid, S, gl, s_tab[warp],
-                                 out + (x0.bq * H + x0.h0) * kHeadDim, lane);
+        group_compute<VT, FUSED, NPL>(vb, H, x0.h0, in0.a, in0.v, in0.r, x0.valid, gl,
+                                      s_tab[warp], out + (x0.bq * H + x0.h0) * kHeadDim, lane);
         x0 = x1;
         in0 = in1;
         cur = nx;
@@ -173,9 +174,19 @@ static cudaError_t launch_group(const Problem& p, const float* lo, const float* 
     int npad_log2 = 2;
     while ((1 << npad_log2) < S) ++npad_log2;
     const unsigned grid = (unsigned)((rows + kRowsPerTile - 1) / kRowsPerTile);
-    msda_forward_group_kernel<VT, FUSED><<<grid, kThreads, 0, s>>>(
-        static_cast<const VT*>(p.value), lo, wl, ref, out, p.B, p.Nq, p.Nv, p.H, p.L, p.P, p.R,
-        npad_log2, p.lv);
+    const VT* v = static_cast<const VT*>(p.value);
+    switch (npad_log2) {
+#define MSDA_GROUP_CASE(NPLV)                                                                    \
+    case NPLV:                                                                                   \
+        msda_forward_group_kernel<VT, FUSED, NPLV><<<grid, kThreads, 0, s>>>(                    \
+            v, lo, wl, ref, out, p.B, p.Nq, p.Nv, p.H, p.L, p.P, p.R, p.lv);                     \
+        break;
+        MSDA_GROUP_CASE(2)
+        MSDA_GROUP_CASE(3)
+        MSDA_GROUP_CASE(4)
+#undef MSDA_GROUP_CASE
+        default: return cudaErrorInvalidValue;
+    }
     return cudaGetLastError();
 }
 

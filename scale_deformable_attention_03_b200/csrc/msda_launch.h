@@ -56,6 +56,11 @@ cudaError_t launch_sca_gather(const Problem& p, const float* ref_cam, const floa
                               const float* logits, const int32_t* idx, const int32_t* count,
                               float* out_rb, cudaStream_t s);
 
+// K3q: the whole SCA forward, query-major (no compaction, no rebatched rows).
+cudaError_t launch_sca_query_major(const Problem& p, const float* ref_cam, const uint8_t* mask,
+                                   const float* off, const float* logits, float* out,
+                                   cudaStream_t s);
+
 // K4: deterministic camera average.
 cudaError_t launch_sca_average(const float* out_rb, const int32_t* pos, const int32_t* hits,
                                int B, int Ncam, int Nq, int H, float* out, cudaStream_t s);
@@ -78,6 +83,19 @@ cudaError_t launch_sca_zero_tail(const int32_t* count, int B, int Ncam, int Nq, 
 #include "msda.h"
 
 namespace msda {
+// Gradients of offsets, logits and reference points (sca_input_grads.cu).
+cudaError_t launch_sca_input_grads(const float* logits, const int32_t* pos,
+                                   const float* grad_loc_rb, const float* grad_attn_rb, int B,
+                                   int Ncam, int Nq, int H, int L, int P, int R, const Levels& lv,
+                                   float* grad_off, float* grad_logits, float* grad_ref_cam,
+                                   cudaStream_t s);
+
+// TSA (tsa.cu): ego-motion reference points and the queue-mean fused forward.
+cudaError_t launch_tsa_reference(const float* ego, int B, int T, int bev_h, int bev_w, double gx,
+                                 double gy, float* ref, cudaStream_t s);
+cudaError_t launch_tsa_forward(const Problem& p, int T, const float* ref, const float* off,
+                               const float* logits, float* out, cudaStream_t s);
+
 // Set the per-thread error message of msda_last_error() and return the code.
 msda_status_t api_fail(msda_status_t code, const char* message);
 msda_status_t api_ok();

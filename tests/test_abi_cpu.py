@@ -36,6 +36,7 @@ def test_header_declares_the_boundary():
               "sca_compact_workspace_size", "sca_compact", "sca_forward", "sca_backward",
               "sca_rebatched_forward", "sca_camera_average", "sca_rebatched_backward",
               "sca_compact_no_alloc", "msda_linear", "msda_linear_timeouts",
+              "sca_module_forward", "sca_backward_inputs", "tsa_reference_points", "tsa_forward", "sca_forward_query_major",
               "msda_status_string", "msda_last_error", "msda_version"):
         assert n in names
 
@@ -179,3 +180,42 @@ def test_linear_rejects_unsupported_shapes(L):
     assert f(FAKE, FAKE, FAKE + 4, None, 128, 256, 256, 0, FAKE, None) == INVALID   # bias
     assert f(FAKE, FAKE, None, None, 128, 256, 256, 9, FAKE, None) == INVALID       # dtype
     assert f(0, 0, None, None, 0, 256, 256, 0, 0, None) == OK                        # empty
+
+
+def test_tsa_reference_points_rejects_bad_arguments(L):
+    f = L.tsa_reference_points
+    assert f(FAKE, -1, 2, 200, 200, 0.512, 0.512, FAKE, None) == INVALID      # B
+    assert f(FAKE, 1, 0, 200, 200, 0.512, 0.512, FAKE, None) == INVALID       # queues
+    assert f(FAKE, 1, 2, 0, 200, 0.512, 0.512, FAKE, None) == INVALID         # empty grid
+    assert f(FAKE, 1, 2, 200, 200, 0.0, 0.512, FAKE, None) == INVALID         # grid length
+    assert f(FAKE, 1, 2, 200, 200, 0.512, float("nan"), FAKE, None) == INVALID
+    assert f(FAKE, 1, 2, 200, 200, 0.512, 0.512, FAKE + 4, None) == INVALID   # alignment
+    assert f(0, 1, 2, 200, 200, 0.512, 0.512, FAKE, None) == INVALID          # null
+    assert f(0, 0, 2, 200, 200, 0.512, 0.512, 0, None) == OK                  # empty batch
+
+
+def test_tsa_forward_rejects_bad_arguments(L):
+    s, st = _levels(((4, 4),))
+    p = ctypes.POINTER(ctypes.c_int64)
+    call = lambda T, d, out=FAKE: L.tsa_forward(  # noqa: E731
+        FAKE, 0, s.ctypes.data_as(p), st.ctypes.data_as(p), FAKE, FAKE, FAKE, T, d, out, None)
+    assert call(0, msda.Dims(*GOOD)) == UNSUPPORTED
+    assert call(5, msda.Dims(*GOOD)) == UNSUPPORTED
+    assert call(2, msda.Dims(*GOOD), FAKE + 4) == INVALID
+    assert call(2, msda.Dims(*GOOD), 0) == INVALID
+    empty = list(GOOD)
+    empty[0] = 0
+    assert call(2, msda.Dims(*empty), 0) == OK
+
+
+def test_sca_query_major_rejects_bad_arguments(L):
+    s, st = _levels(((4, 4),))
+    p = ctypes.POINTER(ctypes.c_int64)
+    call = lambda d, out=FAKE, mask=FAKE: L.sca_forward_query_major(  # noqa: E731
+        FAKE, 0, s.ctypes.data_as(p), st.ctypes.data_as(p), FAKE, mask, FAKE, FAKE, d, out, None)
+    assert call(msda.Dims(1, 33, 8, 16, 2, 1, 4, 1)) == UNSUPPORTED   # Ncam > 32
+    assert call(msda.Dims(1, 0, 8, 16, 2, 1, 4, 1)) == UNSUPPORTED    # no camera
+    assert call(msda.Dims(1, 6, 8, 16, 2, 1, 4, 1), out=0) == INVALID
+    assert call(msda.Dims(1, 6, 8, 16, 2, 1, 4, 1), mask=0) == INVALID
+    assert call(msda.Dims(1, 6, 8, 16, 2, 1, 4, 1), out=FAKE + 8) == INVALID
+    assert call(msda.Dims(1, 6, 0, 16, 2, 1, 4, 1), out=0) == OK       # nothing to do

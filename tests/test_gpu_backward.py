@@ -111,3 +111,51 @@ def test_workload5_training_step_full_size():
     assert_close(gw, rw, True, "workload 5 grad_attention_weights_rb")
     assert_close(gl, rl, True, "workload 5 grad_sampling_locations_rb")
     assert_close(gv, rv, True, "workload 5 grad_value")
+
+
+@pytest.mark.parametrize("seed,B,Ncam,bev,shapes,H,P,R", [
+    (41, 2, 3, (7, 9), [(9, 13), (4, 7)], 2, 4, 2),
+    (42, 1, 6, (30, 40), [(16, 20), (8, 10), (4, 5), (2, 3)], 8, 8, 4),
+    (43, 2, 2, (5, 13), [(6, 7)] * 3, 1, 12, 3),
+])
+def test_sca_backward_inputs(seed, B, Ncam, bev, shapes, H, P, R):
+    """Offsets, logits and reference-point gradients from the rebatched ones,
+    against the oracle's chain rule (itself pinned by finite differences)."""
+    w = inputs.workload3(seed=seed, B=B, Ncam=Ncam, bev_h=bev[0], bev_w=bev[1], shapes=shapes,
+                         H=H, P=P, R=R, rho="uniform", same_mask=False, with_grad=True)
+    mask = dev(w.bev_mask)
+    idx, count, pos, hits = msda.sca_compact(mask)
+    args = (dev(w.value), w.spatial_shapes, w.level_start_index, dev(w.reference_points),
+            dev(w.sampling_offsets), dev(w.attention_logits), dev(w.grad_out), idx, count, hits)
+    gv, gl, gw = msda.sca_rebatched_backward(*args)
+    g_off, g_lg, g_ref = msda.sca_backward_inputs(w.spatial_shapes, w.level_start_index,
+                                                  dev(w.attention_logits), pos, gl, gw, Ncam, R)
+    torch.cuda.synchronize()
+    _, rl, rw = oracle.sca_backward(w.value, w.spatial_shapes, w.level_start_index,
+                                    w.reference_points, w.bev_mask, w.sampling_offsets,
+                                    w.attention_logits, w.grad_out)
+    r_off, r_lg, r_ref = oracle.sca_backward_inputs(w.spatial_shapes, w.bev_mask,
+                                                    w.attention_logits, rl, rw)
+    assert_close(g_off, r_off, False, "grad_sampling_offsets")
+    assert_close(g_lg, r_lg, False, "grad_attention_logits")
+    assert_close(g_ref, r_ref, False, "grad_reference_points_cam")
+
+
+def test_sca_backward_inputs_workload5():
+    w = inputs.workload5()
+    mask = dev(w.bev_mask)
+    idx, count, pos, hits = msda.sca_compact(mask)
+    gv, gl, gw = msda.sca_rebatched_backward(
+        value_tensor(w, True), w.spatial_shapes, w.level_start_index, dev(w.reference_points),
+        dev(w.sampling_offsets), dev(w.attention_logits), dev(w.grad_out), idx, count, hits)
+    g_off, g_lg, g_ref = msda.sca_backward_inputs(w.spatial_shapes, w.level_start_index,
+                                                  dev(w.attention_logits), pos, gl, gw, w.Ncam, w.R)
+    torch.cuda.synchronize()
+    _, rl, rw = oracle.sca_backward(w.value, w.spatial_shapes, w.level_start_index,
+                                    w.reference_points, w.bev_mask, w.sampling_offsets,
+                                    w.attention_logits, w.grad_out)
+    r_off, r_lg, r_ref = oracle.sca_backward_inputs(w.spatial_shapes, w.bev_mask,
+                                                    w.attention_logits, rl, rw)
+    assert_close(g_off, r_off, True, "workload 5 grad_sampling_offsets")
+    assert_close(g_lg, r_lg, True, "workload 5 grad_attention_logits")
+    assert_close(g_ref, r_ref, True, "workload 5 grad_reference_points_cam")
