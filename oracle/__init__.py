@@ -48,11 +48,15 @@ def lib():
                                                   ctypes.c_double, _D, _D]
         L.oracle_tsa_forward.argtypes = [_D, _i, _i, _i, _i, _i, _i, _I64, _I64, _i, _i, _i, _D,
                                          _D, _D, _i, _D]
+        _U32 = ctypes.POINTER(ctypes.c_uint32)
+        L.oracle_philox4x32_10.argtypes = [_U32, _U32, _U32]
+        L.oracle_philox4x32_10.restype = None
+        L.oracle_dropout.argtypes = [_D, ctypes.c_int64, ctypes.c_double, ctypes.c_uint64, _D]
         for f in ("oracle_softmax", "oracle_msda_forward", "oracle_msda_forward_fused",
                   "oracle_fused_locations", "oracle_msda_backward", "oracle_sca_compact",
                   "oracle_sca_forward", "oracle_sca_backward", "oracle_linear",
                   "oracle_sca_backward_inputs", "oracle_tsa_reference_points",
-                  "oracle_tsa_forward"):
+                  "oracle_tsa_forward", "oracle_dropout"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -239,10 +243,11 @@ def round_bf16(a):
 def sca_module_forward(query, query_pos, features, w_value, b_value, w_offsets, b_offsets,
                        w_weights, b_weights, w_output, b_output, reference_points_cam, bev_mask,
                        spatial_shapes, level_start_index, num_levels, num_points,
-                       value_bf16=False):
+                       value_bf16=False, dropout_p=0.0, dropout_seed=0):
     """The SCA module forward ([BQ] 3, 4, 10-13), composed of the oracle's
     projection and SCA: q~ = bf16(q + pos); V = F~ W_v^T + b_v; Delta, a from
-    q~; g = SCA; q_hat = q + bf16(g) W_o^T + b_o.  features [B, Ncam, Nv, C]."""
+    q~; g = SCA; q_hat = q + dropout(bf16(g) W_o^T + b_o).  features
+    [B, Ncam, Nv, C]; dropout_p = 0 is the inference identity."""
     q = _d(query)
     B, Nq, C = q.shape
     _, Ncam, Nv, _ = features.shape
@@ -255,7 +260,8 @@ def sca_module_forward(query, query_pos, features, w_value, b_value, w_offsets, 
     lg = linear(qt, w_weights, b_weights).reshape(B, Nq, H, L, P)
     g = sca_forward(V.reshape(B, Ncam, Nv, H, 32), spatial_shapes, level_start_index,
                     reference_points_cam, bev_mask, off, lg)
-    y = linear(round_bf16(g).reshape(B * Nq, C), w_output, b_output, q.reshape(B * Nq, C))
+    o = linear(round_bf16(g).reshape(B * Nq, C), w_output, b_output)
+    y = q.reshape(B * Nq, C) + (dropout(o, dropout_p, dropout_seed) if dropout_p > 0 else o)
     return y.reshape(B, Nq, C)
 
 
@@ -309,4 +315,22 @@ def tsa_forward(value, spatial_shapes, level_start_index, reference_points, samp
                                   _p(starts, _I64), Nq, P, R, _p(ref, _D), _p(off, _D),
                                   _p(lg, _D), int(coord_f32), _p(out, _D))
     _check(rc, "tsa_forward")
+    return out
+
+
+def philox4x32_10(counter, key):
+    """The four 32-bit output words of Philox4x32-10 (Salmon et al., SC 2011)."""
+    c = np.ascontiguousarray(counter, dtype=np.uint32)
+    k = np.ascontiguousarray(key, dtype=np.uint32)
+    out = np.empty(4, dtype=np.uint32)
+    u32 = ctypes.POINTER(ctypes.c_uint32)
+    lib().oracle_philox4x32_10(_p(c, u32), _p(k, u32), _p(out, u32))
+    return out
+
+
+def dropout(o, p, seed):
+    """Training-time dropout of o (any shape, row-major element order)."""
+    a = _d(o)
+    out = np.empty_like(a)
+    _check(lib().oracle_dropout(_p(a, _D), a.size, float(p), int(seed), _p(out, _D)), "dropout")
     return out

@@ -624,3 +624,46 @@ int oracle_tsa_forward(const double* value, int B, int T, int Nv, int H, int Dh,
     free(per_queue);
     return rc;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Dropout on the module's update branch ([BQ] 12, training time), with the */
+/* counter-based generator Philox4x32-10 (Salmon, Moraes, Dror, Shaw,       */
+/* "Parallel random numbers: as easy as 1, 2, 3", SC 2011)                 */
+/* ------------------------------------------------------------------------ */
+
+void oracle_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4])
+{
+    uint32_t c0 = ctr[0], c1 = ctr[1], c2 = ctr[2], c3 = ctr[3];
+    uint32_t k0 = key[0], k1 = key[1];
+    for (int round = 0; round < 10; ++round) {
+        /* one Philox S-box round: two 32x32 -> 64-bit products */
+        const uint64_t p0 = (uint64_t)0xD2511F53u * c0;
+        const uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
+        const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ k0;
+        const uint32_t n1 = (uint32_t)p1;
+        const uint32_t n2 = (uint32_t)(p0 >> 32) ^ c3 ^ k1;
+        const uint32_t n3 = (uint32_t)p0;
+        c0 = n0; c1 = n1; c2 = n2; c3 = n3;
+        /* key schedule: the Weyl increments (golden ratio, sqrt(3) - 1) */
+        k0 += 0x9E3779B9u;
+        k1 += 0xBB67AE85u;
+    }
+    out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
+}
+
+int oracle_dropout(const double* o, int64_t n, double p, uint64_t seed, double* out)
+{
+    if (!o || !out || n < 0 || !(p >= 0.0) || !(p < 1.0)) return -1;
+    /* element e keeps its value when word e mod 4 of the generator at counter
+     * (e div 4, 0, 0) and key (seed) is at least p * 2^32 */
+    const uint64_t thr = (uint64_t)(p * 4294967296.0);
+    const uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    for (int64_t e = 0; e < n; ++e) {
+        const uint64_t blk = (uint64_t)e >> 2;
+        const uint32_t ctr[4] = {(uint32_t)blk, (uint32_t)(blk >> 32), 0u, 0u};
+        uint32_t u[4];
+        oracle_philox4x32_10(ctr, key, u);
+        out[e] = ((uint64_t)u[e & 3] >= thr) ? o[e] / (1.0 - p) : 0.0;
+    }
+    return 0;
+}

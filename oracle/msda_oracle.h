@@ -15,6 +15,10 @@
  *   [SCA] "Spatial Cross-Attention" walkthrough, Tencent Cloud developer
  *         article 2321140: the bev_mask query rebatch listing and the
  *         scatter-add / clamp(count, 1) average listing.
+ *   [PX]  Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy as
+ *         1, 2, 3", SC 2011: the counter-based generator Philox4x32-10,
+ *         used for training-time dropout (the pages' dropout draws from
+ *         PyTorch's generator, which no second implementation can replay).
  *   [TS]  "【论文阅读】BEVFormer论文解析及Temporal Self-Attention、Spatial
  *         Cross-Attention注意力机制详解及代码示例" (wsisp.com): section 二.2
  *         (TSA between the previous and the current BEV) and the BEV encoder
@@ -163,6 +167,18 @@ int oracle_tsa_forward(const double* value, int B, int T, int Nv, int H, int Dh,
                        int Nq, int P, int R, const double* ref,
                        const double* off, const double* logits,
                        int coord_f32, double* out);
+
+/* Philox4x32-10 ([PX]): ten rounds of two multiply-xor S-boxes with
+ * multipliers 0xD2511F53, 0xCD9E8D57 and key increments 0x9E3779B9,
+ * 0xBB67AE85; out = the four output words for counter ctr and key key. */
+void oracle_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]);
+
+/* Training-time dropout ([BQ] 12: m / (1 - p) * o): element e of o [n] is
+ * kept when word (e mod 4) of Philox4x32-10 at counter (e div 4 as two
+ * 32-bit words low first, 0, 0) and key (seed low, seed high) is
+ * >= floor(p * 2^32), and then scaled by 1 / (1 - p); otherwise 0.
+ * 0 <= p < 1; p = 0 is the identity. */
+int oracle_dropout(const double* o, int64_t n, double p, uint64_t seed, double* out);
 
 #ifdef __cplusplus
 }

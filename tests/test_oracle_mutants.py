@@ -83,6 +83,11 @@ MUTANTS = [
      "out[((int64_t)b * Nq + q) * HD + d] = sum;", 0),
     ("every queue reads queue 0", "sum += per_queue[(((int64_t)b * T + t) * Nq + q) * HD + d];",
      "sum += per_queue[(((int64_t)b * T + 0) * Nq + q) * HD + d];", 0),
+    ("Philox multiplier digits swapped", "(uint64_t)0xD2511F53u * c0", "(uint64_t)0xD2511F35u * c0", 0),
+    ("Philox key not bumped", "k0 += 0x9E3779B9u;", "", 0),
+    ("dropout without the rescale", "? o[e] / (1.0 - p) : 0.0", "? o[e] : 0.0", 0),
+    ("dropout keeps the low draws", "(uint64_t)u[e & 3] >= thr", "(uint64_t)u[e & 3] < thr", 0),
+    ("dropout reads the wrong word", "(uint64_t)u[e & 3] >= thr", "(uint64_t)u[(e >> 2) & 3] >= thr", 0),
 ]
 
 PIN_CALLS = [
@@ -113,6 +118,9 @@ PIN_CALLS = [
     ("tsa_rigid", lambda: pins.test_tsa_reference_points_are_a_rigid_motion()),
     ("tsa_rot90", lambda: pins.test_tsa_quarter_turns_rotate_the_previous_map(90.0, 1)),
     ("tsa_shift", lambda: pins.test_tsa_whole_cell_shift_moves_the_previous_map()),
+    ("philox_kat", lambda: [pins.test_philox_known_answers(*k) for k in pins.PHILOX_KAT]),
+    ("dropout_scale", lambda: pins.test_dropout_keeps_and_scales()),
+    ("dropout_words", lambda: pins.test_dropout_mask_is_the_generator_words()),
 ]
 
 
@@ -140,10 +148,10 @@ def test_pins_catch_planted_mistake(tmp_path, monkeypatch, name, old, new, occ):
                   "oracle_fused_locations", "oracle_msda_backward", "oracle_sca_compact",
                   "oracle_sca_forward", "oracle_sca_backward", "oracle_linear",
                   "oracle_sca_backward_inputs", "oracle_tsa_reference_points",
-                  "oracle_tsa_forward"):
+                  "oracle_tsa_forward", "oracle_dropout", "oracle_philox4x32_10"):
         fn = getattr(mutant, fname)
         fn.argtypes = getattr(good, fname).argtypes
-        fn.restype = ctypes.c_int
+        fn.restype = getattr(good, fname).restype
     monkeypatch.setattr(oracle, "_lib", mutant)
     caught = []
     for pin_name, call in PIN_CALLS:

@@ -723,3 +723,54 @@ def test_tsa_mean_is_symmetric_in_the_queues():
     one = oracle.msda_forward_fused(args[0][:1], w.spatial_shapes, w.level_start_index,
                                     *(x[:1] for x in args[1:]))
     np.testing.assert_allclose(same, one, rtol=0, atol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# training-time dropout (section 12) with Philox4x32-10 (Salmon, Moraes,
+# Dror, Shaw, "Parallel random numbers: as easy as 1, 2, 3", SC 2011)
+# --------------------------------------------------------------------------
+
+# the generator's published known-answer vectors: (counter, key) -> output
+PHILOX_KAT = [
+    ((0, 0, 0, 0), (0, 0), (0x6627E8D5, 0xE169C58D, 0xBC57AC4C, 0x9B00DBD8)),
+    ((0xFFFFFFFF,) * 4, (0xFFFFFFFF,) * 2, (0x408F276D, 0x41C83B0E, 0xA20BC7C6, 0x6D5451FD)),
+    ((0x243F6A88, 0x85A308D3, 0x13198A2E, 0x03707344), (0xA4093822, 0x299F31D0),
+     (0xD16CFE09, 0x94FDCCEB, 0x5001E420, 0x24126EA1)),
+]
+
+
+@pytest.mark.parametrize("ctr,key,want", PHILOX_KAT)
+def test_philox_known_answers(ctr, key, want):
+    assert [int(x) for x in oracle.philox4x32_10(ctr, key)] == list(want)
+
+
+def test_dropout_zero_rate_is_identity():
+    o = _rng(70).standard_normal((13, 7))
+    np.testing.assert_array_equal(oracle.dropout(o, 0.0, 123), o)
+
+
+def test_dropout_keeps_and_scales():
+    """Kept elements are o / (1 - p) exactly, dropped ones 0, the kept
+    fraction is 1 - p within five standard deviations, the mask follows the
+    element index only (not the values), and another seed gives another mask."""
+    p, n = 0.1, 1 << 18
+    o = _rng(71).uniform(1.0, 2.0, n)
+    y = oracle.dropout(o, p, 2024)
+    kept = y != 0
+    np.testing.assert_array_equal(y[kept], o[kept] / (1 - p))
+    sigma = np.sqrt(n * p * (1 - p))
+    assert abs(kept.sum() - n * (1 - p)) < 5 * sigma
+    y2 = oracle.dropout(o * 3.0 + 1.0, p, 2024)
+    np.testing.assert_array_equal(y2 != 0, kept)
+    y3 = oracle.dropout(o, p, 2025)
+    assert 0.1 * n < np.count_nonzero((y3 != 0) != kept) < 0.3 * n
+
+
+def test_dropout_mask_is_the_generator_words():
+    """Element e is kept iff word e mod 4 of Philox at counter (e div 4) and
+    key (seed) is at least p * 2^32 (checked on a few elements by hand)."""
+    p, seed = 0.25, (7 << 32) | 5
+    y = oracle.dropout(np.ones(40), p, seed)
+    for e in (0, 1, 2, 3, 4, 17, 39):
+        u = oracle.philox4x32_10((e // 4, 0, 0, 0), (5, 7))[e % 4]
+        assert (y[e] != 0) == (int(u) >= int(p * 2 ** 32))
