@@ -157,6 +157,17 @@ def input_grads_algorithmic_bytes(w, rows):
                + w.B * w.Nq * S * 3 * 4 + w.Ncam * w.B * w.Nq * w.R * 2 * 4)
 
 
+def sca_backward_algorithmic_bytes(w, rows, hit_queries, value_elem):
+    """sca_backward: the forward's inputs once (value, offsets and logits of
+    seen queries, reference points, mask), grad_out once, grad_value written
+    once (the atomics' read-modify-write is not counted), the rebatched
+    location and weight gradients of the seen rows written once."""
+    S = w.H * w.L * w.P
+    return int(w.value.size * value_elem + hit_queries * S * 3 * 4 + rows * w.R * 2 * 4
+               + w.bev_mask.nbytes + w.B * w.Nq * w.H * 32 * 4 + w.value.size * 4
+               + rows * S * 3 * 4)
+
+
 def kernel_source_digest():
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
@@ -414,6 +425,15 @@ def run_native(args):
     if world > 1:
         dist.barrier()
     clocks = sampler.stop() if sampler else None
+    # the gather again with a warm L2 (no flush between launches), for reference
+    warm_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(min(args.steps, 50))]
+    for a, b in warm_evs:
+        a.record(stream)
+        gather()
+        b.record(stream)
+    torch.cuda.synchronize()
+    warm_gather_ms = float(np.median([a.elapsed_time(b) for a, b in warm_evs]))
     step_ms = [e[0].elapsed_time(e[3]) for e in evs]
     gather_ms = [e[1].elapsed_time(e[2]) for e in evs]
     compact_ms = [e[0].elapsed_time(e[1]) for e in evs]
@@ -480,6 +500,10 @@ def run_native(args):
                  "hbm_frac": nbytes["step"] / (step_mean * 1e-3) / 1e9 / peak,
                  "ms": {"compact": float(np.mean(compact_ms)), "gather": g_ms,
                         "average": float(np.mean(avg_ms)), "step": step_mean},
+                 "step_ms_percentiles": {"p10": float(np.percentile(step_ms, 10)),
+                                         "median": float(np.median(step_ms)),
+                                         "p90": float(np.percentile(step_ms, 90))},
+                 "gather_ms_warm_l2_median": warm_gather_ms,
                  "samples": samples_per_step, "rebatched_rows": rows},
         "e2e": {"value": e2e_gs, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "api": "sca_forward (one call)",
@@ -546,6 +570,25 @@ def measure_next_rows(args, w, tensors, flush, stream, hbm_peak):
     r.update(kernel="sca_query_major_kernel", workload="bevformer-base-sca-forward",
              gsamples_per_s=tensors["samples"] / (ms * 1e-3) / 1e9)
     rows["sca_forward_query_major"] = r
+
+    # the plain fused MSDA: the Deformable-DETR encoder and the TSA queues as a batch
+    for name, wk in (("msda_forward_fused_detr", inputs.workload2()),
+                     ("msda_forward_fused_tsa_batch2", inputs.workload4())):
+        dv = {k: torch.from_numpy(np.ascontiguousarray(a)).cuda() for k, a in (
+            ("value", wk.value), ("ref", wk.reference_points), ("off", wk.sampling_offsets),
+            ("logits", wk.attention_logits))}
+        o = torch.empty((wk.B, wk.Nq, wk.H * 32), dtype=torch.float32, device="cuda")
+        fa = (dv["value"], wk.spatial_shapes, wk.level_start_index, dv["ref"], dv["off"],
+              dv["logits"])
+        ms = timed(lambda: msda.msda_forward_fused(*fa, out=o))
+        S = wk.H * wk.L * wk.P
+        nbytes = (wk.value.nbytes + wk.B * wk.Nq * S * 12 + wk.reference_points.nbytes
+                  + o.numel() * 4)
+        r = hbm(nbytes, ms)
+        r.update(kernel="msda_forward_group_kernel<float, true, 2>", workload=wk.name,
+                 gsamples_per_s=wk.B * wk.Nq * S / (ms * 1e-3) / 1e9)
+        rows[name] = r
+        del dv, o, fa
 
     # f4: TSA, two queues of the 200x200 BEV, ego motion (1.7 m, -0.9 m, 4 deg)
     w4 = inputs.workload4()
@@ -622,6 +665,28 @@ def measure_next_rows(args, w, tensors, flush, stream, hbm_peak):
     r = hbm(input_grads_algorithmic_bytes(w, n_rows), ms)
     r.update(kernel="sca_offset_logit_grads_kernel + sca_reference_grads_kernel")
     rows["sca_backward_inputs"] = r
+    del gl, gw, bufs, gout
+
+    # A10/A11: the SCA backward of the training-step shape (B = 2, bf16 value)
+    w5 = inputs.workload5()
+    d5 = {k: torch.from_numpy(np.ascontiguousarray(a)).cuda() for k, a in (
+        ("ref", w5.reference_points), ("mask", w5.bev_mask), ("off", w5.sampling_offsets),
+        ("logits", w5.attention_logits), ("gout", w5.grad_out))}
+    v5 = torch.from_numpy(w5.value_bf16.view(np.int16)).cuda().view(torch.bfloat16)
+    args5 = (v5, w5.spatial_shapes, w5.level_start_index, d5["ref"], d5["mask"], d5["off"],
+             d5["logits"], d5["gout"])
+    g5 = msda.sca_backward(*args5)
+    _, cnt5, _, hits5 = msda.sca_compact(d5["mask"])
+    rows5, hitq5 = int(cnt5.sum().item()), int((hits5 > 0).sum().item())
+    ms = timed(lambda: msda.sca_backward(*args5, grad_value=g5[0],
+                                         grad_sampling_locations_rb=g5[1],
+                                         grad_attention_weights_rb=g5[2]),
+               n=max(1, iters // 4))
+    r = hbm(sca_backward_algorithmic_bytes(w5, rows5, hitq5, 2), ms)
+    r.update(kernel="sca_backward_kernel (+ compaction, zero fill, zero tail)",
+             workload="bevformer-base SCA training step, B=2, bf16 value",
+             gsamples_per_s=rows5 * w5.H * w5.L * w5.P / (ms * 1e-3) / 1e9)
+    rows["sca_backward"] = r
     return rows
 
 

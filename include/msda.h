@@ -172,6 +172,38 @@ msda_status_t msda_backward(const void* value, msda_dtype_t vdt,
                             float* grad_sampling_locations, float* grad_attention_weights,
                             msda_stream_t stream);
 
+/* Deterministic variants of msda_backward and sca_backward (the pages give no
+ * backward; the derivative is the same).  grad_value is accumulated without
+ * floating-point atomics: every contribution alpha * w_g * grad_out is scaled
+ * by 2^32 (exact), rounded once to a 64-bit integer and added with integer
+ * atomics into a fixed-point copy in the workspace, then rounded once to
+ * fp32.  Integer addition does not depend on order, so grad_value is bitwise
+ * reproducible from run to run, and its error (at most 2^-33 per
+ * contribution before the final rounding) is below that of fp32 sums.  The
+ * partial sums must stay below 2^31 in magnitude.  The other gradients are
+ * deterministic in both variants.  The workspace (caller-owned device
+ * memory, 256-byte aligned, contents ignored) holds the fixed-point copy (and,
+ * for the SCA call, the compaction lists). */
+size_t msda_backward_deterministic_workspace_size(msda_dims_t d);
+msda_status_t msda_backward_deterministic(const void* value, msda_dtype_t vdt,
+                                          const int64_t* spatial_shapes,
+                                          const int64_t* level_start_index,
+                                          const float* sampling_locations,
+                                          const float* attention_weights, const float* grad_out,
+                                          msda_dims_t d, void* workspace, size_t workspace_bytes,
+                                          float* grad_value, float* grad_sampling_locations,
+                                          float* grad_attention_weights, msda_stream_t stream);
+size_t sca_backward_deterministic_workspace_size(msda_dims_t d);
+msda_status_t sca_backward_deterministic(const void* value, msda_dtype_t vdt,
+                                         const int64_t* spatial_shapes,
+                                         const int64_t* level_start_index,
+                                         const float* reference_points_cam,
+                                         const uint8_t* bev_mask, const float* sampling_offsets,
+                                         const float* attention_logits, const float* grad_out,
+                                         msda_dims_t d, void* workspace, size_t workspace_bytes,
+                                         float* grad_value, float* grad_sampling_locations_rb,
+                                         float* grad_attention_weights_rb, msda_stream_t stream);
+
 /* Dense projection on the tensor cores ([BQ] 3 value projection W_v, 4.1
  * offset head W_Delta, 4.2 weight head W_alpha, 11 output projection W_o, 13
  * residual):  y = x w^T (+ bias) (+ residual).
@@ -187,6 +219,19 @@ msda_status_t msda_backward(const void* value, msda_dtype_t vdt,
 msda_status_t msda_linear(const void* x, const void* w, const float* bias,
                           const float* residual, int32_t M, int32_t N, int32_t K,
                           msda_dtype_t y_dtype, void* y, msda_stream_t stream);
+
+/* msda_linear with training-time dropout of x w^T + bias before the residual
+ * is added ([BQ] 12: m / (1 - p) * o):  y = residual + m (x w^T + bias) / (1 - p).
+ * The pages' dropout draws from PyTorch's generator; this mask is element
+ * e = row * N + col kept when word (e mod 4) of the counter-based generator
+ * Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as
+ * easy as 1, 2, 3", SC 2011) at counter (e div 4 low, high, 0, 0) and key
+ * (seed low, seed high) is >= floor(p * 2^32).  0 <= dropout_p < 1 (else
+ * MSDA_ERR_INVALID_ARG); dropout_p = 0 is msda_linear. */
+msda_status_t msda_linear_dropout(const void* x, const void* w, const float* bias,
+                                  const float* residual, int32_t M, int32_t N, int32_t K,
+                                  msda_dtype_t y_dtype, void* y, float dropout_p,
+                                  uint64_t dropout_seed, msda_stream_t stream);
 
 /* Number of msda_linear tiles that gave up waiting on their load or MMA
  * pipeline (each wait is bounded, about a second); 0 in normal operation.
@@ -344,8 +389,9 @@ msda_status_t sca_backward(const void* value, msda_dtype_t vdt,
  * [SCA] listings):
  *   q~ = bf16(q + pos);  V = F~ W_v^T + b_v;  Delta = q~ W_Delta^T + b_Delta;
  *   a = q~ W_alpha^T + b_alpha;  g = sca_forward(V, Delta, a, rho, mask);
- *   q_hat = q + bf16(g) W_o^T + b_o   (dropout is the identity, [BQ] 12;
- *   the LayerNorm after it belongs to the outer layer, [BQ] 13).
+ *   q_hat = q + dropout(bf16(g) W_o^T + b_o)   (dropout as msda_linear_dropout
+ *   with the params' rate and seed, the identity at rate 0, [BQ] 12; the
+ *   LayerNorm after it belongs to the outer layer, [BQ] 13).
  * C = H * 32.  The projections run on msda_linear, so C and H*L*P must be
  * multiples of 256 and C one of 64..256 (BEVFormer-base: C = 256, H = 8,
  * L = 4, P = 8).  Weights use the nn.Linear layout (out x in), bf16; biases
@@ -366,10 +412,13 @@ typedef struct {
     const float* reference_points_cam; /* [Ncam, B, Nq, R, 2] */
     const uint8_t* bev_mask;           /* [Ncam, B, Nq, R] */
     msda_dtype_t value_dtype;          /* storage of V for the sampling: fp32 or bf16 */
+    float dropout_p;                   /* training-time dropout rate in [0, 1); 0 = inference */
+    uint64_t dropout_seed;             /* key of the dropout mask (see msda_linear_dropout) */
 } sca_module_params_t;
 
-/* Bytes of device workspace sca_module_forward needs (q~, V, Delta, a, g and
- * the sca_forward workspace), 256-byte alignment included. */
+/* Bytes of device workspace sca_module_forward needs (q~, V, Delta, a, the
+ * bf16 g and the sca_forward workspace), 256-byte alignment included.  The
+ * camera average stores g directly as bf16, the output projection's operand. */
 size_t sca_module_workspace_size(msda_dims_t d, msda_dtype_t value_dtype);
 
 /*   q_hat [B, Nq, C] fp32, written.  workspace 256-byte aligned. */

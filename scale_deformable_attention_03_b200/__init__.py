@@ -40,7 +40,8 @@ class ScaModuleParams(ctypes.Structure):
     _fields_ = [("query", _vp), ("query_pos", _vp), ("features", _vp), ("w_value", _vp),
                 ("b_value", _vp), ("w_offsets", _vp), ("b_offsets", _vp), ("w_weights", _vp),
                 ("b_weights", _vp), ("w_output", _vp), ("b_output", _vp),
-                ("reference_points_cam", _vp), ("bev_mask", _vp), ("value_dtype", ctypes.c_int)]
+                ("reference_points_cam", _vp), ("bev_mask", _vp), ("value_dtype", ctypes.c_int),
+                ("dropout_p", ctypes.c_float), ("dropout_seed", ctypes.c_uint64)]
 
 
 _lib = None
@@ -59,6 +60,16 @@ def lib():
         L.msda_forward.argtypes = [_vp, st, _i64p, _i64p, _vp, _vp, Dims, _vp, _vp]
         L.msda_forward_fused.argtypes = [_vp, st, _i64p, _i64p, _vp, _vp, _vp, Dims, _vp, _vp]
         L.msda_backward.argtypes = [_vp, st, _i64p, _i64p, _vp, _vp, _vp, Dims, _vp, _vp, _vp, _vp]
+        L.msda_backward_deterministic.argtypes = [_vp, st, _i64p, _i64p, _vp, _vp, _vp, Dims,
+                                                  _vp, ctypes.c_size_t, _vp, _vp, _vp, _vp]
+        L.msda_backward_deterministic.restype = ctypes.c_int
+        L.msda_backward_deterministic_workspace_size.argtypes = [Dims]
+        L.msda_backward_deterministic_workspace_size.restype = ctypes.c_size_t
+        L.sca_backward_deterministic.argtypes = [_vp, st, _i64p, _i64p, _vp, _vp, _vp, _vp, _vp,
+                                                 Dims, _vp, ctypes.c_size_t, _vp, _vp, _vp, _vp]
+        L.sca_backward_deterministic.restype = ctypes.c_int
+        L.sca_backward_deterministic_workspace_size.argtypes = [Dims]
+        L.sca_backward_deterministic_workspace_size.restype = ctypes.c_size_t
         L.msda_workspace_size.argtypes = [Dims]
         L.msda_workspace_size.restype = ctypes.c_size_t
         L.sca_compact_workspace_size.argtypes = [Dims]
@@ -80,6 +91,10 @@ def lib():
         L.msda_linear.argtypes = [_vp, _vp, _vp, _vp, ctypes.c_int32, ctypes.c_int32,
                                   ctypes.c_int32, st, _vp, _vp]
         L.msda_linear.restype = ctypes.c_int
+        L.msda_linear_dropout.argtypes = [_vp, _vp, _vp, _vp, ctypes.c_int32, ctypes.c_int32,
+                                          ctypes.c_int32, st, _vp, ctypes.c_float,
+                                          ctypes.c_uint64, _vp]
+        L.msda_linear_dropout.restype = ctypes.c_int
         L.msda_linear_timeouts.restype = ctypes.c_uint32
         L.sca_module_workspace_size.argtypes = [Dims, ctypes.c_int]
         L.sca_module_workspace_size.restype = ctypes.c_size_t
@@ -243,9 +258,11 @@ def tsa_forward(value, spatial_shapes, level_start_index, reference_points, samp
 
 def msda_backward(value, spatial_shapes, level_start_index, sampling_locations,
                   attention_weights, grad_out, grad_value=None, grad_sampling_locations=None,
-                  grad_attention_weights=None, stream=None):
+                  grad_attention_weights=None, stream=None, deterministic=False, workspace=None):
     """-> (grad_value [B, Nv, H, 32] fp32, grad_sampling_locations,
-    grad_attention_weights)."""
+    grad_attention_weights).  deterministic=True accumulates grad_value in
+    fixed point (bitwise reproducible; needs a workspace, allocated here when
+    not given)."""
     torch = _torch()
     _contig(value, sampling_locations, attention_weights, grad_out)
     B, Nv, H, _ = value.shape
@@ -261,12 +278,17 @@ def msda_backward(value, spatial_shapes, level_start_index, sampling_locations,
         grad_attention_weights = torch.empty(attention_weights.shape, device=dev,
                                              dtype=torch.float32)
     d = Dims(B, 1, Nq, Nv, H, L, P, 1)
-    _check(lib().msda_backward(_ptr(value), _vdt(value), shapes.ctypes.data_as(_i64p),
-                               starts.ctypes.data_as(_i64p), _ptr(sampling_locations),
-                               _ptr(attention_weights), _ptr(grad_out), d, _ptr(grad_value),
-                               _ptr(grad_sampling_locations), _ptr(grad_attention_weights),
-                               _stream(stream)),
-           "msda_backward")
+    args = (_ptr(value), _vdt(value), shapes.ctypes.data_as(_i64p), starts.ctypes.data_as(_i64p),
+            _ptr(sampling_locations), _ptr(attention_weights), _ptr(grad_out), d)
+    outs = (_ptr(grad_value), _ptr(grad_sampling_locations), _ptr(grad_attention_weights),
+            _stream(stream))
+    if deterministic:
+        workspace = _workspace(int(lib().msda_backward_deterministic_workspace_size(d)), dev,
+                               workspace)
+        _check(lib().msda_backward_deterministic(*args, _ptr(workspace), workspace.numel(),
+                                                 *outs), "msda_backward_deterministic")
+    else:
+        _check(lib().msda_backward(*args, *outs), "msda_backward")
     return grad_value, grad_sampling_locations, grad_attention_weights
 
 
@@ -358,9 +380,11 @@ def sca_forward_query_major(value, spatial_shapes, level_start_index, reference_
 def sca_backward(value, spatial_shapes, level_start_index, reference_points_cam, bev_mask,
                  sampling_offsets, attention_logits, grad_out, grad_value=None,
                  grad_sampling_locations_rb=None, grad_attention_weights_rb=None,
-                 workspace=None, stream=None):
+                 workspace=None, stream=None, deterministic=False):
     """-> (grad_value [B, Ncam, Nv, H, 32], grad_sampling_locations_rb
-    [B, Ncam, Nq, H, L, P, 2], grad_attention_weights_rb [B, Ncam, Nq, H, L, P])."""
+    [B, Ncam, Nq, H, L, P, 2], grad_attention_weights_rb [B, Ncam, Nq, H, L, P]).
+    deterministic=True accumulates grad_value in fixed point (bitwise
+    reproducible; the workspace then also holds the fixed-point copy)."""
     torch = _torch()
     _contig(value, reference_points_cam, bev_mask, sampling_offsets, attention_logits, grad_out)
     if bev_mask.dtype == torch.bool:
@@ -376,14 +400,16 @@ def sca_backward(value, spatial_shapes, level_start_index, reference_points_cam,
     if grad_attention_weights_rb is None:
         grad_attention_weights_rb = torch.empty((d.B, d.Ncam, d.Nq, d.H, d.L, d.P), device=dev,
                                                 dtype=torch.float32)
-    workspace = _workspace(msda_workspace_size(d), dev, workspace)
-    _check(lib().sca_backward(_ptr(value), _vdt(value), shapes.ctypes.data_as(_i64p),
-                              starts.ctypes.data_as(_i64p), _ptr(reference_points_cam),
-                              _ptr(bev_mask), _ptr(sampling_offsets), _ptr(attention_logits),
-                              _ptr(grad_out), d, _ptr(workspace), workspace.numel(),
-                              _ptr(grad_value), _ptr(grad_sampling_locations_rb),
-                              _ptr(grad_attention_weights_rb), _stream(stream)),
-           "sca_backward")
+    fn = lib().sca_backward_deterministic if deterministic else lib().sca_backward
+    need = (int(lib().sca_backward_deterministic_workspace_size(d)) if deterministic
+            else msda_workspace_size(d))
+    workspace = _workspace(need, dev, workspace)
+    _check(fn(_ptr(value), _vdt(value), shapes.ctypes.data_as(_i64p),
+              starts.ctypes.data_as(_i64p), _ptr(reference_points_cam), _ptr(bev_mask),
+              _ptr(sampling_offsets), _ptr(attention_logits), _ptr(grad_out), d, _ptr(workspace),
+              workspace.numel(), _ptr(grad_value), _ptr(grad_sampling_locations_rb),
+              _ptr(grad_attention_weights_rb), _stream(stream)),
+           "sca_backward_deterministic" if deterministic else "sca_backward")
     return grad_value, grad_sampling_locations_rb, grad_attention_weights_rb
 
 
@@ -451,10 +477,12 @@ def sca_rebatched_backward(value, spatial_shapes, level_start_index, reference_p
     return grad_value, grad_sampling_locations_rb, grad_attention_weights_rb
 
 
-def msda_linear(x, w, bias=None, residual=None, out=None, out_dtype=None, stream=None):
+def msda_linear(x, w, bias=None, residual=None, out=None, out_dtype=None, stream=None,
+                dropout_p=0.0, dropout_seed=0):
     """y = x w^T (+ bias) (+ residual) on the tensor cores.  x [M, K] bf16,
     w [N, K] bf16, bias [N] fp32, residual [M, N] fp32 -> y [M, N] (fp32, or
-    bf16 when out_dtype / out is bfloat16)."""
+    bf16 when out_dtype / out is bfloat16).  dropout_p > 0 applies
+    training-time dropout to x w^T + bias before the residual."""
     torch = _torch()
     _contig(x, w, bias, residual, out)
     if x.dtype != torch.bfloat16 or w.dtype != torch.bfloat16:
@@ -464,8 +492,9 @@ def msda_linear(x, w, bias=None, residual=None, out=None, out_dtype=None, stream
     if out is None:
         out = torch.empty((M, N), device=x.device, dtype=out_dtype or torch.float32)
     ydt = MSDA_BF16 if out.dtype == torch.bfloat16 else MSDA_F32
-    _check(lib().msda_linear(_ptr(x), _ptr(w), _ptr(bias), _ptr(residual), M, N, K, ydt,
-                             _ptr(out), _stream(stream)),
+    _check(lib().msda_linear_dropout(_ptr(x), _ptr(w), _ptr(bias), _ptr(residual), M, N, K,
+                                     ydt, _ptr(out), float(dropout_p), int(dropout_seed),
+                                     _stream(stream)),
            "msda_linear")
     return out
 
@@ -473,7 +502,8 @@ def msda_linear(x, w, bias=None, residual=None, out=None, out_dtype=None, stream
 def sca_module_forward(query, query_pos, features, w_value, b_value, w_offsets, b_offsets,
                        w_weights, b_weights, w_output, b_output, reference_points_cam, bev_mask,
                        spatial_shapes, level_start_index, num_levels, num_points,
-                       value_dtype=None, out=None, workspace=None, stream=None):
+                       value_dtype=None, out=None, workspace=None, stream=None, dropout_p=0.0,
+                       dropout_seed=0):
     """The SCA module forward: q_hat = q + output_proj(SCA(value_proj(F~),
     offsets(q + pos), weights(q + pos))).  query, query_pos [B, Nq, C] fp32;
     features [B, Ncam, Nv, C] bf16; weights bf16 [out, in]; biases fp32;
@@ -499,7 +529,8 @@ def sca_module_forward(query, query_pos, features, w_value, b_value, w_offsets, 
     prm = ScaModuleParams(*[_ptr(t) for t in (query, query_pos, features, w_value, b_value,
                                               w_offsets, b_offsets, w_weights, b_weights,
                                               w_output, b_output, reference_points_cam,
-                                              bev_mask)], vdt)
+                                              bev_mask)], vdt, float(dropout_p),
+                           int(dropout_seed))
     _check(lib().sca_module_forward(ctypes.byref(prm), shapes.ctypes.data_as(_i64p),
                                     starts.ctypes.data_as(_i64p), d, _ptr(workspace),
                                     workspace.numel(), _ptr(out), _stream(stream)),

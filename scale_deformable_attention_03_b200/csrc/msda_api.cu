@@ -332,9 +332,55 @@ msda_status_t msda_backward(const void* value, msda_dtype_t vdt, const int64_t* 
     cudaError_t e = msda::launch_zero(grad_value, (int64_t)d.B * d.Nv * d.H * MSDA_HEAD_DIM, s);
     if (e == cudaSuccess && d.Nq > 0)
         e = msda::launch_msda_backward(p, sampling_locations, attention_weights, grad_out,
-                                       grad_value, grad_sampling_locations,
+                                       grad_value, nullptr, grad_sampling_locations,
                                        grad_attention_weights, s);
     return cuda_status(e, "msda_backward");
+}
+
+static msda_status_t check_workspace(const void* ws, size_t have, size_t need);
+
+size_t msda_backward_deterministic_workspace_size(msda_dims_t d)
+{
+    if (d.B < 0 || d.Nv < 1 || d.H < 1) return 0;
+    return align256(sizeof(long long) * (size_t)d.B * d.Nv * d.H * MSDA_HEAD_DIM);
+}
+
+msda_status_t msda_backward_deterministic(const void* value, msda_dtype_t vdt,
+                                          const int64_t* spatial_shapes,
+                                          const int64_t* level_start_index,
+                                          const float* sampling_locations,
+                                          const float* attention_weights, const float* grad_out,
+                                          msda_dims_t d, void* workspace, size_t workspace_bytes,
+                                          float* grad_value, float* grad_sampling_locations,
+                                          float* grad_attention_weights, msda_stream_t stream)
+{
+    MSDA_TRY(check_dims(d, false));
+    msda::Levels lv;
+    MSDA_TRY(check_levels(d, spatial_shapes, level_start_index, lv));
+    MSDA_TRY(check_dtype(vdt));
+    if (d.B == 0) return ok();
+    MSDA_PTR(grad_value, 16);
+    if (d.Nq > 0) {
+        MSDA_TRY(check_value(value));
+        MSDA_PTR(sampling_locations, 8);
+        MSDA_PTR(attention_weights, 4);
+        MSDA_PTR(grad_out, 16);
+        MSDA_PTR(grad_sampling_locations, 8);
+        MSDA_PTR(grad_attention_weights, 4);
+    }
+    MSDA_TRY(check_workspace(workspace, workspace_bytes,
+                             msda_backward_deterministic_workspace_size(d)));
+    const cudaStream_t s = (cudaStream_t)stream;
+    const msda::Problem p = make_problem(value, vdt, d, lv);
+    const int64_t n = (int64_t)d.B * d.Nv * d.H * MSDA_HEAD_DIM;
+    long long* acc = static_cast<long long*>(workspace);
+    cudaError_t e = msda::launch_zero(reinterpret_cast<float*>(acc), 2 * n, s);
+    if (e == cudaSuccess && d.Nq > 0)
+        e = msda::launch_msda_backward(p, sampling_locations, attention_weights, grad_out,
+                                       grad_value, acc, grad_sampling_locations,
+                                       grad_attention_weights, s);
+    if (e == cudaSuccess) e = msda::launch_fix_to_float(acc, grad_value, n, s);
+    return cuda_status(e, "msda_backward_deterministic");
 }
 
 size_t msda_workspace_size(msda_dims_t d)
@@ -445,7 +491,7 @@ msda_status_t sca_camera_average(const float* out_rb, const int32_t* pos, const 
     MSDA_PTR(hits, 4);
     MSDA_PTR(out, 16);
     return cuda_status(msda::launch_sca_average(out_rb, pos, hits, d.B, d.Ncam, d.Nq, d.H, out,
-                                                (cudaStream_t)stream),
+                                                false, (cudaStream_t)stream),
                        "sca_camera_average");
 }
 
@@ -455,25 +501,10 @@ msda_status_t sca_forward(const void* value, msda_dtype_t vdt, const int64_t* sp
                           const float* attention_logits, msda_dims_t d, void* workspace,
                           size_t workspace_bytes, float* out, msda_stream_t stream)
 {
-    msda::Levels lv;
-    MSDA_TRY(check_sca_inputs(value, vdt, d, spatial_shapes, level_start_index,
-                              reference_points_cam, sampling_offsets, attention_logits, lv));
-    if ((int64_t)d.B * d.Nq == 0) return ok();
-    MSDA_PTR(bev_mask, 1);
-    MSDA_PTR(out, 16);
-    MSDA_TRY(check_workspace(workspace, workspace_bytes,
-                             msda::sca_workspace_bytes(d.B, d.Ncam, d.Nq, d.H, true)));
-    const cudaStream_t s = (cudaStream_t)stream;
-    const msda::ScaWorkspace w = msda::sca_workspace_carve(workspace, d.B, d.Ncam, d.Nq, d.H, true);
-    const msda::Problem p = make_problem(value, vdt, d, lv);
-    cudaError_t e = msda::launch_sca_compact(bev_mask, d.B, d.Ncam, d.Nq, d.R, w.idx, w.count,
-                                             w.pos, w.hits, w.chunk_counts, s);
-    if (e == cudaSuccess)
-        e = msda::launch_sca_gather(p, reference_points_cam, sampling_offsets, attention_logits,
-                                    w.idx, w.count, w.out_rb, s);
-    if (e == cudaSuccess)
-        e = msda::launch_sca_average(w.out_rb, w.pos, w.hits, d.B, d.Ncam, d.Nq, d.H, out, s);
-    return cuda_status(e, "sca_forward");
+    return msda::sca_forward_to(value, vdt, spatial_shapes, level_start_index,
+                                reference_points_cam, bev_mask, sampling_offsets,
+                                attention_logits, d, workspace, workspace_bytes, out, false,
+                                (cudaStream_t)stream);
 }
 
 msda_status_t sca_forward_query_major(const void* value, msda_dtype_t vdt,
@@ -526,19 +557,11 @@ msda_status_t sca_rebatched_backward(const void* value, msda_dtype_t vdt,
         MSDA_PTR(grad_sampling_locations_rb, 8);
         MSDA_PTR(grad_attention_weights_rb, 4);
     }
-    const cudaStream_t s = (cudaStream_t)stream;
-    const msda::Problem p = make_problem(value, vdt, d, lv);
-    cudaError_t e = msda::launch_zero(grad_value,
-                                      (int64_t)d.B * d.Ncam * d.Nv * d.H * MSDA_HEAD_DIM, s);
-    if (e == cudaSuccess && d.Nq > 0)
-        e = msda::launch_sca_backward_rows(p, reference_points_cam, sampling_offsets,
-                                           attention_logits, grad_out, idx, hits, count,
-                                           grad_value, grad_sampling_locations_rb,
-                                           grad_attention_weights_rb, s);
-    if (e == cudaSuccess && d.Nq > 0)
-        e = msda::launch_sca_zero_tail(count, d.B, d.Ncam, d.Nq, d.H * d.L * d.P,
-                                       grad_sampling_locations_rb, grad_attention_weights_rb, s);
-    return cuda_status(e, "sca_rebatched_backward");
+    return msda::sca_rebatched_backward_to(value, vdt, d, lv, reference_points_cam,
+                                           sampling_offsets, attention_logits, grad_out, idx,
+                                           count, hits, grad_value, nullptr,
+                                           grad_sampling_locations_rb, grad_attention_weights_rb,
+                                           (cudaStream_t)stream);
 }
 
 msda_status_t sca_backward(const void* value, msda_dtype_t vdt, const int64_t* spatial_shapes,
@@ -567,6 +590,46 @@ msda_status_t sca_backward(const void* value, msda_dtype_t vdt, const int64_t* s
                                   reference_points_cam, sampling_offsets, attention_logits,
                                   grad_out, w.idx, w.count, w.hits, d, grad_value,
                                   grad_sampling_locations_rb, grad_attention_weights_rb, stream);
+}
+
+size_t sca_backward_deterministic_workspace_size(msda_dims_t d)
+{
+    if (d.B < 0 || d.Ncam < 1 || d.Nq < 0 || d.Nv < 1 || d.H < 1) return 0;
+    return msda::sca_workspace_bytes(d.B, d.Ncam, d.Nq, d.H, false) +
+           align256(sizeof(long long) * (size_t)d.B * d.Ncam * d.Nv * d.H * MSDA_HEAD_DIM);
+}
+
+msda_status_t sca_backward_deterministic(const void* value, msda_dtype_t vdt,
+                                         const int64_t* spatial_shapes,
+                                         const int64_t* level_start_index,
+                                         const float* reference_points_cam,
+                                         const uint8_t* bev_mask, const float* sampling_offsets,
+                                         const float* attention_logits, const float* grad_out,
+                                         msda_dims_t d, void* workspace, size_t workspace_bytes,
+                                         float* grad_value, float* grad_sampling_locations_rb,
+                                         float* grad_attention_weights_rb, msda_stream_t stream)
+{
+    msda::Levels lv;
+    MSDA_TRY(check_sca_inputs(value, vdt, d, spatial_shapes, level_start_index,
+                              reference_points_cam, sampling_offsets, attention_logits, lv));
+    if (d.B == 0) return ok();
+    if (d.Nq > 0) MSDA_PTR(bev_mask, 1);
+    MSDA_TRY(check_workspace(workspace, workspace_bytes,
+                             sca_backward_deterministic_workspace_size(d)));
+    const cudaStream_t s = (cudaStream_t)stream;
+    const size_t lists = msda::sca_workspace_bytes(d.B, d.Ncam, d.Nq, d.H, false);
+    const msda::ScaWorkspace w = msda::sca_workspace_carve(workspace, d.B, d.Ncam, d.Nq, d.H, false);
+    long long* acc = reinterpret_cast<long long*>(static_cast<char*>(workspace) + lists);
+    if (d.Nq > 0) {
+        const cudaError_t e = msda::launch_sca_compact(bev_mask, d.B, d.Ncam, d.Nq, d.R, w.idx,
+                                                       w.count, w.pos, w.hits, w.chunk_counts, s);
+        if (e != cudaSuccess) return cuda_status(e, "sca_backward_deterministic");
+    }
+    return msda::sca_rebatched_backward_to(value, vdt, d, lv, reference_points_cam,
+                                           sampling_offsets, attention_logits, grad_out, w.idx,
+                                           w.count, w.hits, grad_value, acc,
+                                           grad_sampling_locations_rb, grad_attention_weights_rb,
+                                           s);
 }
 
 }  // extern "C"
@@ -607,4 +670,74 @@ namespace msda {
 msda_status_t api_fail(msda_status_t code, const char* message) { return fail(code, "%s", message); }
 msda_status_t api_ok() { return ok(); }
 msda_status_t api_cuda(cudaError_t e, const char* where) { return cuda_status(e, where); }
+}  // namespace msda
+
+namespace msda {
+
+msda_status_t sca_forward_to(const void* value, msda_dtype_t vdt, const int64_t* spatial_shapes,
+                             const int64_t* level_start_index, const float* reference_points_cam,
+                             const uint8_t* bev_mask, const float* sampling_offsets,
+                             const float* attention_logits, msda_dims_t d, void* workspace,
+                             size_t workspace_bytes, void* out, bool out_bf16, cudaStream_t s)
+{
+    msda::Levels lv;
+    MSDA_TRY(check_sca_inputs(value, vdt, d, spatial_shapes, level_start_index,
+                              reference_points_cam, sampling_offsets, attention_logits, lv));
+    if ((int64_t)d.B * d.Nq == 0) return ok();
+    MSDA_PTR(bev_mask, 1);
+    MSDA_PTR(out, 16);
+    MSDA_TRY(check_workspace(workspace, workspace_bytes,
+                             msda::sca_workspace_bytes(d.B, d.Ncam, d.Nq, d.H, true)));
+    const msda::ScaWorkspace w = msda::sca_workspace_carve(workspace, d.B, d.Ncam, d.Nq, d.H, true);
+    const msda::Problem p = make_problem(value, vdt, d, lv);
+    cudaError_t e = msda::launch_sca_compact(bev_mask, d.B, d.Ncam, d.Nq, d.R, w.idx, w.count,
+                                             w.pos, w.hits, w.chunk_counts, s);
+    if (e == cudaSuccess)
+        e = msda::launch_sca_gather(p, reference_points_cam, sampling_offsets, attention_logits,
+                                    w.idx, w.count, w.out_rb, s);
+    if (e == cudaSuccess)
+        e = msda::launch_sca_average(w.out_rb, w.pos, w.hits, d.B, d.Ncam, d.Nq, d.H, out,
+                                     out_bf16, s);
+    return cuda_status(e, "sca_forward");
+}
+
+}  // namespace msda
+
+namespace msda {
+
+// sca_rebatched_backward after its input checks; acc non-null: the
+// deterministic fixed-point accumulation (acc zeroed here, then rounded into
+// grad_value).
+msda_status_t sca_rebatched_backward_to(const void* value, msda_dtype_t vdt, const msda_dims_t& d,
+                                        const Levels& lv, const float* reference_points_cam,
+                                        const float* sampling_offsets,
+                                        const float* attention_logits, const float* grad_out,
+                                        const int32_t* idx, const int32_t* count,
+                                        const int32_t* hits, float* grad_value, long long* acc,
+                                        float* grad_loc_rb, float* grad_attn_rb, cudaStream_t s)
+{
+    MSDA_PTR(grad_value, 16);
+    if (d.Nq > 0) {
+        MSDA_PTR(grad_out, 16);
+        MSDA_PTR(idx, 4);
+        MSDA_PTR(count, 4);
+        MSDA_PTR(hits, 4);
+        MSDA_PTR(grad_loc_rb, 8);
+        MSDA_PTR(grad_attn_rb, 4);
+    }
+    const Problem p = make_problem(value, vdt, d, lv);
+    const int64_t n = (int64_t)d.B * d.Ncam * d.Nv * d.H * MSDA_HEAD_DIM;
+    cudaError_t e = acc ? launch_zero(reinterpret_cast<float*>(acc), 2 * n, s)
+                        : launch_zero(grad_value, n, s);
+    if (e == cudaSuccess && d.Nq > 0)
+        e = launch_sca_backward_rows(p, reference_points_cam, sampling_offsets, attention_logits,
+                                     grad_out, idx, hits, count, grad_value, acc, grad_loc_rb,
+                                     grad_attn_rb, s);
+    if (e == cudaSuccess && d.Nq > 0)
+        e = launch_sca_zero_tail(count, d.B, d.Ncam, d.Nq, d.H * d.L * d.P, grad_loc_rb,
+                                 grad_attn_rb, s);
+    if (e == cudaSuccess && acc) e = launch_fix_to_float(acc, grad_value, n, s);
+    return cuda_status(e, acc ? "sca_backward_deterministic" : "sca_rebatched_backward");
+}
+
 }  // namespace msda

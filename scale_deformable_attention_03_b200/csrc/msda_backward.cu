@@ -11,6 +11,11 @@
 // alpha w_g grad_out to grad_value with one 16-byte vector reduction
 // (red.global.add.v4.f32); the per-sample scalars are reduced with shuffles
 // and land on the lane that owns the sample, which writes them coalesced.
+// Deterministic variant (DET): instead of fp32 reductions, each contribution
+// is scaled by 2^32 (exact), rounded once to a 64-bit integer and added with
+// red.global.add.u64 into a fixed-point copy of grad_value; integer addition
+// does not depend on order, so the result is bitwise reproducible, and one
+// conversion kernel rounds it to fp32 at the end.
 // The dot products and everything derived from them are formed in double
 // (a product of two fp32 numbers is exact in double): the location gradient
 // multiplies a difference of dot products by alpha * W_l (up to ~40 at
@@ -37,6 +42,14 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
                  "f"(c), "f"(d)
                  : "memory");
+}
+
+constexpr float kFixScale = 4294967296.f;  // 2^32: fixed-point grad_value units
+
+__device__ __forceinline__ void red_add_fix(long long* addr, float v)
+{
+    const long long q = __float2ll_rn(v * kFixScale);
+    asm volatile("red.global.add.u64 [%0], %1;" ::"l"(addr), "l"(q) : "memory");
 }
 
 // d w_g / d lx and d w_g / d ly for neighbour g.
@@ -73,9 +86,10 @@ struct BwdLanes<float> {
     __device__ __forceinline__ static int group(int lane) { return lane >> 3; }
     // sample (within the batch) whose dot product the lane holds after batch()
     __device__ __forceinline__ static int held(int lane) { return lane & 7; }
+    template <bool DET>
     __device__ __forceinline__ double batch(const float* __restrict__ vb,
-                                            float* __restrict__ gvb, const BwdTable& tab,
-                                            int j0, int cnt, int lane) const
+                                            float* __restrict__ gvb, long long* __restrict__ gvi,
+                                            const BwdTable& tab, int j0, int cnt, int lane) const
     {
         const int g = lane >> 3, t = lane & 7;
         double part[8];
@@ -89,7 +103,17 @@ struct BwdLanes<float> {
                 part[k] = (double)go.x * v.x + (double)go.y * v.y + (double)go.z * v.z +
                           (double)go.w * v.w;
                 const float w = tab.alpha[j] * tab.wb[g][j];
-                if (w != 0.f) red_add_v4(gvb + o + 4 * t, w * go.x, w * go.y, w * go.z, w * go.w);
+                if (w != 0.f) {
+                    if (DET) {
+                        long long* dst = gvi + o + 4 * t;
+                        red_add_fix(dst, w * go.x);
+                        red_add_fix(dst + 1, w * go.y);
+                        red_add_fix(dst + 2, w * go.z);
+                        red_add_fix(dst + 3, w * go.w);
+                    } else {
+                        red_add_v4(gvb + o + 4 * t, w * go.x, w * go.y, w * go.z, w * go.w);
+                    }
+                }
             }
         }
         double q[4], r[2];
@@ -131,9 +155,10 @@ struct BwdLanes<__nv_bfloat16> {
     }
     __device__ __forceinline__ static int group(int lane) { return (lane >> 2) & 3; }
     __device__ __forceinline__ static int held(int lane) { return 2 * (lane & 3) + (lane >> 4); }
+    template <bool DET>
     __device__ __forceinline__ double batch(const __nv_bfloat16* __restrict__ vb,
-                                            float* __restrict__ gvb, const BwdTable& tab,
-                                            int j0, int cnt, int lane) const
+                                            float* __restrict__ gvb, long long* __restrict__ gvi,
+                                            const BwdTable& tab, int j0, int cnt, int lane) const
     {
         const int s = lane >> 4, g = (lane >> 2) & 3, t = lane & 3;
         double part[4];
@@ -155,9 +180,15 @@ struct BwdLanes<__nv_bfloat16> {
                 part[k] = d;
                 const float w = tab.alpha[j] * tab.wb[g][j];
                 if (w != 0.f) {
-                    float* dst = gvb + o + 8 * t;
-                    red_add_v4(dst, w * go[0], w * go[1], w * go[2], w * go[3]);
-                    red_add_v4(dst + 4, w * go[4], w * go[5], w * go[6], w * go[7]);
+                    if (DET) {
+                        long long* dst = gvi + o + 8 * t;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) red_add_fix(dst + i, w * go[i]);
+                    } else {
+                        float* dst = gvb + o + 8 * t;
+                        red_add_v4(dst, w * go[0], w * go[1], w * go[2], w * go[3]);
+                        red_add_v4(dst + 4, w * go[4], w * go[5], w * go[6], w * go[7]);
+                    }
                 }
             }
         }
@@ -181,15 +212,17 @@ struct BwdLanes<__nv_bfloat16> {
 
 // Backward of one (row, head).  grow: grad_out of the row's head (32 floats),
 // divided by `scale` (1 for MSDA, max(1, hits) for SCA).  gvb: grad_value of
-// the batch item (and camera).  gloc_row [L, P, 2], gattn_row [L, P].
-template <typename VT, bool FUSED, int NC>
+// the batch item (and camera), or (DET) gvi its fixed-point copy.  gloc_row
+// [L, P, 2], gattn_row [L, P].
+template <typename VT, bool FUSED, int NC, bool DET>
 __device__ __forceinline__ void row_backward(const VT* __restrict__ vb, int H, int h,
                                              const float* __restrict__ lo,
                                              const float* __restrict__ wl,
                                              const float* __restrict__ ref, int n,
                                              const LaneSamples<NC>& ls, BwdTable& tab,
                                              const float* __restrict__ grow, float scale,
-                                             float* __restrict__ gvb, float* __restrict__ gloc_row,
+                                             float* __restrict__ gvb, long long* __restrict__ gvi,
+                                             float* __restrict__ gloc_row,
                                              float* __restrict__ gattn_row, int lane)
 {
     float a[NC];
@@ -229,7 +262,7 @@ __device__ __forceinline__ void row_backward(const VT* __restrict__ vb, int H, i
         float res_w = 0.f, res_x = 0.f, res_y = 0.f;
         const int cnt = min(32, n - c * 32);
         for (int j0 = 0; j0 < cnt; j0 += 8) {
-            const double d = lanes.batch(vb, gvb, tab, j0, cnt, lane);
+            const double d = lanes.template batch<DET>(vb, gvb, gvi, tab, j0, cnt, lane);
             const int js = j0 + held;  // the sample whose D_g this lane holds
             const bool valid = js < cnt;
             double cw = valid ? (double)tab.wb[g][js] * d : 0.0;
@@ -260,11 +293,12 @@ __device__ __forceinline__ void row_backward(const VT* __restrict__ vb, int H, i
     }
 }
 
-template <typename VT, int NC>
+template <typename VT, int NC, bool DET>
 __global__ void __launch_bounds__(kThreads)
 msda_backward_kernel(const VT* __restrict__ value, const float* __restrict__ loc,
                      const float* __restrict__ attn, const float* __restrict__ grad_out,
-                     float* __restrict__ grad_value, float* __restrict__ grad_loc,
+                     float* __restrict__ grad_value, long long* __restrict__ grad_value_fix,
+                     float* __restrict__ grad_loc,
                      float* __restrict__ grad_attn, int B, int Nq, int Nv, int H, int L, int P,
                      Levels levels)
 {
@@ -291,20 +325,22 @@ msda_backward_kernel(const VT* __restrict__ value, const float* __restrict__ loc
         }
         const int64_t item = bq * H + cur.h;
         const int64_t vofs = (int64_t)b * Nv * H * kHeadDim;
-        row_backward<VT, false, NC>(value + vofs, H, cur.h, loc + item * S * 2, attn + item * S,
-                                    nullptr, S, ls, s_tab[warp], grad_out + item * kHeadDim, 1.f,
-                                    grad_value + vofs, grad_loc + item * S * 2,
-                                    grad_attn + item * S, lane);
+        row_backward<VT, false, NC, DET>(value + vofs, H, cur.h, loc + item * S * 2,
+                                         attn + item * S, nullptr, S, ls, s_tab[warp],
+                                         grad_out + item * kHeadDim, 1.f, grad_value + vofs,
+                                         DET ? grad_value_fix + vofs : nullptr,
+                                         grad_loc + item * S * 2, grad_attn + item * S, lane);
     }
 }
 
-template <typename VT, int NC>
+template <typename VT, int NC, bool DET>
 __global__ void __launch_bounds__(kThreads)
 sca_backward_kernel(const VT* __restrict__ value, const float* __restrict__ off,
                     const float* __restrict__ logits, const float* __restrict__ ref_cam,
                     const float* __restrict__ grad_out, const int32_t* __restrict__ idx,
                     const int32_t* __restrict__ hits, const int32_t* __restrict__ count,
-                    float* __restrict__ grad_value, float* __restrict__ grad_loc_rb,
+                    float* __restrict__ grad_value, long long* __restrict__ grad_value_fix,
+                    float* __restrict__ grad_loc_rb,
                     float* __restrict__ grad_attn_rb, int B, int Ncam, int Nq, int Nv, int H,
                     int L, int P, int R, Levels levels)
 {
@@ -341,11 +377,14 @@ sca_backward_kernel(const VT* __restrict__ value, const float* __restrict__ off,
             const int64_t vofs = (int64_t)bc * Nv * H * kHeadDim;
             const int64_t rowh = ((int64_t)bc * Nq + i) * H + h;
             const float scale = (float)max(1, __ldg(hits + bq));
-            row_backward<VT, true, NC>(value + vofs, H, h, off + bqh * S * 2, logits + bqh * S,
-                                       ref_cam + (((int64_t)c * B + b) * Nq + q) * R * 2, S, ls,
-                                       s_tab[warp], grad_out + bqh * kHeadDim, scale,
-                                       grad_value + vofs, grad_loc_rb + rowh * S * 2,
-                                       grad_attn_rb + rowh * S, lane);
+            row_backward<VT, true, NC, DET>(value + vofs, H, h, off + bqh * S * 2,
+                                            logits + bqh * S,
+                                            ref_cam + (((int64_t)c * B + b) * Nq + q) * R * 2, S,
+                                            ls, s_tab[warp], grad_out + bqh * kHeadDim, scale,
+                                            grad_value + vofs,
+                                            DET ? grad_value_fix + vofs : nullptr,
+                                            grad_loc_rb + rowh * S * 2, grad_attn_rb + rowh * S,
+                                            lane);
         }
     }
 }
@@ -392,6 +431,23 @@ cudaError_t launch_zero(float* p, int64_t n, cudaStream_t s)
     return cudaGetLastError();
 }
 
+// grad_value = fixed-point accumulator * 2^-32, rounded once to fp32.
+__global__ void fix_to_float_kernel(const long long* __restrict__ acc, float* __restrict__ out,
+                                    int64_t n)
+{
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x)
+        out[i] = (float)((double)__ldcs(acc + i) * (1.0 / 4294967296.0));
+}
+
+cudaError_t launch_fix_to_float(const long long* acc, float* out, int64_t n, cudaStream_t s)
+{
+    if (n <= 0) return cudaSuccess;
+    const int64_t blocks = std::min<int64_t>((n + 255) / 256, (int64_t)device_sm_count() * 16);
+    fix_to_float_kernel<<<(unsigned)blocks, 256, 0, s>>>(acc, out, n);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_sca_zero_tail(const int32_t* count, int B, int Ncam, int Nq, int S,
                                  float* grad_loc_rb, float* grad_attn_rb, cudaStream_t s)
 {
@@ -403,10 +459,11 @@ cudaError_t launch_sca_zero_tail(const int32_t* count, int B, int Ncam, int Nq, 
     return cudaGetLastError();
 }
 
-template <typename VT>
+template <typename VT, bool DET>
 static cudaError_t launch_msda_backward_t(const Problem& p, const float* loc, const float* attn,
                                           const float* grad_out, float* grad_value,
-                                          float* grad_loc, float* grad_attn, cudaStream_t s)
+                                          long long* grad_value_fix, float* grad_loc,
+                                          float* grad_attn, cudaStream_t s)
 {
     const int64_t rows = (int64_t)p.B * p.Nq;
     if (rows == 0) return cudaSuccess;
@@ -415,9 +472,9 @@ static cudaError_t launch_msda_backward_t(const Problem& p, const float* loc, co
     const int nc = (p.L * p.P + 31) / 32;
 #define MSDA_BWD_CASE(NCV)                                                                       \
     case NCV:                                                                                    \
-        msda_backward_kernel<VT, NCV><<<grid, kThreads, 0, s>>>(                                 \
-            v, loc, attn, grad_out, grad_value, grad_loc, grad_attn, p.B, p.Nq, p.Nv, p.H, p.L,  \
-            p.P, p.lv);                                                                          \
+        msda_backward_kernel<VT, NCV, DET><<<grid, kThreads, 0, s>>>(                            \
+            v, loc, attn, grad_out, grad_value, grad_value_fix, grad_loc, grad_attn, p.B, p.Nq,  \
+            p.Nv, p.H, p.L, p.P, p.lv);                                                          \
         break;
     switch (nc) {
         MSDA_BWD_CASE(1)
@@ -431,13 +488,21 @@ static cudaError_t launch_msda_backward_t(const Problem& p, const float* loc, co
 }
 
 cudaError_t launch_msda_backward(const Problem& p, const float* loc, const float* attn,
-                                 const float* grad_out, float* grad_value, float* grad_loc,
-                                 float* grad_attn, cudaStream_t s)
+                                 const float* grad_out, float* grad_value,
+                                 long long* grad_value_fix, float* grad_loc, float* grad_attn,
+                                 cudaStream_t s)
 {
-    return p.bf16 ? launch_msda_backward_t<__nv_bfloat16>(p, loc, attn, grad_out, grad_value,
-                                                          grad_loc, grad_attn, s)
-                  : launch_msda_backward_t<float>(p, loc, attn, grad_out, grad_value, grad_loc,
-                                                  grad_attn, s);
+    if (grad_value_fix)
+        return p.bf16 ? launch_msda_backward_t<__nv_bfloat16, true>(
+                            p, loc, attn, grad_out, grad_value, grad_value_fix, grad_loc,
+                            grad_attn, s)
+                      : launch_msda_backward_t<float, true>(p, loc, attn, grad_out, grad_value,
+                                                            grad_value_fix, grad_loc, grad_attn, s);
+    return p.bf16 ? launch_msda_backward_t<__nv_bfloat16, false>(p, loc, attn, grad_out,
+                                                                 grad_value, nullptr, grad_loc,
+                                                                 grad_attn, s)
+                  : launch_msda_backward_t<float, false>(p, loc, attn, grad_out, grad_value,
+                                                         nullptr, grad_loc, grad_attn, s);
 }
 
 template <typename K>
@@ -449,12 +514,13 @@ static int bwd_resident_ctas(K kernel)
     return n;
 }
 
-template <typename VT>
+template <typename VT, bool DET>
 static cudaError_t launch_sca_backward_t(const Problem& p, const float* ref_cam, const float* off,
                                          const float* logits, const float* grad_out,
                                          const int32_t* idx, const int32_t* hits,
                                          const int32_t* count, float* grad_value,
-                                         float* grad_loc_rb, float* grad_attn_rb, cudaStream_t s)
+                                         long long* grad_value_fix, float* grad_loc_rb,
+                                         float* grad_attn_rb, cudaStream_t s)
 {
     const int64_t max_rows = (int64_t)p.B * p.Ncam * p.Nq;
     if (max_rows == 0) return cudaSuccess;
@@ -463,11 +529,11 @@ static cudaError_t launch_sca_backward_t(const Problem& p, const float* ref_cam,
     const int nc = (p.L * p.P + 31) / 32;
 #define SCA_BWD_CASE(NCV)                                                                        \
     case NCV: {                                                                                  \
-        static int occ = bwd_resident_ctas(sca_backward_kernel<VT, NCV>);                        \
+        static int occ = bwd_resident_ctas(sca_backward_kernel<VT, NCV, DET>);                   \
         const int64_t grid = std::min<int64_t>(max_ctas, (int64_t)occ * device_sm_count());      \
-        sca_backward_kernel<VT, NCV><<<(unsigned)grid, kThreads, 0, s>>>(                        \
-            v, off, logits, ref_cam, grad_out, idx, hits, count, grad_value, grad_loc_rb,        \
-            grad_attn_rb, p.B, p.Ncam, p.Nq, p.Nv, p.H, p.L, p.P, p.R, p.lv);                    \
+        sca_backward_kernel<VT, NCV, DET><<<(unsigned)grid, kThreads, 0, s>>>(                   \
+            v, off, logits, ref_cam, grad_out, idx, hits, count, grad_value, grad_value_fix,     \
+            grad_loc_rb, grad_attn_rb, p.B, p.Ncam, p.Nq, p.Nv, p.H, p.L, p.P, p.R, p.lv);       \
         break;                                                                                   \
     }
     switch (nc) {
@@ -485,13 +551,23 @@ cudaError_t launch_sca_backward_rows(const Problem& p, const float* ref_cam, con
                                      const float* logits, const float* grad_out,
                                      const int32_t* idx, const int32_t* hits,
                                      const int32_t* count, float* grad_value,
-                                     float* grad_loc_rb, float* grad_attn_rb, cudaStream_t s)
+                                     long long* grad_value_fix, float* grad_loc_rb,
+                                     float* grad_attn_rb, cudaStream_t s)
 {
-    return p.bf16 ? launch_sca_backward_t<__nv_bfloat16>(p, ref_cam, off, logits, grad_out, idx,
-                                                         hits, count, grad_value,
-                                                         grad_loc_rb, grad_attn_rb, s)
-                  : launch_sca_backward_t<float>(p, ref_cam, off, logits, grad_out, idx, hits,
-                                                 count, grad_value, grad_loc_rb, grad_attn_rb, s);
+    if (grad_value_fix)
+        return p.bf16 ? launch_sca_backward_t<__nv_bfloat16, true>(
+                            p, ref_cam, off, logits, grad_out, idx, hits, count, grad_value,
+                            grad_value_fix, grad_loc_rb, grad_attn_rb, s)
+                      : launch_sca_backward_t<float, true>(p, ref_cam, off, logits, grad_out, idx,
+                                                           hits, count, grad_value, grad_value_fix,
+                                                           grad_loc_rb, grad_attn_rb, s);
+    return p.bf16 ? launch_sca_backward_t<__nv_bfloat16, false>(p, ref_cam, off, logits, grad_out,
+                                                                idx, hits, count, grad_value,
+                                                                nullptr, grad_loc_rb,
+                                                                grad_attn_rb, s)
+                  : launch_sca_backward_t<float, false>(p, ref_cam, off, logits, grad_out, idx,
+                                                        hits, count, grad_value, nullptr,
+                                                        grad_loc_rb, grad_attn_rb, s);
 }
 
 }  // namespace msda

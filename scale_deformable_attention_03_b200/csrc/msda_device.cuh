@@ -44,6 +44,11 @@ constexpr int kMaxBatchCameras = 1024;  // B * Ncam limit of the SCA kernels
 #else
 #define MSDA_GATHER_BOUNDS __launch_bounds__(kThreads)
 #endif
+// Minimum resident CTAs of the small-row group kernels (a register cap).
+#ifndef MSDA_GROUP_MIN_CTAS
+#define MSDA_GROUP_MIN_CTAS 3
+#endif
+#define MSDA_GROUP_BOUNDS __launch_bounds__(kThreads, MSDA_GROUP_MIN_CTAS)
 #ifndef MSDA_PAIR_UNROLL
 #define MSDA_PAIR_UNROLL 2     // the same for the bf16 head-pair gather
 #endif
@@ -284,10 +289,6 @@ struct Gather<float> {
             acc[3] += w.x * x0.w + w.y * x1.w + w.z * x2.w + w.w * x3.w;
         }
     }
-    // Lane bits over which the partial sums of one output are spread: the
-    // corner g (bits 4 and 3).  Channel quad t = lane & 7.
-    static constexpr int kSumMasks[2] = {16, 8};
-    __device__ __forceinline__ static int channel0(int lane) { return 4 * (lane & 7); }
     // Sum the four corners; lanes 0..7 store channels 4t..4t+3.
     __device__ __forceinline__ static void store(float (&acc)[4], int lane, float* __restrict__ out)
     {
@@ -361,10 +362,6 @@ struct Gather<__nv_bfloat16> {
             fma8(acc, wb, rb);
         }
     }
-    // Partial sums spread over the sample half (bit 4) and the corner (bits 3,
-    // 2); channel group t = lane & 3.
-    static constexpr int kSumMasks[3] = {16, 8, 4};
-    __device__ __forceinline__ static int channel0(int lane) { return 8 * (lane & 3); }
     // Sum corners and halves; lanes 0..3 store channels 8t..8t+7.
     __device__ __forceinline__ static void store(float (&acc)[8], int lane, float* __restrict__ out)
     {
@@ -381,71 +378,6 @@ struct Gather<__nv_bfloat16> {
         }
     }
 };
-
-// Several heads' partial sums at once (acc[s] = head s, partial over the
-// lanes named by Gather<VT>::kSumMasks).  A butterfly reduce-scatter: at each
-// lane bit, the lane keeps half of the heads it holds (the lower half if the
-// bit is clear) and adds its partner's copy of that half, so G heads cost
-// (G/2 + G/4 + ...) shuffles per element instead of G per bit.  Once a lane
-// holds one head, the remaining bits are plain butterfly sums.
-template <int HELD, int G, int NA>
-__device__ __forceinline__ void reduce_level(float (&acc)[G][NA], int mask, int lane,
-                                             int& head0, bool& writer)
-{
-    if constexpr (HELD > 1) {
-        const bool upper = (lane & mask) != 0;
-#pragma unroll
-        for (int i = 0; i < HELD / 2; ++i)
-#pragma unroll
-            for (int e = 0; e < NA; ++e) {
-                const float keep = upper ? acc[i + HELD / 2][e] : acc[i][e];
-                const float send = upper ? acc[i][e] : acc[i + HELD / 2][e];
-                acc[i][e] = keep + __shfl_xor_sync(0xffffffffu, send, mask);
-            }
-        if (upper) head0 += HELD / 2;
-    } else {
-#pragma unroll
-        for (int e = 0; e < NA; ++e) acc[0][e] += __shfl_xor_sync(0xffffffffu, acc[0][e], mask);
-        writer = writer && (lane & mask) == 0;
-    }
-}
-
-template <int G>
-__host__ __device__ constexpr int held_after(int levels)
-{
-    return (G >> levels) > 0 ? (G >> levels) : 1;
-}
-
-// Reduce G heads' partial sums and store heads 0 .. nheads - 1 of them, each
-// scaled by `scale`, to out_row0 + 32 s.
-template <typename VT, int G>
-__device__ __forceinline__ void store_heads(float (&acc)[G][Gather<VT>::kAcc], int lane,
-                                            float* __restrict__ out_row0, int nheads,
-                                            float scale = 1.f)
-{
-    constexpr int NA = Gather<VT>::kAcc;
-    constexpr int NM = sizeof(Gather<VT>::kSumMasks) / sizeof(int);
-    int head0 = 0;
-    bool writer = true;
-    reduce_level<held_after<G>(0), G, NA>(acc, Gather<VT>::kSumMasks[0], lane, head0, writer);
-    reduce_level<held_after<G>(1), G, NA>(acc, Gather<VT>::kSumMasks[1], lane, head0, writer);
-    if constexpr (NM > 2)
-        reduce_level<held_after<G>(2), G, NA>(acc, Gather<VT>::kSumMasks[2], lane, head0, writer);
-    constexpr int kHeld = held_after<G>(NM);
-    if (!writer) return;
-    const int c0 = Gather<VT>::channel0(lane);
-#pragma unroll
-    for (int i = 0; i < kHeld; ++i) {
-        const int s = head0 + i;
-        if (s < nheads) {
-            float4* o = reinterpret_cast<float4*>(out_row0 + s * kHeadDim + c0);
-#pragma unroll
-            for (int j = 0; j < NA / 4; ++j)
-                o[j] = make_float4(acc[i][4 * j] * scale, acc[i][4 * j + 1] * scale,
-                                   acc[i][4 * j + 2] * scale, acc[i][4 * j + 3] * scale);
-        }
-    }
-}
 
 // Inputs of one row for HP heads, per lane (samples j = c * 32 + lane): the
 // logits (or weights), the pixel offsets (or locations) and, fused, the
@@ -739,20 +671,6 @@ __device__ __forceinline__ void group_table(int H, int h0, float a, float2 v, fl
     }
 }
 
-// The gathers of heads h0 .. h0 + G - 1 (the first nheads of them) from a
-// filled group table, added to acc[s]; NPL = log2(npad), G = 32 >> NPL.  All
-// heads' loads are straight-line code, so they are in flight together.
-template <typename VT, int NPL>
-__device__ __forceinline__ void group_gather(const VT* __restrict__ vb, const WarpTable& tab,
-                                             int nheads, int lane,
-                                             float (&acc)[32 >> NPL][Gather<VT>::kAcc])
-{
-    constexpr int G = 32 >> NPL, Q = (1 << NPL) / 4;
-#pragma unroll
-    for (int s = 0; s < G; ++s)
-        if (s < nheads) Gather<VT>::template run_quads<Q>(vb, tab, lane, acc[s], s << NPL);
-}
-
 // One row, heads h0 .. h0 + G - 1 (those < H), from the lane's preloaded
 // inputs (see group_table); out_row0: head h0's output (+32 per head).
 template <typename VT, bool FUSED, int NPL>
@@ -764,15 +682,15 @@ __device__ __forceinline__ void group_compute(const VT* __restrict__ vb, int H, 
     constexpr int G = 32 >> NPL;
     group_table<FUSED>(H, h0, a, v, r, valid, gl, tab, lane);
     __syncwarp();
-    float acc[G][Gather<VT>::kAcc];
-#pragma unroll
-    for (int s = 0; s < G; ++s)
-#pragma unroll
-        for (int i = 0; i < Gather<VT>::kAcc; ++i) acc[s][i] = 0.f;
     const int nheads = min(G, H - h0);
-    group_gather<VT, NPL>(vb, tab, nheads, lane, acc);
+    for (int s = 0; s < nheads; ++s) {
+        float acc[Gather<VT>::kAcc];
+#pragma unroll
+        for (int i = 0; i < Gather<VT>::kAcc; ++i) acc[i] = 0.f;
+        Gather<VT>::template run_quads<(1 << NPL) / 4>(vb, tab, lane, acc, s << NPL);
+        Gather<VT>::store(acc, lane, out_row0 + s * kHeadDim);
+    }
     __syncwarp();
-    store_heads<VT, G>(acc, lane, out_row0, nheads);
 }
 
 // Walks the (row, head) items of one warp without divisions: items are

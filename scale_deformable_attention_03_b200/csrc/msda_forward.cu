@@ -89,7 +89,7 @@ msda_forward_kernel(const VT* __restrict__ value, const float* __restrict__ lo,
 // K1g: rows with L*P <= 16, G = 32 / npad heads per warp item (see
 // group_compute).  Items are (row, head group), head groups fastest.
 template <typename VT, bool FUSED, int NPL>
-__global__ void MSDA_GATHER_BOUNDS
+__global__ void MSDA_GROUP_BOUNDS
 msda_forward_group_kernel(const VT* __restrict__ value, const float* __restrict__ lo,
                           const float* __restrict__ wl, const float* __restrict__ ref,
                           float* __restrict__ out, int B, int Nq, int Nv, int H, int L, int P,

@@ -61,20 +61,26 @@ cudaError_t launch_sca_query_major(const Problem& p, const float* ref_cam, const
                                    const float* off, const float* logits, float* out,
                                    cudaStream_t s);
 
-// K4: deterministic camera average.
+// K4: deterministic camera average; fp32 or (out_bf16) bf16 output.
 cudaError_t launch_sca_average(const float* out_rb, const int32_t* pos, const int32_t* hits,
-                               int B, int Ncam, int Nq, int H, float* out, cudaStream_t s);
+                               int B, int Ncam, int Nq, int H, void* out, bool out_bf16,
+                               cudaStream_t s);
 
 // Backward.
 cudaError_t launch_zero(float* p, int64_t n, cudaStream_t s);
+// grad_value_fix non-null: deterministic fixed-point accumulation into it
+// (zeroed by the caller) instead of fp32 reductions into grad_value.
 cudaError_t launch_msda_backward(const Problem& p, const float* loc, const float* attn,
-                                 const float* grad_out, float* grad_value, float* grad_loc,
-                                 float* grad_attn, cudaStream_t s);
+                                 const float* grad_out, float* grad_value,
+                                 long long* grad_value_fix, float* grad_loc, float* grad_attn,
+                                 cudaStream_t s);
 cudaError_t launch_sca_backward_rows(const Problem& p, const float* ref_cam, const float* off,
                                      const float* logits, const float* grad_out,
                                      const int32_t* idx, const int32_t* hits,
                                      const int32_t* count, float* grad_value,
-                                     float* grad_loc_rb, float* grad_attn_rb, cudaStream_t s);
+                                     long long* grad_value_fix, float* grad_loc_rb,
+                                     float* grad_attn_rb, cudaStream_t s);
+cudaError_t launch_fix_to_float(const long long* acc, float* out, int64_t n, cudaStream_t s);
 cudaError_t launch_sca_zero_tail(const int32_t* count, int B, int Ncam, int Nq, int S,
                                  float* grad_loc_rb, float* grad_attn_rb, cudaStream_t s);
 
@@ -95,6 +101,24 @@ cudaError_t launch_tsa_reference(const float* ego, int B, int T, int bev_h, int 
                                  double gy, float* ref, cudaStream_t s);
 cudaError_t launch_tsa_forward(const Problem& p, int T, const float* ref, const float* off,
                                const float* logits, float* out, cudaStream_t s);
+
+// sca_forward with its output stored as fp32 or (out_bf16) bf16; validates
+// like sca_forward.
+msda_status_t sca_forward_to(const void* value, msda_dtype_t vdt, const int64_t* spatial_shapes,
+                             const int64_t* level_start_index, const float* reference_points_cam,
+                             const uint8_t* bev_mask, const float* sampling_offsets,
+                             const float* attention_logits, msda_dims_t d, void* workspace,
+                             size_t workspace_bytes, void* out, bool out_bf16,
+                             cudaStream_t stream);
+
+// sca_rebatched_backward after its input checks (acc: see msda_api.cu).
+msda_status_t sca_rebatched_backward_to(const void* value, msda_dtype_t vdt, const msda_dims_t& d,
+                                        const Levels& lv, const float* reference_points_cam,
+                                        const float* sampling_offsets,
+                                        const float* attention_logits, const float* grad_out,
+                                        const int32_t* idx, const int32_t* count,
+                                        const int32_t* hits, float* grad_value, long long* acc,
+                                        float* grad_loc_rb, float* grad_attn_rb, cudaStream_t s);
 
 // Set the per-thread error message of msda_last_error() and return the code.
 msda_status_t api_fail(msda_status_t code, const char* message);

@@ -5,22 +5,29 @@
 //   Y = X W^T (+ bias) (+ residual),  X [M, K] bf16, W [N, K] bf16 (the
 //   nn.Linear weight layout), fp32 accumulation, Y fp32 or bf16.
 //
-// One CTA computes a 128 x 256 tile of Y on the 5th-generation tensor cores:
-//   - one thread issues the TMA loads of the whole K extent (K <= 256) of the
-//     X tile and the W tile into shared memory, 128-byte swizzled, and waits
-//     on an mbarrier for their bytes;
-//   - the same thread issues tcgen05.mma (M = 128, N = 256, K = 16, bf16 in,
-//     fp32 accumulate) into a 256-column TMEM accumulator, then
-//     tcgen05.commit to a second mbarrier;
-//   - four warps read the accumulator rows back with tcgen05.ld (warp w owns
-//     TMEM lanes 32w..32w+31 = tile rows), add bias and residual and store.
-// Every mbarrier wait is bounded: a wait that gives up counts a timeout in a
-// device word (msda_linear_timeouts), skips the rest of the tile and still
-// frees its TMEM.
+// A persistent, warp-specialised kernel on the 5th-generation tensor cores,
+// one CTA per SM, each walking output tiles of 128 x 256 (N-tile major, so a
+// CTA keeps one N-tile for a run of M-tiles):
+//   - warp 0 (one elected thread) loads the W tile of the whole K extent
+//     (K <= 256) once per run of M-tiles, and streams X in 128 x 64 blocks
+//     through a 4-stage shared-memory ring with TMA (128-byte swizzle);
+//   - warp 1 (one thread) issues tcgen05.mma (M = 128, N = 256, K = 16, bf16
+//     in, fp32 accumulate) into one of two 256-column TMEM accumulators and
+//     commits each ring slot back to the loader and each finished tile to the
+//     epilogue;
+//   - warps 2-5 drain the other accumulator meanwhile: tcgen05.ld of their 32
+//     TMEM lanes (tile rows), bias and residual added, the values written to
+//     a swizzled shared-memory buffer and stored by TMA.
+// So loads, tensor-core work and stores of consecutive tiles overlap.  Every
+// mbarrier wait is bounded: a wait that gives up counts a timeout in a device
+// word (msda_linear_timeouts), raises a CTA-wide stop flag that makes the
+// other roles leave their loops, and the CTA still waits (bounded) for its
+// copies in flight and frees its TMEM.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "msda.h"
@@ -34,10 +41,13 @@ constexpr int kBN = 256;   // tile columns (TMEM columns, fp32)
 constexpr int kBK = 64;    // one 128-byte swizzle row of bf16
 constexpr int kMaxK = 256;
 constexpr int kMaxKBlocks = kMaxK / kBK;
-constexpr int kGemmThreads = 128;
-constexpr uint32_t kABlockBytes = kBM * kBK * 2;  // 16 KB
-constexpr uint32_t kBBlockBytes = kBN * kBK * 2;  // 32 KB
-constexpr uint32_t kSpinLimit = 1u << 24;         // mbarrier polls before giving up
+constexpr int kStages = 4;                          // X ring slots
+constexpr int kGemmThreads = 192;                   // 6 warps
+constexpr uint32_t kABlockBytes = kBM * kBK * 2;    // 16 KB
+constexpr uint32_t kBBlockBytes = kBN * kBK * 2;    // 32 KB
+constexpr uint32_t kCBufBytes = 32 * 128;           // 32 rows x 128 bytes
+constexpr uint32_t kSpinLimit = 1u << 24;           // mbarrier polls before giving up
+constexpr uint64_t kWaitNs = 2000000000ull;         // ... or 2 s of wall time
 
 // Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulator (bits
 // 4-5 = 1), A and B bf16 (bits 7-9 = 1, 10-12 = 1), both K-major (bits 15, 16
@@ -46,14 +56,23 @@ constexpr uint32_t kInstrDesc = (1u << 4) | (1u << 7) | (1u << 10) |
                                 ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
 
 struct __align__(8) Ctrl {
-    uint64_t load_bar;
-    uint64_t mma_bar;
+    uint64_t full[kStages];    // X slot loaded (TMA bytes)
+    uint64_t empty[kStages];   // X slot consumed (tcgen05.commit)
+    uint64_t b_full;           // W tile loaded
+    uint64_t b_free;           // the MMAs of a W tile's run are done
+    uint64_t acc_full[2];      // accumulator ready for the epilogue
+    uint64_t acc_empty[2];     // accumulator drained (4 epilogue warps)
+    uint64_t drain;            // every MMA issued so far has finished (stop path)
     uint32_t tmem_base;
-    int failed;
+    volatile int stop;
 };
 
-constexpr size_t kSmemBytes = 1024 /* alignment slack */ + kMaxKBlocks * (kABlockBytes + kBBlockBytes) +
-                              sizeof(Ctrl);
+// Shared memory: W (K/64 blocks of 256 x 64), the X ring, 4 warps x 2
+// epilogue buffers, then the control block; 1024-byte aligned.
+constexpr size_t kSmemB = (size_t)kMaxKBlocks * kBBlockBytes;   // 128 KB
+constexpr size_t kSmemA = (size_t)kStages * kABlockBytes;       // 64 KB
+constexpr size_t kSmemC = (size_t)4 * 2 * kCBufBytes;           // 32 KB
+constexpr size_t kSmemBytes = 1024 + kSmemB + kSmemA + kSmemC + sizeof(Ctrl);
 
 __device__ unsigned int g_gemm_timeouts = 0;
 
@@ -75,9 +94,19 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes)
                  : "memory");
 }
 
-// Wait for the completion of phase `parity`; false after kSpinLimit polls.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity)
+__device__ __forceinline__ uint64_t global_ns()
 {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for the completion of phase `parity`; false after kSpinLimit polls,
+// after kWaitNs of wall time, or once `stop` is raised (when given).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          const volatile int* stop = nullptr)
+{
+    uint64_t t0 = 0;
     for (uint32_t i = 0; i < kSpinLimit; ++i) {
         uint32_t done;
         asm volatile(
@@ -88,8 +117,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity)
             : "r"(smem_u32(bar)), "r"(parity)
             : "memory");
         if (done) return true;
+        if ((i & 255) == 0) {
+            const uint64_t t = global_ns();
+            if (i == 0) t0 = t;
+            else if (t - t0 > kWaitNs) return false;
+            if (stop && *stop) return false;
+        }
     }
     return false;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
@@ -100,6 +140,29 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
         " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
         : "memory");
+}
+
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int x, int y, const void* src)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(x), "r"(y), "r"(smem_u32(src))
+        : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// Wait until at most N committed store groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read()
+{
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ void fence_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // Shared-memory matrix descriptor of a K-major operand in the 128-byte
@@ -157,30 +220,100 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// Training-time dropout of the projection ("BEV(三) ..." section 12): element
+// e = row * N + col keeps its value when word e mod 4 of Philox4x32-10
+// (Salmon et al., SC 2011) at counter (e div 4, 0, 0) and key `seed` is at
+// least `thr` (= floor(p * 2^32)), scaled by 1 / (1 - p); else it is 0.
+struct Dropout {
+    uint32_t thr;
+    float scale;
+    uint32_t key0, key1;
+    int on;
+};
+
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1)
+{
+#pragma unroll
+    for (int round = 0; round < 10; ++round) {
+        const uint32_t hi0 = __umulhi(0xD2511F53u, c.x), lo0 = 0xD2511F53u * c.x;
+        const uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z), lo1 = 0xCD9E8D57u * c.z;
+        c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+        k0 += 0x9E3779B9u;
+        k1 += 0xBB67AE85u;
+    }
+    return c;
+}
+
+// Dropout of the 32 values v of columns col .. col + 31 of `row`.
+__device__ __forceinline__ void apply_dropout(float (&v)[32], int64_t row, int col, int N,
+                                              const Dropout& d)
+{
+    const uint64_t blk0 = (uint64_t)(row * N + col) >> 2;  // col is a multiple of 32
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint64_t blk = blk0 + i;
+        const uint4 u = philox4x32_10(make_uint4((uint32_t)blk, (uint32_t)(blk >> 32), 0u, 0u),
+                                      d.key0, d.key1);
+        v[4 * i] = u.x >= d.thr ? v[4 * i] * d.scale : 0.f;
+        v[4 * i + 1] = u.y >= d.thr ? v[4 * i + 1] * d.scale : 0.f;
+        v[4 * i + 2] = u.z >= d.thr ? v[4 * i + 2] * d.scale : 0.f;
+        v[4 * i + 3] = u.w >= d.thr ? v[4 * i + 3] * d.scale : 0.f;
+    }
+}
+
+__device__ __forceinline__ void note_timeout(Ctrl& ctrl)
+{
+    if (!ctrl.stop) atomicAdd(&g_gemm_timeouts, 1u);
+    ctrl.stop = 1;
+}
+
+// One 32-row x 128-byte epilogue chunk of thread `lane` (its row) into the
+// 128-byte-swizzled buffer the TMA store reads: 16-byte unit c of row r sits
+// at unit c ^ (r mod 8).
+__device__ __forceinline__ void put_row(uint8_t* buf, int lane, const uint32_t (&u)[32])
+{
+    uint8_t* row = buf + lane * 128;
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(row + ((c ^ (lane & 7)) << 4)) =
+            make_uint4(u[4 * c], u[4 * c + 1], u[4 * c + 2], u[4 * c + 3]);
+}
+
 __global__ void __launch_bounds__(kGemmThreads, 1)
 proj_gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
-                 const float* __restrict__ bias, const float* __restrict__ residual,
-                 void* __restrict__ y, int y_bf16, int M, int N, int K)
+                 const __grid_constant__ CUtensorMap map_y, const float* __restrict__ bias,
+                 const float* __restrict__ residual, int y_bf16, int M, int N, int K, Dropout drop)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    uint8_t* sa = smem;                                 // K/64 blocks of 128 x 64 bf16
-    uint8_t* sb = smem + kMaxKBlocks * kABlockBytes;    // K/64 blocks of 256 x 64 bf16
-    Ctrl& ctrl = *reinterpret_cast<Ctrl*>(sb + kMaxKBlocks * kBBlockBytes);
+    uint8_t* sb = smem;
+    uint8_t* sa = sb + kSmemB;
+    uint8_t* sc = sa + kSmemA;
+    Ctrl& ctrl = *reinterpret_cast<Ctrl*>(sc + kSmemC);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.x * kBM, n0 = blockIdx.y * kBN;
     const int kblocks = K / kBK;
+    const int mt = (M + kBM - 1) / kBM;
+    const int ntiles = mt * (N / kBN);
 
     if (threadIdx.x == 0) {
-        mbar_init(&ctrl.load_bar, 1);
-        mbar_init(&ctrl.mma_bar, 1);
-        ctrl.failed = 0;
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&ctrl.full[i], 1);
+            mbar_init(&ctrl.empty[i], 1);
+        }
+        mbar_init(&ctrl.b_full, 1);
+        mbar_init(&ctrl.b_free, 1);
+        mbar_init(&ctrl.drain, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&ctrl.acc_full[i], 1);
+            mbar_init(&ctrl.acc_empty[i], 4);
+        }
+        ctrl.stop = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(&ctrl.tmem_base)),
-                     "r"(kBN)
+                     "r"(2 * kBN)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
@@ -189,87 +322,183 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = ctrl.tmem_base;
 
-    if (threadIdx.x == 0) {
-        mbar_expect_tx(&ctrl.load_bar, (uint32_t)kblocks * (kABlockBytes + kBBlockBytes));
-        for (int kb = 0; kb < kblocks; ++kb) {
-            tma_load_2d(sa + kb * kABlockBytes, &map_x, kb * kBK, m0, &ctrl.load_bar);
-            tma_load_2d(sb + kb * kBBlockBytes, &map_w, kb * kBK, n0, &ctrl.load_bar);
-        }
-        if (mbar_wait(&ctrl.load_bar, 0)) {
-            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            for (int kb = 0; kb < kblocks; ++kb)
-                for (int ks = 0; ks < kBK / 16; ++ks) {
-                    const uint64_t ad = smem_desc_sw128(smem_u32(sa + kb * kABlockBytes) + ks * 32);
-                    const uint64_t bd = smem_desc_sw128(smem_u32(sb + kb * kBBlockBytes) + ks * 32);
-                    umma_bf16(tmem, ad, bd, (kb | ks) != 0);
-                }
-            umma_commit(&ctrl.mma_bar);
-        } else {
-            ctrl.failed = 1;
-            atomicAdd(&g_gemm_timeouts, 1u);
-            mbar_wait(&ctrl.load_bar, 0);  // give copies still in flight a last chance
-        }
-    }
-    __syncthreads();
-    bool ok = !ctrl.failed;
-    if (ok) ok = mbar_wait(&ctrl.mma_bar, 0);
-    if (!ok && threadIdx.x == 0 && !ctrl.failed) atomicAdd(&g_gemm_timeouts, 1u);
-    ok = __all_sync(0xffffffffu, ok);
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-
-    if (ok) {
-        const int row = m0 + warp * 32 + lane;
-        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-        for (int c0 = 0; c0 < kBN; c0 += 32) {
-            uint32_t r[32];
-            tmem_ld32(lane_base + (uint32_t)c0, r);
-            if (row < M) {
-                const int col0 = n0 + c0;
-                float v[32];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-                if (bias) {
-#pragma unroll
-                    for (int j = 0; j < 32; j += 4) {
-                        const float4 b4 = __ldg(reinterpret_cast<const float4*>(bias + col0 + j));
-                        v[j] += b4.x; v[j + 1] += b4.y; v[j + 2] += b4.z; v[j + 3] += b4.w;
+    if (warp == 0) {
+        // ---- loader ----
+        if (lane == 0) {
+            int stage = 0, cur_n = -1, b_loads = 0;
+            uint32_t phase = 0, free_phase = 0;
+            int issued[kStages];  // parity of each slot's last load, -1 = none
+            for (int i = 0; i < kStages; ++i) issued[i] = -1;
+            for (int tile = blockIdx.x; tile < ntiles && !ctrl.stop; tile += gridDim.x) {
+                const int m0 = (tile % mt) * kBM, n_tile = tile / mt;
+                if (n_tile != cur_n) {
+                    if (cur_n >= 0) {
+                        if (!mbar_wait(&ctrl.b_free, free_phase, &ctrl.stop)) {
+                            note_timeout(ctrl);
+                            break;
+                        }
+                        free_phase ^= 1;
                     }
+                    mbar_expect_tx(&ctrl.b_full, (uint32_t)kblocks * kBBlockBytes);
+                    for (int kb = 0; kb < kblocks; ++kb)
+                        tma_load_2d(sb + kb * kBBlockBytes, &map_w, kb * kBK, n_tile * kBN,
+                                    &ctrl.b_full);
+                    ++b_loads;
+                    cur_n = n_tile;
                 }
-                if (residual) {
-                    const float4* rp =
-                        reinterpret_cast<const float4*>(residual + (int64_t)row * N + col0);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const float4 q = __ldcs(rp + j);
-                        v[4 * j] += q.x; v[4 * j + 1] += q.y; v[4 * j + 2] += q.z; v[4 * j + 3] += q.w;
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(&ctrl.empty[stage], phase ^ 1, &ctrl.stop)) {
+                        note_timeout(ctrl);
+                        break;
                     }
-                }
-                if (y_bf16) {
-                    uint4* yp = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(y) +
-                                                         (int64_t)row * N + col0);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        uint4 u;
-                        u.x = pack_bf16x2(v[8 * j], v[8 * j + 1]);
-                        u.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
-                        u.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
-                        u.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
-                        __stcs(yp + j, u);
+                    mbar_expect_tx(&ctrl.full[stage], kABlockBytes);
+                    tma_load_2d(sa + stage * kABlockBytes, &map_x, kb * kBK, m0, &ctrl.full[stage]);
+                    issued[stage] = (int)phase;
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1;
                     }
-                } else {
-                    float4* yp = reinterpret_cast<float4*>(static_cast<float*>(y) + (int64_t)row * N + col0);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        __stcs(yp + j, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
                 }
             }
+            // On a stop, give the copies still in flight a bounded chance to land.
+            if (ctrl.stop) {
+                for (int i = 0; i < kStages; ++i)
+                    if (issued[i] >= 0) mbar_wait(&ctrl.full[i], (uint32_t)issued[i]);
+                if (b_loads > 0) mbar_wait(&ctrl.b_full, (uint32_t)((b_loads - 1) & 1));
+            }
         }
+    } else if (warp == 1) {
+        // ---- tensor-core issuer ----
+        if (lane == 0) {
+            int stage = 0, acc = 0, cur_n = -1;
+            uint32_t phase = 0, acc_phase = 0, b_phase = 0;
+            for (int tile = blockIdx.x; tile < ntiles && !ctrl.stop; tile += gridDim.x) {
+                const int n_tile = tile / mt;
+                if (n_tile != cur_n) {
+                    if (!mbar_wait(&ctrl.b_full, b_phase, &ctrl.stop)) {
+                        note_timeout(ctrl);
+                        break;
+                    }
+                    b_phase ^= 1;
+                    cur_n = n_tile;
+                }
+                if (!mbar_wait(&ctrl.acc_empty[acc], acc_phase ^ 1, &ctrl.stop)) {
+                    note_timeout(ctrl);
+                    break;
+                }
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                const uint32_t d = tmem + (uint32_t)(acc * kBN);
+                bool ok = true;
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(&ctrl.full[stage], phase, &ctrl.stop)) {
+                        note_timeout(ctrl);
+                        ok = false;
+                        break;
+                    }
+                    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+#pragma unroll
+                    for (int ks = 0; ks < kBK / 16; ++ks) {
+                        const uint64_t ad = smem_desc_sw128(smem_u32(sa + stage * kABlockBytes) + ks * 32);
+                        const uint64_t bd = smem_desc_sw128(smem_u32(sb + kb * kBBlockBytes) + ks * 32);
+                        umma_bf16(d, ad, bd, (kb | ks) != 0);
+                    }
+                    umma_commit(&ctrl.empty[stage]);  // the slot is free once these MMAs finish
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+                if (!ok) break;
+                umma_commit(&ctrl.acc_full[acc]);
+                const int next = tile + gridDim.x;
+                if (next < ntiles && next / mt != n_tile) umma_commit(&ctrl.b_free);
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1;
+            }
+            if (ctrl.stop) {  // TMEM is freed below: let issued MMAs finish first
+                umma_commit(&ctrl.drain);
+                mbar_wait(&ctrl.drain, 0);
+            }
+        }
+    } else {
+        // ---- epilogue: warps 2..5, TMEM lane quarter q = warp % 4 ----
+        const int q = warp & 3;
+        uint8_t* cbuf = sc + (size_t)q * 2 * kCBufBytes;
+        int acc = 0, buf = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+            const int m0 = (tile % mt) * kBM, n0 = (tile / mt) * kBN;
+            if (!mbar_wait(&ctrl.acc_full[acc], acc_phase, &ctrl.stop)) {
+                if (lane == 0) note_timeout(ctrl);
+                break;
+            }
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            const int row = m0 + q * 32 + lane;
+            const bool row_ok = row < M;
+            const bool block_ok = m0 + q * 32 < M;
+            const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kBN);
+            const int cols = y_bf16 ? 64 : 32;  // columns per 128-byte store row
+            for (int c0 = 0; c0 < kBN; c0 += cols) {
+                uint32_t u[32];
+                for (int half = 0; half < cols / 32; ++half) {
+                    uint32_t r[32];
+                    tmem_ld32(taddr + (uint32_t)(c0 + 32 * half), r);
+                    float v[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+                    const int col = n0 + c0 + 32 * half;
+                    if (bias) {
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4) {
+                            const float4 b4 = __ldg(reinterpret_cast<const float4*>(bias + col + j));
+                            v[j] += b4.x; v[j + 1] += b4.y; v[j + 2] += b4.z; v[j + 3] += b4.w;
+                        }
+                    }
+                    if (drop.on) apply_dropout(v, row, col, N, drop);
+                    if (residual && row_ok) {
+                        const float4* rp = reinterpret_cast<const float4*>(residual + (int64_t)row * N + col);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const float4 t = __ldcs(rp + j);
+                            v[4 * j] += t.x; v[4 * j + 1] += t.y; v[4 * j + 2] += t.z; v[4 * j + 3] += t.w;
+                        }
+                    }
+                    if (y_bf16) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) u[16 * half + j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) u[j] = __float_as_uint(v[j]);
+                    }
+                }
+                // the buffer written two chunks ago must have been read by its store
+                if (lane == 0) bulk_wait_read<1>();
+                __syncwarp();
+                uint8_t* b = cbuf + buf * kCBufBytes;
+                put_row(b, lane, u);
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0 && block_ok) {
+                    tma_store_2d(&map_y, n0 + c0, m0 + q * 32, b);
+                    bulk_commit();
+                }
+                buf ^= 1;
+            }
+            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctrl.acc_empty[acc]);
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1;
+        }
+        if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+        __syncwarp();
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
     if (warp == 0) {
+        __syncwarp();
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kBN)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * kBN)
                      : "memory");
     }
 }
@@ -309,14 +538,34 @@ bool make_map(CUtensorMap* map, const void* base, int rows, int K, int box_rows)
            CUDA_SUCCESS;
 }
 
+// Y [M, N] (fp32 or bf16) written in boxes of 32 rows x 128 bytes.
+bool make_store_map(CUtensorMap* map, void* base, int M, int N, bool bf16)
+{
+    EncodeTiled enc = encode_tiled();
+    if (enc == nullptr) return false;
+    const int elem = bf16 ? 2 : 4;
+    const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+    const cuuint64_t strides[1] = {(cuuint64_t)N * elem};
+    const cuuint32_t box[2] = {(cuuint32_t)(128 / elem), 32};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+               base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 }  // namespace msda
 
-extern "C" msda_status_t msda_linear(const void* x, const void* w, const float* bias,
-                                     const float* residual, int32_t M, int32_t N, int32_t K,
-                                     msda_dtype_t y_dtype, void* y, msda_stream_t stream)
+extern "C" msda_status_t msda_linear_dropout(const void* x, const void* w, const float* bias,
+                                             const float* residual, int32_t M, int32_t N,
+                                             int32_t K, msda_dtype_t y_dtype, void* y,
+                                             float dropout_p, uint64_t dropout_seed,
+                                             msda_stream_t stream)
 {
     using namespace msda;
+    if (!(dropout_p >= 0.f && dropout_p < 1.f))
+        return api_fail(MSDA_ERR_INVALID_ARG, "dropout_p must be in [0, 1)");
     if (M < 0) return api_fail(MSDA_ERR_INVALID_ARG, "M must be >= 0");
     if (N < kBN || N % kBN != 0)
         return api_fail(MSDA_ERR_UNSUPPORTED, "N must be a positive multiple of 256");
@@ -330,8 +579,9 @@ extern "C" msda_status_t msda_linear(const void* x, const void* w, const float* 
         return api_fail(MSDA_ERR_INVALID_ARG, "x, w and y must be non-null and 16-byte aligned");
     if ((bias && ((uintptr_t)bias & 15)) || (residual && ((uintptr_t)residual & 15)))
         return api_fail(MSDA_ERR_INVALID_ARG, "bias and residual must be 16-byte aligned");
-    CUtensorMap mx, mw;
-    if (!make_map(&mx, x, M, K, kBM) || !make_map(&mw, w, N, K, kBN))
+    CUtensorMap mx, mw, my;
+    if (!make_map(&mx, x, M, K, kBM) || !make_map(&mw, w, N, K, kBN) ||
+        !make_store_map(&my, y, M, N, y_dtype == MSDA_BF16))
         return api_fail(MSDA_ERR_CUDA, "cuTensorMapEncodeTiled failed or is unavailable");
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
@@ -340,10 +590,24 @@ extern "C" msda_status_t msda_linear(const void* x, const void* w, const float* 
                                         (int)kSmemBytes);
     });
     if (attr_err != cudaSuccess) return api_cuda(attr_err, "msda_linear: shared memory size");
-    const dim3 grid((unsigned)((M + kBM - 1) / kBM), (unsigned)(N / kBN));
+    const int64_t ntiles = (int64_t)((M + kBM - 1) / kBM) * (N / kBN);
+    const unsigned grid = (unsigned)std::min<int64_t>(ntiles, device_sm_count());
+    Dropout drop;
+    drop.on = dropout_p > 0.f;
+    drop.thr = (uint32_t)((double)dropout_p * 4294967296.0);
+    drop.scale = (float)(1.0 / (1.0 - (double)dropout_p));
+    drop.key0 = (uint32_t)dropout_seed;
+    drop.key1 = (uint32_t)(dropout_seed >> 32);
     proj_gemm_kernel<<<grid, kGemmThreads, kSmemBytes, (cudaStream_t)stream>>>(
-        mx, mw, bias, residual, y, y_dtype == MSDA_BF16, M, N, K);
+        mx, mw, my, bias, residual, y_dtype == MSDA_BF16, M, N, K, drop);
     return api_cuda(cudaGetLastError(), "msda_linear");
+}
+
+extern "C" msda_status_t msda_linear(const void* x, const void* w, const float* bias,
+                                     const float* residual, int32_t M, int32_t N, int32_t K,
+                                     msda_dtype_t y_dtype, void* y, msda_stream_t stream)
+{
+    return msda_linear_dropout(x, w, bias, residual, M, N, K, y_dtype, y, 0.f, 0, stream);
 }
 
 extern "C" uint32_t msda_linear_timeouts(void)

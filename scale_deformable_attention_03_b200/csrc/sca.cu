@@ -294,11 +294,13 @@ constexpr int kAvgWarps = 8;
 
 // PL: float4 per lane (a power of two >= row4 / 32); rows of up to 16 heads.
 // kAvgBatch cameras' rows are loaded together (8 float4 per lane in flight).
-template <int PL>
+// BF16: the mean is stored rounded to bf16 (to nearest even), the operand
+// type of the output projection that follows it in the SCA module.
+template <int PL, bool BF16>
 __global__ void __launch_bounds__(kAvgWarps * 32)
 sca_average_kernel(const float4* __restrict__ out_rb, const int32_t* __restrict__ pos,
                    const int32_t* __restrict__ hits, int B, int Ncam, int Nq, int row4,
-                   float4* __restrict__ out)
+                   void* __restrict__ out)
 {
     constexpr int kAvgBatch = PL >= 8 ? 1 : 8 / PL;
     const int lane = threadIdx.x & 31;
@@ -344,26 +346,40 @@ sca_average_kernel(const float4* __restrict__ out_rb, const int32_t* __restrict_
 #pragma unroll
     for (int e = 0; e < PL; ++e) {
         const int v4 = lane + 32 * e;
-        if (v4 < row4)
-            __stcs(out + bq * row4 + v4,
-                   make_float4(acc[e].x / n, acc[e].y / n, acc[e].z / n, acc[e].w / n));
+        if (v4 < row4) {
+            const float4 m = make_float4(acc[e].x / n, acc[e].y / n, acc[e].z / n, acc[e].w / n);
+            if constexpr (BF16) {
+                const __nv_bfloat162 lo = __floats2bfloat162_rn(m.x, m.y);
+                const __nv_bfloat162 hi = __floats2bfloat162_rn(m.z, m.w);
+                uint2 u;
+                u.x = *reinterpret_cast<const uint32_t*>(&lo);
+                u.y = *reinterpret_cast<const uint32_t*>(&hi);
+                __stcs(static_cast<uint2*>(out) + bq * row4 + v4, u);
+            } else {
+                __stcs(static_cast<float4*>(out) + bq * row4 + v4, m);
+            }
+        }
     }
 }
 
 cudaError_t launch_sca_average(const float* out_rb, const int32_t* pos, const int32_t* hits,
-                               int B, int Ncam, int Nq, int H, float* out, cudaStream_t s)
+                               int B, int Ncam, int Nq, int H, void* out, bool out_bf16,
+                               cudaStream_t s)
 {
     const int row4 = H * kHeadDim / 4;
     const int64_t rows = (int64_t)B * Nq;
     if (rows == 0) return cudaSuccess;
     const unsigned grid = (unsigned)((rows + kAvgWarps - 1) / kAvgWarps);
     const float4* in = reinterpret_cast<const float4*>(out_rb);
-    float4* o = reinterpret_cast<float4*>(out);
     const int pl = (row4 + 31) / 32;
 #define SCA_AVG_CASE(PLV)                                                                        \
     if (pl <= PLV) {                                                                             \
-        sca_average_kernel<PLV><<<grid, kAvgWarps * 32, 0, s>>>(in, pos, hits, B, Ncam, Nq,      \
-                                                                row4, o);                        \
+        if (out_bf16)                                                                            \
+            sca_average_kernel<PLV, true><<<grid, kAvgWarps * 32, 0, s>>>(in, pos, hits, B,      \
+                                                                          Ncam, Nq, row4, out);  \
+        else                                                                                     \
+            sca_average_kernel<PLV, false><<<grid, kAvgWarps * 32, 0, s>>>(in, pos, hits, B,     \
+                                                                           Ncam, Nq, row4, out); \
         return cudaGetLastError();                                                               \
     }
     SCA_AVG_CASE(1)

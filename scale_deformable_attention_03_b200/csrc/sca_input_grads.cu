@@ -7,6 +7,8 @@
 //   grad_offsets[q, h, l, k]  = sum_c grad_loc_rb[c, pos_c(q), h, l, k] / (W_l, H_l)
 //   grad_logits[q, h, :]      = alpha * (G - <alpha, G>),  G = sum_c grad_attn_rb[...]
 //   grad_ref_cam[c, q, m]     = sum over (h, l, k) with k mod R = m of grad_loc_rb
+// The long sums (the reference points' H*L*P/R terms, <alpha, G>) are formed
+// in double: their terms may cancel.
 #include <cuda_runtime.h>
 
 #include "msda.h"
@@ -17,14 +19,30 @@ namespace {
 
 constexpr int kIgWarps = 8;
 
-// One warp per (batch, query); heads in turn; lanes over the L*P samples.
-template <int NC>
+__device__ __forceinline__ double warp_sum_f64(double v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// One warp per (batch, query); lanes over the L*P samples; heads in chunks
+// of kIgHeads whose loads are issued together (they are independent).
+// REF (all heads in one chunk, R dividing 32): the same pass also forms the
+// reference-point gradients of every camera: sample j of a head has the
+// anchor (j mod P) mod R = j mod R, which is lane mod R for every chunk, so a
+// lane sums its samples over the heads and a butterfly over the lanes of one
+// anchor finishes each camera's sums.
+constexpr int kIgHeads = 8;
+
+template <int NC, bool REF>
 __global__ void __launch_bounds__(kIgWarps * 32)
 sca_offset_logit_grads_kernel(const float* __restrict__ logits, const int32_t* __restrict__ pos,
                               const float* __restrict__ grad_loc_rb,
                               const float* __restrict__ grad_attn_rb, int B, int Ncam, int Nq,
-                              int H, int L, int P, Levels levels, float* __restrict__ grad_off,
-                              float* __restrict__ grad_logits)
+                              int H, int L, int P, int R, Levels levels,
+                              float* __restrict__ grad_off, float* __restrict__ grad_logits,
+                              float* __restrict__ grad_ref_cam)
 {
     __shared__ SmemLevels s_lv;
     stage_levels(s_lv, levels);
@@ -36,66 +54,104 @@ sca_offset_logit_grads_kernel(const float* __restrict__ logits, const int32_t* _
     const int n = L * P, S = H * n;
     const int p = lane < Ncam ? __ldg(pos + ((int64_t)b * Ncam + lane) * Nq + q) : -1;
     const unsigned seen = __ballot_sync(0xffffffffu, p >= 0);
+    if (REF) {  // the cameras that do not see the query get zero reference gradients
+        for (int i = lane; i < Ncam * R * 2; i += 32) {
+            const int c = i / (2 * R);
+            if (!((seen >> c) & 1u))
+                grad_ref_cam[(((int64_t)c * B + b) * Nq + q) * R * 2 + (i - c * 2 * R)] = 0.f;
+        }
+    }
     float wl[NC], hl[NC];
+    bool in[NC];
 #pragma unroll
     for (int c = 0; c < NC; ++c) {
         const int j = c * 32 + lane;
-        const int l = j < n ? j / P : 0;
+        in[c] = j < n;
+        const int l = in[c] ? j / P : 0;
         wl[c] = (float)s_lv.w[l];
         hl[c] = (float)s_lv.h[l];
     }
-    for (int h = 0; h < H; ++h) {
-        float G[NC], gx[NC], gy[NC];
+    for (int h0 = 0; h0 < H; h0 += kIgHeads) {
+        const int nh = min(kIgHeads, H - h0);
+        float G[kIgHeads][NC], gx[kIgHeads][NC], gy[kIgHeads][NC];
 #pragma unroll
-        for (int c = 0; c < NC; ++c) G[c] = gx[c] = gy[c] = 0.f;
+        for (int hh = 0; hh < kIgHeads; ++hh)
+#pragma unroll
+            for (int c = 0; c < NC; ++c) G[hh][c] = gx[hh][c] = gy[hh][c] = 0.f;
         unsigned cams = seen;
         while (cams) {
             const int cam = __ffs(cams) - 1;  // ascending camera order
             cams &= cams - 1;
             const int row = __shfl_sync(0xffffffffu, p, cam);
-            const int64_t r = (((int64_t)b * Ncam + cam) * Nq + row) * S + (int64_t)h * n;
+            const int64_t r = (((int64_t)b * Ncam + cam) * Nq + row) * S + (int64_t)h0 * n;
+            double rx = 0.0, ry = 0.0;
 #pragma unroll
-            for (int c = 0; c < NC; ++c) {
-                const int j = c * 32 + lane;
-                if (j < n) {
-                    G[c] += __ldcs(grad_attn_rb + r + j);
-                    const float2 v = __ldcs(reinterpret_cast<const float2*>(grad_loc_rb) + r + j);
-                    gx[c] += v.x;
-                    gy[c] += v.y;
+            for (int hh = 0; hh < kIgHeads; ++hh)
+#pragma unroll
+                for (int c = 0; c < NC; ++c) {
+                    const int j = c * 32 + lane;
+                    if (hh < nh && in[c]) {
+                        G[hh][c] += __ldcs(grad_attn_rb + r + hh * n + j);
+                        const float2 v =
+                            __ldcs(reinterpret_cast<const float2*>(grad_loc_rb) + r + hh * n + j);
+                        gx[hh][c] += v.x;
+                        gy[hh][c] += v.y;
+                        if (REF) {
+                            rx += v.x;
+                            ry += v.y;
+                        }
+                    }
+                }
+            if (REF) {
+                for (int o = 16; o >= R; o >>= 1) {
+                    rx += __shfl_xor_sync(0xffffffffu, rx, o);
+                    ry += __shfl_xor_sync(0xffffffffu, ry, o);
+                }
+                if (lane < R) {
+                    float* out = grad_ref_cam + (((int64_t)cam * B + b) * Nq + q) * R * 2;
+                    out[2 * lane] = (float)rx;
+                    out[2 * lane + 1] = (float)ry;
                 }
             }
         }
-        const int64_t o = bq * S + (int64_t)h * n;
-        float a[NC];
-        float m = -INFINITY;
+        float a[kIgHeads][NC];
 #pragma unroll
-        for (int c = 0; c < NC; ++c) {
-            const int j = c * 32 + lane;
-            a[c] = j < n ? __ldg(logits + o + j) : -INFINITY;
-            m = fmaxf(m, a[c]);
-        }
-        m = warp_max(m);
-        float z = 0.f;
+        for (int hh = 0; hh < kIgHeads; ++hh)
 #pragma unroll
-        for (int c = 0; c < NC; ++c) {
-            const int j = c * 32 + lane;
-            a[c] = j < n ? expf(a[c] - m) : 0.f;
-            z += a[c];
-        }
-        z = warp_sum(z);
-        float dot = 0.f;
+            for (int c = 0; c < NC; ++c)
+                a[hh][c] = (hh < nh && in[c])
+                               ? __ldg(logits + bq * S + (int64_t)(h0 + hh) * n + c * 32 + lane)
+                               : -INFINITY;
 #pragma unroll
-        for (int c = 0; c < NC; ++c) {
-            a[c] = a[c] / z;
-            dot += a[c] * G[c];
-        }
-        dot = warp_sum(dot);
+        for (int hh = 0; hh < kIgHeads; ++hh) {
+            if (hh >= nh) break;  // warp-uniform
+            float m = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < NC; ++c) {
-            const int j = c * 32 + lane;
-            if (j < n) {
-                grad_logits[o + j] = a[c] * (G[c] - dot);
-                reinterpret_cast<float2*>(grad_off)[o + j] = make_float2(gx[c] / wl[c], gy[c] / hl[c]);
+            for (int c = 0; c < NC; ++c) m = fmaxf(m, a[hh][c]);
+            m = warp_max(m);
+            float z = 0.f;
+#pragma unroll
+            for (int c = 0; c < NC; ++c) {
+                a[hh][c] = in[c] ? expf(a[hh][c] - m) : 0.f;
+                z += a[hh][c];
+            }
+            z = warp_sum(z);
+            double dot = 0.0;
+#pragma unroll
+            for (int c = 0; c < NC; ++c) {
+                a[hh][c] = a[hh][c] / z;
+                dot += (double)a[hh][c] * (double)G[hh][c];
+            }
+            dot = warp_sum_f64(dot);
+            const int64_t o = bq * S + (int64_t)(h0 + hh) * n;
+#pragma unroll
+            for (int c = 0; c < NC; ++c) {
+                const int j = c * 32 + lane;
+                if (in[c]) {
+                    grad_logits[o + j] = (float)((double)a[hh][c] * ((double)G[hh][c] - dot));
+                    reinterpret_cast<float2*>(grad_off)[o + j] =
+                        make_float2(gx[hh][c] / wl[c], gy[hh][c] / hl[c]);
+                }
             }
         }
     }
@@ -122,9 +178,28 @@ sca_reference_grads_kernel(const int32_t* __restrict__ pos, const float* __restr
     }
     const float2* g = reinterpret_cast<const float2*>(grad_loc_rb) +
                       (((int64_t)b * Ncam + c) * Nq + p) * S;
-    float sx[MSDA_MAX_POINTS], sy[MSDA_MAX_POINTS];
+    if (32 % R == 0) {
+        // sample e has anchor (e mod P) mod R = e mod R (R divides P, which
+        // divides L*P): lane + 32 i has the anchor lane mod R for every i
+        double ax = 0.0, ay = 0.0;
+        for (int e = lane; e < S; e += 32) {
+            const float2 v = __ldcs(g + e);
+            ax += v.x;
+            ay += v.y;
+        }
+        for (int o = 16; o >= R; o >>= 1) {
+            ax += __shfl_xor_sync(0xffffffffu, ax, o);
+            ay += __shfl_xor_sync(0xffffffffu, ay, o);
+        }
+        if (lane < R) {
+            out[2 * lane] = (float)ax;
+            out[2 * lane + 1] = (float)ay;
+        }
+        return;
+    }
+    double sx[MSDA_MAX_POINTS], sy[MSDA_MAX_POINTS];
 #pragma unroll
-    for (int m = 0; m < MSDA_MAX_POINTS; ++m) sx[m] = sy[m] = 0.f;
+    for (int m = 0; m < MSDA_MAX_POINTS; ++m) sx[m] = sy[m] = 0.0;
     for (int e = lane; e < S; e += 32) {
         const float2 v = __ldcs(g + e);
         const int m = (e % P) % R;
@@ -138,10 +213,10 @@ sca_reference_grads_kernel(const int32_t* __restrict__ pos, const float* __restr
 #pragma unroll
     for (int m = 0; m < MSDA_MAX_POINTS; ++m) {
         if (m < R) {  // warp-uniform
-            const float x = warp_sum(sx[m]), y = warp_sum(sy[m]);
+            const double x = warp_sum_f64(sx[m]), y = warp_sum_f64(sy[m]);
             if (lane == 0) {
-                out[2 * m] = x;
-                out[2 * m + 1] = y;
+                out[2 * m] = (float)x;
+                out[2 * m + 1] = (float)y;
             }
         }
     }
@@ -159,11 +234,17 @@ cudaError_t launch_sca_input_grads(const float* logits, const int32_t* pos,
     if (rows == 0) return cudaSuccess;
     const unsigned grid = (unsigned)((rows + kIgWarps - 1) / kIgWarps);
     const int nc = (L * P + 31) / 32;
+    const bool fused = H <= kIgHeads && 32 % R == 0;
 #define IG_CASE(NCV)                                                                             \
     case NCV:                                                                                    \
-        sca_offset_logit_grads_kernel<NCV><<<grid, kIgWarps * 32, 0, s>>>(                       \
-            logits, pos, grad_loc_rb, grad_attn_rb, B, Ncam, Nq, H, L, P, lv, grad_off,          \
-            grad_logits);                                                                        \
+        if (fused)                                                                               \
+            sca_offset_logit_grads_kernel<NCV, true><<<grid, kIgWarps * 32, 0, s>>>(             \
+                logits, pos, grad_loc_rb, grad_attn_rb, B, Ncam, Nq, H, L, P, R, lv, grad_off,   \
+                grad_logits, grad_ref_cam);                                                      \
+        else                                                                                     \
+            sca_offset_logit_grads_kernel<NCV, false><<<grid, kIgWarps * 32, 0, s>>>(            \
+                logits, pos, grad_loc_rb, grad_attn_rb, B, Ncam, Nq, H, L, P, R, lv, grad_off,   \
+                grad_logits, grad_ref_cam);                                                      \
         break;
     switch (nc) {
         IG_CASE(1)
@@ -173,6 +254,7 @@ cudaError_t launch_sca_input_grads(const float* logits, const int32_t* pos,
         default: return cudaErrorInvalidValue;
     }
 #undef IG_CASE
+    if (fused) return cudaGetLastError();
     const int64_t crows = (int64_t)Ncam * B * Nq;
     sca_reference_grads_kernel<<<(unsigned)((crows + kIgWarps - 1) / kIgWarps), kIgWarps * 32, 0,
                                  s>>>(pos, grad_loc_rb, B, Ncam, Nq, H * L * P, P, R, grad_ref_cam);

@@ -6,10 +6,12 @@
 //   V     = F~ W_v^T + b_v               (section 3; tensor cores)
 //   Delta = q~ W_Delta^T + b_Delta       (4.1)
 //   a     = q~ W_alpha^T + b_alpha       (4.2)
-//   g     = SCA(V, Delta, a, rho, mask)  (5-10: compaction, fused MSDA, average)
-//   q_hat = q + (bf16(g) W_o^T + b_o)    (11-13; dropout is the identity)
-// It composes the library's own entry points; the only new kernels are the
-// two element-wise conversions below.
+//   g     = SCA(V, Delta, a, rho, mask)  (5-10: compaction, fused MSDA, average;
+//                                         the average stores g as bf16)
+//   q_hat = q + dropout(g W_o^T + b_o)   (11-13; dropout in the projection's
+//                                         epilogue, the identity when p = 0)
+// It composes the library's own kernels; the only new one is the element-wise
+// q + pos conversion below.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -62,7 +64,6 @@ struct ModuleWs {
     void* value;       // [B * Ncam * Nv, C] value dtype
     float* offsets;    // [B * Nq, H L P 2]
     float* logits;     // [B * Nq, H L P]
-    float* g;          // [B * Nq, C]
     void* g16;         // [B * Nq, C] bf16
     void* sca;         // sca_forward workspace
     size_t sca_bytes;
@@ -85,7 +86,6 @@ ModuleWs module_carve(void* base, const msda_dims_t& d, msda_dtype_t vdt)
     w.value = take(rows_v * C * (vdt == MSDA_BF16 ? 2 : 4));
     w.offsets = reinterpret_cast<float*>(take(rows_q * S * 2 * 4));
     w.logits = reinterpret_cast<float*>(take(rows_q * S * 4));
-    w.g = reinterpret_cast<float*>(take(rows_q * C * 4));
     w.g16 = take(rows_q * C * 2);
     w.sca_bytes = msda_workspace_size(d);
     w.sca = take(w.sca_bytes);
@@ -140,12 +140,10 @@ extern "C" msda_status_t sca_module_forward(const sca_module_params_t* p,
     if ((st = msda_linear(w.qt, p->w_weights, p->b_weights, nullptr, (int32_t)rows_q, S, C,
                           MSDA_F32, w.logits, stream)) != MSDA_OK)
         return st;
-    if ((st = sca_forward(w.value, p->value_dtype, spatial_shapes, level_start_index,
-                          p->reference_points_cam, p->bev_mask, w.offsets, w.logits, d, w.sca,
-                          w.sca_bytes, w.g, stream)) != MSDA_OK)
+    if ((st = sca_forward_to(w.value, p->value_dtype, spatial_shapes, level_start_index,
+                             p->reference_points_cam, p->bev_mask, w.offsets, w.logits, d, w.sca,
+                             w.sca_bytes, w.g16, true, s)) != MSDA_OK)
         return st;
-    e = launch_add_to_bf16(w.g, nullptr, w.g16, rows_q * C, s);
-    if (e != cudaSuccess) return api_cuda(e, "sca_module_forward: g to bf16");
-    return msda_linear(w.g16, p->w_output, p->b_output, p->query, (int32_t)rows_q, C, C, MSDA_F32,
-                       q_hat, stream);
+    return msda_linear_dropout(w.g16, p->w_output, p->b_output, p->query, (int32_t)rows_q, C, C,
+                               MSDA_F32, q_hat, p->dropout_p, p->dropout_seed, stream);
 }

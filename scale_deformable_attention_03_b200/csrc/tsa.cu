@@ -65,7 +65,7 @@ __device__ __forceinline__ void scale_acc(float (&acc)[NA], float f)
 // group); the warp builds one table per queue, then each head's output sums
 // the T queues' gathers before its single store.
 template <typename VT, int T, int NPL>
-__global__ void MSDA_GATHER_BOUNDS
+__global__ void MSDA_GROUP_BOUNDS
 tsa_forward_group_kernel(const VT* __restrict__ value, const float* __restrict__ off,
                          const float* __restrict__ logits, const float* __restrict__ ref,
                          float* __restrict__ out, int B, int Nq, int Nv, int H, int L, int P,
@@ -143,16 +143,19 @@ tsa_forward_group_kernel(const VT* __restrict__ value, const float* __restrict__
         __syncwarp();
         const VT* vb = value + (int64_t)x0.b * T * vstride;
         const int nheads = min(G, H - x0.h0);
-        float acc[G][Gather<VT>::kAcc];
+        float* orow = out + (x0.bq * H + x0.h0) * kHeadDim;
+        for (int s = 0; s < nheads; ++s) {
+            float acc[Gather<VT>::kAcc];
 #pragma unroll
-        for (int s = 0; s < G; ++s)
+            for (int i = 0; i < Gather<VT>::kAcc; ++i) acc[i] = 0.f;
 #pragma unroll
-            for (int i = 0; i < Gather<VT>::kAcc; ++i) acc[s][i] = 0.f;
-#pragma unroll
-        for (int t = 0; t < T; ++t)
-            group_gather<VT, NPL>(vb + t * vstride, s_tab[warp][t], nheads, lane, acc);
+            for (int t = 0; t < T; ++t)
+                Gather<VT>::template run_quads<(1 << NPL) / 4>(vb + t * vstride, s_tab[warp][t],
+                                                               lane, acc, s << NPL);
+            scale_acc(acc, inv_t);
+            Gather<VT>::store(acc, lane, orow + s * kHeadDim);
+        }
         __syncwarp();
-        store_heads<VT, G>(acc, lane, out + (x0.bq * H + x0.h0) * kHeadDim, nheads, inv_t);
         x0 = x1;
         in0 = in1;
         cur = nx;

@@ -37,6 +37,8 @@ def test_header_declares_the_boundary():
               "sca_rebatched_forward", "sca_camera_average", "sca_rebatched_backward",
               "sca_compact_no_alloc", "msda_linear", "msda_linear_timeouts",
               "sca_module_forward", "sca_backward_inputs", "tsa_reference_points", "tsa_forward", "sca_forward_query_major",
+              "msda_linear_dropout", "msda_backward_deterministic",
+              "sca_backward_deterministic",
               "msda_status_string", "msda_last_error", "msda_version"):
         assert n in names
 
@@ -219,3 +221,25 @@ def test_sca_query_major_rejects_bad_arguments(L):
     assert call(msda.Dims(1, 6, 8, 16, 2, 1, 4, 1), mask=0) == INVALID
     assert call(msda.Dims(1, 6, 8, 16, 2, 1, 4, 1), out=FAKE + 8) == INVALID
     assert call(msda.Dims(1, 6, 0, 16, 2, 1, 4, 1), out=0) == OK       # nothing to do
+
+
+def test_linear_dropout_rejects_bad_rates(L):
+    f = L.msda_linear_dropout
+    for p in (-0.1, 1.0, 1.5, float("nan")):
+        assert f(FAKE, FAKE, None, None, 128, 256, 256, 0, FAKE, p, 0, None) == INVALID
+    assert f(0, 0, None, None, 0, 256, 256, 0, 0, 0.2, 1, None) == OK   # empty
+
+
+def test_deterministic_backward_workspace_checks(L):
+    s, st = _levels(((4, 4),))
+    p = ctypes.POINTER(ctypes.c_int64)
+    d = msda.Dims(*GOOD)
+    need = L.msda_backward_deterministic_workspace_size(d)
+    assert need >= 1 * 16 * 2 * 32 * 8
+    call = lambda ws, n: L.msda_backward_deterministic(  # noqa: E731
+        FAKE, 0, s.ctypes.data_as(p), st.ctypes.data_as(p), FAKE, FAKE, FAKE, d, ws, n, FAKE,
+        FAKE, FAKE, None)
+    assert call(0, need) == WORKSPACE
+    assert call(FAKE, need - 8) == WORKSPACE
+    sd = msda.Dims(1, 6, 8, 16, 2, 1, 4, 1)
+    assert L.sca_backward_deterministic_workspace_size(sd) >= 6 * 16 * 2 * 32 * 8

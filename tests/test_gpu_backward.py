@@ -113,32 +113,60 @@ def test_workload5_training_step_full_size():
     assert_close(gv, rv, True, "workload 5 grad_value")
 
 
+def _input_grads_both(w, pos, rl, rw):
+    """sca_backward_inputs on the GPU and in the oracle, both fed the same
+    fp32 rebatched gradients (the oracle's, rounded once)."""
+    rl32, rw32 = rl.astype(np.float32), rw.astype(np.float32)
+    got = msda.sca_backward_inputs(w.spatial_shapes, w.level_start_index,
+                                   dev(w.attention_logits), pos, dev(rl32), dev(rw32), w.Ncam,
+                                   w.R)
+    torch.cuda.synchronize()
+    want = oracle.sca_backward_inputs(w.spatial_shapes, w.bev_mask, w.attention_logits, rl32,
+                                      rw32)
+    return got, want
+
+
 @pytest.mark.parametrize("seed,B,Ncam,bev,shapes,H,P,R", [
     (41, 2, 3, (7, 9), [(9, 13), (4, 7)], 2, 4, 2),
     (42, 1, 6, (30, 40), [(16, 20), (8, 10), (4, 5), (2, 3)], 8, 8, 4),
-    (43, 2, 2, (5, 13), [(6, 7)] * 3, 1, 12, 3),
+    (43, 2, 2, (5, 13), [(6, 7)] * 3, 1, 12, 3),       # R = 3: separate reference kernel
+    (44, 1, 4, (9, 11), [(8, 9), (4, 5)], 12, 4, 2),   # 12 heads: two head chunks
 ])
-def test_sca_backward_inputs(seed, B, Ncam, bev, shapes, H, P, R):
+@pytest.mark.parametrize("rho", ["uniform", "coherent"])
+def test_sca_backward_inputs(seed, B, Ncam, bev, shapes, H, P, R, rho):
     """Offsets, logits and reference-point gradients from the rebatched ones,
     against the oracle's chain rule (itself pinned by finite differences)."""
     w = inputs.workload3(seed=seed, B=B, Ncam=Ncam, bev_h=bev[0], bev_w=bev[1], shapes=shapes,
-                         H=H, P=P, R=R, rho="uniform", same_mask=False, with_grad=True)
-    mask = dev(w.bev_mask)
-    idx, count, pos, hits = msda.sca_compact(mask)
-    args = (dev(w.value), w.spatial_shapes, w.level_start_index, dev(w.reference_points),
-            dev(w.sampling_offsets), dev(w.attention_logits), dev(w.grad_out), idx, count, hits)
-    gv, gl, gw = msda.sca_rebatched_backward(*args)
-    g_off, g_lg, g_ref = msda.sca_backward_inputs(w.spatial_shapes, w.level_start_index,
-                                                  dev(w.attention_logits), pos, gl, gw, Ncam, R)
+                         H=H, P=P, R=R, rho=rho, same_mask=False, with_grad=True)
+    idx, count, pos, hits = msda.sca_compact(dev(w.bev_mask))
+    _, rl, rw = oracle.sca_backward(w.value, w.spatial_shapes, w.level_start_index,
+                                    w.reference_points, w.bev_mask, w.sampling_offsets,
+                                    w.attention_logits, w.grad_out)
+    (g_off, g_lg, g_ref), (r_off, r_lg, r_ref) = _input_grads_both(w, pos, rl, rw)
+    assert_close(g_off, r_off, False, "grad_sampling_offsets")
+    assert_close(g_lg, r_lg, False, "grad_attention_logits")
+    assert_close(g_ref, r_ref, False, "grad_reference_points_cam")
+
+
+def test_sca_backward_chain_on_the_gpu():
+    """The GPU's own rebatched gradients through sca_backward_inputs stay
+    within the bf16-path bound of the oracle's chain (the fp32 errors of the
+    first stage are summed over up to H*L*P/R terms by the second)."""
+    w = inputs.workload3(seed=44, bev_h=20, bev_w=25, with_grad=True)
+    idx, count, pos, hits = msda.sca_compact(dev(w.bev_mask))
+    _, gl, gw = msda.sca_rebatched_backward(
+        dev(w.value), w.spatial_shapes, w.level_start_index, dev(w.reference_points),
+        dev(w.sampling_offsets), dev(w.attention_logits), dev(w.grad_out), idx, count, hits)
+    g = msda.sca_backward_inputs(w.spatial_shapes, w.level_start_index, dev(w.attention_logits),
+                                 pos, gl, gw, w.Ncam, w.R)
     torch.cuda.synchronize()
     _, rl, rw = oracle.sca_backward(w.value, w.spatial_shapes, w.level_start_index,
                                     w.reference_points, w.bev_mask, w.sampling_offsets,
                                     w.attention_logits, w.grad_out)
-    r_off, r_lg, r_ref = oracle.sca_backward_inputs(w.spatial_shapes, w.bev_mask,
-                                                    w.attention_logits, rl, rw)
-    assert_close(g_off, r_off, False, "grad_sampling_offsets")
-    assert_close(g_lg, r_lg, False, "grad_attention_logits")
-    assert_close(g_ref, r_ref, False, "grad_reference_points_cam")
+    r = oracle.sca_backward_inputs(w.spatial_shapes, w.bev_mask, w.attention_logits, rl, rw)
+    for got, want, name in zip(g, r, ("offsets", "logits", "reference points")):
+        err = np.abs(got.cpu().numpy().astype(np.float64) - want)
+        assert err.max() <= 1e-4 * (1.0 + np.abs(want).max()), (name, err.max())
 
 
 def test_sca_backward_inputs_workload5():
@@ -148,14 +176,68 @@ def test_sca_backward_inputs_workload5():
     gv, gl, gw = msda.sca_rebatched_backward(
         value_tensor(w, True), w.spatial_shapes, w.level_start_index, dev(w.reference_points),
         dev(w.sampling_offsets), dev(w.attention_logits), dev(w.grad_out), idx, count, hits)
-    g_off, g_lg, g_ref = msda.sca_backward_inputs(w.spatial_shapes, w.level_start_index,
-                                                  dev(w.attention_logits), pos, gl, gw, w.Ncam, w.R)
     torch.cuda.synchronize()
     _, rl, rw = oracle.sca_backward(w.value, w.spatial_shapes, w.level_start_index,
                                     w.reference_points, w.bev_mask, w.sampling_offsets,
                                     w.attention_logits, w.grad_out)
+    # the second stage alone, on the oracle's first-stage gradients: fp32 bound
+    (g_off, g_lg, g_ref), (r_off, r_lg, r_ref) = _input_grads_both(w, pos, rl, rw)
+    assert_close(g_off, r_off, False, "workload 5 grad_sampling_offsets")
+    assert_close(g_lg, r_lg, False, "workload 5 grad_attention_logits")
+    assert_close(g_ref, r_ref, False, "workload 5 grad_reference_points_cam")
+    # the whole GPU chain (bf16 value): the bf16-path bound
+    g_off, g_lg, g_ref = msda.sca_backward_inputs(w.spatial_shapes, w.level_start_index,
+                                                  dev(w.attention_logits), pos, gl, gw, w.Ncam,
+                                                  w.R)
+    torch.cuda.synchronize()
     r_off, r_lg, r_ref = oracle.sca_backward_inputs(w.spatial_shapes, w.bev_mask,
                                                     w.attention_logits, rl, rw)
-    assert_close(g_off, r_off, True, "workload 5 grad_sampling_offsets")
-    assert_close(g_lg, r_lg, True, "workload 5 grad_attention_logits")
-    assert_close(g_ref, r_ref, True, "workload 5 grad_reference_points_cam")
+    assert_close(g_off, r_off, True, "workload 5 chain grad_sampling_offsets")
+    assert_close(g_lg, r_lg, True, "workload 5 chain grad_attention_logits")
+    assert_close(g_ref, r_ref, True, "workload 5 chain grad_reference_points_cam")
+
+
+@pytest.mark.parametrize("case", CASES, ids=[f"case{c[0]}" for c in CASES])
+@pytest.mark.parametrize("bf16", [False, True])
+def test_msda_backward_deterministic(case, bf16):
+    """Fixed-point grad_value: the oracle's derivative within the fp32 bound,
+    and two runs bitwise equal."""
+    seed, B, Nq, H, shapes, P = case
+    s, starts, value, loc, weights, gout = _problem(seed, B, Nq, H, shapes, P)
+    if bf16:
+        bits = inputs.to_bf16_bits(value)
+        value = inputs.bf16_bits_to_f32(bits)
+        vt = dev(bits.view(np.int16)).view(torch.bfloat16)
+    else:
+        vt = dev(value)
+    args = (vt, s, starts, dev(loc), dev(weights), dev(gout))
+    gv, gl, gw = msda.msda_backward(*args, deterministic=True)
+    gv2, gl2, gw2 = msda.msda_backward(*args, deterministic=True)
+    torch.cuda.synchronize()
+    rv, rl, rw = oracle.msda_backward(value, s, starts, loc, weights, gout)
+    assert_close(gv, rv, False, "deterministic grad_value")
+    assert_close(gl, rl, False, "grad_sampling_locations")
+    assert_close(gw, rw, False, "grad_attention_weights")
+    assert torch.equal(gv, gv2) and torch.equal(gl, gl2) and torch.equal(gw, gw2)
+
+
+def test_sca_backward_deterministic_workload5():
+    """The SCA training step with fixed-point grad_value: parity at full size
+    (bf16 value), bitwise equal runs, and within fp32 rounding of the atomic
+    path."""
+    w = inputs.workload5()
+    args = (value_tensor(w, True), w.spatial_shapes, w.level_start_index,
+            dev(w.reference_points), dev(w.bev_mask), dev(w.sampling_offsets),
+            dev(w.attention_logits), dev(w.grad_out))
+    gv, gl, gw = msda.sca_backward(*args, deterministic=True)
+    gv2, _, _ = msda.sca_backward(*args, deterministic=True)
+    ga, _, _ = msda.sca_backward(*args)
+    torch.cuda.synchronize()
+    assert torch.equal(gv, gv2)
+    rv, rl, rw = oracle.sca_backward(w.value, w.spatial_shapes, w.level_start_index,
+                                     w.reference_points, w.bev_mask, w.sampling_offsets,
+                                     w.attention_logits, w.grad_out)
+    assert_close(gv, rv, True, "workload 5 deterministic grad_value")
+    assert_close(gl, rl, True, "workload 5 grad_sampling_locations_rb")
+    assert_close(gw, rw, True, "workload 5 grad_attention_weights_rb")
+    assert_close(gv, ga.cpu().numpy(), False, "deterministic vs atomic grad_value")

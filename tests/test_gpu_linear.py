@@ -50,6 +50,32 @@ def test_linear_matches_oracle(M, N, K, with_bias, with_res, out_bf16):
     assert msda.lib().msda_linear_timeouts() == 0
 
 
+@pytest.mark.parametrize("M,N,K,out_bf16", [
+    (148 * 128 * 3 + 77, 256, 256, False),   # several tiles per CTA, ragged last tile
+    (40000, 512, 256, True),                 # the offset head: a W-tile switch per CTA
+    (9000, 768, 64, False),                  # three W tiles, one K block
+])
+def test_linear_persistent_tiles(M, N, K, out_bf16):
+    """Many tiles per CTA: the X ring and both TMEM accumulators wrap many
+    times and the W tile is reloaded when a CTA's tiles move to a new N-tile."""
+    rng = np.random.Generator(np.random.PCG64(M + N + K))
+    x32, x = _bf16(rng.standard_normal((M, K)).astype(np.float32))
+    w32, w = _bf16((rng.standard_normal((N, K)) / np.sqrt(K)).astype(np.float32))
+    b = rng.standard_normal(N).astype(np.float32)
+    r = rng.standard_normal((M, N)).astype(np.float32)
+    y = msda.msda_linear(x, w, torch.from_numpy(b).cuda(), torch.from_numpy(r).cuda(),
+                         out_dtype=torch.bfloat16 if out_bf16 else torch.float32)
+    torch.cuda.synchronize()
+    ref = oracle.linear(x32, w32, b, r)
+    mag = np.abs(x32) @ np.abs(w32).T + np.abs(b) + np.abs(r)
+    tol = 1e-6 + (K + 2) * 2.0 ** -24 * mag
+    if out_bf16:
+        tol = tol + 2.0 ** -8 * np.abs(ref)
+    err = np.abs(y.float().cpu().numpy().astype(np.float64) - ref)
+    assert np.all(err <= tol), f"max err {err.max():.3e}"
+    assert msda.lib().msda_linear_timeouts() == 0
+
+
 def test_linear_identity_reproduces_input():
     """W = I (N = K = 256): the projection returns x exactly (fp32 output)."""
     rng = np.random.Generator(np.random.PCG64(5))
@@ -58,3 +84,32 @@ def test_linear_identity_reproduces_input():
     y = msda.msda_linear(x, w)
     torch.cuda.synchronize()
     assert np.array_equal(y.cpu().numpy(), x32)
+
+
+@pytest.mark.parametrize("p,seed,out_bf16", [(0.1, 7, False), (0.5, (3 << 40) | 11, False),
+                                             (0.25, 99, True)])
+def test_linear_dropout_matches_oracle(p, seed, out_bf16):
+    """Training-time dropout in the epilogue: y = r + dropout(x w^T + b).  The
+    mask is the same Philox4x32-10 draw on both sides, so any mask difference
+    fails by the size of a value; the bound is the fp32 one scaled by
+    1 / (1 - p) plus one fp32 rounding of the scaling."""
+    M, N, K = 3000, 512, 128
+    rng = np.random.Generator(np.random.PCG64(31))
+    x32, x = _bf16(rng.standard_normal((M, K)).astype(np.float32))
+    w32, w = _bf16((rng.standard_normal((N, K)) / np.sqrt(K)).astype(np.float32))
+    b = rng.standard_normal(N).astype(np.float32)
+    r = rng.standard_normal((M, N)).astype(np.float32)
+    y = msda.msda_linear(x, w, torch.from_numpy(b).cuda(), torch.from_numpy(r).cuda(),
+                         out_dtype=torch.bfloat16 if out_bf16 else torch.float32,
+                         dropout_p=p, dropout_seed=seed)
+    torch.cuda.synchronize()
+    o = oracle.linear(x32, w32, b)
+    ref = r + oracle.dropout(o, p, seed)
+    mag = np.abs(x32) @ np.abs(w32).T + np.abs(b)
+    tol = 1e-6 + (K + 2) * 2.0 ** -24 * mag / (1 - p) + 2.0 ** -23 * np.abs(o) / (1 - p)
+    if out_bf16:
+        tol = tol + 2.0 ** -8 * np.abs(ref)
+    err = np.abs(y.float().cpu().numpy().astype(np.float64) - ref)
+    assert np.all(err <= tol), f"max err {err.max():.3e}"
+    kept = np.count_nonzero(oracle.dropout(np.ones(M * N), p, seed))
+    assert abs(kept - M * N * (1 - p)) < 5 * np.sqrt(M * N * p * (1 - p))

@@ -2,7 +2,9 @@
 cores, SCA, output projection plus residual) against the oracle's
 composition of the same steps, through the C ABI.  Operands are bf16
 (query + pos, features, weights, and g before the output projection), so the
-bf16 bound applies: |q_hat - oracle| <= 2e-2."""
+bf16 bound applies: |q_hat - oracle| <= 2e-2.  With training-time dropout
+both sides draw the mask from Philox4x32-10 on the same element index and
+seed, so a mask difference would show as an error of the size of a value."""
 import numpy as np
 import pytest
 import torch
@@ -18,8 +20,9 @@ def _bf16_tensor(a):
     return torch.from_numpy(inputs.to_bf16_bits(a).view(np.int16)).cuda().view(torch.bfloat16)
 
 
-@pytest.mark.parametrize("value_bf16", [False, True])
-def test_module_matches_oracle(value_bf16):
+@pytest.mark.parametrize("value_bf16,dropout_p", [(False, 0.0), (True, 0.0), (False, 0.1),
+                                                  (True, 0.3)])
+def test_module_matches_oracle(value_bf16, dropout_p):
     rng = np.random.Generator(np.random.PCG64(77))
     w = inputs.workload3(seed=78, bev_h=16, bev_w=20,
                          shapes=[(29, 50), (15, 25), (8, 13), (4, 7)])
@@ -44,11 +47,13 @@ def test_module_matches_oracle(value_bf16):
         t(q), t(pos), _bf16_tensor(feats), _bf16_tensor(wv), t(bv), _bf16_tensor(woff), t(boff),
         _bf16_tensor(ww), t(bw), _bf16_tensor(wo), t(bo), t(w.reference_points), t(w.bev_mask),
         w.spatial_shapes, w.level_start_index, L, P,
-        value_dtype=torch.bfloat16 if value_bf16 else torch.float32)
+        value_dtype=torch.bfloat16 if value_bf16 else torch.float32, dropout_p=dropout_p,
+        dropout_seed=0x1234_5678_9ABC)
     torch.cuda.synchronize()
     ref = oracle.sca_module_forward(q, pos, feats, wv, bv, woff, boff, ww, bw, wo, bo,
                                     w.reference_points, w.bev_mask, w.spatial_shapes,
-                                    w.level_start_index, L, P, value_bf16=value_bf16)
+                                    w.level_start_index, L, P, value_bf16=value_bf16,
+                                    dropout_p=dropout_p, dropout_seed=0x1234_5678_9ABC)
     err = np.abs(out.cpu().numpy().astype(np.float64) - ref)
     assert err.max() <= 2e-2, err.max()
     assert msda.lib().msda_linear_timeouts() == 0
