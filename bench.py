@@ -572,8 +572,10 @@ def measure_next_rows(args, w, tensors, flush, stream, hbm_peak):
     rows["sca_forward_query_major"] = r
 
     # the plain fused MSDA: the Deformable-DETR encoder and the TSA queues as a batch
-    for name, wk in (("msda_forward_fused_detr", inputs.workload2()),
-                     ("msda_forward_fused_tsa_batch2", inputs.workload4())):
+    for name, wk, kname in (
+            ("msda_forward_fused_detr", inputs.workload2(), "msda_forward_group_kernel<float, true, 4>"),
+            ("msda_forward_fused_tsa_batch2", inputs.workload4(),
+             "msda_forward_group_kernel<float, true, 2>")):
         dv = {k: torch.from_numpy(np.ascontiguousarray(a)).cuda() for k, a in (
             ("value", wk.value), ("ref", wk.reference_points), ("off", wk.sampling_offsets),
             ("logits", wk.attention_logits))}
@@ -585,7 +587,7 @@ def measure_next_rows(args, w, tensors, flush, stream, hbm_peak):
         nbytes = (wk.value.nbytes + wk.B * wk.Nq * S * 12 + wk.reference_points.nbytes
                   + o.numel() * 4)
         r = hbm(nbytes, ms)
-        r.update(kernel="msda_forward_group_kernel<float, true, 2>", workload=wk.name,
+        r.update(kernel=kname, workload=wk.name,
                  gsamples_per_s=wk.B * wk.Nq * S / (ms * 1e-3) / 1e9)
         rows[name] = r
         del dv, o, fa
@@ -687,6 +689,19 @@ def measure_next_rows(args, w, tensors, flush, stream, hbm_peak):
              workload="bevformer-base SCA training step, B=2, bf16 value",
              gsamples_per_s=rows5 * w5.H * w5.L * w5.P / (ms * 1e-3) / 1e9)
     rows["sca_backward"] = r
+    ws5 = torch.empty(int(msda.lib().sca_backward_deterministic_workspace_size(
+        msda.Dims(w5.B, w5.Ncam, w5.Nq, w5.Nv, w5.H, w5.L, w5.P, w5.R))), dtype=torch.uint8,
+        device="cuda")
+    ms = timed(lambda: msda.sca_backward(*args5, grad_value=g5[0],
+                                         grad_sampling_locations_rb=g5[1],
+                                         grad_attention_weights_rb=g5[2], workspace=ws5,
+                                         deterministic=True),
+               n=max(1, iters // 4))
+    r = hbm(sca_backward_algorithmic_bytes(w5, rows5, hitq5, 2), ms)
+    r.update(kernel="sca_backward_kernel<..., deterministic> (fixed-point grad_value)",
+             workload="bevformer-base SCA training step, B=2, bf16 value",
+             gsamples_per_s=rows5 * w5.H * w5.L * w5.P / (ms * 1e-3) / 1e9)
+    rows["sca_backward_deterministic"] = r
     return rows
 
 
