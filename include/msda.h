@@ -27,8 +27,10 @@
  *     in the shapes given.  spatial_shapes and level_start_index are HOST
  *     arrays (read during the call, not kept).
  *   - The library allocates no memory and keeps no pointer after returning.
- *     The only state it holds is a per-thread error message and a per-device
- *     cache of the SM count.
+ *     Its only state: a per-thread error message, a per-device cache of the
+ *     SM count, the fixed scratch array of sca_compact_no_alloc, the device
+ *     counter read by msda_linear_timeouts, and (set once) the GEMM kernel's
+ *     shared-memory attribute and the driver's tensor-map encoder.
  *   - Calls are asynchronous on `stream` (NULL = the legacy default stream).
  *     The status covers argument checks and kernel launch errors; errors that
  *     happen while the kernels run surface at the caller's next

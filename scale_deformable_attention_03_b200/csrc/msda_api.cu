@@ -201,7 +201,7 @@ ScaWorkspace sca_workspace_carve(void* base, int B, int Ncam, int Nq, int H, boo
 
 extern "C" {
 
-int32_t msda_version(void) { return 10000; }  // 1.0.0
+int32_t msda_version(void) { return 10100; }  // 1.1.0: module dropout fields, TSA, deterministic backward
 
 const char* msda_status_string(msda_status_t status)
 {
