@@ -243,17 +243,30 @@ def round_bf16(a):
 def sca_module_forward(query, query_pos, features, w_value, b_value, w_offsets, b_offsets,
                        w_weights, b_weights, w_output, b_output, reference_points_cam, bev_mask,
                        spatial_shapes, level_start_index, num_levels, num_points,
-                       value_bf16=False, dropout_p=0.0, dropout_seed=0):
+                       value_bf16=False, dropout_p=0.0, dropout_seed=0, camera_embeds=None,
+                       level_embeds=None):
     """The SCA module forward ([BQ] 3, 4, 10-13), composed of the oracle's
-    projection and SCA: q~ = bf16(q + pos); V = F~ W_v^T + b_v; Delta, a from
-    q~; g = SCA; q_hat = q + dropout(bf16(g) W_o^T + b_o).  features
-    [B, Ncam, Nv, C]; dropout_p = 0 is the inference identity."""
+    projection and SCA: F~ = F + e_cam + e_level ([BQ] 3; the embeddings are
+    optional, absent = already in F); q~ = bf16(q + pos); V = F~ W_v^T + b_v;
+    Delta, a from q~; g = SCA; q_hat = q + dropout(bf16(g) W_o^T + b_o).
+    features [B, Ncam, Nv, C]; camera_embeds [Ncam, C]; level_embeds [L, C]
+    (added to the rows of level l: start_l .. start_l + H_l W_l - 1);
+    dropout_p = 0 is the inference identity."""
     q = _d(query)
     B, Nq, C = q.shape
     _, Ncam, Nv, _ = features.shape
     H, L, P = C // 32, num_levels, num_points
     qt = round_bf16(q + (0.0 if query_pos is None else _d(query_pos))).reshape(B * Nq, C)
-    V = linear(_d(features).reshape(-1, C), w_value, b_value)
+    F = _d(features).copy()
+    if camera_embeds is not None:
+        F += _d(camera_embeds)[None, :, None, :]
+    if level_embeds is not None:
+        shapes, starts = _levels(spatial_shapes, level_start_index)
+        e = _d(level_embeds)
+        for l in range(L):
+            n = int(shapes[l, 0] * shapes[l, 1])
+            F[:, :, starts[l]:starts[l] + n, :] += e[l]
+    V = linear(F.reshape(-1, C), w_value, b_value)
     if value_bf16:
         V = round_bf16(V)
     off = linear(qt, w_offsets, b_offsets).reshape(B, Nq, H, L, P, 2)

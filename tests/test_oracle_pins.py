@@ -774,3 +774,28 @@ def test_dropout_mask_is_the_generator_words():
     for e in (0, 1, 2, 3, 4, 17, 39):
         u = oracle.philox4x32_10((e // 4, 0, 0, 0), (5, 7))[e % 4]
         assert (y[e] != 0) == (int(u) >= int(p * 2 ** 32))
+
+
+def test_module_embeddings_are_added_to_the_features():
+    """[BQ] 3: F~ = F + e_cam + e_level.  Passing the embeddings equals passing
+    features that already hold them, built here by indexing each pixel's
+    camera and level independently (a level per row from the level table)."""
+    rng = _rng(43)
+    B, Ncam, Nq, C, L, P, R = 1, 3, 5, 32, 2, 2, 1
+    shapes, starts, Nv = _levels([(3, 4), (2, 2)])
+    q = rng.standard_normal((B, Nq, C))
+    feats = oracle.round_bf16(rng.standard_normal((B, Ncam, Nv, C)))
+    e_cam = rng.standard_normal((Ncam, C))
+    e_lvl = rng.standard_normal((L, C))
+    ref = rng.uniform(0.1, 0.9, (Ncam, B, Nq, R, 2))
+    mask = np.ones((Ncam, B, Nq, R), np.uint8)
+    S = L * P
+    wv, wo = rng.standard_normal((C, C)) / 8, rng.standard_normal((C, C)) / 8
+    woff, ww = rng.standard_normal((2 * S, C)) / 8, rng.standard_normal((S, C)) / 8
+    level_of_row = np.concatenate([np.full(h * w, l) for l, (h, w) in enumerate(shapes)])
+    tilde = feats + e_cam[None, :, None, :] + e_lvl[level_of_row][None, None, :, :]
+    common = (None, wv, None, woff, None, ww, None, wo, None, ref, mask, shapes, starts, L, P)
+    a = oracle.sca_module_forward(q, None, feats, *common[1:], camera_embeds=e_cam,
+                                  level_embeds=e_lvl)
+    b = oracle.sca_module_forward(q, None, tilde, *common[1:])
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-12)
