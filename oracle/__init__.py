@@ -347,3 +347,23 @@ def dropout(o, p, seed):
     out = np.empty_like(a)
     _check(lib().oracle_dropout(_p(a, _D), a.size, float(p), int(seed), _p(out, _D)), "dropout")
     return out
+
+
+def tsa_backward(value, spatial_shapes, level_start_index, reference_points, sampling_offsets,
+                 attention_logits, num_queues, grad_out, coord_f32=True):
+    """Derivative of tsa_forward (the pages give no backward): queue t of
+    sample b receives grad_out[b] / T; the fused MSDA backward of every queue
+    gives the location and weight gradients, and the chain through the
+    location and the softmax (oracle_sca_backward_inputs with one camera that
+    sees every query) gives those of the offsets, logits and reference points.
+    -> (grad_value [B*T, Nv, H, Dh], grad_offsets [B*T, Nq, H, L, P, 2],
+        grad_logits [B*T, Nq, H, L, P], grad_reference_points [B*T, Nq, R, 2])."""
+    T = int(num_queues)
+    v, ref, off, lg = _d(value), _d(reference_points), _d(sampling_offsets), _d(attention_logits)
+    BT, Nq, R = ref.shape[0], ref.shape[1], ref.shape[2]
+    loc, w = fused_locations(spatial_shapes, ref, off, lg, coord_f32)
+    go = np.repeat(_d(grad_out) / T, T, axis=0)
+    gv, gl, gw = msda_backward(v, spatial_shapes, level_start_index, loc, w, go, coord_f32)
+    seen = np.ones((1, BT, Nq, R), np.uint8)
+    g_off, g_lg, g_ref = sca_backward_inputs(spatial_shapes, seen, lg, gl[:, None], gw[:, None])
+    return gv, g_off, g_lg, g_ref[0]

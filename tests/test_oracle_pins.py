@@ -799,3 +799,42 @@ def test_module_embeddings_are_added_to_the_features():
                                   level_embeds=e_lvl)
     b = oracle.sca_module_forward(q, None, tilde, *common[1:])
     np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-12)
+
+
+def test_tsa_backward_matches_finite_differences():
+    """Central differences through the whole TSA forward (two queues, two
+    levels, R = 2) for the value, offsets, logits and reference points."""
+    rng = _rng(62)
+    B, T, Nq, H, Dh, P, R = 1, 2, 3, 2, 3, 2, 2
+    shapes, starts, Nv = _levels([(4, 5), (2, 3)])
+    L = 2
+    value = rng.standard_normal((B * T, Nv, H, Dh))
+    ref = rng.uniform(0.2, 0.8, (B * T, Nq, R, 2))
+    off = rng.uniform(-0.7, 0.7, (B * T, Nq, H, L, P, 2))
+    logits = rng.standard_normal((B * T, Nq, H, L, P))
+    go = rng.standard_normal((B, Nq, H * Dh))
+    for _ in range(50):  # keep pixel coordinates away from cell boundaries
+        loc, _w = oracle.fused_locations(shapes, ref, off, logits, coord_f32=False)
+        ok = True
+        for l, (Hl, Wl) in enumerate(shapes):
+            for ax, n in ((0, Wl), (1, Hl)):
+                x = loc[..., l, :, ax] * n - 0.5
+                fr = x - np.floor(x)
+                ok &= bool(np.all((fr > 1e-3) & (fr < 1 - 1e-3)))
+        if ok:
+            break
+        off += rng.uniform(-0.05, 0.05, off.shape)
+    assert ok
+
+    def loss():
+        return float(np.sum(go * oracle.tsa_forward(value, shapes, starts, ref, off, logits, T,
+                                                     coord_f32=False)))
+
+    gv, g_off, g_lg, g_ref = oracle.tsa_backward(value, shapes, starts, ref, off, logits, T, go,
+                                                 coord_f32=False)
+    h = 1e-6
+    np.testing.assert_allclose(gv, _central_fd(loss, value, h), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(g_off, _central_fd(loss, off, h), rtol=1e-6, atol=1e-7)
+    np.testing.assert_allclose(g_lg, _central_fd(loss, logits, h), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(g_ref, _central_fd(loss, ref, h), rtol=1e-6, atol=1e-7)
+    assert np.abs(g_off).max() > 0.02
