@@ -54,7 +54,7 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=("native", "reference"), default="native")
     p.add_argument("--value-dtype", choices=("f32", "bf16"), default="f32")
     p.add_argument("--rho", choices=("coherent", "uniform"), default="coherent")
-    p.add_argument("--e2e-steps", type=int, default=5)
+    p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--rows-iters", type=int, default=20,
                    help="timed calls per entry point in the next_rows section (0 = skip)")
     p.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -442,33 +442,59 @@ def run_native(args):
     value_gs = total_samples / (total_ms * 1e-3) / 1e9
 
     # ---- end to end through the one-call C ABI, host buffers ----
+    # Every step copies its inputs from pinned host memory, runs sca_forward
+    # and copies its result back.  Two device buffer sets let the copies of
+    # step i + 1 (copy stream) overlap the kernels of step i (compute stream)
+    # and the read-back of step i - 1 (read-back stream).
     host = {k: torch.from_numpy(np.ascontiguousarray(a)).pin_memory() for k, a in (
         ("value", w.value_bf16.view(np.int16) if bf16 else w.value),
         ("ref", w.reference_points), ("mask", w.bev_mask), ("off", w.sampling_offsets),
         ("logits", w.attention_logits))}
-    host_out = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+    host_out = [torch.empty(out.shape, dtype=torch.float32).pin_memory() for _ in range(2)]
     ws = torch.empty(msda.msda_workspace_size(dims), dtype=torch.uint8, device="cuda")
-    dev_in = {k: torch.empty(v.shape, dtype=v.dtype, device="cuda") for k, v in host.items()}
+    dev_in = [{k: torch.empty(v.shape, dtype=v.dtype, device="cuda") for k, v in host.items()}
+              for _ in range(2)]
+    dev_out = [torch.empty_like(out) for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = host_out.numel() * 4
+    d2h = host_out[0].numel() * 4
+    copy_s, back_s = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    computed = [ev(), ev()]
+    read_back = [ev(), ev()]
 
-    def e2e_step():
-        for k in host:
-            dev_in[k].copy_(host[k], non_blocking=True)
-        v = dev_in["value"].view(torch.bfloat16) if bf16 else dev_in["value"]
-        msda._check(L.sca_forward(P(v), vdt, sp, st, P(dev_in["ref"]), P(dev_in["mask"]),
-                                  P(dev_in["off"]), P(dev_in["logits"]), dims, P(ws), ws.numel(),
-                                  P(out), sptr), "sca_forward")
-        host_out.copy_(out, non_blocking=True)
+    def e2e_step(i):
+        j = i % 2
+        copied = ev()
+        with torch.cuda.stream(copy_s):
+            copy_s.wait_event(computed[j])   # step i - 2 has finished reading set j
+            for k in host:
+                dev_in[j][k].copy_(host[k], non_blocking=True)
+            copied.record(copy_s)
+        stream.wait_event(copied)
+        stream.wait_event(read_back[j])      # step i - 2's result has left dev_out[j]
+        d_in = dev_in[j]
+        v = d_in["value"].view(torch.bfloat16) if bf16 else d_in["value"]
+        msda._check(L.sca_forward(P(v), vdt, sp, st, P(d_in["ref"]), P(d_in["mask"]),
+                                  P(d_in["off"]), P(d_in["logits"]), dims, P(ws), ws.numel(),
+                                  P(dev_out[j]), sptr), "sca_forward")
+        computed[j].record(stream)
+        with torch.cuda.stream(back_s):
+            back_s.wait_event(computed[j])
+            host_out[j].copy_(dev_out[j], non_blocking=True)
+            read_back[j].record(back_s)
 
-    e2e_step()
+    for i in range(2):
+        e2e_step(i)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.e2e_steps):
-        e2e_step()
+    copy_s.wait_event(e0)
+    for i in range(args.e2e_steps):
+        e2e_step(i)
+    stream.wait_stream(back_s)
+    stream.wait_stream(copy_s)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms, e2e_samples = aggregate(e0.elapsed_time(e1), samples_per_step * args.e2e_steps, world)
@@ -507,7 +533,9 @@ def run_native(args):
                  "samples": samples_per_step, "rebatched_rows": rows},
         "e2e": {"value": e2e_gs, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "api": "sca_forward (one call)",
-                "steps": args.e2e_steps},
+                "steps": args.e2e_steps,
+                "pipelining": "copies of step i+1 and read-back of step i-1 overlap the "
+                              "kernels of step i (two buffer sets, three streams)"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
@@ -611,7 +639,20 @@ def measure_next_rows(args, w, tensors, flush, stream, hbm_peak):
     rows["tsa_forward"] = r
     ms = timed(lambda: msda.tsa_reference_points(ego, 200, 200, out=ref4))
     rows["tsa_reference_points"] = hbm(2 * w4.Nq * 8 + 24, ms)
-    del v4, off4, lg4, out4, ref4
+    go4 = torch.randn((1, w4.Nq, w4.H * 32), device="cuda")
+    tws = torch.empty(int(msda.lib().tsa_backward_workspace_size(
+        msda.Dims(1, 1, w4.Nq, w4.Nv, w4.H, w4.L, w4.P, w4.R), 2)), dtype=torch.uint8,
+        device="cuda")
+    ms = timed(lambda: msda.tsa_backward(v4, w4.spatial_shapes, w4.level_start_index, ref4v,
+                                         off4, lg4, 2, go4, workspace=tws))
+    S4 = w4.H * w4.L * w4.P
+    r = hbm(tsa_algorithmic_bytes(w4, 2, 4) + w4.Nq * w4.H * 32 * 4 + w4.value.size * 4
+            + 2 * w4.Nq * (S4 * 3 + w4.R * 2) * 4, ms)
+    r.update(kernel="tsa_backward_kernel + sca_offset_logit_grads_kernel",
+             workload="bevformer-tsa 2 queues x 200x200, H=8, P=4, fp32",
+             gsamples_per_s=2 * w4.Nq * S4 / (ms * 1e-3) / 1e9)
+    rows["tsa_backward"] = r
+    del v4, off4, lg4, out4, ref4, go4, tws
 
     # A12: the value projection of all six cameras' features, M = 6 * 30825
     g = torch.Generator(device="cuda").manual_seed(7)

@@ -157,6 +157,28 @@ msda_status_t tsa_forward(const void* value, msda_dtype_t vdt, const int64_t* sp
                           const float* sampling_offsets, const float* attention_logits,
                           int32_t num_queues, msda_dims_t d, float* out, msda_stream_t stream);
 
+/* TSA backward: the derivative of tsa_forward (the pages give no backward).
+ * Queue t of sample b receives grad_out[b] / T; the fused MSDA backward of
+ * every queue row gives its location and weight gradients (workspace), and
+ * the chain through the location and the softmax gives:
+ *   grad_value             [B*T, Nv, H, 32]       fp32, written (zeroed, then
+ *                                                 accumulated with atomics)
+ *   grad_sampling_offsets  [B*T, Nq, H, L, P, 2]  = d/d s / (W_l, H_l)
+ *   grad_attention_logits  [B*T, Nq, H, L, P]     softmax backward
+ *   grad_reference_points  [B*T, Nq, R, 2]        sum over the points k with
+ *                                                 k mod R = m
+ *   grad_out               [B, Nq, H * 32]
+ * Other arguments as tsa_forward; workspace >= tsa_backward_workspace_size(d,
+ * num_queues) bytes (256-byte aligned). */
+size_t tsa_backward_workspace_size(msda_dims_t d, int32_t num_queues);
+msda_status_t tsa_backward(const void* value, msda_dtype_t vdt, const int64_t* spatial_shapes,
+                           const int64_t* level_start_index, const float* reference_points,
+                           const float* sampling_offsets, const float* attention_logits,
+                           int32_t num_queues, const float* grad_out, msda_dims_t d,
+                           void* workspace, size_t workspace_bytes, float* grad_value,
+                           float* grad_sampling_offsets, float* grad_attention_logits,
+                           float* grad_reference_points, msda_stream_t stream);
+
 /* MSDA backward: the derivative of msda_forward (the pages give no backward;
  * this is the analytic derivative of [BQ] 6 and 8).
  *   grad_out                [B, Nq, H * 32]      fp32
@@ -401,8 +423,13 @@ msda_status_t sca_backward(const void* value, msda_dtype_t vdt,
 typedef struct {
     const float* query;                /* [B, Nq, C] fp32: q, also the residual */
     const float* query_pos;            /* [B, Nq, C] fp32 or NULL: pos */
-    const void* features;              /* [B, Ncam, Nv, C] bf16: F~ = FPN + camera + level
-                                          embeddings, level rows as level_start_index */
+    const void* features;              /* [B, Ncam, Nv, C] bf16: the FPN features F, level
+                                          rows as level_start_index; F~ = F + e_cam +
+                                          e_level ([BQ] 3), the embeddings below (NULL
+                                          = already in F).  They enter the value
+                                          projection as a bias per (camera, level):
+                                          (e_cam + e_level) W_v^T + b_v, computed in
+                                          double, so F itself is never re-rounded */
     const void* w_value;               /* [C, C] bf16 */
     const float* b_value;              /* [C] */
     const void* w_offsets;             /* [H*L*P*2, C] bf16 (rows h, l, k, xy) */
@@ -416,6 +443,8 @@ typedef struct {
     msda_dtype_t value_dtype;          /* storage of V for the sampling: fp32 or bf16 */
     float dropout_p;                   /* training-time dropout rate in [0, 1); 0 = inference */
     uint64_t dropout_seed;             /* key of the dropout mask (see msda_linear_dropout) */
+    const float* camera_embeds;        /* [Ncam, C] fp32 or NULL: e_cam of [BQ] 3 */
+    const float* level_embeds;         /* [L, C] fp32 or NULL: e_level of [BQ] 3 */
 } sca_module_params_t;
 
 /* Bytes of device workspace sca_module_forward needs (q~, V, Delta, a, the

@@ -41,7 +41,8 @@ class ScaModuleParams(ctypes.Structure):
                 ("b_value", _vp), ("w_offsets", _vp), ("b_offsets", _vp), ("w_weights", _vp),
                 ("b_weights", _vp), ("w_output", _vp), ("b_output", _vp),
                 ("reference_points_cam", _vp), ("bev_mask", _vp), ("value_dtype", ctypes.c_int),
-                ("dropout_p", ctypes.c_float), ("dropout_seed", ctypes.c_uint64)]
+                ("dropout_p", ctypes.c_float), ("dropout_seed", ctypes.c_uint64),
+                ("camera_embeds", _vp), ("level_embeds", _vp)]
 
 
 _lib = None
@@ -109,6 +110,11 @@ def lib():
         L.tsa_reference_points.restype = ctypes.c_int
         L.tsa_forward.argtypes = [_vp, st, _i64p, _i64p, _vp, _vp, _vp, i32, Dims, _vp, _vp]
         L.tsa_forward.restype = ctypes.c_int
+        L.tsa_backward_workspace_size.argtypes = [Dims, i32]
+        L.tsa_backward_workspace_size.restype = ctypes.c_size_t
+        L.tsa_backward.argtypes = [_vp, st, _i64p, _i64p, _vp, _vp, _vp, i32, _vp, Dims, _vp,
+                                   ctypes.c_size_t, _vp, _vp, _vp, _vp, _vp]
+        L.tsa_backward.restype = ctypes.c_int
         L.sca_forward_query_major.argtypes = [_vp, st, _i64p, _i64p, _vp, _vp, _vp, _vp, Dims,
                                               _vp, _vp]
         L.sca_forward_query_major.restype = ctypes.c_int
@@ -254,6 +260,35 @@ def tsa_forward(value, spatial_shapes, level_start_index, reference_points, samp
                              _stream(stream)),
            "tsa_forward")
     return out
+
+
+def tsa_backward(value, spatial_shapes, level_start_index, reference_points, sampling_offsets,
+                 attention_logits, num_queues, grad_out, workspace=None, stream=None):
+    """-> (grad_value [B*T, Nv, H, 32], grad_sampling_offsets [B*T, Nq, H, L, P, 2],
+    grad_attention_logits [B*T, Nq, H, L, P], grad_reference_points [B*T, Nq, R, 2])."""
+    torch = _torch()
+    _contig(value, reference_points, sampling_offsets, attention_logits, grad_out)
+    BT, Nv, H, _ = value.shape
+    T = int(num_queues)
+    if T < 1 or BT % T:
+        raise MsdaError("tsa_backward: the value batch is not a multiple of num_queues")
+    _, Nq, _, L, P, _ = sampling_offsets.shape
+    R = reference_points.shape[2]
+    shapes, starts = _levels(spatial_shapes, level_start_index)
+    d = Dims(BT // T, 1, Nq, Nv, H, L, P, R)
+    dev = value.device
+    gv = torch.empty(value.shape, device=dev, dtype=torch.float32)
+    g_off = torch.empty(sampling_offsets.shape, device=dev, dtype=torch.float32)
+    g_lg = torch.empty(attention_logits.shape, device=dev, dtype=torch.float32)
+    g_ref = torch.empty(reference_points.shape, device=dev, dtype=torch.float32)
+    workspace = _workspace(int(lib().tsa_backward_workspace_size(d, T)), dev, workspace)
+    _check(lib().tsa_backward(_ptr(value), _vdt(value), shapes.ctypes.data_as(_i64p),
+                              starts.ctypes.data_as(_i64p), _ptr(reference_points),
+                              _ptr(sampling_offsets), _ptr(attention_logits), T, _ptr(grad_out),
+                              d, _ptr(workspace), workspace.numel(), _ptr(gv), _ptr(g_off),
+                              _ptr(g_lg), _ptr(g_ref), _stream(stream)),
+           "tsa_backward")
+    return gv, g_off, g_lg, g_ref
 
 
 def msda_backward(value, spatial_shapes, level_start_index, sampling_locations,
@@ -503,7 +538,7 @@ def sca_module_forward(query, query_pos, features, w_value, b_value, w_offsets, 
                        w_weights, b_weights, w_output, b_output, reference_points_cam, bev_mask,
                        spatial_shapes, level_start_index, num_levels, num_points,
                        value_dtype=None, out=None, workspace=None, stream=None, dropout_p=0.0,
-                       dropout_seed=0):
+                       dropout_seed=0, camera_embeds=None, level_embeds=None):
     """The SCA module forward: q_hat = q + output_proj(SCA(value_proj(F~),
     offsets(q + pos), weights(q + pos))).  query, query_pos [B, Nq, C] fp32;
     features [B, Ncam, Nv, C] bf16; weights bf16 [out, in]; biases fp32;
@@ -511,7 +546,7 @@ def sca_module_forward(query, query_pos, features, w_value, b_value, w_offsets, 
     -> q_hat [B, Nq, C] fp32."""
     torch = _torch()
     _contig(query, query_pos, features, w_value, w_offsets, w_weights, w_output,
-            reference_points_cam, bev_mask)
+            reference_points_cam, bev_mask, camera_embeds, level_embeds)
     if bev_mask.dtype == torch.bool:
         bev_mask = bev_mask.view(torch.uint8)
     B, Nq, C = query.shape
@@ -530,7 +565,7 @@ def sca_module_forward(query, query_pos, features, w_value, b_value, w_offsets, 
                                               w_offsets, b_offsets, w_weights, b_weights,
                                               w_output, b_output, reference_points_cam,
                                               bev_mask)], vdt, float(dropout_p),
-                           int(dropout_seed))
+                           int(dropout_seed), _ptr(camera_embeds), _ptr(level_embeds))
     _check(lib().sca_module_forward(ctypes.byref(prm), shapes.ctypes.data_as(_i64p),
                                     starts.ctypes.data_as(_i64p), d, _ptr(workspace),
                                     workspace.numel(), _ptr(out), _stream(stream)),

@@ -307,6 +307,63 @@ msda_status_t tsa_forward(const void* value, msda_dtype_t vdt, const int64_t* sp
                        "tsa_forward");
 }
 
+static msda_status_t check_workspace(const void* ws, size_t have, size_t need);
+
+size_t tsa_backward_workspace_size(msda_dims_t d, int32_t num_queues)
+{
+    if (d.B < 0 || d.Nq < 0 || d.H < 1 || d.L < 1 || d.P < 1 || num_queues < 1) return 0;
+    const size_t rows = (size_t)d.B * num_queues * d.Nq;
+    const size_t S = (size_t)d.H * d.L * d.P;
+    return align256(sizeof(float) * rows * S * 2) + align256(sizeof(float) * rows * S);
+}
+
+msda_status_t tsa_backward(const void* value, msda_dtype_t vdt, const int64_t* spatial_shapes,
+                           const int64_t* level_start_index, const float* reference_points,
+                           const float* sampling_offsets, const float* attention_logits,
+                           int32_t num_queues, const float* grad_out, msda_dims_t d,
+                           void* workspace, size_t workspace_bytes, float* grad_value,
+                           float* grad_sampling_offsets, float* grad_attention_logits,
+                           float* grad_reference_points, msda_stream_t stream)
+{
+    MSDA_TRY(check_dims(d, false));
+    MSDA_CHECK(num_queues >= 1 && num_queues <= MSDA_MAX_QUEUES, MSDA_ERR_UNSUPPORTED,
+               "num_queues = %d outside 1..%d", num_queues, MSDA_MAX_QUEUES);
+    MSDA_CHECK((int64_t)d.B * num_queues * d.Nq <= INT32_MAX, MSDA_ERR_UNSUPPORTED,
+               "B * num_queues * Nq exceeds the 32-bit range");
+    msda::Levels lv;
+    MSDA_TRY(check_levels(d, spatial_shapes, level_start_index, lv));
+    MSDA_TRY(check_dtype(vdt));
+    if (d.B == 0) return ok();
+    MSDA_PTR(grad_value, 16);
+    if (d.Nq > 0) {
+        MSDA_TRY(check_value(value));
+        MSDA_PTR(reference_points, 8);
+        MSDA_PTR(sampling_offsets, 8);
+        MSDA_PTR(attention_logits, 4);
+        MSDA_PTR(grad_out, 16);
+        MSDA_PTR(grad_sampling_offsets, 8);
+        MSDA_PTR(grad_attention_logits, 4);
+        MSDA_PTR(grad_reference_points, 8);
+    }
+    MSDA_TRY(check_workspace(workspace, workspace_bytes, tsa_backward_workspace_size(d, num_queues)));
+    const cudaStream_t s = (cudaStream_t)stream;
+    const int BT = d.B * num_queues;
+    const size_t S = (size_t)d.H * d.L * d.P;
+    float* gl = static_cast<float*>(workspace);
+    float* gw = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                         align256(sizeof(float) * (size_t)BT * d.Nq * S * 2));
+    const msda::Problem p = make_problem(value, vdt, d, lv);
+    cudaError_t e = msda::launch_zero(grad_value, (int64_t)BT * d.Nv * d.H * MSDA_HEAD_DIM, s);
+    if (e == cudaSuccess && d.Nq > 0)
+        e = msda::launch_tsa_backward(p, num_queues, reference_points, sampling_offsets,
+                                      attention_logits, grad_out, grad_value, gl, gw, s);
+    if (e == cudaSuccess && d.Nq > 0)
+        e = msda::launch_sca_input_grads(attention_logits, nullptr, gl, gw, BT, 1, d.Nq, d.H, d.L,
+                                         d.P, d.R, lv, grad_sampling_offsets,
+                                         grad_attention_logits, grad_reference_points, s);
+    return cuda_status(e, "tsa_backward");
+}
+
 msda_status_t msda_backward(const void* value, msda_dtype_t vdt, const int64_t* spatial_shapes,
                             const int64_t* level_start_index, const float* sampling_locations,
                             const float* attention_weights, const float* grad_out, msda_dims_t d,
@@ -336,8 +393,6 @@ msda_status_t msda_backward(const void* value, msda_dtype_t vdt, const int64_t* 
                                        grad_attention_weights, s);
     return cuda_status(e, "msda_backward");
 }
-
-static msda_status_t check_workspace(const void* ws, size_t have, size_t need);
 
 size_t msda_backward_deterministic_workspace_size(msda_dims_t d)
 {

@@ -389,6 +389,87 @@ sca_backward_kernel(const VT* __restrict__ value, const float* __restrict__ off,
     }
 }
 
+// TSA: the fused backward of every queue's MSDA; queue t of sample b (value
+// item b * T + t) receives grad_out[b] / T (the queue mean).  Rows are
+// (b * T + t, q); location and weight gradients per queue row.
+template <typename VT, int NC>
+__global__ void __launch_bounds__(kThreads)
+tsa_backward_kernel(const VT* __restrict__ value, const float* __restrict__ off,
+                    const float* __restrict__ logits, const float* __restrict__ ref,
+                    const float* __restrict__ grad_out, float* __restrict__ grad_value,
+                    float* __restrict__ grad_loc, float* __restrict__ grad_attn, int BT, int T,
+                    int Nq, int Nv, int H, int L, int P, int R, Levels levels)
+{
+    __shared__ SmemLevels s_lv;
+    __shared__ __align__(16) BwdTable s_tab[kWarps];
+    stage_levels(s_lv, levels);
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    LaneSamples<NC> ls;
+    lane_samples<NC>(s_lv, L, P, R, lane, ls);
+    const int S = L * P;
+    const int64_t rows = (int64_t)BT * Nq;
+    const int64_t row0 = (int64_t)blockIdx.x * kBwdRowsPerTile;
+    const int bt0 = (int)(row0 / Nq);
+    const int q0 = (int)(row0 - (int64_t)bt0 * Nq);
+    ItemCursor cur(warp, H);
+    for (int it = warp; it < kBwdRowsPerTile * H; it += kWarps, cur.next()) {
+        const int64_t r = row0 + cur.rr;
+        if (r >= rows) break;
+        int q = q0 + cur.rr, bt = bt0;
+        while (q >= Nq) {
+            q -= Nq;
+            ++bt;
+        }
+        const int64_t item = r * H + cur.h;
+        const int64_t gitem = ((int64_t)(bt / T) * Nq + q) * H + cur.h;
+        const int64_t vofs = (int64_t)bt * Nv * H * kHeadDim;
+        row_backward<VT, true, NC, false>(value + vofs, H, cur.h, off + item * S * 2,
+                                          logits + item * S, ref + r * R * 2, S, ls, s_tab[warp],
+                                          grad_out + gitem * kHeadDim, (float)T,
+                                          grad_value + vofs, nullptr, grad_loc + item * S * 2,
+                                          grad_attn + item * S, lane);
+    }
+}
+
+template <typename VT>
+static cudaError_t launch_tsa_backward_t(const Problem& p, int T, const float* ref,
+                                         const float* off, const float* logits,
+                                         const float* grad_out, float* grad_value,
+                                         float* grad_loc, float* grad_attn, cudaStream_t s)
+{
+    const int BT = p.B * T;
+    const int64_t rows = (int64_t)BT * p.Nq;
+    if (rows == 0) return cudaSuccess;
+    const unsigned grid = (unsigned)((rows + kBwdRowsPerTile - 1) / kBwdRowsPerTile);
+    const VT* v = static_cast<const VT*>(p.value);
+    switch ((p.L * p.P + 31) / 32) {
+#define TSA_BWD_CASE(NCV)                                                                        \
+    case NCV:                                                                                    \
+        tsa_backward_kernel<VT, NCV><<<grid, kThreads, 0, s>>>(                                  \
+            v, off, logits, ref, grad_out, grad_value, grad_loc, grad_attn, BT, T, p.Nq, p.Nv,   \
+            p.H, p.L, p.P, p.R, p.lv);                                                           \
+        break;
+        TSA_BWD_CASE(1)
+        TSA_BWD_CASE(2)
+        TSA_BWD_CASE(3)
+        TSA_BWD_CASE(4)
+#undef TSA_BWD_CASE
+        default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_tsa_backward(const Problem& p, int T, const float* ref, const float* off,
+                                const float* logits, const float* grad_out, float* grad_value,
+                                float* grad_loc, float* grad_attn, cudaStream_t s)
+{
+    return p.bf16 ? launch_tsa_backward_t<__nv_bfloat16>(p, T, ref, off, logits, grad_out,
+                                                         grad_value, grad_loc, grad_attn, s)
+                  : launch_tsa_backward_t<float>(p, T, ref, off, logits, grad_out, grad_value,
+                                                 grad_loc, grad_attn, s);
+}
+
 // ---------------------------------------------------------------------------
 
 __device__ __forceinline__ void zero_range(float* __restrict__ p, int64_t n, int64_t tid,

@@ -89,7 +89,8 @@ cudaError_t launch_sca_zero_tail(const int32_t* count, int B, int Ncam, int Nq, 
 #include "msda.h"
 
 namespace msda {
-// Gradients of offsets, logits and reference points (sca_input_grads.cu).
+// Gradients of offsets, logits and reference points (sca_input_grads.cu);
+// pos == null: Ncam = 1 and row i is query i.
 cudaError_t launch_sca_input_grads(const float* logits, const int32_t* pos,
                                    const float* grad_loc_rb, const float* grad_attn_rb, int B,
                                    int Ncam, int Nq, int H, int L, int P, int R, const Levels& lv,
@@ -101,6 +102,22 @@ cudaError_t launch_tsa_reference(const float* ego, int B, int T, int bev_h, int 
                                  double gy, float* ref, cudaStream_t s);
 cudaError_t launch_tsa_forward(const Problem& p, int T, const float* ref, const float* off,
                                const float* logits, float* out, cudaStream_t s);
+
+// The projection with a bias per (camera, level) row group (the embedding
+// prologue of the SCA module): row r is pixel r mod nv of camera
+// (r div nv) mod ncam, level = last l with start[l] <= pixel.
+struct RowBiasArgs {
+    const float* table;  // [ncam * L, N]
+    int nv, ncam, L;
+    int start[8];
+};
+msda_status_t linear_impl(const void* x, const void* w, const float* bias, const float* residual,
+                          int32_t M, int32_t N, int32_t K, msda_dtype_t y_dtype, void* y,
+                          float dropout_p, uint64_t dropout_seed, const RowBiasArgs* rb,
+                          cudaStream_t stream);
+cudaError_t launch_embed_bias(const float* e_cam, const float* e_lvl, const void* w,
+                              const float* b, int ncam, int L, int N, int K, float* table,
+                              cudaStream_t s);
 
 // sca_forward with its output stored as fp32 or (out_bf16) bf16; validates
 // like sca_forward.
@@ -119,6 +136,13 @@ msda_status_t sca_rebatched_backward_to(const void* value, msda_dtype_t vdt, con
                                         const int32_t* idx, const int32_t* count,
                                         const int32_t* hits, float* grad_value, long long* acc,
                                         float* grad_loc_rb, float* grad_attn_rb, cudaStream_t s);
+
+// TSA backward rows (msda_backward.cu): location and weight gradients of
+// every queue row, grad_value accumulated (zeroed by the caller); p.B counts
+// BEV samples, the value holds p.B * T items.
+cudaError_t launch_tsa_backward(const Problem& p, int T, const float* ref, const float* off,
+                                const float* logits, const float* grad_out, float* grad_value,
+                                float* grad_loc, float* grad_attn, cudaStream_t s);
 
 // Set the per-thread error message of msda_last_error() and return the code.
 msda_status_t api_fail(msda_status_t code, const char* message);

@@ -231,6 +231,27 @@ struct Dropout {
     int on;
 };
 
+// A bias per (camera, level) instead of per column ("BEV(三) ..." section 3:
+// F~ = F + e_cam + e_level, and (F + e) W^T = F W^T + e W^T): row r of X is
+// pixel v = r mod nv of camera (r div nv) mod ncam, and its level is the last
+// l with start[l] <= v; the bias row is table[(camera * L + level) * N].
+struct RowBias {
+    const float* table;  // [ncam * L, N] or null (then the plain bias)
+    int nv, ncam, L;
+    int start[8];
+};
+
+__device__ __forceinline__ const float* row_bias(const RowBias& rb, int64_t row, int N)
+{
+    const int64_t v = row % rb.nv;
+    const int c = (int)((row / rb.nv) % rb.ncam);
+    int l = 0;
+#pragma unroll
+    for (int i = 1; i < 8; ++i)
+        if (i < rb.L && rb.start[i] <= v) l = i;
+    return rb.table + ((int64_t)c * rb.L + l) * N;
+}
+
 __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1)
 {
 #pragma unroll
@@ -282,7 +303,8 @@ __device__ __forceinline__ void put_row(uint8_t* buf, int lane, const uint32_t (
 __global__ void __launch_bounds__(kGemmThreads, 1)
 proj_gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
                  const __grid_constant__ CUtensorMap map_y, const float* __restrict__ bias,
-                 const float* __restrict__ residual, int y_bf16, int M, int N, int K, Dropout drop)
+                 const float* __restrict__ residual, int y_bf16, int M, int N, int K, Dropout drop,
+                 RowBias rbias)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -447,10 +469,12 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
 #pragma unroll
                     for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
                     const int col = n0 + c0 + 32 * half;
-                    if (bias) {
+                    const float* brow = bias;
+                    if (rbias.table) brow = row_ok ? row_bias(rbias, row, N) : nullptr;
+                    if (brow) {
 #pragma unroll
                         for (int j = 0; j < 32; j += 4) {
-                            const float4 b4 = __ldg(reinterpret_cast<const float4*>(bias + col + j));
+                            const float4 b4 = __ldg(reinterpret_cast<const float4*>(brow + col + j));
                             v[j] += b4.x; v[j + 1] += b4.y; v[j + 2] += b4.z; v[j + 3] += b4.w;
                         }
                     }
@@ -557,13 +581,62 @@ bool make_store_map(CUtensorMap* map, void* base, int M, int N, bool bf16)
 }  // namespace
 }  // namespace msda
 
+namespace msda {
+
+// Bias table of the embedding prologue: table[c * L + l, n] = b[n] +
+// sum_k (e_cam[c, k] + e_level[l, k]) w[n, k] (double accumulation; either
+// embedding may be null).  One thread per table entry.
+__global__ void embed_bias_kernel(const float* __restrict__ e_cam, const float* __restrict__ e_lvl,
+                                  const __nv_bfloat16* __restrict__ w, const float* __restrict__ b,
+                                  int ncam, int L, int N, int K, float* __restrict__ table)
+{
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (int64_t)ncam * L * N) return;
+    const int n = (int)(i % N);
+    const int cl = (int)(i / N);
+    const int c = cl / L, l = cl - c * L;
+    double acc = b ? (double)b[n] : 0.0;
+    for (int k = 0; k < K; ++k) {
+        const float e = (e_cam ? e_cam[(int64_t)c * K + k] : 0.f) +
+                        (e_lvl ? e_lvl[(int64_t)l * K + k] : 0.f);
+        acc += (double)e * (double)__bfloat162float(w[(int64_t)n * K + k]);
+    }
+    table[i] = (float)acc;
+}
+
+cudaError_t launch_embed_bias(const float* e_cam, const float* e_lvl, const void* w,
+                              const float* b, int ncam, int L, int N, int K, float* table,
+                              cudaStream_t s)
+{
+    const int64_t n = (int64_t)ncam * L * N;
+    if (n == 0) return cudaSuccess;
+    embed_bias_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
+        e_cam, e_lvl, static_cast<const __nv_bfloat16*>(w), b, ncam, L, N, K, table);
+    return cudaGetLastError();
+}
+
+msda_status_t linear_impl(const void* x, const void* w, const float* bias, const float* residual,
+                          int32_t M, int32_t N, int32_t K, msda_dtype_t y_dtype, void* y,
+                          float dropout_p, uint64_t dropout_seed, const RowBiasArgs* rb,
+                          cudaStream_t stream);
+
+}  // namespace msda
+
 extern "C" msda_status_t msda_linear_dropout(const void* x, const void* w, const float* bias,
                                              const float* residual, int32_t M, int32_t N,
                                              int32_t K, msda_dtype_t y_dtype, void* y,
                                              float dropout_p, uint64_t dropout_seed,
                                              msda_stream_t stream)
 {
-    using namespace msda;
+    return msda::linear_impl(x, w, bias, residual, M, N, K, y_dtype, y, dropout_p, dropout_seed,
+                             nullptr, (cudaStream_t)stream);
+}
+
+msda_status_t msda::linear_impl(const void* x, const void* w, const float* bias,
+                                const float* residual, int32_t M, int32_t N, int32_t K,
+                                msda_dtype_t y_dtype, void* y, float dropout_p,
+                                uint64_t dropout_seed, const RowBiasArgs* rb, cudaStream_t stream)
+{
     if (!(dropout_p >= 0.f && dropout_p < 1.f))
         return api_fail(MSDA_ERR_INVALID_ARG, "dropout_p must be in [0, 1)");
     if (M < 0) return api_fail(MSDA_ERR_INVALID_ARG, "M must be >= 0");
@@ -598,8 +671,21 @@ extern "C" msda_status_t msda_linear_dropout(const void* x, const void* w, const
     drop.scale = (float)(1.0 / (1.0 - (double)dropout_p));
     drop.key0 = (uint32_t)dropout_seed;
     drop.key1 = (uint32_t)(dropout_seed >> 32);
-    proj_gemm_kernel<<<grid, kGemmThreads, kSmemBytes, (cudaStream_t)stream>>>(
-        mx, mw, my, bias, residual, y_dtype == MSDA_BF16, M, N, K, drop);
+    RowBias rbias;
+    rbias.table = nullptr;
+    rbias.nv = rbias.ncam = rbias.L = 1;
+    for (int i = 0; i < 8; ++i) rbias.start[i] = 0;
+    if (rb) {
+        if (rb->table == nullptr || rb->nv < 1 || rb->ncam < 1 || rb->L < 1 || rb->L > 8)
+            return api_fail(MSDA_ERR_INVALID_ARG, "bad per-(camera, level) bias");
+        rbias.table = rb->table;
+        rbias.nv = rb->nv;
+        rbias.ncam = rb->ncam;
+        rbias.L = rb->L;
+        for (int i = 0; i < rb->L; ++i) rbias.start[i] = rb->start[i];
+    }
+    proj_gemm_kernel<<<grid, kGemmThreads, kSmemBytes, stream>>>(
+        mx, mw, my, bias, residual, y_dtype == MSDA_BF16, M, N, K, drop, rbias);
     return api_cuda(cudaGetLastError(), "msda_linear");
 }
 

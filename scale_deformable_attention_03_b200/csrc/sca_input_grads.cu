@@ -52,7 +52,8 @@ sca_offset_logit_grads_kernel(const float* __restrict__ logits, const int32_t* _
     if (bq >= (int64_t)B * Nq) return;  // warp-uniform
     const int b = (int)(bq / Nq), q = (int)(bq - (int64_t)b * Nq);
     const int n = L * P, S = H * n;
-    const int p = lane < Ncam ? __ldg(pos + ((int64_t)b * Ncam + lane) * Nq + q) : -1;
+    // pos == null: one camera whose row i is query i (the TSA queues)
+    const int p = lane < Ncam ? (pos ? __ldg(pos + ((int64_t)b * Ncam + lane) * Nq + q) : q) : -1;
     const unsigned seen = __ballot_sync(0xffffffffu, p >= 0);
     if (REF) {  // the cameras that do not see the query get zero reference gradients
         for (int i = lane; i < Ncam * R * 2; i += 32) {
@@ -170,7 +171,7 @@ sca_reference_grads_kernel(const int32_t* __restrict__ pos, const float* __restr
     const int q = (int)(cbq % Nq);
     const int64_t cb = cbq / Nq;
     const int b = (int)(cb % B), c = (int)(cb / B);
-    const int p = __ldg(pos + ((int64_t)b * Ncam + c) * Nq + q);
+    const int p = pos ? __ldg(pos + ((int64_t)b * Ncam + c) * Nq + q) : q;
     float* out = grad_ref_cam + cbq * R * 2;
     if (p < 0) {
         if (lane < 2 * R) out[lane] = 0.f;

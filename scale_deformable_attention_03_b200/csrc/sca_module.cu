@@ -3,7 +3,9 @@
 // the Feature" (sections 3, 4, 10-14; the Tencent Cloud walkthrough's
 // listings), on the GPU end to end:
 //   q~    = q + pos                      (bf16, the projections' operand)
-//   V     = F~ W_v^T + b_v               (section 3; tensor cores)
+//   V     = F~ W_v^T + b_v               (section 3; tensor cores; with
+//           F~ = F + e_cam + e_level, the embeddings enter as a bias per
+//           (camera, level): (e_cam + e_level) W_v^T + b_v)
 //   Delta = q~ W_Delta^T + b_Delta       (4.1)
 //   a     = q~ W_alpha^T + b_alpha       (4.2)
 //   g     = SCA(V, Delta, a, rho, mask)  (5-10: compaction, fused MSDA, average;
@@ -65,6 +67,7 @@ struct ModuleWs {
     float* offsets;    // [B * Nq, H L P 2]
     float* logits;     // [B * Nq, H L P]
     void* g16;         // [B * Nq, C] bf16
+    float* embed_bias; // [Ncam * L, C]: the embedding prologue's bias rows
     void* sca;         // sca_forward workspace
     size_t sca_bytes;
     size_t total;
@@ -87,6 +90,7 @@ ModuleWs module_carve(void* base, const msda_dims_t& d, msda_dtype_t vdt)
     w.offsets = reinterpret_cast<float*>(take(rows_q * S * 2 * 4));
     w.logits = reinterpret_cast<float*>(take(rows_q * S * 4));
     w.g16 = take(rows_q * C * 2);
+    w.embed_bias = reinterpret_cast<float*>(take((size_t)d.Ncam * d.L * C * 4));
     w.sca_bytes = msda_workspace_size(d);
     w.sca = take(w.sca_bytes);
     w.total = off;
@@ -131,9 +135,25 @@ extern "C" msda_status_t sca_module_forward(const sca_module_params_t* p,
     cudaError_t e = launch_add_to_bf16(p->query, p->query_pos, w.qt, rows_q * C, s);
     if (e != cudaSuccess) return api_cuda(e, "sca_module_forward: query + pos");
     msda_status_t st;
-    if ((st = msda_linear(p->features, p->w_value, p->b_value, nullptr, (int32_t)rows_v, C, C,
-                          p->value_dtype, w.value, stream)) != MSDA_OK)
-        return st;
+    if (p->camera_embeds || p->level_embeds) {
+        if (d.L > 8 || ((uintptr_t)p->camera_embeds & 3) || ((uintptr_t)p->level_embeds & 3))
+            return api_fail(MSDA_ERR_INVALID_ARG, "embeddings: L <= 8, 4-byte aligned arrays");
+        e = launch_embed_bias(p->camera_embeds, p->level_embeds, p->w_value, p->b_value, d.Ncam,
+                              d.L, C, C, w.embed_bias, s);
+        if (e != cudaSuccess) return api_cuda(e, "sca_module_forward: embedding bias");
+        RowBiasArgs rb;
+        rb.table = w.embed_bias;
+        rb.nv = d.Nv;
+        rb.ncam = d.Ncam;
+        rb.L = d.L;
+        for (int l = 0; l < 8; ++l) rb.start[l] = l < d.L ? (int)level_start_index[l] : 0;
+        st = linear_impl(p->features, p->w_value, nullptr, nullptr, (int32_t)rows_v, C, C,
+                         p->value_dtype, w.value, 0.f, 0, &rb, s);
+    } else {
+        st = msda_linear(p->features, p->w_value, p->b_value, nullptr, (int32_t)rows_v, C, C,
+                         p->value_dtype, w.value, stream);
+    }
+    if (st != MSDA_OK) return st;
     if ((st = msda_linear(w.qt, p->w_offsets, p->b_offsets, nullptr, (int32_t)rows_q, S * 2, C,
                           MSDA_F32, w.offsets, stream)) != MSDA_OK)
         return st;

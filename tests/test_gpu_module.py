@@ -20,9 +20,10 @@ def _bf16_tensor(a):
     return torch.from_numpy(inputs.to_bf16_bits(a).view(np.int16)).cuda().view(torch.bfloat16)
 
 
-@pytest.mark.parametrize("value_bf16,dropout_p", [(False, 0.0), (True, 0.0), (False, 0.1),
-                                                  (True, 0.3)])
-def test_module_matches_oracle(value_bf16, dropout_p):
+@pytest.mark.parametrize("value_bf16,dropout_p,embeds", [(False, 0.0, False), (True, 0.0, False),
+                                                         (False, 0.1, False), (True, 0.3, False),
+                                                         (False, 0.0, True), (True, 0.1, True)])
+def test_module_matches_oracle(value_bf16, dropout_p, embeds):
     rng = np.random.Generator(np.random.PCG64(77))
     w = inputs.workload3(seed=78, bev_h=16, bev_w=20,
                          shapes=[(29, 50), (15, 25), (8, 13), (4, 7)])
@@ -41,19 +42,23 @@ def test_module_matches_oracle(value_bf16, dropout_p):
     bv, bo = (rng.standard_normal(C) * 0.1).astype(np.float32), (rng.standard_normal(C) * 0.1).astype(np.float32)
     boff, bw = rng.standard_normal(2 * S).astype(np.float32), rng.standard_normal(S).astype(np.float32)
 
+    e_cam = (rng.standard_normal((Ncam, C)) * 0.5).astype(np.float32) if embeds else None
+    e_lvl = (rng.standard_normal((L, C)) * 0.5).astype(np.float32) if embeds else None
+
     def t(a):
-        return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+        return None if a is None else torch.from_numpy(np.ascontiguousarray(a)).cuda()
     out = msda.sca_module_forward(
         t(q), t(pos), _bf16_tensor(feats), _bf16_tensor(wv), t(bv), _bf16_tensor(woff), t(boff),
         _bf16_tensor(ww), t(bw), _bf16_tensor(wo), t(bo), t(w.reference_points), t(w.bev_mask),
         w.spatial_shapes, w.level_start_index, L, P,
         value_dtype=torch.bfloat16 if value_bf16 else torch.float32, dropout_p=dropout_p,
-        dropout_seed=0x1234_5678_9ABC)
+        dropout_seed=0x1234_5678_9ABC, camera_embeds=t(e_cam), level_embeds=t(e_lvl))
     torch.cuda.synchronize()
     ref = oracle.sca_module_forward(q, pos, feats, wv, bv, woff, boff, ww, bw, wo, bo,
                                     w.reference_points, w.bev_mask, w.spatial_shapes,
                                     w.level_start_index, L, P, value_bf16=value_bf16,
-                                    dropout_p=dropout_p, dropout_seed=0x1234_5678_9ABC)
+                                    dropout_p=dropout_p, dropout_seed=0x1234_5678_9ABC,
+                                    camera_embeds=e_cam, level_embeds=e_lvl)
     err = np.abs(out.cpu().numpy().astype(np.float64) - ref)
     assert err.max() <= 2e-2, err.max()
     assert msda.lib().msda_linear_timeouts() == 0

@@ -123,3 +123,49 @@ def test_tsa_forward_empty():
     out = msda.tsa_forward(v, s, starts, torch.zeros((0, 16, 1, 2), device="cuda"), z,
                            torch.zeros((0, 16, 8, 1, 4), device="cuda"), 2)
     assert out.shape == (0, 16, 256)
+
+
+def _chain_close(got, want, what):
+    """The chain from the kernel's own fp32 location and weight gradients: sums
+    of up to H*L*P terms that may cancel, bounded relative to the largest."""
+    err = np.abs(got.cpu().numpy().astype(np.float64) - want)
+    assert err.max() <= 1e-4 * (1.0 + np.abs(want).max()), (what, err.max())
+
+
+@pytest.mark.parametrize("case", [CASES[0], CASES[2], CASES[4], CASES[5]],
+                         ids=["case80", "case82", "case84", "case85"])
+@pytest.mark.parametrize("bf16", [False, True])
+def test_tsa_backward(case, bf16):
+    seed, B, T, shapes, H, P, R = case
+    s, starts, value, vt, ref, off, logits = _problem(seed, B, T, shapes, H, P, R, bf16)
+    Nq = ref.shape[1]
+    go = np.random.Generator(np.random.PCG64(seed + 500)).standard_normal(
+        (B, Nq, H * 32)).astype(np.float32)
+    gv, g_off, g_lg, g_ref = msda.tsa_backward(vt, s, starts, dev(ref), dev(off), dev(logits), T,
+                                               dev(go))
+    torch.cuda.synchronize()
+    rv, r_off, r_lg, r_ref = oracle.tsa_backward(value, s, starts, ref, off, logits, T, go)
+    assert_close(gv, rv, False, "tsa grad_value")
+    assert_close(g_off, r_off, False, "tsa grad_sampling_offsets")
+    _chain_close(g_lg, r_lg, "tsa grad_attention_logits")
+    _chain_close(g_ref, r_ref, "tsa grad_reference_points")
+
+
+def test_tsa_backward_bevformer_base_full_size():
+    w = inputs.workload4()
+    ego = np.array([[[1.7, -0.9, 4.0], [0.0, 0.0, 0.0]]], np.float32)
+    ref = oracle.tsa_reference_points(200, 200, ego).astype(np.float32).reshape(2, -1, 1, 2)
+    go = np.random.Generator(np.random.PCG64(89)).standard_normal(
+        (1, w.Nq, w.H * 32)).astype(np.float32)
+    gv, g_off, g_lg, g_ref = msda.tsa_backward(dev(w.value), w.spatial_shapes,
+                                               w.level_start_index, dev(ref),
+                                               dev(w.sampling_offsets), dev(w.attention_logits),
+                                               2, dev(go))
+    torch.cuda.synchronize()
+    rv, r_off, r_lg, r_ref = oracle.tsa_backward(w.value, w.spatial_shapes, w.level_start_index,
+                                                 ref, w.sampling_offsets, w.attention_logits, 2,
+                                                 go)
+    assert_close(gv, rv, False, "tsa 200x200 grad_value")
+    assert_close(g_off, r_off, False, "tsa 200x200 grad_sampling_offsets")
+    _chain_close(g_lg, r_lg, "tsa 200x200 grad_attention_logits")
+    _chain_close(g_ref, r_ref, "tsa 200x200 grad_reference_points")
