@@ -586,6 +586,16 @@ def measure_next_rows(args, w, tensors, flush, stream, hbm_peak):
 
     rows = {}
     bf16 = args.value_dtype == "bf16"
+    with_cpu = args.cpu_seconds > 0
+
+    def cpu_rate(call, work, unit, what):
+        """The oracle timed on one host core on a bounded slice of the same
+        workload (one call), as work per second."""
+        t0 = time.perf_counter()
+        call()
+        el = time.perf_counter() - t0
+        return {"value": work / el, "unit": unit, "cores": 1, "kind": "oracle",
+                "sample": f"{what}: {el:.2f} s on one host core"}
     value, ref, mask, off, logits = (tensors[k] for k in ("value", "ref", "mask", "off",
                                                           "logits"))
     shapes, starts = w.spatial_shapes, w.level_start_index
@@ -617,6 +627,17 @@ def measure_next_rows(args, w, tensors, flush, stream, hbm_peak):
         r = hbm(nbytes, ms)
         r.update(kernel=kname, workload=wk.name,
                  gsamples_per_s=wk.B * wk.Nq * S / (ms * 1e-3) / 1e9)
+        if with_cpu:
+            import oracle
+            nq = wk.Nq
+            sl = (slice(None), slice(0, nq))
+            r["cpu_oracle"] = cpu_rate(
+                lambda: oracle.msda_forward_fused(
+                    wk.value, wk.spatial_shapes, wk.level_start_index,
+                    np.ascontiguousarray(wk.reference_points[sl]),
+                    np.ascontiguousarray(wk.sampling_offsets[sl]),
+                    np.ascontiguousarray(wk.attention_logits[sl])),
+                wk.B * nq * S / 1e9, UNIT, f"all {nq} queries")
         rows[name] = r
         del dv, o, fa
 
@@ -636,6 +657,18 @@ def measure_next_rows(args, w, tensors, flush, stream, hbm_peak):
     r.update(kernel="tsa_forward_group_kernel<float, 2, 2>",
              workload="bevformer-tsa 2 queues x 200x200, H=8, P=4, fp32",
              gsamples_per_s=2 * w4.Nq * w4.H * w4.L * w4.P / (ms * 1e-3) / 1e9)
+    nq4 = 20000
+    sl4 = (slice(None), slice(0, nq4))
+    if with_cpu:
+        import oracle
+        ref4_np = oracle.tsa_reference_points(
+            200, 200, np.array([[[1.7, -0.9, 4.0], [0.0, 0.0, 0.0]]])).reshape(2, -1, 1, 2)
+        r["cpu_oracle"] = cpu_rate(
+            lambda: oracle.tsa_forward(w4.value, w4.spatial_shapes, w4.level_start_index,
+                                       np.ascontiguousarray(ref4_np[sl4]),
+                                       np.ascontiguousarray(w4.sampling_offsets[sl4]),
+                                       np.ascontiguousarray(w4.attention_logits[sl4]), 2),
+            2 * nq4 * w4.H * w4.L * w4.P / 1e9, UNIT, f"the first {nq4} BEV queries")
     rows["tsa_forward"] = r
     ms = timed(lambda: msda.tsa_reference_points(ego, 200, 200, out=ref4))
     rows["tsa_reference_points"] = hbm(2 * w4.Nq * 8 + 24, ms)
@@ -651,6 +684,15 @@ def measure_next_rows(args, w, tensors, flush, stream, hbm_peak):
     r.update(kernel="tsa_backward_kernel + sca_offset_logit_grads_kernel",
              workload="bevformer-tsa 2 queues x 200x200, H=8, P=4, fp32",
              gsamples_per_s=2 * w4.Nq * S4 / (ms * 1e-3) / 1e9)
+    if with_cpu:
+        go4_np = np.random.Generator(np.random.PCG64(4)).standard_normal((1, nq4, w4.H * 32))
+        r["cpu_oracle"] = cpu_rate(
+            lambda: oracle.tsa_backward(w4.value, w4.spatial_shapes, w4.level_start_index,
+                                        np.ascontiguousarray(ref4_np[sl4]),
+                                        np.ascontiguousarray(w4.sampling_offsets[sl4]),
+                                        np.ascontiguousarray(w4.attention_logits[sl4]), 2,
+                                        go4_np),
+            2 * nq4 * S4 / 1e9, UNIT, f"the first {nq4} BEV queries")
     rows["tsa_backward"] = r
     del v4, off4, lg4, out4, ref4, go4, tws
 
@@ -669,6 +711,14 @@ def measure_next_rows(args, w, tensors, flush, stream, hbm_peak):
         tflops = 2.0 * M * N * K / (ms * 1e-3) / 1e12
         r.update(kernel="proj_gemm_kernel (tcgen05)", shape=[M, N, K], y_dtype=y_dtype,
                  tflops=tflops, tensor_frac=tflops / peak_tf, tensor_peak_source=peak_tf_src)
+        if with_cpu and y_dtype == "f32":
+            import oracle
+            mc = 10000
+            xs = x[:mc].float().cpu().numpy()
+            wts = wt.float().cpu().numpy()
+            r["cpu_oracle"] = cpu_rate(lambda: oracle.linear(xs, wts),
+                                       2.0 * mc * N * K / 1e12, "TFLOP/s",
+                                       f"{mc} rows of the same projection")
         rows[f"msda_linear_value_proj_{y_dtype}"] = r
     del x, y
 
@@ -729,6 +779,19 @@ def measure_next_rows(args, w, tensors, flush, stream, hbm_peak):
     r.update(kernel="sca_backward_kernel (+ compaction, zero fill, zero tail)",
              workload="bevformer-base SCA training step, B=2, bf16 value",
              gsamples_per_s=rows5 * w5.H * w5.L * w5.P / (ms * 1e-3) / 1e9)
+    if with_cpu:
+        import oracle
+        nq5 = 1000
+        q5 = slice(0, nq5)
+        m5 = np.ascontiguousarray(w5.bev_mask[:, :, q5])
+        seen5 = int(np.count_nonzero(m5.any(-1)))
+        r["cpu_oracle"] = cpu_rate(
+            lambda: oracle.sca_backward(w5.value, w5.spatial_shapes, w5.level_start_index,
+                                        np.ascontiguousarray(w5.reference_points[:, :, q5]), m5,
+                                        np.ascontiguousarray(w5.sampling_offsets[:, q5]),
+                                        np.ascontiguousarray(w5.attention_logits[:, q5]),
+                                        np.ascontiguousarray(w5.grad_out[:, q5])),
+            seen5 * w5.H * w5.L * w5.P / 1e9, UNIT, f"the first {nq5} BEV queries")
     rows["sca_backward"] = r
     ws5 = torch.empty(int(msda.lib().sca_backward_deterministic_workspace_size(
         msda.Dims(w5.B, w5.Ncam, w5.Nq, w5.Nv, w5.H, w5.L, w5.P, w5.R))), dtype=torch.uint8,

@@ -15,7 +15,9 @@
 // is scaled by 2^32 (exact), rounded once to a 64-bit integer and added with
 // red.global.add.u64 into a fixed-point copy of grad_value; integer addition
 // does not depend on order, so the result is bitwise reproducible, and one
-// conversion kernel rounds it to fp32 at the end.
+// conversion kernel rounds it to fp32 at the end.  The 64-bit adds are
+// issued lane per channel (one warp instruction adds a whole 256-byte corner
+// slice, eight full L2 sectors), from a per-sample copy of the coefficients.
 // The dot products and everything derived from them are formed in double
 // (a product of two fp32 numbers is exact in double): the location gradient
 // multiplies a difference of dot products by alpha * W_l (up to ~40 at
@@ -28,6 +30,13 @@
 namespace msda {
 
 constexpr int kBwdRowsPerTile = 2;
+
+// The four corners of one sample, for the deterministic adds (read as two
+// broadcast 16-byte loads).
+struct __align__(16) DetEntry {
+    int off[4];
+    float wa[4];  // alpha * bilinear weight
+};
 
 struct BwdTable {
     int off[4][kMetaStride];
@@ -102,17 +111,9 @@ struct BwdLanes<float> {
                 const float4 v = __ldg(reinterpret_cast<const float4*>(vb + o + 4 * t));
                 part[k] = (double)go.x * v.x + (double)go.y * v.y + (double)go.z * v.z +
                           (double)go.w * v.w;
-                const float w = tab.alpha[j] * tab.wb[g][j];
-                if (w != 0.f) {
-                    if (DET) {
-                        long long* dst = gvi + o + 4 * t;
-                        red_add_fix(dst, w * go.x);
-                        red_add_fix(dst + 1, w * go.y);
-                        red_add_fix(dst + 2, w * go.z);
-                        red_add_fix(dst + 3, w * go.w);
-                    } else {
-                        red_add_v4(gvb + o + 4 * t, w * go.x, w * go.y, w * go.z, w * go.w);
-                    }
+                if (!DET) {
+                    const float w = tab.alpha[j] * tab.wb[g][j];
+                    if (w != 0.f) red_add_v4(gvb + o + 4 * t, w * go.x, w * go.y, w * go.z, w * go.w);
                 }
             }
         }
@@ -178,13 +179,9 @@ struct BwdLanes<__nv_bfloat16> {
 #pragma unroll
                 for (int i = 0; i < 8; ++i) d += (double)go[i] * v[i];
                 part[k] = d;
-                const float w = tab.alpha[j] * tab.wb[g][j];
-                if (w != 0.f) {
-                    if (DET) {
-                        long long* dst = gvi + o + 8 * t;
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) red_add_fix(dst + i, w * go[i]);
-                    } else {
+                if (!DET) {
+                    const float w = tab.alpha[j] * tab.wb[g][j];
+                    if (w != 0.f) {
                         float* dst = gvb + o + 8 * t;
                         red_add_v4(dst, w * go[0], w * go[1], w * go[2], w * go[3]);
                         red_add_v4(dst + 4, w * go[4], w * go[5], w * go[6], w * go[7]);
@@ -222,9 +219,12 @@ __device__ __forceinline__ void row_backward(const VT* __restrict__ vb, int H, i
                                              const LaneSamples<NC>& ls, BwdTable& tab,
                                              const float* __restrict__ grow, float scale,
                                              float* __restrict__ gvb, long long* __restrict__ gvi,
+                                             DetEntry* __restrict__ det,
                                              float* __restrict__ gloc_row,
                                              float* __restrict__ gattn_row, int lane)
 {
+    // DET: channel `lane` of the row's upstream gradient, as BwdLanes forms it
+    const float go_c = DET ? __ldg(grow + lane) / scale : 0.f;
     float a[NC];
     row_weights<FUSED, NC>(wl, n, lane, a);
     BwdLanes<VT> lanes;
@@ -258,11 +258,28 @@ __device__ __forceinline__ void row_backward(const VT* __restrict__ vb, int H, i
         tab.lx[lane] = cr.lx;
         tab.ly[lane] = cr.ly;
         tab.alpha[lane] = a[c];
+        if (DET) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                det[lane].off[q] = cr.off[q];
+                det[lane].wa[q] = a[c] * cr.w[q];  // the same product as the fp32 path
+            }
+        }
         __syncwarp();
         float res_w = 0.f, res_x = 0.f, res_y = 0.f;
         const int cnt = min(32, n - c * 32);
         for (int j0 = 0; j0 < cnt; j0 += 8) {
             const double d = lanes.template batch<DET>(vb, gvb, gvi, tab, j0, cnt, lane);
+            if (DET) {  // lane = channel: one 256-byte slice per (sample, corner)
+                for (int j = j0; j < min(j0 + 8, cnt); ++j) {
+                    const int4 o = *reinterpret_cast<const int4*>(det[j].off);
+                    const float4 w = *reinterpret_cast<const float4*>(det[j].wa);
+                    if (o.x >= 0 && w.x != 0.f) red_add_fix(gvi + o.x + lane, w.x * go_c);
+                    if (o.y >= 0 && w.y != 0.f) red_add_fix(gvi + o.y + lane, w.y * go_c);
+                    if (o.z >= 0 && w.z != 0.f) red_add_fix(gvi + o.z + lane, w.z * go_c);
+                    if (o.w >= 0 && w.w != 0.f) red_add_fix(gvi + o.w + lane, w.w * go_c);
+                }
+            }
             const int js = j0 + held;  // the sample whose D_g this lane holds
             const bool valid = js < cnt;
             double cw = valid ? (double)tab.wb[g][js] * d : 0.0;
@@ -304,6 +321,7 @@ msda_backward_kernel(const VT* __restrict__ value, const float* __restrict__ loc
 {
     __shared__ SmemLevels s_lv;
     __shared__ __align__(16) BwdTable s_tab[kWarps];
+    __shared__ DetEntry s_det[DET ? kWarps : 1][kMetaStride];
     stage_levels(s_lv, levels);
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -329,7 +347,8 @@ msda_backward_kernel(const VT* __restrict__ value, const float* __restrict__ loc
                                          attn + item * S, nullptr, S, ls, s_tab[warp],
                                          grad_out + item * kHeadDim, 1.f, grad_value + vofs,
                                          DET ? grad_value_fix + vofs : nullptr,
-                                         grad_loc + item * S * 2, grad_attn + item * S, lane);
+                                         s_det[DET ? warp : 0], grad_loc + item * S * 2,
+                                         grad_attn + item * S, lane);
     }
 }
 
@@ -346,6 +365,7 @@ sca_backward_kernel(const VT* __restrict__ value, const float* __restrict__ off,
 {
     __shared__ SmemLevels s_lv;
     __shared__ __align__(16) BwdTable s_tab[kWarps];
+    __shared__ DetEntry s_det[DET ? kWarps : 1][kMetaStride];
     __shared__ int s_prefix[kMaxBatchCameras + 1];
     const int nbc = B * Ncam;
     stage_levels(s_lv, levels);
@@ -383,8 +403,8 @@ sca_backward_kernel(const VT* __restrict__ value, const float* __restrict__ off,
                                             ls, s_tab[warp], grad_out + bqh * kHeadDim, scale,
                                             grad_value + vofs,
                                             DET ? grad_value_fix + vofs : nullptr,
-                                            grad_loc_rb + rowh * S * 2, grad_attn_rb + rowh * S,
-                                            lane);
+                                            s_det[DET ? warp : 0], grad_loc_rb + rowh * S * 2,
+                                            grad_attn_rb + rowh * S, lane);
         }
     }
 }
@@ -427,8 +447,8 @@ tsa_backward_kernel(const VT* __restrict__ value, const float* __restrict__ off,
         row_backward<VT, true, NC, false>(value + vofs, H, cur.h, off + item * S * 2,
                                           logits + item * S, ref + r * R * 2, S, ls, s_tab[warp],
                                           grad_out + gitem * kHeadDim, (float)T,
-                                          grad_value + vofs, nullptr, grad_loc + item * S * 2,
-                                          grad_attn + item * S, lane);
+                                          grad_value + vofs, nullptr, nullptr,
+                                          grad_loc + item * S * 2, grad_attn + item * S, lane);
     }
 }
 

@@ -44,6 +44,10 @@ constexpr int kMaxBatchCameras = 1024;  // B * Ncam limit of the SCA kernels
 #else
 #define MSDA_GATHER_BOUNDS __launch_bounds__(kThreads)
 #endif
+// Consecutive rows per CTA tile of the small-row group kernels.
+#ifndef MSDA_GROUP_ROWS_PER_TILE
+#define MSDA_GROUP_ROWS_PER_TILE 16
+#endif
 // Minimum resident CTAs of the small-row group kernels (a register cap).
 #ifndef MSDA_GROUP_MIN_CTAS
 #define MSDA_GROUP_MIN_CTAS 3

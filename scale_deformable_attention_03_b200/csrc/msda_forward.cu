@@ -12,6 +12,7 @@
 namespace msda {
 
 constexpr int kRowsPerTile = MSDA_ROWS_PER_TILE;
+constexpr int kGroupRowsPerTile = MSDA_GROUP_ROWS_PER_TILE;
 
 template <typename VT, bool FUSED, int NC, int HP>
 __global__ void MSDA_GATHER_BOUNDS
@@ -87,7 +88,9 @@ msda_forward_kernel(const VT* __restrict__ value, const float* __restrict__ lo,
 }
 
 // K1g: rows with L*P <= 16, G = 32 / npad heads per warp item (see
-// group_compute).  Items are (row, head group), head groups fastest.
+// group_compute).  Items are (row, head group), head groups fastest; a CTA
+// owns kGroupRowsPerTile consecutive rows (more than K1: a row has fewer
+// samples, and neighbouring queries share more of their reads).
 template <typename VT, bool FUSED, int NPL>
 __global__ void MSDA_GROUP_BOUNDS
 msda_forward_group_kernel(const VT* __restrict__ value, const float* __restrict__ lo,
@@ -108,10 +111,10 @@ msda_forward_group_kernel(const VT* __restrict__ value, const float* __restrict_
     const int G = 32 >> npad_log2;
     const int HG = (H + G - 1) / G;  // head groups per row
     const int64_t rows = (int64_t)B * Nq;
-    const int64_t row0 = (int64_t)blockIdx.x * kRowsPerTile;
+    const int64_t row0 = (int64_t)blockIdx.x * kGroupRowsPerTile;
     const int b0 = (int)(row0 / Nq);
     const int q0 = (int)(row0 - (int64_t)b0 * Nq);
-    const int n_items = kRowsPerTile * HG;
+    const int n_items = kGroupRowsPerTile * HG;
 
     struct Item {
         bool ok, valid;
@@ -173,7 +176,7 @@ static cudaError_t launch_group(const Problem& p, const float* lo, const float* 
     const int S = p.L * p.P;
     int npad_log2 = 2;
     while ((1 << npad_log2) < S) ++npad_log2;
-    const unsigned grid = (unsigned)((rows + kRowsPerTile - 1) / kRowsPerTile);
+    const unsigned grid = (unsigned)((rows + kGroupRowsPerTile - 1) / kGroupRowsPerTile);
     const VT* v = static_cast<const VT*>(p.value);
     switch (npad_log2) {
 #define MSDA_GROUP_CASE(NPLV)                                                                    \

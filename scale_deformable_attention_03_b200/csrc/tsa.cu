@@ -15,6 +15,7 @@
 namespace msda {
 
 constexpr int kTsaRowsPerTile = MSDA_ROWS_PER_TILE;
+constexpr int kTsaGroupRowsPerTile = MSDA_GROUP_ROWS_PER_TILE;
 
 // One thread per (b, t, q).  The listing reads delta_x, delta_y (metres) and
 // the yaw in degrees from the CAN bus and uses 0.512 m BEV cells, then breaks
@@ -84,10 +85,10 @@ tsa_forward_group_kernel(const VT* __restrict__ value, const float* __restrict__
     const int S = L * P;
     const int HG = (H + G - 1) / G;
     const int64_t rows = (int64_t)B * Nq;
-    const int64_t row0 = (int64_t)blockIdx.x * kTsaRowsPerTile;
+    const int64_t row0 = (int64_t)blockIdx.x * kTsaGroupRowsPerTile;
     const int b0 = (int)(row0 / Nq);
     const int q0 = (int)(row0 - (int64_t)b0 * Nq);
-    const int n_items = kTsaRowsPerTile * HG;
+    const int n_items = kTsaGroupRowsPerTile * HG;
     const int64_t vstride = (int64_t)Nv * H * kHeadDim;
     const float inv_t = 1.f / (float)T;
 
@@ -253,6 +254,8 @@ static cudaError_t launch_tsa_t(const Problem& p, const float* ref, const float*
     const int64_t rows = (int64_t)p.B * p.Nq;
     if (rows == 0) return cudaSuccess;
     const unsigned grid = (unsigned)((rows + kTsaRowsPerTile - 1) / kTsaRowsPerTile);
+    const unsigned group_grid =
+        (unsigned)((rows + kTsaGroupRowsPerTile - 1) / kTsaGroupRowsPerTile);
     const VT* v = static_cast<const VT*>(p.value);
     const int S = p.L * p.P;
     if (S <= 16 && p.H > 1) {
@@ -261,7 +264,7 @@ static cudaError_t launch_tsa_t(const Problem& p, const float* ref, const float*
         switch (npad_log2) {
 #define TSA_GROUP_CASE(NPLV)                                                                     \
     case NPLV:                                                                                   \
-        tsa_forward_group_kernel<VT, T, NPLV><<<grid, kThreads, 0, s>>>(                         \
+        tsa_forward_group_kernel<VT, T, NPLV><<<group_grid, kThreads, 0, s>>>(                   \
             v, off, logits, ref, out, p.B, p.Nq, p.Nv, p.H, p.L, p.P, p.R, p.lv);                \
         break;
             TSA_GROUP_CASE(2)
