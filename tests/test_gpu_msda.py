@@ -98,16 +98,25 @@ CASES = [
 
 
 @pytest.mark.parametrize("case", CASES, ids=[f"case{c[0]}" for c in CASES])
-def test_random_shapes(case):
+@pytest.mark.parametrize("bf16", [False, True])
+def test_random_shapes(case, bf16):
+    """Every kernel layout: one head per warp (one to four sample chunks),
+    head pairs (bf16, even H), several heads per warp (L*P <= 16), 1-pixel
+    levels, 8 levels of 16 points."""
     seed, B, Nq, H, shapes, P, R = case
     s, starts, value, loc, logits, ref, off = _random_problem(seed, B, Nq, H, shapes, P, R)
     L = len(shapes)
+    vt = dev(value)
+    if bf16:
+        bits = inputs.to_bf16_bits(value)
+        value = inputs.bf16_bits_to_f32(bits)
+        vt = dev(bits.view(np.int16)).view(torch.bfloat16)
     weights = softmax_weights(logits, L * P)
-    out = msda.msda_forward(dev(value), s, starts, dev(loc), dev(weights))
-    out_f = msda.msda_forward_fused(dev(value), s, starts, dev(ref), dev(off), dev(logits))
+    out = msda.msda_forward(vt, s, starts, dev(loc), dev(weights))
+    out_f = msda.msda_forward_fused(vt, s, starts, dev(ref), dev(off), dev(logits))
     torch.cuda.synchronize()
-    assert_close(out, oracle.msda_forward(value, s, starts, loc, weights), False, "given")
-    assert_close(out_f, oracle.msda_forward_fused(value, s, starts, ref, off, logits), False,
+    assert_close(out, oracle.msda_forward(value, s, starts, loc, weights), bf16, "given")
+    assert_close(out_f, oracle.msda_forward_fused(value, s, starts, ref, off, logits), bf16,
                  "fused")
 
 
