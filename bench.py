@@ -639,6 +639,26 @@ def measure_next_rows(args, w, tensors, flush, stream, hbm_peak):
                     np.ascontiguousarray(wk.attention_logits[sl])),
                 wk.B * nq * S / 1e9, UNIT, f"all {nq} queries")
         rows[name] = r
+        if name == "msda_forward_fused_detr":
+            # the same encoder's backward from given locations and weights
+            # (prepared with plain torch ops, outside the timed region)
+            wh = torch.tensor([[w_, h_] for h_, w_ in wk.spatial_shapes], dtype=torch.float32,
+                              device="cuda").view(1, 1, 1, wk.L, 1, 2)
+            loc = (dv["ref"].view(wk.B, wk.Nq, 1, 1, 1, 2) + dv["off"] / wh).contiguous()
+            wts = torch.softmax(dv["logits"].view(wk.B, wk.Nq, wk.H, -1), -1).view(
+                dv["logits"].shape).contiguous()
+            gout = torch.randn((wk.B, wk.Nq, wk.H * 32), device="cuda")
+            grads = msda.msda_backward(dv["value"], wk.spatial_shapes, wk.level_start_index,
+                                       loc, wts, gout)
+            ms = timed(lambda: msda.msda_backward(dv["value"], wk.spatial_shapes,
+                                                  wk.level_start_index, loc, wts, gout, *grads))
+            # value read and grad_value written once, locations and weights
+            # read and their gradients written once, grad_out read once
+            r = hbm(2 * wk.value.nbytes + wk.B * wk.Nq * S * 12 * 2 + gout.numel() * 4, ms)
+            r.update(kernel="zero_kernel + backward_group_kernel<float, 4, false, false>",
+                     workload=wk.name, gsamples_per_s=wk.B * wk.Nq * S / (ms * 1e-3) / 1e9)
+            rows["msda_backward_detr"] = r
+            del loc, wts, gout, grads
         del dv, o, fa
 
     # f4: TSA, two queues of the 200x200 BEV, ego motion (1.7 m, -0.9 m, 4 deg)
@@ -681,7 +701,7 @@ def measure_next_rows(args, w, tensors, flush, stream, hbm_peak):
     S4 = w4.H * w4.L * w4.P
     r = hbm(tsa_algorithmic_bytes(w4, 2, 4) + w4.Nq * w4.H * 32 * 4 + w4.value.size * 4
             + 2 * w4.Nq * (S4 * 3 + w4.R * 2) * 4, ms)
-    r.update(kernel="tsa_backward_kernel + sca_offset_logit_grads_kernel",
+    r.update(kernel="backward_group_kernel<float, 2, true, false> + sca_offset_logit_grads_kernel",
              workload="bevformer-tsa 2 queues x 200x200, H=8, P=4, fp32",
              gsamples_per_s=2 * w4.Nq * S4 / (ms * 1e-3) / 1e9)
     if with_cpu:

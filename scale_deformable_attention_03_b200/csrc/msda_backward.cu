@@ -73,6 +73,40 @@ __device__ __forceinline__ double dw_dly(int g, float lx)
     return (g >> 1) ? a : -a;
 }
 
+// Butterfly reduce-scatter over the lanes that differ only in the low bits
+// of t (three bits for eight entries, two for four): lane t ends with the
+// full sum of entry t (t mod the entry count).
+__device__ __forceinline__ double reduce_scatter8(const double (&part)[8], int t)
+{
+    double q[4], r[2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const bool hi = t & 4;
+        q[i] = (hi ? part[i + 4] : part[i]) +
+               __shfl_xor_sync(0xffffffffu, hi ? part[i] : part[i + 4], 4);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const bool hi = t & 2;
+        r[i] = (hi ? q[i + 2] : q[i]) + __shfl_xor_sync(0xffffffffu, hi ? q[i] : q[i + 2], 2);
+    }
+    const bool hi = t & 1;
+    return (hi ? r[1] : r[0]) + __shfl_xor_sync(0xffffffffu, hi ? r[0] : r[1], 1);
+}
+
+__device__ __forceinline__ double reduce_scatter4(const double (&part)[4], int t)
+{
+    double q[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const bool hi = t & 2;
+        q[i] = (hi ? part[i + 2] : part[i]) +
+               __shfl_xor_sync(0xffffffffu, hi ? part[i] : part[i + 2], 2);
+    }
+    const bool hi = t & 1;
+    return (hi ? q[1] : q[0]) + __shfl_xor_sync(0xffffffffu, hi ? q[0] : q[1], 1);
+}
+
 // Samples are processed eight at a time.  Each lane forms its partial dot
 // products <grad_out, V_g> for the eight samples (over its own channels), and
 // a butterfly reduce-scatter over the lanes that share a corner leaves every
@@ -117,20 +151,7 @@ struct BwdLanes<float> {
                 }
             }
         }
-        double q[4], r[2];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const bool hi = t & 4;
-            q[i] = (hi ? part[i + 4] : part[i]) +
-                   __shfl_xor_sync(0xffffffffu, hi ? part[i] : part[i + 4], 4);
-        }
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const bool hi = t & 2;
-            r[i] = (hi ? q[i + 2] : q[i]) + __shfl_xor_sync(0xffffffffu, hi ? q[i] : q[i + 2], 2);
-        }
-        const bool hi = t & 1;
-        return (hi ? r[1] : r[0]) + __shfl_xor_sync(0xffffffffu, hi ? r[0] : r[1], 1);
+        return reduce_scatter8(part, t);
     }
     __device__ __forceinline__ static double reduce_groups(double v)
     {
@@ -189,15 +210,7 @@ struct BwdLanes<__nv_bfloat16> {
                 }
             }
         }
-        double q[2];
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const bool hi = t & 2;
-            q[i] = (hi ? part[i + 2] : part[i]) +
-                   __shfl_xor_sync(0xffffffffu, hi ? part[i] : part[i + 2], 2);
-        }
-        const bool hi = t & 1;
-        return (hi ? q[1] : q[0]) + __shfl_xor_sync(0xffffffffu, hi ? q[0] : q[1], 1);
+        return reduce_scatter4(part, t);
     }
     __device__ __forceinline__ static double reduce_groups(double v)
     {
@@ -308,6 +321,223 @@ __device__ __forceinline__ void row_backward(const VT* __restrict__ vb, int H, i
         }
         __syncwarp();
     }
+}
+
+// ---------------------------------------------------------------------------
+// Grouped backward for rows of L*P <= 16 samples, in the forward's group
+// layout (see group_compute): a warp takes G = 32 / npad heads of one row and
+// lane (s, k) builds sample k of head h0 + s, so the softmax, the corner
+// decision and the table cost one pass per 32 samples instead of one per
+// head.  The batches of eight then walk the 32-entry table in order, each
+// sample with its own head's upstream gradient (a per-warp copy of grad_out,
+// already divided by the scale).
+
+struct __align__(16) GroupBwdTable {
+    int2 ow[32][4];        // corner g of sample j: offset (-1 outside), alpha * w_g (bits)
+    float2 l[32];          // (lx, ly) of sample j
+    float go[32 * 8];      // grad_out / scale of the heads, head s at 32 s
+};
+
+template <typename VT>
+struct GroupBwdLanes;
+
+// fp32 value: lanes 8g + t hold corner g, channels 4t..4t+3 (as BwdLanes).
+template <>
+struct GroupBwdLanes<float> {
+    __device__ __forceinline__ static int group(int lane) { return lane >> 3; }
+    __device__ __forceinline__ static int held(int lane) { return lane & 7; }
+    __device__ __forceinline__ static int holder(int u) { return u; }
+    template <bool DET>
+    __device__ __forceinline__ static double corner(const float* __restrict__ vb,
+                                                    float* __restrict__ gvb, int2 e, float4 go,
+                                                    int t)
+    {
+        if (e.x < 0) return 0.0;
+        const float4 v = __ldg(reinterpret_cast<const float4*>(vb + e.x + 4 * t));
+        if (!DET) {
+            const float w = __int_as_float(e.y);
+            if (w != 0.f) red_add_v4(gvb + e.x + 4 * t, w * go.x, w * go.y, w * go.z, w * go.w);
+        }
+        return (double)go.x * v.x + (double)go.y * v.y + (double)go.z * v.z + (double)go.w * v.w;
+    }
+    // Samples j0 .. j0 + 7; with npad = 4 the second four belong to the next head.
+    template <int NPL, bool DET>
+    __device__ __forceinline__ static double batch(const float* __restrict__ vb,
+                                                   float* __restrict__ gvb,
+                                                   const GroupBwdTable& tab, int j0, int lane)
+    {
+        const int g = lane >> 3, t = lane & 7;
+        const float* gs = tab.go + (j0 >> NPL) * kHeadDim + 4 * t;
+        const float4 ga = *reinterpret_cast<const float4*>(gs);
+        const float4 gb = NPL == 2 ? *reinterpret_cast<const float4*>(gs + kHeadDim) : ga;
+        double part[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            part[k] = corner<DET>(vb, gvb, tab.ow[j0 + k][g], (NPL == 2 && k >= 4) ? gb : ga, t);
+        return reduce_scatter8(part, t);
+    }
+};
+
+// bf16 value: lanes 16s + 4g + t hold corner g, channels 8t..8t+7, of the
+// samples j0 + 2k + s (as BwdLanes).
+template <>
+struct GroupBwdLanes<__nv_bfloat16> {
+    __device__ __forceinline__ static int group(int lane) { return (lane >> 2) & 3; }
+    __device__ __forceinline__ static int held(int lane) { return 2 * (lane & 3) + (lane >> 4); }
+    __device__ __forceinline__ static int holder(int u) { return 16 * (u & 1) + (u >> 1); }
+    template <bool DET>
+    __device__ __forceinline__ static double corner(const __nv_bfloat16* __restrict__ vb,
+                                                    float* __restrict__ gvb, int2 e, float4 g0,
+                                                    float4 g1, int t)
+    {
+        if (e.x < 0) return 0.0;
+        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(vb + e.x + 8 * t));
+        float v[8];
+        bf16x2_to_f32(raw.x, v[0], v[1]);
+        bf16x2_to_f32(raw.y, v[2], v[3]);
+        bf16x2_to_f32(raw.z, v[4], v[5]);
+        bf16x2_to_f32(raw.w, v[6], v[7]);
+        if (!DET) {
+            const float w = __int_as_float(e.y);
+            if (w != 0.f) {
+                float* dst = gvb + e.x + 8 * t;
+                red_add_v4(dst, w * g0.x, w * g0.y, w * g0.z, w * g0.w);
+                red_add_v4(dst + 4, w * g1.x, w * g1.y, w * g1.z, w * g1.w);
+            }
+        }
+        return (double)g0.x * v[0] + (double)g0.y * v[1] + (double)g0.z * v[2] +
+               (double)g0.w * v[3] + (double)g1.x * v[4] + (double)g1.y * v[5] +
+               (double)g1.z * v[6] + (double)g1.w * v[7];
+    }
+    template <int NPL, bool DET>
+    __device__ __forceinline__ static double batch(const __nv_bfloat16* __restrict__ vb,
+                                                   float* __restrict__ gvb,
+                                                   const GroupBwdTable& tab, int j0, int lane)
+    {
+        const int s = lane >> 4, g = (lane >> 2) & 3, t = lane & 3;
+        const float4* gs =
+            reinterpret_cast<const float4*>(tab.go + (j0 >> NPL) * kHeadDim + 8 * t);
+        const float4 ga0 = gs[0], ga1 = gs[1];
+        const float4 gb0 = NPL == 2 ? gs[kHeadDim / 4] : ga0;
+        const float4 gb1 = NPL == 2 ? gs[kHeadDim / 4 + 1] : ga1;
+        double part[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const bool second = NPL == 2 && k >= 2;  // samples j0 + 4 .. j0 + 7
+            part[k] = corner<DET>(vb, gvb, tab.ow[j0 + 2 * k + s][g], second ? gb0 : ga0,
+                                  second ? gb1 : ga1, t);
+        }
+        return reduce_scatter4(part, t);
+    }
+};
+
+// One row, heads h0 .. h0 + G - 1 (those < H).  The lane's inputs come
+// preloaded: a (logit, or the weight when !FUSED), v (offset, or the
+// location), r (reference point), `valid` = the lane's sample exists, go =
+// the lane's channel of each head's grad_out / scale.  gvb / gvi: grad_value
+// of the batch item or its fixed-point copy; gloc0 [G, S, 2] and gattn0
+// [G, S]: head h0's gradients (+S per head).
+template <typename VT, bool FUSED, int NPL, bool DET>
+__device__ __forceinline__ void group_backward(const VT* __restrict__ vb, int H, int h0, int S,
+                                               float a, float2 v, float2 r, bool valid,
+                                               const float (&go)[32 >> NPL], const GroupLane& gl,
+                                               GroupBwdTable& tab, float* __restrict__ gvb,
+                                               long long* __restrict__ gvi,
+                                               float* __restrict__ gloc0,
+                                               float* __restrict__ gattn0, int lane)
+{
+    constexpr int G = 32 >> NPL;
+    constexpr int npad = 1 << NPL;
+    if (FUSED) {
+        const float m = segment_max(a, npad);
+        const float e = valid ? expf(a - m) : 0.f;
+        const float z = segment_sum(e, npad);
+        a = valid ? e / z : 0.f;
+    } else if (!valid) {
+        a = 0.f;
+    }
+    Corners cr;
+    if (valid) {
+        float sx = v.x, sy = v.y;
+        if (FUSED) {
+            sx = __fadd_rn(r.x, __fdiv_rn(v.x, (float)gl.w));
+            sy = __fadd_rn(r.y, __fdiv_rn(v.y, (float)gl.h));
+        }
+        locate(sx, sy, gl.h, gl.w, gl.start, H, h0 + gl.s, cr);
+    } else {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            cr.off[g] = -1;
+            cr.w[g] = 0.f;
+        }
+        cr.lx = cr.ly = 0.f;
+        cr.valid = false;
+    }
+    int4* row = reinterpret_cast<int4*>(tab.ow[lane]);
+    row[0] = make_int4(cr.off[0], __float_as_int(a * cr.w[0]), cr.off[1],
+                       __float_as_int(a * cr.w[1]));
+    row[1] = make_int4(cr.off[2], __float_as_int(a * cr.w[2]), cr.off[3],
+                       __float_as_int(a * cr.w[3]));
+    tab.l[lane] = make_float2(cr.lx, cr.ly);
+#pragma unroll
+    for (int i = 0; i < G; ++i) tab.go[i * kHeadDim + lane] = go[i];
+    __syncwarp();
+
+    using Lanes = GroupBwdLanes<VT>;
+    const int g = Lanes::group(lane);
+    const int held = Lanes::held(lane);
+    const int nheads = min(G, H - h0);
+    float res_w = 0.f, res_x = 0.f, res_y = 0.f;
+#pragma unroll
+    for (int j0 = 0; j0 < 32; j0 += 8) {
+        if ((j0 >> NPL) >= nheads) break;
+        const double d = Lanes::template batch<NPL, DET>(vb, gvb, tab, j0, lane);
+        if (DET) {  // lane = channel: one 256-byte slice per (sample, corner)
+#pragma unroll
+            for (int j = j0; j < j0 + 8; ++j) {
+                const int4* e = reinterpret_cast<const int4*>(tab.ow[j]);
+                const int4 p = e[0], q = e[1];
+                const float go_c = tab.go[(j >> NPL) * kHeadDim + lane];
+                if (p.x >= 0 && __int_as_float(p.y) != 0.f)
+                    red_add_fix(gvi + p.x + lane, __int_as_float(p.y) * go_c);
+                if (p.z >= 0 && __int_as_float(p.w) != 0.f)
+                    red_add_fix(gvi + p.z + lane, __int_as_float(p.w) * go_c);
+                if (q.x >= 0 && __int_as_float(q.y) != 0.f)
+                    red_add_fix(gvi + q.x + lane, __int_as_float(q.y) * go_c);
+                if (q.z >= 0 && __int_as_float(q.w) != 0.f)
+                    red_add_fix(gvi + q.z + lane, __int_as_float(q.w) * go_c);
+            }
+        }
+        // d = D_g of sample j0 + held; its bilinear weight and the weight's
+        // derivatives follow from (lx, ly) as in locate()
+        const float2 l = tab.l[j0 + held];
+        const float hx = __fsub_rn(1.f, l.x), hy = __fsub_rn(1.f, l.y);
+        const float wg = __fmul_rn((g & 1) ? l.x : hx, (g >> 1) ? l.y : hy);
+        double cw = (double)wg * d;
+        double cx = dw_dlx(g, l.y) * d;
+        double cy = dw_dly(g, l.x) * d;
+        cw = BwdLanes<VT>::reduce_groups(cw);
+        cx = BwdLanes<VT>::reduce_groups(cx);
+        cy = BwdLanes<VT>::reduce_groups(cy);
+        // sample j0 + u lands on lane j0 + u
+        const int src = Lanes::holder(lane & 7);
+        const float tw = __shfl_sync(0xffffffffu, (float)cw, src);
+        const float tx = __shfl_sync(0xffffffffu, (float)cx, src);
+        const float ty = __shfl_sync(0xffffffffu, (float)cy, src);
+        if ((lane & ~7) == j0) {
+            res_w = tw;
+            res_x = tx;
+            res_y = ty;
+        }
+    }
+    if (valid) {
+        const int j = gl.s * S + gl.k;
+        gattn0[j] = res_w;
+        *reinterpret_cast<float2*>(gloc0 + 2 * j) =
+            make_float2(cr.valid ? a * (float)gl.w * res_x : 0.f,
+                        cr.valid ? a * (float)gl.h * res_y : 0.f);
+    }
+    __syncwarp();
 }
 
 template <typename VT, int NC, bool DET>
@@ -452,6 +682,137 @@ tsa_backward_kernel(const VT* __restrict__ value, const float* __restrict__ off,
     }
 }
 
+constexpr int kBwdGroupRowsPerTile = MSDA_GROUP_ROWS_PER_TILE;
+
+// Rows with L*P <= 16: a warp item is (row, head group), see group_backward.
+// TSA: rows are (b * T + t, q), each queue receiving grad_out[b] / T.  MSDA
+// (T = 1, !FUSED): rows are (b, q) with the locations and weights given.
+template <typename VT, int NPL, bool FUSED, bool DET>
+__global__ void __launch_bounds__(kThreads)
+backward_group_kernel(const VT* __restrict__ value, const float* __restrict__ off,
+                      const float* __restrict__ logits, const float* __restrict__ ref,
+                      const float* __restrict__ grad_out, float* __restrict__ grad_value,
+                      long long* __restrict__ grad_value_fix, float* __restrict__ grad_loc,
+                      float* __restrict__ grad_attn, int BT, int T, int Nq, int Nv, int H, int L,
+                      int P, int R, Levels levels)
+{
+    constexpr int G = 32 >> NPL;
+    __shared__ SmemLevels s_lv;
+    __shared__ GroupBwdTable s_tab[kWarps];
+    stage_levels(s_lv, levels);
+    __syncthreads();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    GroupLane gl;
+    group_lane(s_lv, L, P, R, NPL, lane, gl);
+    const int S = L * P;
+    const int HG = (H + G - 1) / G;
+    const int64_t rows = (int64_t)BT * Nq;
+    const int64_t row0 = (int64_t)blockIdx.x * kBwdGroupRowsPerTile;
+    const int bt0 = (int)(row0 / Nq);
+    const int q0 = (int)(row0 - (int64_t)bt0 * Nq);
+    const int n_items = kBwdGroupRowsPerTile * HG;
+    const int64_t vstride = (int64_t)Nv * H * kHeadDim;
+    const float scale = (float)T;
+
+    struct Item {
+        bool ok, valid;
+        int bt, q, h0;
+        int64_t r;
+    };
+    auto resolve = [&](int it, const ItemCursor& cur) {
+        Item x;
+        x.r = row0 + cur.rr;
+        x.ok = it < n_items && x.r < rows;
+        x.h0 = cur.h * G;
+        x.valid = gl.in && x.h0 + gl.s < H;
+        x.q = q0 + cur.rr;
+        x.bt = bt0;
+        while (x.q >= Nq) {
+            x.q -= Nq;
+            ++x.bt;
+        }
+        return x;
+    };
+    struct In {
+        float a;
+        float2 v, r;
+        float go[G];
+    };
+    auto fetch = [&](const Item& x, In& in) {
+        const int64_t row_h = (x.r * H + x.h0 + gl.s) * S + gl.k;
+        in.a = x.valid ? ld_stream(logits + row_h) : (FUSED ? -INFINITY : 0.f);
+        in.v = x.valid ? ld_stream2(off + 2 * row_h) : make_float2(0.f, 0.f);
+        in.r = (FUSED && x.valid)
+                   ? __ldg(reinterpret_cast<const float2*>(ref + x.r * R * 2) + gl.m)
+                   : make_float2(0.f, 0.f);
+        const int64_t gitem = ((int64_t)(x.bt / T) * Nq + x.q) * H + x.h0;
+#pragma unroll
+        for (int i = 0; i < G; ++i)
+            in.go[i] = x.h0 + i < H ? __ldg(grad_out + (gitem + i) * kHeadDim + lane) / scale
+                                    : 0.f;
+    };
+
+    ItemCursor cur(warp, HG);
+    int it = warp;
+    Item x0 = resolve(it, cur);
+    In in0, in1;
+    if (x0.ok) fetch(x0, in0);
+    while (x0.ok) {
+        ItemCursor nx = cur;
+        nx.next();
+        const Item x1 = resolve(it + kWarps, nx);
+        if (x1.ok) fetch(x1, in1);
+        const int64_t vofs = (int64_t)x0.bt * vstride;
+        const int64_t item0 = x0.r * H + x0.h0;
+        group_backward<VT, FUSED, NPL, DET>(value + vofs, H, x0.h0, S, in0.a, in0.v, in0.r,
+                                            x0.valid, in0.go, gl, s_tab[warp], grad_value + vofs,
+                                            DET ? grad_value_fix + vofs : nullptr,
+                                            grad_loc + item0 * S * 2, grad_attn + item0 * S,
+                                            lane);
+        x0 = x1;
+        in0 = in1;
+        cur = nx;
+        it += kWarps;
+    }
+}
+
+// npad = L*P rounded up to a power of two, at least 4; 0 when the row is
+// too long for the group kernels (or H = 1, where a warp would hold one head).
+static int group_npl(int S, int H)
+{
+    if (S > 16 || H < 2) return 0;
+    int npl = 2;
+    while ((1 << npl) < S) ++npl;
+    return npl;
+}
+
+template <typename VT, bool FUSED, bool DET>
+static cudaError_t launch_backward_group(const Problem& p, int npl, int BT, int T,
+                                         const float* ref, const float* off, const float* logits,
+                                         const float* grad_out, float* grad_value,
+                                         long long* grad_value_fix, float* grad_loc,
+                                         float* grad_attn, cudaStream_t s)
+{
+    const int64_t rows = (int64_t)BT * p.Nq;
+    const unsigned grid = (unsigned)((rows + kBwdGroupRowsPerTile - 1) / kBwdGroupRowsPerTile);
+    const VT* v = static_cast<const VT*>(p.value);
+    switch (npl) {
+#define BWD_GROUP_CASE(NPLV)                                                                     \
+    case NPLV:                                                                                   \
+        backward_group_kernel<VT, NPLV, FUSED, DET><<<grid, kThreads, 0, s>>>(                   \
+            v, off, logits, ref, grad_out, grad_value, grad_value_fix, grad_loc, grad_attn, BT,  \
+            T, p.Nq, p.Nv, p.H, p.L, p.P, p.R, p.lv);                                            \
+        break;
+        BWD_GROUP_CASE(2)
+        BWD_GROUP_CASE(3)
+        BWD_GROUP_CASE(4)
+#undef BWD_GROUP_CASE
+        default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
 template <typename VT>
 static cudaError_t launch_tsa_backward_t(const Problem& p, int T, const float* ref,
                                          const float* off, const float* logits,
@@ -461,6 +822,10 @@ static cudaError_t launch_tsa_backward_t(const Problem& p, int T, const float* r
     const int BT = p.B * T;
     const int64_t rows = (int64_t)BT * p.Nq;
     if (rows == 0) return cudaSuccess;
+    if (const int npl = group_npl(p.L * p.P, p.H))
+        return launch_backward_group<VT, true, false>(p, npl, BT, T, ref, off, logits, grad_out,
+                                                      grad_value, nullptr, grad_loc, grad_attn,
+                                                      s);
     const unsigned grid = (unsigned)((rows + kBwdRowsPerTile - 1) / kBwdRowsPerTile);
     const VT* v = static_cast<const VT*>(p.value);
     switch ((p.L * p.P + 31) / 32) {
@@ -568,6 +933,10 @@ static cudaError_t launch_msda_backward_t(const Problem& p, const float* loc, co
 {
     const int64_t rows = (int64_t)p.B * p.Nq;
     if (rows == 0) return cudaSuccess;
+    if (const int npl = group_npl(p.L * p.P, p.H))
+        return launch_backward_group<VT, false, DET>(p, npl, p.B, 1, nullptr, loc, attn, grad_out,
+                                                     grad_value, grad_value_fix, grad_loc,
+                                                     grad_attn, s);
     const unsigned grid = (unsigned)((rows + kBwdRowsPerTile - 1) / kBwdRowsPerTile);
     const VT* v = static_cast<const VT*>(p.value);
     const int nc = (p.L * p.P + 31) / 32;

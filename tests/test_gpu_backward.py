@@ -35,6 +35,13 @@ CASES = [
     (2, 2, 300, 8, [(20, 30), (10, 15), (5, 8), (3, 4)], 4),
     (3, 1, 77, 2, [(6, 5), (3, 3), (1, 9)], 12),     # two chunks
     (4, 1, 40, 3, [(7, 9)] * 8, 16),                 # four chunks
+    # rows of <= 16 samples take the head-group kernel: eight heads of four
+    # samples per warp, a partial group (H = 5 in groups of four), padded
+    # sample slots (3 of 4, 12 of 16)
+    (5, 2, 53, 8, [(9, 11)], 4),
+    (6, 1, 41, 5, [(6, 7), (3, 4)], 3),
+    (7, 3, 37, 6, [(5, 9)], 3),
+    (8, 1, 33, 2, [(4, 4), (2, 3), (3, 2)], 4),
 ]
 
 

@@ -132,8 +132,7 @@ def _chain_close(got, want, what):
     assert err.max() <= 1e-4 * (1.0 + np.abs(want).max()), (what, err.max())
 
 
-@pytest.mark.parametrize("case", [CASES[0], CASES[2], CASES[4], CASES[5]],
-                         ids=["case80", "case82", "case84", "case85"])
+@pytest.mark.parametrize("case", CASES, ids=[f"case{c[0]}" for c in CASES])
 @pytest.mark.parametrize("bf16", [False, True])
 def test_tsa_backward(case, bf16):
     seed, B, T, shapes, H, P, R = case
