@@ -163,17 +163,29 @@ struct BwdLanes<float> {
 
 // bf16 value: lanes 16s + 4g + t hold corner g, channels 8t..8t+7, of the
 // samples j0 + 2k + s.  After batch(), lane (s, g, t) holds D_g of sample
-// j0 + 2t + s.
+// j0 + 2t + s.  The grad_value reductions use another channel split so that
+// every 16-byte vector add has its 32-byte sector's other half in the same
+// instruction (one L2 sector operation instead of two): lanes t = 2p + h add
+// channels 16p + 4h .. +3 in the first instruction and 16p + 8 + 4h .. +3 in
+// the second (red_channel).
+__device__ __forceinline__ int red_channel(int t) { return 16 * (t >> 1) + 4 * (t & 1); }
+
 template <>
 struct BwdLanes<__nv_bfloat16> {
-    float go[8];
+    float go[8];  // channels 8t .. 8t+7 (dot products)
+    float gr[8];  // channels red_channel(t) + 0..3 and + 8..11 (reductions)
     __device__ __forceinline__ void load_grad(const float* __restrict__ grow, float scale,
                                               int lane)
     {
-        const float4* g4 = reinterpret_cast<const float4*>(grow) + 2 * (lane & 3);
-        const float4 a = __ldg(g4), b = __ldg(g4 + 1);
+        const int t = lane & 3;
+        const float4* g4 = reinterpret_cast<const float4*>(grow);
+        const float4 a = __ldg(g4 + 2 * t), b = __ldg(g4 + 2 * t + 1);
         go[0] = a.x / scale; go[1] = a.y / scale; go[2] = a.z / scale; go[3] = a.w / scale;
         go[4] = b.x / scale; go[5] = b.y / scale; go[6] = b.z / scale; go[7] = b.w / scale;
+        const int rc = red_channel(t) / 4;
+        const float4 c = __ldg(g4 + rc), d = __ldg(g4 + rc + 2);
+        gr[0] = c.x / scale; gr[1] = c.y / scale; gr[2] = c.z / scale; gr[3] = c.w / scale;
+        gr[4] = d.x / scale; gr[5] = d.y / scale; gr[6] = d.z / scale; gr[7] = d.w / scale;
     }
     __device__ __forceinline__ static int group(int lane) { return (lane >> 2) & 3; }
     __device__ __forceinline__ static int held(int lane) { return 2 * (lane & 3) + (lane >> 4); }
@@ -203,9 +215,9 @@ struct BwdLanes<__nv_bfloat16> {
                 if (!DET) {
                     const float w = tab.alpha[j] * tab.wb[g][j];
                     if (w != 0.f) {
-                        float* dst = gvb + o + 8 * t;
-                        red_add_v4(dst, w * go[0], w * go[1], w * go[2], w * go[3]);
-                        red_add_v4(dst + 4, w * go[4], w * go[5], w * go[6], w * go[7]);
+                        float* dst = gvb + o + red_channel(t);
+                        red_add_v4(dst, w * gr[0], w * gr[1], w * gr[2], w * gr[3]);
+                        red_add_v4(dst + 8, w * gr[4], w * gr[5], w * gr[6], w * gr[7]);
                     }
                 }
             }
@@ -385,10 +397,13 @@ struct GroupBwdLanes<__nv_bfloat16> {
     __device__ __forceinline__ static int group(int lane) { return (lane >> 2) & 3; }
     __device__ __forceinline__ static int held(int lane) { return 2 * (lane & 3) + (lane >> 4); }
     __device__ __forceinline__ static int holder(int u) { return 16 * (u & 1) + (u >> 1); }
+    // g0, g1: channels 8t .. 8t+7 of the sample's head; rs: the head's
+    // channels red_channel(t) + 0..3 and + 8..11 (see BwdLanes), read from
+    // the shared copy only when the add happens
     template <bool DET>
     __device__ __forceinline__ static double corner(const __nv_bfloat16* __restrict__ vb,
                                                     float* __restrict__ gvb, int2 e, float4 g0,
-                                                    float4 g1, int t)
+                                                    float4 g1, const float4* rs, int t)
     {
         if (e.x < 0) return 0.0;
         const uint4 raw = __ldg(reinterpret_cast<const uint4*>(vb + e.x + 8 * t));
@@ -400,9 +415,10 @@ struct GroupBwdLanes<__nv_bfloat16> {
         if (!DET) {
             const float w = __int_as_float(e.y);
             if (w != 0.f) {
-                float* dst = gvb + e.x + 8 * t;
-                red_add_v4(dst, w * g0.x, w * g0.y, w * g0.z, w * g0.w);
-                red_add_v4(dst + 4, w * g1.x, w * g1.y, w * g1.z, w * g1.w);
+                const float4 r0 = rs[0], r1 = rs[2];
+                float* dst = gvb + e.x + red_channel(t);
+                red_add_v4(dst, w * r0.x, w * r0.y, w * r0.z, w * r0.w);
+                red_add_v4(dst + 8, w * r1.x, w * r1.y, w * r1.z, w * r1.w);
             }
         }
         return (double)g0.x * v[0] + (double)g0.y * v[1] + (double)g0.z * v[2] +
@@ -415,8 +431,9 @@ struct GroupBwdLanes<__nv_bfloat16> {
                                                    const GroupBwdTable& tab, int j0, int lane)
     {
         const int s = lane >> 4, g = (lane >> 2) & 3, t = lane & 3;
-        const float4* gs =
-            reinterpret_cast<const float4*>(tab.go + (j0 >> NPL) * kHeadDim + 8 * t);
+        const float* head = tab.go + (j0 >> NPL) * kHeadDim;
+        const float4* gs = reinterpret_cast<const float4*>(head + 8 * t);
+        const float4* rs = reinterpret_cast<const float4*>(head + red_channel(t));
         const float4 ga0 = gs[0], ga1 = gs[1];
         const float4 gb0 = NPL == 2 ? gs[kHeadDim / 4] : ga0;
         const float4 gb1 = NPL == 2 ? gs[kHeadDim / 4 + 1] : ga1;
@@ -425,7 +442,7 @@ struct GroupBwdLanes<__nv_bfloat16> {
         for (int k = 0; k < 4; ++k) {
             const bool second = NPL == 2 && k >= 2;  // samples j0 + 4 .. j0 + 7
             part[k] = corner<DET>(vb, gvb, tab.ow[j0 + 2 * k + s][g], second ? gb0 : ga0,
-                                  second ? gb1 : ga1, t);
+                                  second ? gb1 : ga1, second ? rs + kHeadDim / 4 : rs, t);
         }
         return reduce_scatter4(part, t);
     }
@@ -688,7 +705,7 @@ constexpr int kBwdGroupRowsPerTile = MSDA_GROUP_ROWS_PER_TILE;
 // TSA: rows are (b * T + t, q), each queue receiving grad_out[b] / T.  MSDA
 // (T = 1, !FUSED): rows are (b, q) with the locations and weights given.
 template <typename VT, int NPL, bool FUSED, bool DET>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 3)
 backward_group_kernel(const VT* __restrict__ value, const float* __restrict__ off,
                       const float* __restrict__ logits, const float* __restrict__ ref,
                       const float* __restrict__ grad_out, float* __restrict__ grad_value,
