@@ -129,13 +129,35 @@ struct BwdLanes<float> {
     __device__ __forceinline__ static int group(int lane) { return lane >> 3; }
     // sample (within the batch) whose dot product the lane holds after batch()
     __device__ __forceinline__ static int held(int lane) { return lane & 7; }
-    template <bool DET>
+    template <bool DET, bool LF>
     __device__ __forceinline__ double batch(const float* __restrict__ vb,
                                             float* __restrict__ gvb, long long* __restrict__ gvi,
                                             const BwdTable& tab, int j0, int cnt, int lane) const
     {
         const int g = lane >> 3, t = lane & 7;
         double part[8];
+        if (!DET && LF) {  // every load of the batch in flight before its reductions
+            int o[8];
+            float4 v[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int j = j0 + k;
+                o[k] = j < cnt ? tab.off[g][j] : -1;
+                v[k] = o[k] >= 0 ? __ldg(reinterpret_cast<const float4*>(vb + o[k] + 4 * t))
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const float w = o[k] >= 0 ? tab.alpha[j0 + k] * tab.wb[g][j0 + k] : 0.f;
+                if (w != 0.f)
+                    red_add_v4(gvb + o[k] + 4 * t, w * go.x, w * go.y, w * go.z, w * go.w);
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                part[k] = (double)go.x * v[k].x + (double)go.y * v[k].y +
+                          (double)go.z * v[k].z + (double)go.w * v[k].w;
+            return reduce_scatter8(part, t);
+        }
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
             const int j = j0 + k;
@@ -189,13 +211,47 @@ struct BwdLanes<__nv_bfloat16> {
     }
     __device__ __forceinline__ static int group(int lane) { return (lane >> 2) & 3; }
     __device__ __forceinline__ static int held(int lane) { return 2 * (lane & 3) + (lane >> 4); }
-    template <bool DET>
+    template <bool DET, bool LF>
     __device__ __forceinline__ double batch(const __nv_bfloat16* __restrict__ vb,
                                             float* __restrict__ gvb, long long* __restrict__ gvi,
                                             const BwdTable& tab, int j0, int cnt, int lane) const
     {
         const int s = lane >> 4, g = (lane >> 2) & 3, t = lane & 3;
         double part[4];
+        if (!DET && LF) {  // every load of the batch in flight before its reductions
+            int o[4];
+            uint4 raw[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int j = j0 + 2 * k + s;
+                o[k] = j < cnt ? tab.off[g][j] : -1;
+                raw[k] = o[k] >= 0 ? __ldg(reinterpret_cast<const uint4*>(vb + o[k] + 8 * t))
+                                   : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int j = j0 + 2 * k + s;
+                const float w = o[k] >= 0 ? tab.alpha[j] * tab.wb[g][j] : 0.f;
+                if (w != 0.f) {
+                    float* dst = gvb + o[k] + red_channel(t);
+                    red_add_v4(dst, w * gr[0], w * gr[1], w * gr[2], w * gr[3]);
+                    red_add_v4(dst + 8, w * gr[4], w * gr[5], w * gr[6], w * gr[7]);
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                float v[8];
+                bf16x2_to_f32(raw[k].x, v[0], v[1]);
+                bf16x2_to_f32(raw[k].y, v[2], v[3]);
+                bf16x2_to_f32(raw[k].z, v[4], v[5]);
+                bf16x2_to_f32(raw[k].w, v[6], v[7]);
+                double d = 0.0;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) d += (double)go[i] * v[i];
+                part[k] = d;
+            }
+            return reduce_scatter4(part, t);
+        }
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const int j = j0 + 2 * k + s;
@@ -235,8 +291,10 @@ struct BwdLanes<__nv_bfloat16> {
 // Backward of one (row, head).  grow: grad_out of the row's head (32 floats),
 // divided by `scale` (1 for MSDA, max(1, hits) for SCA).  gvb: grad_value of
 // the batch item (and camera), or (DET) gvi its fixed-point copy.  gloc_row
-// [L, P, 2], gattn_row [L, P].
-template <typename VT, bool FUSED, int NC, bool DET>
+// [L, P, 2], gattn_row [L, P].  LF: issue a batch's eight corner loads before
+// its grad_value reductions (more registers; faster in the persistent SCA
+// kernel, whose grid is sized to the resident CTAs, slower elsewhere).
+template <typename VT, bool FUSED, int NC, bool DET, bool LF = false>
 __device__ __forceinline__ void row_backward(const VT* __restrict__ vb, int H, int h,
                                              const float* __restrict__ lo,
                                              const float* __restrict__ wl,
@@ -294,7 +352,7 @@ __device__ __forceinline__ void row_backward(const VT* __restrict__ vb, int H, i
         float res_w = 0.f, res_x = 0.f, res_y = 0.f;
         const int cnt = min(32, n - c * 32);
         for (int j0 = 0; j0 < cnt; j0 += 8) {
-            const double d = lanes.template batch<DET>(vb, gvb, gvi, tab, j0, cnt, lane);
+            const double d = lanes.template batch<DET, LF>(vb, gvb, gvi, tab, j0, cnt, lane);
             if (DET) {  // lane = channel: one 256-byte slice per (sample, corner)
                 for (int j = j0; j < min(j0 + 8, cnt); ++j) {
                     const int4 o = *reinterpret_cast<const int4*>(det[j].off);
@@ -644,7 +702,7 @@ sca_backward_kernel(const VT* __restrict__ value, const float* __restrict__ off,
             const int64_t vofs = (int64_t)bc * Nv * H * kHeadDim;
             const int64_t rowh = ((int64_t)bc * Nq + i) * H + h;
             const float scale = (float)max(1, __ldg(hits + bq));
-            row_backward<VT, true, NC, DET>(value + vofs, H, h, off + bqh * S * 2,
+            row_backward<VT, true, NC, DET, true>(value + vofs, H, h, off + bqh * S * 2,
                                             logits + bqh * S,
                                             ref_cam + (((int64_t)c * B + b) * Nq + q) * R * 2, S,
                                             ls, s_tab[warp], grad_out + bqh * kHeadDim, scale,
