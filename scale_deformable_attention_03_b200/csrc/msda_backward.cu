@@ -38,12 +38,12 @@ struct __align__(16) DetEntry {
     float wa[4];  // alpha * bilinear weight
 };
 
+// Sample table of one (row, head): corner g of sample j as (element offset,
+// -1 outside; alpha * w_g as float bits), and the sample's fractions (lx, ly),
+// from which w_g and its derivatives are formed again.
 struct BwdTable {
-    int off[4][kMetaStride];
-    float wb[4][kMetaStride];  // bilinear weight without alpha
-    float lx[kMetaStride];
-    float ly[kMetaStride];
-    float alpha[kMetaStride];
+    int2 ow[4][kMetaStride];
+    float2 l[kMetaStride];
 };
 
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d)
@@ -107,6 +107,29 @@ __device__ __forceinline__ double reduce_scatter4(const double (&part)[4], int t
     return (hi ? q[1] : q[0]) + __shfl_xor_sync(0xffffffffu, hi ? q[0] : q[1], 1);
 }
 
+// Sums over the four corner-group lanes, scattered: afterwards the lane of
+// group g holds the total of c[g].  `stride` is the lane distance between
+// neighbouring groups.  Three double shuffles for three sums (c[3] unused).
+__device__ __forceinline__ double reduce_scatter_groups(const double (&c)[4], int g, int stride)
+{
+    const bool hi2 = g & 2;
+    const double a0 =
+        (hi2 ? c[2] : c[0]) + __shfl_xor_sync(0xffffffffu, hi2 ? c[0] : c[2], 2 * stride);
+    const double a1 =
+        (hi2 ? c[3] : c[1]) + __shfl_xor_sync(0xffffffffu, hi2 ? c[1] : c[3], 2 * stride);
+    const bool hi1 = g & 1;
+    return (hi1 ? a1 : a0) + __shfl_xor_sync(0xffffffffu, hi1 ? a0 : a1, stride);
+}
+
+// w_g (as locate() rounds it) and, in double, d w_g / d lx and d w_g / d ly.
+__device__ __forceinline__ void corner_weight(int g, float2 l, float& wg, double& dx, double& dy)
+{
+    const float hx = __fsub_rn(1.f, l.x), hy = __fsub_rn(1.f, l.y);
+    wg = __fmul_rn((g & 1) ? l.x : hx, (g >> 1) ? l.y : hy);
+    dx = dw_dlx(g, l.y);
+    dy = dw_dly(g, l.x);
+}
+
 // Samples are processed eight at a time.  Each lane forms its partial dot
 // products <grad_out, V_g> for the eight samples (over its own channels), and
 // a butterfly reduce-scatter over the lanes that share a corner leaves every
@@ -126,9 +149,12 @@ struct BwdLanes<float> {
         const float4 v = __ldg(reinterpret_cast<const float4*>(grow) + (lane & 7));
         go = make_float4(v.x / scale, v.y / scale, v.z / scale, v.w / scale);
     }
+    static constexpr int kStride = 8;  // lanes between corner groups
     __device__ __forceinline__ static int group(int lane) { return lane >> 3; }
     // sample (within the batch) whose dot product the lane holds after batch()
     __device__ __forceinline__ static int held(int lane) { return lane & 7; }
+    // a group-0 lane holding sample u of the batch
+    __device__ __forceinline__ static int holder(int u) { return u; }
     template <bool DET, bool LF>
     __device__ __forceinline__ double batch(const float* __restrict__ vb,
                                             float* __restrict__ gvb, long long* __restrict__ gvi,
@@ -142,13 +168,13 @@ struct BwdLanes<float> {
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
                 const int j = j0 + k;
-                o[k] = j < cnt ? tab.off[g][j] : -1;
+                o[k] = j < cnt ? tab.ow[g][j].x : -1;
                 v[k] = o[k] >= 0 ? __ldg(reinterpret_cast<const float4*>(vb + o[k] + 4 * t))
                                  : make_float4(0.f, 0.f, 0.f, 0.f);
             }
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
-                const float w = o[k] >= 0 ? tab.alpha[j0 + k] * tab.wb[g][j0 + k] : 0.f;
+                const float w = o[k] >= 0 ? __int_as_float(tab.ow[g][j0 + k].y) : 0.f;
                 if (w != 0.f)
                     red_add_v4(gvb + o[k] + 4 * t, w * go.x, w * go.y, w * go.z, w * go.w);
             }
@@ -161,25 +187,18 @@ struct BwdLanes<float> {
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
             const int j = j0 + k;
-            const int o = j < cnt ? tab.off[g][j] : -1;
+            const int2 e = j < cnt ? tab.ow[g][j] : make_int2(-1, 0);
             part[k] = 0.0;
-            if (o >= 0) {
-                const float4 v = __ldg(reinterpret_cast<const float4*>(vb + o + 4 * t));
+            if (e.x >= 0) {
+                const float4 v = __ldg(reinterpret_cast<const float4*>(vb + e.x + 4 * t));
                 part[k] = (double)go.x * v.x + (double)go.y * v.y + (double)go.z * v.z +
                           (double)go.w * v.w;
-                if (!DET) {
-                    const float w = tab.alpha[j] * tab.wb[g][j];
-                    if (w != 0.f) red_add_v4(gvb + o + 4 * t, w * go.x, w * go.y, w * go.z, w * go.w);
-                }
+                const float w = __int_as_float(e.y);
+                if (!DET && w != 0.f)
+                    red_add_v4(gvb + e.x + 4 * t, w * go.x, w * go.y, w * go.z, w * go.w);
             }
         }
         return reduce_scatter8(part, t);
-    }
-    __device__ __forceinline__ static double reduce_groups(double v)
-    {
-        v += __shfl_xor_sync(0xffffffffu, v, 8);
-        v += __shfl_xor_sync(0xffffffffu, v, 16);
-        return v;
     }
 };
 
@@ -209,8 +228,10 @@ struct BwdLanes<__nv_bfloat16> {
         gr[0] = c.x / scale; gr[1] = c.y / scale; gr[2] = c.z / scale; gr[3] = c.w / scale;
         gr[4] = d.x / scale; gr[5] = d.y / scale; gr[6] = d.z / scale; gr[7] = d.w / scale;
     }
+    static constexpr int kStride = 4;
     __device__ __forceinline__ static int group(int lane) { return (lane >> 2) & 3; }
     __device__ __forceinline__ static int held(int lane) { return 2 * (lane & 3) + (lane >> 4); }
+    __device__ __forceinline__ static int holder(int u) { return 16 * (u & 1) + (u >> 1); }
     template <bool DET, bool LF>
     __device__ __forceinline__ double batch(const __nv_bfloat16* __restrict__ vb,
                                             float* __restrict__ gvb, long long* __restrict__ gvi,
@@ -224,14 +245,14 @@ struct BwdLanes<__nv_bfloat16> {
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const int j = j0 + 2 * k + s;
-                o[k] = j < cnt ? tab.off[g][j] : -1;
+                o[k] = j < cnt ? tab.ow[g][j].x : -1;
                 raw[k] = o[k] >= 0 ? __ldg(reinterpret_cast<const uint4*>(vb + o[k] + 8 * t))
                                    : make_uint4(0u, 0u, 0u, 0u);
             }
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const int j = j0 + 2 * k + s;
-                const float w = o[k] >= 0 ? tab.alpha[j] * tab.wb[g][j] : 0.f;
+                const float w = o[k] >= 0 ? __int_as_float(tab.ow[g][j].y) : 0.f;
                 if (w != 0.f) {
                     float* dst = gvb + o[k] + red_channel(t);
                     red_add_v4(dst, w * gr[0], w * gr[1], w * gr[2], w * gr[3]);
@@ -255,10 +276,10 @@ struct BwdLanes<__nv_bfloat16> {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const int j = j0 + 2 * k + s;
-            const int o = j < cnt ? tab.off[g][j] : -1;
+            const int2 e = j < cnt ? tab.ow[g][j] : make_int2(-1, 0);
             part[k] = 0.0;
-            if (o >= 0) {
-                const uint4 raw = __ldg(reinterpret_cast<const uint4*>(vb + o + 8 * t));
+            if (e.x >= 0) {
+                const uint4 raw = __ldg(reinterpret_cast<const uint4*>(vb + e.x + 8 * t));
                 float v[8];
                 bf16x2_to_f32(raw.x, v[0], v[1]);
                 bf16x2_to_f32(raw.y, v[2], v[3]);
@@ -268,23 +289,15 @@ struct BwdLanes<__nv_bfloat16> {
 #pragma unroll
                 for (int i = 0; i < 8; ++i) d += (double)go[i] * v[i];
                 part[k] = d;
-                if (!DET) {
-                    const float w = tab.alpha[j] * tab.wb[g][j];
-                    if (w != 0.f) {
-                        float* dst = gvb + o + red_channel(t);
-                        red_add_v4(dst, w * gr[0], w * gr[1], w * gr[2], w * gr[3]);
-                        red_add_v4(dst + 8, w * gr[4], w * gr[5], w * gr[6], w * gr[7]);
-                    }
+                const float w = __int_as_float(e.y);
+                if (!DET && w != 0.f) {
+                    float* dst = gvb + e.x + red_channel(t);
+                    red_add_v4(dst, w * gr[0], w * gr[1], w * gr[2], w * gr[3]);
+                    red_add_v4(dst + 8, w * gr[4], w * gr[5], w * gr[6], w * gr[7]);
                 }
             }
         }
         return reduce_scatter4(part, t);
-    }
-    __device__ __forceinline__ static double reduce_groups(double v)
-    {
-        v += __shfl_xor_sync(0xffffffffu, v, 4);
-        v += __shfl_xor_sync(0xffffffffu, v, 8);
-        return v;
     }
 };
 
@@ -310,10 +323,11 @@ __device__ __forceinline__ void row_backward(const VT* __restrict__ vb, int H, i
     const float go_c = DET ? __ldg(grow + lane) / scale : 0.f;
     float a[NC];
     row_weights<FUSED, NC>(wl, n, lane, a);
-    BwdLanes<VT> lanes;
+    using Lanes = BwdLanes<VT>;
+    Lanes lanes;
     lanes.load_grad(grow, scale, lane);
-    const int g = BwdLanes<VT>::group(lane);
-    const int held = BwdLanes<VT>::held(lane);
+    const int g = Lanes::group(lane);
+    const int held = Lanes::held(lane);
 #pragma unroll
     for (int c = 0; c < NC; ++c) {
         const int j = c * 32 + lane;
@@ -334,13 +348,9 @@ __device__ __forceinline__ void row_backward(const VT* __restrict__ vb, int H, i
             cr.lx = cr.ly = 0.f;
         }
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            tab.off[q][lane] = cr.off[q];
-            tab.wb[q][lane] = cr.w[q];
-        }
-        tab.lx[lane] = cr.lx;
-        tab.ly[lane] = cr.ly;
-        tab.alpha[lane] = a[c];
+        for (int q = 0; q < 4; ++q)
+            tab.ow[q][lane] = make_int2(cr.off[q], __float_as_int(a[c] * cr.w[q]));
+        tab.l[lane] = make_float2(cr.lx, cr.ly);
         if (DET) {
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -364,19 +374,22 @@ __device__ __forceinline__ void row_backward(const VT* __restrict__ vb, int H, i
                 }
             }
             const int js = j0 + held;  // the sample whose D_g this lane holds
-            const bool valid = js < cnt;
-            double cw = valid ? (double)tab.wb[g][js] * d : 0.0;
-            double cx = valid ? dw_dlx(g, tab.ly[js]) * d : 0.0;
-            double cy = valid ? dw_dly(g, tab.lx[js]) * d : 0.0;
-            cw = BwdLanes<VT>::reduce_groups(cw);
-            cx = BwdLanes<VT>::reduce_groups(cx);
-            cy = BwdLanes<VT>::reduce_groups(cy);
-            // the owner of sample j0 + u is lane j0 + u; fetch from a lane holding it
-            const int u = lane & 7;
-            const int src = std::is_same<VT, float>::value ? u : 16 * (u & 1) + (u >> 1);
-            const float tw = __shfl_sync(0xffffffffu, (float)cw, src);
-            const float tx = __shfl_sync(0xffffffffu, (float)cx, src);
-            const float ty = __shfl_sync(0xffffffffu, (float)cy, src);
+            double c4[4] = {0.0, 0.0, 0.0, 0.0};
+            if (js < cnt) {
+                float wg;
+                double dx, dy;
+                corner_weight(g, tab.l[js], wg, dx, dy);
+                c4[0] = (double)wg * d;
+                c4[1] = dx * d;
+                c4[2] = dy * d;
+            }
+            // lanes of group 0, 1, 2 now hold the weight, x and y sums
+            const float r = (float)reduce_scatter_groups(c4, g, Lanes::kStride);
+            // the owner of sample j0 + u is lane j0 + u; fetch from the lanes holding it
+            const int src = Lanes::holder(lane & 7);
+            const float tw = __shfl_sync(0xffffffffu, r, src);
+            const float tx = __shfl_sync(0xffffffffu, r, src + Lanes::kStride);
+            const float ty = __shfl_sync(0xffffffffu, r, src + 2 * Lanes::kStride);
             if ((lane & ~7) == j0) {
                 res_w = tw;
                 res_x = tx;
@@ -585,20 +598,16 @@ __device__ __forceinline__ void group_backward(const VT* __restrict__ vb, int H,
         }
         // d = D_g of sample j0 + held; its bilinear weight and the weight's
         // derivatives follow from (lx, ly) as in locate()
-        const float2 l = tab.l[j0 + held];
-        const float hx = __fsub_rn(1.f, l.x), hy = __fsub_rn(1.f, l.y);
-        const float wg = __fmul_rn((g & 1) ? l.x : hx, (g >> 1) ? l.y : hy);
-        double cw = (double)wg * d;
-        double cx = dw_dlx(g, l.y) * d;
-        double cy = dw_dly(g, l.x) * d;
-        cw = BwdLanes<VT>::reduce_groups(cw);
-        cx = BwdLanes<VT>::reduce_groups(cx);
-        cy = BwdLanes<VT>::reduce_groups(cy);
+        float wg;
+        double dx, dy;
+        corner_weight(g, tab.l[j0 + held], wg, dx, dy);
+        const double c4[4] = {(double)wg * d, dx * d, dy * d, 0.0};
+        const float r = (float)reduce_scatter_groups(c4, g, BwdLanes<VT>::kStride);
         // sample j0 + u lands on lane j0 + u
         const int src = Lanes::holder(lane & 7);
-        const float tw = __shfl_sync(0xffffffffu, (float)cw, src);
-        const float tx = __shfl_sync(0xffffffffu, (float)cx, src);
-        const float ty = __shfl_sync(0xffffffffu, (float)cy, src);
+        const float tw = __shfl_sync(0xffffffffu, r, src);
+        const float tx = __shfl_sync(0xffffffffu, r, src + BwdLanes<VT>::kStride);
+        const float ty = __shfl_sync(0xffffffffu, r, src + 2 * BwdLanes<VT>::kStride);
         if ((lane & ~7) == j0) {
             res_w = tw;
             res_x = tx;
@@ -615,8 +624,10 @@ __device__ __forceinline__ void group_backward(const VT* __restrict__ vb, int H,
     __syncwarp();
 }
 
+// Register caps: four CTAs per SM for fp32 value, three for bf16 rows of up
+// to 32 samples, two for longer bf16 rows.
 template <typename VT, int NC, bool DET>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, sizeof(VT) == 4 ? 4 : (NC == 1 ? 3 : 2))
 msda_backward_kernel(const VT* __restrict__ value, const float* __restrict__ loc,
                      const float* __restrict__ attn, const float* __restrict__ grad_out,
                      float* __restrict__ grad_value, long long* __restrict__ grad_value_fix,
