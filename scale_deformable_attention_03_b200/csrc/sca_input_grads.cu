@@ -158,6 +158,95 @@ sca_offset_logit_grads_kernel(const float* __restrict__ logits, const int32_t* _
     }
 }
 
+// Rows of L*P <= 16 samples, in the forward's group layout: lane (s, k)
+// takes sample k of head h0 + s (npad = L*P rounded up to a power of two,
+// G = 32 / npad heads per pass), so the softmax and <alpha, G> are segmented
+// reductions over npad lanes instead of whole-warp ones for a few samples.
+// REF (all heads in one pass, R dividing npad): lane mod R is the sample's
+// anchor, and a butterfly over the lanes of one anchor gives each camera's
+// reference-point sums, as in the per-head kernel.
+__device__ __forceinline__ double segment_sum_f64(double v, int npad)
+{
+    for (int o = npad >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+template <int NPL, bool REF>
+__global__ void __launch_bounds__(kIgWarps * 32)
+sca_offset_logit_grads_group_kernel(const float* __restrict__ logits,
+                                    const int32_t* __restrict__ pos,
+                                    const float* __restrict__ grad_loc_rb,
+                                    const float* __restrict__ grad_attn_rb, int B, int Ncam,
+                                    int Nq, int H, int L, int P, int R, Levels levels,
+                                    float* __restrict__ grad_off, float* __restrict__ grad_logits,
+                                    float* __restrict__ grad_ref_cam)
+{
+    constexpr int npad = 1 << NPL;
+    constexpr int G = 32 >> NPL;
+    __shared__ SmemLevels s_lv;
+    stage_levels(s_lv, levels);
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    const int64_t bq = (int64_t)blockIdx.x * kIgWarps + (threadIdx.x >> 5);
+    if (bq >= (int64_t)B * Nq) return;  // warp-uniform
+    const int b = (int)(bq / Nq), q = (int)(bq - (int64_t)b * Nq);
+    const int n = L * P, S = H * n;
+    const int p = lane < Ncam ? (pos ? __ldg(pos + ((int64_t)b * Ncam + lane) * Nq + q) : q) : -1;
+    const unsigned seen = __ballot_sync(0xffffffffu, p >= 0);
+    if (REF) {
+        for (int i = lane; i < Ncam * R * 2; i += 32) {
+            const int c = i / (2 * R);
+            if (!((seen >> c) & 1u))
+                grad_ref_cam[(((int64_t)c * B + b) * Nq + q) * R * 2 + (i - c * 2 * R)] = 0.f;
+        }
+    }
+    const int s = lane >> NPL, k = lane & (npad - 1);
+    const bool kin = k < n;
+    const int l = kin ? k / P : 0;
+    const float wl = (float)s_lv.w[l], hl = (float)s_lv.h[l];
+    for (int h0 = 0; h0 < H; h0 += G) {
+        const bool in = kin && h0 + s < H;
+        const int64_t e = (int64_t)(h0 + s) * n + k;  // element within the row
+        float Gs = 0.f, gx = 0.f, gy = 0.f;
+        unsigned cams = seen;
+        while (cams) {
+            const int cam = __ffs(cams) - 1;  // ascending camera order
+            cams &= cams - 1;
+            const int row = __shfl_sync(0xffffffffu, p, cam);
+            const int64_t r = (((int64_t)b * Ncam + cam) * Nq + row) * S;
+            float2 v = make_float2(0.f, 0.f);
+            if (in) {
+                Gs += __ldcs(grad_attn_rb + r + e);
+                v = __ldcs(reinterpret_cast<const float2*>(grad_loc_rb) + r + e);
+                gx += v.x;
+                gy += v.y;
+            }
+            if (REF) {
+                double rx = v.x, ry = v.y;
+                for (int o = 16; o >= R; o >>= 1) {
+                    rx += __shfl_xor_sync(0xffffffffu, rx, o);
+                    ry += __shfl_xor_sync(0xffffffffu, ry, o);
+                }
+                if (lane < R) {
+                    float* out = grad_ref_cam + (((int64_t)cam * B + b) * Nq + q) * R * 2;
+                    out[2 * lane] = (float)rx;
+                    out[2 * lane + 1] = (float)ry;
+                }
+            }
+        }
+        const float a = in ? __ldg(logits + bq * S + e) : -INFINITY;
+        const float m = segment_max(a, npad);
+        const float ex = in ? expf(a - m) : 0.f;
+        const float z = segment_sum(ex, npad);
+        const float alpha = in ? ex / z : 0.f;
+        const double dot = segment_sum_f64((double)alpha * (double)Gs, npad);
+        if (in) {
+            grad_logits[bq * S + e] = (float)((double)alpha * ((double)Gs - dot));
+            reinterpret_cast<float2*>(grad_off)[bq * S + e] = make_float2(gx / wl, gy / hl);
+        }
+    }
+}
+
 // One warp per (camera, batch, query): the row's H*L*P location gradients
 // summed per anchor m = k mod R (zero when the camera does not see the query).
 __global__ void __launch_bounds__(kIgWarps * 32)
@@ -234,8 +323,32 @@ cudaError_t launch_sca_input_grads(const float* logits, const int32_t* pos,
     const int64_t rows = (int64_t)B * Nq;
     if (rows == 0) return cudaSuccess;
     const unsigned grid = (unsigned)((rows + kIgWarps - 1) / kIgWarps);
-    const int nc = (L * P + 31) / 32;
-    const bool fused = H <= kIgHeads && 32 % R == 0;
+    const int n = L * P;
+    const int nc = (n + 31) / 32;
+    bool fused = H <= kIgHeads && 32 % R == 0;
+    if (n <= 16) {
+        int npl = 2;
+        while ((1 << npl) < n) ++npl;
+        fused = H <= (32 >> npl) && (1 << npl) % R == 0;
+#define IG_GROUP_CASE(NPLV)                                                                      \
+    case NPLV:                                                                                   \
+        if (fused)                                                                               \
+            sca_offset_logit_grads_group_kernel<NPLV, true><<<grid, kIgWarps * 32, 0, s>>>(      \
+                logits, pos, grad_loc_rb, grad_attn_rb, B, Ncam, Nq, H, L, P, R, lv, grad_off,   \
+                grad_logits, grad_ref_cam);                                                      \
+        else                                                                                     \
+            sca_offset_logit_grads_group_kernel<NPLV, false><<<grid, kIgWarps * 32, 0, s>>>(     \
+                logits, pos, grad_loc_rb, grad_attn_rb, B, Ncam, Nq, H, L, P, R, lv, grad_off,   \
+                grad_logits, grad_ref_cam);                                                      \
+        break;
+        switch (npl) {
+            IG_GROUP_CASE(2)
+            IG_GROUP_CASE(3)
+            IG_GROUP_CASE(4)
+            default: return cudaErrorInvalidValue;
+        }
+#undef IG_GROUP_CASE
+    } else {
 #define IG_CASE(NCV)                                                                             \
     case NCV:                                                                                    \
         if (fused)                                                                               \
@@ -247,14 +360,15 @@ cudaError_t launch_sca_input_grads(const float* logits, const int32_t* pos,
                 logits, pos, grad_loc_rb, grad_attn_rb, B, Ncam, Nq, H, L, P, R, lv, grad_off,   \
                 grad_logits, grad_ref_cam);                                                      \
         break;
-    switch (nc) {
-        IG_CASE(1)
-        IG_CASE(2)
-        IG_CASE(3)
-        IG_CASE(4)
-        default: return cudaErrorInvalidValue;
-    }
+        switch (nc) {
+            IG_CASE(1)
+            IG_CASE(2)
+            IG_CASE(3)
+            IG_CASE(4)
+            default: return cudaErrorInvalidValue;
+        }
 #undef IG_CASE
+    }
     if (fused) return cudaGetLastError();
     const int64_t crows = (int64_t)Ncam * B * Nq;
     sca_reference_grads_kernel<<<(unsigned)((crows + kIgWarps - 1) / kIgWarps), kIgWarps * 32, 0,

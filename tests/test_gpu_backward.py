@@ -138,6 +138,12 @@ def _input_grads_both(w, pos, rl, rw):
     (42, 1, 6, (30, 40), [(16, 20), (8, 10), (4, 5), (2, 3)], 8, 8, 4),
     (43, 2, 2, (5, 13), [(6, 7)] * 3, 1, 12, 3),       # R = 3: separate reference kernel
     (44, 1, 4, (9, 11), [(8, 9), (4, 5)], 12, 4, 2),   # 12 heads: two head chunks
+    # rows of <= 16 samples (the head-group kernel): eight heads of four samples
+    # with the reference points fused, padded slots (12 of 16) in three passes,
+    # and R = 3 not dividing the four-lane segment (separate reference kernel)
+    (45, 2, 3, (6, 8), [(10, 12)], 8, 4, 4),
+    (46, 1, 5, (7, 7), [(6, 9), (3, 5), (2, 2)], 5, 4, 1),
+    (47, 2, 4, (5, 9), [(7, 7)], 3, 3, 3),
 ])
 @pytest.mark.parametrize("rho", ["uniform", "coherent"])
 def test_sca_backward_inputs(seed, B, Ncam, bev, shapes, H, P, R, rho):
