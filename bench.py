@@ -701,7 +701,8 @@ def measure_next_rows(args, w, tensors, flush, stream, hbm_peak):
     S4 = w4.H * w4.L * w4.P
     r = hbm(tsa_algorithmic_bytes(w4, 2, 4) + w4.Nq * w4.H * 32 * 4 + w4.value.size * 4
             + 2 * w4.Nq * (S4 * 3 + w4.R * 2) * 4, ms)
-    r.update(kernel="backward_group_kernel<float, 2, true, false> + sca_offset_logit_grads_kernel",
+    r.update(kernel="zero_kernel + backward_group_kernel<float, 2, true, false> + "
+                    "sca_offset_logit_grads_group_kernel<2, true>",
              workload="bevformer-tsa 2 queues x 200x200, H=8, P=4, fp32",
              gsamples_per_s=2 * w4.Nq * S4 / (ms * 1e-3) / 1e9)
     if with_cpu:
@@ -776,7 +777,7 @@ def measure_next_rows(args, w, tensors, flush, stream, hbm_peak):
     ms = timed(lambda: msda.sca_backward_inputs(shapes, starts, logits, pos, gl, gw, w.Ncam,
                                                 w.R, out=bufs))
     r = hbm(input_grads_algorithmic_bytes(w, n_rows), ms)
-    r.update(kernel="sca_offset_logit_grads_kernel + sca_reference_grads_kernel")
+    r.update(kernel="sca_offset_logit_grads_kernel<1, true> (reference points fused)")
     rows["sca_backward_inputs"] = r
     del gl, gw, bufs, gout
 
