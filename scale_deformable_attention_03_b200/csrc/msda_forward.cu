@@ -15,7 +15,7 @@ constexpr int kRowsPerTile = MSDA_ROWS_PER_TILE;
 constexpr int kGroupRowsPerTile = MSDA_GROUP_ROWS_PER_TILE;
 
 template <typename VT, bool FUSED, int NC, int HP>
-__global__ void MSDA_GATHER_BOUNDS
+__global__ void MSDA_GATHER_BOUNDS(VT, NC)
 msda_forward_kernel(const VT* __restrict__ value, const float* __restrict__ lo,
                     const float* __restrict__ wl, const float* __restrict__ ref,
                     float* __restrict__ out, int B, int Nq, int Nv, int H, int L, int P, int R,

@@ -146,7 +146,7 @@ cudaError_t launch_sca_compact(const uint8_t* mask, int B, int Ncam, int Nq, int
 // Offsets and logits come from the BEV query and are shared by its cameras;
 // the reference points are the camera's own.
 template <typename VT, int NC, int HP>
-__global__ void MSDA_GATHER_BOUNDS
+__global__ void MSDA_GATHER_BOUNDS(VT, NC)
 sca_gather_kernel(const VT* __restrict__ value, const float* __restrict__ off,
                   const float* __restrict__ logits, const float* __restrict__ ref_cam,
                   const int32_t* __restrict__ idx, const int32_t* __restrict__ count,

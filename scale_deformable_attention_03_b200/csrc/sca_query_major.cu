@@ -50,7 +50,7 @@ __device__ __forceinline__ void divide_acc(float (&acc)[NA], unsigned seen)
 }
 
 template <typename VT, int NC, int HP>
-__global__ void MSDA_GATHER_BOUNDS
+__global__ void MSDA_GATHER_BOUNDS(VT, NC)
 sca_query_major_kernel(const VT* __restrict__ value, const float* __restrict__ off,
                        const float* __restrict__ logits, const float* __restrict__ ref_cam,
                        const uint8_t* __restrict__ mask, float* __restrict__ out, int B,

@@ -167,7 +167,7 @@ tsa_forward_group_kernel(const VT* __restrict__ value, const float* __restrict__
 // Rows with more samples: a warp item is (b, q, h); the T queues' gathers
 // accumulate into the same partial sums.
 template <typename VT, int NC, int T>
-__global__ void MSDA_GATHER_BOUNDS
+__global__ void MSDA_GATHER_BOUNDS(VT, NC)
 tsa_forward_kernel(const VT* __restrict__ value, const float* __restrict__ off,
                    const float* __restrict__ logits, const float* __restrict__ ref,
                    float* __restrict__ out, int B, int Nq, int Nv, int H, int L, int P, int R,
