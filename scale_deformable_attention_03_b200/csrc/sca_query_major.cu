@@ -19,6 +19,13 @@ namespace msda {
 
 constexpr int kQmRowsPerTile = MSDA_ROWS_PER_TILE;
 
+// Register budget: an explicit four-CTA bound for fp32 rows of up to 32
+// samples (2 % faster here than the compiler's own choice), otherwise as the
+// other forward gathers.
+#define MSDA_QM_BOUNDS(VT, NC)                                                           \
+    __launch_bounds__(kThreads, (NC) == 1 ? (sizeof(VT) == 4 ? 4 : MSDA_MIN_CTAS_BF16)   \
+                                          : ((NC) == 2 ? 2 : 1))
+
 // Camera lane: does camera `lane` (< Ncam) see query (b, q)?
 __device__ __forceinline__ unsigned seeing_cameras(const uint8_t* __restrict__ mask, int B,
                                                    int Ncam, int Nq, int R, int b, int q, int lane)
@@ -50,7 +57,7 @@ __device__ __forceinline__ void divide_acc(float (&acc)[NA], unsigned seen)
 }
 
 template <typename VT, int NC, int HP>
-__global__ void MSDA_GATHER_BOUNDS(VT, NC)
+__global__ void MSDA_QM_BOUNDS(VT, NC)
 sca_query_major_kernel(const VT* __restrict__ value, const float* __restrict__ off,
                        const float* __restrict__ logits, const float* __restrict__ ref_cam,
                        const uint8_t* __restrict__ mask, float* __restrict__ out, int B,
