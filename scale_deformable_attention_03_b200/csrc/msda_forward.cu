@@ -91,8 +91,14 @@ msda_forward_kernel(const VT* __restrict__ value, const float* __restrict__ lo,
 // group_compute).  Items are (row, head group), head groups fastest; a CTA
 // owns kGroupRowsPerTile consecutive rows (more than K1: a row has fewer
 // samples, and neighbouring queries share more of their reads).
+// Register budget: rows of up to four samples (eight heads per warp) run
+// fastest at four CTAs per SM (TSA queues as a batch of two: 140 -> 119 us),
+// longer rows at the group kernels' three.
+#ifndef MSDA_GROUP4_MIN_CTAS
+#define MSDA_GROUP4_MIN_CTAS 4
+#endif
 template <typename VT, bool FUSED, int NPL>
-__global__ void MSDA_GROUP_BOUNDS
+__global__ void __launch_bounds__(kThreads, NPL == 2 ? MSDA_GROUP4_MIN_CTAS : MSDA_GROUP_MIN_CTAS)
 msda_forward_group_kernel(const VT* __restrict__ value, const float* __restrict__ lo,
                           const float* __restrict__ wl, const float* __restrict__ ref,
                           float* __restrict__ out, int B, int Nq, int Nv, int H, int L, int P,
