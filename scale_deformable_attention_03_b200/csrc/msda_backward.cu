@@ -773,8 +773,14 @@ constexpr int kBwdGroupRowsPerTile = MSDA_GROUP_ROWS_PER_TILE;
 // Rows with L*P <= 16: a warp item is (row, head group), see group_backward.
 // TSA: rows are (b * T + t, q), each queue receiving grad_out[b] / T.  MSDA
 // (T = 1, !FUSED): rows are (b, q) with the locations and weights given.
+// Register budget: rows of up to four samples (eight heads per warp) run
+// fastest at four CTAs per SM despite small spills (TSA backward 0.48 ->
+// 0.43 ms), longer rows at three.
+#ifndef MSDA_BWD_GROUP4_MIN_CTAS
+#define MSDA_BWD_GROUP4_MIN_CTAS 4
+#endif
 template <typename VT, int NPL, bool FUSED, bool DET>
-__global__ void __launch_bounds__(kThreads, 3)
+__global__ void __launch_bounds__(kThreads, NPL == 2 ? MSDA_BWD_GROUP4_MIN_CTAS : 3)
 backward_group_kernel(const VT* __restrict__ value, const float* __restrict__ off,
                       const float* __restrict__ logits, const float* __restrict__ ref,
                       const float* __restrict__ grad_out, float* __restrict__ grad_value,
