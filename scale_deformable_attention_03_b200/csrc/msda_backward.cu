@@ -162,7 +162,7 @@ struct BwdLanes<float> {
     {
         const int g = lane >> 3, t = lane & 7;
         double part[8];
-        if (!DET && LF) {  // every load of the batch in flight before its reductions
+        if constexpr (!DET && LF) {  // every load of the batch in flight before its reductions
             int o[8];
             float4 v[8];
 #pragma unroll
@@ -183,22 +183,23 @@ struct BwdLanes<float> {
                 part[k] = (double)go.x * v[k].x + (double)go.y * v[k].y +
                           (double)go.z * v[k].z + (double)go.w * v[k].w;
             return reduce_scatter8(part, t);
-        }
+        } else {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const int j = j0 + k;
-            const int2 e = j < cnt ? tab.ow[g][j] : make_int2(-1, 0);
-            part[k] = 0.0;
-            if (e.x >= 0) {
-                const float4 v = __ldg(reinterpret_cast<const float4*>(vb + e.x + 4 * t));
-                part[k] = (double)go.x * v.x + (double)go.y * v.y + (double)go.z * v.z +
-                          (double)go.w * v.w;
-                const float w = __int_as_float(e.y);
-                if (!DET && w != 0.f)
-                    red_add_v4(gvb + e.x + 4 * t, w * go.x, w * go.y, w * go.z, w * go.w);
+            for (int k = 0; k < 8; ++k) {
+                const int j = j0 + k;
+                const int2 e = j < cnt ? tab.ow[g][j] : make_int2(-1, 0);
+                part[k] = 0.0;
+                if (e.x >= 0) {
+                    const float4 v = __ldg(reinterpret_cast<const float4*>(vb + e.x + 4 * t));
+                    part[k] = (double)go.x * v.x + (double)go.y * v.y + (double)go.z * v.z +
+                              (double)go.w * v.w;
+                    const float w = __int_as_float(e.y);
+                    if (!DET && w != 0.f)
+                        red_add_v4(gvb + e.x + 4 * t, w * go.x, w * go.y, w * go.z, w * go.w);
+                }
             }
+            return reduce_scatter8(part, t);
         }
-        return reduce_scatter8(part, t);
     }
 };
 
@@ -239,7 +240,7 @@ struct BwdLanes<__nv_bfloat16> {
     {
         const int s = lane >> 4, g = (lane >> 2) & 3, t = lane & 3;
         double part[4];
-        if (!DET && LF) {  // every load of the batch in flight before its reductions
+        if constexpr (!DET && LF) {  // every load of the batch in flight before its reductions
             int o[4];
             uint4 raw[4];
 #pragma unroll
@@ -272,32 +273,33 @@ struct BwdLanes<__nv_bfloat16> {
                 part[k] = d;
             }
             return reduce_scatter4(part, t);
-        }
+        } else {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int j = j0 + 2 * k + s;
-            const int2 e = j < cnt ? tab.ow[g][j] : make_int2(-1, 0);
-            part[k] = 0.0;
-            if (e.x >= 0) {
-                const uint4 raw = __ldg(reinterpret_cast<const uint4*>(vb + e.x + 8 * t));
-                float v[8];
-                bf16x2_to_f32(raw.x, v[0], v[1]);
-                bf16x2_to_f32(raw.y, v[2], v[3]);
-                bf16x2_to_f32(raw.z, v[4], v[5]);
-                bf16x2_to_f32(raw.w, v[6], v[7]);
-                double d = 0.0;
+            for (int k = 0; k < 4; ++k) {
+                const int j = j0 + 2 * k + s;
+                const int2 e = j < cnt ? tab.ow[g][j] : make_int2(-1, 0);
+                part[k] = 0.0;
+                if (e.x >= 0) {
+                    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(vb + e.x + 8 * t));
+                    float v[8];
+                    bf16x2_to_f32(raw.x, v[0], v[1]);
+                    bf16x2_to_f32(raw.y, v[2], v[3]);
+                    bf16x2_to_f32(raw.z, v[4], v[5]);
+                    bf16x2_to_f32(raw.w, v[6], v[7]);
+                    double d = 0.0;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) d += (double)go[i] * v[i];
-                part[k] = d;
-                const float w = __int_as_float(e.y);
-                if (!DET && w != 0.f) {
-                    float* dst = gvb + e.x + red_channel(t);
-                    red_add_v4(dst, w * gr[0], w * gr[1], w * gr[2], w * gr[3]);
-                    red_add_v4(dst + 8, w * gr[4], w * gr[5], w * gr[6], w * gr[7]);
+                    for (int i = 0; i < 8; ++i) d += (double)go[i] * v[i];
+                    part[k] = d;
+                    const float w = __int_as_float(e.y);
+                    if (!DET && w != 0.f) {
+                        float* dst = gvb + e.x + red_channel(t);
+                        red_add_v4(dst, w * gr[0], w * gr[1], w * gr[2], w * gr[3]);
+                        red_add_v4(dst + 8, w * gr[4], w * gr[5], w * gr[6], w * gr[7]);
+                    }
                 }
             }
+            return reduce_scatter4(part, t);
         }
-        return reduce_scatter4(part, t);
     }
 };
 
@@ -779,8 +781,12 @@ constexpr int kBwdGroupRowsPerTile = MSDA_GROUP_ROWS_PER_TILE;
 #ifndef MSDA_BWD_GROUP4_MIN_CTAS
 #define MSDA_BWD_GROUP4_MIN_CTAS 4
 #endif
+#ifndef MSDA_BWD_GROUP_MIN_CTAS
+#define MSDA_BWD_GROUP_MIN_CTAS 3
+#endif
 template <typename VT, int NPL, bool FUSED, bool DET>
-__global__ void __launch_bounds__(kThreads, NPL == 2 ? MSDA_BWD_GROUP4_MIN_CTAS : 3)
+__global__ void __launch_bounds__(kThreads,
+                                  NPL == 2 ? MSDA_BWD_GROUP4_MIN_CTAS : MSDA_BWD_GROUP_MIN_CTAS)
 backward_group_kernel(const VT* __restrict__ value, const float* __restrict__ off,
                       const float* __restrict__ logits, const float* __restrict__ ref,
                       const float* __restrict__ grad_out, float* __restrict__ grad_value,
