@@ -8,9 +8,13 @@
 //   d out / d V_g = alpha w_g   (neighbours inside the map only).
 // One warp per (row, head) with the forward's lane layout.  For every sample
 // each lane forms dot_g = <grad_out, V_g> over its channels and adds
-// alpha w_g grad_out to grad_value with one 16-byte vector reduction
-// (red.global.add.v4.f32); the per-sample scalars are reduced with shuffles
-// and land on the lane that owns the sample, which writes them coalesced.
+// alpha w_g grad_out to grad_value with 16-byte vector reductions
+// (red.global.add.v4.f32, paired across lanes so that every instruction
+// covers whole 32-byte L2 sectors); the per-sample scalars are reduced with
+// shuffles and land on the lane that owns the sample, which writes them
+// coalesced.  Rows of at most 16 samples take the head-group form
+// (backward_group_kernel): one warp builds a 32-sample table for several
+// heads of a row, as the forward's group kernels do.
 // Deterministic variant (DET): instead of fp32 reductions, each contribution
 // is scaled by 2^32 (exact), rounded once to a 64-bit integer and added with
 // red.global.add.u64 into a fixed-point copy of grad_value; integer addition
