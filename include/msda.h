@@ -298,9 +298,11 @@ msda_status_t sca_compact(const uint8_t* bev_mask, msda_dims_t d, void* workspac
  *   - Limit: B * Ncam * ceil(Nq / 1024) <= MSDA_NO_ALLOC_COUNT_SLOTS, else
  *     MSDA_ERR_UNSUPPORTED with a message (e.g. B = 1, Ncam = 6 allows
  *     Nq up to about 11 million).
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current) and remembers it; make
- *     that first call before any stream capture.
+ *   - The first call in a CUDA context looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and remembers it for
+ *     that context, keyed by the context's unique id: after cudaDeviceReset,
+ *     or in another context, the next call looks it up again.  Make the first
+ *     call in each context before any stream capture.
  *   - Every call shares the one array per device and leaves its counts
  *     there; calls whose work overlaps on the GPU (different streams, or
  *     different host threads, without ordering) race on it.  Calls on one
@@ -478,6 +480,34 @@ msda_status_t sca_backward_inputs(const int64_t* spatial_shapes, const int64_t* 
                                   const float* grad_attention_weights_rb, msda_dims_t d,
                                   float* grad_sampling_offsets, float* grad_attention_logits,
                                   float* grad_reference_points_cam, msda_stream_t stream);
+
+/* The whole SCA backward down to the SCA inputs, in one call ([BQ] 4.2
+ * softmax, 5 location, 6 bilinear read, 8 weighted sum, 10 camera average;
+ * the pages give no backward, this is the analytic derivative):
+ * sca_compact, the rebatched backward and sca_backward_inputs' chain, with
+ * the location gradients kept to double accuracy between the two stages
+ * (the softmax weight and each location gradient are formed in double and
+ * passed on as fp32 value plus fp32 rounding residual, summed in double), so
+ * that the chained sums over up to H*L*P terms stay within the fp32 bound of
+ * the exact derivative.
+ *   inputs as sca_backward; grad_out [B, Nq, H*32] fp32
+ *   grad_value                [B, Ncam, Nv, H, 32]  fp32, fully written
+ *   grad_sampling_offsets     [B, Nq, H, L, P, 2]   fp32
+ *   grad_attention_logits     [B, Nq, H, L, P]      fp32
+ *   grad_reference_points_cam [Ncam, B, Nq, R, 2]   fp32 (zero where the
+ *                                                   camera does not see q)
+ *   workspace: sca_backward_full_workspace_size(d) bytes, 256-byte aligned
+ *   (compaction lists and the rebatched gradients with residuals).
+ * grad_value is accumulated with fp32 atomics (order-dependent rounding). */
+size_t sca_backward_full_workspace_size(msda_dims_t d);
+msda_status_t sca_backward_full(const void* value, msda_dtype_t vdt,
+                                const int64_t* spatial_shapes, const int64_t* level_start_index,
+                                const float* reference_points_cam, const uint8_t* bev_mask,
+                                const float* sampling_offsets, const float* attention_logits,
+                                const float* grad_out, msda_dims_t d, void* workspace,
+                                size_t workspace_bytes, float* grad_value,
+                                float* grad_sampling_offsets, float* grad_attention_logits,
+                                float* grad_reference_points_cam, msda_stream_t stream);
 
 /* Fixed text for a status code. */
 const char* msda_status_string(msda_status_t status);

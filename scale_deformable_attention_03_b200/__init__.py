@@ -105,6 +105,11 @@ def lib():
         L.sca_backward_inputs.argtypes = [_i64p, _i64p, _vp, _vp, _vp, _vp, Dims, _vp, _vp, _vp,
                                           _vp]
         L.sca_backward_inputs.restype = ctypes.c_int
+        L.sca_backward_full_workspace_size.argtypes = [Dims]
+        L.sca_backward_full_workspace_size.restype = ctypes.c_size_t
+        L.sca_backward_full.argtypes = [_vp, st, _i64p, _i64p, _vp, _vp, _vp, _vp, _vp, Dims,
+                                        _vp, ctypes.c_size_t, _vp, _vp, _vp, _vp, _vp]
+        L.sca_backward_full.restype = ctypes.c_int
         i32, f64 = ctypes.c_int32, ctypes.c_double
         L.tsa_reference_points.argtypes = [_vp, i32, i32, i32, i32, f64, f64, _vp, _vp]
         L.tsa_reference_points.restype = ctypes.c_int
@@ -446,6 +451,39 @@ def sca_backward(value, spatial_shapes, level_start_index, reference_points_cam,
               _ptr(grad_attention_weights_rb), _stream(stream)),
            "sca_backward_deterministic" if deterministic else "sca_backward")
     return grad_value, grad_sampling_locations_rb, grad_attention_weights_rb
+
+
+def sca_backward_full(value, spatial_shapes, level_start_index, reference_points_cam, bev_mask,
+                      sampling_offsets, attention_logits, grad_out, out=None, workspace=None,
+                      stream=None):
+    """The SCA backward down to its inputs -> (grad_value [B, Ncam, Nv, H, 32],
+    grad_sampling_offsets [B, Nq, H, L, P, 2], grad_attention_logits
+    [B, Nq, H, L, P], grad_reference_points_cam [Ncam, B, Nq, R, 2]); `out`
+    may supply the four tensors."""
+    torch = _torch()
+    _contig(value, reference_points_cam, bev_mask, sampling_offsets, attention_logits, grad_out)
+    if bev_mask.dtype == torch.bool:
+        bev_mask = bev_mask.view(torch.uint8)
+    d = _sca_dims(value, sampling_offsets, reference_points_cam)
+    shapes, starts = _levels(spatial_shapes, level_start_index)
+    dev = value.device
+    if out is not None:
+        gv, g_off, g_lg, g_ref = out
+        _contig(gv, g_off, g_lg, g_ref)
+    else:
+        gv = torch.empty(value.shape, device=dev, dtype=torch.float32)
+        g_off = torch.empty(sampling_offsets.shape, device=dev, dtype=torch.float32)
+        g_lg = torch.empty(attention_logits.shape, device=dev, dtype=torch.float32)
+        g_ref = torch.empty(reference_points_cam.shape, device=dev, dtype=torch.float32)
+    workspace = _workspace(int(lib().sca_backward_full_workspace_size(d)), dev, workspace)
+    _check(lib().sca_backward_full(_ptr(value), _vdt(value), shapes.ctypes.data_as(_i64p),
+                                   starts.ctypes.data_as(_i64p), _ptr(reference_points_cam),
+                                   _ptr(bev_mask), _ptr(sampling_offsets), _ptr(attention_logits),
+                                   _ptr(grad_out), d, _ptr(workspace), workspace.numel(),
+                                   _ptr(gv), _ptr(g_off), _ptr(g_lg), _ptr(g_ref),
+                                   _stream(stream)),
+           "sca_backward_full")
+    return gv, g_off, g_lg, g_ref
 
 
 def sca_rebatched_forward(value, spatial_shapes, level_start_index, reference_points_cam,

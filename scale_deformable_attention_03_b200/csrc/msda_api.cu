@@ -201,7 +201,7 @@ ScaWorkspace sca_workspace_carve(void* base, int B, int Ncam, int Nq, int H, boo
 
 extern "C" {
 
-int32_t msda_version(void) { return 10100; }  // 1.1.0: module dropout fields, TSA, deterministic backward
+int32_t msda_version(void) { return 10200; }  // 1.2.0: sca_backward_full, precise TSA chain, four-lane gather
 
 const char* msda_status_string(msda_status_t status)
 {
@@ -314,7 +314,8 @@ size_t tsa_backward_workspace_size(msda_dims_t d, int32_t num_queues)
     if (d.B < 0 || d.Nq < 0 || d.H < 1 || d.L < 1 || d.P < 1 || num_queues < 1) return 0;
     const size_t rows = (size_t)d.B * num_queues * d.Nq;
     const size_t S = (size_t)d.H * d.L * d.P;
-    return align256(sizeof(float) * rows * S * 2) + align256(sizeof(float) * rows * S);
+    // per queue row: location gradients, their fp32 rounding residuals, weight gradients
+    return 2 * align256(sizeof(float) * rows * S * 2) + align256(sizeof(float) * rows * S);
 }
 
 msda_status_t tsa_backward(const void* value, msda_dtype_t vdt, const int64_t* spatial_shapes,
@@ -349,18 +350,19 @@ msda_status_t tsa_backward(const void* value, msda_dtype_t vdt, const int64_t* s
     const cudaStream_t s = (cudaStream_t)stream;
     const int BT = d.B * num_queues;
     const size_t S = (size_t)d.H * d.L * d.P;
+    const size_t loc_bytes = align256(sizeof(float) * (size_t)BT * d.Nq * S * 2);
     float* gl = static_cast<float*>(workspace);
-    float* gw = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                         align256(sizeof(float) * (size_t)BT * d.Nq * S * 2));
+    float* gl_lo = reinterpret_cast<float*>(static_cast<char*>(workspace) + loc_bytes);
+    float* gw = reinterpret_cast<float*>(static_cast<char*>(workspace) + 2 * loc_bytes);
     const msda::Problem p = make_problem(value, vdt, d, lv);
     cudaError_t e = msda::launch_zero(grad_value, (int64_t)BT * d.Nv * d.H * MSDA_HEAD_DIM, s);
     if (e == cudaSuccess && d.Nq > 0)
         e = msda::launch_tsa_backward(p, num_queues, reference_points, sampling_offsets,
-                                      attention_logits, grad_out, grad_value, gl, gw, s);
+                                      attention_logits, grad_out, grad_value, gl, gl_lo, gw, s);
     if (e == cudaSuccess && d.Nq > 0)
         e = msda::launch_sca_input_grads(attention_logits, nullptr, gl, gw, BT, 1, d.Nq, d.H, d.L,
                                          d.P, d.R, lv, grad_sampling_offsets,
-                                         grad_attention_logits, grad_reference_points, s);
+                                         grad_attention_logits, grad_reference_points, s, gl_lo);
     return cuda_status(e, "tsa_backward");
 }
 
@@ -688,6 +690,65 @@ msda_status_t sca_backward_deterministic(const void* value, msda_dtype_t vdt,
 }
 
 }  // extern "C"
+
+extern "C" size_t sca_backward_full_workspace_size(msda_dims_t d)
+{
+    if (d.B < 0 || d.Ncam < 1 || d.Nq < 0 || d.H < 1 || d.L < 1 || d.P < 1) return 0;
+    const size_t rows = (size_t)d.B * d.Ncam * d.Nq;
+    const size_t S = (size_t)d.H * d.L * d.P;
+    return msda::sca_workspace_bytes(d.B, d.Ncam, d.Nq, d.H, false) +
+           2 * align256(sizeof(float) * rows * S * 2) + align256(sizeof(float) * rows * S);
+}
+
+extern "C" msda_status_t sca_backward_full(
+    const void* value, msda_dtype_t vdt, const int64_t* spatial_shapes,
+    const int64_t* level_start_index, const float* reference_points_cam, const uint8_t* bev_mask,
+    const float* sampling_offsets, const float* attention_logits, const float* grad_out,
+    msda_dims_t d, void* workspace, size_t workspace_bytes, float* grad_value,
+    float* grad_sampling_offsets, float* grad_attention_logits, float* grad_reference_points_cam,
+    msda_stream_t stream)
+{
+    msda::Levels lv;
+    MSDA_TRY(check_sca_inputs(value, vdt, d, spatial_shapes, level_start_index,
+                              reference_points_cam, sampling_offsets, attention_logits, lv));
+    MSDA_TRY(check_compact(d));
+    if (d.B == 0) return ok();
+    MSDA_PTR(grad_value, 16);
+    if (d.Nq > 0) {
+        MSDA_PTR(bev_mask, 1);
+        MSDA_PTR(grad_out, 16);
+        MSDA_PTR(grad_sampling_offsets, 8);
+        MSDA_PTR(grad_attention_logits, 4);
+        MSDA_PTR(grad_reference_points_cam, 4);
+    }
+    MSDA_TRY(check_workspace(workspace, workspace_bytes, sca_backward_full_workspace_size(d)));
+    const cudaStream_t s = (cudaStream_t)stream;
+    const msda::ScaWorkspace w = msda::sca_workspace_carve(workspace, d.B, d.Ncam, d.Nq, d.H, false);
+    const size_t rows = (size_t)d.B * d.Ncam * d.Nq;
+    const size_t S = (size_t)d.H * d.L * d.P;
+    char* rest = static_cast<char*>(workspace) +
+                 msda::sca_workspace_bytes(d.B, d.Ncam, d.Nq, d.H, false);
+    const size_t loc_bytes = align256(sizeof(float) * rows * S * 2);
+    float* gl = reinterpret_cast<float*>(rest);
+    float* gl_lo = reinterpret_cast<float*>(rest + loc_bytes);
+    float* gw = reinterpret_cast<float*>(rest + 2 * loc_bytes);
+    const msda::Problem p = make_problem(value, vdt, d, lv);
+    cudaError_t e = msda::launch_zero(grad_value,
+                                      (int64_t)d.B * d.Ncam * d.Nv * d.H * MSDA_HEAD_DIM, s);
+    if (e == cudaSuccess && d.Nq > 0)
+        e = msda::launch_sca_compact(bev_mask, d.B, d.Ncam, d.Nq, d.R, w.idx, w.count, w.pos,
+                                     w.hits, w.chunk_counts, s);
+    if (e == cudaSuccess && d.Nq > 0)
+        e = msda::launch_sca_backward_rows(p, reference_points_cam, sampling_offsets,
+                                           attention_logits, grad_out, w.idx, w.hits, w.count,
+                                           grad_value, nullptr, gl, gw, s, gl_lo);
+    if (e == cudaSuccess && d.Nq > 0)
+        e = msda::launch_sca_input_grads(attention_logits, w.pos, gl, gw, d.B, d.Ncam, d.Nq, d.H,
+                                         d.L, d.P, d.R, lv, grad_sampling_offsets,
+                                         grad_attention_logits, grad_reference_points_cam, s,
+                                         gl_lo);
+    return cuda_status(e, "sca_backward_full");
+}
 
 extern "C" msda_status_t sca_backward_inputs(const int64_t* spatial_shapes,
                                              const int64_t* level_start_index,

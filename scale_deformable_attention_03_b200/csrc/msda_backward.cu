@@ -65,6 +65,57 @@ __device__ __forceinline__ void red_add_fix(long long* addr, float v)
     asm volatile("red.global.add.u64 [%0], %1;" ::"l"(addr), "l"(q) : "memory");
 }
 
+__device__ __forceinline__ double warp_sum_d(double v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ double segment_sum_d(double v, int npad)
+{
+    for (int o = npad >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// row_weights with the softmax formed in double ("BEV(三)..." section 4.2):
+// ad = exp(x - max) / sum in double, a = ad rounded once to fp32.
+template <bool FUSED, int NC>
+__device__ __forceinline__ void row_weights_f64(const float* __restrict__ src, int n, int lane,
+                                                float (&a)[NC], double (&ad)[NC])
+{
+    float x[NC];
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+        const int j = c * 32 + lane;
+        x[c] = (j < n) ? ld_stream(src + j) : (FUSED ? -INFINITY : 0.f);
+    }
+    if (!FUSED) {
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+            a[c] = x[c];
+            ad[c] = x[c];
+        }
+        return;
+    }
+    float m = x[0];
+#pragma unroll
+    for (int c = 1; c < NC; ++c) m = fmaxf(m, x[c]);
+    m = warp_max(m);
+    double z = 0.0;
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+        ad[c] = (c * 32 + lane < n) ? exp((double)x[c] - (double)m) : 0.0;
+        z += ad[c];
+    }
+    z = warp_sum_d(z);
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+        ad[c] = ad[c] / z;
+        a[c] = (float)ad[c];
+    }
+}
+
 // d w_g / d lx and d w_g / d ly for neighbour g.
 __device__ __forceinline__ double dw_dlx(int g, float ly)
 {
@@ -313,7 +364,12 @@ struct BwdLanes<__nv_bfloat16> {
 // [L, P, 2], gattn_row [L, P].  LF: issue a batch's eight corner loads before
 // its grad_value reductions (more registers; faster in the persistent SCA
 // kernel, whose grid is sized to the resident CTAs, slower elsewhere).
-template <typename VT, bool FUSED, int NC, bool DET, bool LF = false>
+// PREC (the precise location gradients that the chain to offsets and
+// reference points sums): the softmax weight and the location gradient are
+// formed in double, and gloc_lo_row receives the residual of the fp32
+// rounding (gloc = hi, gloc_lo = fp32(exact - hi)), so that sums over many
+// samples keep double accuracy.
+template <typename VT, bool FUSED, int NC, bool DET, bool LF = false, bool PREC = false>
 __device__ __forceinline__ void row_backward(const VT* __restrict__ vb, int H, int h,
                                              const float* __restrict__ lo,
                                              const float* __restrict__ wl,
@@ -323,12 +379,17 @@ __device__ __forceinline__ void row_backward(const VT* __restrict__ vb, int H, i
                                              float* __restrict__ gvb, long long* __restrict__ gvi,
                                              DetEntry* __restrict__ det,
                                              float* __restrict__ gloc_row,
-                                             float* __restrict__ gattn_row, int lane)
+                                             float* __restrict__ gattn_row, int lane,
+                                             float* __restrict__ gloc_lo_row = nullptr)
 {
     // DET: channel `lane` of the row's upstream gradient, as BwdLanes forms it
     const float go_c = DET ? __ldg(grow + lane) / scale : 0.f;
     float a[NC];
-    row_weights<FUSED, NC>(wl, n, lane, a);
+    double ad[NC];
+    if constexpr (PREC)
+        row_weights_f64<FUSED, NC>(wl, n, lane, a, ad);
+    else
+        row_weights<FUSED, NC>(wl, n, lane, a);
     using Lanes = BwdLanes<VT>;
     Lanes lanes;
     lanes.load_grad(grow, scale, lane);
@@ -365,7 +426,8 @@ __device__ __forceinline__ void row_backward(const VT* __restrict__ vb, int H, i
             }
         }
         __syncwarp();
-        float res_w = 0.f, res_x = 0.f, res_y = 0.f;
+        float res_w = 0.f;
+        typename std::conditional<PREC, double, float>::type res_x = 0, res_y = 0;
         const int cnt = min(32, n - c * 32);
         for (int j0 = 0; j0 < cnt; j0 += 8) {
             const double d = lanes.template batch<DET, LF>(vb, gvb, gvi, tab, j0, cnt, lane);
@@ -390,12 +452,13 @@ __device__ __forceinline__ void row_backward(const VT* __restrict__ vb, int H, i
                 c4[2] = dy * d;
             }
             // lanes of group 0, 1, 2 now hold the weight, x and y sums
-            const float r = (float)reduce_scatter_groups(c4, g, Lanes::kStride);
+            using R = typename std::conditional<PREC, double, float>::type;
+            const R r = (R)reduce_scatter_groups(c4, g, Lanes::kStride);
             // the owner of sample j0 + u is lane j0 + u; fetch from the lanes holding it
             const int src = Lanes::holder(lane & 7);
-            const float tw = __shfl_sync(0xffffffffu, r, src);
-            const float tx = __shfl_sync(0xffffffffu, r, src + Lanes::kStride);
-            const float ty = __shfl_sync(0xffffffffu, r, src + 2 * Lanes::kStride);
+            const float tw = __shfl_sync(0xffffffffu, (float)r, src);
+            const R tx = __shfl_sync(0xffffffffu, r, src + Lanes::kStride);
+            const R ty = __shfl_sync(0xffffffffu, r, src + 2 * Lanes::kStride);
             if ((lane & ~7) == j0) {
                 res_w = tw;
                 res_x = tx;
@@ -404,9 +467,18 @@ __device__ __forceinline__ void row_backward(const VT* __restrict__ vb, int H, i
         }
         if (j < n) {
             gattn_row[j] = res_w;
-            const float al = a[c];
-            *reinterpret_cast<float2*>(gloc_row + 2 * j) =
-                make_float2(cr.valid ? al * Wl * res_x : 0.f, cr.valid ? al * Hl * res_y : 0.f);
+            if constexpr (PREC) {
+                const double gx = cr.valid ? ad[c] * (double)Wl * res_x : 0.0;
+                const double gy = cr.valid ? ad[c] * (double)Hl * res_y : 0.0;
+                const float hx = (float)gx, hy = (float)gy;
+                *reinterpret_cast<float2*>(gloc_row + 2 * j) = make_float2(hx, hy);
+                *reinterpret_cast<float2*>(gloc_lo_row + 2 * j) =
+                    make_float2((float)(gx - (double)hx), (float)(gy - (double)hy));
+            } else {
+                const float al = a[c];
+                *reinterpret_cast<float2*>(gloc_row + 2 * j) = make_float2(
+                    cr.valid ? al * Wl * res_x : 0.f, cr.valid ? al * Hl * res_y : 0.f);
+            }
         }
         __syncwarp();
     }
@@ -531,25 +603,37 @@ struct GroupBwdLanes<__nv_bfloat16> {
 // the lane's channel of each head's grad_out / scale.  gvb / gvi: grad_value
 // of the batch item or its fixed-point copy; gloc0 [G, S, 2] and gattn0
 // [G, S]: head h0's gradients (+S per head).
-template <typename VT, bool FUSED, int NPL, bool DET>
+// PREC: as in row_backward (double softmax and location gradients, the fp32
+// rounding residual of the location gradients into gloc_lo0).
+template <typename VT, bool FUSED, int NPL, bool DET, bool PREC = false>
 __device__ __forceinline__ void group_backward(const VT* __restrict__ vb, int H, int h0, int S,
                                                float a, float2 v, float2 r, bool valid,
                                                const float (&go)[32 >> NPL], const GroupLane& gl,
                                                GroupBwdTable& tab, float* __restrict__ gvb,
                                                long long* __restrict__ gvi,
                                                float* __restrict__ gloc0,
-                                               float* __restrict__ gattn0, int lane)
+                                               float* __restrict__ gattn0, int lane,
+                                               float* __restrict__ gloc_lo0 = nullptr)
 {
     constexpr int G = 32 >> NPL;
     constexpr int npad = 1 << NPL;
+    double ad = 0.0;
     if (FUSED) {
         const float m = segment_max(a, npad);
-        const float e = valid ? expf(a - m) : 0.f;
-        const float z = segment_sum(e, npad);
-        a = valid ? e / z : 0.f;
+        if constexpr (PREC) {
+            const double e = valid ? exp((double)a - (double)m) : 0.0;
+            const double z = segment_sum_d(e, npad);
+            ad = valid ? e / z : 0.0;
+            a = (float)ad;
+        } else {
+            const float e = valid ? expf(a - m) : 0.f;
+            const float z = segment_sum(e, npad);
+            a = valid ? e / z : 0.f;
+        }
     } else if (!valid) {
         a = 0.f;
     }
+    if (!FUSED) ad = a;
     Corners cr;
     if (valid) {
         float sx = v.x, sy = v.y;
@@ -581,7 +665,9 @@ __device__ __forceinline__ void group_backward(const VT* __restrict__ vb, int H,
     const int g = Lanes::group(lane);
     const int held = Lanes::held(lane);
     const int nheads = min(G, H - h0);
-    float res_w = 0.f, res_x = 0.f, res_y = 0.f;
+    using R = typename std::conditional<PREC, double, float>::type;
+    float res_w = 0.f;
+    R res_x = 0, res_y = 0;
 #pragma unroll
     for (int j0 = 0; j0 < 32; j0 += 8) {
         if ((j0 >> NPL) >= nheads) break;
@@ -608,12 +694,12 @@ __device__ __forceinline__ void group_backward(const VT* __restrict__ vb, int H,
         double dx, dy;
         corner_weight(g, tab.l[j0 + held], wg, dx, dy);
         const double c4[4] = {(double)wg * d, dx * d, dy * d, 0.0};
-        const float r = (float)reduce_scatter_groups(c4, g, BwdLanes<VT>::kStride);
+        const R r = (R)reduce_scatter_groups(c4, g, BwdLanes<VT>::kStride);
         // sample j0 + u lands on lane j0 + u
         const int src = Lanes::holder(lane & 7);
-        const float tw = __shfl_sync(0xffffffffu, r, src);
-        const float tx = __shfl_sync(0xffffffffu, r, src + BwdLanes<VT>::kStride);
-        const float ty = __shfl_sync(0xffffffffu, r, src + 2 * BwdLanes<VT>::kStride);
+        const float tw = __shfl_sync(0xffffffffu, (float)r, src);
+        const R tx = __shfl_sync(0xffffffffu, r, src + BwdLanes<VT>::kStride);
+        const R ty = __shfl_sync(0xffffffffu, r, src + 2 * BwdLanes<VT>::kStride);
         if ((lane & ~7) == j0) {
             res_w = tw;
             res_x = tx;
@@ -623,9 +709,18 @@ __device__ __forceinline__ void group_backward(const VT* __restrict__ vb, int H,
     if (valid) {
         const int j = gl.s * S + gl.k;
         gattn0[j] = res_w;
-        *reinterpret_cast<float2*>(gloc0 + 2 * j) =
-            make_float2(cr.valid ? a * (float)gl.w * res_x : 0.f,
-                        cr.valid ? a * (float)gl.h * res_y : 0.f);
+        if constexpr (PREC) {
+            const double gx = cr.valid ? ad * (double)gl.w * res_x : 0.0;
+            const double gy = cr.valid ? ad * (double)gl.h * res_y : 0.0;
+            const float hx = (float)gx, hy = (float)gy;
+            *reinterpret_cast<float2*>(gloc0 + 2 * j) = make_float2(hx, hy);
+            *reinterpret_cast<float2*>(gloc_lo0 + 2 * j) =
+                make_float2((float)(gx - (double)hx), (float)(gy - (double)hy));
+        } else {
+            *reinterpret_cast<float2*>(gloc0 + 2 * j) =
+                make_float2(cr.valid ? a * (float)gl.w * res_x : 0.f,
+                            cr.valid ? a * (float)gl.h * res_y : 0.f);
+        }
     }
     __syncwarp();
 }
@@ -674,14 +769,17 @@ msda_backward_kernel(const VT* __restrict__ value, const float* __restrict__ loc
     }
 }
 
-template <typename VT, int NC, bool DET>
+// PREC: precise location gradients with their rounding residual into
+// grad_loc_lo_rb (see row_backward), for the chain to offsets and reference
+// points.
+template <typename VT, int NC, bool DET, bool PREC>
 __global__ void __launch_bounds__(kThreads)
 sca_backward_kernel(const VT* __restrict__ value, const float* __restrict__ off,
                     const float* __restrict__ logits, const float* __restrict__ ref_cam,
                     const float* __restrict__ grad_out, const int32_t* __restrict__ idx,
                     const int32_t* __restrict__ hits, const int32_t* __restrict__ count,
                     float* __restrict__ grad_value, long long* __restrict__ grad_value_fix,
-                    float* __restrict__ grad_loc_rb,
+                    float* __restrict__ grad_loc_rb, float* __restrict__ grad_loc_lo_rb,
                     float* __restrict__ grad_attn_rb, int B, int Ncam, int Nq, int Nv, int H,
                     int L, int P, int R, Levels levels)
 {
@@ -691,7 +789,7 @@ sca_backward_kernel(const VT* __restrict__ value, const float* __restrict__ off,
     __shared__ int s_prefix[kMaxBatchCameras + 1];
     const int nbc = B * Ncam;
     stage_levels(s_lv, levels);
-    stage_row_prefix(count, nbc, s_prefix);
+    stage_row_prefix(count, nbc, Nq, s_prefix);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     LaneSamples<NC> ls;
     lane_samples<NC>(s_lv, L, P, R, lane, ls);
@@ -719,14 +817,13 @@ sca_backward_kernel(const VT* __restrict__ value, const float* __restrict__ off,
             const int64_t vofs = (int64_t)bc * Nv * H * kHeadDim;
             const int64_t rowh = ((int64_t)bc * Nq + i) * H + h;
             const float scale = (float)max(1, __ldg(hits + bq));
-            row_backward<VT, true, NC, DET, true>(value + vofs, H, h, off + bqh * S * 2,
-                                            logits + bqh * S,
-                                            ref_cam + (((int64_t)c * B + b) * Nq + q) * R * 2, S,
-                                            ls, s_tab[warp], grad_out + bqh * kHeadDim, scale,
-                                            grad_value + vofs,
-                                            DET ? grad_value_fix + vofs : nullptr,
-                                            s_det[DET ? warp : 0], grad_loc_rb + rowh * S * 2,
-                                            grad_attn_rb + rowh * S, lane);
+            row_backward<VT, true, NC, DET, true, PREC>(
+                value + vofs, H, h, off + bqh * S * 2, logits + bqh * S,
+                ref_cam + (((int64_t)c * B + b) * Nq + q) * R * 2, S, ls, s_tab[warp],
+                grad_out + bqh * kHeadDim, scale, grad_value + vofs,
+                DET ? grad_value_fix + vofs : nullptr, s_det[DET ? warp : 0],
+                grad_loc_rb + rowh * S * 2, grad_attn_rb + rowh * S, lane,
+                PREC ? grad_loc_lo_rb + rowh * S * 2 : nullptr);
         }
     }
 }
@@ -739,8 +836,9 @@ __global__ void __launch_bounds__(kThreads)
 tsa_backward_kernel(const VT* __restrict__ value, const float* __restrict__ off,
                     const float* __restrict__ logits, const float* __restrict__ ref,
                     const float* __restrict__ grad_out, float* __restrict__ grad_value,
-                    float* __restrict__ grad_loc, float* __restrict__ grad_attn, int BT, int T,
-                    int Nq, int Nv, int H, int L, int P, int R, Levels levels)
+                    float* __restrict__ grad_loc, float* __restrict__ grad_loc_lo,
+                    float* __restrict__ grad_attn, int BT, int T, int Nq, int Nv, int H, int L,
+                    int P, int R, Levels levels)
 {
     __shared__ SmemLevels s_lv;
     __shared__ __align__(16) BwdTable s_tab[kWarps];
@@ -766,11 +864,11 @@ tsa_backward_kernel(const VT* __restrict__ value, const float* __restrict__ off,
         const int64_t item = r * H + cur.h;
         const int64_t gitem = ((int64_t)(bt / T) * Nq + q) * H + cur.h;
         const int64_t vofs = (int64_t)bt * Nv * H * kHeadDim;
-        row_backward<VT, true, NC, false>(value + vofs, H, cur.h, off + item * S * 2,
-                                          logits + item * S, ref + r * R * 2, S, ls, s_tab[warp],
-                                          grad_out + gitem * kHeadDim, (float)T,
-                                          grad_value + vofs, nullptr, nullptr,
-                                          grad_loc + item * S * 2, grad_attn + item * S, lane);
+        row_backward<VT, true, NC, false, false, true>(
+            value + vofs, H, cur.h, off + item * S * 2, logits + item * S, ref + r * R * 2, S, ls,
+            s_tab[warp], grad_out + gitem * kHeadDim, (float)T, grad_value + vofs, nullptr,
+            nullptr, grad_loc + item * S * 2, grad_attn + item * S, lane,
+            grad_loc_lo + item * S * 2);
     }
 }
 
@@ -788,15 +886,15 @@ constexpr int kBwdGroupRowsPerTile = MSDA_GROUP_ROWS_PER_TILE;
 #ifndef MSDA_BWD_GROUP_MIN_CTAS
 #define MSDA_BWD_GROUP_MIN_CTAS 3
 #endif
-template <typename VT, int NPL, bool FUSED, bool DET>
+template <typename VT, int NPL, bool FUSED, bool DET, bool PREC>
 __global__ void __launch_bounds__(kThreads,
                                   NPL == 2 ? MSDA_BWD_GROUP4_MIN_CTAS : MSDA_BWD_GROUP_MIN_CTAS)
 backward_group_kernel(const VT* __restrict__ value, const float* __restrict__ off,
                       const float* __restrict__ logits, const float* __restrict__ ref,
                       const float* __restrict__ grad_out, float* __restrict__ grad_value,
                       long long* __restrict__ grad_value_fix, float* __restrict__ grad_loc,
-                      float* __restrict__ grad_attn, int BT, int T, int Nq, int Nv, int H, int L,
-                      int P, int R, Levels levels)
+                      float* __restrict__ grad_loc_lo, float* __restrict__ grad_attn, int BT,
+                      int T, int Nq, int Nv, int H, int L, int P, int R, Levels levels)
 {
     constexpr int G = 32 >> NPL;
     __shared__ SmemLevels s_lv;
@@ -867,11 +965,10 @@ backward_group_kernel(const VT* __restrict__ value, const float* __restrict__ of
         if (x1.ok) fetch(x1, in1);
         const int64_t vofs = (int64_t)x0.bt * vstride;
         const int64_t item0 = x0.r * H + x0.h0;
-        group_backward<VT, FUSED, NPL, DET>(value + vofs, H, x0.h0, S, in0.a, in0.v, in0.r,
-                                            x0.valid, in0.go, gl, s_tab[warp], grad_value + vofs,
-                                            DET ? grad_value_fix + vofs : nullptr,
-                                            grad_loc + item0 * S * 2, grad_attn + item0 * S,
-                                            lane);
+        group_backward<VT, FUSED, NPL, DET, PREC>(
+            value + vofs, H, x0.h0, S, in0.a, in0.v, in0.r, x0.valid, in0.go, gl, s_tab[warp],
+            grad_value + vofs, DET ? grad_value_fix + vofs : nullptr, grad_loc + item0 * S * 2,
+            grad_attn + item0 * S, lane, PREC ? grad_loc_lo + item0 * S * 2 : nullptr);
         x0 = x1;
         in0 = in1;
         cur = nx;
@@ -889,12 +986,13 @@ static int group_npl(int S, int H)
     return npl;
 }
 
-template <typename VT, bool FUSED, bool DET>
+template <typename VT, bool FUSED, bool DET, bool PREC = false>
 static cudaError_t launch_backward_group(const Problem& p, int npl, int BT, int T,
                                          const float* ref, const float* off, const float* logits,
                                          const float* grad_out, float* grad_value,
                                          long long* grad_value_fix, float* grad_loc,
-                                         float* grad_attn, cudaStream_t s)
+                                         float* grad_attn, cudaStream_t s,
+                                         float* grad_loc_lo = nullptr)
 {
     const int64_t rows = (int64_t)BT * p.Nq;
     const unsigned grid = (unsigned)((rows + kBwdGroupRowsPerTile - 1) / kBwdGroupRowsPerTile);
@@ -902,9 +1000,9 @@ static cudaError_t launch_backward_group(const Problem& p, int npl, int BT, int 
     switch (npl) {
 #define BWD_GROUP_CASE(NPLV)                                                                     \
     case NPLV:                                                                                   \
-        backward_group_kernel<VT, NPLV, FUSED, DET><<<grid, kThreads, 0, s>>>(                   \
-            v, off, logits, ref, grad_out, grad_value, grad_value_fix, grad_loc, grad_attn, BT,  \
-            T, p.Nq, p.Nv, p.H, p.L, p.P, p.R, p.lv);                                            \
+        backward_group_kernel<VT, NPLV, FUSED, DET, PREC><<<grid, kThreads, 0, s>>>(             \
+            v, off, logits, ref, grad_out, grad_value, grad_value_fix, grad_loc, grad_loc_lo,    \
+            grad_attn, BT, T, p.Nq, p.Nv, p.H, p.L, p.P, p.R, p.lv);                             \
         break;
         BWD_GROUP_CASE(2)
         BWD_GROUP_CASE(3)
@@ -919,23 +1017,24 @@ template <typename VT>
 static cudaError_t launch_tsa_backward_t(const Problem& p, int T, const float* ref,
                                          const float* off, const float* logits,
                                          const float* grad_out, float* grad_value,
-                                         float* grad_loc, float* grad_attn, cudaStream_t s)
+                                         float* grad_loc, float* grad_loc_lo, float* grad_attn,
+                                         cudaStream_t s)
 {
     const int BT = p.B * T;
     const int64_t rows = (int64_t)BT * p.Nq;
     if (rows == 0) return cudaSuccess;
     if (const int npl = group_npl(p.L * p.P, p.H))
-        return launch_backward_group<VT, true, false>(p, npl, BT, T, ref, off, logits, grad_out,
-                                                      grad_value, nullptr, grad_loc, grad_attn,
-                                                      s);
+        return launch_backward_group<VT, true, false, true>(p, npl, BT, T, ref, off, logits,
+                                                            grad_out, grad_value, nullptr,
+                                                            grad_loc, grad_attn, s, grad_loc_lo);
     const unsigned grid = (unsigned)((rows + kBwdRowsPerTile - 1) / kBwdRowsPerTile);
     const VT* v = static_cast<const VT*>(p.value);
     switch ((p.L * p.P + 31) / 32) {
 #define TSA_BWD_CASE(NCV)                                                                        \
     case NCV:                                                                                    \
         tsa_backward_kernel<VT, NCV><<<grid, kThreads, 0, s>>>(                                  \
-            v, off, logits, ref, grad_out, grad_value, grad_loc, grad_attn, BT, T, p.Nq, p.Nv,   \
-            p.H, p.L, p.P, p.R, p.lv);                                                           \
+            v, off, logits, ref, grad_out, grad_value, grad_loc, grad_loc_lo, grad_attn, BT, T,  \
+            p.Nq, p.Nv, p.H, p.L, p.P, p.R, p.lv);                                               \
         break;
         TSA_BWD_CASE(1)
         TSA_BWD_CASE(2)
@@ -949,12 +1048,14 @@ static cudaError_t launch_tsa_backward_t(const Problem& p, int T, const float* r
 
 cudaError_t launch_tsa_backward(const Problem& p, int T, const float* ref, const float* off,
                                 const float* logits, const float* grad_out, float* grad_value,
-                                float* grad_loc, float* grad_attn, cudaStream_t s)
+                                float* grad_loc, float* grad_loc_lo, float* grad_attn,
+                                cudaStream_t s)
 {
     return p.bf16 ? launch_tsa_backward_t<__nv_bfloat16>(p, T, ref, off, logits, grad_out,
-                                                         grad_value, grad_loc, grad_attn, s)
+                                                         grad_value, grad_loc, grad_loc_lo,
+                                                         grad_attn, s)
                   : launch_tsa_backward_t<float>(p, T, ref, off, logits, grad_out, grad_value,
-                                                 grad_loc, grad_attn, s);
+                                                 grad_loc, grad_loc_lo, grad_attn, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -984,7 +1085,8 @@ __global__ void sca_zero_tail_kernel(const int32_t* __restrict__ count, int Nq, 
                                      float* __restrict__ grad_attn_rb)
 {
     const int bc = blockIdx.y;
-    const int64_t first = (int64_t)bc * Nq + __ldg(count + bc), last = (int64_t)bc * Nq + Nq;
+    const int n = min(max(__ldg(count + bc), 0), Nq);  // inconsistent counts stay in the block
+    const int64_t first = (int64_t)bc * Nq + n, last = (int64_t)bc * Nq + Nq;
     const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t nthreads = (int64_t)gridDim.x * blockDim.x;
     zero_range(grad_loc_rb + first * S * 2, (last - first) * S * 2, tid, nthreads);
@@ -1086,13 +1188,14 @@ static int bwd_resident_ctas(K kernel)
     return n;
 }
 
-template <typename VT, bool DET>
+template <typename VT, bool DET, bool PREC>
 static cudaError_t launch_sca_backward_t(const Problem& p, const float* ref_cam, const float* off,
                                          const float* logits, const float* grad_out,
                                          const int32_t* idx, const int32_t* hits,
                                          const int32_t* count, float* grad_value,
                                          long long* grad_value_fix, float* grad_loc_rb,
-                                         float* grad_attn_rb, cudaStream_t s)
+                                         float* grad_loc_lo_rb, float* grad_attn_rb,
+                                         cudaStream_t s)
 {
     const int64_t max_rows = (int64_t)p.B * p.Ncam * p.Nq;
     if (max_rows == 0) return cudaSuccess;
@@ -1101,11 +1204,12 @@ static cudaError_t launch_sca_backward_t(const Problem& p, const float* ref_cam,
     const int nc = (p.L * p.P + 31) / 32;
 #define SCA_BWD_CASE(NCV)                                                                        \
     case NCV: {                                                                                  \
-        static int occ = bwd_resident_ctas(sca_backward_kernel<VT, NCV, DET>);                   \
+        static int occ = bwd_resident_ctas(sca_backward_kernel<VT, NCV, DET, PREC>);             \
         const int64_t grid = std::min<int64_t>(max_ctas, (int64_t)occ * device_sm_count());      \
-        sca_backward_kernel<VT, NCV, DET><<<(unsigned)grid, kThreads, 0, s>>>(                   \
+        sca_backward_kernel<VT, NCV, DET, PREC><<<(unsigned)grid, kThreads, 0, s>>>(             \
             v, off, logits, ref_cam, grad_out, idx, hits, count, grad_value, grad_value_fix,     \
-            grad_loc_rb, grad_attn_rb, p.B, p.Ncam, p.Nq, p.Nv, p.H, p.L, p.P, p.R, p.lv);       \
+            grad_loc_rb, grad_loc_lo_rb, grad_attn_rb, p.B, p.Ncam, p.Nq, p.Nv, p.H, p.L, p.P,   \
+            p.R, p.lv);                                                                          \
         break;                                                                                   \
     }
     switch (nc) {
@@ -1124,22 +1228,20 @@ cudaError_t launch_sca_backward_rows(const Problem& p, const float* ref_cam, con
                                      const int32_t* idx, const int32_t* hits,
                                      const int32_t* count, float* grad_value,
                                      long long* grad_value_fix, float* grad_loc_rb,
-                                     float* grad_attn_rb, cudaStream_t s)
+                                     float* grad_attn_rb, cudaStream_t s, float* grad_loc_lo_rb)
 {
+#define SCA_BWD_ARGS                                                                             \
+    p, ref_cam, off, logits, grad_out, idx, hits, count, grad_value, grad_value_fix, grad_loc_rb, \
+        grad_loc_lo_rb, grad_attn_rb, s
     if (grad_value_fix)
-        return p.bf16 ? launch_sca_backward_t<__nv_bfloat16, true>(
-                            p, ref_cam, off, logits, grad_out, idx, hits, count, grad_value,
-                            grad_value_fix, grad_loc_rb, grad_attn_rb, s)
-                      : launch_sca_backward_t<float, true>(p, ref_cam, off, logits, grad_out, idx,
-                                                           hits, count, grad_value, grad_value_fix,
-                                                           grad_loc_rb, grad_attn_rb, s);
-    return p.bf16 ? launch_sca_backward_t<__nv_bfloat16, false>(p, ref_cam, off, logits, grad_out,
-                                                                idx, hits, count, grad_value,
-                                                                nullptr, grad_loc_rb,
-                                                                grad_attn_rb, s)
-                  : launch_sca_backward_t<float, false>(p, ref_cam, off, logits, grad_out, idx,
-                                                        hits, count, grad_value, nullptr,
-                                                        grad_loc_rb, grad_attn_rb, s);
+        return p.bf16 ? launch_sca_backward_t<__nv_bfloat16, true, false>(SCA_BWD_ARGS)
+                      : launch_sca_backward_t<float, true, false>(SCA_BWD_ARGS);
+    if (grad_loc_lo_rb)
+        return p.bf16 ? launch_sca_backward_t<__nv_bfloat16, false, true>(SCA_BWD_ARGS)
+                      : launch_sca_backward_t<float, false, true>(SCA_BWD_ARGS);
+    return p.bf16 ? launch_sca_backward_t<__nv_bfloat16, false, false>(SCA_BWD_ARGS)
+                  : launch_sca_backward_t<float, false, false>(SCA_BWD_ARGS);
+#undef SCA_BWD_ARGS
 }
 
 }  // namespace msda

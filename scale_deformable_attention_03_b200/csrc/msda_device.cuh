@@ -733,15 +733,18 @@ struct ItemCursor {
 };
 
 // Row offsets of the rebatched layout: s_prefix[bc] = sum of count[0..bc),
-// s_prefix[n] = total rows.  Warp 0 scans; the whole block must call this.
-__device__ __forceinline__ void stage_row_prefix(const int32_t* __restrict__ count, int n,
+// s_prefix[n] = total rows.  Each count is clamped to [0, cap] (cap = Nq, the
+// capacity of a (batch, camera) block of rows), so inconsistent counts never
+// address rows outside their block.  Warp 0 scans; the whole block must call
+// this.
+__device__ __forceinline__ void stage_row_prefix(const int32_t* __restrict__ count, int n, int cap,
                                                  int* s_prefix)
 {
     if (threadIdx.x < 32) {
         const int lane = threadIdx.x;
         int run = 0;
         for (int base = 0; base < n; base += 32) {
-            const int v = (base + lane < n) ? __ldg(count + base + lane) : 0;
+            const int v = (base + lane < n) ? min(max(__ldg(count + base + lane), 0), cap) : 0;
             int incl = v;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {

@@ -56,6 +56,13 @@ cudaError_t launch_sca_gather(const Problem& p, const float* ref_cam, const floa
                               const float* logits, const int32_t* idx, const int32_t* count,
                               float* out_rb, cudaStream_t s);
 
+// K3 with four lanes per (row, head) for rows of up to 32 samples
+// (sca_gather_quad.cu); sca_gather_quad_fits says whether a problem qualifies.
+bool sca_gather_quad_fits(const Problem& p);
+cudaError_t launch_sca_gather_quad(const Problem& p, const float* ref_cam, const float* off,
+                                   const float* logits, const int32_t* idx, const int32_t* count,
+                                   float* out_rb, cudaStream_t s);
+
 // K3q: the whole SCA forward, query-major (no compaction, no rebatched rows).
 cudaError_t launch_sca_query_major(const Problem& p, const float* ref_cam, const uint8_t* mask,
                                    const float* off, const float* logits, float* out,
@@ -74,12 +81,16 @@ cudaError_t launch_msda_backward(const Problem& p, const float* loc, const float
                                  const float* grad_out, float* grad_value,
                                  long long* grad_value_fix, float* grad_loc, float* grad_attn,
                                  cudaStream_t s);
+// grad_loc_lo_rb non-null: the precise location gradients (softmax and
+// location gradient in double), with the fp32 rounding residual of each
+// location gradient written there (not with grad_value_fix).
 cudaError_t launch_sca_backward_rows(const Problem& p, const float* ref_cam, const float* off,
                                      const float* logits, const float* grad_out,
                                      const int32_t* idx, const int32_t* hits,
                                      const int32_t* count, float* grad_value,
                                      long long* grad_value_fix, float* grad_loc_rb,
-                                     float* grad_attn_rb, cudaStream_t s);
+                                     float* grad_attn_rb, cudaStream_t s,
+                                     float* grad_loc_lo_rb = nullptr);
 cudaError_t launch_fix_to_float(const long long* acc, float* out, int64_t n, cudaStream_t s);
 cudaError_t launch_sca_zero_tail(const int32_t* count, int B, int Ncam, int Nq, int S,
                                  float* grad_loc_rb, float* grad_attn_rb, cudaStream_t s);
@@ -90,12 +101,13 @@ cudaError_t launch_sca_zero_tail(const int32_t* count, int B, int Ncam, int Nq, 
 
 namespace msda {
 // Gradients of offsets, logits and reference points (sca_input_grads.cu);
-// pos == null: Ncam = 1 and row i is query i.
+// pos == null: Ncam = 1 and row i is query i.  grad_loc_lo_rb (may be null):
+// the fp32 rounding residuals of grad_loc_rb, added in double.
 cudaError_t launch_sca_input_grads(const float* logits, const int32_t* pos,
                                    const float* grad_loc_rb, const float* grad_attn_rb, int B,
                                    int Ncam, int Nq, int H, int L, int P, int R, const Levels& lv,
                                    float* grad_off, float* grad_logits, float* grad_ref_cam,
-                                   cudaStream_t s);
+                                   cudaStream_t s, const float* grad_loc_lo_rb = nullptr);
 
 // TSA (tsa.cu): ego-motion reference points and the queue-mean fused forward.
 cudaError_t launch_tsa_reference(const float* ego, int B, int T, int bev_h, int bev_w, double gx,
@@ -142,7 +154,8 @@ msda_status_t sca_rebatched_backward_to(const void* value, msda_dtype_t vdt, con
 // BEV samples, the value holds p.B * T items.
 cudaError_t launch_tsa_backward(const Problem& p, int T, const float* ref, const float* off,
                                 const float* logits, const float* grad_out, float* grad_value,
-                                float* grad_loc, float* grad_attn, cudaStream_t s);
+                                float* grad_loc, float* grad_loc_lo, float* grad_attn,
+                                cudaStream_t s);
 
 // Set the per-thread error message of msda_last_error() and return the code.
 msda_status_t api_fail(msda_status_t code, const char* message);

@@ -1,7 +1,8 @@
 // SCA forward pieces (Tencent Cloud "Spatial Cross-Attention" walkthrough,
 // rebatch and average listings; "BEV(三) BEVFormer ..." section 10):
 //   K2a sca_count_kernel    hits per query, seeing queries per 1024-query chunk
-//   K2b sca_scatter_kernel  stable ranks -> idx / pos / count / row prefix
+//   K2s sca_chunk_scan_kernel  per-camera prefix of the chunk counts, count
+//   K2b sca_scatter_kernel  stable ranks -> idx / pos
 //   K3  sca_gather_kernel   fused MSDA over every camera's seeing queries
 //   K4  sca_average_kernel  per-query sum over cameras / max(1, hits)
 // Nothing here synchronises with the host: the rebatched row counts live in
@@ -65,10 +66,29 @@ sca_count_kernel(const uint8_t* __restrict__ mask, int B, int Ncam, int Nq, int 
     }
 }
 
+// Exclusive prefix of the per-chunk counts of one (batch, camera), in place,
+// and the camera's total into count[bc]: one warp per (batch, camera), so the
+// scatter pass reads one base per chunk instead of summing earlier chunks.
+__global__ void __launch_bounds__(32)
+sca_chunk_scan_kernel(int32_t* __restrict__ chunk_counts, int nchunks, int32_t* __restrict__ count)
+{
+    const int bc = blockIdx.x, lane = threadIdx.x;
+    int32_t* cc = chunk_counts + (int64_t)bc * nchunks;
+    int run = 0;
+    for (int base = 0; base < nchunks; base += 32) {
+        const int i = base + lane;
+        const int v = i < nchunks ? cc[i] : 0;
+        const int incl = warp_inclusive_scan(v, lane);
+        if (i < nchunks) cc[i] = run + incl - v;
+        run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) count[bc] = run;
+}
+
 __global__ void __launch_bounds__(kCompactChunk)
 sca_scatter_kernel(const uint8_t* __restrict__ mask, int B, int Ncam, int Nq, int R, int nchunks,
-                   const int32_t* __restrict__ chunk_counts, int32_t* __restrict__ idx,
-                   int32_t* __restrict__ count, int32_t* __restrict__ pos)
+                   const int32_t* __restrict__ chunk_base, const int32_t* __restrict__ count,
+                   int32_t* __restrict__ idx, int32_t* __restrict__ pos)
 {
     __shared__ int s_base[kMaxCameras], s_total[kMaxCameras];
     __shared__ int s_wpre[kMaxCameras][32];
@@ -78,21 +98,10 @@ sca_scatter_kernel(const uint8_t* __restrict__ mask, int B, int Ncam, int Nq, in
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     // seeing queries of camera `warp` in earlier chunks, and in all chunks
-    if (warp < Ncam) {
-        const int32_t* cc = chunk_counts + ((int64_t)b * Ncam + warp) * nchunks;
-        int before = 0, all = 0;
-        for (int i = lane; i < nchunks; i += 32) {
-            const int v = cc[i];
-            all += v;
-            if (i < chunk) before += v;
-        }
-        before = warp_sum_int(before);
-        all = warp_sum_int(all);
-        if (lane == 0) {
-            s_base[warp] = before;
-            s_total[warp] = all;
-            if (chunk == 0) count[(int64_t)b * Ncam + warp] = all;
-        }
+    if (warp < Ncam && lane == 0) {
+        const int64_t bc = (int64_t)b * Ncam + warp;
+        s_base[warp] = chunk_base[bc * nchunks + chunk];
+        s_total[warp] = count[bc];
     }
     uint32_t hitbits = 0;
     for (int c = 0; c < Ncam; ++c) {
@@ -134,8 +143,9 @@ cudaError_t launch_sca_compact(const uint8_t* mask, int B, int Ncam, int Nq, int
     const dim3 grid(nchunks, B);
     sca_count_kernel<<<grid, kCompactChunk, 0, s>>>(mask, B, Ncam, Nq, R, nchunks, hits,
                                                     chunk_counts);
+    sca_chunk_scan_kernel<<<B * Ncam, 32, 0, s>>>(chunk_counts, nchunks, count);
     sca_scatter_kernel<<<grid, kCompactChunk, 0, s>>>(mask, B, Ncam, Nq, R, nchunks,
-                                                      chunk_counts, idx, count, pos);
+                                                      chunk_counts, count, idx, pos);
     return cudaGetLastError();
 }
 
@@ -159,7 +169,7 @@ sca_gather_kernel(const VT* __restrict__ value, const float* __restrict__ off,
     __shared__ int s_prefix[kMaxBatchCameras + 1];
     const int nbc = B * Ncam;
     stage_levels(s_lv, levels);
-    stage_row_prefix(count, nbc, s_prefix);
+    stage_row_prefix(count, nbc, Nq, s_prefix);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     LaneSamples<NC> ls;
@@ -276,10 +286,16 @@ static cudaError_t launch_gather_t(const Problem& p, const float* ref_cam, const
     return cudaGetLastError();
 }
 
+#ifndef MSDA_GATHER_QUAD
+#define MSDA_GATHER_QUAD 1  // rows of <= 32 samples take the four-lane gather
+#endif
+
 cudaError_t launch_sca_gather(const Problem& p, const float* ref_cam, const float* off,
                               const float* logits, const int32_t* idx, const int32_t* count,
                               float* out_rb, cudaStream_t s)
 {
+    if (MSDA_GATHER_QUAD && sca_gather_quad_fits(p))
+        return launch_sca_gather_quad(p, ref_cam, off, logits, idx, count, out_rb, s);
     if (!p.bf16) return launch_gather_t<float, 1>(p, ref_cam, off, logits, idx, count, out_rb, s);
     if (p.H % 2 == 0)
         return launch_gather_t<__nv_bfloat16, 2>(p, ref_cam, off, logits, idx, count, out_rb, s);

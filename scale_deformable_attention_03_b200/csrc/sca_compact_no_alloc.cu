@@ -9,6 +9,7 @@
 // running, because cudaMalloc can block and cudaFree synchronises the device.
 // This entry point keeps the scratch in a fixed array that the library itself
 // owns, so the caller passes only its inputs and outputs.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdio>
@@ -27,10 +28,51 @@ static __device__ __align__(256) int32_t g_chunk_counts[MSDA_NO_ALLOC_COUNT_SLOT
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mutex;
-void* g_address[kMaxDevices] = {nullptr};  // device address of g_chunk_counts, per device
 
-// The array's address on the current device, looked up the first time this
-// device calls in (with the device current) and remembered afterwards.
+// The array's device address is a property of the CUDA context that loaded
+// the module, not of the device ordinal: after cudaDeviceReset, or with
+// another context current, the old address is stale.  So each remembered
+// address carries the unique id of the context it was looked up in
+// (cuCtxGetId), and a lookup in any other context asks again.
+struct Remembered {
+    unsigned long long ctx_id;
+    void* address;
+};
+Remembered g_remembered[kMaxDevices] = {};
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique id of the current context; 0 when there is none yet or the driver
+// entry points are unavailable (then nothing is remembered).
+unsigned long long current_context_id()
+{
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static bool looked_up = false;
+    if (!looked_up) {
+        cudaDriverEntryPointQueryResult q1, q2;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", reinterpret_cast<void**>(&get_current),
+                                    cudaEnableDefault, &q1) != cudaSuccess ||
+            q1 != cudaDriverEntryPointSuccess)
+            get_current = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", reinterpret_cast<void**>(&get_id),
+                                    cudaEnableDefault, &q2) != cudaSuccess ||
+            q2 != cudaDriverEntryPointSuccess)
+            get_id = nullptr;
+        looked_up = true;
+    }
+    if (get_current == nullptr || get_id == nullptr) return 0;
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+    if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
+// The array's address in the current context of the current device: looked
+// up (cudaGetSymbolAddress, with that device current) the first time a
+// context calls in, and remembered for that context afterwards.
 cudaError_t chunk_counts_address(void** out)
 {
     int dev = 0;
@@ -38,13 +80,18 @@ cudaError_t chunk_counts_address(void** out)
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(g_mutex);
-    if (g_address[dev] == nullptr) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_chunk_counts);
-        if (e != cudaSuccess) return e;
-        g_address[dev] = p;
+    const unsigned long long id = current_context_id();
+    Remembered& r = g_remembered[dev];
+    if (id != 0 && r.ctx_id == id && r.address != nullptr) {
+        *out = r.address;
+        return cudaSuccess;
     }
-    *out = g_address[dev];
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_chunk_counts);  // also creates the context if needed
+    if (e != cudaSuccess) return e;
+    r.ctx_id = current_context_id();
+    r.address = r.ctx_id != 0 ? p : nullptr;
+    *out = p;
     return cudaSuccess;
 }
 

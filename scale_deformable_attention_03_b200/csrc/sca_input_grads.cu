@@ -7,8 +7,11 @@
 //   grad_offsets[q, h, l, k]  = sum_c grad_loc_rb[c, pos_c(q), h, l, k] / (W_l, H_l)
 //   grad_logits[q, h, :]      = alpha * (G - <alpha, G>),  G = sum_c grad_attn_rb[...]
 //   grad_ref_cam[c, q, m]     = sum over (h, l, k) with k mod R = m of grad_loc_rb
-// The long sums (the reference points' H*L*P/R terms, <alpha, G>) are formed
-// in double: their terms may cancel.
+// The long sums (the reference points' H*L*P/R terms, <alpha, G>) and the
+// camera sums of the offsets are formed in double: their terms may cancel.
+// When the row kernels provide the fp32 rounding residuals of the location
+// gradients (grad_loc_lo_rb), each term enters the sums as hi + lo, so the
+// chain keeps the double accuracy of the precise location gradients.
 #include <cuda_runtime.h>
 
 #include "msda.h"
@@ -39,6 +42,7 @@ template <int NC, bool REF>
 __global__ void __launch_bounds__(kIgWarps * 32)
 sca_offset_logit_grads_kernel(const float* __restrict__ logits, const int32_t* __restrict__ pos,
                               const float* __restrict__ grad_loc_rb,
+                              const float* __restrict__ grad_loc_lo_rb,
                               const float* __restrict__ grad_attn_rb, int B, int Ncam, int Nq,
                               int H, int L, int P, int R, Levels levels,
                               float* __restrict__ grad_off, float* __restrict__ grad_logits,
@@ -74,11 +78,15 @@ sca_offset_logit_grads_kernel(const float* __restrict__ logits, const int32_t* _
     }
     for (int h0 = 0; h0 < H; h0 += kIgHeads) {
         const int nh = min(kIgHeads, H - h0);
-        float G[kIgHeads][NC], gx[kIgHeads][NC], gy[kIgHeads][NC];
+        float G[kIgHeads][NC];
+        double gx[kIgHeads][NC], gy[kIgHeads][NC];
 #pragma unroll
         for (int hh = 0; hh < kIgHeads; ++hh)
 #pragma unroll
-            for (int c = 0; c < NC; ++c) G[hh][c] = gx[hh][c] = gy[hh][c] = 0.f;
+            for (int c = 0; c < NC; ++c) {
+                G[hh][c] = 0.f;
+                gx[hh][c] = gy[hh][c] = 0.0;
+            }
         unsigned cams = seen;
         while (cams) {
             const int cam = __ffs(cams) - 1;  // ascending camera order
@@ -95,11 +103,17 @@ sca_offset_logit_grads_kernel(const float* __restrict__ logits, const int32_t* _
                         G[hh][c] += __ldcs(grad_attn_rb + r + hh * n + j);
                         const float2 v =
                             __ldcs(reinterpret_cast<const float2*>(grad_loc_rb) + r + hh * n + j);
-                        gx[hh][c] += v.x;
-                        gy[hh][c] += v.y;
+                        const float2 lo =
+                            grad_loc_lo_rb ? __ldcs(reinterpret_cast<const float2*>(grad_loc_lo_rb) +
+                                                    r + hh * n + j)
+                                           : make_float2(0.f, 0.f);
+                        const double vx = (double)v.x + (double)lo.x;
+                        const double vy = (double)v.y + (double)lo.y;
+                        gx[hh][c] += vx;
+                        gy[hh][c] += vy;
                         if (REF) {
-                            rx += v.x;
-                            ry += v.y;
+                            rx += vx;
+                            ry += vy;
                         }
                     }
                 }
@@ -151,7 +165,8 @@ sca_offset_logit_grads_kernel(const float* __restrict__ logits, const int32_t* _
                 if (in[c]) {
                     grad_logits[o + j] = (float)((double)a[hh][c] * ((double)G[hh][c] - dot));
                     reinterpret_cast<float2*>(grad_off)[o + j] =
-                        make_float2(gx[hh][c] / wl[c], gy[hh][c] / hl[c]);
+                        make_float2((float)(gx[hh][c] / (double)wl[c]),
+                                    (float)(gy[hh][c] / (double)hl[c]));
                 }
             }
         }
@@ -176,6 +191,7 @@ __global__ void __launch_bounds__(kIgWarps * 32)
 sca_offset_logit_grads_group_kernel(const float* __restrict__ logits,
                                     const int32_t* __restrict__ pos,
                                     const float* __restrict__ grad_loc_rb,
+                                    const float* __restrict__ grad_loc_lo_rb,
                                     const float* __restrict__ grad_attn_rb, int B, int Ncam,
                                     int Nq, int H, int L, int P, int R, Levels levels,
                                     float* __restrict__ grad_off, float* __restrict__ grad_logits,
@@ -207,22 +223,28 @@ sca_offset_logit_grads_group_kernel(const float* __restrict__ logits,
     for (int h0 = 0; h0 < H; h0 += G) {
         const bool in = kin && h0 + s < H;
         const int64_t e = (int64_t)(h0 + s) * n + k;  // element within the row
-        float Gs = 0.f, gx = 0.f, gy = 0.f;
+        float Gs = 0.f;
+        double gx = 0.0, gy = 0.0;
         unsigned cams = seen;
         while (cams) {
             const int cam = __ffs(cams) - 1;  // ascending camera order
             cams &= cams - 1;
             const int row = __shfl_sync(0xffffffffu, p, cam);
             const int64_t r = (((int64_t)b * Ncam + cam) * Nq + row) * S;
-            float2 v = make_float2(0.f, 0.f);
+            double vx = 0.0, vy = 0.0;
             if (in) {
                 Gs += __ldcs(grad_attn_rb + r + e);
-                v = __ldcs(reinterpret_cast<const float2*>(grad_loc_rb) + r + e);
-                gx += v.x;
-                gy += v.y;
+                const float2 v = __ldcs(reinterpret_cast<const float2*>(grad_loc_rb) + r + e);
+                const float2 lo = grad_loc_lo_rb
+                                      ? __ldcs(reinterpret_cast<const float2*>(grad_loc_lo_rb) + r + e)
+                                      : make_float2(0.f, 0.f);
+                vx = (double)v.x + (double)lo.x;
+                vy = (double)v.y + (double)lo.y;
+                gx += vx;
+                gy += vy;
             }
             if (REF) {
-                double rx = v.x, ry = v.y;
+                double rx = vx, ry = vy;
                 for (int o = 16; o >= R; o >>= 1) {
                     rx += __shfl_xor_sync(0xffffffffu, rx, o);
                     ry += __shfl_xor_sync(0xffffffffu, ry, o);
@@ -242,7 +264,8 @@ sca_offset_logit_grads_group_kernel(const float* __restrict__ logits,
         const double dot = segment_sum_f64((double)alpha * (double)Gs, npad);
         if (in) {
             grad_logits[bq * S + e] = (float)((double)alpha * ((double)Gs - dot));
-            reinterpret_cast<float2*>(grad_off)[bq * S + e] = make_float2(gx / wl, gy / hl);
+            reinterpret_cast<float2*>(grad_off)[bq * S + e] =
+                make_float2((float)(gx / (double)wl), (float)(gy / (double)hl));
         }
     }
 }
@@ -251,8 +274,8 @@ sca_offset_logit_grads_group_kernel(const float* __restrict__ logits,
 // summed per anchor m = k mod R (zero when the camera does not see the query).
 __global__ void __launch_bounds__(kIgWarps * 32)
 sca_reference_grads_kernel(const int32_t* __restrict__ pos, const float* __restrict__ grad_loc_rb,
-                           int B, int Ncam, int Nq, int S, int P, int R,
-                           float* __restrict__ grad_ref_cam)
+                           const float* __restrict__ grad_loc_lo_rb, int B, int Ncam, int Nq,
+                           int S, int P, int R, float* __restrict__ grad_ref_cam)
 {
     const int lane = threadIdx.x & 31;
     const int64_t cbq = (int64_t)blockIdx.x * kIgWarps + (threadIdx.x >> 5);  // (c * B + b) * Nq + q
@@ -266,16 +289,19 @@ sca_reference_grads_kernel(const int32_t* __restrict__ pos, const float* __restr
         if (lane < 2 * R) out[lane] = 0.f;
         return;
     }
-    const float2* g = reinterpret_cast<const float2*>(grad_loc_rb) +
-                      (((int64_t)b * Ncam + c) * Nq + p) * S;
+    const int64_t row = (((int64_t)b * Ncam + c) * Nq + p) * S;
+    const float2* g = reinterpret_cast<const float2*>(grad_loc_rb) + row;
+    const float2* glo =
+        grad_loc_lo_rb ? reinterpret_cast<const float2*>(grad_loc_lo_rb) + row : nullptr;
     if (32 % R == 0) {
         // sample e has anchor (e mod P) mod R = e mod R (R divides P, which
         // divides L*P): lane + 32 i has the anchor lane mod R for every i
         double ax = 0.0, ay = 0.0;
         for (int e = lane; e < S; e += 32) {
             const float2 v = __ldcs(g + e);
-            ax += v.x;
-            ay += v.y;
+            const float2 lo = glo ? __ldcs(glo + e) : make_float2(0.f, 0.f);
+            ax += (double)v.x + (double)lo.x;
+            ay += (double)v.y + (double)lo.y;
         }
         for (int o = 16; o >= R; o >>= 1) {
             ax += __shfl_xor_sync(0xffffffffu, ax, o);
@@ -292,12 +318,13 @@ sca_reference_grads_kernel(const int32_t* __restrict__ pos, const float* __restr
     for (int m = 0; m < MSDA_MAX_POINTS; ++m) sx[m] = sy[m] = 0.0;
     for (int e = lane; e < S; e += 32) {
         const float2 v = __ldcs(g + e);
+        const float2 lo = glo ? __ldcs(glo + e) : make_float2(0.f, 0.f);
         const int m = (e % P) % R;
 #pragma unroll
         for (int mm = 0; mm < MSDA_MAX_POINTS; ++mm)
             if (mm == m) {
-                sx[mm] += v.x;
-                sy[mm] += v.y;
+                sx[mm] += (double)v.x + (double)lo.x;
+                sy[mm] += (double)v.y + (double)lo.y;
             }
     }
 #pragma unroll
@@ -318,7 +345,7 @@ cudaError_t launch_sca_input_grads(const float* logits, const int32_t* pos,
                                    const float* grad_loc_rb, const float* grad_attn_rb, int B,
                                    int Ncam, int Nq, int H, int L, int P, int R, const Levels& lv,
                                    float* grad_off, float* grad_logits, float* grad_ref_cam,
-                                   cudaStream_t s)
+                                   cudaStream_t s, const float* grad_loc_lo_rb)
 {
     const int64_t rows = (int64_t)B * Nq;
     if (rows == 0) return cudaSuccess;
@@ -334,11 +361,13 @@ cudaError_t launch_sca_input_grads(const float* logits, const int32_t* pos,
     case NPLV:                                                                                   \
         if (fused)                                                                               \
             sca_offset_logit_grads_group_kernel<NPLV, true><<<grid, kIgWarps * 32, 0, s>>>(      \
-                logits, pos, grad_loc_rb, grad_attn_rb, B, Ncam, Nq, H, L, P, R, lv, grad_off,   \
+                logits, pos, grad_loc_rb, grad_loc_lo_rb, grad_attn_rb, B, Ncam, Nq, H, L, P, R, \
+                lv, grad_off,                                                                    \
                 grad_logits, grad_ref_cam);                                                      \
         else                                                                                     \
             sca_offset_logit_grads_group_kernel<NPLV, false><<<grid, kIgWarps * 32, 0, s>>>(     \
-                logits, pos, grad_loc_rb, grad_attn_rb, B, Ncam, Nq, H, L, P, R, lv, grad_off,   \
+                logits, pos, grad_loc_rb, grad_loc_lo_rb, grad_attn_rb, B, Ncam, Nq, H, L, P, R, \
+                lv, grad_off,                                                                    \
                 grad_logits, grad_ref_cam);                                                      \
         break;
         switch (npl) {
@@ -353,11 +382,13 @@ cudaError_t launch_sca_input_grads(const float* logits, const int32_t* pos,
     case NCV:                                                                                    \
         if (fused)                                                                               \
             sca_offset_logit_grads_kernel<NCV, true><<<grid, kIgWarps * 32, 0, s>>>(             \
-                logits, pos, grad_loc_rb, grad_attn_rb, B, Ncam, Nq, H, L, P, R, lv, grad_off,   \
+                logits, pos, grad_loc_rb, grad_loc_lo_rb, grad_attn_rb, B, Ncam, Nq, H, L, P, R, \
+                lv, grad_off,                                                                    \
                 grad_logits, grad_ref_cam);                                                      \
         else                                                                                     \
             sca_offset_logit_grads_kernel<NCV, false><<<grid, kIgWarps * 32, 0, s>>>(            \
-                logits, pos, grad_loc_rb, grad_attn_rb, B, Ncam, Nq, H, L, P, R, lv, grad_off,   \
+                logits, pos, grad_loc_rb, grad_loc_lo_rb, grad_attn_rb, B, Ncam, Nq, H, L, P, R, \
+                lv, grad_off,                                                                    \
                 grad_logits, grad_ref_cam);                                                      \
         break;
         switch (nc) {
@@ -372,7 +403,8 @@ cudaError_t launch_sca_input_grads(const float* logits, const int32_t* pos,
     if (fused) return cudaGetLastError();
     const int64_t crows = (int64_t)Ncam * B * Nq;
     sca_reference_grads_kernel<<<(unsigned)((crows + kIgWarps - 1) / kIgWarps), kIgWarps * 32, 0,
-                                 s>>>(pos, grad_loc_rb, B, Ncam, Nq, H * L * P, P, R, grad_ref_cam);
+                                 s>>>(pos, grad_loc_rb, grad_loc_lo_rb, B, Ncam, Nq, H * L * P, P,
+                                      R, grad_ref_cam);
     return cudaGetLastError();
 }
 

@@ -65,7 +65,8 @@ def test_msda_backward_random(case, bf16):
 
 
 def test_msda_backward_workload2():
-    w = inputs.workload2(max_queries=6000)
+    """The Deformable-DETR encoder at full size (all 19 947 queries)."""
+    w = inputs.workload2()
     loc, weights = oracle.fused_locations(w.spatial_shapes, w.reference_points,
                                           w.sampling_offsets, w.attention_logits)
     loc, weights = loc.astype(np.float32), weights.astype(np.float32)
@@ -79,6 +80,25 @@ def test_msda_backward_workload2():
     assert_close(gw, rw, False, "grad_attention_weights")
     assert_close(gl, rl, False, "grad_sampling_locations")
     assert_close(gv, rv, False, "grad_value")
+
+
+def test_msda_backward_tsa_queues_full_size():
+    """The two 200x200 TSA queues as a plain MSDA batch of two (workload 4),
+    locations and weights from the oracle's fused location step."""
+    w = inputs.workload4()
+    loc, weights = oracle.fused_locations(w.spatial_shapes, w.reference_points,
+                                          w.sampling_offsets, w.attention_logits)
+    loc, weights = loc.astype(np.float32), weights.astype(np.float32)
+    gout = np.random.Generator(np.random.PCG64(6)).standard_normal(
+        (w.B, w.Nq, w.H * 32)).astype(np.float32)
+    gv, gl, gw = msda.msda_backward(dev(w.value), w.spatial_shapes, w.level_start_index,
+                                    dev(loc), dev(weights), dev(gout))
+    torch.cuda.synchronize()
+    rv, rl, rw = oracle.msda_backward(w.value, w.spatial_shapes, w.level_start_index, loc,
+                                      weights, gout)
+    assert_close(gw, rw, False, "tsa queues grad_attention_weights")
+    assert_close(gl, rl, False, "tsa queues grad_sampling_locations")
+    assert_close(gv, rv, False, "tsa queues grad_value")
 
 
 def _sca_bwd(w, bf16):
@@ -103,6 +123,62 @@ def test_sca_backward_random(seed, B, Ncam, bev, shapes, H, P, R):
     assert_close(gw, rw, False, "grad_attention_weights_rb")
     assert_close(gl, rl, False, "grad_sampling_locations_rb")
     assert_close(gv, rv, False, "grad_value")
+
+
+def test_sca_backward_workload3_full_size():
+    """The BEVFormer-base SCA backward with fp32 value (B = 1) at full size:
+    the rebatched gradients and grad_value at the fp32 bound."""
+    w = inputs.workload3(seed=1003, with_grad=True)
+    (gv, gl, gw), (rv, rl, rw) = _sca_bwd(w, False)
+    assert_close(gw, rw, False, "workload 3 grad_attention_weights_rb")
+    assert_close(gl, rl, False, "workload 3 grad_sampling_locations_rb")
+    assert_close(gv, rv, False, "workload 3 grad_value")
+
+
+def _full_both(w, bf16):
+    """sca_backward_full on the GPU; the oracle's derivative and chain."""
+    got = msda.sca_backward_full(value_tensor(w, bf16), w.spatial_shapes, w.level_start_index,
+                                 dev(w.reference_points), dev(w.bev_mask),
+                                 dev(w.sampling_offsets), dev(w.attention_logits),
+                                 dev(w.grad_out))
+    torch.cuda.synchronize()
+    rv, rl, rw = oracle.sca_backward(w.value, w.spatial_shapes, w.level_start_index,
+                                     w.reference_points, w.bev_mask, w.sampling_offsets,
+                                     w.attention_logits, w.grad_out)
+    want = (rv,) + tuple(oracle.sca_backward_inputs(w.spatial_shapes, w.bev_mask,
+                                                    w.attention_logits, rl, rw))
+    return got, want
+
+
+FULL_NAMES = ("grad_value", "grad_sampling_offsets", "grad_attention_logits",
+              "grad_reference_points_cam")
+
+
+@pytest.mark.parametrize("seed,B,Ncam,bev,shapes,H,P,R", [
+    (51, 2, 3, (7, 9), [(9, 13), (4, 7)], 2, 4, 2),
+    (52, 1, 6, (30, 40), [(16, 20), (8, 10), (4, 5), (2, 3)], 8, 8, 4),
+    (53, 2, 2, (5, 13), [(6, 7)] * 3, 1, 12, 3),       # R = 3: separate reference kernel
+    (54, 1, 4, (9, 11), [(8, 9), (4, 5)], 12, 4, 2),   # 12 heads: two head chunks
+    (55, 2, 3, (6, 8), [(10, 12)], 8, 4, 4),           # rows of 4 samples: group chain
+    (56, 1, 2, (4, 6), [(5, 6)] * 5, 2, 16, 4),        # 80 samples: three chunks
+])
+@pytest.mark.parametrize("rho", ["uniform", "coherent"])
+def test_sca_backward_full(seed, B, Ncam, bev, shapes, H, P, R, rho):
+    """The whole SCA backward to its inputs, at the fp32 element bound."""
+    w = inputs.workload3(seed=seed, B=B, Ncam=Ncam, bev_h=bev[0], bev_w=bev[1], shapes=shapes,
+                         H=H, P=P, R=R, rho=rho, same_mask=False, with_grad=True)
+    got, want = _full_both(w, False)
+    for g, r, name in zip(got, want, FULL_NAMES):
+        assert_close(g, r, False, name)
+
+
+def test_sca_backward_full_workload3_full_size():
+    """BEVFormer-base (fp32 value, B = 1): value, offset, logit and
+    reference-point gradients at the fp32 element bound."""
+    w = inputs.workload3(seed=1003, with_grad=True)
+    got, want = _full_both(w, False)
+    for g, r, name in zip(got, want, FULL_NAMES):
+        assert_close(g, r, False, "workload 3 " + name)
 
 
 def test_workload5_training_step_full_size():
@@ -161,27 +237,6 @@ def test_sca_backward_inputs(seed, B, Ncam, bev, shapes, H, P, R, rho):
     assert_close(g_ref, r_ref, False, "grad_reference_points_cam")
 
 
-def test_sca_backward_chain_on_the_gpu():
-    """The GPU's own rebatched gradients through sca_backward_inputs stay
-    within the bf16-path bound of the oracle's chain (the fp32 errors of the
-    first stage are summed over up to H*L*P/R terms by the second)."""
-    w = inputs.workload3(seed=44, bev_h=20, bev_w=25, with_grad=True)
-    idx, count, pos, hits = msda.sca_compact(dev(w.bev_mask))
-    _, gl, gw = msda.sca_rebatched_backward(
-        dev(w.value), w.spatial_shapes, w.level_start_index, dev(w.reference_points),
-        dev(w.sampling_offsets), dev(w.attention_logits), dev(w.grad_out), idx, count, hits)
-    g = msda.sca_backward_inputs(w.spatial_shapes, w.level_start_index, dev(w.attention_logits),
-                                 pos, gl, gw, w.Ncam, w.R)
-    torch.cuda.synchronize()
-    _, rl, rw = oracle.sca_backward(w.value, w.spatial_shapes, w.level_start_index,
-                                    w.reference_points, w.bev_mask, w.sampling_offsets,
-                                    w.attention_logits, w.grad_out)
-    r = oracle.sca_backward_inputs(w.spatial_shapes, w.bev_mask, w.attention_logits, rl, rw)
-    for got, want, name in zip(g, r, ("offsets", "logits", "reference points")):
-        err = np.abs(got.cpu().numpy().astype(np.float64) - want)
-        assert err.max() <= 1e-4 * (1.0 + np.abs(want).max()), (name, err.max())
-
-
 def test_sca_backward_inputs_workload5():
     w = inputs.workload5()
     mask = dev(w.bev_mask)
@@ -198,16 +253,10 @@ def test_sca_backward_inputs_workload5():
     assert_close(g_off, r_off, False, "workload 5 grad_sampling_offsets")
     assert_close(g_lg, r_lg, False, "workload 5 grad_attention_logits")
     assert_close(g_ref, r_ref, False, "workload 5 grad_reference_points_cam")
-    # the whole GPU chain (bf16 value): the bf16-path bound
-    g_off, g_lg, g_ref = msda.sca_backward_inputs(w.spatial_shapes, w.level_start_index,
-                                                  dev(w.attention_logits), pos, gl, gw, w.Ncam,
-                                                  w.R)
-    torch.cuda.synchronize()
-    r_off, r_lg, r_ref = oracle.sca_backward_inputs(w.spatial_shapes, w.bev_mask,
-                                                    w.attention_logits, rl, rw)
-    assert_close(g_off, r_off, True, "workload 5 chain grad_sampling_offsets")
-    assert_close(g_lg, r_lg, True, "workload 5 chain grad_attention_logits")
-    assert_close(g_ref, r_ref, True, "workload 5 chain grad_reference_points_cam")
+    # the whole GPU chain in one call (bf16 value): the bf16-path bound
+    got, want = _full_both(w, True)
+    for g, r, name in zip(got, want, FULL_NAMES):
+        assert_close(g, r, True, "workload 5 sca_backward_full " + name)
 
 
 @pytest.mark.parametrize("case", CASES, ids=[f"case{c[0]}" for c in CASES])

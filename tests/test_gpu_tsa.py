@@ -125,13 +125,6 @@ def test_tsa_forward_empty():
     assert out.shape == (0, 16, 256)
 
 
-def _chain_close(got, want, what):
-    """The chain from the kernel's own fp32 location and weight gradients: sums
-    of up to H*L*P terms that may cancel, bounded relative to the largest."""
-    err = np.abs(got.cpu().numpy().astype(np.float64) - want)
-    assert err.max() <= 1e-4 * (1.0 + np.abs(want).max()), (what, err.max())
-
-
 @pytest.mark.parametrize("case", CASES, ids=[f"case{c[0]}" for c in CASES])
 @pytest.mark.parametrize("bf16", [False, True])
 def test_tsa_backward(case, bf16):
@@ -146,8 +139,8 @@ def test_tsa_backward(case, bf16):
     rv, r_off, r_lg, r_ref = oracle.tsa_backward(value, s, starts, ref, off, logits, T, go)
     assert_close(gv, rv, False, "tsa grad_value")
     assert_close(g_off, r_off, False, "tsa grad_sampling_offsets")
-    _chain_close(g_lg, r_lg, "tsa grad_attention_logits")
-    _chain_close(g_ref, r_ref, "tsa grad_reference_points")
+    assert_close(g_lg, r_lg, False, "tsa grad_attention_logits")
+    assert_close(g_ref, r_ref, False, "tsa grad_reference_points")
 
 
 def test_tsa_backward_bevformer_base_full_size():
@@ -166,5 +159,5 @@ def test_tsa_backward_bevformer_base_full_size():
                                                  go)
     assert_close(gv, rv, False, "tsa 200x200 grad_value")
     assert_close(g_off, r_off, False, "tsa 200x200 grad_sampling_offsets")
-    _chain_close(g_lg, r_lg, "tsa 200x200 grad_attention_logits")
-    _chain_close(g_ref, r_ref, "tsa 200x200 grad_reference_points")
+    assert_close(g_lg, r_lg, False, "tsa 200x200 grad_attention_logits")
+    assert_close(g_ref, r_ref, False, "tsa 200x200 grad_reference_points")
