@@ -27,7 +27,6 @@ import argparse
 import hashlib
 import json
 import os
-import re
 import sys
 import time
 
@@ -41,9 +40,10 @@ UNIT = "Gsamples/s"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 L2_FLUSH_BYTES = 256 << 20
-PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "sca_gather_bevformer_base.md")
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "traffic.json")
 KERNEL_SOURCES = ("scale_deformable_attention_03_b200/csrc/msda_device.cuh",
-                  "scale_deformable_attention_03_b200/csrc/sca.cu")
+                  "scale_deformable_attention_03_b200/csrc/sca.cu",
+                  "scale_deformable_attention_03_b200/csrc/sca_gather_quad.cu")
 
 
 def parse_args(argv=None):
@@ -100,6 +100,11 @@ def algorithmic_bytes(w, rows, hit_queries, value_elem):
     step = (value + w.B * w.Nq * offsets_logits_per_query + w.reference_points.nbytes
             + w.bev_mask.nbytes + w.B * w.Nq * out_row)
     return {"gather": int(gather), "step": int(step)}
+
+
+def gather_kernel_name(w):
+    """The rebatched-gather kernel sca_rebatched_forward launches here."""
+    return ("sca_gather_quad_kernel" if w.L * w.P <= 32 else "sca_gather_kernel")
 
 
 def aggregate(local_ms_total, local_samples, world):
@@ -177,17 +182,30 @@ def kernel_source_digest():
 
 
 def recorded_traffic(value_dtype):
-    """DRAM bytes per gather launch from the committed ncu summary, when it
-    was taken on the current kernel sources; None otherwise."""
+    """DRAM bytes per gather launch from the committed ncu record
+    (profiles/traffic.json), when it was taken on the current kernel sources;
+    None otherwise."""
     try:
-        text = open(PROFILE_TRAFFIC).read()
+        with open(TRAFFIC_RECORD) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if rec.get("kernel_sources_sha256_16") != kernel_source_digest():
+        return None
+    v = rec.get("dram_bytes_per_launch", {}).get(value_dtype)
+    return int(v) if v is not None else None
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
     except OSError:
-        return None
-    m = re.search(r"kernel_sources_sha256_16:\s*([0-9a-f]+)", text)
-    t = re.search(rf"traffic_bytes_per_launch_{value_dtype}:\s*([0-9]+)", text)
-    if not m or not t or m.group(1) != kernel_source_digest():
-        return None
-    return int(t.group(1))
+        pass
+    import platform
+    return platform.processor() or "unknown"
 
 
 class ClockSampler:
@@ -260,32 +278,58 @@ class ClockSampler:
 # CPU baseline: the oracle as it stands, one host core
 # --------------------------------------------------------------------------
 
-def oracle_step(w, n_queries):
-    """One oracle SCA forward over the first n_queries BEV queries of the
-    workload (all cameras, full value maps). Returns sampled points."""
+def oracle_step(w, q0, q1, value64=None):
+    """One oracle SCA forward over BEV queries q0 .. q1 - 1 of the workload
+    (all cameras, full value maps). Returns sampled points."""
     import oracle
-    q = slice(0, n_queries)
-    out = oracle.sca_forward(w.value, w.spatial_shapes, w.level_start_index,
+    q = slice(q0, q1)
+    out = oracle.sca_forward(w.value if value64 is None else value64, w.spatial_shapes,
+                             w.level_start_index,
                              np.ascontiguousarray(w.reference_points[:, :, q]),
                              np.ascontiguousarray(w.bev_mask[:, :, q]),
                              np.ascontiguousarray(w.sampling_offsets[:, q]),
                              np.ascontiguousarray(w.attention_logits[:, q]))
-    assert out.shape[1] == n_queries
+    assert out.shape[1] == q1 - q0
     rows = int(np.count_nonzero(w.bev_mask[:, :, q].any(-1)))
     return rows * w.H * w.L * w.P
 
 
 def cpu_baseline(w, min_seconds):
+    """The oracle as it stands on the host cores: full workload passes on one
+    core, then passes split into query slices over every core (threads: the
+    C oracle runs without the Python lock).  The value map is widened to
+    double once, outside the timed passes (the oracle's input type)."""
+    import concurrent.futures as cf
+    import oracle
+    oracle.lib()
+    v64 = np.ascontiguousarray(w.value, dtype=np.float64)
     done, samples, t0 = 0, 0, time.perf_counter()
     while True:
-        samples += oracle_step(w, w.Nq)
+        samples += oracle_step(w, 0, w.Nq, v64)
         done += 1
-        el = time.perf_counter() - t0
-        if el >= min_seconds:
+        el1 = time.perf_counter() - t0
+        if el1 >= min_seconds:
             break
-    return {"value": samples / el / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{done} full workload pass(es) of the C oracle (double), "
-                      f"{el:.1f} s on one host core"}
+    one = samples / el1 / 1e9
+    cores = os.cpu_count() or 1
+    step = max(200, (w.Nq // (4 * cores)) // 200 * 200)  # whole BEV rows per slice
+    slices = [(q, min(w.Nq, q + step)) for q in range(0, w.Nq, step)]
+    done_m, samples_m = 0, 0
+    with cf.ThreadPoolExecutor(max_workers=cores) as ex:
+        t0 = time.perf_counter()
+        while True:
+            samples_m += sum(ex.map(lambda s: oracle_step(w, s[0], s[1], v64), slices))
+            done_m += 1
+            elm = time.perf_counter() - t0
+            if elm >= min_seconds / 2:
+                break
+    many = samples_m / elm / 1e9
+    return {"value": many, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "cpu_model": cpu_model(),
+            "sample": f"{done_m} full workload pass(es) of the C oracle (double) split into "
+                      f"{len(slices)} query slices over {cores} threads, {elm:.1f} s",
+            "single_core": {"value": one, "unit": UNIT, "cores": 1,
+                            "sample": f"{done} full workload pass(es) on one core, {el1:.1f} s"}}
 
 
 def run_reference(args):
@@ -297,16 +341,16 @@ def run_reference(args):
     oracle_build.build()
     w = inputs.workload3(seed=rank_seed(0), value_dtype=args.value_dtype, rho=args.rho)
     t0 = time.perf_counter()
-    oracle_step(w, w.Nq)
+    oracle_step(w, 0, w.Nq)
     t_full = time.perf_counter() - t0
     budget = 150.0  # seconds for warm-up + timed steps
     frac = min(1.0, budget / max(1e-9, (args.steps + args.warmup) * t_full))
     nq = max(200, int(w.Nq * frac) // 200 * 200)  # whole BEV rows of 200 cells
     for _ in range(args.warmup):
-        oracle_step(w, nq)
+        oracle_step(w, 0, nq)
     samples, t0 = 0, time.perf_counter()
     for _ in range(args.steps):
-        samples += oracle_step(w, nq)
+        samples += oracle_step(w, 0, nq)
     el = time.perf_counter() - t0
     value = samples / el / 1e9
     sample = (f"first {nq} of {w.Nq} BEV queries per step (all 6 cameras, full value maps), "
@@ -318,7 +362,7 @@ def run_reference(args):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(args),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": sample},
+                         "cpu_model": cpu_model(), "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -329,23 +373,16 @@ def run_reference(args):
 # native arm
 # --------------------------------------------------------------------------
 
-def run_native(args):
+def measure_replica(args, rank, world, barrier):
+    """The device section of one replica: the timed SCA forward steps, the
+    warm-L2 gather, the end-to-end leg through sca_forward with host buffers
+    and (one GPU) the further entry points.  barrier() is called at the same
+    points on every rank.  Returns this rank's local results."""
     import torch
-    import torch.distributed as dist
 
     import scale_deformable_attention_03_b200 as msda
     from scale_deformable_attention_03_b200 import inputs
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world != args.gpus:
-        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
     msda.lib()  # fail loudly before any work when the library is missing
     stream = torch.cuda.current_stream()
 
@@ -390,7 +427,7 @@ def run_native(args):
         msda._check(L.sca_camera_average(P(out_rb), P(pos), P(hits), dims, P(out), sptr),
                     "sca_camera_average")
 
-    launches_per_step = 4  # two compaction kernels, the gather, the average
+    launches_per_step = 5  # three compaction kernels, the gather, the average
     compact()
     torch.cuda.synchronize()
     rows = int(count.sum().item())
@@ -407,8 +444,7 @@ def run_native(args):
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
-    if world > 1:
-        dist.barrier()
+    barrier()
     torch.cuda.synchronize()
     if sampler:
         sampler.start()
@@ -422,8 +458,7 @@ def run_native(args):
         average()
         e[3].record(stream)
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    barrier()
     clocks = sampler.stop() if sampler else None
     # the gather again with a warm L2 (no flush between launches), for reference
     warm_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -438,9 +473,6 @@ def run_native(args):
     gather_ms = [e[1].elapsed_time(e[2]) for e in evs]
     compact_ms = [e[0].elapsed_time(e[1]) for e in evs]
     avg_ms = [e[2].elapsed_time(e[3]) for e in evs]
-    total_ms, total_samples = aggregate(sum(step_ms), samples_per_step * args.steps, world)
-    value_gs = total_samples / (total_ms * 1e-3) / 1e9
-
     # ---- end to end through the one-call C ABI, host buffers ----
     # Every step copies its inputs from pinned host memory, runs sca_forward
     # and copies its result back.  Two device buffer sets let the copies of
@@ -486,8 +518,7 @@ def run_native(args):
     for i in range(2):
         e2e_step(i)
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     copy_s.wait_event(e0)
@@ -497,18 +528,68 @@ def run_native(args):
     stream.wait_stream(copy_s)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms, e2e_samples = aggregate(e0.elapsed_time(e1), samples_per_step * args.e2e_steps, world)
-    e2e_gs = e2e_samples / (e2e_ms * 1e-3) / 1e9
+    res = {"w": w, "bf16": bf16, "step_ms": step_ms, "gather_ms": gather_ms,
+           "compact_ms": compact_ms, "avg_ms": avg_ms, "warm_gather_ms": warm_gather_ms,
+           "samples_per_step": samples_per_step, "rows": rows, "nbytes": nbytes,
+           "e2e_ms": e0.elapsed_time(e1), "h2d": int(h2d), "d2h": int(d2h), "clocks": clocks,
+           "launches_per_step": launches_per_step}
+    if world == 1 and args.rows_iters > 0:
+        tensors = {"value": value, "ref": ref, "mask": mask, "off": off, "logits": logits,
+                   "step_bytes": nbytes["step"], "samples": samples_per_step}
+        peak, _ = measured_hbm_peak()
+        res["next_rows"] = measure_next_rows(args, w, tensors, flush, stream, peak)
+    return res
 
+
+def run_native(args, backend="nccl", replica=measure_replica):
+    """One replica per rank (weak scaling): the device section (`replica`),
+    then the job time (max over ranks of the summed step times) and work (sum
+    over ranks) through the process group; rank 0 prints the JSON line."""
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    if backend == "nccl":
+        import torch
+        torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        kw = {}
+        if backend == "nccl":
+            import torch
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    res = replica(args, rank, world, barrier)
+    step_ms = res["step_ms"]
+    total_ms, total_samples = aggregate(sum(step_ms), res["samples_per_step"] * args.steps, world)
+    value_gs = total_samples / (total_ms * 1e-3) / 1e9
+    e2e_ms, e2e_samples = aggregate(res["e2e_ms"], res["samples_per_step"] * args.e2e_steps, world)
+    e2e_gs = e2e_samples / (e2e_ms * 1e-3) / 1e9
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
         return 0
-
+    w, nbytes = res["w"], res["nbytes"]
+    gather_ms, compact_ms, avg_ms = res["gather_ms"], res["compact_ms"], res["avg_ms"]
+    warm_gather_ms, samples_per_step = res["warm_gather_ms"], res["samples_per_step"]
+    rows, h2d, d2h, clocks = res["rows"], res["h2d"], res["d2h"], res["clocks"]
+    launches_per_step = res["launches_per_step"]
     peak, peak_src = measured_hbm_peak()
     g_ms = float(np.mean(gather_ms))
-    achieved = nbytes["gather"] / (g_ms * 1e-3) / 1e9
+    # the step's algorithmic bytes (value once, every query's offsets and
+    # logits, reference points, mask, output once) over the dominant kernel's
+    # time; the gather's own bytes (with its rebatched rows) beside it
+    achieved = nbytes["step"] / (g_ms * 1e-3) / 1e9
+    achieved_own = nbytes["gather"] / (g_ms * 1e-3) / 1e9
     traffic = recorded_traffic(args.value_dtype)
     step_mean = float(np.mean(step_ms))
     line = {
@@ -518,8 +599,13 @@ def run_native(args):
         "data": "synthetic", "config": workload_config(args),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "sca_gather_kernel", "peak_source": peak_src,
-                     "algorithmic_bytes_per_launch": nbytes["gather"],
+                     "kernel": gather_kernel_name(w), "peak_source": peak_src,
+                     "algorithmic_bytes_per_launch": nbytes["step"],
+                     "algorithmic_bytes_note": "the step's bytes (value, offsets and logits "
+                                               "of every query, reference points, mask, "
+                                               "output), each once",
+                     "gather_own_bytes_per_launch": nbytes["gather"],
+                     "gather_own_frac": achieved_own / peak,
                      "launch_ms": g_ms},
         "step": {"algorithmic_bytes": nbytes["step"],
                  "hbm_gbs": nbytes["step"] / (step_mean * 1e-3) / 1e9,
@@ -539,14 +625,14 @@ def run_native(args):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
-    if world == 1 and args.rows_iters > 0:
-        tensors = {"value": value, "ref": ref, "mask": mask, "off": off, "logits": logits,
-                   "step_bytes": nbytes["step"], "samples": samples_per_step}
-        line["next_rows"] = measure_next_rows(args, w, tensors, flush, stream, peak)
-    if world == 1:
+    if "next_rows" in res:
+        line["next_rows"] = res["next_rows"]
+    if world == 1 and args.cpu_seconds > 0:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     print(json.dumps(line), flush=True)
     return 0
+
+
 
 
 # --------------------------------------------------------------------------
@@ -608,6 +694,31 @@ def measure_next_rows(args, w, tensors, flush, stream, hbm_peak):
     r.update(kernel="sca_query_major_kernel", workload="bevformer-base-sca-forward",
              gsamples_per_s=tensors["samples"] / (ms * 1e-3) / 1e9)
     rows["sca_forward_query_major"] = r
+
+    # the same SCA forward with bf16 value (BEVFormer-base's bf16 variant):
+    # the rebatched step (sca_forward's kernels) and the query-major kernel
+    if not bf16:
+        vb16 = value.to(torch.bfloat16)  # round to nearest even, as the inputs module does
+        step_b16 = tensors["step_bytes"] - w.value.size * 2
+        ws16 = torch.empty(msda.msda_workspace_size(msda.Dims(w.B, w.Ncam, w.Nq, w.Nv, w.H,
+                                                              w.L, w.P, w.R)),
+                           dtype=torch.uint8, device="cuda")
+        ms = timed(lambda: msda.sca_forward(vb16, shapes, starts, ref, mask, off, logits,
+                                            out=out, workspace=ws16))
+        r = hbm(step_b16, ms)
+        r.update(kernel="sca_count + sca_chunk_scan + sca_scatter + "
+                        f"{gather_kernel_name(w)}<bf16> + sca_average",
+                 workload="bevformer-base-sca-forward, bf16 value",
+                 gsamples_per_s=tensors["samples"] / (ms * 1e-3) / 1e9)
+        rows["sca_forward_bf16"] = r
+        ms = timed(lambda: msda.sca_forward_query_major(vb16, shapes, starts, ref, mask, off,
+                                                        logits, out=out))
+        r = hbm(step_b16, ms)
+        r.update(kernel="sca_query_major_kernel<bf16>",
+                 workload="bevformer-base-sca-forward, bf16 value",
+                 gsamples_per_s=tensors["samples"] / (ms * 1e-3) / 1e9)
+        rows["sca_forward_query_major_bf16"] = r
+        del vb16, ws16
 
     # the plain fused MSDA: the Deformable-DETR encoder and the TSA queues as a batch
     for name, wk, kname in (
@@ -827,6 +938,23 @@ def measure_next_rows(args, w, tensors, flush, stream, hbm_peak):
              workload="bevformer-base SCA training step, B=2, bf16 value",
              gsamples_per_s=rows5 * w5.H * w5.L * w5.P / (ms * 1e-3) / 1e9)
     rows["sca_backward_deterministic"] = r
+    # the whole backward to the SCA inputs (precise chain) in one call
+    wsf = torch.empty(int(msda.lib().sca_backward_full_workspace_size(
+        msda.Dims(w5.B, w5.Ncam, w5.Nq, w5.Nv, w5.H, w5.L, w5.P, w5.R))), dtype=torch.uint8,
+        device="cuda")
+    full_out = (g5[0], torch.empty_like(d5["off"]), torch.empty_like(d5["logits"]),
+                torch.empty_like(d5["ref"]))
+    ms = timed(lambda: msda.sca_backward_full(*args5, out=full_out, workspace=wsf),
+               n=max(1, iters // 4))
+    S5 = w5.H * w5.L * w5.P
+    r = hbm(sca_backward_algorithmic_bytes(w5, rows5, hitq5, 2) - rows5 * S5 * 3 * 4
+            + w5.B * w5.Nq * S5 * 3 * 4 + w5.reference_points.nbytes, ms)
+    r.update(kernel="sca_backward_kernel<..., precise> + sca_offset_logit_grads_kernel "
+                    "(+ compaction, zero fill)",
+             workload="bevformer-base SCA training step, B=2, bf16 value",
+             gsamples_per_s=rows5 * S5 / (ms * 1e-3) / 1e9)
+    rows["sca_backward_full"] = r
+    del wsf, full_out
     return rows
 
 
