@@ -268,7 +268,7 @@ def tsa_forward(value, spatial_shapes, level_start_index, reference_points, samp
 
 
 def tsa_backward(value, spatial_shapes, level_start_index, reference_points, sampling_offsets,
-                 attention_logits, num_queues, grad_out, workspace=None, stream=None):
+                 attention_logits, num_queues, grad_out, workspace=None, stream=None, out=None):
     """-> (grad_value [B*T, Nv, H, 32], grad_sampling_offsets [B*T, Nq, H, L, P, 2],
     grad_attention_logits [B*T, Nq, H, L, P], grad_reference_points [B*T, Nq, R, 2])."""
     torch = _torch()
@@ -282,10 +282,14 @@ def tsa_backward(value, spatial_shapes, level_start_index, reference_points, sam
     shapes, starts = _levels(spatial_shapes, level_start_index)
     d = Dims(BT // T, 1, Nq, Nv, H, L, P, R)
     dev = value.device
-    gv = torch.empty(value.shape, device=dev, dtype=torch.float32)
-    g_off = torch.empty(sampling_offsets.shape, device=dev, dtype=torch.float32)
-    g_lg = torch.empty(attention_logits.shape, device=dev, dtype=torch.float32)
-    g_ref = torch.empty(reference_points.shape, device=dev, dtype=torch.float32)
+    if out is not None:
+        gv, g_off, g_lg, g_ref = out
+        _contig(gv, g_off, g_lg, g_ref)
+    else:
+        gv = torch.empty(value.shape, device=dev, dtype=torch.float32)
+        g_off = torch.empty(sampling_offsets.shape, device=dev, dtype=torch.float32)
+        g_lg = torch.empty(attention_logits.shape, device=dev, dtype=torch.float32)
+        g_ref = torch.empty(reference_points.shape, device=dev, dtype=torch.float32)
     workspace = _workspace(int(lib().tsa_backward_workspace_size(d, T)), dev, workspace)
     _check(lib().tsa_backward(_ptr(value), _vdt(value), shapes.ctypes.data_as(_i64p),
                               starts.ctypes.data_as(_i64p), _ptr(reference_points),
@@ -354,19 +358,24 @@ def _workspace(nbytes, device, workspace):
     return workspace
 
 
-def sca_compact(bev_mask, workspace=None, stream=None):
+def sca_compact(bev_mask, workspace=None, stream=None, out=None):
     """bev_mask [Ncam, B, Nq, R] (uint8 / bool) -> (idx [B, Ncam, Nq],
-    count [B, Ncam], pos [B, Ncam, Nq], hits [B, Nq]), int32."""
+    count [B, Ncam], pos [B, Ncam, Nq], hits [B, Nq]), int32; `out` may
+    supply the four tensors."""
     torch = _torch()
     _contig(bev_mask)
     if bev_mask.dtype == torch.bool:
         bev_mask = bev_mask.view(torch.uint8)
     Ncam, B, Nq, R = bev_mask.shape
     dev = bev_mask.device
-    idx = torch.empty((B, Ncam, Nq), dtype=torch.int32, device=dev)
-    count = torch.empty((B, Ncam), dtype=torch.int32, device=dev)
-    pos = torch.empty((B, Ncam, Nq), dtype=torch.int32, device=dev)
-    hits = torch.empty((B, Nq), dtype=torch.int32, device=dev)
+    if out is not None:
+        idx, count, pos, hits = out
+        _contig(idx, count, pos, hits)
+    else:
+        idx = torch.empty((B, Ncam, Nq), dtype=torch.int32, device=dev)
+        count = torch.empty((B, Ncam), dtype=torch.int32, device=dev)
+        pos = torch.empty((B, Ncam, Nq), dtype=torch.int32, device=dev)
+        hits = torch.empty((B, Nq), dtype=torch.int32, device=dev)
     d = Dims(B, Ncam, Nq, 1, 1, 1, 1, R)
     nbytes = sca_compact_workspace_size(d)
     workspace = _workspace(nbytes, dev, workspace)
