@@ -262,6 +262,14 @@ msda_status_t msda_linear_dropout(const void* x, const void* w, const float* bia
  * Reads a device word, so it synchronises with the device. */
 uint32_t msda_linear_timeouts(void);
 
+/* Test hook of the bounded-wait path (no counterpart on the pages): the next
+ * msda_linear launch holds back the first X-tile load of its first CTA.  That
+ * CTA's tensor-core wait then runs out (about two seconds), counts one
+ * timeout (msda_linear_timeouts), raises its stop flag, waits for the copies
+ * it did issue and frees its tensor memory; the other CTAs finish normally.
+ * The output of that one call is incomplete.  Synchronises with the device. */
+msda_status_t msda_linear_test_withhold_load(void);
+
 /* Bytes of device workspace sca_forward / sca_backward need for these
  * sizes: the compaction lists and, for the forward, the rebatched rows
  * (B * Ncam * Nq * H * 32 floats, of which only the seeing rows are used). */

@@ -97,6 +97,7 @@ def lib():
                                           ctypes.c_uint64, _vp]
         L.msda_linear_dropout.restype = ctypes.c_int
         L.msda_linear_timeouts.restype = ctypes.c_uint32
+        L.msda_linear_test_withhold_load.restype = ctypes.c_int
         L.sca_module_workspace_size.argtypes = [Dims, ctypes.c_int]
         L.sca_module_workspace_size.restype = ctypes.c_size_t
         L.sca_module_forward.argtypes = [ctypes.POINTER(ScaModuleParams), _i64p, _i64p, Dims, _vp,

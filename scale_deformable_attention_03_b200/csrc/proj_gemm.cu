@@ -75,6 +75,10 @@ constexpr size_t kSmemC = (size_t)4 * 2 * kCBufBytes;           // 32 KB
 constexpr size_t kSmemBytes = 1024 + kSmemB + kSmemA + kSmemC + sizeof(Ctrl);
 
 __device__ unsigned int g_gemm_timeouts = 0;
+// Test switch of the bounded-wait path (msda_linear_test_withhold_load): when
+// set, CTA 0 of the next launch clears it and holds back its first X-tile
+// load, so that its tensor-core wait runs out.
+__device__ int g_gemm_withhold = 0;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p)
 {
@@ -351,6 +355,9 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
             uint32_t phase = 0, free_phase = 0;
             int issued[kStages];  // parity of each slot's last load, -1 = none
             for (int i = 0; i < kStages; ++i) issued[i] = -1;
+            // the test switch: withhold the first X-tile load (its slot's
+            // barrier is then never completed, and nothing is in flight to it)
+            bool withhold = blockIdx.x == 0 && atomicExch(&g_gemm_withhold, 0) != 0;
             for (int tile = blockIdx.x; tile < ntiles && !ctrl.stop; tile += gridDim.x) {
                 const int m0 = (tile % mt) * kBM, n_tile = tile / mt;
                 if (n_tile != cur_n) {
@@ -373,9 +380,14 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
                         note_timeout(ctrl);
                         break;
                     }
-                    mbar_expect_tx(&ctrl.full[stage], kABlockBytes);
-                    tma_load_2d(sa + stage * kABlockBytes, &map_x, kb * kBK, m0, &ctrl.full[stage]);
-                    issued[stage] = (int)phase;
+                    if (withhold) {
+                        withhold = false;
+                    } else {
+                        mbar_expect_tx(&ctrl.full[stage], kABlockBytes);
+                        tma_load_2d(sa + stage * kABlockBytes, &map_x, kb * kBK, m0,
+                                    &ctrl.full[stage]);
+                        issued[stage] = (int)phase;
+                    }
                     if (++stage == kStages) {
                         stage = 0;
                         phase ^= 1;
@@ -701,4 +713,11 @@ extern "C" uint32_t msda_linear_timeouts(void)
     unsigned int v = 0;
     if (cudaMemcpyFromSymbol(&v, msda::g_gemm_timeouts, sizeof(v)) != cudaSuccess) return 0xFFFFFFFFu;
     return v;
+}
+
+extern "C" msda_status_t msda_linear_test_withhold_load(void)
+{
+    const int one = 1;
+    return msda::api_cuda(cudaMemcpyToSymbol(msda::g_gemm_withhold, &one, sizeof(one)),
+                          "msda_linear_test_withhold_load");
 }

@@ -38,7 +38,7 @@ def test_header_declares_the_boundary():
               "sca_compact_no_alloc", "msda_linear", "msda_linear_timeouts",
               "sca_module_forward", "sca_backward_inputs", "tsa_reference_points", "tsa_forward", "sca_forward_query_major",
               "msda_linear_dropout", "msda_backward_deterministic", "tsa_backward",
-              "sca_backward_deterministic", "sca_backward_full", "sca_backward_full_workspace_size",
+              "sca_backward_deterministic", "sca_backward_full", "sca_backward_full_workspace_size", "msda_linear_test_withhold_load",
               "msda_status_string", "msda_last_error", "msda_version"):
         assert n in names
 
