@@ -102,9 +102,13 @@ def algorithmic_bytes(w, rows, hit_queries, value_elem):
     return {"gather": int(gather), "step": int(step)}
 
 
-def gather_kernel_name(w):
-    """The rebatched-gather kernel sca_rebatched_forward launches here."""
-    return ("sca_gather_quad_kernel" if w.L * w.P <= 32 else "sca_gather_kernel")
+def gather_kernel_name(w, bf16=False):
+    """The rebatched-gather kernel sca_rebatched_forward launches here: the
+    four-lane kernel for fp32 value and rows of up to 32 samples, else the
+    table kernel (head pairs for bf16 value)."""
+    if not bf16 and w.L * w.P <= 32:
+        return "sca_gather_quad_kernel<float>"
+    return "sca_gather_kernel<bf16, 1, 2>" if bf16 else "sca_gather_kernel<float>"
 
 
 def aggregate(local_ms_total, local_samples, world):
@@ -599,7 +603,7 @@ def run_native(args, backend="nccl", replica=measure_replica):
         "data": "synthetic", "config": workload_config(args),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": gather_kernel_name(w), "peak_source": peak_src,
+                     "kernel": gather_kernel_name(w, res["bf16"]), "peak_source": peak_src,
                      "algorithmic_bytes_per_launch": nbytes["step"],
                      "algorithmic_bytes_note": "the step's bytes (value, offsets and logits "
                                                "of every query, reference points, mask, "
@@ -707,7 +711,7 @@ def measure_next_rows(args, w, tensors, flush, stream, hbm_peak):
                                             out=out, workspace=ws16))
         r = hbm(step_b16, ms)
         r.update(kernel="sca_count + sca_chunk_scan + sca_scatter + "
-                        f"{gather_kernel_name(w)}<bf16> + sca_average",
+                        f"{gather_kernel_name(w, True)} + sca_average",
                  workload="bevformer-base-sca-forward, bf16 value",
                  gsamples_per_s=tensors["samples"] / (ms * 1e-3) / 1e9)
         rows["sca_forward_bf16"] = r

@@ -184,7 +184,12 @@ sca_gather_kernel(const VT* __restrict__ value, const float* __restrict__ off,
         bool ok, skip;
         int h, bc, in_row, ref_row, out_row;
     };
-    for (int64_t tile = blockIdx.x; tile * kScaRowsPerTile < total; tile += gridDim.x) {
+#ifndef MSDA_GATHER_CHUNK
+#define MSDA_GATHER_CHUNK 1  // consecutive tiles per CTA within each window of the row list
+#endif
+    constexpr int kChunk = MSDA_GATHER_CHUNK;
+    for (int64_t tile = (int64_t)blockIdx.x * kChunk; tile * kScaRowsPerTile < total;
+         tile = ((tile + 1) % kChunk) ? tile + 1 : tile + 1 + (int64_t)(gridDim.x - 1) * kChunk) {
         const int r0 = (int)(tile * kScaRowsPerTile);
         // lane i < kScaRowsPerTile resolves row r0 + i of the tile: one coalesced index load
         int my_bc = 0, my_in = -1, my_ref = 0, my_out = 0;
@@ -286,15 +291,22 @@ static cudaError_t launch_gather_t(const Problem& p, const float* ref_cam, const
     return cudaGetLastError();
 }
 
+// Which gather serves rows of <= 32 samples: the four-lane kernel
+// (sca_gather_quad.cu) measured faster for fp32 value (0.466 vs 0.498 ms on
+// the BEVFormer-base step), the head-pair table kernel below for bf16 value
+// (0.372 vs 0.417 ms).
 #ifndef MSDA_GATHER_QUAD
-#define MSDA_GATHER_QUAD 1  // rows of <= 32 samples take the four-lane gather
+#define MSDA_GATHER_QUAD 1
+#endif
+#ifndef MSDA_GATHER_QUAD_BF16
+#define MSDA_GATHER_QUAD_BF16 0
 #endif
 
 cudaError_t launch_sca_gather(const Problem& p, const float* ref_cam, const float* off,
                               const float* logits, const int32_t* idx, const int32_t* count,
                               float* out_rb, cudaStream_t s)
 {
-    if (MSDA_GATHER_QUAD && sca_gather_quad_fits(p))
+    if ((p.bf16 ? MSDA_GATHER_QUAD_BF16 : MSDA_GATHER_QUAD) && sca_gather_quad_fits(p))
         return launch_sca_gather_quad(p, ref_cam, off, logits, idx, count, out_rb, s);
     if (!p.bf16) return launch_gather_t<float, 1>(p, ref_cam, off, logits, idx, count, out_rb, s);
     if (p.H % 2 == 0)

@@ -30,13 +30,13 @@
 namespace msda {
 
 #ifndef MSDA_QUAD_MIN_CTAS_F32
-#define MSDA_QUAD_MIN_CTAS_F32 0
+#define MSDA_QUAD_MIN_CTAS_F32 3
 #endif
 #ifndef MSDA_QUAD_MIN_CTAS_BF16
 #define MSDA_QUAD_MIN_CTAS_BF16 0
 #endif
 #ifndef MSDA_QUAD_PREFETCH
-#define MSDA_QUAD_PREFETCH 1  // load the next tile's logits and offsets during this tile
+#define MSDA_QUAD_PREFETCH 0  // 1: load the next tile's logits and offsets during this tile
 #endif
 
 namespace {
@@ -189,46 +189,80 @@ __device__ __forceinline__ void quad_load(const float* __restrict__ lg,
 }
 
 // Softmax over the item's n logits (section 4.2: max-subtracted, each head
-// its own L * P logits) and the sampling locations rho_m + (dx / W_l, dy / H_l)
-// (section 5), in place.  Lanes of dead items get alpha = 0 and NaN
-// locations, which read nothing.
-__device__ __forceinline__ void quad_prepare(QuadIn& in, const QuadMeta* s_meta,
-                                             const float* __restrict__ rf, int n, int t, bool live)
+// its own L * P logits), in place; lanes of dead items get alpha = 0.
+__device__ __forceinline__ void quad_softmax(float (&a)[8], int n, int t, bool live)
 {
     float m = -INFINITY;
 #pragma unroll
-    for (int r = 0; r < 8; ++r) m = fmaxf(m, in.a[r]);
+    for (int r = 0; r < 8; ++r) m = fmaxf(m, a[r]);
     m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
     m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
     float z = 0.f;
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
         const int j = 8 * t + r;
-        in.a[r] = (live && j < n) ? expf(in.a[r] - m) : 0.f;
-        z += in.a[r];
+        a[r] = (live && j < n) ? expf(a[r] - m) : 0.f;
+        z += a[r];
     }
     z += __shfl_xor_sync(0xffffffffu, z, 1);
     z += __shfl_xor_sync(0xffffffffu, z, 2);
     const float zi = live ? z : 1.f;
 #pragma unroll
+    for (int r = 0; r < 8; ++r) a[r] = a[r] / zi;
+}
+
+// Offsets in level pixels -> normalised offsets dx / W_l, dy / H_l (one IEEE
+// division each, section 5), in place.
+__device__ __forceinline__ void quad_scale_offsets(float (&x)[8], float (&y)[8],
+                                                   const QuadMeta* s_meta, int n, int t, bool live)
+{
+#pragma unroll
     for (int r = 0; r < 8; ++r) {
         const int j = 8 * t + r;
-        in.a[r] = in.a[r] / zi;
         if (live && j < n) {
             const QuadMeta mt = s_meta[quad_meta_slot(j)];
-            const float2 ref = __ldg(reinterpret_cast<const float2*>(rf) + mt.m);
-            in.x[r] = __fadd_rn(ref.x, __fdiv_rn(in.x[r], (float)mt.w));
-            in.y[r] = __fadd_rn(ref.y, __fdiv_rn(in.y[r], (float)mt.h));
-        } else {
-            in.x[r] = __int_as_float(0x7fffffff);  // NaN: no corner is read
-            in.y[r] = in.x[r];
+            x[r] = __fdiv_rn(x[r], (float)mt.w);
+            y[r] = __fdiv_rn(y[r], (float)mt.h);
         }
     }
 }
 
+// Sampling locations rho_m + (dx / W_l, dy / H_l) of the lane's samples from
+// the normalised offsets and one reference-point row rf [R, 2]; samples that
+// do not exist (or dead items) get NaN, which reads nothing.
+__device__ __forceinline__ void quad_locations(const float (&nx)[8], const float (&ny)[8],
+                                               float (&sx)[8], float (&sy)[8],
+                                               const QuadMeta* s_meta,
+                                               const float* __restrict__ rf, int n, int t,
+                                               bool live)
+{
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+        const int j = 8 * t + r;
+        if (live && j < n) {
+            const QuadMeta mt = s_meta[quad_meta_slot(j)];
+            const float2 ref = __ldg(reinterpret_cast<const float2*>(rf) + mt.m);
+            sx[r] = __fadd_rn(ref.x, nx[r]);
+            sy[r] = __fadd_rn(ref.y, ny[r]);
+        } else {
+            sx[r] = __int_as_float(0x7fffffff);  // NaN: no corner is read
+            sy[r] = sx[r];
+        }
+    }
+}
+
+// Softmax weights and sampling locations of one rebatched row, in place.
+__device__ __forceinline__ void quad_prepare(QuadIn& in, const QuadMeta* s_meta,
+                                             const float* __restrict__ rf, int n, int t, bool live)
+{
+    quad_softmax(in.a, n, t, live);
+    quad_scale_offsets(in.x, in.y, s_meta, n, t, live);
+    quad_locations(in.x, in.y, in.x, in.y, s_meta, rf, n, t, live);
+}
+
 // Samples whose corner loads are issued together (a power of two <= 8).
 #ifndef MSDA_QUAD_STEP_F32
-#define MSDA_QUAD_STEP_F32 2
+#define MSDA_QUAD_STEP_F32 1
 #endif
 #ifndef MSDA_QUAD_STEP_BF16
 #define MSDA_QUAD_STEP_BF16 4
@@ -242,6 +276,35 @@ template <typename VT>
 struct QuadBounds {
     static constexpr int kMin = sizeof(VT) == 4 ? MSDA_QUAD_MIN_CTAS_F32 : MSDA_QUAD_MIN_CTAS_BF16;
 };
+
+// The corner loop of one item: every sample j of the quad's item, taken from
+// register j mod 8 of quad lane j / 8 (alpha, s_x, s_y), added into acc.
+template <typename VT>
+__device__ __forceinline__ void quad_gather(const VT* __restrict__ vb, int H, int h, int t, int n,
+                                            const float (&a)[8], const float (&x)[8],
+                                            const float (&y)[8], const QuadMeta* s_meta,
+                                            float (&acc)[8])
+{
+    // The register index must be a constant, so r is the unrolled outer
+    // loop; each pass of the inner loop handles kStep samples (their corner
+    // loads in flight together).
+    const int quads_of_8 = (n + 7) >> 3;
+    constexpr int kStep = QuadStep<VT>::kSamples;
+#pragma unroll
+    for (int r0 = 0; r0 < 8; r0 += kStep) {
+#pragma unroll 1
+        for (int src = 0; src < quads_of_8; ++src) {
+#pragma unroll
+            for (int r = r0; r < r0 + kStep; ++r) {
+                const float al = __shfl_sync(0xffffffffu, a[r], src, 4);
+                const float sx = __shfl_sync(0xffffffffu, x[r], src, 4);
+                const float sy = __shfl_sync(0xffffffffu, y[r], src, 4);
+                const QuadMeta mt = s_meta[quad_meta_slot(8 * src + r)];
+                quad_sample<VT>(vb, H, h, t, al, sx, sy, mt, acc);
+            }
+        }
+    }
+}
 
 }  // namespace
 
@@ -277,8 +340,14 @@ sca_gather_quad_kernel(const VT* __restrict__ value, const float* __restrict__ o
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int u = lane >> 2, t = lane & 3;
-    const int64_t n_items = (int64_t)s_prefix[nbc] * H;
-    const int64_t n_tiles = (n_items + 7) >> 3;
+#ifndef MSDA_QUAD_HEADSPEC
+#define MSDA_QUAD_HEADSPEC 0  // 1: a CTA tile is 64 rows of one head (grid a multiple of H)
+#endif
+    const int total_rows = s_prefix[nbc];
+    const int64_t n_items = (int64_t)total_rows * H;
+    const int64_t n_tiles = MSDA_QUAD_HEADSPEC
+                                ? (((int64_t)total_rows + kWarps * 8 - 1) / (kWarps * 8)) * H * kWarps
+                                : (n_items + 7) >> 3;
     const int64_t stride = (int64_t)gridDim.x * kWarps;
     int bc = 0;  // this quad's (batch, camera): its rows only grow
 
@@ -290,10 +359,18 @@ sca_gather_quad_kernel(const VT* __restrict__ value, const float* __restrict__ o
     };
     auto resolve = [&](int64_t tile) {
         Item it{false, 0, 0, 0, 0, logits, off};
+#if MSDA_QUAD_HEADSPEC
+        const int64_t X = tile / kWarps;
+        const int64_t row64 = (X / H) * (kWarps * 8) + (tile - X * kWarps) * 8 + u;
+        if (tile < n_tiles && row64 < total_rows) {
+            const int row = (int)row64;
+            it.h = (int)(X % H);
+#else
         const int64_t item = tile * 8 + u;
         if (tile < n_tiles && item < n_items) {
             const int row = (int)(item / H);
             it.h = (int)(item - (int64_t)row * H);
+#endif
             while (row >= s_prefix[bc + 1]) ++bc;
             const int i = row - s_prefix[bc];
             const int b = bc / Ncam, c = bc - b * Ncam;
@@ -311,13 +388,25 @@ sca_gather_quad_kernel(const VT* __restrict__ value, const float* __restrict__ o
         return it;
     };
 
-    int64_t tile = (int64_t)blockIdx.x * kWarps + warp;
+#ifndef MSDA_QUAD_CHUNK
+#define MSDA_QUAD_CHUNK 1  // consecutive warp-tile groups per CTA within each window
+#endif
+    // CTA k takes kChunk consecutive groups of kWarps warp tiles, then skips
+    // to its groups in the next window of gridDim.x * kChunk groups
+    constexpr int kChunk = MSDA_QUAD_CHUNK;
+    auto advance = [&](int64_t t0) {
+        const int64_t g = t0 / kWarps;  // the group (kWarps consecutive tiles) of t0
+        return ((g + 1) % kChunk) ? t0 + kWarps
+                                  : t0 + kWarps + (int64_t)(gridDim.x - 1) * kChunk * kWarps;
+    };
+    (void)stride;
+    int64_t tile = (int64_t)blockIdx.x * kChunk * kWarps + warp;
     if (tile >= n_tiles) return;  // warp-uniform
     Item cur = resolve(tile);
     QuadIn in;
     quad_load(cur.lg, cur.of, n, t, cur.live, vec, in);
     while (true) {
-        const int64_t next_tile = tile + stride;
+        const int64_t next_tile = advance(tile);
 #if MSDA_QUAD_PREFETCH
         const Item nxt = resolve(next_tile);
         QuadIn in_next;
@@ -329,26 +418,7 @@ sca_gather_quad_kernel(const VT* __restrict__ value, const float* __restrict__ o
         float acc[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-        // Sample j = 8 src + r lives in register r of lane src of the quad.
-        // The register index must be a constant, so r is the unrolled outer
-        // loop; each pass of the inner loop handles kStep samples (their
-        // corner loads in flight together).
-        const int quads_of_8 = (n + 7) >> 3;
-        constexpr int kStep = QuadStep<VT>::kSamples;
-#pragma unroll
-        for (int r0 = 0; r0 < 8; r0 += kStep) {
-#pragma unroll 1
-            for (int src = 0; src < quads_of_8; ++src) {
-#pragma unroll
-                for (int r = r0; r < r0 + kStep; ++r) {
-                    const float a = __shfl_sync(0xffffffffu, in.a[r], src, 4);
-                    const float sx = __shfl_sync(0xffffffffu, in.x[r], src, 4);
-                    const float sy = __shfl_sync(0xffffffffu, in.y[r], src, 4);
-                    const QuadMeta mt = s_meta[quad_meta_slot(8 * src + r)];
-                    quad_sample<VT>(vb, H, cur.h, t, a, sx, sy, mt, acc);
-                }
-            }
-        }
+        quad_gather<VT>(vb, H, cur.h, t, n, in.a, in.x, in.y, s_meta, acc);
         if (cur.live) {
             float4* o = reinterpret_cast<float4*>(
                 out_rb + ((int64_t)cur.out_row * H + cur.h) * kHeadDim + 8 * t);
@@ -383,7 +453,8 @@ static cudaError_t launch_quad_t(const Problem& p, const float* ref_cam, const f
             n = 1;
         return n;
     }();
-    const int64_t grid = std::min<int64_t>(max_ctas, (int64_t)occ * device_sm_count());
+    int64_t grid = std::min<int64_t>(max_ctas, (int64_t)occ * device_sm_count());
+    if (MSDA_QUAD_HEADSPEC && grid > p.H) grid -= grid % p.H;  // a CTA keeps one head
     const bool vec = p.L * p.P == kQuadSamples && ((uintptr_t)off & 15) == 0 &&
                      ((uintptr_t)logits & 15) == 0;
     sca_gather_quad_kernel<VT><<<(unsigned)grid, kThreads, 0, s>>>(

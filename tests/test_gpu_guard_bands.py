@@ -187,7 +187,9 @@ def test_linear(M, N, K, out_bf16):
 
 
 def test_sca_module_forward():
-    w = _sca_problem(seed=66, B=1, Ncam=2, bev=(4, 6), shapes=((6, 8), (3, 4)), H=8, P=4, R=4)
+    # C = 256 and H * L * P = 256: the projections' N (2 * 256, 256) are multiples of 256
+    w = _sca_problem(seed=66, B=1, Ncam=2, bev=(4, 6), shapes=((6, 8), (3, 4), (2, 2), (1, 2)),
+                     H=8, P=8, R=4)
     C, S = w.H * 32, w.H * w.L * w.P
     gen = torch.Generator(device="cuda").manual_seed(66)
     q = torch.randn((w.B, w.Nq, C), device="cuda", generator=gen)
