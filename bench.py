@@ -700,29 +700,38 @@ def measure_next_rows(args, w, tensors, flush, stream, hbm_peak):
     rows["sca_forward_query_major"] = r
 
     # the same SCA forward with bf16 value (BEVFormer-base's bf16 variant):
-    # the rebatched step (sca_forward's kernels) and the query-major kernel
+    # sca_forward (which takes the query-major kernel for bf16 value) and the
+    # rebatched steps (compaction, head-pair gather, camera average)
     if not bf16:
         vb16 = value.to(torch.bfloat16)  # round to nearest even, as the inputs module does
         step_b16 = tensors["step_bytes"] - w.value.size * 2
-        ws16 = torch.empty(msda.msda_workspace_size(msda.Dims(w.B, w.Ncam, w.Nq, w.Nv, w.H,
-                                                              w.L, w.P, w.R)),
-                           dtype=torch.uint8, device="cuda")
+        dims16 = msda.Dims(w.B, w.Ncam, w.Nq, w.Nv, w.H, w.L, w.P, w.R)
+        ws16 = torch.empty(msda.msda_workspace_size(dims16), dtype=torch.uint8, device="cuda")
         ms = timed(lambda: msda.sca_forward(vb16, shapes, starts, ref, mask, off, logits,
                                             out=out, workspace=ws16))
+        r = hbm(step_b16, ms)
+        r.update(kernel="sca_query_major_kernel<bf16, 1, 2> (sca_forward's bf16 path)",
+                 workload="bevformer-base-sca-forward, bf16 value",
+                 gsamples_per_s=tensors["samples"] / (ms * 1e-3) / 1e9)
+        rows["sca_forward_bf16"] = r
+        cws16 = torch.empty(max(16, msda.sca_compact_workspace_size(dims16)), dtype=torch.uint8,
+                            device="cuda")
+        lists = msda.sca_compact(mask, workspace=cws16)
+        rb16 = torch.empty((w.B, w.Ncam, w.Nq, w.H * 32), dtype=torch.float32, device="cuda")
+
+        def staged16():
+            msda.sca_compact(mask, workspace=cws16, out=lists)
+            msda.sca_rebatched_forward(vb16, shapes, starts, ref, off, logits, lists[0],
+                                       lists[1], out_rb=rb16)
+            msda.sca_camera_average(rb16, lists[2], lists[3], out=out)
+        ms = timed(staged16)
         r = hbm(step_b16, ms)
         r.update(kernel="sca_count + sca_chunk_scan + sca_scatter + "
                         f"{gather_kernel_name(w, True)} + sca_average",
                  workload="bevformer-base-sca-forward, bf16 value",
                  gsamples_per_s=tensors["samples"] / (ms * 1e-3) / 1e9)
-        rows["sca_forward_bf16"] = r
-        ms = timed(lambda: msda.sca_forward_query_major(vb16, shapes, starts, ref, mask, off,
-                                                        logits, out=out))
-        r = hbm(step_b16, ms)
-        r.update(kernel="sca_query_major_kernel<bf16>",
-                 workload="bevformer-base-sca-forward, bf16 value",
-                 gsamples_per_s=tensors["samples"] / (ms * 1e-3) / 1e9)
-        rows["sca_forward_query_major_bf16"] = r
-        del vb16, ws16
+        rows["sca_rebatched_step_bf16"] = r
+        del vb16, ws16, cws16, rb16, lists
 
     # the plain fused MSDA: the Deformable-DETR encoder and the TSA queues as a batch
     for name, wk, kname in (

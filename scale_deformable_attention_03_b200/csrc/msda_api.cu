@@ -790,6 +790,10 @@ msda_status_t api_cuda(cudaError_t e, const char* where) { return cuda_status(e,
 
 namespace msda {
 
+#ifndef MSDA_SCA_FORWARD_QM_BF16
+#define MSDA_SCA_FORWARD_QM_BF16 1
+#endif
+
 msda_status_t sca_forward_to(const void* value, msda_dtype_t vdt, const int64_t* spatial_shapes,
                              const int64_t* level_start_index, const float* reference_points_cam,
                              const uint8_t* bev_mask, const float* sampling_offsets,
@@ -806,6 +810,14 @@ msda_status_t sca_forward_to(const void* value, msda_dtype_t vdt, const int64_t*
                              msda::sca_workspace_bytes(d.B, d.Ncam, d.Nq, d.H, true)));
     const msda::ScaWorkspace w = msda::sca_workspace_carve(workspace, d.B, d.Ncam, d.Nq, d.H, true);
     const msda::Problem p = make_problem(value, vdt, d, lv);
+    // bf16 value with an fp32 result: the query-major kernel computes the same
+    // function in one pass (no compaction, rebatched rows or average kernel)
+    // and measured faster there (0.401 vs 0.424 ms on the BEVFormer-base step)
+    if (MSDA_SCA_FORWARD_QM_BF16 && vdt == MSDA_BF16 && !out_bf16)
+        return cuda_status(msda::launch_sca_query_major(p, reference_points_cam, bev_mask,
+                                                        sampling_offsets, attention_logits,
+                                                        static_cast<float*>(out), s),
+                           "sca_forward");
     cudaError_t e = msda::launch_sca_compact(bev_mask, d.B, d.Ncam, d.Nq, d.R, w.idx, w.count,
                                              w.pos, w.hits, w.chunk_counts, s);
     if (e == cudaSuccess)

@@ -272,10 +272,31 @@ struct QuadStep {
     static constexpr int kSamples = sizeof(VT) == 4 ? MSDA_QUAD_STEP_F32 : MSDA_QUAD_STEP_BF16;
 };
 
+// 1: the quads keep their samples' (alpha, s_x, s_y) in shared memory and
+// read them there in the corner loop (no registers held, no shuffles).
+#ifndef MSDA_QUAD_SMEM
+#define MSDA_QUAD_SMEM 0
+#endif
+constexpr int kQuadSmemStride = kQuadSamples + 1;  // quads u of a warp on distinct banks
+
 template <typename VT>
 struct QuadBounds {
     static constexpr int kMin = sizeof(VT) == 4 ? MSDA_QUAD_MIN_CTAS_F32 : MSDA_QUAD_MIN_CTAS_BF16;
 };
+
+// The corner loop of one item from the warp's shared-memory copy of its
+// quads' samples: sa, sx, sy point at this quad's row of 32 (+1) entries.
+template <typename VT>
+__device__ __forceinline__ void quad_gather_smem(const VT* __restrict__ vb, int H, int h, int t,
+                                                 int n, const float* sa, const float* sx,
+                                                 const float* sy, const QuadMeta* s_meta,
+                                                 float (&acc)[8])
+{
+    constexpr int kStep = QuadStep<VT>::kSamples;
+#pragma unroll kStep
+    for (int j = 0; j < n; ++j)
+        quad_sample<VT>(vb, H, h, t, sa[j], sx[j], sy[j], s_meta[quad_meta_slot(j)], acc);
+}
 
 // The corner loop of one item: every sample j of the quad's item, taken from
 // register j mod 8 of quad lane j / 8 (alpha, s_x, s_y), added into acc.
@@ -323,6 +344,7 @@ sca_gather_quad_kernel(const VT* __restrict__ value, const float* __restrict__ o
 {
     __shared__ QuadMeta s_meta[kQuadMetaSlots];
     __shared__ int s_prefix[kMaxBatchCameras + 1];
+    __shared__ float s_in[MSDA_QUAD_SMEM ? kWarps : 1][3][8][kQuadSmemStride];
     const int n = L * P;
     if (threadIdx.x < kQuadSamples) {
         const int j = threadIdx.x;
@@ -418,7 +440,24 @@ sca_gather_quad_kernel(const VT* __restrict__ value, const float* __restrict__ o
         float acc[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#if MSDA_QUAD_SMEM
+        {
+            float* sa = s_in[warp][0][u];
+            float* sx = s_in[warp][1][u];
+            float* sy = s_in[warp][2][u];
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                sa[8 * t + r] = in.a[r];
+                sx[8 * t + r] = in.x[r];
+                sy[8 * t + r] = in.y[r];
+            }
+            __syncwarp();
+            quad_gather_smem<VT>(vb, H, cur.h, t, n, sa, sx, sy, s_meta, acc);
+            __syncwarp();  // read before the next item overwrites
+        }
+#else
         quad_gather<VT>(vb, H, cur.h, t, n, in.a, in.x, in.y, s_meta, acc);
+#endif
         if (cur.live) {
             float4* o = reinterpret_cast<float4*>(
                 out_rb + ((int64_t)cur.out_row * H + cur.h) * kHeadDim + 8 * t);

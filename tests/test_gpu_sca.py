@@ -111,6 +111,26 @@ def test_empty_mask():
     assert torch.all(out == 0)
 
 
+def test_rebatched_bf16_full_size():
+    """The staged rebatched path with bf16 value (head-pair gather) at the
+    full BEVFormer-base size; sca_forward takes the query-major kernel for bf16
+    value, so the two agree within the bf16-path bound of the oracle."""
+    w = inputs.workload3(value_dtype="bf16")
+    v = value_tensor(w, True)
+    args = (v, w.spatial_shapes, w.level_start_index, dev(w.reference_points))
+    idx, count, pos, hits = msda.sca_compact(dev(w.bev_mask))
+    rows = msda.sca_rebatched_forward(*args, dev(w.sampling_offsets), dev(w.attention_logits),
+                                      idx, count)
+    staged = msda.sca_camera_average(rows, pos, hits)
+    whole = msda.sca_forward(*args, dev(w.bev_mask), dev(w.sampling_offsets),
+                             dev(w.attention_logits))
+    torch.cuda.synchronize()
+    ref = oracle.sca_forward(w.value, w.spatial_shapes, w.level_start_index, w.reference_points,
+                             w.bev_mask, w.sampling_offsets, w.attention_logits)
+    assert_close(staged, ref, True, "staged bf16 SCA")
+    assert_close(whole, ref, True, "sca_forward bf16")
+
+
 def test_staged_calls_equal_sca_forward():
     """sca_compact + sca_rebatched_forward + sca_camera_average is sca_forward,
     bit for bit, and the rebatched rows match the oracle's."""
