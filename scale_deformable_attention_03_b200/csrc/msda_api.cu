@@ -585,7 +585,7 @@ msda_status_t sca_forward_query_major(const void* value, msda_dtype_t vdt,
     MSDA_PTR(out, 16);
     const msda::Problem p = make_problem(value, vdt, d, lv);
     return cuda_status(msda::launch_sca_query_major(p, reference_points_cam, bev_mask,
-                                                    sampling_offsets, attention_logits, out,
+                                                    sampling_offsets, attention_logits, out, false,
                                                     (cudaStream_t)stream),
                        "sca_forward_query_major");
 }
@@ -810,13 +810,15 @@ msda_status_t sca_forward_to(const void* value, msda_dtype_t vdt, const int64_t*
                              msda::sca_workspace_bytes(d.B, d.Ncam, d.Nq, d.H, true)));
     const msda::ScaWorkspace w = msda::sca_workspace_carve(workspace, d.B, d.Ncam, d.Nq, d.H, true);
     const msda::Problem p = make_problem(value, vdt, d, lv);
-    // bf16 value with an fp32 result: the query-major kernel computes the same
-    // function in one pass (no compaction, rebatched rows or average kernel)
-    // and measured faster there (0.401 vs 0.424 ms on the BEVFormer-base step)
-    if (MSDA_SCA_FORWARD_QM_BF16 && vdt == MSDA_BF16 && !out_bf16)
+    // bf16 value: the query-major kernel computes the same function in one
+    // pass (no compaction, rebatched rows or average kernel: the camera mean
+    // is formed in registers and stored once, as fp32 or, for the SCA module,
+    // as the bf16 operand of the output projection) and measured faster there
+    // (0.401 vs 0.424 ms on the BEVFormer-base step)
+    if (MSDA_SCA_FORWARD_QM_BF16 && vdt == MSDA_BF16)
         return cuda_status(msda::launch_sca_query_major(p, reference_points_cam, bev_mask,
-                                                        sampling_offsets, attention_logits,
-                                                        static_cast<float*>(out), s),
+                                                        sampling_offsets, attention_logits, out,
+                                                        out_bf16, s),
                            "sca_forward");
     cudaError_t e = msda::launch_sca_compact(bev_mask, d.B, d.Ncam, d.Nq, d.R, w.idx, w.count,
                                              w.pos, w.hits, w.chunk_counts, s);

@@ -772,11 +772,8 @@ msda_backward_kernel(const VT* __restrict__ value, const float* __restrict__ loc
 // PREC: precise location gradients with their rounding residual into
 // grad_loc_lo_rb (see row_backward), for the chain to offsets and reference
 // points.
-#ifndef MSDA_BWD_SCA_MIN_CTAS
-#define MSDA_BWD_SCA_MIN_CTAS 1  // register cap of the SCA row backward (resident CTAs per SM)
-#endif
 template <typename VT, int NC, bool DET, bool PREC>
-__global__ void __launch_bounds__(kThreads, MSDA_BWD_SCA_MIN_CTAS)
+__global__ void __launch_bounds__(kThreads)
 sca_backward_kernel(const VT* __restrict__ value, const float* __restrict__ off,
                     const float* __restrict__ logits, const float* __restrict__ ref_cam,
                     const float* __restrict__ grad_out, const int32_t* __restrict__ idx,
@@ -1226,10 +1223,6 @@ static cudaError_t launch_sca_backward_t(const Problem& p, const float* ref_cam,
     return cudaGetLastError();
 }
 
-#ifndef MSDA_BWD_QUAD
-#define MSDA_BWD_QUAD 1  // rows of <= 32 samples take the four-lane backward
-#endif
-
 cudaError_t launch_sca_backward_rows(const Problem& p, const float* ref_cam, const float* off,
                                      const float* logits, const float* grad_out,
                                      const int32_t* idx, const int32_t* hits,
@@ -1237,10 +1230,6 @@ cudaError_t launch_sca_backward_rows(const Problem& p, const float* ref_cam, con
                                      long long* grad_value_fix, float* grad_loc_rb,
                                      float* grad_attn_rb, cudaStream_t s, float* grad_loc_lo_rb)
 {
-    if (MSDA_BWD_QUAD && sca_backward_quad_fits(p))
-        return launch_sca_backward_quad(p, ref_cam, off, logits, grad_out, idx, hits, count,
-                                        grad_value, grad_value_fix, grad_loc_rb, grad_loc_lo_rb,
-                                        grad_attn_rb, s);
 #define SCA_BWD_ARGS                                                                             \
     p, ref_cam, off, logits, grad_out, idx, hits, count, grad_value, grad_value_fix, grad_loc_rb, \
         grad_loc_lo_rb, grad_attn_rb, s

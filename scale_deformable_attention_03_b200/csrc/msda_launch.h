@@ -64,9 +64,10 @@ cudaError_t launch_sca_gather_quad(const Problem& p, const float* ref_cam, const
                                    float* out_rb, cudaStream_t s);
 
 // K3q: the whole SCA forward, query-major (no compaction, no rebatched rows).
+// out_bf16: the result stored as bf16 (bf16 value only).
 cudaError_t launch_sca_query_major(const Problem& p, const float* ref_cam, const uint8_t* mask,
-                                   const float* off, const float* logits, float* out,
-                                   cudaStream_t s);
+                                   const float* off, const float* logits, void* out,
+                                   bool out_bf16, cudaStream_t s);
 
 // K4: deterministic camera average; fp32 or (out_bf16) bf16 output.
 cudaError_t launch_sca_average(const float* out_rb, const int32_t* pos, const int32_t* hits,
@@ -91,15 +92,6 @@ cudaError_t launch_sca_backward_rows(const Problem& p, const float* ref_cam, con
                                      long long* grad_value_fix, float* grad_loc_rb,
                                      float* grad_attn_rb, cudaStream_t s,
                                      float* grad_loc_lo_rb = nullptr);
-// K6 in the four-lane layout for rows of up to 32 samples (sca_backward_quad.cu):
-// the arguments of launch_sca_backward_rows.
-bool sca_backward_quad_fits(const Problem& p);
-cudaError_t launch_sca_backward_quad(const Problem& p, const float* ref_cam, const float* off,
-                                     const float* logits, const float* grad_out,
-                                     const int32_t* idx, const int32_t* hits,
-                                     const int32_t* count, float* grad_value,
-                                     long long* grad_value_fix, float* grad_loc_rb,
-                                     float* grad_loc_lo_rb, float* grad_attn_rb, cudaStream_t s);
 cudaError_t launch_fix_to_float(const long long* acc, float* out, int64_t n, cudaStream_t s);
 cudaError_t launch_sca_zero_tail(const int32_t* count, int B, int Ncam, int Nq, int S,
                                  float* grad_loc_rb, float* grad_attn_rb, cudaStream_t s);

@@ -56,11 +56,45 @@ __device__ __forceinline__ void divide_acc(float (&acc)[NA], unsigned seen)
     for (int i = 0; i < NA; ++i) acc[i] *= inv;
 }
 
-template <typename VT, int NC, int HP>
+// Eight channels rounded to bf16 (to nearest even) in one 16-byte store.
+__device__ __forceinline__ void store_bf16x8(__nv_bfloat16* dst, const float (&v)[8])
+{
+    uint32_t u[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 p = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+        u[i] = *reinterpret_cast<const uint32_t*>(&p);
+    }
+    *reinterpret_cast<uint4*>(dst) = make_uint4(u[0], u[1], u[2], u[3]);
+}
+
+// The bf16-output form of pair_store (HP = 2) and Gather<bf16>::store (HP = 1)
+// for bf16 value: the mean rounded to bf16, the operand type of the output
+// projection that follows it in the SCA module.
+template <int HP>
+__device__ __forceinline__ void store_row_bf16(float (&acc)[8], int lane,
+                                               __nv_bfloat16* __restrict__ out_row0)
+{
+    const int g = (lane >> 2) & 3, t = lane & 3;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 4);
+        acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 8);
+        if (HP == 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 16);
+    }
+    if (HP == 2) {
+        if (g == 0) store_bf16x8(out_row0 + (lane >> 4) * kHeadDim + 8 * t, acc);
+    } else if (lane < 4) {
+        store_bf16x8(out_row0 + 8 * t, acc);
+    }
+}
+
+// OUT16: the result is stored as bf16 (bf16 value only).
+template <typename VT, int NC, int HP, bool OUT16>
 __global__ void MSDA_QM_BOUNDS(VT, NC)
 sca_query_major_kernel(const VT* __restrict__ value, const float* __restrict__ off,
                        const float* __restrict__ logits, const float* __restrict__ ref_cam,
-                       const uint8_t* __restrict__ mask, float* __restrict__ out, int B,
+                       const uint8_t* __restrict__ mask, void* __restrict__ out, int B,
                        int Ncam, int Nq, int Nv, int H, int L, int P, int R, Levels levels)
 {
     using Table = typename std::conditional<HP == 2, PairTable, WarpTable>::type;
@@ -149,11 +183,14 @@ sca_query_major_kernel(const VT* __restrict__ value, const float* __restrict__ o
             }
         }
         divide_acc(acc, x0.seen);
-        float* orow = out + (x0.bq * H + x0.h) * kHeadDim;
-        if constexpr (HP == 2)
-            pair_store(acc, lane, orow);
-        else
-            Gather<VT>::store(acc, lane, orow);
+        const int64_t orow = (x0.bq * H + x0.h) * kHeadDim;
+        if constexpr (OUT16) {
+            store_row_bf16<HP>(acc, lane, static_cast<__nv_bfloat16*>(out) + orow);
+        } else if constexpr (HP == 2) {
+            pair_store(acc, lane, static_cast<float*>(out) + orow);
+        } else {
+            Gather<VT>::store(acc, lane, static_cast<float*>(out) + orow);
+        }
         x0 = x1;
         in0 = in1;
         cur = nx;
@@ -161,9 +198,9 @@ sca_query_major_kernel(const VT* __restrict__ value, const float* __restrict__ o
     }
 }
 
-template <typename VT, int HP>
+template <typename VT, int HP, bool OUT16 = false>
 static cudaError_t launch_qm_t(const Problem& p, const float* ref_cam, const uint8_t* mask,
-                               const float* off, const float* logits, float* out, cudaStream_t s)
+                               const float* off, const float* logits, void* out, cudaStream_t s)
 {
     const int64_t rows = (int64_t)p.B * p.Nq;
     if (rows == 0) return cudaSuccess;
@@ -172,7 +209,7 @@ static cudaError_t launch_qm_t(const Problem& p, const float* ref_cam, const uin
     switch ((p.L * p.P + 31) / 32) {
 #define SCA_QM_CASE(NCV)                                                                         \
     case NCV:                                                                                    \
-        sca_query_major_kernel<VT, NCV, HP><<<grid, kThreads, 0, s>>>(                           \
+        sca_query_major_kernel<VT, NCV, HP, OUT16><<<grid, kThreads, 0, s>>>(                    \
             v, off, logits, ref_cam, mask, out, p.B, p.Ncam, p.Nq, p.Nv, p.H, p.L, p.P, p.R,     \
             p.lv);                                                                               \
         break;
@@ -187,13 +224,18 @@ static cudaError_t launch_qm_t(const Problem& p, const float* ref_cam, const uin
 }
 
 cudaError_t launch_sca_query_major(const Problem& p, const float* ref_cam, const uint8_t* mask,
-                                   const float* off, const float* logits, float* out,
-                                   cudaStream_t s)
+                                   const float* off, const float* logits, void* out,
+                                   bool out_bf16, cudaStream_t s)
 {
-    if (!p.bf16) return launch_qm_t<float, 1>(p, ref_cam, mask, off, logits, out, s);
+    if (!p.bf16) {
+        if (out_bf16) return cudaErrorInvalidValue;  // bf16 output serves bf16 value only
+        return launch_qm_t<float, 1>(p, ref_cam, mask, off, logits, out, s);
+    }
     if (p.H % 2 == 0)
-        return launch_qm_t<__nv_bfloat16, 2>(p, ref_cam, mask, off, logits, out, s);
-    return launch_qm_t<__nv_bfloat16, 1>(p, ref_cam, mask, off, logits, out, s);
+        return out_bf16 ? launch_qm_t<__nv_bfloat16, 2, true>(p, ref_cam, mask, off, logits, out, s)
+                        : launch_qm_t<__nv_bfloat16, 2>(p, ref_cam, mask, off, logits, out, s);
+    return out_bf16 ? launch_qm_t<__nv_bfloat16, 1, true>(p, ref_cam, mask, off, logits, out, s)
+                    : launch_qm_t<__nv_bfloat16, 1>(p, ref_cam, mask, off, logits, out, s);
 }
 
 }  // namespace msda
