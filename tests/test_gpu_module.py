@@ -20,14 +20,19 @@ def _bf16_tensor(a):
     return torch.from_numpy(inputs.to_bf16_bits(a).view(np.int16)).cuda().view(torch.bfloat16)
 
 
-@pytest.mark.parametrize("value_bf16,dropout_p,embeds", [(False, 0.0, False), (True, 0.0, False),
-                                                         (False, 0.1, False), (True, 0.3, False),
-                                                         (False, 0.0, True), (True, 0.1, True)])
-def test_module_matches_oracle(value_bf16, dropout_p, embeds):
+SMALL = dict(bev_h=16, bev_w=20, shapes=[(29, 50), (15, 25), (8, 13), (4, 7)])
+FULL = {}  # the BEVFormer-base sizes: 200 x 200 BEV, 6 cameras, 4 levels
+
+
+@pytest.mark.parametrize("size,value_bf16,dropout_p,embeds", [
+    ("small", False, 0.0, False), ("small", True, 0.0, False), ("small", False, 0.1, False),
+    ("small", True, 0.3, False), ("small", False, 0.0, True), ("small", True, 0.1, True),
+    ("full", False, 0.0, False), ("full", True, 0.1, True),
+])
+def test_module_matches_oracle(size, value_bf16, dropout_p, embeds):
     timeouts0 = msda.lib().msda_linear_timeouts()
     rng = np.random.Generator(np.random.PCG64(77))
-    w = inputs.workload3(seed=78, bev_h=16, bev_w=20,
-                         shapes=[(29, 50), (15, 25), (8, 13), (4, 7)])
+    w = inputs.workload3(seed=78, **(SMALL if size == "small" else FULL))
     B, Ncam, Nq, Nv, H, L, P = w.B, w.Ncam, w.Nq, w.Nv, w.H, w.L, w.P
     C, S = H * 32, H * L * P
     q = rng.standard_normal((B, Nq, C)).astype(np.float32)
