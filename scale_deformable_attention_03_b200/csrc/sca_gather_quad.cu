@@ -57,13 +57,25 @@ struct QuadCorner<float> {
 #pragma unroll
         for (int e = 0; e < 8; ++e) r.v[e] = 0.f;
     }
-    // 32 bytes in one 256-bit load (read-only path).
-    __device__ __forceinline__ static void load(const float* p, Raw& r)
+    // 32 bytes in one 256-bit load (read-only path); policy 1: not allocated
+    // in L1, 2: kept in L1 preferentially (the level's reuse decides).
+    __device__ __forceinline__ static void load(const float* p, Raw& r, int policy = 0)
     {
-        asm volatile("ld.global.nc.v8.f32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-                     : "=f"(r.v[0]), "=f"(r.v[1]), "=f"(r.v[2]), "=f"(r.v[3]), "=f"(r.v[4]),
-                       "=f"(r.v[5]), "=f"(r.v[6]), "=f"(r.v[7])
-                     : "l"(p));
+        if (policy == 1)
+            asm volatile("ld.global.nc.L1::no_allocate.v8.f32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                         : "=f"(r.v[0]), "=f"(r.v[1]), "=f"(r.v[2]), "=f"(r.v[3]), "=f"(r.v[4]),
+                           "=f"(r.v[5]), "=f"(r.v[6]), "=f"(r.v[7])
+                         : "l"(p));
+        else if (policy == 2)
+            asm volatile("ld.global.nc.L1::evict_last.v8.f32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                         : "=f"(r.v[0]), "=f"(r.v[1]), "=f"(r.v[2]), "=f"(r.v[3]), "=f"(r.v[4]),
+                           "=f"(r.v[5]), "=f"(r.v[6]), "=f"(r.v[7])
+                         : "l"(p));
+        else
+            asm volatile("ld.global.nc.v8.f32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                         : "=f"(r.v[0]), "=f"(r.v[1]), "=f"(r.v[2]), "=f"(r.v[3]), "=f"(r.v[4]),
+                           "=f"(r.v[5]), "=f"(r.v[6]), "=f"(r.v[7])
+                         : "l"(p));
     }
     __device__ __forceinline__ static void fma(float (&acc)[8], float w, const Raw& r)
     {
@@ -78,7 +90,7 @@ struct QuadCorner<__nv_bfloat16> {
         uint4 u;
     };
     __device__ __forceinline__ static void zero(Raw& r) { r.u = make_uint4(0u, 0u, 0u, 0u); }
-    __device__ __forceinline__ static void load(const __nv_bfloat16* p, Raw& r)
+    __device__ __forceinline__ static void load(const __nv_bfloat16* p, Raw& r, int = 0)
     {
         r.u = __ldg(reinterpret_cast<const uint4*>(p));
     }
@@ -102,9 +114,26 @@ struct QuadCorner<__nv_bfloat16> {
 
 // Level geometry and anchor of sample j, stored at j + j / 8 so that the
 // four lanes of a quad (samples 8t + r) read four different bank groups.
+// m: the anchor in bits 0-7, the L1 policy of the level's corner loads above.
 struct __align__(16) QuadMeta {
     int w, h, start, m;
 };
+
+// L1 policy per level: the finest MSDA_QUAD_NOALLOC_LEVELS levels are read
+// without allocating in L1 (little reuse), the coarsest MSDA_QUAD_KEEP_LEVELS
+// levels with evict-last (their slices are met again by neighbouring rows).
+#ifndef MSDA_QUAD_NOALLOC_LEVELS
+#define MSDA_QUAD_NOALLOC_LEVELS 0
+#endif
+#ifndef MSDA_QUAD_KEEP_LEVELS
+#define MSDA_QUAD_KEEP_LEVELS 0
+#endif
+__device__ __forceinline__ int quad_level_policy(int l, int L)
+{
+    if (l < MSDA_QUAD_NOALLOC_LEVELS) return 1;
+    if (l >= L - MSDA_QUAD_KEEP_LEVELS) return 2;
+    return 0;
+}
 constexpr int kQuadMetaSlots = kQuadSamples + kQuadSamples / 8;
 
 __device__ __forceinline__ int quad_meta_slot(int j) { return j + (j >> 3); }
@@ -131,15 +160,16 @@ __device__ __forceinline__ void quad_sample(const VT* __restrict__ vb, int H, in
     const bool y0in = valid && y0 >= 0, y1in = valid && y0 + 1 < mt.h;
     const int pix = H * kHeadDim;  // elements per pixel
     const int base = ((mt.start + y0 * mt.w + x0) * H + h) * kHeadDim + 8 * t;
+    const int pol = mt.m >> 8;
     typename C::Raw r0, r1, r2, r3;
     C::zero(r0);
     C::zero(r1);
     C::zero(r2);
     C::zero(r3);
-    if (x0in && y0in) C::load(vb + base, r0);
-    if (x1in && y0in) C::load(vb + base + pix, r1);
-    if (x0in && y1in) C::load(vb + base + mt.w * pix, r2);
-    if (x1in && y1in) C::load(vb + base + (mt.w + 1) * pix, r3);
+    if (x0in && y0in) C::load(vb + base, r0, pol);
+    if (x1in && y0in) C::load(vb + base + pix, r1, pol);
+    if (x0in && y1in) C::load(vb + base + mt.w * pix, r2, pol);
+    if (x1in && y1in) C::load(vb + base + (mt.w + 1) * pix, r3, pol);
     C::fma(acc, __fmul_rn(__fmul_rn(hx, hy), alpha), r0);
     C::fma(acc, __fmul_rn(__fmul_rn(lx, hy), alpha), r1);
     C::fma(acc, __fmul_rn(__fmul_rn(hx, ly), alpha), r2);
@@ -241,7 +271,7 @@ __device__ __forceinline__ void quad_locations(const float (&nx)[8], const float
         const int j = 8 * t + r;
         if (live && j < n) {
             const QuadMeta mt = s_meta[quad_meta_slot(j)];
-            const float2 ref = __ldg(reinterpret_cast<const float2*>(rf) + mt.m);
+            const float2 ref = __ldg(reinterpret_cast<const float2*>(rf) + (mt.m & 0xff));
             sx[r] = __fadd_rn(ref.x, nx[r]);
             sy[r] = __fadd_rn(ref.y, ny[r]);
         } else {
@@ -353,7 +383,9 @@ sca_gather_quad_kernel(const VT* __restrict__ value, const float* __restrict__ o
             const int l = j / P, k = j - l * P;
 #pragma unroll
             for (int i = 0; i < kMaxLevels; ++i)  // constant indices: Levels stays in registers
-                if (i == l) mt = QuadMeta{levels.w[i], levels.h[i], levels.start[i], k % R};
+                if (i == l)
+                    mt = QuadMeta{levels.w[i], levels.h[i], levels.start[i],
+                                  (k % R) | (quad_level_policy(l, L) << 8)};
         }
         s_meta[quad_meta_slot(j)] = mt;
     }
