@@ -57,17 +57,12 @@ struct QuadCorner<float> {
 #pragma unroll
         for (int e = 0; e < 8; ++e) r.v[e] = 0.f;
     }
-    // 32 bytes in one 256-bit load (read-only path); policy 1: not allocated
-    // in L1, 2: kept in L1 preferentially (the level's reuse decides).
-    __device__ __forceinline__ static void load(const float* p, Raw& r, int policy = 0)
+    // 32 bytes in one 256-bit load (read-only path); NA: not allocated in L1.
+    template <bool NA>
+    __device__ __forceinline__ static void load(const float* p, Raw& r)
     {
-        if (policy == 1)
+        if constexpr (NA)
             asm volatile("ld.global.nc.L1::no_allocate.v8.f32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-                         : "=f"(r.v[0]), "=f"(r.v[1]), "=f"(r.v[2]), "=f"(r.v[3]), "=f"(r.v[4]),
-                           "=f"(r.v[5]), "=f"(r.v[6]), "=f"(r.v[7])
-                         : "l"(p));
-        else if (policy == 2)
-            asm volatile("ld.global.nc.L1::evict_last.v8.f32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
                          : "=f"(r.v[0]), "=f"(r.v[1]), "=f"(r.v[2]), "=f"(r.v[3]), "=f"(r.v[4]),
                            "=f"(r.v[5]), "=f"(r.v[6]), "=f"(r.v[7])
                          : "l"(p));
@@ -90,9 +85,15 @@ struct QuadCorner<__nv_bfloat16> {
         uint4 u;
     };
     __device__ __forceinline__ static void zero(Raw& r) { r.u = make_uint4(0u, 0u, 0u, 0u); }
-    __device__ __forceinline__ static void load(const __nv_bfloat16* p, Raw& r, int = 0)
+    template <bool NA>
+    __device__ __forceinline__ static void load(const __nv_bfloat16* p, Raw& r)
     {
-        r.u = __ldg(reinterpret_cast<const uint4*>(p));
+        if constexpr (NA)
+            asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(r.u.x), "=r"(r.u.y), "=r"(r.u.z), "=r"(r.u.w)
+                         : "l"(p));
+        else
+            r.u = __ldg(reinterpret_cast<const uint4*>(p));
     }
     __device__ __forceinline__ static void fma(float (&acc)[8], float w, const Raw& r)
     {
@@ -114,26 +115,16 @@ struct QuadCorner<__nv_bfloat16> {
 
 // Level geometry and anchor of sample j, stored at j + j / 8 so that the
 // four lanes of a quad (samples 8t + r) read four different bank groups.
-// m: the anchor in bits 0-7, the L1 policy of the level's corner loads above.
 struct __align__(16) QuadMeta {
     int w, h, start, m;
 };
 
-// L1 policy per level: the finest MSDA_QUAD_NOALLOC_LEVELS levels are read
-// without allocating in L1 (little reuse), the coarsest MSDA_QUAD_KEEP_LEVELS
-// levels with evict-last (their slices are met again by neighbouring rows).
+// The finest MSDA_QUAD_NOALLOC_LEVELS levels read their corners without
+// allocating in L1: those slices are rarely met again, and L1 is left to the
+// coarse levels, whose slices neighbouring rows read again.
 #ifndef MSDA_QUAD_NOALLOC_LEVELS
-#define MSDA_QUAD_NOALLOC_LEVELS 0
+#define MSDA_QUAD_NOALLOC_LEVELS 3
 #endif
-#ifndef MSDA_QUAD_KEEP_LEVELS
-#define MSDA_QUAD_KEEP_LEVELS 0
-#endif
-__device__ __forceinline__ int quad_level_policy(int l, int L)
-{
-    if (l < MSDA_QUAD_NOALLOC_LEVELS) return 1;
-    if (l >= L - MSDA_QUAD_KEEP_LEVELS) return 2;
-    return 0;
-}
 constexpr int kQuadMetaSlots = kQuadSamples + kQuadSamples / 8;
 
 __device__ __forceinline__ int quad_meta_slot(int j) { return j + (j >> 3); }
@@ -141,7 +132,7 @@ __device__ __forceinline__ int quad_meta_slot(int j) { return j + (j >> 3); }
 // One sample of a quad: corner decision ("BEV(三)..." section 6: x = W s_x -
 // 1/2, binary32, never contracted; a neighbour outside the map reads
 // nothing), then the four corner reads weighted by alpha * w_g.
-template <typename VT>
+template <typename VT, bool NA>
 __device__ __forceinline__ void quad_sample(const VT* __restrict__ vb, int H, int h, int t,
                                             float alpha, float sx, float sy, const QuadMeta& mt,
                                             float (&acc)[8])
@@ -160,16 +151,15 @@ __device__ __forceinline__ void quad_sample(const VT* __restrict__ vb, int H, in
     const bool y0in = valid && y0 >= 0, y1in = valid && y0 + 1 < mt.h;
     const int pix = H * kHeadDim;  // elements per pixel
     const int base = ((mt.start + y0 * mt.w + x0) * H + h) * kHeadDim + 8 * t;
-    const int pol = mt.m >> 8;
     typename C::Raw r0, r1, r2, r3;
     C::zero(r0);
     C::zero(r1);
     C::zero(r2);
     C::zero(r3);
-    if (x0in && y0in) C::load(vb + base, r0, pol);
-    if (x1in && y0in) C::load(vb + base + pix, r1, pol);
-    if (x0in && y1in) C::load(vb + base + mt.w * pix, r2, pol);
-    if (x1in && y1in) C::load(vb + base + (mt.w + 1) * pix, r3, pol);
+    if (x0in && y0in) C::template load<NA>(vb + base, r0);
+    if (x1in && y0in) C::template load<NA>(vb + base + pix, r1);
+    if (x0in && y1in) C::template load<NA>(vb + base + mt.w * pix, r2);
+    if (x1in && y1in) C::template load<NA>(vb + base + (mt.w + 1) * pix, r3);
     C::fma(acc, __fmul_rn(__fmul_rn(hx, hy), alpha), r0);
     C::fma(acc, __fmul_rn(__fmul_rn(lx, hy), alpha), r1);
     C::fma(acc, __fmul_rn(__fmul_rn(hx, ly), alpha), r2);
@@ -271,7 +261,7 @@ __device__ __forceinline__ void quad_locations(const float (&nx)[8], const float
         const int j = 8 * t + r;
         if (live && j < n) {
             const QuadMeta mt = s_meta[quad_meta_slot(j)];
-            const float2 ref = __ldg(reinterpret_cast<const float2*>(rf) + (mt.m & 0xff));
+            const float2 ref = __ldg(reinterpret_cast<const float2*>(rf) + mt.m);
             sx[r] = __fadd_rn(ref.x, nx[r]);
             sy[r] = __fadd_rn(ref.y, ny[r]);
         } else {
@@ -318,43 +308,60 @@ struct QuadBounds {
 // quads' samples: sa, sx, sy point at this quad's row of 32 (+1) entries.
 template <typename VT>
 __device__ __forceinline__ void quad_gather_smem(const VT* __restrict__ vb, int H, int h, int t,
-                                                 int n, const float* sa, const float* sx,
+                                                 int n, int P, const float* sa, const float* sx,
                                                  const float* sy, const QuadMeta* s_meta,
                                                  float (&acc)[8])
 {
     constexpr int kStep = QuadStep<VT>::kSamples;
+    const int na_samples = min(n, MSDA_QUAD_NOALLOC_LEVELS * P);
 #pragma unroll kStep
-    for (int j = 0; j < n; ++j)
-        quad_sample<VT>(vb, H, h, t, sa[j], sx[j], sy[j], s_meta[quad_meta_slot(j)], acc);
+    for (int j = 0; j < na_samples; ++j)
+        quad_sample<VT, true>(vb, H, h, t, sa[j], sx[j], sy[j], s_meta[quad_meta_slot(j)], acc);
+#pragma unroll kStep
+    for (int j = na_samples; j < n; ++j)
+        quad_sample<VT, false>(vb, H, h, t, sa[j], sx[j], sy[j], s_meta[quad_meta_slot(j)], acc);
 }
 
 // The corner loop of one item: every sample j of the quad's item, taken from
 // register j mod 8 of quad lane j / 8 (alpha, s_x, s_y), added into acc.
-template <typename VT>
-__device__ __forceinline__ void quad_gather(const VT* __restrict__ vb, int H, int h, int t, int n,
-                                            const float (&a)[8], const float (&x)[8],
-                                            const float (&y)[8], const QuadMeta* s_meta,
-                                            float (&acc)[8])
+template <typename VT, bool NA>
+__device__ __forceinline__ void quad_gather_range(const VT* __restrict__ vb, int H, int h, int t,
+                                                  int src0, int src1, const float (&a)[8],
+                                                  const float (&x)[8], const float (&y)[8],
+                                                  const QuadMeta* s_meta, float (&acc)[8])
 {
     // The register index must be a constant, so r is the unrolled outer
     // loop; each pass of the inner loop handles kStep samples (their corner
     // loads in flight together).
-    const int quads_of_8 = (n + 7) >> 3;
     constexpr int kStep = QuadStep<VT>::kSamples;
 #pragma unroll
     for (int r0 = 0; r0 < 8; r0 += kStep) {
 #pragma unroll 1
-        for (int src = 0; src < quads_of_8; ++src) {
+        for (int src = src0; src < src1; ++src) {
 #pragma unroll
             for (int r = r0; r < r0 + kStep; ++r) {
                 const float al = __shfl_sync(0xffffffffu, a[r], src, 4);
                 const float sx = __shfl_sync(0xffffffffu, x[r], src, 4);
                 const float sy = __shfl_sync(0xffffffffu, y[r], src, 4);
                 const QuadMeta mt = s_meta[quad_meta_slot(8 * src + r)];
-                quad_sample<VT>(vb, H, h, t, al, sx, sy, mt, acc);
+                quad_sample<VT, NA>(vb, H, h, t, al, sx, sy, mt, acc);
             }
         }
     }
+}
+
+// Groups of eight samples wholly inside the finest MSDA_QUAD_NOALLOC_LEVELS
+// levels (the row's first NOALLOC * P samples) load without allocating in L1.
+template <typename VT>
+__device__ __forceinline__ void quad_gather(const VT* __restrict__ vb, int H, int h, int t, int n,
+                                            int P, const float (&a)[8], const float (&x)[8],
+                                            const float (&y)[8], const QuadMeta* s_meta,
+                                            float (&acc)[8])
+{
+    const int quads_of_8 = (n + 7) >> 3;
+    const int na_groups = min(quads_of_8, (MSDA_QUAD_NOALLOC_LEVELS * P) >> 3);
+    quad_gather_range<VT, true>(vb, H, h, t, 0, na_groups, a, x, y, s_meta, acc);
+    quad_gather_range<VT, false>(vb, H, h, t, na_groups, quads_of_8, a, x, y, s_meta, acc);
 }
 
 }  // namespace
@@ -383,9 +390,7 @@ sca_gather_quad_kernel(const VT* __restrict__ value, const float* __restrict__ o
             const int l = j / P, k = j - l * P;
 #pragma unroll
             for (int i = 0; i < kMaxLevels; ++i)  // constant indices: Levels stays in registers
-                if (i == l)
-                    mt = QuadMeta{levels.w[i], levels.h[i], levels.start[i],
-                                  (k % R) | (quad_level_policy(l, L) << 8)};
+                if (i == l) mt = QuadMeta{levels.w[i], levels.h[i], levels.start[i], k % R};
         }
         s_meta[quad_meta_slot(j)] = mt;
     }
@@ -484,11 +489,11 @@ sca_gather_quad_kernel(const VT* __restrict__ value, const float* __restrict__ o
                 sy[8 * t + r] = in.y[r];
             }
             __syncwarp();
-            quad_gather_smem<VT>(vb, H, cur.h, t, n, sa, sx, sy, s_meta, acc);
+            quad_gather_smem<VT>(vb, H, cur.h, t, n, P, sa, sx, sy, s_meta, acc);
             __syncwarp();  // read before the next item overwrites
         }
 #else
-        quad_gather<VT>(vb, H, cur.h, t, n, in.a, in.x, in.y, s_meta, acc);
+        quad_gather<VT>(vb, H, cur.h, t, n, P, in.a, in.x, in.y, s_meta, acc);
 #endif
         if (cur.live) {
             float4* o = reinterpret_cast<float4*>(
