@@ -57,25 +57,6 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
                  : "memory");
 }
 
-// Corner loads that do not allocate in L1 (the finest levels' slices are
-// rarely met again; leaving L1 to the coarse levels raises their hit rate).
-__device__ __forceinline__ float4 ld_na_f4(const float* p)
-{
-    float4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "l"(p));
-    return v;
-}
-__device__ __forceinline__ uint4 ld_na_u4(const void* p)
-{
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
-
 constexpr float kFixScale = 4294967296.f;  // 2^32: fixed-point grad_value units
 
 __device__ __forceinline__ void red_add_fix(long long* addr, float v)
@@ -232,8 +213,7 @@ struct BwdLanes<float> {
     template <bool DET, bool LF>
     __device__ __forceinline__ double batch(const float* __restrict__ vb,
                                             float* __restrict__ gvb, long long* __restrict__ gvi,
-                                            const BwdTable& tab, int j0, int cnt, int lane,
-                                            bool na = false) const
+                                            const BwdTable& tab, int j0, int cnt, int lane) const
     {
         const int g = lane >> 3, t = lane & 7;
         double part[8];
@@ -244,9 +224,8 @@ struct BwdLanes<float> {
             for (int k = 0; k < 8; ++k) {
                 const int j = j0 + k;
                 o[k] = j < cnt ? tab.ow[g][j].x : -1;
-                v[k] = o[k] < 0 ? make_float4(0.f, 0.f, 0.f, 0.f)
-                       : na     ? ld_na_f4(vb + o[k] + 4 * t)
-                                : __ldg(reinterpret_cast<const float4*>(vb + o[k] + 4 * t));
+                v[k] = o[k] >= 0 ? __ldg(reinterpret_cast<const float4*>(vb + o[k] + 4 * t))
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
             }
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
@@ -312,8 +291,7 @@ struct BwdLanes<__nv_bfloat16> {
     template <bool DET, bool LF>
     __device__ __forceinline__ double batch(const __nv_bfloat16* __restrict__ vb,
                                             float* __restrict__ gvb, long long* __restrict__ gvi,
-                                            const BwdTable& tab, int j0, int cnt, int lane,
-                                            bool na = false) const
+                                            const BwdTable& tab, int j0, int cnt, int lane) const
     {
         const int s = lane >> 4, g = (lane >> 2) & 3, t = lane & 3;
         double part[4];
@@ -324,9 +302,8 @@ struct BwdLanes<__nv_bfloat16> {
             for (int k = 0; k < 4; ++k) {
                 const int j = j0 + 2 * k + s;
                 o[k] = j < cnt ? tab.ow[g][j].x : -1;
-                raw[k] = o[k] < 0 ? make_uint4(0u, 0u, 0u, 0u)
-                         : na     ? ld_na_u4(vb + o[k] + 8 * t)
-                                  : __ldg(reinterpret_cast<const uint4*>(vb + o[k] + 8 * t));
+                raw[k] = o[k] >= 0 ? __ldg(reinterpret_cast<const uint4*>(vb + o[k] + 8 * t))
+                                   : make_uint4(0u, 0u, 0u, 0u);
             }
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
@@ -403,8 +380,7 @@ __device__ __forceinline__ void row_backward(const VT* __restrict__ vb, int H, i
                                              DetEntry* __restrict__ det,
                                              float* __restrict__ gloc_row,
                                              float* __restrict__ gattn_row, int lane,
-                                             float* __restrict__ gloc_lo_row = nullptr,
-                                             int na_samples = 0)
+                                             float* __restrict__ gloc_lo_row = nullptr)
 {
     // DET: channel `lane` of the row's upstream gradient, as BwdLanes forms it
     const float go_c = DET ? __ldg(grow + lane) / scale : 0.f;
@@ -454,10 +430,7 @@ __device__ __forceinline__ void row_backward(const VT* __restrict__ vb, int H, i
         typename std::conditional<PREC, double, float>::type res_x = 0, res_y = 0;
         const int cnt = min(32, n - c * 32);
         for (int j0 = 0; j0 < cnt; j0 += 8) {
-            // batches wholly inside the row's first na_samples samples (the
-            // finest levels) read their corners without allocating in L1
-            const bool na = c * 32 + j0 + 8 <= na_samples;
-            const double d = lanes.template batch<DET, LF>(vb, gvb, gvi, tab, j0, cnt, lane, na);
+            const double d = lanes.template batch<DET, LF>(vb, gvb, gvi, tab, j0, cnt, lane);
             if (DET) {  // lane = channel: one 256-byte slice per (sample, corner)
                 for (int j = j0; j < min(j0 + 8, cnt); ++j) {
                     const int4 o = *reinterpret_cast<const int4*>(det[j].off);
@@ -799,10 +772,6 @@ msda_backward_kernel(const VT* __restrict__ value, const float* __restrict__ loc
 // PREC: precise location gradients with their rounding residual into
 // grad_loc_lo_rb (see row_backward), for the chain to offsets and reference
 // points.
-// Finest levels whose corner loads bypass L1 in the SCA row backward.
-#ifndef MSDA_BWD_NOALLOC_LEVELS
-#define MSDA_BWD_NOALLOC_LEVELS 0
-#endif
 template <typename VT, int NC, bool DET, bool PREC>
 __global__ void __launch_bounds__(kThreads)
 sca_backward_kernel(const VT* __restrict__ value, const float* __restrict__ off,
@@ -854,7 +823,7 @@ sca_backward_kernel(const VT* __restrict__ value, const float* __restrict__ off,
                 grad_out + bqh * kHeadDim, scale, grad_value + vofs,
                 DET ? grad_value_fix + vofs : nullptr, s_det[DET ? warp : 0],
                 grad_loc_rb + rowh * S * 2, grad_attn_rb + rowh * S, lane,
-                PREC ? grad_loc_lo_rb + rowh * S * 2 : nullptr, MSDA_BWD_NOALLOC_LEVELS * P);
+                PREC ? grad_loc_lo_rb + rowh * S * 2 : nullptr);
         }
     }
 }

@@ -529,32 +529,14 @@ struct PairTable {
     float w[2][4][kMetaStride];
 };
 
-// 16-byte corner load that does not allocate in L1.
-__device__ __forceinline__ uint4 ldg_na_u4(const void* p)
-{
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
-
-// Finest levels whose bf16 head-pair corner loads bypass L1 (their slices
-// are rarely met again; the coarse levels keep L1 to themselves).
-#ifndef MSDA_PAIR_NOALLOC_LEVELS
-#define MSDA_PAIR_NOALLOC_LEVELS 0
-#endif
-
 // Heads h0 and h0 + 1 of one row from normalised weights, added to the
-// lane's partial sums (see pair_store for the lane layout).  Table quads
-// wholly inside the row's first na_samples samples load without allocating
-// in L1.
+// lane's partial sums (see pair_store for the lane layout).
 template <bool FUSED, int NC>
 __device__ __forceinline__ void pair_gather(const __nv_bfloat16* __restrict__ vb, int H, int h0,
                                             const RowIn<FUSED, NC, 2>& in,
                                             const float2 (&rf)[NC], int n,
                                             const LaneSamples<NC>& ls, PairTable& tab,
-                                            float (&acc)[8], int lane, int na_samples = 0)
+                                            float (&acc)[8], int lane)
 {
     const int half = lane >> 4, g = (lane >> 2) & 3, t = lane & 3;
     const __nv_bfloat16* v = vb + 8 * t;
@@ -577,17 +559,10 @@ __device__ __forceinline__ void pair_gather(const __nv_bfloat16* __restrict__ vb
             const int4 o = *reinterpret_cast<const int4*>(&tab.off[half][g][4 * p]);
             const float4 w = *reinterpret_cast<const float4*>(&tab.w[half][g][4 * p]);
             uint4 r0 = make_uint4(0u, 0u, 0u, 0u), r1 = r0, r2 = r0, r3 = r0;
-            if (c * 32 + 4 * p + 4 <= na_samples) {
-                if (o.x >= 0) r0 = ldg_na_u4(v + o.x);
-                if (o.y >= 0) r1 = ldg_na_u4(v + o.y);
-                if (o.z >= 0) r2 = ldg_na_u4(v + o.z);
-                if (o.w >= 0) r3 = ldg_na_u4(v + o.w);
-            } else {
-                if (o.x >= 0) r0 = __ldg(reinterpret_cast<const uint4*>(v + o.x));
-                if (o.y >= 0) r1 = __ldg(reinterpret_cast<const uint4*>(v + o.y));
-                if (o.z >= 0) r2 = __ldg(reinterpret_cast<const uint4*>(v + o.z));
-                if (o.w >= 0) r3 = __ldg(reinterpret_cast<const uint4*>(v + o.w));
-            }
+            if (o.x >= 0) r0 = __ldg(reinterpret_cast<const uint4*>(v + o.x));
+            if (o.y >= 0) r1 = __ldg(reinterpret_cast<const uint4*>(v + o.y));
+            if (o.z >= 0) r2 = __ldg(reinterpret_cast<const uint4*>(v + o.z));
+            if (o.w >= 0) r3 = __ldg(reinterpret_cast<const uint4*>(v + o.w));
             Gather<__nv_bfloat16>::fma8(acc, w.x, r0);
             Gather<__nv_bfloat16>::fma8(acc, w.y, r1);
             Gather<__nv_bfloat16>::fma8(acc, w.z, r2);
@@ -620,15 +595,14 @@ template <bool FUSED, int NC>
 __device__ __forceinline__ void row_compute_pair(const __nv_bfloat16* __restrict__ vb, int H,
                                                  int h0, RowIn<FUSED, NC, 2>& in, int n,
                                                  const LaneSamples<NC>& ls, PairTable& tab,
-                                                 float* __restrict__ out_row0, int lane,
-                                                 int na_samples = 0)
+                                                 float* __restrict__ out_row0, int lane)
 {
     normalise<FUSED, NC>(in.a[0], ls);
     normalise<FUSED, NC>(in.a[1], ls);
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-    pair_gather<FUSED, NC>(vb, H, h0, in, in.rf, n, ls, tab, acc, lane, na_samples);
+    pair_gather<FUSED, NC>(vb, H, h0, in, in.rf, n, ls, tab, acc, lane);
     pair_store(acc, lane, out_row0);
 }
 

@@ -239,8 +239,7 @@ sca_gather_kernel(const VT* __restrict__ value, const float* __restrict__ off,
                 const VT* vb = value + (int64_t)x0.bc * Nv * H * kHeadDim;
                 float* orow = out_rb + ((int64_t)x0.out_row * H + x0.h) * kHeadDim;
                 if constexpr (HP == 2)
-                    row_compute_pair<true, NC>(vb, H, x0.h, in0, S, ls, s_tab[warp], orow, lane,
-                                               MSDA_PAIR_NOALLOC_LEVELS * P);
+                    row_compute_pair<true, NC>(vb, H, x0.h, in0, S, ls, s_tab[warp], orow, lane);
                 else
                     row_compute<VT, true, NC>(vb, H, x0.h, in0, S, ls, s_tab[warp], orow, lane);
             }

@@ -173,8 +173,7 @@ sca_query_major_kernel(const VT* __restrict__ value, const float* __restrict__ o
                              rf_next);
             const VT* vb = value + ((int64_t)x0.b * Ncam + cam) * vstride;
             if constexpr (HP == 2)
-                pair_gather<true, NC>(vb, H, x0.h, in0, rf, S, ls, s_tab[warp], acc, lane,
-                                      MSDA_PAIR_NOALLOC_LEVELS * P);
+                pair_gather<true, NC>(vb, H, x0.h, in0, rf, S, ls, s_tab[warp], acc, lane);
             else
                 head_gather<VT, true, NC>(vb, H, x0.h, in0.a[0], in0.lo[0], rf, S, ls,
                                           s_tab[warp], acc, lane);
