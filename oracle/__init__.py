@@ -42,6 +42,7 @@ def lib():
         L.oracle_sca_backward.argtypes = [_D, _i, _i, _i, _i, _i, _i, _I64, _I64, _i, _i, _i, _D,
                                           _U8, _D, _D, _D, _i, _D, _D, _D]
         L.oracle_linear.argtypes = [_D, _D, _D, _D, _i, _i, _i, _D]
+        L.oracle_sca_camera_average.argtypes = [_D, _I32, _I32, _i, _i, _i, ctypes.c_int64, _D]
         L.oracle_sca_backward_inputs.argtypes = [_i, _i, _i, _i, _i, _I64, _i, _i, _U8, _D, _D,
                                                  _D, _D, _D, _D]
         L.oracle_tsa_reference_points.argtypes = [_i, _i, _i, _i, ctypes.c_double,
@@ -55,6 +56,7 @@ def lib():
         for f in ("oracle_softmax", "oracle_msda_forward", "oracle_msda_forward_fused",
                   "oracle_fused_locations", "oracle_msda_backward", "oracle_sca_compact",
                   "oracle_sca_forward", "oracle_sca_backward", "oracle_linear",
+                  "oracle_sca_camera_average",
                   "oracle_sca_backward_inputs", "oracle_tsa_reference_points",
                   "oracle_tsa_forward", "oracle_dropout"):
             getattr(L, f).restype = ctypes.c_int
@@ -192,6 +194,21 @@ def sca_forward(value, spatial_shapes, level_start_index, reference_points_cam, 
                                   _p(rb, _D) if rb is not None else None)
     _check(rc, "sca_forward")
     return (out, rb) if return_rebatched else out
+
+
+def sca_camera_average(out_rb, pos, hits):
+    """out_rb [B, Ncam, Nq, HD], pos [B, Ncam, Nq], hits [B, Nq] (int32, as
+    sca_compact gives them) -> out [B, Nq, HD]: the seeing cameras' rows
+    summed in ascending camera order, divided by max(1, hits)."""
+    rb = _d(out_rb)
+    B, Ncam, Nq, HD = rb.shape
+    p = np.ascontiguousarray(pos, dtype=np.int32)
+    h = np.ascontiguousarray(hits, dtype=np.int32)
+    out = np.empty((B, Nq, HD))
+    rc = lib().oracle_sca_camera_average(_p(rb, _D), _p(p, _I32), _p(h, _I32), B, Ncam, Nq, HD,
+                                         _p(out, _D))
+    _check(rc, "sca_camera_average")
+    return out
 
 
 def sca_backward(value, spatial_shapes, level_start_index, reference_points_cam, bev_mask,

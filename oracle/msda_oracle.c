@@ -444,6 +444,30 @@ int oracle_sca_forward(const double* value, int B, int Ncam, int Nv, int H, int 
     return 0;
 }
 
+int oracle_sca_camera_average(const double* out_rb, const int32_t* pos, const int32_t* hits,
+                              int B, int Ncam, int Nq, int64_t HD, double* out)
+{
+    if (out_rb == NULL || pos == NULL || hits == NULL || out == NULL || B < 0 || Ncam < 1 ||
+        Nq < 0 || HD < 1)
+        return -1;
+    for (int b = 0; b < B; ++b)
+        for (int q = 0; q < Nq; ++q) {
+            const int64_t bq = (int64_t)b * Nq + q;
+            double* o = out + bq * HD;
+            for (int64_t d = 0; d < HD; ++d) o[d] = 0.0;
+            for (int c = 0; c < Ncam; ++c) {          /* scatter-add, ascending camera */
+                const int64_t bc = (int64_t)b * Ncam + c;
+                const int32_t i = pos[bc * Nq + q];
+                if (i < 0) continue;
+                if (i >= Nq) return -1;
+                for (int64_t d = 0; d < HD; ++d) o[d] += out_rb[(bc * Nq + i) * HD + d];
+            }
+            const int n = hits[bq] > 1 ? hits[bq] : 1;   /* clamp(count, 1) */
+            for (int64_t d = 0; d < HD; ++d) o[d] /= (double)n;
+        }
+    return 0;
+}
+
 int oracle_sca_backward(const double* value, int B, int Ncam, int Nv, int H, int Dh,
                         int L, const int64_t* shapes, const int64_t* starts,
                         int Nq, int P, int R, const double* ref_cam,

@@ -110,6 +110,14 @@ int oracle_sca_forward(const double* value, int B, int Ncam, int Nv, int H, int 
                        const double* logits, int coord_f32,
                        double* out, double* out_rb);
 
+/* SCA camera average on its own ([SCA] scatter-add and clamp(count, 1)
+ * listing; [BQ] 10): for every (b, q), the rows out_rb[b, c, pos[b, c, q]] of
+ * the cameras c with pos >= 0, added in ascending c, divided by
+ * max(1, hits[b, q]).  out_rb [B, Ncam, Nq, HD]; pos [B, Ncam, Nq];
+ * hits [B, Nq]; out [B, Nq, HD]. */
+int oracle_sca_camera_average(const double* out_rb, const int32_t* pos, const int32_t* hits,
+                              int B, int Ncam, int Nq, int64_t HD, double* out);
+
 /* SCA backward (derivative of oracle_sca_forward w.r.t. value and the
  * rebatched sampling locations and attention weights).
  * grad_out [B, Nq, H*Dh] -> grad_value [B, Ncam, Nv, H, Dh],

@@ -48,6 +48,14 @@ MUTANTS = [
      "oracle_softmax(logit_row, H * L, P, attn_row);", 0),
     ("softmax without normalisation", "for (int i = 0; i < n; ++i) w[i] /= z;", "", 0),
     ("average over all cameras", "int n = sc.hits[bq] > 1 ? sc.hits[bq] : 1;", "int n = Ncam;", 1),
+    ("average step over all cameras", "const int n = hits[bq] > 1 ? hits[bq] : 1;",
+     "const int n = Ncam;", 0),
+    ("average step without the clamp", "const int n = hits[bq] > 1 ? hits[bq] : 1;",
+     "const int n = hits[bq];", 0),
+    ("average step reads camera 0's positions", "const int32_t i = pos[bc * Nq + q];",
+     "const int32_t i = pos[(int64_t)b * Ncam * Nq + q];", 0),
+    ("average step reads the query's row", "o[d] += out_rb[(bc * Nq + i) * HD + d];",
+     "o[d] += out_rb[(bc * Nq + q) * HD + d];", 0),
     ("only anchor 0 decides a hit", "for (int r = 0; r < R; ++r)\n                    if (bev_mask",
      "for (int r = 0; r < 1; ++r)\n                    if (bev_mask", 0),
     ("camera 0 reference points everywhere",
@@ -107,6 +115,8 @@ PIN_CALLS = [
     ("compaction", lambda: pins.test_compaction_brute_force()),
     ("sca_mean", lambda: pins.test_sca_equals_per_query_camera_mean(False)),
     ("sca_rebatch", lambda: pins.test_sca_rebatched_rows_follow_compaction()),
+    ("average_mean", lambda: pins.test_camera_average_is_the_mean_of_the_seeing_cameras()),
+    ("average_closed", lambda: pins.test_camera_average_closed_forms()),
     ("msda_fd", lambda: pins.test_msda_backward_matches_finite_differences()),
     ("msda_fd_border", lambda: pins.test_msda_backward_with_partly_outside_samples()),
     ("linearity", lambda: pins.test_msda_backward_linearity()),
@@ -148,7 +158,8 @@ def test_pins_catch_planted_mistake(tmp_path, monkeypatch, name, old, new, occ):
                   "oracle_fused_locations", "oracle_msda_backward", "oracle_sca_compact",
                   "oracle_sca_forward", "oracle_sca_backward", "oracle_linear",
                   "oracle_sca_backward_inputs", "oracle_tsa_reference_points",
-                  "oracle_tsa_forward", "oracle_dropout", "oracle_philox4x32_10"):
+                  "oracle_tsa_forward", "oracle_dropout", "oracle_philox4x32_10",
+                  "oracle_sca_camera_average"):
         fn = getattr(mutant, fname)
         fn.argtypes = getattr(good, fname).argtypes
         fn.restype = getattr(good, fname).restype

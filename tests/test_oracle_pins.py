@@ -400,6 +400,54 @@ def test_sca_rebatched_rows_follow_compaction():
         np.testing.assert_allclose(out[b], acc / np.maximum(hits[b], 1)[:, None], rtol=1e-14)
 
 
+def test_camera_average_is_the_mean_of_the_seeing_cameras():
+    """The average step on its own: for every query, numpy's mean over the
+    rows of the cameras whose mask sees it (each row found through idx, not
+    through pos), zero for a query no camera sees."""
+    rng = _rng(12)
+    Ncam, B, Nq, R, HD = 4, 2, 37, 2, 5
+    mask = _random_mask(rng, Ncam, B, Nq, R, 0.3)
+    mask[:, 0, 0, :] = 0          # a query no camera sees
+    mask[:, 0, 1, 0] = 1          # a query every camera sees
+    idx, _, pos, hits = oracle.sca_compact(mask)
+    rb = rng.standard_normal((B, Ncam, Nq, HD))
+    out = oracle.sca_camera_average(rb, pos, hits)
+    for b in range(B):
+        for q in range(Nq):
+            cams = [c for c in range(Ncam) if mask[c, b, q].any()]
+            rows = [rb[b, c, list(idx[b, c]).index(q)] for c in cams]
+            expect = np.mean(rows, axis=0) if rows else np.zeros(HD)
+            np.testing.assert_allclose(out[b, q], expect, rtol=1e-13, atol=1e-15)
+    assert np.all(out[0, 0] == 0.0)
+
+
+def test_camera_average_closed_forms():
+    """One seeing camera returns its row unchanged; six cameras with equal
+    rows of small integers return that row exactly; rows past a camera's
+    count are never read."""
+    Ncam, B, Nq, HD = 6, 1, 3, 4
+    mask = np.zeros((Ncam, B, Nq, 1), np.uint8)
+    mask[2, 0, 0, 0] = 1          # query 0: camera 2 only
+    mask[:, 0, 1, 0] = 1          # query 1: all six
+    _, cnt, pos, hits = oracle.sca_compact(mask)
+    rb = np.full((B, Ncam, Nq, HD), np.nan)
+    for c in range(Ncam):
+        rb[0, c, :cnt[0, c]] = 3.0
+    rb[0, 2, 0] = [1.0, -2.0, 0.5, 7.0]
+    out = oracle.sca_camera_average(rb, pos, hits)
+    np.testing.assert_array_equal(out[0, 0], [1.0, -2.0, 0.5, 7.0])
+    np.testing.assert_array_equal(out[0, 1], np.full(HD, 3.0))
+    np.testing.assert_array_equal(out[0, 2], np.zeros(HD))
+
+
+def test_camera_average_of_the_rebatched_rows_is_sca_forward():
+    t = _tiny_sca(13)
+    out, rb = oracle.sca_forward(t["value"], t["shapes"], t["starts"], t["ref"], t["mask"],
+                                 t["off"], t["logits"], coord_f32=False, return_rebatched=True)
+    _, _, pos, hits = oracle.sca_compact(t["mask"])
+    np.testing.assert_array_equal(oracle.sca_camera_average(rb, pos, hits), out)
+
+
 # --------------------------------------------------------------------------
 # backward: central finite differences and linearity
 # --------------------------------------------------------------------------
