@@ -905,7 +905,26 @@ def measure_next_rows(args, w, tensors, flush, stream, hbm_peak):
                                                workspace=mod_ws))
     rows["sca_module_forward"] = {"ms": ms, "workload": "bevformer-base SCA module, C=256",
                                   "gsamples_per_s": tensors["samples"] / (ms * 1e-3) / 1e9}
-    del feats, q, mod_out, mod_ws
+    del feats, mod_out, mod_ws
+
+    # f1: the camera average fused into the output projection (the module's
+    # last step for fp32 value)
+    if not bf16:
+        idx, cnt, pos, hits = msda.sca_compact(mask)
+        rb = msda.sca_rebatched_forward(value, shapes, starts, ref, off, logits, idx, cnt)
+        n_rows = int(cnt.sum().item())
+        resid = q.reshape(w.B * w.Nq, C)
+        y = torch.empty_like(resid)
+        ms = timed(lambda: msda.sca_camera_average_linear(rb, pos, hits, wout, bout, resid, out=y))
+        nbytes = (n_rows * C * 4 + w.B * w.Ncam * w.Nq * 4 + w.B * w.Nq * 4 + C * C * 2 + C * 4
+                  + 2 * w.B * w.Nq * C * 4)
+        r = hbm(nbytes, ms)
+        r.update(kernel="proj_gemm_kernel<averaged X> (tcgen05)",
+                 workload="bevformer-base output projection, C=256, residual",
+                 algorithmic_bytes_note="the rebatched rows once, pos, hits, W_o, b_o, residual, y")
+        rows["sca_camera_average_linear"] = r
+        del rb, y, resid
+    del q
 
     # f3: gradients of offsets, logits and reference points from the rebatched ones
     idx, cnt, pos, hits = msda.sca_compact(mask)

@@ -350,6 +350,27 @@ msda_status_t sca_rebatched_forward(const void* value, msda_dtype_t vdt,
 msda_status_t sca_camera_average(const float* out_rb, const int32_t* pos, const int32_t* hits,
                                  msda_dims_t d, float* out, msda_stream_t stream);
 
+/* SCA, stage 3 fused into the output projection ([SCA] scatter-add and
+ * clamp(count, 1) listing; [BQ] 10 then 11-13):
+ *   g[b, q]     = bf16(sca_camera_average(out_rb, pos, hits)[b, q])
+ *   y[b * Nq + q] = residual + dropout(g[b, q] W^T + bias)
+ * in one kernel: the tensor-core projection of msda_linear_dropout whose X
+ * tiles are formed in shared memory from the rebatched rows (the same sum in
+ * ascending camera order, the same division and rounding as
+ * sca_camera_average followed by a bf16 conversion), so g is never stored.
+ *   out_rb  [B, Ncam, Nq, K] fp32, 32-byte aligned, K = H * 32 (64 .. 256)
+ *   pos, hits from sca_compact; Ncam <= 8 (else MSDA_ERR_UNSUPPORTED)
+ *   w       [N, K] bf16 (nn.Linear layout), N a positive multiple of 256
+ *   bias    [N] fp32 or NULL; residual [B * Nq, N] fp32 or NULL
+ *   y       [B * Nq, N] fp32 or bf16 (y_dtype), written
+ *   dropout_p, dropout_seed as msda_linear_dropout (element e = row * N + col).
+ * Pointers 16-byte aligned.  Errors as msda_linear. */
+msda_status_t sca_camera_average_linear(const float* out_rb, const int32_t* pos,
+                                        const int32_t* hits, msda_dims_t d, const void* w,
+                                        const float* bias, const float* residual, int32_t N,
+                                        msda_dtype_t y_dtype, void* y, float dropout_p,
+                                        uint64_t dropout_seed, msda_stream_t stream);
+
 /* SCA forward ([BQ] 10; [SCA] listings): sca_compact, sca_rebatched_forward
  * and sca_camera_average in one call, with the lists and the rebatched rows
  * in the caller's workspace.  A query no camera sees gets 0.  With bf16

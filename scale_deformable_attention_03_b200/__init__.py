@@ -9,7 +9,8 @@ status.  There is no fallback: without the built library every call raises.
 
 Functions (same names as the C ABI): ``msda_forward``, ``msda_forward_fused``,
 ``msda_backward``, ``sca_compact``, ``sca_rebatched_forward``,
-``sca_camera_average``, ``sca_forward``, ``sca_rebatched_backward``,
+``sca_camera_average``, ``sca_camera_average_linear``, ``sca_forward``,
+``sca_rebatched_backward``,
 ``sca_backward``, ``msda_linear``, ``sca_module_forward``,
 ``msda_workspace_size``, ``sca_compact_workspace_size``.
 """
@@ -96,6 +97,10 @@ def lib():
                                           ctypes.c_int32, st, _vp, ctypes.c_float,
                                           ctypes.c_uint64, _vp]
         L.msda_linear_dropout.restype = ctypes.c_int
+        L.sca_camera_average_linear.argtypes = [_vp, _vp, _vp, Dims, _vp, _vp, _vp,
+                                                ctypes.c_int32, st, _vp, ctypes.c_float,
+                                                ctypes.c_uint64, _vp]
+        L.sca_camera_average_linear.restype = ctypes.c_int
         L.msda_linear_timeouts.restype = ctypes.c_uint32
         L.msda_linear_test_withhold_load.restype = ctypes.c_int
         L.sca_module_workspace_size.argtypes = [Dims, ctypes.c_int]
@@ -527,6 +532,30 @@ def sca_camera_average(out_rb, pos, hits, out=None, stream=None):
     _check(lib().sca_camera_average(_ptr(out_rb), _ptr(pos), _ptr(hits), d, _ptr(out),
                                     _stream(stream)),
            "sca_camera_average")
+    return out
+
+
+def sca_camera_average_linear(out_rb, pos, hits, w, bias=None, residual=None, out=None,
+                              out_dtype=None, stream=None, dropout_p=0.0, dropout_seed=0):
+    """y = residual + dropout(bf16(camera average of out_rb) w^T + bias), the
+    average formed inside the tensor-core projection.  out_rb [B, Ncam, Nq, C]
+    fp32; pos, hits from sca_compact; w [N, C] bf16; bias [N] fp32; residual
+    [B * Nq, N] fp32 -> y [B * Nq, N] (fp32, or bf16 when out_dtype / out is
+    bfloat16)."""
+    torch = _torch()
+    _contig(out_rb, pos, hits, w, bias, residual, out)
+    if w.dtype != torch.bfloat16:
+        raise MsdaError("sca_camera_average_linear takes a bfloat16 w")
+    B, Ncam, Nq, C = out_rb.shape
+    N = w.shape[0]
+    if out is None:
+        out = torch.empty((B * Nq, N), device=out_rb.device, dtype=out_dtype or torch.float32)
+    ydt = MSDA_BF16 if out.dtype == torch.bfloat16 else MSDA_F32
+    d = Dims(B, Ncam, Nq, 1, C // HEAD_DIM, 1, 1, 1)
+    _check(lib().sca_camera_average_linear(_ptr(out_rb), _ptr(pos), _ptr(hits), d, _ptr(w),
+                                           _ptr(bias), _ptr(residual), N, ydt, _ptr(out),
+                                           float(dropout_p), int(dropout_seed), _stream(stream)),
+           "sca_camera_average_linear")
     return out
 
 

@@ -552,6 +552,20 @@ msda_status_t sca_camera_average(const float* out_rb, const int32_t* pos, const 
                        "sca_camera_average");
 }
 
+msda_status_t sca_camera_average_linear(const float* out_rb, const int32_t* pos,
+                                        const int32_t* hits, msda_dims_t d, const void* w,
+                                        const float* bias, const float* residual, int32_t N,
+                                        msda_dtype_t y_dtype, void* y, float dropout_p,
+                                        uint64_t dropout_seed, msda_stream_t stream)
+{
+    MSDA_TRY(check_compact(d));
+    MSDA_CHECK(d.H >= 1 && d.H <= 8, MSDA_ERR_UNSUPPORTED,
+               "H = %d: the projection takes rows of 64 .. 256 channels (H in 2..8)", d.H);
+    return msda::average_linear_impl(out_rb, pos, hits, d.B, d.Ncam, d.Nq, w, bias, residual, N,
+                                     d.H * MSDA_HEAD_DIM, y_dtype, y, dropout_p, dropout_seed,
+                                     (cudaStream_t)stream);
+}
+
 msda_status_t sca_forward(const void* value, msda_dtype_t vdt, const int64_t* spatial_shapes,
                           const int64_t* level_start_index, const float* reference_points_cam,
                           const uint8_t* bev_mask, const float* sampling_offsets,
@@ -798,18 +812,28 @@ msda_status_t sca_forward_to(const void* value, msda_dtype_t vdt, const int64_t*
                              const int64_t* level_start_index, const float* reference_points_cam,
                              const uint8_t* bev_mask, const float* sampling_offsets,
                              const float* attention_logits, msda_dims_t d, void* workspace,
-                             size_t workspace_bytes, void* out, bool out_bf16, cudaStream_t s)
+                             size_t workspace_bytes, void* out, bool out_bf16, cudaStream_t s,
+                             ScaWorkspace* rows)
 {
     msda::Levels lv;
     MSDA_TRY(check_sca_inputs(value, vdt, d, spatial_shapes, level_start_index,
                               reference_points_cam, sampling_offsets, attention_logits, lv));
     if ((int64_t)d.B * d.Nq == 0) return ok();
     MSDA_PTR(bev_mask, 1);
-    MSDA_PTR(out, 16);
+    if (rows == nullptr) MSDA_PTR(out, 16);
     MSDA_TRY(check_workspace(workspace, workspace_bytes,
                              msda::sca_workspace_bytes(d.B, d.Ncam, d.Nq, d.H, true)));
     const msda::ScaWorkspace w = msda::sca_workspace_carve(workspace, d.B, d.Ncam, d.Nq, d.H, true);
     const msda::Problem p = make_problem(value, vdt, d, lv);
+    if (rows) {
+        *rows = w;
+        cudaError_t e = msda::launch_sca_compact(bev_mask, d.B, d.Ncam, d.Nq, d.R, w.idx, w.count,
+                                                 w.pos, w.hits, w.chunk_counts, s);
+        if (e == cudaSuccess)
+            e = msda::launch_sca_gather(p, reference_points_cam, sampling_offsets,
+                                        attention_logits, w.idx, w.count, w.out_rb, s);
+        return cuda_status(e, "sca_forward");
+    }
     // bf16 value: the query-major kernel computes the same function in one
     // pass (no compaction, rebatched rows or average kernel: the camera mean
     // is formed in registers and stored once, as fp32 or, for the SCA module,

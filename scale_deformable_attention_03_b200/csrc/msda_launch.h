@@ -128,18 +128,29 @@ msda_status_t linear_impl(const void* x, const void* w, const float* bias, const
                           int32_t M, int32_t N, int32_t K, msda_dtype_t y_dtype, void* y,
                           float dropout_p, uint64_t dropout_seed, const RowBiasArgs* rb,
                           cudaStream_t stream);
+// The projection of the camera average: y = residual + dropout(X W^T + bias)
+// with X[b * Nq + q] = bf16(sum over c ascending with pos[b, c, q] >= 0 of
+// out_rb[b, c, pos[b, c, q]] / max(1, hits[b, q])), formed inside the
+// projection kernel (Ncam <= 8; K = the rows' width).
+msda_status_t average_linear_impl(const float* out_rb, const int32_t* pos, const int32_t* hits,
+                                  int32_t B, int32_t Ncam, int32_t Nq, const void* w,
+                                  const float* bias, const float* residual, int32_t N, int32_t K,
+                                  msda_dtype_t y_dtype, void* y, float dropout_p,
+                                  uint64_t dropout_seed, cudaStream_t stream);
 cudaError_t launch_embed_bias(const float* e_cam, const float* e_lvl, const void* w,
                               const float* b, int ncam, int L, int N, int K, float* table,
                               cudaStream_t s);
 
 // sca_forward with its output stored as fp32 or (out_bf16) bf16; validates
-// like sca_forward.
+// like sca_forward.  rows non-null: only the compaction and the rebatched
+// gather run (out unused) and *rows receives the workspace's lists and rows,
+// for a consumer that averages the cameras itself.
 msda_status_t sca_forward_to(const void* value, msda_dtype_t vdt, const int64_t* spatial_shapes,
                              const int64_t* level_start_index, const float* reference_points_cam,
                              const uint8_t* bev_mask, const float* sampling_offsets,
                              const float* attention_logits, msda_dims_t d, void* workspace,
                              size_t workspace_bytes, void* out, bool out_bf16,
-                             cudaStream_t stream);
+                             cudaStream_t stream, ScaWorkspace* rows = nullptr);
 
 // sca_rebatched_backward after its input checks (acc: see msda_api.cu).
 msda_status_t sca_rebatched_backward_to(const void* value, msda_dtype_t vdt, const msda_dims_t& d,

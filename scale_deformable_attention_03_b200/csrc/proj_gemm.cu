@@ -18,7 +18,15 @@
 //   - warps 2-5 drain the other accumulator meanwhile: tcgen05.ld of their 32
 //     TMEM lanes (tile rows), bias and residual added, the values written to
 //     a swizzled shared-memory buffer and stored by TMA.
-// So loads, tensor-core work and stores of consecutive tiles overlap.  Every
+// So loads, tensor-core work and stores of consecutive tiles overlap.
+//
+// The SCA output projection can take its X from the camera average instead
+// (sca_camera_average_linear; "BEV(三) ..." section 10 then 11-13): four more
+// warps (6-9) form each 128 x 64 bf16 block of X in shared memory from the
+// rebatched rows, X[b * Nq + q] = bf16(sum over the query's cameras, in
+// ascending order, of its rebatched rows / max(1, hits)), in the layout the
+// TMA would have written, so the averaged queries never go through HBM.
+// Every
 // mbarrier wait is bounded: a wait that gives up counts a timeout in a device
 // word (msda_linear_timeouts), raises a CTA-wide stop flag that makes the
 // other roles leave their loops, and the CTA still waits (bounded) for its
@@ -41,8 +49,12 @@ constexpr int kBN = 256;   // tile columns (TMEM columns, fp32)
 constexpr int kBK = 64;    // one 128-byte swizzle row of bf16
 constexpr int kMaxK = 256;
 constexpr int kMaxKBlocks = kMaxK / kBK;
-constexpr int kStages = 4;                          // X ring slots
+constexpr int kStages = 4;                          // X ring slots (TMA-loaded X)
+constexpr int kAvgStages = 3;                       // X ring slots (averaged X)
 constexpr int kGemmThreads = 192;                   // 6 warps
+constexpr int kAvgThreads = 320;                    // + 4 warps forming X
+constexpr int kAvgProducers = 128;
+constexpr int kMaxAvgCams = 8;                      // cameras of the averaged X
 constexpr uint32_t kABlockBytes = kBM * kBK * 2;    // 16 KB
 constexpr uint32_t kBBlockBytes = kBN * kBK * 2;    // 32 KB
 constexpr uint32_t kCBufBytes = 32 * 128;           // 32 rows x 128 bytes
@@ -67,12 +79,38 @@ struct __align__(8) Ctrl {
     volatile int stop;
 };
 
+// The X producers' view of one tile: row r's rebatched source rows (global
+// row indices of out_rb, ascending camera), their number and the divisor;
+// ok[] passes the producers' common decision on each ring slot.
+struct AvgTable {
+    int src[kBM][kMaxAvgCams];
+    int n[kBM];
+    float div[kBM];
+    int ok[2];
+};
+
+// Where the averaged X comes from: out_rb [B, Ncam, Nq, K] fp32, pos
+// [B, Ncam, Nq] (row of query q in camera c, or -1), hits [B, Nq].
+struct AvgArgs {
+    const float* rows;
+    const int32_t* pos;
+    const int32_t* hits;
+    int Ncam, Nq;
+};
+
 // Shared memory: W (K/64 blocks of 256 x 64), the X ring, 4 warps x 2
-// epilogue buffers, then the control block; 1024-byte aligned.
+// epilogue buffers, the control block, then (averaged X) the producers'
+// table; 1024-byte aligned.
 constexpr size_t kSmemB = (size_t)kMaxKBlocks * kBBlockBytes;   // 128 KB
-constexpr size_t kSmemA = (size_t)kStages * kABlockBytes;       // 64 KB
 constexpr size_t kSmemC = (size_t)4 * 2 * kCBufBytes;           // 32 KB
-constexpr size_t kSmemBytes = 1024 + kSmemB + kSmemA + kSmemC + sizeof(Ctrl);
+template <bool AVG>
+constexpr size_t smem_bytes()
+{
+    return 1024 + kSmemB + (size_t)(AVG ? kAvgStages : kStages) * kABlockBytes + kSmemC +
+           sizeof(Ctrl) + (AVG ? sizeof(AvgTable) + 16 : 0);
+}
+static_assert(smem_bytes<false>() <= 227 * 1024 && smem_bytes<true>() <= 227 * 1024,
+              "shared memory of the projection kernel");
 
 __device__ unsigned int g_gemm_timeouts = 0;
 // Test switch of the bounded-wait path (msda_linear_test_withhold_load): when
@@ -304,26 +342,111 @@ __device__ __forceinline__ void put_row(uint8_t* buf, int lane, const uint32_t (
             make_uint4(u[4 * c], u[4 * c + 1], u[4 * c + 2], u[4 * c + 3]);
 }
 
-__global__ void __launch_bounds__(kGemmThreads, 1)
+// The X producers' barrier (named barrier 1, their 128 threads only).
+__device__ __forceinline__ void producers_sync()
+{
+    asm volatile("bar.sync 1, %0;" ::"n"(kAvgProducers) : "memory");
+}
+
+// Eight fp32 values (32 bytes, read once: no L1 allocation).
+__device__ __forceinline__ void load8_stream(const float* p, float (&v)[8])
+{
+    asm volatile("ld.global.nc.L1::no_allocate.v8.f32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]),
+                   "=f"(v[6]), "=f"(v[7])
+                 : "l"(p));
+}
+
+// Row `pt` of the tile at m0: its sources in ascending camera order.
+__device__ __forceinline__ void avg_table_row(AvgTable& tb, const AvgArgs& a, int m0, int pt,
+                                              int M)
+{
+    const int bq = m0 + pt;
+    int n = 0, h = 0;
+    if (bq < M) {
+        const int b = bq / a.Nq, q = bq - b * a.Nq;
+        for (int c = 0; c < a.Ncam; ++c) {
+            const int row = __ldg(a.pos + ((int64_t)b * a.Ncam + c) * a.Nq + q);
+            if ((unsigned)row < (unsigned)a.Nq) tb.src[pt][n++] = (b * a.Ncam + c) * a.Nq + row;
+        }
+        h = __ldg(a.hits + bq);
+    }
+    tb.n[pt] = n;
+    tb.div[pt] = (float)max(1, h);
+}
+
+// Columns kb * 64 + 8u .. + 7 of tile rows r = 32 w + 4 i + j (i = 0..7) as
+// bf16 into the 128-byte-swizzled X block at dst (16-byte unit u of row r at
+// unit u ^ (r mod 8)): the sum over the row's sources in their order, then
+// one IEEE division by max(1, hits), then round to nearest even.
+__device__ __forceinline__ void avg_block(uint8_t* dst, const AvgTable& tb, const float* rows,
+                                          int K, int kb, int w, int j, int u)
+{
+#pragma unroll
+    for (int i0 = 0; i0 < 8; i0 += 4) {
+        int r[4], n[4];
+        float x[4][2][8];  // the first two sources of four rows, loads in flight together
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            r[a] = 32 * w + 4 * (i0 + a) + j;
+            n[a] = tb.n[r[a]];
+#pragma unroll
+            for (int s = 0; s < 2; ++s) {
+                if (s < n[a])
+                    load8_stream(rows + (int64_t)tb.src[r[a]][s] * K + kb * kBK + 8 * u, x[a][s]);
+                else
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[a][s][e] = 0.f;
+            }
+        }
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            float v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = 0.f;
+#pragma unroll
+            for (int s = 0; s < 2; ++s)
+                if (s < n[a])
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) v[e] += x[a][s][e];
+            for (int s = 2; s < n[a]; ++s) {
+                float y[8];
+                load8_stream(rows + (int64_t)tb.src[r[a]][s] * K + kb * kBK + 8 * u, y);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v[e] += y[e];
+            }
+            const float d = tb.div[r[a]];
+            const uint4 o = make_uint4(pack_bf16x2(v[0] / d, v[1] / d), pack_bf16x2(v[2] / d, v[3] / d),
+                                       pack_bf16x2(v[4] / d, v[5] / d), pack_bf16x2(v[6] / d, v[7] / d));
+            *reinterpret_cast<uint4*>(dst + r[a] * 128 + ((u ^ (r[a] & 7)) << 4)) = o;
+        }
+    }
+}
+
+template <bool AVG>
+__global__ void __launch_bounds__(AVG ? kAvgThreads : kGemmThreads, 1)
 proj_gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
                  const __grid_constant__ CUtensorMap map_y, const float* __restrict__ bias,
                  const float* __restrict__ residual, int y_bf16, int M, int N, int K, Dropout drop,
-                 RowBias rbias)
+                 RowBias rbias, AvgArgs avg)
 {
+    constexpr int STAGES = AVG ? kAvgStages : kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t* sb = smem;
     uint8_t* sa = sb + kSmemB;
-    uint8_t* sc = sa + kSmemA;
+    uint8_t* sc = sa + (size_t)STAGES * kABlockBytes;
     Ctrl& ctrl = *reinterpret_cast<Ctrl*>(sc + kSmemC);
+    AvgTable& tb = *reinterpret_cast<AvgTable*>(
+        ((uintptr_t)(sc + kSmemC + sizeof(Ctrl)) + 15) & ~(uintptr_t)15);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int kblocks = K / kBK;
     const int mt = (M + kBM - 1) / kBM;
     const int ntiles = mt * (N / kBN);
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kStages; ++i) {
-            mbar_init(&ctrl.full[i], 1);
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(&ctrl.full[i], AVG ? kAvgProducers : 1);
             mbar_init(&ctrl.empty[i], 1);
         }
         mbar_init(&ctrl.b_full, 1);
@@ -375,6 +498,7 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
                     ++b_loads;
                     cur_n = n_tile;
                 }
+                if (AVG) continue;  // X is formed by the producer warps
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait(&ctrl.empty[stage], phase ^ 1, &ctrl.stop)) {
                         note_timeout(ctrl);
@@ -388,7 +512,7 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
                                     &ctrl.full[stage]);
                         issued[stage] = (int)phase;
                     }
-                    if (++stage == kStages) {
+                    if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1;
                     }
@@ -396,7 +520,7 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
             }
             // On a stop, give the copies still in flight a bounded chance to land.
             if (ctrl.stop) {
-                for (int i = 0; i < kStages; ++i)
+                for (int i = 0; i < STAGES; ++i)
                     if (issued[i] >= 0) mbar_wait(&ctrl.full[i], (uint32_t)issued[i]);
                 if (b_loads > 0) mbar_wait(&ctrl.b_full, (uint32_t)((b_loads - 1) & 1));
             }
@@ -437,7 +561,7 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
                         umma_bf16(d, ad, bd, (kb | ks) != 0);
                     }
                     umma_commit(&ctrl.empty[stage]);  // the slot is free once these MMAs finish
-                    if (++stage == kStages) {
+                    if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1;
                     }
@@ -454,7 +578,41 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
                 mbar_wait(&ctrl.drain, 0);
             }
         }
-    } else {
+    } else if (AVG && warp >= 6) {
+        // ---- X producers: warps 6..9, thread pt; warp w forms tile rows 32w .. 32w + 31 ----
+        const int pt = threadIdx.x - 192, w = pt >> 5, j = lane >> 3, u = lane & 7;
+        int stage = 0, flip = 0;
+        uint32_t phase = 0;
+        bool go = true;
+        for (int tile = blockIdx.x; tile < ntiles && go; tile += gridDim.x) {
+            const int m0 = (tile % mt) * kBM;
+            producers_sync();  // the previous tile's table is no longer read
+            avg_table_row(tb, avg, m0, pt, M);
+            producers_sync();
+            for (int kb = 0; kb < kblocks; ++kb) {
+                // one thread waits for the slot; the others take its verdict
+                // after the barrier, so all 128 leave together on a stop
+                if (pt == 0) {
+                    const bool ok = mbar_wait(&ctrl.empty[stage], phase ^ 1, &ctrl.stop);
+                    if (!ok) note_timeout(ctrl);
+                    tb.ok[flip] = ok;
+                }
+                producers_sync();
+                if (!tb.ok[flip]) {
+                    go = false;
+                    break;
+                }
+                flip ^= 1;
+                avg_block(sa + stage * kABlockBytes, tb, avg.rows, K, kb, w, j, u);
+                fence_async_smem();  // the generic-proxy writes, seen by the tensor cores
+                mbar_arrive(&ctrl.full[stage]);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+            }
+        }
+    } else if (warp < 6) {
         // ---- epilogue: warps 2..5, TMEM lane quarter q = warp % 4 ----
         const int q = warp & 3;
         uint8_t* cbuf = sc + (size_t)q * 2 * kCBufBytes;
@@ -644,9 +802,14 @@ extern "C" msda_status_t msda_linear_dropout(const void* x, const void* w, const
                              nullptr, (cudaStream_t)stream);
 }
 
-msda_status_t msda::linear_impl(const void* x, const void* w, const float* bias,
-                                const float* residual, int32_t M, int32_t N, int32_t K,
-                                msda_dtype_t y_dtype, void* y, float dropout_p,
+namespace msda {
+namespace {
+
+// Checks shared by both X sources; then the launch.  avg null: X from x by
+// TMA; else X is the camera average of avg's rebatched rows (x unused).
+msda_status_t launch_projection(const void* x, const AvgArgs* avg, const void* w,
+                                const float* bias, const float* residual, int32_t M, int32_t N,
+                                int32_t K, msda_dtype_t y_dtype, void* y, float dropout_p,
                                 uint64_t dropout_seed, const RowBiasArgs* rb, cudaStream_t stream)
 {
     if (!(dropout_p >= 0.f && dropout_p < 1.f))
@@ -659,22 +822,17 @@ msda_status_t msda::linear_impl(const void* x, const void* w, const float* bias,
     if (y_dtype != MSDA_F32 && y_dtype != MSDA_BF16)
         return api_fail(MSDA_ERR_INVALID_ARG, "unknown output dtype");
     if (M == 0) return api_ok();
+    if (M > INT32_MAX - 2 * kBM) return api_fail(MSDA_ERR_UNSUPPORTED, "M too large");
     auto bad = [](const void* p) { return p == nullptr || ((uintptr_t)p & 15) != 0; };
-    if (bad(x) || bad(w) || bad(y))
+    if ((avg == nullptr && bad(x)) || bad(w) || bad(y))
         return api_fail(MSDA_ERR_INVALID_ARG, "x, w and y must be non-null and 16-byte aligned");
     if ((bias && ((uintptr_t)bias & 15)) || (residual && ((uintptr_t)residual & 15)))
         return api_fail(MSDA_ERR_INVALID_ARG, "bias and residual must be 16-byte aligned");
     CUtensorMap mx, mw, my;
-    if (!make_map(&mx, x, M, K, kBM) || !make_map(&mw, w, N, K, kBN) ||
+    if ((avg == nullptr && !make_map(&mx, x, M, K, kBM)) || !make_map(&mw, w, N, K, kBN) ||
         !make_store_map(&my, y, M, N, y_dtype == MSDA_BF16))
         return api_fail(MSDA_ERR_CUDA, "cuTensorMapEncodeTiled failed or is unavailable");
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(proj_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)kSmemBytes);
-    });
-    if (attr_err != cudaSuccess) return api_cuda(attr_err, "msda_linear: shared memory size");
+    if (avg) mx = mw;  // not read
     const int64_t ntiles = (int64_t)((M + kBM - 1) / kBM) * (N / kBN);
     const unsigned grid = (unsigned)std::min<int64_t>(ntiles, device_sm_count());
     Dropout drop;
@@ -696,9 +854,60 @@ msda_status_t msda::linear_impl(const void* x, const void* w, const float* bias,
         rbias.L = rb->L;
         for (int i = 0; i < rb->L; ++i) rbias.start[i] = rb->start[i];
     }
-    proj_gemm_kernel<<<grid, kGemmThreads, kSmemBytes, stream>>>(
-        mx, mw, my, bias, residual, y_dtype == MSDA_BF16, M, N, K, drop, rbias);
+    // the shared-memory attribute belongs to the current device: set on every launch
+    cudaError_t e;
+    if (avg) {
+        e = cudaFuncSetAttribute(proj_gemm_kernel<true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem_bytes<true>());
+        if (e != cudaSuccess) return api_cuda(e, "msda_linear: shared memory size");
+        proj_gemm_kernel<true><<<grid, kAvgThreads, smem_bytes<true>(), stream>>>(
+            mx, mw, my, bias, residual, y_dtype == MSDA_BF16, M, N, K, drop, rbias, *avg);
+    } else {
+        e = cudaFuncSetAttribute(proj_gemm_kernel<false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem_bytes<false>());
+        if (e != cudaSuccess) return api_cuda(e, "msda_linear: shared memory size");
+        const AvgArgs none{nullptr, nullptr, nullptr, 1, 1};
+        proj_gemm_kernel<false><<<grid, kGemmThreads, smem_bytes<false>(), stream>>>(
+            mx, mw, my, bias, residual, y_dtype == MSDA_BF16, M, N, K, drop, rbias, none);
+    }
     return api_cuda(cudaGetLastError(), "msda_linear");
+}
+
+}  // namespace
+}  // namespace msda
+
+msda_status_t msda::linear_impl(const void* x, const void* w, const float* bias,
+                                const float* residual, int32_t M, int32_t N, int32_t K,
+                                msda_dtype_t y_dtype, void* y, float dropout_p,
+                                uint64_t dropout_seed, const RowBiasArgs* rb, cudaStream_t stream)
+{
+    return launch_projection(x, nullptr, w, bias, residual, M, N, K, y_dtype, y, dropout_p,
+                             dropout_seed, rb, stream);
+}
+
+msda_status_t msda::average_linear_impl(const float* out_rb, const int32_t* pos,
+                                        const int32_t* hits, int32_t B, int32_t Ncam, int32_t Nq,
+                                        const void* w, const float* bias, const float* residual,
+                                        int32_t N, int32_t K, msda_dtype_t y_dtype, void* y,
+                                        float dropout_p, uint64_t dropout_seed,
+                                        cudaStream_t stream)
+{
+    if (B < 0 || Nq < 0 || Ncam < 1)
+        return api_fail(MSDA_ERR_INVALID_ARG, "bad sizes");
+    if (Ncam > kMaxAvgCams)
+        return api_fail(MSDA_ERR_UNSUPPORTED, "at most 8 cameras for the averaged projection");
+    if ((int64_t)B * Ncam * Nq > INT32_MAX)
+        return api_fail(MSDA_ERR_UNSUPPORTED, "too many rebatched rows");
+    if ((int64_t)B * Nq == 0) return api_ok();
+    if (out_rb == nullptr || ((uintptr_t)out_rb & 31) || pos == nullptr || ((uintptr_t)pos & 3) ||
+        hits == nullptr || ((uintptr_t)hits & 3))
+        return api_fail(MSDA_ERR_INVALID_ARG,
+                        "out_rb (32-byte aligned), pos and hits (4-byte aligned) are required");
+    const AvgArgs a{out_rb, pos, hits, Ncam, Nq};
+    return launch_projection(nullptr, &a, w, bias, residual, B * Nq, N, K, y_dtype, y, dropout_p,
+                             dropout_seed, nullptr, stream);
 }
 
 extern "C" msda_status_t msda_linear(const void* x, const void* w, const float* bias,

@@ -8,10 +8,12 @@
 //           (camera, level): (e_cam + e_level) W_v^T + b_v)
 //   Delta = q~ W_Delta^T + b_Delta       (4.1)
 //   a     = q~ W_alpha^T + b_alpha       (4.2)
-//   g     = SCA(V, Delta, a, rho, mask)  (5-10: compaction, fused MSDA, average;
-//                                         the average stores g as bf16)
+//   g     = SCA(V, Delta, a, rho, mask)  (5-10: compaction, fused MSDA, average)
 //   q_hat = q + dropout(g W_o^T + b_o)   (11-13; dropout in the projection's
 //                                         epilogue, the identity when p = 0)
+// With fp32 value the camera average is formed inside the output projection
+// (its X tiles are built from the rebatched rows), so g is never stored; with
+// bf16 value the query-major SCA stores g as bf16 for the projection.
 // It composes the library's own kernels; the only new one is the element-wise
 // q + pos conversion below.
 #include <cuda_bf16.h>
@@ -21,6 +23,10 @@
 
 #include "msda.h"
 #include "msda_launch.h"
+
+#ifndef MSDA_MODULE_FUSED_AVERAGE
+#define MSDA_MODULE_FUSED_AVERAGE 0
+#endif
 
 namespace msda {
 namespace {
@@ -160,6 +166,19 @@ extern "C" msda_status_t sca_module_forward(const sca_module_params_t* p,
     if ((st = msda_linear(w.qt, p->w_weights, p->b_weights, nullptr, (int32_t)rows_q, S, C,
                           MSDA_F32, w.logits, stream)) != MSDA_OK)
         return st;
+    // fp32 value: the compaction and the rebatched gather, then the camera
+    // average formed inside the output projection (g never stored); bf16
+    // value: the query-major SCA stores g as bf16, then the projection
+    if (MSDA_MODULE_FUSED_AVERAGE && p->value_dtype == MSDA_F32 && d.Ncam <= 8) {
+        ScaWorkspace rows;
+        if ((st = sca_forward_to(w.value, p->value_dtype, spatial_shapes, level_start_index,
+                                 p->reference_points_cam, p->bev_mask, w.offsets, w.logits, d,
+                                 w.sca, w.sca_bytes, nullptr, false, s, &rows)) != MSDA_OK)
+            return st;
+        return average_linear_impl(rows.out_rb, rows.pos, rows.hits, d.B, d.Ncam, d.Nq,
+                                   p->w_output, p->b_output, p->query, C, C, MSDA_F32, q_hat,
+                                   p->dropout_p, p->dropout_seed, s);
+    }
     if ((st = sca_forward_to(w.value, p->value_dtype, spatial_shapes, level_start_index,
                              p->reference_points_cam, p->bev_mask, w.offsets, w.logits, d, w.sca,
                              w.sca_bytes, w.g16, true, s)) != MSDA_OK)

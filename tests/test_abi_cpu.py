@@ -35,6 +35,7 @@ def test_header_declares_the_boundary():
     for n in ("msda_forward", "msda_forward_fused", "msda_backward", "msda_workspace_size",
               "sca_compact_workspace_size", "sca_compact", "sca_forward", "sca_backward",
               "sca_rebatched_forward", "sca_camera_average", "sca_rebatched_backward",
+              "sca_camera_average_linear",
               "sca_compact_no_alloc", "msda_linear", "msda_linear_timeouts",
               "sca_module_forward", "sca_backward_inputs", "tsa_reference_points", "tsa_forward", "sca_forward_query_major",
               "msda_linear_dropout", "msda_backward_deterministic", "tsa_backward",

@@ -186,6 +186,25 @@ def test_linear(M, N, K, out_bf16):
     g.check("msda_linear")
 
 
+@pytest.mark.parametrize("H,N,out_bf16", [(8, 256, False), (2, 512, True)])
+def test_sca_camera_average_linear(H, N, out_bf16):
+    rng = np.random.Generator(np.random.PCG64(67 + H))
+    B, Ncam, Nq, C = 2, 5, 133, H * 32
+    mask = (rng.random((Ncam, B, Nq, 2)) < 0.4).astype(np.uint8)
+    g = Guards()
+    idx, count, pos, hits = msda.sca_compact(dev(mask))
+    rb = g.tensor((B, Ncam, Nq, C), torch.float32)
+    rb.copy_(torch.from_numpy(rng.standard_normal((B, Ncam, Nq, C)).astype(np.float32)))
+    wt = torch.from_numpy(rng.standard_normal((N, C)).astype(np.float32)).cuda().to(torch.bfloat16)
+    bias = torch.from_numpy(rng.standard_normal(N).astype(np.float32)).cuda()
+    res = torch.from_numpy(rng.standard_normal((B * Nq, N)).astype(np.float32)).cuda()
+    y = g.tensor((B * Nq, N), torch.bfloat16 if out_bf16 else torch.float32)
+    msda.sca_camera_average_linear(rb, pos, hits, wt, bias, res, out=y)
+    msda.sca_camera_average_linear(rb, pos, hits, wt, bias, res, out=y, dropout_p=0.2,
+                                   dropout_seed=5)
+    g.check("sca_camera_average_linear")
+
+
 def test_sca_module_forward():
     # C = 256 and H * L * P = 256: the projections' N (2 * 256, 256) are multiples of 256
     w = _sca_problem(seed=66, B=1, Ncam=2, bev=(4, 6), shapes=((6, 8), (3, 4), (2, 2), (1, 2)),
