@@ -49,12 +49,13 @@ constexpr int kBN = 256;   // tile columns (TMEM columns, fp32)
 constexpr int kBK = 64;    // one 128-byte swizzle row of bf16
 constexpr int kMaxK = 256;
 constexpr int kMaxKBlocks = kMaxK / kBK;
-constexpr int kStages = 4;                          // X ring slots (TMA-loaded X)
-constexpr int kAvgStages = 3;                       // X ring slots (averaged X)
+constexpr int kStages = 4;                          // X ring slots
 constexpr int kGemmThreads = 192;                   // 6 warps
-constexpr int kAvgThreads = 320;                    // + 4 warps forming X
-constexpr int kAvgProducers = 128;
+constexpr int kAvgThreads = 256;                    // + 2 warps forming X (64 rows each;
+                                                    // 8 warps keep 255 registers a thread)
+constexpr int kAvgProducers = 64;
 constexpr int kMaxAvgCams = 8;                      // cameras of the averaged X
+constexpr int kAvgRowsPerBatch = 8;                 // rows whose source loads fly together
 constexpr uint32_t kABlockBytes = kBM * kBK * 2;    // 16 KB
 constexpr uint32_t kBBlockBytes = kBN * kBK * 2;    // 32 KB
 constexpr uint32_t kCBufBytes = 32 * 128;           // 32 rows x 128 bytes
@@ -79,16 +80,6 @@ struct __align__(8) Ctrl {
     volatile int stop;
 };
 
-// The X producers' view of one tile: row r's rebatched source rows (global
-// row indices of out_rb, ascending camera), their number and the divisor;
-// ok[] passes the producers' common decision on each ring slot.
-struct AvgTable {
-    int src[kBM][kMaxAvgCams];
-    int n[kBM];
-    float div[kBM];
-    int ok[2];
-};
-
 // Where the averaged X comes from: out_rb [B, Ncam, Nq, K] fp32, pos
 // [B, Ncam, Nq] (row of query q in camera c, or -1), hits [B, Nq].
 struct AvgArgs {
@@ -99,18 +90,14 @@ struct AvgArgs {
 };
 
 // Shared memory: W (K/64 blocks of 256 x 64), the X ring, 4 warps x 2
-// epilogue buffers, the control block, then (averaged X) the producers'
-// table; 1024-byte aligned.
+// epilogue buffers, then the control block; 1024-byte aligned.
 constexpr size_t kSmemB = (size_t)kMaxKBlocks * kBBlockBytes;   // 128 KB
+constexpr size_t kSmemA = (size_t)kStages * kABlockBytes;       // 64 KB
 constexpr size_t kSmemC = (size_t)4 * 2 * kCBufBytes;           // 32 KB
-template <bool AVG>
-constexpr size_t smem_bytes()
-{
-    return 1024 + kSmemB + (size_t)(AVG ? kAvgStages : kStages) * kABlockBytes + kSmemC +
-           sizeof(Ctrl) + (AVG ? sizeof(AvgTable) + 16 : 0);
-}
-static_assert(smem_bytes<false>() <= 227 * 1024 && smem_bytes<true>() <= 227 * 1024,
-              "shared memory of the projection kernel");
+constexpr size_t kSmemBytes = 1024 + kSmemB + kSmemA + kSmemC + sizeof(Ctrl);
+static_assert(kSmemBytes <= 227 * 1024, "shared memory of the projection kernel");
+static_assert((kStages & (kStages - 1)) == 0 && kStages >= kMaxKBlocks,
+              "a tile's K-blocks fit the ring, whose size is a power of two");
 
 __device__ unsigned int g_gemm_timeouts = 0;
 // Test switch of the bounded-wait path (msda_linear_test_withhold_load): when
@@ -342,83 +329,144 @@ __device__ __forceinline__ void put_row(uint8_t* buf, int lane, const uint32_t (
             make_uint4(u[4 * c], u[4 * c + 1], u[4 * c + 2], u[4 * c + 3]);
 }
 
-// The X producers' barrier (named barrier 1, their 128 threads only).
-__device__ __forceinline__ void producers_sync()
+// Eight fp32 values (32 bytes, read once: no L1 allocation) when `on`; else
+// v keeps what it holds.  A predicated load, no branch, so that a batch's
+// loads all leave before the first is used.
+__device__ __forceinline__ void load8_stream(const float* p, bool on, float (&v)[8])
 {
-    asm volatile("bar.sync 1, %0;" ::"n"(kAvgProducers) : "memory");
+    asm volatile(
+        "{\n .reg .pred q;\n setp.ne.b32 q, %9, 0;\n"
+        " @q ld.global.nc.L1::no_allocate.v8.f32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n}\n"
+        : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]), "+f"(v[6]),
+          "+f"(v[7])
+        : "l"(p), "r"((int)on));
 }
 
-// Eight fp32 values (32 bytes, read once: no L1 allocation).
-__device__ __forceinline__ void load8_stream(const float* p, float (&v)[8])
-{
-    asm volatile("ld.global.nc.L1::no_allocate.v8.f32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-                 : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]),
-                   "=f"(v[6]), "=f"(v[7])
-                 : "l"(p));
-}
+// One tile row's sources in ascending camera order (global rows of out_rb),
+// their number and the divisor max(1, hits).
+struct AvgRow {
+    int src[kMaxAvgCams];
+    int n;
+    int div;  // max(1, hits)
+};
 
-// Row `pt` of the tile at m0: its sources in ascending camera order.
-__device__ __forceinline__ void avg_table_row(AvgTable& tb, const AvgArgs& a, int m0, int pt,
-                                              int M)
+// The raw lists of tile row bq (its camera positions and hits), loaded ahead
+// of their use.
+struct AvgRaw {
+    int pos[kMaxAvgCams];
+    int hits;
+};
+
+__device__ __forceinline__ void avg_load_raw(AvgRaw& raw, const AvgArgs& a, int bq, int M)
 {
-    const int bq = m0 + pt;
-    int n = 0, h = 0;
+#pragma unroll
+    for (int c = 0; c < kMaxAvgCams; ++c) raw.pos[c] = -1;
+    raw.hits = 0;
     if (bq < M) {
         const int b = bq / a.Nq, q = bq - b * a.Nq;
-        for (int c = 0; c < a.Ncam; ++c) {
-            const int row = __ldg(a.pos + ((int64_t)b * a.Ncam + c) * a.Nq + q);
-            if ((unsigned)row < (unsigned)a.Nq) tb.src[pt][n++] = (b * a.Ncam + c) * a.Nq + row;
-        }
-        h = __ldg(a.hits + bq);
+#pragma unroll
+        for (int c = 0; c < kMaxAvgCams; ++c)
+            if (c < a.Ncam) raw.pos[c] = __ldg(a.pos + ((int64_t)b * a.Ncam + c) * a.Nq + q);
+        raw.hits = __ldg(a.hits + bq);
     }
-    tb.n[pt] = n;
-    tb.div[pt] = (float)max(1, h);
 }
 
-// Columns kb * 64 + 8u .. + 7 of tile rows r = 32 w + 4 i + j (i = 0..7) as
-// bf16 into the 128-byte-swizzled X block at dst (16-byte unit u of row r at
-// unit u ^ (r mod 8)): the sum over the row's sources in their order, then
-// one IEEE division by max(1, hits), then round to nearest even.
-__device__ __forceinline__ void avg_block(uint8_t* dst, const AvgTable& tb, const float* rows,
-                                          int K, int kb, int w, int j, int u)
+__device__ __forceinline__ void avg_compact(AvgRow& row, const AvgRaw& raw, const AvgArgs& a,
+                                            int bq, int M)
 {
+    row.n = 0;
 #pragma unroll
-    for (int i0 = 0; i0 < 8; i0 += 4) {
-        int r[4], n[4];
-        float x[4][2][8];  // the first two sources of four rows, loads in flight together
+    for (int c = 0; c < kMaxAvgCams; ++c) row.src[c] = 0;
+    if (bq < M) {
+        const int b = bq / a.Nq;
 #pragma unroll
-        for (int a = 0; a < 4; ++a) {
-            r[a] = 32 * w + 4 * (i0 + a) + j;
-            n[a] = tb.n[r[a]];
+        for (int c = 0; c < kMaxAvgCams; ++c) {
+            if ((unsigned)raw.pos[c] < (unsigned)a.Nq) {
+                // row.n <= c: compile-time-indexed selects keep src in registers
+#pragma unroll
+                for (int k = 0; k <= c; ++k)
+                    if (k == row.n) row.src[k] = (b * a.Ncam + c) * a.Nq + raw.pos[c];
+                ++row.n;
+            }
+        }
+    }
+    row.div = max(1, raw.hits);
+}
+
+// 32 tile rows of a producer warp (tile row r0 + i is held by lane i:
+// its sources in ascending camera order as global rows of out_rb, their
+// number n and the divisor) into the X slots of the tile: lane l forms
+// channels 8l .. 8l + 7 of every row (one coalesced K * 4-byte read per
+// source row), bf16 unit l mod 8 of the row in K-block l / 8, written where
+// the 128-byte-swizzled TMA layout puts it (unit u of row r at u ^ (r mod 8)).
+// The sum runs over the sources in order from 0, then one IEEE division by
+// max(1, hits), then round to nearest even: the camera average's arithmetic.
+__device__ __forceinline__ void avg_rows(uint8_t* sa, int s0, const float* rows,
+                                         const AvgRow& t, int K, int rbase, int lane)
+{
+    const bool active = 8 * lane < K;
+    const int u = lane & 7;
+    // K-block lane / 8 sits in ring slot (s0 + lane / 8) mod 4
+    uint8_t* slot = sa + ((s0 + (lane >> 3)) & (kStages - 1)) * kABlockBytes;
+    const float* col = rows + 8 * lane;
+#pragma unroll 1
+    for (int r0 = 0; r0 < 32; r0 += kAvgRowsPerBatch) {
+        float x[kAvgRowsPerBatch][2][8];  // the first two sources of the batch's rows
+        int nr[kAvgRowsPerBatch];
+#pragma unroll
+        for (int a = 0; a < kAvgRowsPerBatch; ++a) {
+            nr[a] = __shfl_sync(0xffffffffu, t.n, r0 + a);
 #pragma unroll
             for (int s = 0; s < 2; ++s) {
-                if (s < n[a])
-                    load8_stream(rows + (int64_t)tb.src[r[a]][s] * K + kb * kBK + 8 * u, x[a][s]);
-                else
+                const int row = __shfl_sync(0xffffffffu, t.src[s], r0 + a);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) x[a][s][e] = 0.f;
+                for (int e = 0; e < 8; ++e) x[a][s][e] = 0.f;
+                load8_stream(col + (int64_t)row * K, s < nr[a] && active, x[a][s]);
             }
         }
 #pragma unroll
-        for (int a = 0; a < 4; ++a) {
+        for (int a = 0; a < kAvgRowsPerBatch; ++a) {
             float v[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) v[e] = 0.f;
 #pragma unroll
             for (int s = 0; s < 2; ++s)
-                if (s < n[a])
+                if (s < nr[a])
 #pragma unroll
                     for (int e = 0; e < 8; ++e) v[e] += x[a][s][e];
-            for (int s = 2; s < n[a]; ++s) {
-                float y[8];
-                load8_stream(rows + (int64_t)tb.src[r[a]][s] * K + kb * kBK + 8 * u, y);
+            if (nr[a] > 2) {  // warp-uniform: more than two seeing cameras
+                float y[kMaxAvgCams - 2][8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) v[e] += y[e];
+                for (int s = 2; s < kMaxAvgCams; ++s) {
+                    const int row = __shfl_sync(0xffffffffu, t.src[s], r0 + a);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) y[s - 2][e] = 0.f;
+                    load8_stream(col + (int64_t)row * K, s < nr[a] && active, y[s - 2]);
+                }
+#pragma unroll
+                for (int s = 2; s < kMaxAvgCams; ++s)
+                    if (s < nr[a])
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) v[e] += y[s - 2][e];
             }
-            const float d = tb.div[r[a]];
-            const uint4 o = make_uint4(pack_bf16x2(v[0] / d, v[1] / d), pack_bf16x2(v[2] / d, v[3] / d),
-                                       pack_bf16x2(v[4] / d, v[5] / d), pack_bf16x2(v[6] / d, v[7] / d));
-            *reinterpret_cast<uint4*>(dst + r[a] * 128 + ((u ^ (r[a] & 7)) << 4)) = o;
+            const int d = __shfl_sync(0xffffffffu, t.div, r0 + a);
+            // v / d, correctly rounded: for d a power of two the product with
+            // the exact 1 / d is the same number, without the division routine
+            if ((d & (d - 1)) == 0) {  // warp-uniform
+                const float rd = __int_as_float((127 - (31 - __clz(d))) << 23);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v[e] = __fmul_rn(v[e], rd);
+            } else {
+                const float df = (float)d;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v[e] = __fdiv_rn(v[e], df);
+            }
+            if (active) {
+                const int r = rbase + r0 + a;
+                const uint4 o = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                           pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+                *reinterpret_cast<uint4*>(slot + r * 128 + ((u ^ (r & 7)) << 4)) = o;
+            }
         }
     }
 }
@@ -430,15 +478,13 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
                  const float* __restrict__ residual, int y_bf16, int M, int N, int K, Dropout drop,
                  RowBias rbias, AvgArgs avg)
 {
-    constexpr int STAGES = AVG ? kAvgStages : kStages;
+    constexpr int STAGES = kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t* sb = smem;
     uint8_t* sa = sb + kSmemB;
-    uint8_t* sc = sa + (size_t)STAGES * kABlockBytes;
+    uint8_t* sc = sa + kSmemA;
     Ctrl& ctrl = *reinterpret_cast<Ctrl*>(sc + kSmemC);
-    AvgTable& tb = *reinterpret_cast<AvgTable*>(
-        ((uintptr_t)(sc + kSmemC + sizeof(Ctrl)) + 15) & ~(uintptr_t)15);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int kblocks = K / kBK;
     const int mt = (M + kBM - 1) / kBM;
@@ -498,23 +544,24 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
                     ++b_loads;
                     cur_n = n_tile;
                 }
-                if (AVG) continue;  // X is formed by the producer warps
-                for (int kb = 0; kb < kblocks; ++kb) {
-                    if (!mbar_wait(&ctrl.empty[stage], phase ^ 1, &ctrl.stop)) {
-                        note_timeout(ctrl);
-                        break;
-                    }
-                    if (withhold) {
-                        withhold = false;
-                    } else {
-                        mbar_expect_tx(&ctrl.full[stage], kABlockBytes);
-                        tma_load_2d(sa + stage * kABlockBytes, &map_x, kb * kBK, m0,
-                                    &ctrl.full[stage]);
-                        issued[stage] = (int)phase;
-                    }
-                    if (++stage == STAGES) {
-                        stage = 0;
-                        phase ^= 1;
+                if constexpr (!AVG) {  // else X is formed by the producer warps
+                    for (int kb = 0; kb < kblocks; ++kb) {
+                        if (!mbar_wait(&ctrl.empty[stage], phase ^ 1, &ctrl.stop)) {
+                            note_timeout(ctrl);
+                            break;
+                        }
+                        if (withhold) {
+                            withhold = false;
+                        } else {
+                            mbar_expect_tx(&ctrl.full[stage], kABlockBytes);
+                            tma_load_2d(sa + stage * kABlockBytes, &map_x, kb * kBK, m0,
+                                        &ctrl.full[stage]);
+                            issued[stage] = (int)phase;
+                        }
+                        if (++stage == STAGES) {
+                            stage = 0;
+                            phase ^= 1;
+                        }
                     }
                 }
             }
@@ -579,38 +626,51 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
             }
         }
     } else if (AVG && warp >= 6) {
-        // ---- X producers: warps 6..9, thread pt; warp w forms tile rows 32w .. 32w + 31 ----
-        const int pt = threadIdx.x - 192, w = pt >> 5, j = lane >> 3, u = lane & 7;
-        int stage = 0, flip = 0;
+        // ---- X producers: warps 6, 7; warp w forms tile rows 64w .. 64w + 63 ----
+        // Each warp works on its own: one lane waits for the tile's slots and
+        // the warp takes its verdict, so a stop leaves no warp behind.  The
+        // lists of the warp's next tile are loaded while it forms this one.
+        const int rbase = 64 * (warp - 6);
+        int stage = 0;
         uint32_t phase = 0;
-        bool go = true;
-        for (int tile = blockIdx.x; tile < ntiles && go; tile += gridDim.x) {
+        AvgRaw raw[2];
+        int tile = blockIdx.x;
+        if (tile < ntiles) {
             const int m0 = (tile % mt) * kBM;
-            producers_sync();  // the previous tile's table is no longer read
-            avg_table_row(tb, avg, m0, pt, M);
-            producers_sync();
+            avg_load_raw(raw[0], avg, m0 + rbase + lane, M);
+            avg_load_raw(raw[1], avg, m0 + rbase + 32 + lane, M);
+        }
+        for (; tile < ntiles; tile += gridDim.x) {
+            const int m0 = (tile % mt) * kBM;
+            AvgRow cur[2];
+            avg_compact(cur[0], raw[0], avg, m0 + rbase + lane, M);
+            avg_compact(cur[1], raw[1], avg, m0 + rbase + 32 + lane, M);
+            const int next = tile + gridDim.x;
+            if (next < ntiles) {
+                const int mn = (next % mt) * kBM;
+                avg_load_raw(raw[0], avg, mn + rbase + lane, M);
+                avg_load_raw(raw[1], avg, mn + rbase + 32 + lane, M);
+            }
+            // the tile's K-blocks go to the next kblocks ring slots (from s0,
+            // wrapping), as the tensor-core issuer takes them
+            const int s0 = stage;
+            bool ok = true;
             for (int kb = 0; kb < kblocks; ++kb) {
-                // one thread waits for the slot; the others take its verdict
-                // after the barrier, so all 128 leave together on a stop
-                if (pt == 0) {
-                    const bool ok = mbar_wait(&ctrl.empty[stage], phase ^ 1, &ctrl.stop);
-                    if (!ok) note_timeout(ctrl);
-                    tb.ok[flip] = ok;
-                }
-                producers_sync();
-                if (!tb.ok[flip]) {
-                    go = false;
-                    break;
-                }
-                flip ^= 1;
-                avg_block(sa + stage * kABlockBytes, tb, avg.rows, K, kb, w, j, u);
-                fence_async_smem();  // the generic-proxy writes, seen by the tensor cores
-                mbar_arrive(&ctrl.full[stage]);
+                if (lane == 0 && ok) ok = mbar_wait(&ctrl.empty[stage], phase ^ 1, &ctrl.stop);
                 if (++stage == STAGES) {
                     stage = 0;
                     phase ^= 1;
                 }
             }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) {
+                if (lane == 0) note_timeout(ctrl);
+                break;
+            }
+            avg_rows(sa, s0, avg.rows, cur[0], K, rbase, lane);
+            avg_rows(sa, s0, avg.rows, cur[1], K, rbase + 32, lane);
+            fence_async_smem();  // the generic-proxy writes, seen by the tensor cores
+            for (int kb = 0; kb < kblocks; ++kb) mbar_arrive(&ctrl.full[(s0 + kb) & (STAGES - 1)]);
         }
     } else if (warp < 6) {
         // ---- epilogue: warps 2..5, TMEM lane quarter q = warp % 4 ----
@@ -859,17 +919,17 @@ msda_status_t launch_projection(const void* x, const AvgArgs* avg, const void* w
     if (avg) {
         e = cudaFuncSetAttribute(proj_gemm_kernel<true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem_bytes<true>());
+                                 (int)kSmemBytes);
         if (e != cudaSuccess) return api_cuda(e, "msda_linear: shared memory size");
-        proj_gemm_kernel<true><<<grid, kAvgThreads, smem_bytes<true>(), stream>>>(
+        proj_gemm_kernel<true><<<grid, kAvgThreads, kSmemBytes, stream>>>(
             mx, mw, my, bias, residual, y_dtype == MSDA_BF16, M, N, K, drop, rbias, *avg);
     } else {
         e = cudaFuncSetAttribute(proj_gemm_kernel<false>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem_bytes<false>());
+                                 (int)kSmemBytes);
         if (e != cudaSuccess) return api_cuda(e, "msda_linear: shared memory size");
         const AvgArgs none{nullptr, nullptr, nullptr, 1, 1};
-        proj_gemm_kernel<false><<<grid, kGemmThreads, smem_bytes<false>(), stream>>>(
+        proj_gemm_kernel<false><<<grid, kGemmThreads, kSmemBytes, stream>>>(
             mx, mw, my, bias, residual, y_dtype == MSDA_BF16, M, N, K, drop, rbias, none);
     }
     return api_cuda(cudaGetLastError(), "msda_linear");
