@@ -35,6 +35,9 @@ namespace msda {
 #ifndef MSDA_QUAD_MIN_CTAS_BF16
 #define MSDA_QUAD_MIN_CTAS_BF16 0
 #endif
+#ifndef MSDA_QUAD_FFMA2
+#define MSDA_QUAD_FFMA2 1  // fp32 value: the corner adds as packed fp32x2 FMAs
+#endif
 #ifndef MSDA_QUAD_PREFETCH
 #define MSDA_QUAD_PREFETCH 0  // 1: load the next tile's logits and offsets during this tile
 #endif
@@ -74,8 +77,20 @@ struct QuadCorner<float> {
     }
     __device__ __forceinline__ static void fma(float (&acc)[8], float w, const Raw& r)
     {
+#if MSDA_QUAD_FFMA2
+        // two channels per instruction: fma.rn.f32x2 is two IEEE fp32 fused
+        // multiply-adds, the same results as fmaf on each
+#pragma unroll
+        for (int e = 0; e < 8; e += 2)
+            asm("{\n .reg .b64 a, c, w;\n"
+                " mov.b64 a, {%2, %3};\n mov.b64 c, {%0, %1};\n mov.b64 w, {%4, %4};\n"
+                " fma.rn.f32x2 c, w, a, c;\n mov.b64 {%0, %1}, c;\n}\n"
+                : "+f"(acc[e]), "+f"(acc[e + 1])
+                : "f"(r.v[e]), "f"(r.v[e + 1]), "f"(w));
+#else
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = fmaf(w, r.v[e], acc[e]);
+#endif
     }
 };
 
