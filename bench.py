@@ -447,7 +447,9 @@ def measure_replica(args, rank, world, barrier):
         msda._check(L.sca_camera_average(P(out_rb), P(pos), P(hits), dims, P(out), sptr),
                     "sca_camera_average")
 
-    launches_per_step = 5  # three compaction kernels, the gather, the average
+    # compaction (count, scatter; a scan pass between them above 64 chunks of
+    # 1024 queries), the gather, the average
+    launches_per_step = 4 if (w.Nq + 1023) // 1024 <= 64 else 5
     compact()
     torch.cuda.synchronize()
     rows = int(count.sum().item())

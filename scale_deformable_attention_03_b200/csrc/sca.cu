@@ -2,6 +2,7 @@
 // rebatch and average listings; "BEV(三) BEVFormer ..." section 10):
 //   K2a sca_count_kernel    hits per query, seeing queries per 1024-query chunk
 //   K2s sca_chunk_scan_kernel  per-camera prefix of the chunk counts, count
+//                              (only above 64 chunks; below, K2b sums them)
 //   K2b sca_scatter_kernel  stable ranks -> idx / pos
 //   K3  sca_gather_kernel   fused MSDA over every camera's seeing queries
 //   K4  sca_average_kernel  per-query sum over cameras / max(1, hits)
@@ -85,10 +86,17 @@ sca_chunk_scan_kernel(int32_t* __restrict__ chunk_counts, int nchunks, int32_t* 
     if (lane == 0) count[bc] = run;
 }
 
+// inline_scan (at most kInlineScanChunks chunks): the chunk counts are still
+// per chunk, and warp c sums camera c's counts of the earlier chunks and of
+// all chunks itself (chunk 0's CTA writes count), so no scan pass runs
+// between the count and scatter passes.  Otherwise chunk_base holds the scan
+// pass's exclusive prefixes and count its totals.
+constexpr int kInlineScanChunks = 64;
+
 __global__ void __launch_bounds__(kCompactChunk)
 sca_scatter_kernel(const uint8_t* __restrict__ mask, int B, int Ncam, int Nq, int R, int nchunks,
-                   const int32_t* __restrict__ chunk_base, const int32_t* __restrict__ count,
-                   int32_t* __restrict__ idx, int32_t* __restrict__ pos)
+                   const int32_t* __restrict__ chunk_base, int32_t* __restrict__ count,
+                   int32_t* __restrict__ idx, int32_t* __restrict__ pos, bool inline_scan)
 {
     __shared__ int s_base[kMaxCameras], s_total[kMaxCameras];
     __shared__ int s_wpre[kMaxCameras][32];
@@ -98,10 +106,26 @@ sca_scatter_kernel(const uint8_t* __restrict__ mask, int B, int Ncam, int Nq, in
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     // seeing queries of camera `warp` in earlier chunks, and in all chunks
-    if (warp < Ncam && lane == 0) {
+    if (warp < Ncam) {
         const int64_t bc = (int64_t)b * Ncam + warp;
-        s_base[warp] = chunk_base[bc * nchunks + chunk];
-        s_total[warp] = count[bc];
+        if (inline_scan) {
+            int before = 0, all = 0;
+            for (int i = lane; i < nchunks; i += 32) {
+                const int v = __ldg(chunk_base + bc * nchunks + i);
+                all += v;
+                if (i < chunk) before += v;
+            }
+            before = warp_sum_int(before);
+            all = warp_sum_int(all);
+            if (lane == 0) {
+                s_base[warp] = before;
+                s_total[warp] = all;
+                if (chunk == 0) count[bc] = all;
+            }
+        } else if (lane == 0) {
+            s_base[warp] = chunk_base[bc * nchunks + chunk];
+            s_total[warp] = count[bc];
+        }
     }
     uint32_t hitbits = 0;
     for (int c = 0; c < Ncam; ++c) {
@@ -143,9 +167,11 @@ cudaError_t launch_sca_compact(const uint8_t* mask, int B, int Ncam, int Nq, int
     const dim3 grid(nchunks, B);
     sca_count_kernel<<<grid, kCompactChunk, 0, s>>>(mask, B, Ncam, Nq, R, nchunks, hits,
                                                     chunk_counts);
-    sca_chunk_scan_kernel<<<B * Ncam, 32, 0, s>>>(chunk_counts, nchunks, count);
+    const bool inline_scan = nchunks <= kInlineScanChunks;
+    if (!inline_scan)
+        sca_chunk_scan_kernel<<<B * Ncam, 32, 0, s>>>(chunk_counts, nchunks, count);
     sca_scatter_kernel<<<grid, kCompactChunk, 0, s>>>(mask, B, Ncam, Nq, R, nchunks,
-                                                      chunk_counts, count, idx, pos);
+                                                      chunk_counts, count, idx, pos, inline_scan);
     return cudaGetLastError();
 }
 

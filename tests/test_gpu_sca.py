@@ -41,6 +41,9 @@ def test_compaction_workload3_bit_exact():
     ((1, 1, 31, 2), 0.5),       # less than a warp
     ((32, 1, 2048, 3), 0.05),   # the camera limit
     ((5, 2, 4097, 8), 0.02),
+    ((6, 1, 65536, 2), 0.1),    # 64 chunks: the scatter pass sums the chunk counts itself
+    ((6, 1, 65537, 2), 0.1),    # 65 chunks: the separate scan pass
+    ((2, 2, 150000, 1), 0.05),  # 147 chunks per (batch, camera)
 ])
 def test_compaction_random_bit_exact(shape, p):
     rng = np.random.Generator(np.random.PCG64(sum(shape)))
