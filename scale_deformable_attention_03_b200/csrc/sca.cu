@@ -345,18 +345,29 @@ cudaError_t launch_sca_gather(const Problem& p, const float* ref_cam, const floa
 // coalesced, four cameras' loads in flight at a time), sums them in ascending
 // camera order and divides by max(1, hits) (the clamp of the average listing).
 constexpr int kAvgWarps = 8;
+// Rows of up to 256 channels (PL <= 2): eight resident CTAs (32 registers)
+// with one camera row in flight per warp measured faster than four CTAs with
+// four rows in flight (0.0205 vs 0.0266 ms after the gather, BEVFormer-base):
+// the positions -> rows chain is latency-bound, and more warps hide it.
+#ifndef MSDA_AVG_MIN_BLOCKS
+#define MSDA_AVG_MIN_BLOCKS 8  // resident CTAs asked of the register allocation (PL <= 2)
+#endif
+#ifndef MSDA_AVG_INFLIGHT
+#define MSDA_AVG_INFLIGHT 2  // float4 per lane loaded together
+#endif
 
 // PL: float4 per lane (a power of two >= row4 / 32); rows of up to 16 heads.
-// kAvgBatch cameras' rows are loaded together (8 float4 per lane in flight).
-// BF16: the mean is stored rounded to bf16 (to nearest even), the operand
-// type of the output projection that follows it in the SCA module.
+// kAvgBatch cameras' rows are loaded together (MSDA_AVG_INFLIGHT float4 per
+// lane in flight).  BF16: the mean is stored rounded to bf16 (to nearest
+// even), the operand type of the output projection that follows it in the
+// SCA module.
 template <int PL, bool BF16>
-__global__ void __launch_bounds__(kAvgWarps * 32)
+__global__ void __launch_bounds__(kAvgWarps * 32, PL <= 2 ? MSDA_AVG_MIN_BLOCKS : 1)
 sca_average_kernel(const float4* __restrict__ out_rb, const int32_t* __restrict__ pos,
                    const int32_t* __restrict__ hits, int B, int Ncam, int Nq, int row4,
                    void* __restrict__ out)
 {
-    constexpr int kAvgBatch = PL >= 8 ? 1 : 8 / PL;
+    constexpr int kAvgBatch = PL >= MSDA_AVG_INFLIGHT ? 1 : MSDA_AVG_INFLIGHT / PL;
     const int lane = threadIdx.x & 31;
     const int64_t bq = (int64_t)blockIdx.x * kAvgWarps + (threadIdx.x >> 5);
     if (bq >= (int64_t)B * Nq) return;  // warp-uniform
@@ -396,12 +407,19 @@ sca_average_kernel(const float4* __restrict__ out_rb, const int32_t* __restrict_
                     acc[e].w += x[k][e].w;
                 }
     }
-    const float n = (float)max(1, __ldg(hits + bq));
+    const int hn = max(1, __ldg(hits + bq));
+    // division by a power of two is the product with its exact reciprocal:
+    // the same correctly rounded quotient without the division routine
+    const bool pow2 = (hn & (hn - 1)) == 0;  // warp-uniform
+    const float n = (float)hn;
+    const float rn = __int_as_float((127 - (31 - __clz(hn))) << 23);
+    auto quot = [&](float a) { return pow2 ? __fmul_rn(a, rn) : __fdiv_rn(a, n); };
 #pragma unroll
     for (int e = 0; e < PL; ++e) {
         const int v4 = lane + 32 * e;
         if (v4 < row4) {
-            const float4 m = make_float4(acc[e].x / n, acc[e].y / n, acc[e].z / n, acc[e].w / n);
+            const float4 m = make_float4(quot(acc[e].x), quot(acc[e].y), quot(acc[e].z),
+                                         quot(acc[e].w));
             if constexpr (BF16) {
                 const __nv_bfloat162 lo = __floats2bfloat162_rn(m.x, m.y);
                 const __nv_bfloat162 hi = __floats2bfloat162_rn(m.z, m.w);
