@@ -21,13 +21,13 @@
 // So loads, tensor-core work and stores of consecutive tiles overlap.
 //
 // The SCA output projection can take its X from the camera average instead
-// (sca_camera_average_linear; "BEV(三) ..." section 10 then 11-13): four more
-// warps (6-9) form each 128 x 64 bf16 block of X in shared memory from the
-// rebatched rows, X[b * Nq + q] = bf16(sum over the query's cameras, in
+// (sca_camera_average_linear; "BEV(三) ..." section 10 then 11-13): two more
+// warps (6, 7) form the tile's 128 x K bf16 rows of X in shared memory from
+// the rebatched rows, X[b * Nq + q] = bf16(sum over the query's cameras, in
 // ascending order, of its rebatched rows / max(1, hits)), in the layout the
 // TMA would have written, so the averaged queries never go through HBM.
-// Every
-// mbarrier wait is bounded: a wait that gives up counts a timeout in a device
+//
+// Every mbarrier wait is bounded: a wait that gives up counts a timeout in a device
 // word (msda_linear_timeouts), raises a CTA-wide stop flag that makes the
 // other roles leave their loops, and the CTA still waits (bounded) for its
 // copies in flight and frees its TMEM.
