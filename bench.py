@@ -744,12 +744,37 @@ def measure_next_rows(args, w, tensors, flush, stream, hbm_peak):
             msda.sca_camera_average(rb16, lists[2], lists[3], out=out)
         ms = timed(staged16)
         r = hbm(step_b16, ms)
-        r.update(kernel="sca_count + sca_chunk_scan + sca_scatter + "
+        r.update(kernel="sca_count + sca_scatter + "
                         f"{gather_kernel_name(w, True)} + sca_average",
                  workload="bevformer-base-sca-forward, bf16 value",
                  gsamples_per_s=tensors["samples"] / (ms * 1e-3) / 1e9)
         rows["sca_rebatched_step_bf16"] = r
         del vb16, ws16, cws16, rb16, lists
+
+    # the tiny single-level MSDA (16 x 16 map, 256 queries, two heads): given
+    # locations and host-softmaxed weights; launch-latency bound, so the time
+    # (not a bandwidth fraction) is the figure
+    wk = inputs.workload1()
+    a = wk.attention_logits.astype(np.float64)
+    wts1 = np.exp(a - a.max(-1, keepdims=True))
+    wts1 = (wts1 / wts1.sum(-1, keepdims=True)).astype(np.float32)
+    v1, l1, w1 = (torch.from_numpy(np.ascontiguousarray(x)).cuda()
+                  for x in (wk.value, wk.sampling_locations, wts1))
+    o1 = torch.empty((wk.B, wk.Nq, wk.H * 32), dtype=torch.float32, device="cuda")
+    ms = timed(lambda: msda.msda_forward(v1, wk.spatial_shapes, wk.level_start_index, l1, w1,
+                                         out=o1))
+    S1 = wk.H * wk.L * wk.P
+    r = {"ms": ms, "us": ms * 1e3, "workload": wk.name, "samples": wk.B * wk.Nq * S1,
+         "kernel": "msda_forward_group_kernel (rows of L·P <= 16)",
+         "note": "0.15 MB of algorithmic bytes: bound by launch latency, not by memory"}
+    if with_cpu:
+        import oracle
+        r["cpu_oracle"] = cpu_rate(
+            lambda: oracle.msda_forward(wk.value, wk.spatial_shapes, wk.level_start_index,
+                                        wk.sampling_locations, wts1),
+            wk.B * wk.Nq * S1 / 1e9, UNIT, "the whole workload")
+    rows["msda_forward_tiny"] = r
+    del v1, l1, w1, o1
 
     # the plain fused MSDA: the Deformable-DETR encoder and the TSA queues as a batch
     for name, wk, kname in (

@@ -32,6 +32,9 @@ constexpr int kMetaStride = 36;         // words per corner row of the sample ta
 constexpr int kMaxBatchCameras = 1024;  // B * Ncam limit of the SCA kernels
 
 // Build-time tuning of the gather kernels (defaults are the tuned values).
+#ifndef MSDA_BF16_FFMA2
+#define MSDA_BF16_FFMA2 1  // bf16 corner adds as packed fp32x2 FMAs (0: scalar FMAs)
+#endif
 #ifndef MSDA_GATHER_UNROLL
 #define MSDA_GATHER_UNROLL 4   // table quads unrolled in the gather loop
 #endif
@@ -321,6 +324,19 @@ struct Gather<__nv_bfloat16> {
     static constexpr int kAcc = 8;
     __device__ __forceinline__ static void fma8(float (&acc)[8], float w, uint4 r)
     {
+#if MSDA_BF16_FFMA2
+        // bf16 pair -> fp32 pair (the low half shifted up, the high half
+        // masked), then two fused multiply-adds in one fma.rn.f32x2
+        const uint32_t u[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            asm("{\n .reg .b32 lo, hi;\n .reg .b64 a, c, w;\n"
+                " shl.b32 lo, %2, 16;\n and.b32 hi, %2, 0xffff0000;\n"
+                " mov.b64 a, {lo, hi};\n mov.b64 c, {%0, %1};\n mov.b64 w, {%3, %3};\n"
+                " fma.rn.f32x2 c, w, a, c;\n mov.b64 {%0, %1}, c;\n}\n"
+                : "+f"(acc[2 * i]), "+f"(acc[2 * i + 1])
+                : "r"(u[i]), "f"(w));
+#else
         float a, b;
         bf16x2_to_f32(r.x, a, b);
         acc[0] += w * a;
@@ -334,6 +350,7 @@ struct Gather<__nv_bfloat16> {
         bf16x2_to_f32(r.w, a, b);
         acc[6] += w * a;
         acc[7] += w * b;
+#endif
     }
     // samples base .. base + cnt - 1 of the table (base a multiple of 4)
     __device__ __forceinline__ static void run(const __nv_bfloat16* __restrict__ vb,
