@@ -10,9 +10,14 @@ status.  There is no fallback: without the built library every call raises.
 Functions (same names as the C ABI): ``msda_forward``, ``msda_forward_fused``,
 ``msda_backward``, ``sca_compact``, ``sca_rebatched_forward``,
 ``sca_camera_average``, ``sca_camera_average_linear``, ``sca_forward``,
-``sca_rebatched_backward``,
-``sca_backward``, ``msda_linear``, ``sca_module_forward``,
-``msda_workspace_size``, ``sca_compact_workspace_size``.
+``sca_forward_query_major``, ``sca_rebatched_backward``, ``sca_backward``
+and ``msda_backward`` (``deterministic=True``: the fixed-point variants),
+``sca_backward_full``,
+``sca_backward_inputs``, ``tsa_reference_points``, ``tsa_forward``,
+``tsa_backward``, ``msda_linear`` (with dropout), ``sca_module_forward``,
+``msda_workspace_size``, ``sca_compact_workspace_size``; the remaining C
+entry points (workspace sizes, status strings, the no-alloc compaction, the
+GEMM's timeout counter and test switch) are reached through ``lib()``.
 """
 import ctypes
 import os
