@@ -1,0 +1,98 @@
+"""A seeded sweep over the SCA problem space: batch, cameras, BEV size, level
+count and shapes (one-pixel levels included), heads, points and anchors,
+reference points and value dtype, drawn once from a fixed generator.  Each
+problem runs every SCA entry point (the one-call forward, the staged calls,
+the query-major kernel, the training backward in both accumulation modes and
+the whole backward chain) against the oracle: fp32 value at the fp32 element
+bound, bf16 value at the bf16 bound (the oracle reading the same bf16
+values); the staged calls must equal the one-call
+forward bit for bit when both take the rebatched path, and the two grad_value
+accumulations must agree with each other within the fp32 bound.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import scale_deformable_attention_03_b200 as msda
+from scale_deformable_attention_03_b200 import inputs
+
+from .gpu_util import assert_close, dev, value_tensor
+
+pytestmark = pytest.mark.gpu
+
+
+def _draw(n, seed=2024):
+    """n problems (seed, B, Ncam, (bev_h, bev_w), shapes, H, P, R, rho)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    out = []
+    for i in range(n):
+        L = int(rng.integers(1, 5))
+        shapes = [(int(rng.integers(1, 24)), int(rng.integers(1, 24))) for _ in range(L)]
+        H = int(rng.choice([1, 2, 3, 4, 6, 8, 12, 16]))
+        R = int(rng.choice([1, 2, 4]))
+        P = R * int(rng.integers(1, 16 // R + 1))
+        out.append((3000 + i, int(rng.integers(1, 3)), int(rng.integers(1, 9)),
+                    (int(rng.integers(1, 17)), int(rng.integers(1, 17))), shapes, H, P, R,
+                    str(rng.choice(["uniform", "coherent"]))))
+    return out
+
+
+PROBLEMS = _draw(24)
+
+
+def _workload(case, bf16):
+    seed, B, Ncam, bev, shapes, H, P, R, rho = case
+    return inputs.workload3(seed=seed, B=B, Ncam=Ncam, bev_h=bev[0], bev_w=bev[1],
+                            shapes=shapes, H=H, P=P, R=R, rho=rho, same_mask=False,
+                            with_grad=True, value_dtype="bf16" if bf16 else "f32")
+
+
+@pytest.mark.parametrize("case", PROBLEMS, ids=[f"p{c[0]}" for c in PROBLEMS])
+@pytest.mark.parametrize("bf16", [False, True])
+def test_forward_entry_points(case, bf16):
+    w = _workload(case, bf16)
+    v = value_tensor(w, bf16)
+    args = (v, w.spatial_shapes, w.level_start_index, dev(w.reference_points))
+    mask, off, lg = dev(w.bev_mask), dev(w.sampling_offsets), dev(w.attention_logits)
+    whole = msda.sca_forward(*args, mask, off, lg)
+    qm = msda.sca_forward_query_major(*args, mask, off, lg)
+    idx, count, pos, hits = msda.sca_compact(mask)
+    rows = msda.sca_rebatched_forward(*args, off, lg, idx, count)
+    staged = msda.sca_camera_average(rows, pos, hits)
+    torch.cuda.synchronize()
+    ref = oracle.sca_forward(w.value, w.spatial_shapes, w.level_start_index, w.reference_points,
+                             w.bev_mask, w.sampling_offsets, w.attention_logits)
+    assert_close(whole, ref, bf16, "sca_forward")
+    assert_close(qm, ref, bf16, "sca_forward_query_major")
+    assert_close(staged, ref, bf16, "staged forward")
+    if not bf16:  # both take the rebatched path: the same kernels, the same bits
+        assert torch.equal(staged, whole)
+
+
+@pytest.mark.parametrize("case", PROBLEMS, ids=[f"p{c[0]}" for c in PROBLEMS])
+@pytest.mark.parametrize("bf16", [False, True])
+def test_backward_entry_points(case, bf16):
+    w = _workload(case, bf16)
+    args = (value_tensor(w, bf16), w.spatial_shapes, w.level_start_index,
+            dev(w.reference_points), dev(w.bev_mask), dev(w.sampling_offsets),
+            dev(w.attention_logits), dev(w.grad_out))
+    gv, gl, gw = msda.sca_backward(*args)
+    gvd, gld, gwd = msda.sca_backward(*args, deterministic=True)
+    full = msda.sca_backward_full(*args)
+    torch.cuda.synchronize()
+    rv, rl, rw = oracle.sca_backward(w.value, w.spatial_shapes, w.level_start_index,
+                                     w.reference_points, w.bev_mask, w.sampling_offsets,
+                                     w.attention_logits, w.grad_out)
+    for name, g, r in (("grad_value", gv, rv), ("grad_sampling_locations_rb", gl, rl),
+                       ("grad_attention_weights_rb", gw, rw),
+                       ("deterministic grad_value", gvd, rv),
+                       ("deterministic grad_sampling_locations_rb", gld, rl),
+                       ("deterministic grad_attention_weights_rb", gwd, rw)):
+        assert_close(g, r, bf16, name)
+    assert_close(gv, gvd.cpu().numpy(), False, "atomic vs fixed-point grad_value")
+    want = (rv,) + tuple(oracle.sca_backward_inputs(w.spatial_shapes, w.bev_mask,
+                                                    w.attention_logits, rl, rw))
+    for g, r, name in zip(full, want, ("grad_value", "grad_sampling_offsets",
+                                       "grad_attention_logits", "grad_reference_points_cam")):
+        assert_close(g, r, bf16, f"sca_backward_full {name}")
