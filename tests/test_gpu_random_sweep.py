@@ -1,4 +1,4 @@
-"""A seeded sweep over the SCA problem space: batch, cameras, BEV size, level
+"""Seeded sweeps over the problem space.  SCA: batch, cameras, BEV size, level
 count and shapes (one-pixel levels included), heads, points and anchors,
 reference points and value dtype, drawn once from a fixed generator.  Each
 problem runs every SCA entry point (the one-call forward, the staged calls,
@@ -7,7 +7,10 @@ the whole backward chain) against the oracle: fp32 value at the fp32 element
 bound, bf16 value at the bf16 bound (the oracle reading the same bf16
 values); the staged calls must equal the one-call
 forward bit for bit when both take the rebatched path, and the two grad_value
-accumulations must agree with each other within the fp32 bound.
+accumulations must agree with each other within the fp32 bound.  Plain MSDA:
+batch, queries, heads, levels, points and anchors, locations partly outside
+their levels, through msda_forward, msda_forward_fused and msda_backward (both
+accumulation modes).
 """
 import numpy as np
 import pytest
@@ -96,3 +99,62 @@ def test_backward_entry_points(case, bf16):
     for g, r, name in zip(full, want, ("grad_value", "grad_sampling_offsets",
                                        "grad_attention_logits", "grad_reference_points_cam")):
         assert_close(g, r, bf16, f"sca_backward_full {name}")
+
+
+def _draw_msda(n, seed=2025):
+    """n plain-MSDA problems (seed, B, Nq, H, shapes, P, R)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    out = []
+    for i in range(n):
+        L = int(rng.integers(1, 5))
+        shapes = [(int(rng.integers(1, 24)), int(rng.integers(1, 24))) for _ in range(L)]
+        R = int(rng.choice([1, 2, 4]))
+        P = R * int(rng.integers(1, 16 // R + 1))
+        out.append((4000 + i, int(rng.integers(1, 4)), int(rng.integers(1, 300)),
+                    int(rng.choice([1, 2, 3, 4, 5, 8, 12, 16])), shapes, P, R))
+    return out
+
+
+MSDA_PROBLEMS = _draw_msda(24)
+
+
+@pytest.mark.parametrize("case", MSDA_PROBLEMS, ids=[f"m{c[0]}" for c in MSDA_PROBLEMS])
+@pytest.mark.parametrize("bf16", [False, True])
+def test_msda_entry_points(case, bf16):
+    """msda_forward (given locations and weights; about a third of the
+    locations lie partly or wholly outside their level), msda_forward_fused,
+    msda_backward in both accumulation modes, against the oracle."""
+    seed, B, Nq, H, shapes, P, R = case
+    rng = np.random.Generator(np.random.PCG64(seed))
+    s, starts, Nv = inputs.level_table(shapes)
+    L = len(shapes)
+    value = rng.standard_normal((B, Nv, H, 32)).astype(np.float32)
+    if bf16:
+        bits = inputs.to_bf16_bits(value)
+        value = inputs.bf16_bits_to_f32(bits)
+        vt = dev(bits.view(np.int16)).view(torch.bfloat16)
+    else:
+        vt = dev(value)
+    loc = rng.uniform(-0.2, 1.2, (B, Nq, H, L, P, 2)).astype(np.float32)
+    logits = rng.standard_normal((B, Nq, H, L, P)).astype(np.float32)
+    weights = oracle.softmax(logits, L * P).reshape(logits.shape).astype(np.float32)
+    ref = rng.uniform(-0.2, 1.2, (B, Nq, R, 2)).astype(np.float32)
+    off = (rng.standard_normal((B, Nq, H, L, P, 2)) * 3).astype(np.float32)
+    gout = rng.standard_normal((B, Nq, H * 32)).astype(np.float32)
+
+    out = msda.msda_forward(vt, s, starts, dev(loc), dev(weights))
+    fused = msda.msda_forward_fused(vt, s, starts, dev(ref), dev(off), dev(logits))
+    gv, gl, gw = msda.msda_backward(vt, s, starts, dev(loc), dev(weights), dev(gout))
+    gvd, gld, gwd = msda.msda_backward(vt, s, starts, dev(loc), dev(weights), dev(gout),
+                                       deterministic=True)
+    torch.cuda.synchronize()
+    assert_close(out, oracle.msda_forward(value, s, starts, loc, weights), bf16, "msda_forward")
+    assert_close(fused, oracle.msda_forward_fused(value, s, starts, ref, off, logits), bf16,
+                 "msda_forward_fused")
+    rv, rl, rw = oracle.msda_backward(value, s, starts, loc, weights, gout)
+    for name, g, r in (("grad_value", gv, rv), ("grad_sampling_locations", gl, rl),
+                       ("grad_attention_weights", gw, rw),
+                       ("deterministic grad_value", gvd, rv),
+                       ("deterministic grad_sampling_locations", gld, rl),
+                       ("deterministic grad_attention_weights", gwd, rw)):
+        assert_close(g, r, bf16, name)
