@@ -878,10 +878,10 @@ constexpr int kBwdGroupRowsPerTile = MSDA_GROUP_ROWS_PER_TILE;
 // TSA: rows are (b * T + t, q), each queue receiving grad_out[b] / T.  MSDA
 // (T = 1, !FUSED): rows are (b, q) with the locations and weights given.
 // Register budget: rows of up to four samples (eight heads per warp) run
-// fastest at four CTAs per SM despite small spills (TSA backward 0.48 ->
-// 0.43 ms), longer rows at three.
+// fastest at five CTAs per SM despite spills (TSA backward 0.48 -> 0.43 ms
+// at four, 0.425 ms at five; six gained nothing more), longer rows at three.
 #ifndef MSDA_BWD_GROUP4_MIN_CTAS
-#define MSDA_BWD_GROUP4_MIN_CTAS 4
+#define MSDA_BWD_GROUP4_MIN_CTAS 5
 #endif
 #ifndef MSDA_BWD_GROUP_MIN_CTAS
 #define MSDA_BWD_GROUP_MIN_CTAS 3
