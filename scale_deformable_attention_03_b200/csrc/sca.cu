@@ -362,7 +362,7 @@ constexpr int kAvgWarps = 8;
 // even), the operand type of the output projection that follows it in the
 // SCA module.
 template <int PL, bool BF16>
-__global__ void __launch_bounds__(kAvgWarps * 32, PL <= 2 ? MSDA_AVG_MIN_BLOCKS : 1)
+__global__ void __launch_bounds__(kAvgWarps * 32, PL <= 2 ? MSDA_AVG_MIN_BLOCKS : 0)
 sca_average_kernel(const float4* __restrict__ out_rb, const int32_t* __restrict__ pos,
                    const int32_t* __restrict__ hits, int B, int Ncam, int Nq, int row4,
                    void* __restrict__ out)

@@ -46,7 +46,7 @@ constexpr int kIgHeads = 8;
 #endif
 
 template <int NC, bool REF>
-__global__ void __launch_bounds__(kIgWarps * 32, NC == 1 ? MSDA_IG_MIN_BLOCKS : 1)
+__global__ void __launch_bounds__(kIgWarps * 32, NC == 1 ? MSDA_IG_MIN_BLOCKS : 0)
 sca_offset_logit_grads_kernel(const float* __restrict__ logits, const int32_t* __restrict__ pos,
                               const float* __restrict__ grad_loc_rb,
                               const float* __restrict__ grad_loc_lo_rb,
