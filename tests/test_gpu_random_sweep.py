@@ -1,6 +1,7 @@
 """Seeded sweeps over the problem space.  SCA: batch, cameras, BEV size, level
 count and shapes (one-pixel levels included), heads, points and anchors,
-reference points and value dtype, drawn once from a fixed generator.  Each
+reference points and value dtype, drawn once from a fixed generator, plus two
+problems at the compiled limits (L = 8, P = 16, 32 cameras; B * Ncam = 1024).  Each
 problem runs every SCA entry point (the one-call forward, the staged calls,
 the query-major kernel, the training backward in both accumulation modes and
 the whole backward chain) against the oracle: fp32 value at the fp32 element
@@ -41,7 +42,16 @@ def _draw(n, seed=2024):
     return out
 
 
-PROBLEMS = _draw(24)
+# The compiled limits, beside the drawn problems: eight levels of sixteen
+# points (rows of 128 samples, four sample chunks) with sixteen anchors over 32
+# cameras, and B * Ncam = 1024 batch-cameras (the largest row-prefix table).
+LIMITS = [
+    (3900, 1, 32, (4, 5), [(9, 11), (7, 8), (5, 6), (4, 4), (3, 3), (2, 2), (1, 2), (1, 1)],
+     2, 16, 16, "uniform"),
+    (3901, 32, 32, (2, 3), [(3, 4)], 1, 2, 2, "uniform"),
+]
+
+PROBLEMS = _draw(24) + LIMITS
 
 
 def _workload(case, bf16):
