@@ -718,8 +718,8 @@ def measure_next_rows(args, w, tensors, flush, stream, hbm_peak):
     rows["sca_forward_query_major"] = r
 
     # the same SCA forward with bf16 value (BEVFormer-base's bf16 variant):
-    # sca_forward (which takes the query-major kernel for bf16 value) and the
-    # rebatched steps (compaction, head-pair gather, camera average)
+    # sca_forward (compaction, head-pair gather, camera average) and the
+    # query-major kernel
     if not bf16:
         vb16 = value.to(torch.bfloat16)  # round to nearest even, as the inputs module does
         step_b16 = tensors["step_bytes"] - w.value.size * 2
@@ -728,28 +728,19 @@ def measure_next_rows(args, w, tensors, flush, stream, hbm_peak):
         ms = timed(lambda: msda.sca_forward(vb16, shapes, starts, ref, mask, off, logits,
                                             out=out, workspace=ws16))
         r = hbm(step_b16, ms)
-        r.update(kernel="sca_query_major_kernel<bf16, 1, 2> (sca_forward's bf16 path)",
+        r.update(kernel="sca_count + sca_scatter + "
+                        f"{gather_kernel_name(w, True)} + sca_average (sca_forward's bf16 path)",
                  workload="bevformer-base-sca-forward, bf16 value",
                  gsamples_per_s=tensors["samples"] / (ms * 1e-3) / 1e9)
         rows["sca_forward_bf16"] = r
-        cws16 = torch.empty(max(16, msda.sca_compact_workspace_size(dims16)), dtype=torch.uint8,
-                            device="cuda")
-        lists = msda.sca_compact(mask, workspace=cws16)
-        rb16 = torch.empty((w.B, w.Ncam, w.Nq, w.H * 32), dtype=torch.float32, device="cuda")
-
-        def staged16():
-            msda.sca_compact(mask, workspace=cws16, out=lists)
-            msda.sca_rebatched_forward(vb16, shapes, starts, ref, off, logits, lists[0],
-                                       lists[1], out_rb=rb16)
-            msda.sca_camera_average(rb16, lists[2], lists[3], out=out)
-        ms = timed(staged16)
+        ms = timed(lambda: msda.sca_forward_query_major(vb16, shapes, starts, ref, mask, off,
+                                                        logits, out=out))
         r = hbm(step_b16, ms)
-        r.update(kernel="sca_count + sca_scatter + "
-                        f"{gather_kernel_name(w, True)} + sca_average",
+        r.update(kernel="sca_query_major_kernel<bf16, 1, 2>",
                  workload="bevformer-base-sca-forward, bf16 value",
                  gsamples_per_s=tensors["samples"] / (ms * 1e-3) / 1e9)
-        rows["sca_rebatched_step_bf16"] = r
-        del vb16, ws16, cws16, rb16, lists
+        rows["sca_forward_query_major_bf16"] = r
+        del vb16, ws16
 
     # the tiny single-level MSDA (16 x 16 map, 256 queries, two heads): given
     # locations and host-softmaxed weights; launch-latency bound, so the time

@@ -373,11 +373,8 @@ msda_status_t sca_camera_average_linear(const float* out_rb, const int32_t* pos,
 
 /* SCA forward ([BQ] 10; [SCA] listings): sca_compact, sca_rebatched_forward
  * and sca_camera_average in one call, with the lists and the rebatched rows
- * in the caller's workspace.  A query no camera sees gets 0.  With bf16
- * value the same function is computed by the query-major kernel of
- * sca_forward_query_major (faster there; the workspace is then unused), so
- * the fp32 and bf16 results round differently (both within the oracle's
- * bounds). */
+ * in the caller's workspace, bit for bit the result of those three calls.
+ * A query no camera sees gets 0. */
 /*   value                [B, Ncam, Nv, H, 32]   fp32 or bf16
  *   reference_points_cam [Ncam, B, Nq, R, 2]    fp32
  *   bev_mask             [Ncam, B, Nq, R]       uint8

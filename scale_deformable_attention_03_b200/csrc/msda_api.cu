@@ -804,8 +804,12 @@ msda_status_t api_cuda(cudaError_t e, const char* where) { return cuda_status(e,
 
 namespace msda {
 
+// 1: bf16 value takes the query-major kernel (one pass: no compaction,
+// rebatched rows or average kernel; the camera mean formed in registers).
+// On the BEVFormer-base step the rebatched kernels are faster for both value
+// types (bf16: 0.377 against 0.390 ms), so both take them.
 #ifndef MSDA_SCA_FORWARD_QM_BF16
-#define MSDA_SCA_FORWARD_QM_BF16 1
+#define MSDA_SCA_FORWARD_QM_BF16 0
 #endif
 
 msda_status_t sca_forward_to(const void* value, msda_dtype_t vdt, const int64_t* spatial_shapes,
@@ -834,11 +838,9 @@ msda_status_t sca_forward_to(const void* value, msda_dtype_t vdt, const int64_t*
                                         attention_logits, w.idx, w.count, w.out_rb, s);
         return cuda_status(e, "sca_forward");
     }
-    // bf16 value: the query-major kernel computes the same function in one
-    // pass (no compaction, rebatched rows or average kernel: the camera mean
-    // is formed in registers and stored once, as fp32 or, for the SCA module,
-    // as the bf16 operand of the output projection) and measured faster there
-    // (0.401 vs 0.424 ms on the BEVFormer-base step)
+    // the query-major kernel computes the same function (the camera mean is
+    // stored once, as fp32 or, for the SCA module, as the bf16 operand of the
+    // output projection)
     if (MSDA_SCA_FORWARD_QM_BF16 && vdt == MSDA_BF16)
         return cuda_status(msda::launch_sca_query_major(p, reference_points_cam, bev_mask,
                                                         sampling_offsets, attention_logits, out,

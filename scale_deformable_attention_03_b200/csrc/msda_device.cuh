@@ -24,6 +24,14 @@
 
 namespace msda {
 
+// Programmatic dependent launch (see launch_pdl): let the next kernel in the
+// stream begin launching, and wait for the kernel before this one.
+__device__ __forceinline__ void pdl_trigger()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 constexpr int kHeadDim = 32;
 constexpr int kMaxLevels = 8;
 constexpr int kWarps = 8;               // warps per CTA

@@ -40,13 +40,36 @@ ScaWorkspace sca_workspace_carve(void* base, int B, int Ncam, int Nq, int H, boo
 
 int device_sm_count();
 
+// Programmatic dependent launch: the kernel may begin while the kernel before
+// it in the stream is still running, once every CTA of that kernel has
+// executed pdl_trigger() (or exited).  The kernel must call pdl_wait(), which
+// returns when that grid has completed and its writes are visible, before it
+// reads anything an earlier kernel wrote or writes anything an earlier kernel
+// reads.  After a kernel that never triggers, it starts as an ordinary launch.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args&&... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // K1 / K1f: msda_forward (given locations, weights) and msda_forward_fused.
 cudaError_t launch_msda_forward(const Problem& p, const float* loc, const float* attn,
                                 float* out, cudaStream_t s);
 cudaError_t launch_msda_forward_fused(const Problem& p, const float* ref, const float* off,
                                       const float* logits, float* out, cudaStream_t s);
 
-// K2: compaction (two launches).
+// K2: compaction (two launches; three above 64 chunks of 1024 queries).
 cudaError_t launch_sca_compact(const uint8_t* mask, int B, int Ncam, int Nq, int R,
                                int32_t* idx, int32_t* count, int32_t* pos, int32_t* hits,
                                int32_t* chunk_counts, cudaStream_t s);

@@ -1,9 +1,9 @@
 // SCA forward pieces (Tencent Cloud "Spatial Cross-Attention" walkthrough,
 // rebatch and average listings; "BEV(三) BEVFormer ..." section 10):
-//   K2a sca_count_kernel    hits per query, seeing queries per 1024-query chunk
+//   K2a sca_count_kernel    seeing queries per (1024-query chunk, camera)
 //   K2s sca_chunk_scan_kernel  per-camera prefix of the chunk counts, count
 //                              (only above 64 chunks; below, K2b sums them)
-//   K2b sca_scatter_kernel  stable ranks -> idx / pos
+//   K2b sca_scatter_kernel  stable ranks -> idx / pos, hits per query
 //   K3  sca_gather_kernel   fused MSDA over every camera's seeing queries
 //   K4  sca_average_kernel  per-query sum over cameras / max(1, hits)
 // Nothing here synchronises with the host: the rebatched row counts live in
@@ -15,7 +15,6 @@
 
 namespace msda {
 
-constexpr int kMaxCameras = 32;
 constexpr int kScaRowsPerTile = MSDA_ROWS_PER_TILE;  // <= 32: a lane resolves each row
 
 __device__ __forceinline__ int warp_sum_int(int v)
@@ -35,35 +34,46 @@ __device__ __forceinline__ int warp_inclusive_scan(int v, int lane)
     return v;
 }
 
-// A camera sees query q when any of its R anchor bytes is non-zero.
-__device__ __forceinline__ bool seen(const uint8_t* __restrict__ mask, int64_t at, int R)
+// A camera sees query q when any of its R anchor bytes is non-zero.  With
+// `word` (R = 1, 2, 4 or 8 and the mask aligned to R bytes) the R bytes are
+// read as one word.
+__device__ __forceinline__ bool seen(const uint8_t* __restrict__ mask, int64_t at, int R,
+                                     bool word)
 {
+    const uint8_t* p = mask + at * R;
+    if (word) {
+        switch (R) {
+            case 1: return __ldg(p) != 0;
+            case 2: return __ldg(reinterpret_cast<const unsigned short*>(p)) != 0;
+            case 4: return __ldg(reinterpret_cast<const unsigned int*>(p)) != 0;
+            case 8: return __ldg(reinterpret_cast<const unsigned long long*>(p)) != 0;
+            default: break;
+        }
+    }
     bool hit = false;
-    for (int r = 0; r < R; ++r) hit |= __ldg(mask + at * R + r) != 0;
+    for (int r = 0; r < R; ++r) hit |= __ldg(p + r) != 0;
     return hit;
 }
 
+// One CTA per (1024-query chunk, batch-camera): the camera's seeing queries
+// in the chunk.
 __global__ void __launch_bounds__(kCompactChunk)
-sca_count_kernel(const uint8_t* __restrict__ mask, int B, int Ncam, int Nq, int R, int nchunks,
-                 int32_t* __restrict__ hits, int32_t* __restrict__ chunk_counts)
+sca_count_kernel(const uint8_t* __restrict__ mask, int B, int Ncam, int Nq, int R, bool word,
+                 int nchunks, int32_t* __restrict__ chunk_counts)
 {
-    __shared__ int s_cnt[kMaxCameras][32];
-    const int chunk = blockIdx.x, b = blockIdx.y;
+    __shared__ int s_cnt[kCompactChunk / 32];
+    pdl_trigger();  // the scatter pass reads the counts only after its pdl_wait
+    const int chunk = blockIdx.x, bc = blockIdx.y;
+    const int b = bc / Ncam, c = bc - b * Ncam;
     const int q = chunk * kCompactChunk + threadIdx.x;
-    const bool valid = q < Nq;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    int nh = 0;
-    for (int c = 0; c < Ncam; ++c) {
-        const bool hit = valid && seen(mask, ((int64_t)c * B + b) * Nq + q, R);
-        nh += hit;
-        const unsigned bal = __ballot_sync(0xffffffffu, hit);
-        if (lane == 0) s_cnt[c][warp] = __popc(bal);
-    }
-    if (valid) hits[(int64_t)b * Nq + q] = nh;
+    const bool hit = q < Nq && seen(mask, ((int64_t)c * B + b) * Nq + q, R, word);
+    const unsigned bal = __ballot_sync(0xffffffffu, hit);
+    if (lane == 0) s_cnt[warp] = __popc(bal);
     __syncthreads();
-    if (warp < Ncam) {
-        const int v = warp_sum_int(s_cnt[warp][lane]);
-        if (lane == 0) chunk_counts[((int64_t)b * Ncam + warp) * nchunks + chunk] = v;
+    if (warp == 0) {
+        const int v = warp_sum_int(lane < kCompactChunk / 32 ? s_cnt[lane] : 0);
+        if (lane == 0) chunk_counts[(int64_t)bc * nchunks + chunk] = v;
     }
 }
 
@@ -87,74 +97,81 @@ sca_chunk_scan_kernel(int32_t* __restrict__ chunk_counts, int nchunks, int32_t* 
 }
 
 // inline_scan (at most kInlineScanChunks chunks): the chunk counts are still
-// per chunk, and warp c sums camera c's counts of the earlier chunks and of
-// all chunks itself (chunk 0's CTA writes count), so no scan pass runs
+// per chunk, and warp 0 sums the camera's counts of the earlier chunks and of
+// all chunks itself (the chunk-0 CTA writes count), so no scan pass runs
 // between the count and scatter passes.  Otherwise chunk_base holds the scan
 // pass's exclusive prefixes and count its totals.
 constexpr int kInlineScanChunks = 64;
 
+// One CTA per (chunk, batch-camera), as the count pass: the stable ranks of
+// the camera's seeing queries -> idx / pos; the camera-0 CTAs also write the
+// queries' hit counts.
 __global__ void __launch_bounds__(kCompactChunk)
-sca_scatter_kernel(const uint8_t* __restrict__ mask, int B, int Ncam, int Nq, int R, int nchunks,
-                   const int32_t* __restrict__ chunk_base, int32_t* __restrict__ count,
-                   int32_t* __restrict__ idx, int32_t* __restrict__ pos, bool inline_scan)
+sca_scatter_kernel(const uint8_t* __restrict__ mask, int B, int Ncam, int Nq, int R, bool word,
+                   int nchunks, const int32_t* __restrict__ chunk_base, int32_t* __restrict__ count,
+                   int32_t* __restrict__ idx, int32_t* __restrict__ pos, int32_t* __restrict__ hits,
+                   bool inline_scan)
 {
-    __shared__ int s_base[kMaxCameras], s_total[kMaxCameras];
-    __shared__ int s_wpre[kMaxCameras][32];
-    const int chunk = blockIdx.x, b = blockIdx.y;
+    __shared__ int s_base, s_total;
+    __shared__ int s_wpre[kCompactChunk / 32];
+    const int chunk = blockIdx.x, bc = blockIdx.y;
+    const int b = bc / Ncam, c = bc - b * Ncam;
     const int q = chunk * kCompactChunk + threadIdx.x;
     const bool valid = q < Nq;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // seeing queries of camera `warp` in earlier chunks, and in all chunks
-    if (warp < Ncam) {
-        const int64_t bc = (int64_t)b * Ncam + warp;
+    pdl_trigger();  // the gather reads the lists only after its pdl_wait
+    // the mask part first: it does not depend on the passes before
+    const bool hit = valid && seen(mask, ((int64_t)c * B + b) * Nq + q, R, word);
+    const unsigned bal = __ballot_sync(0xffffffffu, hit);
+    if (lane == 0) s_wpre[warp] = __popc(bal);
+    int nh = hit;
+    if (c == 0 && valid) {  // the query's seeing cameras, once per (b, q)
+#pragma unroll 4
+        for (int c2 = 1; c2 < Ncam; ++c2)
+            nh += seen(mask, ((int64_t)c2 * B + b) * Nq + q, R, word);
+    }
+    // a programmatic dependent of the count (or scan) pass: the counts are
+    // read, and the outputs written, only after that grid has completed
+    pdl_wait();
+    if (c == 0 && valid) hits[(int64_t)b * Nq + q] = nh;
+    // seeing queries of the camera in earlier chunks, and in all chunks
+    if (warp == 0) {
         if (inline_scan) {
             int before = 0, all = 0;
             for (int i = lane; i < nchunks; i += 32) {
-                const int v = __ldg(chunk_base + bc * nchunks + i);
+                const int v = __ldg(chunk_base + (int64_t)bc * nchunks + i);
                 all += v;
                 if (i < chunk) before += v;
             }
             before = warp_sum_int(before);
             all = warp_sum_int(all);
             if (lane == 0) {
-                s_base[warp] = before;
-                s_total[warp] = all;
+                s_base = before;
+                s_total = all;
                 if (chunk == 0) count[bc] = all;
             }
         } else if (lane == 0) {
-            s_base[warp] = chunk_base[bc * nchunks + chunk];
-            s_total[warp] = count[bc];
+            s_base = chunk_base[(int64_t)bc * nchunks + chunk];
+            s_total = count[bc];
         }
     }
-    uint32_t hitbits = 0;
-    for (int c = 0; c < Ncam; ++c) {
-        const bool hit = valid && seen(mask, ((int64_t)c * B + b) * Nq + q, R);
-        hitbits |= (uint32_t)hit << c;
-        const unsigned bal = __ballot_sync(0xffffffffu, hit);
-        if (lane == 0) s_wpre[c][warp] = __popc(bal);
+    __syncthreads();
+    if (warp == 0) {  // exclusive scan of the per-warp counts
+        const int v = s_wpre[lane];
+        s_wpre[lane] = warp_inclusive_scan(v, lane) - v;
     }
     __syncthreads();
-    if (warp < Ncam) {  // exclusive scan of the per-warp counts of camera `warp`
-        const int v = s_wpre[warp][lane];
-        s_wpre[warp][lane] = warp_inclusive_scan(v, lane) - v;
-    }
-    __syncthreads();
-    const unsigned below = (1u << lane) - 1u;
-    for (int c = 0; c < Ncam; ++c) {
-        const bool hit = (hitbits >> c) & 1u;
-        const unsigned bal = __ballot_sync(0xffffffffu, hit);
-        const int64_t bc = (int64_t)b * Ncam + c;
-        if (valid) {
-            if (hit) {
-                const int r = s_base[c] + s_wpre[c][warp] + __popc(bal & below);
-                idx[bc * Nq + r] = q;
-                pos[bc * Nq + q] = r;
-            } else {
-                pos[bc * Nq + q] = -1;
-            }
-            if (q >= s_total[c]) idx[bc * Nq + q] = -1;
+    if (valid) {
+        const int64_t row0 = (int64_t)bc * Nq;
+        if (hit) {
+            const int r = s_base + s_wpre[warp] + __popc(bal & ((1u << lane) - 1u));
+            idx[row0 + r] = q;
+            pos[row0 + q] = r;
+        } else {
+            pos[row0 + q] = -1;
         }
+        if (q >= s_total) idx[row0 + q] = -1;
     }
 }
 
@@ -164,15 +181,16 @@ cudaError_t launch_sca_compact(const uint8_t* mask, int B, int Ncam, int Nq, int
 {
     if (B == 0) return cudaSuccess;
     const int nchunks = Nq > 0 ? (Nq + kCompactChunk - 1) / kCompactChunk : 1;
-    const dim3 grid(nchunks, B);
-    sca_count_kernel<<<grid, kCompactChunk, 0, s>>>(mask, B, Ncam, Nq, R, nchunks, hits,
+    const bool word = (R == 1 || R == 2 || R == 4 || R == 8) && (uintptr_t)mask % R == 0;
+    const dim3 grid(nchunks, B * Ncam);
+    sca_count_kernel<<<grid, kCompactChunk, 0, s>>>(mask, B, Ncam, Nq, R, word, nchunks,
                                                     chunk_counts);
     const bool inline_scan = nchunks <= kInlineScanChunks;
     if (!inline_scan)
         sca_chunk_scan_kernel<<<B * Ncam, 32, 0, s>>>(chunk_counts, nchunks, count);
-    sca_scatter_kernel<<<grid, kCompactChunk, 0, s>>>(mask, B, Ncam, Nq, R, nchunks,
-                                                      chunk_counts, count, idx, pos, inline_scan);
-    return cudaGetLastError();
+    // the scatter pass's mask loads overlap the end of the pass before it
+    return launch_pdl(sca_scatter_kernel, grid, dim3(kCompactChunk), 0, s, mask, B, Ncam, Nq, R,
+                      word, nchunks, chunk_counts, count, idx, pos, hits, inline_scan);
 }
 
 // Rows are ordered (b, c, i): at any time the whole GPU works on a narrow
@@ -194,7 +212,9 @@ sca_gather_kernel(const VT* __restrict__ value, const float* __restrict__ off,
     __shared__ __align__(16) Table s_tab[kWarps];
     __shared__ int s_prefix[kMaxBatchCameras + 1];
     const int nbc = B * Ncam;
+    pdl_trigger();  // the average pass reads the rows only after its pdl_wait
     stage_levels(s_lv, levels);
+    pdl_wait();  // the compaction lists are complete
     stage_row_prefix(count, nbc, Nq, s_prefix);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -301,9 +321,11 @@ static cudaError_t launch_gather_t(const Problem& p, const float* ref_cam, const
     case NCV: {                                                                                  \
         static int occ = resident_ctas(sca_gather_kernel<VT, NCV, HP>, kThreads);                \
         const int64_t grid = std::min<int64_t>(max_tiles, (int64_t)occ * device_sm_count());     \
-        sca_gather_kernel<VT, NCV, HP><<<(unsigned)grid, kThreads, 0, s>>>(                      \
-            v, off, logits, ref_cam, idx, count, out_rb, p.B, p.Ncam, p.Nq, p.Nv, p.H, p.L,      \
-            p.P, p.R, p.lv);                                                                     \
+        const cudaError_t e = launch_pdl(sca_gather_kernel<VT, NCV, HP>, dim3((unsigned)grid),   \
+                                         dim3(kThreads), 0, s, v, off, logits, ref_cam, idx,     \
+                                         count, out_rb, p.B, p.Ncam, p.Nq, p.Nv, p.H, p.L, p.P,  \
+                                         p.R, p.lv);                                             \
+        if (e != cudaSuccess) return e;                                                          \
         break;                                                                                   \
     }
     switch (nc) {
@@ -368,6 +390,7 @@ sca_average_kernel(const float4* __restrict__ out_rb, const int32_t* __restrict_
                    void* __restrict__ out)
 {
     constexpr int kAvgBatch = PL >= MSDA_AVG_INFLIGHT ? 1 : MSDA_AVG_INFLIGHT / PL;
+    pdl_wait();  // the rows, positions and hit counts are complete
     const int lane = threadIdx.x & 31;
     const int64_t bq = (int64_t)blockIdx.x * kAvgWarps + (threadIdx.x >> 5);
     if (bq >= (int64_t)B * Nq) return;  // warp-uniform
@@ -447,12 +470,10 @@ cudaError_t launch_sca_average(const float* out_rb, const int32_t* pos, const in
 #define SCA_AVG_CASE(PLV)                                                                        \
     if (pl <= PLV) {                                                                             \
         if (out_bf16)                                                                            \
-            sca_average_kernel<PLV, true><<<grid, kAvgWarps * 32, 0, s>>>(in, pos, hits, B,      \
-                                                                          Ncam, Nq, row4, out);  \
-        else                                                                                     \
-            sca_average_kernel<PLV, false><<<grid, kAvgWarps * 32, 0, s>>>(in, pos, hits, B,     \
-                                                                           Ncam, Nq, row4, out); \
-        return cudaGetLastError();                                                               \
+            return launch_pdl(sca_average_kernel<PLV, true>, dim3(grid), dim3(kAvgWarps * 32), 0, \
+                              s, in, pos, hits, B, Ncam, Nq, row4, out);                         \
+        return launch_pdl(sca_average_kernel<PLV, false>, dim3(grid), dim3(kAvgWarps * 32), 0,   \
+                          s, in, pos, hits, B, Ncam, Nq, row4, out);                             \
     }
     SCA_AVG_CASE(1)
     SCA_AVG_CASE(2)

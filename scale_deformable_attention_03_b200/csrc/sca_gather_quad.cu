@@ -410,6 +410,8 @@ sca_gather_quad_kernel(const VT* __restrict__ value, const float* __restrict__ o
         s_meta[quad_meta_slot(j)] = mt;
     }
     const int nbc = B * Ncam;
+    pdl_trigger();  // the average pass reads the rows only after its pdl_wait
+    pdl_wait();     // the compaction lists are complete
     stage_row_prefix(count, nbc, Nq, s_prefix);  // block barrier: s_meta is visible after it
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -548,10 +550,9 @@ static cudaError_t launch_quad_t(const Problem& p, const float* ref_cam, const f
     if (MSDA_QUAD_HEADSPEC && grid > p.H) grid -= grid % p.H;  // a CTA keeps one head
     const bool vec = p.L * p.P == kQuadSamples && ((uintptr_t)off & 15) == 0 &&
                      ((uintptr_t)logits & 15) == 0;
-    sca_gather_quad_kernel<VT><<<(unsigned)grid, kThreads, 0, s>>>(
-        static_cast<const VT*>(p.value), off, logits, ref_cam, idx, count, out_rb, p.B, p.Ncam,
-        p.Nq, p.Nv, p.H, p.L, p.P, p.R, p.lv, vec);
-    return cudaGetLastError();
+    return launch_pdl(sca_gather_quad_kernel<VT>, dim3((unsigned)grid), dim3(kThreads), 0, s,
+                      static_cast<const VT*>(p.value), off, logits, ref_cam, idx, count, out_rb,
+                      p.B, p.Ncam, p.Nq, p.Nv, p.H, p.L, p.P, p.R, p.lv, vec);
 }
 
 bool sca_gather_quad_fits(const Problem& p) { return p.L * p.P <= kQuadSamples; }

@@ -11,9 +11,11 @@
 //   g     = SCA(V, Delta, a, rho, mask)  (5-10: compaction, fused MSDA, average)
 //   q_hat = q + dropout(g W_o^T + b_o)   (11-13; dropout in the projection's
 //                                         epilogue, the identity when p = 0)
-// With fp32 value the camera average is formed inside the output projection
-// (its X tiles are built from the rebatched rows), so g is never stored; with
-// bf16 value the query-major SCA stores g as bf16 for the projection.
+// The SCA runs compaction, the rebatched gather and the camera average, which
+// stores g as the projection's bf16 operand.  Built with
+// MSDA_MODULE_FUSED_AVERAGE = 1, fp32 value forms the camera average inside
+// the output projection instead (its X tiles built from the rebatched rows,
+// g never stored), which measured slower on the BEVFormer-base module.
 // It composes the library's own kernels; the only new one is the element-wise
 // q + pos conversion below.
 #include <cuda_bf16.h>
@@ -166,9 +168,10 @@ extern "C" msda_status_t sca_module_forward(const sca_module_params_t* p,
     if ((st = msda_linear(w.qt, p->w_weights, p->b_weights, nullptr, (int32_t)rows_q, S, C,
                           MSDA_F32, w.logits, stream)) != MSDA_OK)
         return st;
-    // fp32 value: the compaction and the rebatched gather, then the camera
-    // average formed inside the output projection (g never stored); bf16
-    // value: the query-major SCA stores g as bf16, then the projection
+    // MSDA_MODULE_FUSED_AVERAGE with fp32 value: the compaction and the
+    // rebatched gather, then the camera average formed inside the output
+    // projection (g never stored); otherwise the SCA stores g as bf16, then
+    // the projection
     if (MSDA_MODULE_FUSED_AVERAGE && p->value_dtype == MSDA_F32 && d.Ncam <= 8) {
         ScaWorkspace rows;
         if ((st = sca_forward_to(w.value, p->value_dtype, spatial_shapes, level_start_index,

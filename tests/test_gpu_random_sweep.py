@@ -7,7 +7,7 @@ the query-major kernel, the training backward in both accumulation modes and
 the whole backward chain) against the oracle: fp32 value at the fp32 element
 bound, bf16 value at the bf16 bound (the oracle reading the same bf16
 values); the staged calls must equal the one-call
-forward bit for bit when both take the rebatched path, and the two grad_value
+forward bit for bit (both run the rebatched kernels), and the two grad_value
 accumulations must agree with each other within the fp32 bound.  Plain MSDA:
 batch, queries, heads, levels, points and anchors, locations partly outside
 their levels, through msda_forward, msda_forward_fused and msda_backward (both
@@ -79,8 +79,7 @@ def test_forward_entry_points(case, bf16):
     assert_close(whole, ref, bf16, "sca_forward")
     assert_close(qm, ref, bf16, "sca_forward_query_major")
     assert_close(staged, ref, bf16, "staged forward")
-    if not bf16:  # both take the rebatched path: the same kernels, the same bits
-        assert torch.equal(staged, whole)
+    assert torch.equal(staged, whole)  # the same kernels, the same bits
 
 
 @pytest.mark.parametrize("case", PROBLEMS, ids=[f"p{c[0]}" for c in PROBLEMS])
