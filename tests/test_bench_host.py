@@ -106,7 +106,7 @@ def _stub_replica(args, rank, world, barrier):
     barrier()   # before the end-to-end leg
     k = 1 + rank
     return {"w": _FakeW(), "bf16": False, "step_ms": [0.5 * k] * args.steps,
-            "gather_ms": [0.4 * k] * args.steps, "compact_ms": [0.05] * args.steps,
+            "staged_ms": [0.51 * k] * args.steps, "gather_ms": [0.4 * k] * args.steps, "compact_ms": [0.05] * args.steps,
             "avg_ms": [0.05] * args.steps, "warm_gather_ms": 0.3,
             "samples_per_step": 1000 * k + seed % 7, "rows": 10, "seed": seed,
             "nbytes": {"step": 4_000_000, "gather": 5_000_000},

@@ -116,8 +116,8 @@ def test_empty_mask():
 
 def test_rebatched_bf16_full_size():
     """The staged rebatched path with bf16 value (head-pair gather) at the
-    full BEVFormer-base size; sca_forward takes the query-major kernel for bf16
-    value, so the two agree within the bf16-path bound of the oracle."""
+    full BEVFormer-base size, against the oracle and bit for bit against
+    sca_forward, which runs the same kernels."""
     w = inputs.workload3(value_dtype="bf16")
     v = value_tensor(w, True)
     args = (v, w.spatial_shapes, w.level_start_index, dev(w.reference_points))
@@ -132,6 +132,41 @@ def test_rebatched_bf16_full_size():
                              w.bev_mask, w.sampling_offsets, w.attention_logits)
     assert_close(staged, ref, True, "staged bf16 SCA")
     assert_close(whole, ref, True, "sca_forward bf16")
+    assert torch.equal(staged, whole)
+
+
+def test_back_to_back_calls_share_one_workspace():
+    """Consecutive calls on one stream with different masks and inputs, one
+    workspace and one set of lists, no host synchronisation in between: each
+    result must be its own.  The compaction's later passes, the gather and the
+    camera average begin while the kernel before them finishes (programmatic
+    dependent launches); this checks that a call's lists and rows are never
+    read before they are complete, nor overwritten while the call before
+    still reads them."""
+    ws = [inputs.workload3(seed=s, bev_h=40, bev_w=50, rho=rho, same_mask=False)
+          for s, rho in ((41, "coherent"), (42, "uniform"), (43, "coherent"))]
+    ws[1].bev_mask[:, :, ::3, :] = 0  # fewer rows than the call before it
+    dims = msda.Dims(ws[0].B, ws[0].Ncam, ws[0].Nq, ws[0].Nv, ws[0].H, ws[0].L, ws[0].P,
+                     ws[0].R)
+    workspace = torch.empty(msda.msda_workspace_size(dims), dtype=torch.uint8, device="cuda")
+    dev_args = [(dev(w.value), w.spatial_shapes, w.level_start_index, dev(w.reference_points),
+                 dev(w.bev_mask), dev(w.sampling_offsets), dev(w.attention_logits)) for w in ws]
+    outs = [msda.sca_forward(*a, workspace=workspace) for a in dev_args + dev_args[:1]]
+    lists = msda.sca_compact(dev_args[0][4])
+    rows = torch.empty((ws[0].B, ws[0].Ncam, ws[0].Nq, ws[0].H * 32), device="cuda")
+    staged = []
+    for a in dev_args:
+        msda.sca_compact(a[4], out=lists)
+        msda.sca_rebatched_forward(*a[:4], a[5], a[6], lists[0], lists[1], out_rb=rows)
+        staged.append(msda.sca_camera_average(rows, lists[2], lists[3]))
+    torch.cuda.synchronize()
+    for k, w in enumerate(ws):
+        ref = oracle.sca_forward(w.value, w.spatial_shapes, w.level_start_index,
+                                 w.reference_points, w.bev_mask, w.sampling_offsets,
+                                 w.attention_logits)
+        assert_close(outs[k], ref, False, f"sca_forward call {k}")
+        assert torch.equal(staged[k], outs[k]), f"staged call {k}"
+    assert torch.equal(outs[3], outs[0])
 
 
 def test_staged_calls_equal_sca_forward():
