@@ -125,6 +125,40 @@ def test_sca_backward_random(seed, B, Ncam, bev, shapes, H, P, R):
     assert_close(gv, rv, False, "grad_value")
 
 
+@pytest.mark.parametrize("case", ["no camera sees anything", "one camera blind",
+                                  "every camera sees everything", "sixteen heads"])
+@pytest.mark.parametrize("deterministic", [False, True])
+def test_sca_backward_padding_rows(case, deterministic):
+    """The rebatched gradients' rows count .. Nq-1 of every (batch, camera)
+    hold no row and must come back zero: outputs pre-filled with NaN,
+    compared with the oracle element by element, including the case with no
+    rebatched row at all and a head count above the warps per CTA."""
+    H, P, R = (16, 4, 2) if case == "sixteen heads" else (4, 4, 2)
+    w = inputs.workload3(seed=35, B=2, Ncam=3, bev_h=9, bev_w=11, shapes=[(7, 9), (3, 4)],
+                         H=H, P=P, R=R, rho="uniform", same_mask=False, with_grad=True)
+    if case == "no camera sees anything":
+        w.bev_mask[:] = 0
+    elif case == "one camera blind":
+        w.bev_mask[1] = 0
+    elif case == "every camera sees everything":
+        w.bev_mask[:] = 1
+    B, Ncam, Nq, L = w.B, w.Ncam, w.Nq, w.L
+    gl = torch.full((B, Ncam, Nq, H, L, P, 2), float("nan"), device="cuda")
+    gw = torch.full((B, Ncam, Nq, H, L, P), float("nan"), device="cuda")
+    gv, gl, gw = msda.sca_backward(dev(w.value), w.spatial_shapes, w.level_start_index,
+                                   dev(w.reference_points), dev(w.bev_mask),
+                                   dev(w.sampling_offsets), dev(w.attention_logits),
+                                   dev(w.grad_out), grad_sampling_locations_rb=gl,
+                                   grad_attention_weights_rb=gw, deterministic=deterministic)
+    torch.cuda.synchronize()
+    rv, rl, rw = oracle.sca_backward(w.value, w.spatial_shapes, w.level_start_index,
+                                     w.reference_points, w.bev_mask, w.sampling_offsets,
+                                     w.attention_logits, w.grad_out)
+    assert_close(gw, rw, False, f"{case}: grad_attention_weights_rb")
+    assert_close(gl, rl, False, f"{case}: grad_sampling_locations_rb")
+    assert_close(gv, rv, False, f"{case}: grad_value")
+
+
 def test_sca_backward_workload3_full_size():
     """The BEVFormer-base SCA backward with fp32 value (B = 1) at full size:
     the rebatched gradients and grad_value at the fp32 bound."""
