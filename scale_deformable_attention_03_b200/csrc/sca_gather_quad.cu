@@ -476,6 +476,8 @@ sca_gather_quad_kernel(const VT* __restrict__ value, const float* __restrict__ o
                                   : t0 + kWarps + (int64_t)(gridDim.x - 1) * kChunk * kWarps;
     };
     (void)stride;
+    // with out_rb on 32 bytes, each lane's eight output channels are too
+    const bool out32 = ((uintptr_t)out_rb & 31) == 0;
     int64_t tile = (int64_t)blockIdx.x * kChunk * kWarps + warp;
     if (tile >= n_tiles) return;  // warp-uniform
     Item cur = resolve(tile);
@@ -515,8 +517,15 @@ sca_gather_quad_kernel(const VT* __restrict__ value, const float* __restrict__ o
         if (cur.live) {
             float4* o = reinterpret_cast<float4*>(
                 out_rb + ((int64_t)cur.out_row * H + cur.h) * kHeadDim + 8 * t);
-            o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-            o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+            if (out32) {  // the lane's 32 bytes in one store
+                asm volatile("st.global.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(o),
+                             "f"(acc[0]), "f"(acc[1]), "f"(acc[2]), "f"(acc[3]), "f"(acc[4]),
+                             "f"(acc[5]), "f"(acc[6]), "f"(acc[7])
+                             : "memory");
+            } else {
+                o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+            }
         }
         if (next_tile >= n_tiles) break;  // warp-uniform
         tile = next_tile;
