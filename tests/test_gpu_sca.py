@@ -135,6 +135,29 @@ def test_rebatched_bf16_full_size():
     assert torch.equal(staged, whole)
 
 
+def test_rebatched_rows_into_16_byte_aligned_buffer():
+    """The gather writes each lane's eight channels with one 32-byte store
+    when out_rb is 32-byte aligned and with two 16-byte stores otherwise:
+    the same rows either way."""
+    w = inputs.workload3(seed=45, bev_h=20, bev_w=30)
+    args = (dev(w.value), w.spatial_shapes, w.level_start_index, dev(w.reference_points),
+            dev(w.sampling_offsets), dev(w.attention_logits))
+    idx, count, pos, hits = msda.sca_compact(dev(w.bev_mask))
+    shape = (w.B, w.Ncam, w.Nq, w.H * 32)
+    n = w.B * w.Ncam * w.Nq * w.H * 32
+    store = torch.zeros(n + 8, device="cuda")
+    assert store.data_ptr() % 32 == 0
+    aligned = msda.sca_rebatched_forward(*args, idx, count, out_rb=store[:n].view(shape))
+    off16 = msda.sca_rebatched_forward(*args, idx, count,
+                                       out_rb=torch.zeros(n + 8, device="cuda")[4:4 + n].view(shape))
+    torch.cuda.synchronize()
+    assert off16.data_ptr() % 32 == 16
+    cnt = count.cpu().numpy().reshape(-1)
+    for bc in range(len(cnt)):
+        b, c = divmod(bc, w.Ncam)
+        assert torch.equal(aligned[b, c, :cnt[bc]], off16[b, c, :cnt[bc]])
+
+
 def test_back_to_back_calls_share_one_workspace():
     """Consecutive calls on one stream with different masks and inputs, one
     workspace and one set of lists, no host synchronisation in between: each
