@@ -90,11 +90,13 @@ struct AvgArgs {
 };
 
 // Shared memory: W (K/64 blocks of 256 x 64), the X ring, 4 warps x 2
-// epilogue buffers, then the control block; 1024-byte aligned.
+// epilogue buffers, the bias (a plain bias of N = 256), then the control
+// block; 1024-byte aligned.
 constexpr size_t kSmemB = (size_t)kMaxKBlocks * kBBlockBytes;   // 128 KB
 constexpr size_t kSmemA = (size_t)kStages * kABlockBytes;       // 64 KB
 constexpr size_t kSmemC = (size_t)4 * 2 * kCBufBytes;           // 32 KB
-constexpr size_t kSmemBytes = 1024 + kSmemB + kSmemA + kSmemC + sizeof(Ctrl);
+constexpr size_t kSmemBias = (size_t)kBN * 4;                     // 1 KB: the bias of N = 256
+constexpr size_t kSmemBytes = 1024 + kSmemB + kSmemA + kSmemC + kSmemBias + sizeof(Ctrl);
 static_assert(kSmemBytes <= 227 * 1024, "shared memory of the projection kernel");
 static_assert((kStages & (kStages - 1)) == 0 && kStages >= kMaxKBlocks,
               "a tile's K-blocks fit the ring, whose size is a power of two");
@@ -484,7 +486,8 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
     uint8_t* sb = smem;
     uint8_t* sa = sb + kSmemB;
     uint8_t* sc = sa + kSmemA;
-    Ctrl& ctrl = *reinterpret_cast<Ctrl*>(sc + kSmemC);
+    float* s_bias = reinterpret_cast<float*>(sc + kSmemC);
+    Ctrl& ctrl = *reinterpret_cast<Ctrl*>(sc + kSmemC + kSmemBias);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int kblocks = K / kBK;
     const int mt = (M + kBM - 1) / kBM;
@@ -676,6 +679,13 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
         // ---- epilogue: warps 2..5, TMEM lane quarter q = warp % 4 ----
         const int q = warp & 3;
         uint8_t* cbuf = sc + (size_t)q * 2 * kCBufBytes;
+        // a plain bias of one W tile (N = 256) is read from shared memory:
+        // staged once by the four epilogue warps, before any of their waits
+        const bool bias_smem = bias != nullptr && rbias.table == nullptr && N == kBN;
+        if (bias_smem) {
+            for (int i = (warp - 2) * 32 + lane; i < kBN; i += 128) s_bias[i] = __ldg(bias + i);
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+        }
         int acc = 0, buf = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
@@ -699,9 +709,15 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
 #pragma unroll
                     for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
                     const int col = n0 + c0 + 32 * half;
-                    const float* brow = bias;
+                    const float* brow = bias_smem ? s_bias - n0 : bias;
                     if (rbias.table) brow = row_ok ? row_bias(rbias, row, N) : nullptr;
-                    if (brow) {
+                    if (bias_smem) {
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4) {
+                            const float4 b4 = *reinterpret_cast<const float4*>(brow + col + j);
+                            v[j] += b4.x; v[j + 1] += b4.y; v[j + 2] += b4.z; v[j + 3] += b4.w;
+                        }
+                    } else if (brow) {
 #pragma unroll
                         for (int j = 0; j < 32; j += 4) {
                             const float4 b4 = __ldg(reinterpret_cast<const float4*>(brow + col + j));
