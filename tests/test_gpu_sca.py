@@ -158,6 +158,44 @@ def test_rebatched_rows_into_16_byte_aligned_buffer():
         assert torch.equal(aligned[b, c, :cnt[bc]], off16[b, c, :cnt[bc]])
 
 
+def test_sca_forward_in_a_cuda_graph():
+    """sca_forward captured once into a CUDA graph (its launches, the
+    overlapping ones included, become graph nodes) and replayed on new inputs
+    copied into the captured buffers: each replay equals a direct call bit
+    for bit."""
+    ws = [inputs.workload3(seed=s, bev_h=30, bev_w=40) for s in (46, 47)]
+    w0 = ws[0]
+    dims = msda.Dims(w0.B, w0.Ncam, w0.Nq, w0.Nv, w0.H, w0.L, w0.P, w0.R)
+    workspace = torch.empty(msda.msda_workspace_size(dims), dtype=torch.uint8, device="cuda")
+    bufs = [dev(w0.value), dev(w0.reference_points), dev(w0.bev_mask), dev(w0.sampling_offsets),
+            dev(w0.attention_logits)]
+    out = torch.empty((w0.B, w0.Nq, w0.H * 32), device="cuda")
+
+    def call(stream=None):
+        msda.sca_forward(bufs[0], w0.spatial_shapes, w0.level_start_index, bufs[1], bufs[2],
+                         bufs[3], bufs[4], out=out, workspace=workspace, stream=stream)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        call(side)  # warm-up outside the capture
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call(torch.cuda.current_stream())
+    for w in ws + ws[:1]:
+        for b, a in zip(bufs, (w.value, w.reference_points, w.bev_mask, w.sampling_offsets,
+                               w.attention_logits)):
+            b.copy_(torch.from_numpy(np.ascontiguousarray(a)))
+        graph.replay()
+        direct = msda.sca_forward(dev(w.value), w.spatial_shapes, w.level_start_index,
+                                  dev(w.reference_points), dev(w.bev_mask),
+                                  dev(w.sampling_offsets), dev(w.attention_logits))
+        torch.cuda.synchronize()
+        assert torch.equal(out, direct)
+    del graph
+
+
 def test_back_to_back_calls_share_one_workspace():
     """Consecutive calls on one stream with different masks and inputs, one
     workspace and one set of lists, no host synchronisation in between: each
