@@ -149,4 +149,9 @@ def test_bench_replica_path_two_ranks_gloo(tmp_path):
     assert abs(line["ms_per_step"] - slowest_ms / 4) < 1e-12
     e2e_work = 2 * ((1000 + s0 % 7) + (2000 + s1 % 7))
     assert abs(line["e2e"]["value"] - e2e_work / (2.0 * 2 * 2 * 1e-3) / 1e9) < 1e-12
+    # rank 0's own stage times: the one-call step and the instrumented pass
+    ms = line["step"]["ms"]
+    assert abs(ms["step"] - 0.5) < 1e-12 and abs(ms["staged_step"] - 0.51) < 1e-12
+    assert abs(ms["gather"] - 0.4) < 1e-12 and "sca_forward call" in line["step"]["timing"]
+    assert line["gpu_launches"] == 5 * 4 and line["roofline"]["launch_ms"] == ms["gather"]
     assert "cpu_baseline" not in line and "next_rows" not in line
