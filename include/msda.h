@@ -35,6 +35,11 @@
  *     The status covers argument checks and kernel launch errors; errors that
  *     happen while the kernels run surface at the caller's next
  *     synchronisation.  Nothing is launched when the arguments are rejected.
+ *     Some kernels are programmatic dependent launches (the SCA compaction's
+ *     second pass, the rebatched gather, the camera average): they may begin
+ *     while the kernel before them in the stream finishes and wait for it
+ *     before they read or write memory, so stream order holds as usual, and
+ *     the calls can be captured into CUDA graphs.
  *   - Outputs are fully overwritten (including gradients and padded rows).
  *   - Value rows: pixel (y, x) of level l is row level_start_index[l] +
  *     y * W_l + x; a row holds H heads of MSDA_HEAD_DIM channels.
