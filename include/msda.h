@@ -37,9 +37,9 @@
  *     synchronisation.  Nothing is launched when the arguments are rejected.
  *     Some kernels are programmatic dependent launches (the SCA compaction's
  *     second pass, the rebatched gather, the camera average): they may begin
- *     while the kernel before them in the stream finishes and wait for it
- *     before they read or write memory, so stream order holds as usual, and
- *     the calls can be captured into CUDA graphs.
+ *     while the kernel before them in the stream finishes, and wait for it
+ *     before they read what it may write or write anything, so stream order
+ *     holds as usual, and the calls can be captured into CUDA graphs.
  *   - Outputs are fully overwritten (including gradients and padded rows).
  *   - Value rows: pixel (y, x) of level l is row level_start_index[l] +
  *     y * W_l + x; a row holds H heads of MSDA_HEAD_DIM channels.
