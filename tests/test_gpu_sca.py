@@ -55,6 +55,28 @@ def test_compaction_all_or_nothing(fill):
     _assert_compaction_equal(np.full((6, 2, 3000, 4), fill, np.uint8))
 
 
+@pytest.mark.parametrize("R", [1, 2, 4, 8, 3])
+def test_compaction_mask_at_odd_address(R):
+    """The compaction reads a query's R anchor bytes as one word when R is
+    1, 2, 4 or 8 and the mask is aligned to R bytes, byte by byte otherwise:
+    a mask one byte past an aligned address (and R = 3) takes the byte path,
+    with the same lists."""
+    rng = np.random.Generator(np.random.PCG64(60 + R))
+    Ncam, B, Nq = 5, 2, 2500
+    mask = (rng.random((Ncam, B, Nq, R)) < 0.3).astype(np.uint8)
+    mask[:, :, ::7, :] = 0
+    buf = torch.zeros(mask.size + 16, dtype=torch.uint8, device="cuda")
+    off = buf[1:1 + mask.size].view(mask.shape)
+    off.copy_(torch.from_numpy(mask))
+    aligned = dev(mask)
+    got_off = [t.cpu().numpy() for t in msda.sca_compact(off)]
+    got = [t.cpu().numpy() for t in msda.sca_compact(aligned)]
+    want = oracle.sca_compact(mask)
+    for name, a, b, c in zip(("idx", "count", "pos", "hits"), got_off, got, want):
+        assert np.array_equal(a, c), f"{name} (odd address)"
+        assert np.array_equal(b, c), f"{name} (aligned)"
+
+
 def test_compaction_non_binary_mask_bytes():
     rng = np.random.Generator(np.random.PCG64(3))
     mask = rng.integers(0, 256, (4, 1, 999, 4)).astype(np.uint8) * (rng.random((4, 1, 999, 4)) < 0.2)
